@@ -1,0 +1,893 @@
+/*
+ * kvq_oracle.c -- CPU oracle for the low-bit KV cache (TEST INFRASTRUCTURE).
+ *
+ * This file is the plain, slow, obviously-correct statement of what the hot
+ * path computes.  Only the tests, the package smoke check and the benchmark's
+ * CPU-baseline leg may load it.  It shares no code, header, table or constant
+ * generator with the CUDA library: the byte layout, the sign generator and the
+ * rotation constant are all restated here from their written definitions.
+ *
+ * Sources (cited by page title and section):
+ *   [SRFT]  "When Quantization Is Free: An int4 KV Cache That Outruns fp16 on
+ *           Apple Silicon" -- Methodology 1 (random-sign rotation, SRHT as the
+ *           Hadamard alternative), Methodology 2 (fused kernel: sign in
+ *           registers, butterfly passes, per-group scaling, rounding, nibble
+ *           packing).
+ *   [CERT]  "Runtime-Certified Bounded-Error Quantized Attention" --
+ *           Methodology 1 (tier 1: INT8 keys / INT4 values with scales,
+ *           offsets and per-block error descriptors; tier 2: fp16 originals in
+ *           pinned host RAM), Methodology 2 (key term E_key from the per-token
+ *           score perturbation, value term E_val from per-block reconstruction
+ *           errors weighted by block mass), Methodology 3 (top-K* promotion of
+ *           blocks to fp16).
+ *   [OSCAR] "OSCAR: Offline Spectral Covariance-Aware Rotation for 2-bit KV
+ *           cache quantization" -- 2.2 Algorithm design (Hadamard factor of the
+ *           rotation, clipping thresholds; paged INT2 history; fused kernel
+ *           doing unpack, dequantization, inverse rotation and attention).
+ *
+ * Precision: the codec (rotation, statistics, scale/zero, codes) is fp32 with
+ * every operation rounded separately (build with -ffp-contract=off), because
+ * the quantised codes are integers decided by floating point and both sides
+ * must take that decision in the same precision.  Attention is fp64.
+ *
+ * Readings of points the pages leave open are listed next to the code that
+ * takes them.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define KVQO_INT4_ASYM 0
+#define KVQO_INT8_SYM 1
+#define KVQO_INT2_ASYM 2
+
+#define KVQO_PAGE_TOKENS 16
+#define KVQO_HEADER_BYTES 256
+#define KVQO_MAXD 256
+
+typedef struct {
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t head_dim;
+    int32_t k_fmt;
+    int32_t v_fmt;
+    int32_t k_group;
+    int32_t v_group;
+    float clip_ratio;
+    uint64_t rotation_seed;
+    int32_t rotate;
+    int32_t page_tokens;
+    int32_t num_pages;
+    int32_t bound_block_tokens;
+} kvqo_config;
+
+/* ------------------------------------------------------------------------- */
+/* IEEE binary16 conversions, written from the format definition.            */
+/* ------------------------------------------------------------------------- */
+
+/* binary16 bits -> fp32 value (exact). */
+float kvqo_h2f(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int m = h & 0x3ff;
+    float v;
+    if (e == 0)
+        v = ldexpf((float)m, -24); /* subnormal: m * 2^-24 */
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexpf((float)(m | 0x400), e - 25); /* (1024+m) * 2^(e-15-10) */
+    return sign ? -v : v;
+}
+
+/* round-half-to-even of a non-negative double that holds few bits. */
+static double rhe(double q)
+{
+    double n = floor(q);
+    double f = q - n;
+    if (f > 0.5) return n + 1.0;
+    if (f < 0.5) return n;
+    return (fmod(n, 2.0) == 0.0) ? n : n + 1.0;
+}
+
+/* Magnitude |x| (finite, >= 0) -> binary16 bits of the value on the fp16 grid
+ * selected by `mode`: 0 = nearest-even, 1 = up (away from zero for the
+ * magnitude), 2 = down (toward zero).  Overflow handling is left to the
+ * caller. */
+static uint32_t mag_to_h(double a, int mode)
+{
+    double step;
+    int e = 0;
+    if (a < ldexp(1.0, -14)) {
+        step = ldexp(1.0, -24); /* subnormal grid */
+    } else {
+        int E;
+        frexp(a, &E); /* a = f * 2^E, f in [0.5,1) */
+        e = E - 1;    /* 2^e <= a < 2^(e+1) */
+        step = ldexp(1.0, e - 10);
+    }
+    double q = a / step; /* exact: a has at most 24 significant bits */
+    double n;
+    if (mode == 0) n = rhe(q);
+    else if (mode == 1) n = ceil(q);
+    else n = floor(q);
+    if (a < ldexp(1.0, -14)) return (uint32_t)n; /* n == 1024 is the smallest normal */
+    /* n in [1024, 2048]; n == 2048 carries into the exponent correctly */
+    return (uint32_t)(((e + 15) << 10) + ((int)n - 1024));
+}
+
+/* fp32 -> binary16, round to nearest, ties to even. */
+uint16_t kvqo_f2h_rn(float x)
+{
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    if (isnan(x)) return 0x7e00;
+    double a = fabs((double)x);
+    if (a >= 65520.0) return sign | 0x7c00; /* at or past max + half ulp */
+    return sign | (uint16_t)mag_to_h(a, 0);
+}
+
+/* fp32 -> binary16, round toward +infinity. */
+uint16_t kvqo_f2h_ru(float x)
+{
+    if (isnan(x)) return 0x7e00;
+    double a = fabs((double)x);
+    if (!signbit(x)) {
+        if (a > 65504.0) return 0x7c00;
+        return (uint16_t)mag_to_h(a, 1);
+    }
+    if (a > 65504.0) return 0xfbff; /* -65504 is the least fp16 >= x */
+    return 0x8000 | (uint16_t)mag_to_h(a, 2);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Rotation R = c_d * H_d * diag(s)                                          */
+/* ------------------------------------------------------------------------- */
+
+/* SplitMix64 (Steele, Lea, Flood; Vigna's reference generator): the state
+ * advances by the golden-ratio increment and each output is the state passed
+ * through the two xor-shift-multiply rounds. */
+static uint64_t splitmix64_next(uint64_t *state)
+{
+    uint64_t z = (*state += 0x9E3779B97F4A7C15ULL);
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+    return z ^ (z >> 31);
+}
+
+uint64_t kvqo_splitmix64_output(uint64_t seed, int index)
+{
+    uint64_t st = seed, z = 0;
+    for (int i = 0; i <= index; i++) z = splitmix64_next(&st);
+    return z;
+}
+
+/* [SRFT] Methodology 1: a fixed random sign vector s.  Reading: one vector per
+ * cache, s_i = -1 when the top bit of the i-th SplitMix64 output (state seeded
+ * with rotation_seed) is set, else +1; the same s serves every head, K and V. */
+void kvqo_signs(uint64_t seed, int d, float *s)
+{
+    uint64_t st = seed;
+    for (int i = 0; i < d; i++) s[i] = (splitmix64_next(&st) >> 63) ? -1.0f : 1.0f;
+}
+
+/* c_d = 1/sqrt(d) rounded to fp32. */
+float kvqo_rot_scale_f32(int d) { return (float)(1.0 / sqrt((double)d)); }
+
+/* [SRFT] Methodology 1-2 with the Hadamard choice (SRHT), [OSCAR] 2.2
+ * (H_Had factor): y = c_d * H_d * diag(s) * x in fp32.  H_d is the Sylvester
+ * (natural-order) Hadamard matrix applied as log2(d) butterfly stages with
+ * half-width h = 1, 2, 4, ..., d/2; each stage maps the pair (j, j+h), j&h==0,
+ * to (a+b, a-b).  Stages run in that order and every operation rounds on its
+ * own; the codec's integer decisions depend on this exact order. */
+void kvqo_rotate_f32(const float *x, const float *s, int d, int rotate, float *y)
+{
+    if (!rotate) {
+        for (int i = 0; i < d; i++) y[i] = x[i];
+        return;
+    }
+    for (int i = 0; i < d; i++) y[i] = x[i] * s[i];
+    for (int h = 1; h < d; h <<= 1)
+        for (int j = 0; j < d; j++)
+            if (!(j & h)) {
+                float a = y[j], b = y[j + h];
+                y[j] = a + b;
+                y[j + h] = a - b;
+            }
+    float c = kvqo_rot_scale_f32(d);
+    for (int i = 0; i < d; i++) y[i] = y[i] * c;
+}
+
+static void fwht_f64(double *y, int d)
+{
+    for (int h = 1; h < d; h <<= 1)
+        for (int j = 0; j < d; j++)
+            if (!(j & h)) {
+                double a = y[j], b = y[j + h];
+                y[j] = a + b;
+                y[j + h] = a - b;
+            }
+}
+
+/* fp64 forward rotation R x (used for queries and for the exact fp16 rows). */
+void kvqo_rotate_f64(const double *x, const float *s, int d, int rotate, double *y)
+{
+    if (!rotate) {
+        for (int i = 0; i < d; i++) y[i] = x[i];
+        return;
+    }
+    for (int i = 0; i < d; i++) y[i] = x[i] * (double)s[i];
+    fwht_f64(y, d);
+    double c = 1.0 / sqrt((double)d);
+    for (int i = 0; i < d; i++) y[i] *= c;
+}
+
+/* fp64 inverse rotation R^T x = diag(s) * H_d * c_d * x ([OSCAR] 2.2b: the
+ * fused kernel applies the inverse rotation to the attention output). */
+void kvqo_inv_rotate_f64(const double *x, const float *s, int d, int rotate, double *y)
+{
+    if (!rotate) {
+        for (int i = 0; i < d; i++) y[i] = x[i];
+        return;
+    }
+    for (int i = 0; i < d; i++) y[i] = x[i];
+    fwht_f64(y, d);
+    double c = 1.0 / sqrt((double)d);
+    for (int i = 0; i < d; i++) y[i] = y[i] * c * (double)s[i];
+}
+
+/* ------------------------------------------------------------------------- */
+/* Codec for one token-head row                                              */
+/* ------------------------------------------------------------------------- */
+
+static int fmt_bits(int fmt) { return fmt == KVQO_INT4_ASYM ? 4 : fmt == KVQO_INT8_SYM ? 8 : 2; }
+
+/* Quantise one rotated row y[0..d).
+ *
+ * Asymmetric formats (int4, int2) -- [SRFT] Methodology 2 (per-group
+ * statistics, rounding), [CERT] Methodology 1 (scales/offsets):
+ *   lo = min, hi = max over the group; with clip ratio r < 1 ([OSCAR] 2.2a,
+ *   clipping thresholds) both ends are scaled by r (reading: toward zero);
+ *   scale_h = fp16_rn((hi - lo) / (2^b - 1)); zero_h = fp16_rn(lo);
+ *   inv = 1 / float(scale_h) (0 when scale_h == 0);
+ *   code = clamp(rint((y - float(zero_h)) * inv), 0, 2^b - 1), ties to even.
+ * Reading: "zero" is an additive fp16 offset equal to the group minimum.
+ *
+ * Symmetric int8 ([SRFT] Methodology 2, absmax; [CERT] Methodology 1, INT8
+ * keys): a = max |y| over the row (the config fixes one scale per token-head);
+ *   scale_h = fp16_ru(a / 127) -- rounding up keeps |y| * inv <= 127;
+ *   code = clamp(rint(y * inv), -127, 127).
+ *
+ * Outputs: code[d], scale_h[ng], zero_h[ng] (zero unused for int8), and the
+ * fp32 descriptors max|y - yhat| and max|y| with yhat = float(code)*scale
+ * (+ zero), each operation rounded on its own. */
+static void quantize_row(int fmt, int group, float clip, const float *y, int d, int16_t *code,
+                         uint16_t *scale_h, uint16_t *zero_h, float *err_max, float *abs_max)
+{
+    float emax = 0.0f, amax = 0.0f;
+    if (fmt == KVQO_INT8_SYM) {
+        float a = 0.0f;
+        for (int i = 0; i < d; i++) a = fmaxf(a, fabsf(y[i]));
+        float sf_raw = a / 127.0f;
+        uint16_t sh = kvqo_f2h_ru(sf_raw);
+        float sf = kvqo_h2f(sh);
+        float inv = (sf == 0.0f) ? 0.0f : 1.0f / sf;
+        for (int i = 0; i < d; i++) {
+            float v = y[i] * inv;
+            float r = rintf(v);
+            if (r < -127.0f) r = -127.0f;
+            if (r > 127.0f) r = 127.0f;
+            code[i] = (int16_t)r;
+            float yhat = (float)code[i] * sf;
+            emax = fmaxf(emax, fabsf(y[i] - yhat));
+            amax = fmaxf(amax, fabsf(y[i]));
+        }
+        scale_h[0] = sh;
+        zero_h[0] = 0;
+    } else {
+        int bits = fmt_bits(fmt);
+        float qmax = (float)((1 << bits) - 1);
+        int ng = d / group;
+        for (int g = 0; g < ng; g++) {
+            const float *yg = y + g * group;
+            float lo = yg[0], hi = yg[0];
+            for (int i = 1; i < group; i++) {
+                lo = fminf(lo, yg[i]);
+                hi = fmaxf(hi, yg[i]);
+            }
+            if (clip < 1.0f) {
+                lo = lo * clip;
+                hi = hi * clip;
+            }
+            float sf_raw = (hi - lo) / qmax;
+            uint16_t sh = kvqo_f2h_rn(sf_raw);
+            uint16_t zh = kvqo_f2h_rn(lo);
+            float sf = kvqo_h2f(sh), zf = kvqo_h2f(zh);
+            float inv = (sf == 0.0f) ? 0.0f : 1.0f / sf;
+            for (int i = 0; i < group; i++) {
+                float v = (yg[i] - zf) * inv;
+                float r = rintf(v);
+                if (r < 0.0f) r = 0.0f;
+                if (r > qmax) r = qmax;
+                int16_t c = (int16_t)r;
+                code[g * group + i] = c;
+                float yhat = (float)c * sf + zf;
+                emax = fmaxf(emax, fabsf(yg[i] - yhat));
+                amax = fmaxf(amax, fabsf(yg[i]));
+            }
+            scale_h[g] = sh;
+            zero_h[g] = zh;
+        }
+    }
+    *err_max = emax;
+    *abs_max = amax;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Paged pool layout (restated here from the written layout definition)      */
+/* ------------------------------------------------------------------------- */
+/* pool  = [header: 256 B][pages: num_pages x page_bytes][descriptors]
+ * page  = num_kv_heads chunks, chunk = [K codes][K meta][V codes][V meta]
+ * codes = 16 tokens; a token's code row is the sequential bit stream of its d
+ *         codes (int4: byte j = code[2j] | code[2j+1] << 4; int2: byte j holds
+ *         codes 4j..4j+3 from the low bits up; int8: two's complement bytes),
+ *         stored 16 bytes at a time "chunk-major": chunk c of token t sits at
+ *         (c*16 + t)*16 inside the region, so one 16-byte load is one whole
+ *         int4 group of 32.
+ * meta  = 16 tokens x row meta; asymmetric: ng fp16 scales then ng fp16
+ *         zeros; int8: one fp16 scale.
+ * descriptors (only when bound blocks are on): per (page, kv head) four fp32
+ *         {max key error, max value error, max |value|, 0} over the page. */
+
+static int row_code_bytes(int fmt, int d) { return d * fmt_bits(fmt) / 8; }
+static int row_meta_bytes(int fmt, int d, int group) { return fmt == KVQO_INT8_SYM ? 2 : 4 * (d / group); }
+static size_t region_code_bytes(int fmt, int d) { return (size_t)KVQO_PAGE_TOKENS * row_code_bytes(fmt, d); }
+static size_t region_meta_bytes(int fmt, int d, int g) { return (size_t)KVQO_PAGE_TOKENS * row_meta_bytes(fmt, d, g); }
+
+static size_t chunk_bytes(const kvqo_config *c)
+{
+    int d = c->head_dim;
+    return region_code_bytes(c->k_fmt, d) + region_meta_bytes(c->k_fmt, d, c->k_group) +
+           region_code_bytes(c->v_fmt, d) + region_meta_bytes(c->v_fmt, d, c->v_group);
+}
+
+size_t kvqo_page_bytes(const kvqo_config *c) { return (size_t)c->num_kv_heads * chunk_bytes(c); }
+
+size_t kvqo_desc_offset(const kvqo_config *c)
+{
+    return KVQO_HEADER_BYTES + (size_t)c->num_pages * kvqo_page_bytes(c);
+}
+
+size_t kvqo_pool_bytes(const kvqo_config *c)
+{
+    size_t n = kvqo_desc_offset(c);
+    if (c->bound_block_tokens > 0) n += (size_t)c->num_pages * c->num_kv_heads * 16;
+    return n;
+}
+
+/* byte offset of the region (tensor 0 = K, 1 = V) of (page, kv head) */
+static size_t region_base(const kvqo_config *c, int page, int kvh, int tensor, int meta)
+{
+    int d = c->head_dim;
+    size_t off = KVQO_HEADER_BYTES + (size_t)page * kvqo_page_bytes(c) + (size_t)kvh * chunk_bytes(c);
+    if (tensor == 1) off += region_code_bytes(c->k_fmt, d) + region_meta_bytes(c->k_fmt, d, c->k_group);
+    if (meta) off += region_code_bytes(tensor ? c->v_fmt : c->k_fmt, d);
+    return off;
+}
+
+static void pack_row(const kvqo_config *c, uint8_t *pool, int page, int tok, int kvh, int tensor, const int16_t *code,
+                     const uint16_t *scale_h, const uint16_t *zero_h)
+{
+    int d = c->head_dim;
+    int fmt = tensor ? c->v_fmt : c->k_fmt;
+    int group = tensor ? c->v_group : c->k_group;
+    int rb = row_code_bytes(fmt, d);
+    uint8_t stream[KVQO_MAXD];
+    memset(stream, 0, sizeof(stream));
+    int bits = fmt_bits(fmt);
+    for (int i = 0; i < d; i++) {
+        unsigned v = (unsigned)code[i] & ((1u << bits) - 1u);
+        stream[(i * bits) / 8] |= (uint8_t)(v << ((i * bits) % 8));
+    }
+    uint8_t *codes = pool + region_base(c, page, kvh, tensor, 0);
+    for (int ch = 0; ch < rb / 16; ch++) memcpy(codes + ((size_t)ch * 16 + tok) * 16, stream + ch * 16, 16);
+    uint8_t *meta = pool + region_base(c, page, kvh, tensor, 1) + (size_t)tok * row_meta_bytes(fmt, d, group);
+    if (fmt == KVQO_INT8_SYM) {
+        memcpy(meta, &scale_h[0], 2);
+    } else {
+        int ng = d / group;
+        for (int g = 0; g < ng; g++) {
+            memcpy(meta + 2 * g, &scale_h[g], 2);
+            memcpy(meta + 2 * ng + 2 * g, &zero_h[g], 2);
+        }
+    }
+}
+
+/* Read back the codes, scales and zeros of one stored row (inverse of
+ * pack_row). */
+void kvqo_read_row(const kvqo_config *c, const uint8_t *pool, int slot, int kvh, int tensor, int16_t *code,
+                   uint16_t *scale_h, uint16_t *zero_h)
+{
+    int d = c->head_dim;
+    int fmt = tensor ? c->v_fmt : c->k_fmt;
+    int group = tensor ? c->v_group : c->k_group;
+    int page = slot / KVQO_PAGE_TOKENS, tok = slot % KVQO_PAGE_TOKENS;
+    int rb = row_code_bytes(fmt, d);
+    uint8_t stream[KVQO_MAXD];
+    const uint8_t *codes = pool + region_base(c, page, kvh, tensor, 0);
+    for (int ch = 0; ch < rb / 16; ch++) memcpy(stream + ch * 16, codes + ((size_t)ch * 16 + tok) * 16, 16);
+    int bits = fmt_bits(fmt);
+    for (int i = 0; i < d; i++) {
+        unsigned v = (stream[(i * bits) / 8] >> ((i * bits) % 8)) & ((1u << bits) - 1u);
+        if (fmt == KVQO_INT8_SYM) code[i] = (int16_t)(int8_t)v;
+        else code[i] = (int16_t)v;
+    }
+    const uint8_t *meta = pool + region_base(c, page, kvh, tensor, 1) + (size_t)tok * row_meta_bytes(fmt, d, group);
+    if (fmt == KVQO_INT8_SYM) {
+        memcpy(&scale_h[0], meta, 2);
+        zero_h[0] = 0;
+    } else {
+        int ng = d / group;
+        for (int g = 0; g < ng; g++) {
+            memcpy(&scale_h[g], meta + 2 * g, 2);
+            memcpy(&zero_h[g], meta + 2 * ng + 2 * g, 2);
+        }
+    }
+}
+
+/* Dequantise one stored row in the rotated domain, fp64:
+ * asymmetric: code * scale + zero; int8: code * scale. */
+void kvqo_dequant_row(const kvqo_config *c, const uint8_t *pool, int slot, int kvh, int tensor, double *out)
+{
+    int d = c->head_dim;
+    int fmt = tensor ? c->v_fmt : c->k_fmt;
+    int group = tensor ? c->v_group : c->k_group;
+    int16_t code[KVQO_MAXD];
+    uint16_t sh[KVQO_MAXD], zh[KVQO_MAXD];
+    kvqo_read_row(c, pool, slot, kvh, tensor, code, sh, zh);
+    for (int i = 0; i < d; i++) {
+        if (fmt == KVQO_INT8_SYM) {
+            out[i] = (double)code[i] * (double)kvqo_h2f(sh[0]);
+        } else {
+            int g = i / group;
+            out[i] = (double)code[i] * (double)kvqo_h2f(sh[g]) + (double)kvqo_h2f(zh[g]);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Configuration check                                                       */
+/* ------------------------------------------------------------------------- */
+
+static int fmt_ok(int fmt, int group, int d)
+{
+    if (fmt == KVQO_INT8_SYM) return 1;
+    if (fmt != KVQO_INT4_ASYM && fmt != KVQO_INT2_ASYM) return 0;
+    if (group <= 0 || d % group) return 0;
+    return 1;
+}
+
+int kvqo_config_ok(const kvqo_config *c)
+{
+    int d = c->head_dim;
+    if (d != 64 && d != 128) return 0;
+    if (c->num_kv_heads <= 0 || c->num_q_heads <= 0 || c->num_q_heads % c->num_kv_heads) return 0;
+    if (c->page_tokens != KVQO_PAGE_TOKENS || c->num_pages <= 0) return 0;
+    if (!fmt_ok(c->k_fmt, c->k_group, d) || !fmt_ok(c->v_fmt, c->v_group, d)) return 0;
+    if (!(c->clip_ratio > 0.0f && c->clip_ratio <= 1.0f)) return 0;
+    if (c->bound_block_tokens < 0 || c->bound_block_tokens % KVQO_PAGE_TOKENS) return 0;
+    return 1;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Append: rotate + quantise + pack ([SRFT] Methodology 2, the fused path)   */
+/* ------------------------------------------------------------------------- */
+
+/* k, v: fp16 bits [n_tok][num_kv_heads][head_dim].  slot_mapping[n] < 0 skips
+ * token n.  Returns 0, or -1 for a slot outside the pool (nothing written for
+ * that token).  Also writes, when y_out is not NULL, the fp32 rotated rows
+ * [n_tok][num_kv_heads][2][head_dim] (K then V). */
+int kvqo_append(const kvqo_config *c, uint8_t *pool, const uint16_t *k, const uint16_t *v,
+                const int32_t *slot_mapping, int n_tok, float *y_out)
+{
+    if (!kvqo_config_ok(c)) return -2;
+    int d = c->head_dim, hkv = c->num_kv_heads;
+    float s[KVQO_MAXD], x[KVQO_MAXD], y[KVQO_MAXD];
+    kvqo_signs(c->rotation_seed, d, s);
+    int rc = 0;
+    for (int n = 0; n < n_tok; n++) {
+        int slot = slot_mapping[n];
+        if (slot < 0) continue;
+        if (slot >= c->num_pages * KVQO_PAGE_TOKENS) {
+            rc = -1;
+            continue;
+        }
+        int page = slot / KVQO_PAGE_TOKENS, tok = slot % KVQO_PAGE_TOKENS;
+        for (int kvh = 0; kvh < hkv; kvh++) {
+            for (int tensor = 0; tensor < 2; tensor++) {
+                const uint16_t *src = (tensor ? v : k) + ((size_t)n * hkv + kvh) * d;
+                int fmt = tensor ? c->v_fmt : c->k_fmt;
+                int group = tensor ? c->v_group : c->k_group;
+                for (int i = 0; i < d; i++) x[i] = kvqo_h2f(src[i]);
+                kvqo_rotate_f32(x, s, d, c->rotate, y);
+                if (y_out) memcpy(y_out + (((size_t)n * hkv + kvh) * 2 + tensor) * d, y, sizeof(float) * d);
+                int16_t code[KVQO_MAXD];
+                uint16_t sh[KVQO_MAXD], zh[KVQO_MAXD];
+                float emax, amax;
+                quantize_row(fmt, group, fmt == KVQO_INT8_SYM ? 1.0f : c->clip_ratio, y, d, code, sh, zh, &emax,
+                             &amax);
+                pack_row(c, pool, page, tok, kvh, tensor, code, sh, zh);
+                if (c->bound_block_tokens > 0) {
+                    float *desc = (float *)(pool + kvqo_desc_offset(c) + ((size_t)page * hkv + kvh) * 16);
+                    if (tensor == 0) {
+                        desc[0] = fmaxf(desc[0], emax);
+                    } else {
+                        desc[1] = fmaxf(desc[1], emax);
+                        desc[2] = fmaxf(desc[2], amax);
+                    }
+                }
+            }
+        }
+    }
+    return rc;
+}
+
+/* Dequantise stored rows: out [n][num_kv_heads][head_dim] fp64 (rotated
+ * domain); k_out or v_out may be NULL. */
+void kvqo_dequant(const kvqo_config *c, const uint8_t *pool, const int32_t *slots, int n, double *k_out, double *v_out)
+{
+    int d = c->head_dim, hkv = c->num_kv_heads;
+    for (int i = 0; i < n; i++)
+        for (int kvh = 0; kvh < hkv; kvh++) {
+            if (k_out) kvqo_dequant_row(c, pool, slots[i], kvh, 0, k_out + ((size_t)i * hkv + kvh) * d);
+            if (v_out) kvqo_dequant_row(c, pool, slots[i], kvh, 1, v_out + ((size_t)i * hkv + kvh) * d);
+        }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Attention (fp64)                                                          */
+/* ------------------------------------------------------------------------- */
+
+/* Softmax attention of one rotated query over T rotated keys/values, split
+ * into n_split contiguous token ranges whose partial states (m, l, acc) are
+ * merged by the log-sum-exp rule M = max m_i, L = sum e^{m_i-M} l_i,
+ * o = sum e^{m_i-M} acc_i / L.  n_split = 1 is the plain single pass.
+ * T = 0 gives the zero vector. */
+void kvqo_attend(const double *qr, const double *K, const double *V, int T, int d, double scale, int n_split,
+                 double *o)
+{
+    for (int i = 0; i < d; i++) o[i] = 0.0;
+    if (T <= 0) return;
+    if (n_split < 1) n_split = 1;
+    if (n_split > T) n_split = T;
+    double *acc = (double *)calloc((size_t)n_split * d, sizeof(double));
+    double *m = (double *)malloc(sizeof(double) * n_split);
+    double *l = (double *)calloc((size_t)n_split, sizeof(double));
+    double *sc = (double *)malloc(sizeof(double) * T);
+    for (int t = 0; t < T; t++) {
+        double dot = 0.0;
+        for (int i = 0; i < d; i++) dot += qr[i] * K[(size_t)t * d + i];
+        sc[t] = scale * dot;
+    }
+    for (int sp = 0; sp < n_split; sp++) {
+        int t0 = (int)((long long)T * sp / n_split), t1 = (int)((long long)T * (sp + 1) / n_split);
+        double mx = -INFINITY;
+        for (int t = t0; t < t1; t++) mx = fmax(mx, sc[t]);
+        m[sp] = mx;
+        for (int t = t0; t < t1; t++) {
+            double p = exp(sc[t] - mx);
+            l[sp] += p;
+            for (int i = 0; i < d; i++) acc[(size_t)sp * d + i] += p * V[(size_t)t * d + i];
+        }
+    }
+    double M = -INFINITY;
+    for (int sp = 0; sp < n_split; sp++) M = fmax(M, m[sp]);
+    double L = 0.0;
+    for (int sp = 0; sp < n_split; sp++) L += exp(m[sp] - M) * l[sp];
+    for (int sp = 0; sp < n_split; sp++) {
+        double w = exp(m[sp] - M) / L;
+        for (int i = 0; i < d; i++) o[i] += w * acc[(size_t)sp * d + i];
+    }
+    free(acc);
+    free(m);
+    free(l);
+    free(sc);
+}
+
+static int slot_of(const int32_t *block_table, int max_pages, int b, int t)
+{
+    return block_table[(size_t)b * max_pages + t / KVQO_PAGE_TOKENS] * KVQO_PAGE_TOKENS + t % KVQO_PAGE_TOKENS;
+}
+
+static int decode_args_ok(const kvqo_config *c, const int32_t *block_table, int max_pages, const int32_t *ctx_lens,
+                          int B)
+{
+    for (int b = 0; b < B; b++) {
+        int T = ctx_lens[b];
+        if (T < 0 || T > max_pages * KVQO_PAGE_TOKENS) return 0;
+        for (int p = 0; p < (T + KVQO_PAGE_TOKENS - 1) / KVQO_PAGE_TOKENS; p++) {
+            int pg = block_table[(size_t)b * max_pages + p];
+            if (pg < 0 || pg >= c->num_pages) return 0;
+        }
+    }
+    return 1;
+}
+
+/* Decode attention over the quantised cache ([OSCAR] 2.2b fused kernel:
+ * unpack, dequantise, attention, inverse rotation; the split/LSE merge is the
+ * flash-decoding form the hot path uses).  Per sequence b and query head h:
+ *   kv head = h / (Hq/Hkv) (contiguous grouping; the pages are silent),
+ *   q_r = R q, s_t = scale * q_r . khat_t for t in [0, ctx_lens[b]) read
+ *   through the block table, p = softmax(s), o = R^T sum_t p_t vhat_t.
+ * q: fp16 bits [B][Hq][d]; out: fp64 [B][Hq][d].  scale <= 0 means 1/sqrt(d).
+ * sel (optional, [B][Hkv]) restricts the work to the flagged pairs; rows of
+ * other pairs are left untouched.  Returns 0, or -1 for a bad table/length. */
+int kvqo_decode(const kvqo_config *c, const uint8_t *pool, const uint16_t *q, const int32_t *block_table,
+                int max_pages, const int32_t *ctx_lens, int B, double scale, int n_split, const int32_t *sel,
+                double *out)
+{
+    if (!kvqo_config_ok(c)) return -2;
+    if (!decode_args_ok(c, block_table, max_pages, ctx_lens, B)) return -1;
+    int d = c->head_dim, hq = c->num_q_heads, hkv = c->num_kv_heads, g = hq / hkv;
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    float s[KVQO_MAXD];
+    kvqo_signs(c->rotation_seed, d, s);
+    for (int b = 0; b < B; b++) {
+        int T = ctx_lens[b];
+        for (int kvh = 0; kvh < hkv; kvh++) {
+            if (sel && !sel[b * hkv + kvh]) continue;
+            double *K = (double *)malloc(sizeof(double) * ((size_t)T * d + 1));
+            double *V = (double *)malloc(sizeof(double) * ((size_t)T * d + 1));
+            for (int t = 0; t < T; t++) {
+                int slot = slot_of(block_table, max_pages, b, t);
+                kvqo_dequant_row(c, pool, slot, kvh, 0, K + (size_t)t * d);
+                kvqo_dequant_row(c, pool, slot, kvh, 1, V + (size_t)t * d);
+            }
+            for (int hh = 0; hh < g; hh++) {
+                int h = kvh * g + hh;
+                double qx[KVQO_MAXD], qr[KVQO_MAXD], orot[KVQO_MAXD];
+                for (int i = 0; i < d; i++) qx[i] = (double)kvqo_h2f(q[((size_t)b * hq + h) * d + i]);
+                kvqo_rotate_f64(qx, s, d, c->rotate, qr);
+                kvqo_attend(qr, K, V, T, d, scale, n_split, orot);
+                kvqo_inv_rotate_f64(orot, s, d, c->rotate, out + ((size_t)b * hq + h) * d);
+            }
+            free(K);
+            free(V);
+        }
+    }
+    return 0;
+}
+
+/* Unquantised reference: softmax attention in fp64 over fp16 K/V rows stored
+ * per slot ([num_slots][Hkv][d]) with no rotation -- the quality yardstick
+ * ([CERT] Methodology 1: the fp16 originals are the ground truth). */
+int kvqo_decode_fp16(const kvqo_config *c, const uint16_t *k_slots, const uint16_t *v_slots, const uint16_t *q,
+                     const int32_t *block_table, int max_pages, const int32_t *ctx_lens, int B, double scale,
+                     const int32_t *sel, double *out)
+{
+    if (!decode_args_ok(c, block_table, max_pages, ctx_lens, B)) return -1;
+    int d = c->head_dim, hq = c->num_q_heads, hkv = c->num_kv_heads, g = hq / hkv;
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    for (int b = 0; b < B; b++) {
+        int T = ctx_lens[b];
+        for (int kvh = 0; kvh < hkv; kvh++) {
+            if (sel && !sel[b * hkv + kvh]) continue;
+            double *K = (double *)malloc(sizeof(double) * ((size_t)T * d + 1));
+            double *V = (double *)malloc(sizeof(double) * ((size_t)T * d + 1));
+            for (int t = 0; t < T; t++) {
+                size_t row = ((size_t)slot_of(block_table, max_pages, b, t) * hkv + kvh) * d;
+                for (int i = 0; i < d; i++) {
+                    K[(size_t)t * d + i] = kvqo_h2f(k_slots[row + i]);
+                    V[(size_t)t * d + i] = kvqo_h2f(v_slots[row + i]);
+                }
+            }
+            for (int hh = 0; hh < g; hh++) {
+                int h = kvh * g + hh;
+                double qx[KVQO_MAXD];
+                for (int i = 0; i < d; i++) qx[i] = (double)kvqo_h2f(q[((size_t)b * hq + h) * d + i]);
+                kvqo_attend(qx, K, V, T, d, scale, 1, out + ((size_t)b * hq + h) * d);
+            }
+            free(K);
+            free(V);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Certified decode ([CERT] Methodology 1-3)                                 */
+/* ------------------------------------------------------------------------- */
+
+/* Number of blocks promoted out of n_blocks: ceil(frac * n_blocks), computed
+ * in fp64 with a 1e-9 guard so an exact product is not bumped up by rounding,
+ * clamped to [0, n_blocks]. */
+int kvqo_promote_count(double frac, int n_blocks)
+{
+    if (frac <= 0.0 || n_blocks <= 0) return 0;
+    int k = (int)ceil(frac * (double)n_blocks - 1e-9);
+    if (k < 0) k = 0;
+    if (k > n_blocks) k = n_blocks;
+    return k;
+}
+
+/* Per-block bound, in the rotated domain, for one query head.  Reading of
+ * [CERT] Methodology 2 (the pages give the two terms but print no formula):
+ *   Delta_b = scale * ||q_r||_1 * eps_b        (eps_b: max |k - khat| in b)
+ *   P_b     = sum_{t in b} phat_t               (mass under quantised scores)
+ *   A       = ln sum_b P_b e^{Delta_b}
+ *   bound_b = P_b * ((e^{Delta_b + A} - 1) * nu_b + eta_b)
+ * with eta_b = max |v - vhat| and nu_b = max |v| over the block.  Then
+ * ||o_r,exact - o_r,quant||_inf <= sum_b bound_b: the key term bounds the
+ * total-variation shift of the softmax (p_t/phat_t = e^{delta_t}/Z with
+ * e^{-A} <= Z <= e^{A} by Jensen), the value term is the mass-weighted
+ * reconstruction error. */
+static void block_bounds_one_head(const double *phat, int T, int block, const double *eps, const double *eta,
+                                  const double *nu, double qnorm1, double scale, double *bound)
+{
+    int nb = (T + block - 1) / block;
+    double *P = (double *)calloc((size_t)nb + 1, sizeof(double));
+    for (int t = 0; t < T; t++) P[t / block] += phat[t];
+    double sumexp = 0.0;
+    for (int b = 0; b < nb; b++) sumexp += P[b] * exp(scale * qnorm1 * eps[b]);
+    double A = log(sumexp);
+    for (int b = 0; b < nb; b++) {
+        double Db = scale * qnorm1 * eps[b];
+        bound[b] = P[b] * ((exp(Db + A) - 1.0) * nu[b] + eta[b]);
+    }
+    free(P);
+}
+
+/* Certified decode.  For every (sequence, kv head): compute per-block bounds
+ * for each query head of the group, score each block by the largest of them,
+ * promote the top ceil(frac * n_blocks) blocks (ties to the lower block index;
+ * a partial last block counts) to their exact fp16 originals from tier 2
+ * (rotated in fp64), and run attention with promoted blocks exact and all
+ * others dequantised.  k_slots/v_slots: tier-2 fp16 rows [num_slots][Hkv][d].
+ * promoted (optional): [B][Hkv][max_promote] block indices in descending score
+ * order, -1 padded.  score_out (optional): [B][Hkv][max_blocks].
+ * bound_sum_out (optional): [B][Hq], sum_b bound_b of each head (all blocks
+ * quantised).  quant_out (optional): [B][Hq][d] the plain quantised output. */
+int kvqo_decode_certified(const kvqo_config *c, const uint8_t *pool, const uint16_t *k_slots,
+                          const uint16_t *v_slots, const uint16_t *q, const int32_t *block_table, int max_pages,
+                          const int32_t *ctx_lens, int B, double scale, double frac, const int32_t *sel,
+                          double *out, int32_t *promoted, int max_promote, double *score_out, int max_blocks,
+                          double *bound_sum_out)
+{
+    if (!kvqo_config_ok(c) || c->bound_block_tokens <= 0) return -2;
+    if (!decode_args_ok(c, block_table, max_pages, ctx_lens, B)) return -1;
+    int d = c->head_dim, hq = c->num_q_heads, hkv = c->num_kv_heads, g = hq / hkv;
+    int block = c->bound_block_tokens;
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    float s[KVQO_MAXD];
+    kvqo_signs(c->rotation_seed, d, s);
+    for (int b = 0; b < B; b++) {
+        int T = ctx_lens[b];
+        int nb = (T + block - 1) / block;
+        for (int kvh = 0; kvh < hkv; kvh++) {
+            if (sel && !sel[b * hkv + kvh]) continue;
+            size_t n = (size_t)T * d + 1;
+            double *K = (double *)malloc(sizeof(double) * n), *V = (double *)malloc(sizeof(double) * n);
+            double *eps = (double *)calloc((size_t)nb + 1, sizeof(double));
+            double *eta = (double *)calloc((size_t)nb + 1, sizeof(double));
+            double *nu = (double *)calloc((size_t)nb + 1, sizeof(double));
+            double *score = (double *)calloc((size_t)nb + 1, sizeof(double));
+            double *bound = (double *)calloc((size_t)nb + 1, sizeof(double));
+            double *phat = (double *)malloc(sizeof(double) * ((size_t)T + 1));
+            double *sc = (double *)malloc(sizeof(double) * ((size_t)T + 1));
+            for (int t = 0; t < T; t++) {
+                int slot = slot_of(block_table, max_pages, b, t);
+                kvqo_dequant_row(c, pool, slot, kvh, 0, K + (size_t)t * d);
+                kvqo_dequant_row(c, pool, slot, kvh, 1, V + (size_t)t * d);
+            }
+            /* block descriptors: max over the block's pages */
+            for (int p = 0; p < (T + KVQO_PAGE_TOKENS - 1) / KVQO_PAGE_TOKENS; p++) {
+                int pg = block_table[(size_t)b * max_pages + p];
+                const float *desc = (const float *)(pool + kvqo_desc_offset(c) + ((size_t)pg * hkv + kvh) * 16);
+                int blk = p * KVQO_PAGE_TOKENS / block;
+                eps[blk] = fmax(eps[blk], (double)desc[0]);
+                eta[blk] = fmax(eta[blk], (double)desc[1]);
+                nu[blk] = fmax(nu[blk], (double)desc[2]);
+            }
+            double qr[16][KVQO_MAXD];
+            for (int hh = 0; hh < g && hh < 16; hh++) {
+                int h = kvh * g + hh;
+                double qx[KVQO_MAXD], qn = 0.0;
+                for (int i = 0; i < d; i++) qx[i] = (double)kvqo_h2f(q[((size_t)b * hq + h) * d + i]);
+                kvqo_rotate_f64(qx, s, d, c->rotate, qr[hh]);
+                for (int i = 0; i < d; i++) qn += fabs(qr[hh][i]);
+                double mx = -INFINITY, L = 0.0;
+                for (int t = 0; t < T; t++) {
+                    double dot = 0.0;
+                    for (int i = 0; i < d; i++) dot += qr[hh][i] * K[(size_t)t * d + i];
+                    sc[t] = scale * dot;
+                    mx = fmax(mx, sc[t]);
+                }
+                for (int t = 0; t < T; t++) L += exp(sc[t] - mx);
+                for (int t = 0; t < T; t++) phat[t] = exp(sc[t] - mx) / L;
+                block_bounds_one_head(phat, T, block, eps, eta, nu, qn, scale, bound);
+                double bs = 0.0;
+                for (int bb = 0; bb < nb; bb++) {
+                    score[bb] = (hh == 0) ? bound[bb] : fmax(score[bb], bound[bb]);
+                    bs += bound[bb];
+                }
+                if (bound_sum_out) bound_sum_out[(size_t)b * hq + h] = bs;
+            }
+            if (score_out)
+                for (int bb = 0; bb < nb && bb < max_blocks; bb++) score_out[((size_t)b * hkv + kvh) * max_blocks + bb] = score[bb];
+            /* selection: top k by score, ties to the lower index */
+            int k = kvqo_promote_count(frac, nb);
+            char *taken = (char *)calloc((size_t)nb + 1, 1);
+            for (int r = 0; r < k; r++) {
+                int best = -1;
+                for (int bb = 0; bb < nb; bb++)
+                    if (!taken[bb] && (best < 0 || score[bb] > score[best])) best = bb;
+                taken[best] = 1;
+                if (promoted && r < max_promote) promoted[((size_t)b * hkv + kvh) * max_promote + r] = best;
+            }
+            if (promoted)
+                for (int r = k; r < max_promote; r++) promoted[((size_t)b * hkv + kvh) * max_promote + r] = -1;
+            /* promoted blocks use the exact rotated fp16 originals */
+            for (int t = 0; t < T; t++) {
+                if (!taken[t / block]) continue;
+                int slot = slot_of(block_table, max_pages, b, t);
+                double xk[KVQO_MAXD], xv[KVQO_MAXD];
+                size_t row = ((size_t)slot * hkv + kvh) * d;
+                for (int i = 0; i < d; i++) {
+                    xk[i] = kvqo_h2f(k_slots[row + i]);
+                    xv[i] = kvqo_h2f(v_slots[row + i]);
+                }
+                kvqo_rotate_f64(xk, s, d, c->rotate, K + (size_t)t * d);
+                kvqo_rotate_f64(xv, s, d, c->rotate, V + (size_t)t * d);
+            }
+            for (int hh = 0; hh < g; hh++) {
+                int h = kvh * g + hh;
+                double orot[KVQO_MAXD];
+                kvqo_attend(qr[hh], K, V, T, d, scale, 1, orot);
+                kvqo_inv_rotate_f64(orot, s, d, c->rotate, out + ((size_t)b * hq + h) * d);
+            }
+            free(taken);
+            free(K);
+            free(V);
+            free(eps);
+            free(eta);
+            free(nu);
+            free(score);
+            free(bound);
+            free(phat);
+            free(sc);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Array helpers for the tests                                               */
+/* ------------------------------------------------------------------------- */
+
+void kvqo_f2h_rn_n(const float *x, uint16_t *h, size_t n)
+{
+    for (size_t i = 0; i < n; i++) h[i] = kvqo_f2h_rn(x[i]);
+}
+
+void kvqo_f2h_ru_n(const float *x, uint16_t *h, size_t n)
+{
+    for (size_t i = 0; i < n; i++) h[i] = kvqo_f2h_ru(x[i]);
+}
+
+void kvqo_h2f_n(const uint16_t *h, float *x, size_t n)
+{
+    for (size_t i = 0; i < n; i++) x[i] = kvqo_h2f(h[i]);
+}
+
+/* Quantise already-rotated rows y[n][d] on their own (no pool): codes
+ * [n][d], scales/zeros [n][d/group] (int8: one scale per row). */
+void kvqo_quantize_rows(int fmt, int group, float clip, const float *y, int n, int d, int16_t *code,
+                        uint16_t *scale_h, uint16_t *zero_h, float *err_max, float *abs_max)
+{
+    int ng = (fmt == KVQO_INT8_SYM) ? 1 : d / group;
+    for (int r = 0; r < n; r++)
+        quantize_row(fmt, group, fmt == KVQO_INT8_SYM ? 1.0f : clip, y + (size_t)r * d, d, code + (size_t)r * d,
+                     scale_h + (size_t)r * ng, zero_h + (size_t)r * ng, err_max + r, abs_max + r);
+}
