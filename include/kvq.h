@@ -1,0 +1,169 @@
+/*
+ * kvq.h -- C ABI of the B200 low-bit KV cache: quantise-on-append of K/V and
+ * split-K decode attention over the packed, paged cache.
+ *
+ * What the calls compute (page titles and sections):
+ *  - Rotation: R = c_d * H_d * diag(s), a fixed random sign vector s followed by
+ *    the (Sylvester) Walsh-Hadamard transform, c_d = fp32(1/sqrt(d))
+ *    ["When Quantization Is Free", Methodology 1 (random-sign rotation, SRHT);
+ *    "OSCAR", 2.2 (Hadamard factor of the rotation)].
+ *  - Codec: per-group asymmetric int4 (group 32) and int2 (group = head_dim,
+ *    optional clip ratio) with fp16 scale and fp16 zero; symmetric int8 per
+ *    token-head with an fp16 scale ["When Quantization Is Free", Methodology 2
+ *    (per-group scaling, rounding, nibble packing); "Runtime-Certified
+ *    Bounded-Error Quantized Attention", Methodology 1 (INT8 keys, INT4 values,
+ *    scales/offsets); "OSCAR", 2.2 (INT2 history, clipping thresholds)].
+ *  - Decode: softmax attention of one new query per sequence over the paged
+ *    cache, dequantised in registers, merged across context splits by the
+ *    log-sum-exp rule, inverse-rotated ["OSCAR", 2.2b (fused kernel: unpack,
+ *    dequantise, inverse rotation, attention over a paged cache)].
+ *  - Certified mode: per-block key/value error bounds, top-fraction promotion
+ *    of blocks to their fp16 originals held in pinned host memory
+ *    ["Runtime-Certified Bounded-Error Quantized Attention", Methodology 1-3].
+ *
+ * Conventions for every call:
+ *  - All tensors are caller-owned device memory unless stated (the library
+ *    never allocates device memory).  fp16 tensors are passed as void*.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call is asynchronous on that stream and never synchronises, except
+ *    kvq_create_cache (zero-fills the pool) and kvq_sync_status.
+ *  - Argument checks run on the host before any launch; a failed check returns
+ *    an error status and launches nothing.  A failed launch returns
+ *    KVQ_ERR_CUDA.  Conditions only the device can see (a block-table entry or
+ *    slot outside the pool, a bounded wait that ran out) are recorded in a
+ *    status word inside the pool; kvq_sync_status reports and clears it.
+ *  - Calls on one cache are not thread-safe with respect to each other.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1,  /* NULL pointer, bad size, misaligned buffer     */
+    KVQ_ERR_UNSUPPORTED = 2,  /* valid but not built (format/head_dim/GQA mix)  */
+    KVQ_ERR_CAPACITY = 3,     /* pool or workspace smaller than required        */
+    KVQ_ERR_OUT_OF_RANGE = 4, /* device saw a slot/page index outside the pool  */
+    KVQ_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed           */
+    KVQ_ERR_TIMEOUT = 6       /* a bounded device-side wait ran out             */
+} kvq_status;
+
+typedef enum {
+    KVQ_INT4_ASYM = 0, /* 4-bit codes, group 32, fp16 scale + fp16 zero         */
+    KVQ_INT8_SYM = 1,  /* 8-bit signed codes, one fp16 scale per token-head     */
+    KVQ_INT2_ASYM = 2  /* 2-bit codes, group = head_dim, fp16 scale + fp16 zero */
+} kvq_fmt;
+
+typedef struct {
+    int32_t num_q_heads;        /* Hq; Hq / Hkv (the GQA group) must be 1..8          */
+    int32_t num_kv_heads;       /* Hkv                                                */
+    int32_t head_dim;           /* d: 64 or 128                                       */
+    int32_t k_fmt, v_fmt;       /* kvq_fmt of keys / values (values: int4 or int2)    */
+    int32_t k_group, v_group;   /* int4: 32; int2: head_dim; int8: head_dim           */
+    float clip_ratio;           /* (0, 1]; scales both ends of int2/int4 groups       */
+    uint64_t rotation_seed;     /* SplitMix64 state that draws the sign vector        */
+    int32_t rotate;             /* 1 = sign + Hadamard rotation, 0 = identity         */
+    int32_t page_tokens;        /* tokens per page; must be 16                        */
+    int32_t num_pages;          /* pages in the pool                                  */
+    int32_t bound_block_tokens; /* 0 = no error descriptors; else a multiple of 16    */
+} kvq_config;
+
+typedef struct kvq_cache kvq_cache; /* opaque; owned by the library */
+
+/* Tier-2 store of the certified mode: the original fp16 K and V rows indexed
+ * by slot, [num_pages*16][Hkv][d] each, in pinned host memory mapped into the
+ * device address space (the pointers given must be device-accessible, e.g.
+ * from cudaHostGetDevicePointer).  The caller keeps it current (it is the
+ * ground truth the pages call tier 2). */
+typedef struct {
+    const void *k_host;
+    const void *v_host;
+    float promote_frac; /* fraction of bound blocks per (seq, kv head) promoted */
+} kvq_tier2;
+
+/* Bytes of device memory the pool of `cfg` needs; 0 if cfg is invalid.
+ * Layout: [256-byte header][num_pages pages][descriptors].  A page holds
+ * num_kv_heads chunks [K codes][K meta][V codes][V meta] of 16 tokens.  Codes
+ * of a token are its sequential bit stream (int4: byte j = code[2j] |
+ * code[2j+1] << 4; int2: four codes per byte from the low bits up; int8:
+ * two's complement) cut into 16-byte chunks stored chunk-major, chunk c of
+ * token t at (c*16 + t)*16, so one 16-byte load is a whole int4 group.  Meta
+ * rows are fp16 scales then fp16 zeros (int8: one scale).  Descriptors (when
+ * bound_block_tokens > 0): per (page, kv head) four fp32 {max key error, max
+ * value error, max |value|, 0}. */
+size_t kvq_pool_bytes(const kvq_config *cfg);
+
+/* Create a cache over caller-owned device memory `pool_dev` of `pool_bytes`
+ * (>= kvq_pool_bytes, 256-byte aligned).  Zero-fills the pool (synchronous)
+ * and draws the sign vector from rotation_seed.  *out receives the handle. */
+kvq_status kvq_create_cache(const kvq_config *cfg, void *pool_dev, size_t pool_bytes, kvq_cache **out);
+
+/* Release the handle (the pool memory stays the caller's). */
+kvq_status kvq_destroy_cache(kvq_cache *cache);
+
+/* Quantise-on-append ["When Quantization Is Free", Methodology 2]: rotate,
+ * quantise and pack n_tok tokens of k and v (fp16, [n_tok][Hkv][d], 16-byte
+ * aligned) into the slots slot_mapping[0..n_tok) (int32, device).  A negative
+ * slot skips the token; a slot >= num_pages*16 is skipped and recorded as
+ * KVQ_ERR_OUT_OF_RANGE in the status word.  With descriptors on, each row's
+ * max |k - khat|, max |v - vhat| and max |v| are max-reduced into its page's
+ * descriptor (reset a page with kvq_reset_pages before reusing it). */
+kvq_status kvq_append(kvq_cache *cache, const void *k, const void *v, const int32_t *slot_mapping, int32_t n_tok,
+                      void *stream);
+
+/* Zero the descriptors of n pages listed in page_ids (int32, device). */
+kvq_status kvq_reset_pages(kvq_cache *cache, const int32_t *page_ids, int32_t n, void *stream);
+
+/* Workspace bytes kvq_decode_attn needs for `batch` sequences with block
+ * tables of max_pages_per_seq entries.  The workspace must be zero-filled
+ * before its first use; every decode call leaves it ready for the next one. */
+size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int32_t batch, int32_t max_pages_per_seq);
+
+/* Decode attention ["OSCAR", 2.2b]: for each sequence b and query head h,
+ * out[b][h] = R^T softmax(scale * (R q[b][h]) . khat_t) . vhat_t over the
+ * ctx_lens[b] tokens whose pages block_table[b][0..] lists (16 tokens a page),
+ * with kv head h / (Hq/Hkv).
+ *   q:           fp16 [batch][Hq][d] (device)
+ *   block_table: int32 [batch][max_pages_per_seq] (device)
+ *   ctx_lens:    int32 [batch] (device), 0 <= ctx_lens[b] <= 16*max_pages_per_seq
+ *   softmax_scale: <= 0 means 1/sqrt(d)
+ *   tier2:       NULL, or the certified-mode store (needs bound_block_tokens)
+ *   workspace:   >= kvq_decode_workspace_bytes, zero-filled before first use;
+ *                one workspace must not serve two decode calls that overlap
+ *   out:         fp16 [batch][Hq][d] (device)
+ *   promoted_out (certified mode, optional): int32 [batch][Hkv][kmax] block
+ *                indices promoted, highest bound first, -1 padded, where
+ *                kmax = ceil(promote_frac * ceil(16*max_pages_per_seq / block)).
+ * An empty context gives a zero output row. */
+kvq_status kvq_decode_attn(kvq_cache *cache, const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
+                           const int32_t *ctx_lens, int32_t batch, float softmax_scale, const kvq_tier2 *tier2,
+                           void *workspace, size_t ws_bytes, void *out, int32_t *promoted_out, void *stream);
+
+/* Read back n stored rows (slots[0..n), int32 device) per kv head:
+ *   k_out, v_out: fp32 [n][Hkv][d] rotated-domain dequantised values
+ *                 (code*scale + zero, one rounding), may be NULL;
+ *   codes_out:    uint8 [n][Hkv][2][d] codes in channel order (K then V;
+ *                 int8 as two's complement), may be NULL;
+ *   meta_out:     uint16 [n][Hkv][2][8] fp16 scales in [0,4) and zeros in
+ *                 [4,8) (unused entries 0), may be NULL. */
+kvq_status kvq_dequant_debug(kvq_cache *cache, const int32_t *slots, int32_t n, float *k_out, float *v_out,
+                             uint8_t *codes_out, uint16_t *meta_out, void *stream);
+
+/* Synchronise the cache's last stream use and return (then clear) the device
+ * status word: KVQ_OK, KVQ_ERR_OUT_OF_RANGE or KVQ_ERR_TIMEOUT. */
+kvq_status kvq_sync_status(kvq_cache *cache);
+
+/* Static description of a status code. */
+const char *kvq_status_string(kvq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -1,0 +1,262 @@
+// kvq_api.cu -- the C ABI: argument checks on the host, cache handle, kernel
+// launches on the caller's stream, workspace sizing and the status word.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "kvq_internal.cuh"
+
+using namespace kvq;
+
+namespace {
+
+// SplitMix64 (Steele, Lea & Flood 2014): add the golden-ratio increment to the
+// state, then two xor-shift-multiply rounds and a final xor-shift.
+uint64_t splitmix64_next(uint64_t &state)
+{
+    uint64_t z = (state += 0x9E3779B97F4A7C15ULL);
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+    return z ^ (z >> 31);
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+kvq_status check_config(const kvq_config *c)
+{
+    if (!c) return KVQ_ERR_INVALID_ARG;
+    if (c->head_dim != 64 && c->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+    if (c->num_kv_heads <= 0 || c->num_q_heads <= 0 || c->num_q_heads % c->num_kv_heads) return KVQ_ERR_INVALID_ARG;
+    if (c->num_q_heads / c->num_kv_heads > kMaxGqa) return KVQ_ERR_UNSUPPORTED;
+    if (c->page_tokens != kPageTokens) return KVQ_ERR_UNSUPPORTED;
+    if (c->num_pages <= 0) return KVQ_ERR_INVALID_ARG;
+    const int fmts[2] = {c->k_fmt, c->v_fmt}, groups[2] = {c->k_group, c->v_group};
+    for (int t = 0; t < 2; t++) {
+        switch (fmts[t]) {
+        case KVQ_INT4_ASYM:
+            if (groups[t] != 32) return KVQ_ERR_UNSUPPORTED;
+            break;
+        case KVQ_INT2_ASYM:
+            if (groups[t] != c->head_dim) return KVQ_ERR_UNSUPPORTED;
+            break;
+        case KVQ_INT8_SYM:
+            if (t == 1) return KVQ_ERR_UNSUPPORTED;  // values: int4 or int2
+            if (groups[t] != c->head_dim) return KVQ_ERR_UNSUPPORTED;
+            break;
+        default: return KVQ_ERR_INVALID_ARG;
+        }
+    }
+    if (!(c->clip_ratio > 0.0f && c->clip_ratio <= 1.0f)) return KVQ_ERR_INVALID_ARG;
+    if (c->bound_block_tokens < 0 || c->bound_block_tokens % kPageTokens) return KVQ_ERR_INVALID_ARG;
+    if (c->rotate != 0 && c->rotate != 1) return KVQ_ERR_INVALID_ARG;
+    return KVQ_OK;
+}
+
+struct SplitPlan {
+    int pages_per_warp, pages_per_split, n_splits;
+};
+
+// Split the context so that the largest sequence fills about two CTAs per SM
+// when every sequence is as long as the block table allows.
+SplitPlan plan_splits(const kvq_cache *c, int batch, int max_pages)
+{
+    SplitPlan s{};
+    const long long work = (long long)batch * c->L.hkv * max_pages;
+    const long long target = 2LL * c->num_sms;
+    long long per_cta = (work + target - 1) / target;
+    if (per_cta < 1) per_cta = 1;
+    s.pages_per_warp = (int)((per_cta + kDecodeWarps - 1) / kDecodeWarps);
+    s.pages_per_split = s.pages_per_warp * kDecodeWarps;
+    s.n_splits = (max_pages + s.pages_per_split - 1) / s.pages_per_split;
+    if (s.n_splits < 1) s.n_splits = 1;
+    return s;
+}
+
+size_t counters_bytes(int batch, int hkv) { return ((size_t)batch * hkv * 4 + 255) / 256 * 256; }
+
+kvq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t kvq_pool_bytes(const kvq_config *cfg)
+{
+    if (check_config(cfg) != KVQ_OK) return 0;
+    const Layout L = make_layout(*cfg);
+    size_t n = kHeaderBytes + (size_t)cfg->num_pages * L.page_bytes;
+    if (cfg->bound_block_tokens > 0) n += (size_t)cfg->num_pages * cfg->num_kv_heads * 16;
+    return n;
+}
+
+kvq_status kvq_create_cache(const kvq_config *cfg, void *pool_dev, size_t pool_bytes, kvq_cache **out)
+{
+    if (!out) return KVQ_ERR_INVALID_ARG;
+    *out = nullptr;
+    const kvq_status st = check_config(cfg);
+    if (st != KVQ_OK) return st;
+    if (!pool_dev || !aligned(pool_dev, 256)) return KVQ_ERR_INVALID_ARG;
+    if (pool_bytes < kvq_pool_bytes(cfg)) return KVQ_ERR_CAPACITY;
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, pool_dev) != cudaSuccess) {
+        cudaGetLastError();
+        return KVQ_ERR_INVALID_ARG;
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return KVQ_ERR_INVALID_ARG;
+
+    kvq_cache *c = new (std::nothrow) kvq_cache();
+    if (!c) return KVQ_ERR_CUDA;
+    c->cfg = *cfg;
+    c->L = make_layout(*cfg);
+    c->pool = static_cast<unsigned char *>(pool_dev);
+    c->pool_bytes = pool_bytes;
+    c->device = attr.device;
+    c->last_stream = nullptr;
+    if (cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
+        delete c;
+        return KVQ_ERR_CUDA;
+    }
+    // sign vector: s_i = -1 when the top bit of the i-th SplitMix64 output is set
+    uint64_t state = cfg->rotation_seed;
+    for (int i = 0; i < cfg->head_dim; i++) c->signs[i] = (splitmix64_next(state) >> 63) ? -1.0f : 1.0f;
+    for (int i = cfg->head_dim; i < kMaxD; i++) c->signs[i] = 1.0f;
+    for (int w = 0; w < kMaxD / 2; w++)
+        c->sign_xor[w] = (c->signs[2 * w] < 0 ? 0x00008000u : 0u) | (c->signs[2 * w + 1] < 0 ? 0x80000000u : 0u);
+    c->rot_scale = (float)(1.0 / sqrt((double)cfg->head_dim));
+    if (cudaMemset(pool_dev, 0, kvq_pool_bytes(cfg)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        delete c;
+        return KVQ_ERR_CUDA;
+    }
+    *out = c;
+    return KVQ_OK;
+}
+
+kvq_status kvq_destroy_cache(kvq_cache *cache)
+{
+    if (!cache) return KVQ_ERR_INVALID_ARG;
+    delete cache;
+    return KVQ_OK;
+}
+
+kvq_status kvq_append(kvq_cache *c, const void *k, const void *v, const int32_t *slot_mapping, int32_t n_tok,
+                      void *stream)
+{
+    if (!c || n_tok < 0) return KVQ_ERR_INVALID_ARG;
+    if (n_tok == 0) return KVQ_OK;
+    if (!k || !v || !slot_mapping || !aligned(k, 16) || !aligned(v, 16) || !aligned(slot_mapping, 4))
+        return KVQ_ERR_INVALID_ARG;
+    AppendParams p{};
+    p.k = static_cast<const __half *>(k);
+    p.v = static_cast<const __half *>(v);
+    p.slots = slot_mapping;
+    p.n_tok = n_tok;
+    p.pool = c->pool;
+    p.L = c->L;
+    p.clip = c->cfg.clip_ratio;
+    p.rot_scale = c->rot_scale;
+    p.rotate = c->cfg.rotate;
+    memcpy(p.sign_xor, c->sign_xor, sizeof(p.sign_xor));
+    c->last_stream = stream;
+    return cuda_status(launch_append(p, c->cfg.k_group, c->cfg.v_group, static_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_reset_pages(kvq_cache *c, const int32_t *page_ids, int32_t n, void *stream)
+{
+    if (!c || n < 0 || (n > 0 && !page_ids)) return KVQ_ERR_INVALID_ARG;
+    if (n == 0 || c->L.desc_off == 0) return KVQ_OK;
+    c->last_stream = stream;
+    return cuda_status(launch_reset_pages(c->pool, c->L, page_ids, n, static_cast<cudaStream_t>(stream)));
+}
+
+size_t kvq_decode_workspace_bytes(const kvq_cache *c, int32_t batch, int32_t max_pages_per_seq)
+{
+    if (!c || batch < 0 || max_pages_per_seq < 1) return 0;
+    const SplitPlan s = plan_splits(c, batch, max_pages_per_seq);
+    const size_t part = (size_t)batch * c->L.hkv * s.n_splits * c->L.g * (c->L.d + 4) * sizeof(float);
+    return counters_bytes(batch, c->L.hkv) + part;
+}
+
+kvq_status kvq_decode_attn(kvq_cache *c, const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
+                           const int32_t *ctx_lens, int32_t batch, float softmax_scale, const kvq_tier2 *tier2,
+                           void *workspace, size_t ws_bytes, void *out, int32_t *promoted_out, void *stream)
+{
+    (void)promoted_out;
+    if (!c || batch < 0 || max_pages_per_seq < 1) return KVQ_ERR_INVALID_ARG;
+    if (batch == 0) return KVQ_OK;
+    if (!q || !block_table || !ctx_lens || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
+    if (!decode_supported(c->L)) return KVQ_ERR_UNSUPPORTED;
+    if (tier2) return KVQ_ERR_UNSUPPORTED;
+    if (ws_bytes < kvq_decode_workspace_bytes(c, batch, max_pages_per_seq)) return KVQ_ERR_CAPACITY;
+    const SplitPlan s = plan_splits(c, batch, max_pages_per_seq);
+    DecodeParams p{};
+    p.pool = c->pool;
+    p.q = static_cast<const __half *>(q);
+    p.block_table = block_table;
+    p.ctx_lens = ctx_lens;
+    p.max_pages = max_pages_per_seq;
+    p.batch = batch;
+    p.L = c->L;
+    const float scale = softmax_scale > 0.0f ? softmax_scale : (float)(1.0 / sqrt((double)c->L.d));
+    p.qscale = scale * 1.4426950408889634f;  // log2(e)
+    p.rot_scale = c->rot_scale;
+    p.rotate = c->cfg.rotate;
+    memcpy(p.signs, c->signs, sizeof(p.signs));
+    p.pages_per_split = s.pages_per_split;
+    p.pages_per_warp = s.pages_per_warp;
+    p.n_splits = s.n_splits;
+    p.counters = static_cast<unsigned int *>(workspace);
+    p.part = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + counters_bytes(batch, c->L.hkv));
+    p.out = static_cast<__half *>(out);
+    c->last_stream = stream;
+    const dim3 grid(s.n_splits, c->L.hkv, batch);
+    return cuda_status(launch_decode(p, grid, static_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_dequant_debug(kvq_cache *c, const int32_t *slots, int32_t n, float *k_out, float *v_out,
+                             uint8_t *codes_out, uint16_t *meta_out, void *stream)
+{
+    if (!c || n < 0) return KVQ_ERR_INVALID_ARG;
+    if (n == 0) return KVQ_OK;
+    if (!slots) return KVQ_ERR_INVALID_ARG;
+    DequantParams p{};
+    p.pool = c->pool;
+    p.slots = slots;
+    p.n = n;
+    p.L = c->L;
+    p.k_out = k_out;
+    p.v_out = v_out;
+    p.codes_out = codes_out;
+    p.meta_out = meta_out;
+    c->last_stream = stream;
+    return cuda_status(launch_dequant(p, static_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_sync_status(kvq_cache *c)
+{
+    if (!c) return KVQ_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(c->last_stream)) != cudaSuccess) return KVQ_ERR_CUDA;
+    unsigned int st = 0;
+    if (cudaMemcpy(&st, c->pool, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (st != 0 && cudaMemset(c->pool, 0, sizeof(st)) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return KVQ_ERR_CUDA;
+    return static_cast<kvq_status>(st);
+}
+
+const char *kvq_status_string(kvq_status s)
+{
+    switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_CAPACITY: return "buffer smaller than required";
+    case KVQ_ERR_OUT_OF_RANGE: return "slot or page index outside the pool";
+    case KVQ_ERR_CUDA: return "CUDA runtime error";
+    case KVQ_ERR_TIMEOUT: return "bounded device wait ran out";
+    default: return "unknown status";
+    }
+}
+
+}  // extern "C"

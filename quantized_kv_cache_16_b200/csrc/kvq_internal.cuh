@@ -1,0 +1,239 @@
+// kvq_internal.cuh -- internal definitions shared by the library's .cu files:
+// the pool layout, the cache handle, kernel parameter blocks and the inline
+// PTX wrappers (bulk copy + mbarrier, ldmatrix, mma.sync).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kPageTokens = 16;
+constexpr int kHeaderBytes = 256;
+constexpr int kMaxD = 128;
+constexpr int kMaxGqa = 8;
+
+// Status word lives at the start of the pool header.
+struct PoolHeader {
+    unsigned int status;
+    unsigned int pad[63];
+};
+
+inline __host__ __device__ int fmt_bits(int fmt) { return fmt == KVQ_INT4_ASYM ? 4 : fmt == KVQ_INT8_SYM ? 8 : 2; }
+
+// Byte layout of the pool (see kvq_pool_bytes in kvq.h).
+struct Layout {
+    int d, hq, hkv, g;
+    int k_fmt, v_fmt;
+    int k_row_code, v_row_code;  // code bytes of one token row
+    int k_row_meta, v_row_meta;  // meta bytes of one token row
+    int k_codes, k_meta, v_codes, v_meta;  // region offsets inside a chunk
+    int chunk_bytes;                       // one (page, kv head)
+    long long page_bytes;
+    int num_pages;
+    long long desc_off;  // from the pool start; 0 when descriptors are off
+    int bound_block;
+};
+
+inline __host__ Layout make_layout(const kvq_config &c)
+{
+    Layout L{};
+    L.d = c.head_dim;
+    L.hq = c.num_q_heads;
+    L.hkv = c.num_kv_heads;
+    L.g = c.num_q_heads / c.num_kv_heads;
+    L.k_fmt = c.k_fmt;
+    L.v_fmt = c.v_fmt;
+    L.k_row_code = L.d * fmt_bits(c.k_fmt) / 8;
+    L.v_row_code = L.d * fmt_bits(c.v_fmt) / 8;
+    L.k_row_meta = c.k_fmt == KVQ_INT8_SYM ? 2 : 4 * (L.d / c.k_group);
+    L.v_row_meta = c.v_fmt == KVQ_INT8_SYM ? 2 : 4 * (L.d / c.v_group);
+    L.k_codes = 0;
+    L.k_meta = kPageTokens * L.k_row_code;
+    L.v_codes = L.k_meta + kPageTokens * L.k_row_meta;
+    L.v_meta = L.v_codes + kPageTokens * L.v_row_code;
+    L.chunk_bytes = L.v_meta + kPageTokens * L.v_row_meta;
+    L.page_bytes = (long long)L.hkv * L.chunk_bytes;
+    L.num_pages = c.num_pages;
+    L.bound_block = c.bound_block_tokens;
+    L.desc_off = c.bound_block_tokens > 0 ? kHeaderBytes + (long long)c.num_pages * L.page_bytes : 0;
+    return L;
+}
+
+}  // namespace kvq
+
+struct kvq_cache {
+    kvq_config cfg;
+    kvq::Layout L;
+    unsigned char *pool;
+    size_t pool_bytes;
+    int device;
+    int num_sms;
+    float signs[kvq::kMaxD];       // +1 / -1
+    uint32_t sign_xor[kvq::kMaxD / 2];  // per half2 word: 0x8000 / 0x80000000 where the sign is -1
+    float rot_scale;               // fp32(1/sqrt(d))
+    void *last_stream;
+};
+
+namespace kvq {
+
+// ---------------------------------------------------------------- kernels ---
+
+struct AppendParams {
+    const __half *k;
+    const __half *v;
+    const int32_t *slots;
+    int n_tok;
+    unsigned char *pool;
+    Layout L;
+    float clip;
+    float rot_scale;
+    int rotate;
+    uint32_t sign_xor[kMaxD / 2];
+};
+
+struct DecodeParams {
+    const unsigned char *pool;
+    const __half *q;
+    const int32_t *block_table;
+    const int32_t *ctx_lens;
+    int max_pages;
+    int batch;
+    Layout L;
+    float qscale;  // softmax scale * log2(e)
+    float rot_scale;
+    int rotate;
+    float signs[kMaxD];
+    int pages_per_split;
+    int pages_per_warp;
+    int n_splits;
+    float *part;              // [B][Hkv][n_splits][g][d + 4]
+    unsigned int *counters;   // [B][Hkv]
+    __half *out;
+};
+
+struct DequantParams {
+    const unsigned char *pool;
+    const int32_t *slots;
+    int n;
+    Layout L;
+    float *k_out;
+    float *v_out;
+    uint8_t *codes_out;
+    uint16_t *meta_out;
+};
+
+// launchers (return cudaGetLastError() of the launch)
+cudaError_t launch_append(const AppendParams &p, int k_group, int v_group, cudaStream_t s);
+cudaError_t launch_decode(const DecodeParams &p, dim3 grid, cudaStream_t s);
+cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
+cudaError_t launch_reset_pages(unsigned char *pool, Layout L, const int32_t *pages, int n, cudaStream_t s);
+bool decode_supported(const Layout &L);
+constexpr int kDecodeWarps = 8;
+constexpr int kDecodeThreads = kDecodeWarps * 32;
+
+// ------------------------------------------------------------- device util ---
+
+__device__ __forceinline__ void set_status(const unsigned char *pool, unsigned int code)
+{
+    unsigned int *st = reinterpret_cast<unsigned int *>(const_cast<unsigned char *>(pool));
+    atomicCAS(st, 0u, code);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, unsigned count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Arm the barrier for `bytes` and start a bulk global->shared copy that
+// completes the transaction on it.  src/dst 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(phase)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `phase` of the barrier, giving up after ~limit_ns.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t phase, unsigned long long limit_ns)
+{
+    if (mbar_try_wait(bar, phase)) return true;
+    unsigned long long t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, phase)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t &r0, uint32_t &r1)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// D(16x8 f32) += A(16x16 f16, row) * B(16x8 f16, col)
+__device__ __forceinline__ void mma16816(float *d, const uint32_t *a, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+
+}  // namespace kvq

@@ -1,0 +1,149 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs.
+
+  append  -> pool bytes (codes, scales, zeros, descriptors) bit-exact;
+  dequant -> kvq_dequant_debug values equal fp32(oracle fp64 dequant), codes equal;
+  decode  -> max |gpu - oracle| <= 2e-3 and rel-L2 <= 1e-3 against the
+             oracle's fp64 attention over the same dequantised cache.
+
+Sizes span several pages, several splits and a ragged tail; the full-size
+workloads run in the launch configuration the benchmark uses.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+import workloads as W
+from _cases import TOL_MAX_ABS, TOL_REL_L2, attn_errors, build_pair
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import quantized_kv_cache_16_b200 as K
+    K.lib()  # fails loudly if the library is missing
+
+
+def _decode_check(pair, step=0, extra=0, softmax_scale=0.0):
+    import torch
+    wl = pair.wl
+    q = W.queries(wl, step)
+    out = pair.cache.decode(torch.from_numpy(q).cuda(), pair.block_table(), pair.ctx(extra),
+                            softmax_scale=softmax_scale)
+    got = out.float().cpu().numpy()
+    ctx = [t + extra for t in wl.ctx]
+    want = O.decode(pair.ocfg, pair.opool, q, pair.pages.block_table, ctx, scale=softmax_scale)
+    max_abs, rel = attn_errors(got, want)
+    assert max_abs <= TOL_MAX_ABS and rel <= TOL_REL_L2, f"max_abs={max_abs:.3e} rel={rel:.3e}"
+    assert pair.cache.sync_status() == 0
+    return got, want
+
+
+SMALL = [
+    ("tiny", W.tiny()),
+    ("llama-1000", W.scaled(W.llama(), 1000)),
+    ("llama-ragged", W.scaled(W.llama(), 17)),
+    ("paged-B5", W.scaled(W.paged(), [37, 300, 16, 1, 513])),
+    ("int8k-2000", W.scaled(W.certified(), 2000)),
+    ("int2-B2", W.scaled(W.int2(), [3000, 777])),
+]
+
+
+@pytest.mark.parametrize("name,wl", SMALL, ids=[s[0] for s in SMALL])
+def test_append_bytes_bit_exact(name, wl):
+    pair = build_pair(wl)
+    gpu = pair.cache.pool.cpu().numpy()
+    assert gpu.shape == pair.opool.shape
+    diff = np.nonzero(gpu[256:] != pair.opool[256:])[0]
+    assert diff.size == 0, f"{diff.size} bytes differ, first at pool offset {256 + diff[0]}"
+
+
+@pytest.mark.parametrize("name,wl", SMALL, ids=[s[0] for s in SMALL])
+def test_dequant_debug_matches_oracle(name, wl):
+    import torch
+    pair = build_pair(wl)
+    slots = np.concatenate([pair.pages.slots(b, 0, wl.ctx[b]) for b in range(wl.B)])
+    pick = np.random.default_rng(0).choice(slots, size=min(200, len(slots)), replace=False).astype(np.int32)
+    k, v, codes, meta = pair.cache.dequant(torch.from_numpy(pick).cuda())
+    ko, vo = O.dequant(pair.ocfg, pair.opool, pick)
+    assert np.array_equal(k.cpu().numpy(), ko.astype(np.float32))
+    assert np.array_equal(v.cpu().numpy(), vo.astype(np.float32))
+    codes = codes.cpu().numpy()
+    for i, s in enumerate(pick[:20]):
+        for kvh in range(wl.Hkv):
+            for t in range(2):
+                c, _, _ = O.read_row(pair.ocfg, pair.opool, int(s), kvh, t)
+                fmt = wl.v_fmt if t else wl.k_fmt
+                want = c.astype(np.int64) & (0xFF if fmt == O.INT8_SYM else 0xF if fmt == O.INT4_ASYM else 0x3)
+                assert np.array_equal(codes[i, kvh, t].astype(np.int64), want)
+
+
+@pytest.mark.parametrize("name,wl", SMALL, ids=[s[0] for s in SMALL])
+def test_decode_matches_oracle(name, wl):
+    pair = build_pair(wl)
+    _decode_check(pair)
+
+
+def test_decode_edge_lengths():
+    """Empty context (zero output), one token, exactly one page, page + 1."""
+    wl = W.scaled(W.llama(), [0, 1, 16, 17])
+    pair = build_pair(wl)
+    got, _ = _decode_check(pair)
+    assert not got[0].any()
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (64, 8), (6, 2)])
+def test_decode_gqa_group_sizes(hq, hkv):
+    import dataclasses
+    wl = dataclasses.replace(W.scaled(W.llama(), [700, 45]), Hq=hq, Hkv=hkv)
+    _decode_check(build_pair(wl))
+
+
+def test_decode_without_rotation_and_explicit_scale():
+    wl = W.scaled(W.llama(), [900])
+    pair = build_pair(wl, rotate=0)
+    gpu = pair.cache.pool.cpu().numpy()
+    assert np.array_equal(gpu[256:], pair.opool[256:])
+    _decode_check(pair, softmax_scale=0.05)
+
+
+def test_decode_steps_append_then_attend():
+    """The decode step of the benchmark: append one token per sequence, then
+    attend over the grown context, several steps in a row, with the workspace
+    reused (its counters must come back to zero after every call)."""
+    import torch
+    wl = W.scaled(W.paged(), [100, 31, 260], steps=3)
+    pair = build_pair(wl, extra_tokens=wl.steps)
+    for step in range(wl.steps):
+        k, v = W.step_kv(wl, step)
+        slots = np.array([pair.pages.slot(b, wl.ctx[b] + step) for b in range(wl.B)], np.int32)
+        pair.cache.append(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(), torch.from_numpy(slots).cuda())
+        assert O.append(pair.ocfg, pair.opool, k, v, slots) == 0
+        got1, _ = _decode_check(pair, step=step, extra=step + 1)
+        got2, _ = _decode_check(pair, step=step, extra=step + 1)
+        assert np.array_equal(got1, got2)
+    gpu = pair.cache.pool.cpu().numpy()
+    assert np.array_equal(gpu[256:], pair.opool[256:])
+
+
+FULL = [
+    ("tiny-d64-T256", W.tiny),
+    ("llama3-8b-layer-T32768", lambda: W.scaled(W.llama(), 32768)),
+    ("paged-B16", W.paged),
+    ("int8k-int4v-T131072", lambda: W.scaled(W.certified(), 131072)),
+    ("int2-B4-T65536", W.int2),
+]
+
+
+@pytest.mark.parametrize("name,make", FULL, ids=[f[0] for f in FULL])
+def test_full_size_workloads(name, make):
+    """Full sizes: pool bytes bit-exact, every output row within tolerance."""
+    wl = make()
+    pair = build_pair(wl)
+    gpu = pair.cache.pool.cpu().numpy()
+    diff = np.nonzero(gpu[256:] != pair.opool[256:])[0]
+    assert diff.size == 0, f"{diff.size} bytes differ, first at {256 + diff[0]}"
+    _decode_check(pair)
