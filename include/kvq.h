@@ -136,7 +136,9 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int32_t batch, int32_t
  *   tier2:       NULL, or the certified-mode store (needs bound_block_tokens)
  *   workspace:   >= kvq_decode_workspace_bytes, zero-filled before first use;
  *                one workspace must not serve two decode calls that overlap
- *   out:         fp16 [batch][Hq][d] (device)
+ *   out:         fp32 [batch][Hq][d] (device, 16-byte aligned); fp32 so the
+ *                result keeps the kernel's accuracy (an fp16 store alone
+ *                would round outputs of magnitude 32 by up to 0.008)
  *   promoted_out (certified mode, optional): int32 [batch][Hkv][kmax] block
  *                indices promoted, highest bound first, -1 padded, where
  *                kmax = ceil(promote_frac * ceil(16*max_pages_per_seq / block)).

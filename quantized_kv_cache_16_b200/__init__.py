@@ -210,7 +210,7 @@ class Cache:
         import torch
         batch, max_pages = block_table.shape
         if out is None:
-            out = torch.empty_like(q)
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
         ws = self.workspace_for(batch, max_pages)
         kvq_decode_attn(self.handle, q, block_table, max_pages, ctx_lens, batch, softmax_scale, tier2, ws,
                         ws.numel(), out, promoted_out, stream)

@@ -209,7 +209,7 @@ kvq_status kvq_decode_attn(kvq_cache *c, const void *q, const int32_t *block_tab
     p.n_splits = s.n_splits;
     p.counters = static_cast<unsigned int *>(workspace);
     p.part = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + counters_bytes(batch, c->L.hkv));
-    p.out = static_cast<__half *>(out);
+    p.out = static_cast<float *>(out);
     c->last_stream = stream;
     const dim3 grid(s.n_splits, c->L.hkv, batch);
     return cuda_status(launch_decode(p, grid, static_cast<cudaStream_t>(stream)));

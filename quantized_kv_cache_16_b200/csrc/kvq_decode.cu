@@ -19,13 +19,13 @@
 //       a page's max exceeds it by more than 8 (exact: any reference works).
 //   PV  on tensor cores with M = channels: A = value codes of 16 tokens
 //       transposed by ldmatrix.trans (exact fp16 integers), B = p * scale of
-//       each token and group rounded once to fp16; the zero term is one MMA of
-//       the fp16 zeros against p.
+//       each token and group split into fp16 hi + lo (two MMAs); the zero term
+//       is the fp16 zeros against p (hi + lo).
 //
 // The 8 warps' (m, l, acc) are merged through shared memory into one partial
 // per (sequence, kv head, split, head); the last CTA of each (sequence, kv
 // head) to finish merges all splits by the log-sum-exp rule, applies the
-// inverse rotation R^T = diag(s) H c_d and writes fp16.
+// inverse rotation R^T = diag(s) H c_d and writes fp32.
 #include <math.h>
 
 #include "kvq_internal.cuh"
@@ -87,6 +87,14 @@ __device__ __forceinline__ uint32_t i8pair(uint32_t w, int sel)
 }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) { return h2_bits(__floats2half2_rn(lo, hi)); }
+
+// (x0, x1) ~= hi + lo with hi = fp16(x) and lo = fp16(x - hi), packed pairs.
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uint32_t &lo)
+{
+    const __half2 h = __floats2half2_rn(x0, x1);
+    hi = h2_bits(h);
+    lo = pack_h2(x0 - __low2float(h), x1 - __high2float(h));
+}
 
 // ------------------------------------------------------------ key codecs ---
 // B operand of QK: thread (r = lane/4, j = lane%4) holds for k-step ks the
@@ -557,17 +565,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
                 sv[q][gi] = valid ? h2f_bits(*reinterpret_cast<const uint16_t *>(mrow + 2 * gi)) : 0.f;
             zv[q] = (valid && r < VC::NG) ? *reinterpret_cast<const uint16_t *>(mrow + 2 * VC::NG + 2 * r) : 0;
         }
+        // p and p*scale enter the MMAs as fp16 hi + lo pairs (two MMAs each),
+        // so the weights carry ~22 bits instead of fp16's 11
         {
-            const uint32_t pb0 = pack_h2(pr[0], pr[1]), pb1 = pack_h2(pr[2], pr[3]);
+            uint32_t ph[2], pl[2];
+            split_pair(pr[0], pr[1], ph[0], pl[0]);
+            split_pair(pr[2], pr[3], ph[1], pl[1]);
             const uint32_t az[4] = {uint32_t(zv[0]) | (uint32_t(zv[1]) << 16), 0u,
                                     uint32_t(zv[2]) | (uint32_t(zv[3]) << 16), 0u};
-            mma16816(oz, az, pb0, pb1);
+            mma16816(oz, az, ph[0], ph[1]);
+            mma16816(oz, az, pl[0], pl[1]);
         }
-        uint32_t wb[VC::NG][2];
+        uint32_t wh[VC::NG][2], wl[VC::NG][2];
 #pragma unroll
         for (int gi = 0; gi < VC::NG; gi++) {
-            wb[gi][0] = pack_h2(pr[0] * sv[0][gi], pr[1] * sv[1][gi]);
-            wb[gi][1] = pack_h2(pr[2] * sv[2][gi], pr[3] * sv[3][gi]);
+            split_pair(pr[0] * sv[0][gi], pr[1] * sv[1][gi], wh[gi][0], wl[gi][0]);
+            split_pair(pr[2] * sv[2][gi], pr[3] * sv[3][gi], wh[gi][1], wl[gi][1]);
         }
         uint32_t vA[VC::NCH], vB[VC::NCH];
         ld_rows_t<VC::NCH>(sb + C::V_CODES, lane, vA, vB);
@@ -579,7 +592,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
                 uint32_t a[4];
                 VC::afrag(vA[c], vB[c], u, a);
                 const int gi = VC::group_of_mt(mt);
-                mma16816(oacc[mt], a, wb[gi][0], wb[gi][1]);
+                mma16816(oacc[mt], a, wh[gi][0], wh[gi][1]);
+                mma16816(oacc[mt], a, wl[gi][0], wl[gi][1]);
             }
         }
 
@@ -692,14 +706,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
 #pragma unroll
             for (int e = 0; e < E; e++) o[e] *= p.rot_scale * p.signs[lane * E + e];
         }
-        __half *dst = p.out + ((long long)b * L.hq + kvh * g + h) * D + lane * E;
+        float *dst = p.out + ((long long)b * L.hq + kvh * g + h) * D + lane * E;
         if constexpr (E == 4) {
-            uint2 u;
-            u.x = pack_h2(o[0], o[1]);
-            u.y = pack_h2(o[2], o[3]);
-            *reinterpret_cast<uint2 *>(dst) = u;
+            *reinterpret_cast<float4 *>(dst) = make_float4(o[0], o[1], o[2], o[3]);
         } else {
-            *reinterpret_cast<uint32_t *>(dst) = pack_h2(o[0], o[1]);
+            *reinterpret_cast<float2 *>(dst) = make_float2(o[0], o[1]);
         }
     }
 }

@@ -112,7 +112,7 @@ struct DecodeParams {
     int n_splits;
     float *part;              // [B][Hkv][n_splits][g][d + 4]
     unsigned int *counters;   // [B][Hkv]
-    __half *out;
+    float *out;
 };
 
 struct DequantParams {

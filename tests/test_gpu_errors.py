@@ -63,7 +63,7 @@ def test_decode_checks_arguments_and_indices():
     ctx = pair.ctx()
     ws_need = K.kvq_decode_workspace_bytes(c.handle, 1, bt.shape[1])
     ws = torch.zeros(ws_need, dtype=torch.uint8, device="cuda")
-    out = torch.empty_like(q)
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
     with pytest.raises(K.KvqError) as e:
         K.kvq_decode_attn(c.handle, q, bt, bt.shape[1], ctx, 1, 0.0, None, ws, ws_need - 256, out)
     assert e.value.status == K.KVQ_ERR_CAPACITY
@@ -82,4 +82,4 @@ def test_decode_checks_arguments_and_indices():
     # and the next plain call is clean and finite
     K.kvq_decode_attn(c.handle, q, bt, bt.shape[1], ctx, 1, 0.0, None, ws, ws_need, out)
     assert c.sync_status() == K.KVQ_OK
-    assert torch.isfinite(out.float()).all()
+    assert torch.isfinite(out).all()
