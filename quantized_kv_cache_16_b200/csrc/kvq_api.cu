@@ -70,6 +70,12 @@ SplitPlan plan_splits(const kvq_cache *c, int batch, int max_pages)
     s.pages_per_warp = (int)((per_cta + kDecodeWarps - 1) / kDecodeWarps);
     s.pages_per_split = s.pages_per_warp * kDecodeWarps;
     s.n_splits = (max_pages + s.pages_per_split - 1) / s.pages_per_split;
+    // the final merge holds every split's weight in shared memory
+    while (s.n_splits > decode_max_splits(c->L)) {
+        s.pages_per_warp *= 2;
+        s.pages_per_split = s.pages_per_warp * kDecodeWarps;
+        s.n_splits = (max_pages + s.pages_per_split - 1) / s.pages_per_split;
+    }
     if (s.n_splits < 1) s.n_splits = 1;
     return s;
 }

@@ -4,28 +4,32 @@
 //
 // Grid (split, kv head, sequence); 8 warps per CTA.  Each warp streams its
 // own contiguous run of 16-token pages: one bulk copy per (page, kv head)
-// chunk into a 4-deep shared-memory ring guarded by mbarriers.  Per page:
+// chunk into a shared-memory ring guarded by mbarriers.  Per page (16 tokens),
+// with the MMA row dimension over tokens:
 //
-//   QK  on tensor cores (mma.m16n8k16, fp32 accumulate).  B = the key codes of
-//       8 tokens, turned into fp16 integers exactly (magic-number unpack, no
-//       rounding); A = the rotated, pre-scaled query of the GQA group split
-//       into an fp16 high part (rows 0..g-1) and low part (rows 8..8+g-1), so
-//       q ~= hi + lo to ~22 bits.  One accumulator per quantisation group;
-//       the per-token group scale is applied in fp32 afterwards and the
-//       group-zero term  sum_g zero[t][g] * sum_{i in g} q_i  is one more MMA
-//       with the fp16 zeros as B.  So scores = sum_g s_g (q.c_g) + z_g qsum_g,
-//       the dequantised dot product, without ever rounding a dequantised key.
-//   softmax online in the log2 domain, with the running max raised only when
+//   QK  int8 tensor cores (mma.m16n8k32.s8, exact int32): A = the key codes of
+//       the 16 tokens as bytes (int4/int2 codes unpack with a mask and shift;
+//       int8 codes are used as stored); B = the rotated, pre-scaled query of
+//       every head of the GQA group as three signed 7-bit digits
+//       q*2^E = d1*2^14 + d2*2^7 + d3 (~21 bits), one column per (head, digit).
+//       One MMA per quantisation group; the digits recombine in int32, the
+//       group scale applies in fp32, and the group-zero term
+//       sum_g zero[t][g] * sum_{i in g} q_i is one fp16 MMA (zeros exact,
+//       query sums as hi + lo).  No dequantised key is ever rounded.
+//   softmax online in the log2 domain; lane (r, j) owns head j for tokens r
+//       and r+8, so the running max, sum and the accumulator columns of a
+//       head all live in the same lanes.  The running max is raised only when
 //       a page's max exceeds it by more than 8 (exact: any reference works).
-//   PV  on tensor cores with M = channels: A = value codes of 16 tokens
-//       transposed by ldmatrix.trans (exact fp16 integers), B = p * scale of
-//       each token and group split into fp16 hi + lo (two MMAs); the zero term
-//       is the fp16 zeros against p (hi + lo).
+//   PV  fp16 tensor cores with M = channels: A = value codes of 16 tokens
+//       transposed by ldmatrix.trans (exact fp16 integers); B = p * scale of
+//       each token and group as an (fp16 hi, fp16 lo) column pair per head,
+//       transposed into B layout with movmatrix; the zero term is the fp16
+//       zeros against p (hi, lo) in one more MMA.
 //
-// The 8 warps' (m, l, acc) are merged through shared memory into one partial
-// per (sequence, kv head, split, head); the last CTA of each (sequence, kv
-// head) to finish merges all splits by the log-sum-exp rule, applies the
-// inverse rotation R^T = diag(s) H c_d and writes fp32.
+// The 8 warps' (m, l, acc) merge through shared memory into one partial per
+// (sequence, kv head, split, head); the last CTA of each (sequence, kv head)
+// merges all splits by the log-sum-exp rule with every thread loading in
+// parallel, applies the inverse rotation R^T = diag(s) H c_d, writes fp32.
 #include <math.h>
 
 #include "kvq_internal.cuh"
@@ -37,9 +41,7 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per stage wait
 
 // fp16x2 constants (bit patterns)
-constexpr uint32_t kH1024 = 0x64006400u;   // (1024, 1024)
-constexpr uint32_t kH1152 = 0x64806480u;   // (1152, 1152)
-constexpr uint32_t kMagicB = 0x64646464u;  // bytes 0x64 for PRMT
+constexpr uint32_t kH1024 = 0x64006400u;  // (1024, 1024)
 
 __device__ __forceinline__ uint32_t hsub2u(uint32_t a, uint32_t b)
 {
@@ -51,17 +53,13 @@ __device__ __forceinline__ uint32_t hfma2u(uint32_t a, uint32_t b, uint32_t c)
     return h2_bits(__hfma2(bits_h2(a), bits_h2(b), bits_h2(c)));
 }
 
-// Nibbles at bits [0,4) and [16,20) of w as exact fp16 integers.
-__device__ __forceinline__ uint32_t nib0(uint32_t w) { return hsub2u((w & 0x000F000Fu) | kH1024, kH1024); }
-// Nibbles at bits [4,8) and [20,24): (1024 + 16c) / 16 - 64 = c exactly.
-__device__ __forceinline__ uint32_t nib1(uint32_t w)
-{
-    return hfma2u((w & 0x00F000F0u) | kH1024, 0x2C002C00u /*1/16*/, 0xD400D400u /*-64*/);
-}
-// Nibble n (0..3) of each 16-bit half.
+// Nibble n (0..3) of each 16-bit half of w as exact fp16 integers:
+// (w & mask) | 0x6400 is 1024 + c * 16^(n&1); subtract / rescale exactly.
 __device__ __forceinline__ uint32_t nib(uint32_t w, int n)
 {
-    return (n & 1) ? nib1(n & 2 ? w >> 8 : w) : nib0(n & 2 ? w >> 8 : w);
+    const uint32_t x = (n & 2) ? (w >> 8) : w;
+    if (n & 1) return hfma2u((x & 0x00F000F0u) | kH1024, 0x2C002C00u /*1/16*/, 0xD400D400u /*-64*/);
+    return hsub2u((x & 0x000F000Fu) | kH1024, kH1024);
 }
 
 // 2-bit field f (0..7) of each 16-bit half as exact fp16 integers.
@@ -78,94 +76,99 @@ __device__ __forceinline__ uint32_t fld2(uint32_t w, int f)
     }
 }
 
-// Signed bytes 0,1 (sel 0) or 2,3 (sel 1) of w as exact fp16 integers.
-__device__ __forceinline__ uint32_t i8pair(uint32_t w, int sel)
-{
-    const uint32_t biased = w ^ 0x80808080u;  // c + 128 as unsigned bytes
-    const uint32_t x = __byte_perm(biased, kMagicB, sel ? 0x7362 : 0x5140);
-    return hsub2u(x, kH1152);
-}
-
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) { return h2_bits(__floats2half2_rn(lo, hi)); }
 
-// (x0, x1) ~= hi + lo with hi = fp16(x) and lo = fp16(x - hi), packed pairs.
-__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uint32_t &lo)
+// x ~= hi + lo, returned as the fp16 pair (hi, lo).
+__device__ __forceinline__ uint32_t hilo(float x)
 {
-    const __half2 h = __floats2half2_rn(x0, x1);
-    hi = h2_bits(h);
-    lo = pack_h2(x0 - __low2float(h), x1 - __high2float(h));
+    const float hf = __half2float(__float2half_rn(x));
+    return pack_h2(x, x - hf);
+}
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t movm_t(uint32_t x)
+{
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// D(16x8 s32) += A(16x32 s8, row) * B(32x8 s8, col)
+__device__ __forceinline__ void imma16832(int *d, const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // ------------------------------------------------------------ key codecs ---
-// B operand of QK: thread (r = lane/4, j = lane%4) holds for k-step ks the
-// fp16 pairs at virtual k (2j, 2j+1) and (2j+8, 2j+9) of token r.  chan()
-// maps a virtual (ks, kk) to the physical channel, which the query fragment
-// follows; the unpack never needs to reorder codes.
+// A operand of the QK IMMA: thread (r, j) holds, for k-step kq (32 virtual
+// channels), 4 bytes at virtual k = 4j..4j+3 and 4j+16..4j+19 of tokens r and
+// r+8.  chan(kq, k) maps virtual k to the physical channel; the query digits
+// follow the same map, so the codes never need reordering.
 
 template <int FMT, int D> struct KCodec;
 
 template <int D> struct KCodec<KVQ_INT4_ASYM, D> {
     static constexpr int NCH = D / 32;  // 16-byte chunks per token row (= groups)
     static constexpr int NG = D / 32;
+    static constexpr int KQ = D / 32;   // IMMA k-steps
     static constexpr bool ZERO = true;
     static constexpr int ROW_META = 4 * NG;
-    __device__ static int chan(int ks, int kk)
+    __device__ static int chan(int kq, int k) { return 32 * kq + 8 * ((k & 15) >> 2) + 2 * (k & 3) + (k >> 4); }
+    __device__ static int group_of_kq(int kq) { return kq; }
+    // w[c] / w8[c]: word j of chunk c for tokens r / r+8
+    __device__ static void afrag(const uint32_t (&w)[NCH], const uint32_t (&w8)[NCH], int kq, uint32_t (&a)[4])
     {
-        const int jj = (kk & 7) >> 1, e = kk & 1, hb = kk >> 3;
-        return 32 * (ks >> 1) + 8 * jj + 2 * (ks & 1) + hb + 4 * e;
-    }
-    __device__ static int group_of_chan(int ch) { return ch / 32; }
-    __device__ static int group_of_chunk(int c) { return c; }
-    static constexpr int KS_PER_CHUNK = 2;
-    __device__ static void unpack(uint32_t w, uint32_t (&b)[KS_PER_CHUNK][2])
-    {
-        b[0][0] = nib(w, 0);
-        b[0][1] = nib(w, 1);
-        b[1][0] = nib(w, 2);
-        b[1][1] = nib(w, 3);
+        a[0] = w[kq] & 0x0F0F0F0Fu;
+        a[1] = w8[kq] & 0x0F0F0F0Fu;
+        a[2] = (w[kq] >> 4) & 0x0F0F0F0Fu;
+        a[3] = (w8[kq] >> 4) & 0x0F0F0F0Fu;
     }
 };
 
 template <int D> struct KCodec<KVQ_INT8_SYM, D> {
     static constexpr int NCH = D / 16;
     static constexpr int NG = 1;
+    static constexpr int KQ = D / 32;
     static constexpr bool ZERO = false;
     static constexpr int ROW_META = 2;
-    __device__ static int chan(int ks, int kk)
+    __device__ static int chan(int kq, int k) { return 32 * kq + k; }
+    __device__ static int group_of_kq(int) { return 0; }
+    __device__ static void afrag(const uint32_t (&w)[NCH], const uint32_t (&w8)[NCH], int kq, uint32_t (&a)[4])
     {
-        const int jj = (kk & 7) >> 1, e = kk & 1, hb = kk >> 3;
-        return 16 * ks + 4 * jj + 2 * hb + e;
-    }
-    __device__ static int group_of_chan(int) { return 0; }
-    __device__ static int group_of_chunk(int) { return 0; }
-    static constexpr int KS_PER_CHUNK = 1;
-    __device__ static void unpack(uint32_t w, uint32_t (&b)[KS_PER_CHUNK][2])
-    {
-        b[0][0] = i8pair(w, 0);
-        b[0][1] = i8pair(w, 1);
+        a[0] = w[2 * kq];
+        a[1] = w8[2 * kq];
+        a[2] = w[2 * kq + 1];
+        a[3] = w8[2 * kq + 1];
     }
 };
 
 template <int D> struct KCodec<KVQ_INT2_ASYM, D> {
     static constexpr int NCH = D / 64;
     static constexpr int NG = 1;
+    static constexpr int KQ = D / 32;
     static constexpr bool ZERO = true;
     static constexpr int ROW_META = 4;
-    __device__ static int chan(int ks, int kk)
+    __device__ static int chan(int kq, int k)
     {
-        const int jj = (kk & 7) >> 1, e = kk & 1, hb = kk >> 3;
-        return 64 * (ks >> 2) + 16 * jj + 2 * (ks & 3) + hb + 8 * e;
+        return 64 * (kq >> 1) + 16 * ((k & 15) >> 2) + 4 * (k & 3) + 2 * (kq & 1) + (k >> 4);
     }
-    __device__ static int group_of_chan(int) { return 0; }
-    __device__ static int group_of_chunk(int) { return 0; }
-    static constexpr int KS_PER_CHUNK = 4;
-    __device__ static void unpack(uint32_t w, uint32_t (&b)[KS_PER_CHUNK][2])
+    __device__ static int group_of_kq(int) { return 0; }
+    __device__ static void afrag(const uint32_t (&w)[NCH], const uint32_t (&w8)[NCH], int kq, uint32_t (&a)[4])
     {
-#pragma unroll
-        for (int u = 0; u < 4; u++) {
-            b[u][0] = fld2(w, 2 * u);
-            b[u][1] = fld2(w, 2 * u + 1);
-        }
+        const int c = kq >> 1, s = 2 * (kq & 1);
+        a[0] = (w[c] >> (2 * s)) & 0x03030303u;
+        a[1] = (w8[c] >> (2 * s)) & 0x03030303u;
+        a[2] = (w[c] >> (2 * s + 2)) & 0x03030303u;
+        a[3] = (w8[c] >> (2 * s + 2)) & 0x03030303u;
     }
 };
 
@@ -211,9 +214,11 @@ template <int D> struct VCodec<KVQ_INT2_ASYM, D> {
     }
 };
 
-template <int KF, int VF, int D> struct Cfg {
+template <int KF, int VF, int D, bool G8> struct Cfg {
     using K = KCodec<KF, D>;
     using V = VCodec<VF, D>;
+    static constexpr int NH = G8 ? 2 : 1;  // heads per lane (j, j+4)
+    static constexpr int NT = G8 ? 3 : 2;  // IMMA n-tiles of query digits
     static constexpr int K_CODES = 0;
     static constexpr int K_META = 16 * (D * (KF == KVQ_INT4_ASYM ? 4 : KF == KVQ_INT8_SYM ? 8 : 2) / 8);
     static constexpr int V_CODES = K_META + 16 * K::ROW_META;
@@ -221,63 +226,61 @@ template <int KF, int VF, int D> struct Cfg {
     static constexpr int CHUNK = V_META + 16 * V::ROW_META;
     static constexpr int NST = CHUNK > 3000 ? 3 : 4;
     static constexpr int STAGE = (CHUNK + 127) / 128 * 128;
-    static constexpr int KST = D / 16;  // k-steps of QK
-    static constexpr int MT = D / 16;   // m-tiles of PV
-    static constexpr int E = D / 32;    // elements per lane in warp-wide vectors
+    static constexpr int MT = D / 16;  // m-tiles of PV
+    static constexpr int E = D / 32;   // elements per lane in warp-wide vectors
     // shared memory map
-    static constexpr int OFF_QS = kDecodeWarps * NST * STAGE;
-    static constexpr int OFF_QSUM = OFF_QS + kMaxGqa * D * 4;
-    static constexpr int OFF_BAR = OFF_QSUM + kMaxGqa * 4 * 4;
+    static constexpr int RING = kDecodeWarps * NST * STAGE;
+    static constexpr int OFF_QF = RING;                             // f32 [8][D]
+    static constexpr int OFF_QV = OFF_QF + kMaxGqa * D * 4;          // s8 [NT][KQ][8][32]
+    static constexpr int OFF_QSUM = OFF_QV + NT * K::KQ * 8 * 32;    // f32 [8][4]
+    static constexpr int OFF_QEXP = OFF_QSUM + kMaxGqa * 4 * 4;      // i32 [8]
+    static constexpr int OFF_BAR = OFF_QEXP + kMaxGqa * 4;
     static constexpr int OFF_FLAG = OFF_BAR + kDecodeWarps * NST * 8;
     static constexpr int SMEM = OFF_FLAG + 16;
-    // merge scratch (aliases the stage ring after the page loop)
-    static constexpr int MERGE_ACC = 0;                                       // [W][8][D]
-    static constexpr int MERGE_Z = MERGE_ACC + kDecodeWarps * kMaxGqa * D * 4;  // [W][4][8]
-    static constexpr int MERGE_M = MERGE_Z + kDecodeWarps * 4 * kMaxGqa * 4;    // [W][8]
-    static constexpr int MERGE_L = MERGE_M + kDecodeWarps * kMaxGqa * 4;        // [W][8]
-    static_assert(MERGE_L + kDecodeWarps * kMaxGqa * 4 <= OFF_QS, "merge scratch must fit in the stage ring");
+    // merge scratch (aliases the ring after the page loop)
+    static constexpr int MERGE_ACC = 0;                                         // [W][8][D]
+    static constexpr int MERGE_Z = MERGE_ACC + kDecodeWarps * kMaxGqa * D * 4;    // [W][4][8]
+    static constexpr int MERGE_M = MERGE_Z + kDecodeWarps * 4 * kMaxGqa * 4;      // [W][8]
+    static constexpr int MERGE_L = MERGE_M + kDecodeWarps * kMaxGqa * 4;          // [W][8]
+    static_assert(MERGE_L + kDecodeWarps * kMaxGqa * 4 <= RING, "merge scratch must fit in the ring");
+    static_assert(OFF_BAR % 8 == 0, "mbarriers need 8-byte alignment");
 };
 
-// Load NCH 16-byte chunks of rows [8*nt, 8*nt+8) of a chunk-major code region
-// (non-transposed): out[c] = bytes [4j, 4j+4) of chunk c of token 8*nt + r.
+// Key chunks, not transposed, tokens r (w) and r+8 (w8): ldmatrix.x4 over the
+// matrices (c, tok 0-7), (c, tok 8-15), (c+1, tok 0-7), (c+1, tok 8-15).
 template <int NCH>
-__device__ __forceinline__ void ld_rows(uint32_t base, int nt, int lane, uint32_t (&w)[NCH])
-{
-    const int row = lane & 7, mi = lane >> 3;
-    if constexpr (NCH >= 4) {
-#pragma unroll
-        for (int q = 0; q < NCH / 4; q++) {
-            const uint32_t addr = base + ((4 * q + mi) * 16 + 8 * nt + row) * 16;
-            ldsm_x4(addr, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-        }
-    } else if constexpr (NCH == 2) {
-        const uint32_t addr = base + (((mi & 1)) * 16 + 8 * nt + row) * 16;
-        ldsm_x2(addr, w[0], w[1]);
-    } else {
-        const uint32_t addr = base + (8 * nt + row) * 16;
-        uint32_t dummy;
-        ldsm_x2(addr, w[0], dummy);
-    }
-}
-
-// Load NCH chunks of a value region transposed: wA[c] = tokens (2j, 2j+1),
-// wB[c] = tokens (2j+8, 2j+9), 16-bit piece r of chunk c.
-template <int NCH>
-__device__ __forceinline__ void ld_rows_t(uint32_t base, int lane, uint32_t (&wA)[NCH], uint32_t (&wB)[NCH])
+__device__ __forceinline__ void ld_krows(uint32_t base, int lane, uint32_t (&w)[NCH], uint32_t (&w8)[NCH])
 {
     const int row = lane & 7, mi = lane >> 3;
     if constexpr (NCH >= 2) {
 #pragma unroll
         for (int q = 0; q < NCH / 2; q++) {
             const int c = 2 * q + (mi >> 1), tok = (mi & 1) * 8 + row;
-            const uint32_t addr = base + (c * 16 + tok) * 16;
-            ldsm_x4_t(addr, wA[2 * q], wB[2 * q], wA[2 * q + 1], wB[2 * q + 1]);
+            ldsm_x4(base + (c * 16 + tok) * 16, w[2 * q], w8[2 * q], w[2 * q + 1], w8[2 * q + 1]);
         }
     } else {
         const int tok = (mi & 1) * 8 + row;
-        const uint32_t addr = base + tok * 16;
         uint32_t d0, d1;
-        ldsm_x4_t(addr, wA[0], wB[0], d0, d1);
+        ldsm_x4(base + tok * 16, w[0], w8[0], d0, d1);
+    }
+}
+
+// Value chunks transposed: wA[c] = tokens (2j, 2j+1), wB[c] = tokens
+// (2j+8, 2j+9), 16-bit piece r of chunk c.
+template <int NCH>
+__device__ __forceinline__ void ld_vrows_t(uint32_t base, int lane, uint32_t (&wA)[NCH], uint32_t (&wB)[NCH])
+{
+    const int row = lane & 7, mi = lane >> 3;
+    if constexpr (NCH >= 2) {
+#pragma unroll
+        for (int q = 0; q < NCH / 2; q++) {
+            const int c = 2 * q + (mi >> 1), tok = (mi & 1) * 8 + row;
+            ldsm_x4_t(base + (c * 16 + tok) * 16, wA[2 * q], wB[2 * q], wA[2 * q + 1], wB[2 * q + 1]);
+        }
+    } else {
+        const int tok = (mi & 1) * 8 + row;
+        uint32_t d0, d1;
+        ldsm_x4_t(base + tok * 16, wA[0], wB[0], d0, d1);
     }
 }
 
@@ -306,14 +309,34 @@ __device__ __forceinline__ void fwht_warp(float (&x)[D / 32], int lane)
 
 __device__ __forceinline__ float h2f_bits(uint16_t u) { return __half2float(__ushort_as_half(u)); }
 
-template <int D, int KF, int VF>
-__global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_constant__ DecodeParams p)
+// Which (head, digit) a query-digit column holds; digit -1 = unused column.
+template <bool G8>
+__device__ __forceinline__ void col_src(int nt, int n, int &head, int &digit)
 {
-    using C = Cfg<KF, VF, D>;
+    if (!G8) {
+        head = n >> 1;
+        digit = nt == 0 ? (n & 1) : ((n & 1) ? -1 : 2);
+    } else {
+        if (nt < 2) {
+            head = 4 * nt + (n >> 1);
+            digit = n & 1;
+        } else {
+            head = (n & 1) ? 4 + (n >> 1) : (n >> 1);
+            digit = 2;
+        }
+    }
+}
+
+template <int D, int KF, int VF, bool G8>
+__global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(const __grid_constant__ DecodeParams p)
+{
+    using C = Cfg<KF, VF, D, G8>;
     using KC = typename C::K;
     using VC = typename C::V;
     constexpr int E = C::E;
     constexpr int NST = C::NST;
+    constexpr int NH = C::NH;
+    constexpr int NT = C::NT;
 
     const Layout &L = p.L;
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -331,14 +354,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
     if (split >= n_active) return;
 
     extern __shared__ __align__(128) unsigned char smem[];
-    float *qs = reinterpret_cast<float *>(smem + C::OFF_QS);
+    float *qf = reinterpret_cast<float *>(smem + C::OFF_QF);
+    int8_t *qv = reinterpret_cast<int8_t *>(smem + C::OFF_QV);
     float *qsum = reinterpret_cast<float *>(smem + C::OFF_QSUM);
+    int *qexp = reinterpret_cast<int *>(smem + C::OFF_QEXP);
     int *sflag = reinterpret_cast<int *>(smem + C::OFF_FLAG);
     const uint32_t bar0 = smem_u32(smem + C::OFF_BAR) + warp * NST * 8;
     const uint32_t stage0 = smem_u32(smem) + warp * NST * C::STAGE;
     const unsigned char *stage0_ptr = smem + warp * NST * C::STAGE;
 
-    // ---- query: rotate, pre-scale, group sums (warp w handles head w) ----
+    // ---- query: rotate, pre-scale, digit exponent, group sums (warp h) ----
     for (int h = warp; h < g; h += kDecodeWarps) {
         const __half *qh = p.q + ((long long)b * L.hq + kvh * g + h) * D + lane * E;
         float x[E];
@@ -361,16 +386,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
             fwht_warp<D>(x, lane);
             sc *= p.rot_scale;
         }
+        float amax = 0.f;
 #pragma unroll
         for (int e = 0; e < E; e++) {
             x[e] *= sc;
-            qs[h * D + lane * E + e] = x[e];
+            qf[h * D + lane * E + e] = x[e];
+            amax = fmaxf(amax, fabsf(x[e]));
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, m));
+        if (lane == 0) {
+            int ex = 0;
+            if (amax > 0.f) frexpf(amax, &ex);  // amax < 2^ex
+            qexp[h] = 20 - ex;                  // |q * 2^E| < 2^20
         }
         if constexpr (KC::ZERO) {
             float s = 0.f;
 #pragma unroll
             for (int e = 0; e < E; e++) s += x[e];
-            // lanes sharing a group: int4 -> 32/E lanes, int2 -> all 32
             constexpr int LANES = (KF == KVQ_INT4_ASYM) ? 32 / E : 32;
 #pragma unroll
             for (int m = 1; m < LANES; m <<= 1) s += __shfl_xor_sync(kFull, s, m);
@@ -382,6 +415,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
         fence_mbar_init();
     }
     __syncthreads();
+    // signed 7-bit digits of q*2^E in the virtual channel order of the codes
+    for (int idx = tid; idx < NT * KC::KQ * 8 * 32; idx += kDecodeThreads) {
+        const int k = idx & 31, col = (idx >> 5) & 7, kq = (idx >> 8) % KC::KQ, nt = (idx >> 8) / KC::KQ;
+        int head, digit;
+        col_src<G8>(nt, col, head, digit);
+        int v = 0;
+        if (digit >= 0 && head < g) {
+            const int Q = __float2int_rn(ldexpf(qf[head * D + KC::chan(kq, k)], qexp[head]));
+            const int d3 = ((Q + 64) & 127) - 64;
+            const int R = (Q - d3) >> 7;
+            const int d2 = ((R + 64) & 127) - 64;
+            const int d1 = (R - d2) >> 7;
+            v = digit == 0 ? d1 : digit == 1 ? d2 : d3;
+        }
+        qv[idx] = (int8_t)v;
+    }
+    __syncthreads();
 
     // ---- this warp's pages ----
     const int p_begin = split * p.pages_per_split + warp * p.pages_per_warp;
@@ -390,7 +440,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
     const int32_t *bt = p.block_table + (long long)b * p.max_pages;
     const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
 
-    // page ids of pages [i0, i0+32) of this warp, one per lane
     auto fetch_ids = [&](int i0) -> int {
         const int i = i0 + lane;
         int pg = -1;
@@ -419,40 +468,49 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
     };
     for (int i = 0; i < NST && i < npg; i++) issue(i);
 
-    // ---- query fragments (A operands) ----
-    uint32_t aq[C::KST][4];
+    // ---- per-lane constants: query digit B fragments, zero-term B fragments ----
+    uint32_t qb[NT][KC::KQ][2];
 #pragma unroll
-    for (int ks = 0; ks < C::KST; ks++) {
+    for (int nt = 0; nt < NT; nt++)
 #pragma unroll
-        for (int half = 0; half < 2; half++) {
-            const int kk = 2 * j + 8 * half;
-            uint32_t hi = 0, lo = 0;
-            if (r < g) {
-                const float x0 = qs[r * D + KC::chan(ks, kk)], x1 = qs[r * D + KC::chan(ks, kk + 1)];
-                const __half2 h2 = __floats2half2_rn(x0, x1);
-                hi = h2_bits(h2);
-                lo = pack_h2(x0 - __low2float(h2), x1 - __high2float(h2));
-            }
-            aq[ks][2 * half] = hi;
-            aq[ks][2 * half + 1] = lo;
+        for (int kq = 0; kq < KC::KQ; kq++) {
+            const int8_t *src = qv + ((nt * KC::KQ + kq) * 8 + r) * 32;
+            qb[nt][kq][0] = *reinterpret_cast<const uint32_t *>(src + 4 * j);
+            qb[nt][kq][1] = *reinterpret_cast<const uint32_t *>(src + 16 + 4 * j);
         }
-    }
-    uint32_t aqz[4] = {0, 0, 0, 0};
+    uint32_t zb[NH];
+#pragma unroll
+    for (int t = 0; t < NH; t++) zb[t] = 0u;
     if constexpr (KC::ZERO) {
-        if (r < g && 2 * j < KC::NG) {
-            const float x0 = qsum[r * 4 + 2 * j];
-            const float x1 = (2 * j + 1 < KC::NG) ? qsum[r * 4 + 2 * j + 1] : 0.f;
-            const __half2 h2 = __floats2half2_rn(x0, x1);
-            aqz[0] = h2_bits(h2);
-            aqz[1] = pack_h2(x0 - __low2float(h2), x1 - __high2float(h2));
+#pragma unroll
+        for (int t = 0; t < NH; t++) {
+            const int head = (r >> 1) + 4 * t;
+            if (head < g && 2 * j < KC::NG) {
+                float q0 = qsum[head * 4 + 2 * j];
+                float q1 = (2 * j + 1 < KC::NG) ? qsum[head * 4 + 2 * j + 1] : 0.f;
+                if (r & 1) {  // low part
+                    q0 -= __half2float(__float2half_rn(q0));
+                    q1 -= __half2float(__float2half_rn(q1));
+                }
+                zb[t] = pack_h2(q0, q1);
+            }
         }
     }
-
-    float oacc[C::MT][4];
+    float qinv[NH];
 #pragma unroll
-    for (int mt = 0; mt < C::MT; mt++) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
-    float oz[4] = {0.f, 0.f, 0.f, 0.f};
-    float m_run = -INFINITY, l_part = 0.f;
+    for (int t = 0; t < NH; t++) qinv[t] = (j + 4 * t < g) ? ldexpf(1.f, -qexp[j + 4 * t]) : 0.f;
+
+    float oacc[NH][C::MT][4];
+    float oz[NH][4];
+    float m_run[NH], l_part[NH];
+#pragma unroll
+    for (int t = 0; t < NH; t++) {
+#pragma unroll
+        for (int mt = 0; mt < C::MT; mt++) oacc[t][mt][0] = oacc[t][mt][1] = oacc[t][mt][2] = oacc[t][mt][3] = 0.f;
+        oz[t][0] = oz[t][1] = oz[t][2] = oz[t][3] = 0.f;
+        m_run[t] = -INFINITY;
+        l_part[t] = 0.f;
+    }
 
     for (int i = 0; i < npg; i++) {
         const int st = i % NST;
@@ -470,130 +528,188 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
         const uint32_t sb = stage0 + st * C::STAGE;
         const unsigned char *sp = stage0_ptr + st * C::STAGE;
         const bool page_ok = (vbits >> st) & 1u;
+        const bool ragged = nvalid < kPageTokens || !page_ok;
 
-        // per-thread tokens of the score fragment / PV B operand
-        const int tk[4] = {2 * j, 2 * j + 1, 2 * j + 8, 2 * j + 9};
-
-        // ---------------- QK ----------------
-        float sk[4][KC::NG];
+        // ---------------- QK: scores of tokens r, r+8 for the lane's heads ----
+        float s_r[NH], s_r8[NH];
+        {
+            uint32_t kw[KC::NCH], kw8[KC::NCH];
+            ld_krows<KC::NCH>(sb + C::K_CODES, lane, kw, kw8);
+            const unsigned char *meta_r = sp + C::K_META + r * KC::ROW_META;
+            const unsigned char *meta_r8 = sp + C::K_META + (r + 8) * KC::ROW_META;
+            float zr[NH], zr8[NH];
 #pragma unroll
-        for (int q = 0; q < 4; q++) {
-            const unsigned char *mrow = sp + C::K_META + tk[q] * KC::ROW_META;
-#pragma unroll
-            for (int gi = 0; gi < KC::NG; gi++) sk[q][gi] = h2f_bits(*reinterpret_cast<const uint16_t *>(mrow + 2 * gi));
-        }
-        float sc[4];
-#pragma unroll
-        for (int nt = 0; nt < 2; nt++) {
-            uint32_t kw[KC::NCH];
-            ld_rows<KC::NCH>(sb + C::K_CODES, nt, lane, kw);
-            float dz[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int t = 0; t < NH; t++) zr[t] = zr8[t] = 0.f;
             if constexpr (KC::ZERO) {
-                const unsigned char *mrow = sp + C::K_META + (8 * nt + r) * KC::ROW_META + 2 * KC::NG;
-                uint32_t bz = 0;
+                uint32_t a[4] = {0u, 0u, 0u, 0u};
                 if constexpr (KC::NG >= 2) {
-                    if (2 * j < KC::NG) bz = *reinterpret_cast<const uint32_t *>(mrow + 4 * j);
+                    if (2 * j < KC::NG) {
+                        a[0] = *reinterpret_cast<const uint32_t *>(meta_r + 2 * KC::NG + 4 * j);
+                        a[1] = *reinterpret_cast<const uint32_t *>(meta_r8 + 2 * KC::NG + 4 * j);
+                    }
                 } else {
-                    if (j == 0) bz = *reinterpret_cast<const uint16_t *>(mrow);
+                    if (j == 0) {
+                        a[0] = *reinterpret_cast<const uint16_t *>(meta_r + 2);
+                        a[1] = *reinterpret_cast<const uint16_t *>(meta_r8 + 2);
+                    }
                 }
-                mma16816(dz, aqz, bz, 0u);
+#pragma unroll
+                for (int t = 0; t < NH; t++) {
+                    float dz[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma16816(dz, a, zb[t], 0u);
+                    zr[t] = dz[0] + dz[1];
+                    zr8[t] = dz[2] + dz[3];
+                }
             }
-            float s0 = dz[0] + dz[2], s1 = dz[1] + dz[3];
+            float acc_r[NH], acc_r8[NH];
+#pragma unroll
+            for (int t = 0; t < NH; t++) acc_r[t] = acc_r8[t] = 0.f;
 #pragma unroll
             for (int gi = 0; gi < KC::NG; gi++) {
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                int d[NT][4];
 #pragma unroll
-                for (int c = 0; c < KC::NCH; c++) {
-                    if (KC::group_of_chunk(c) != gi) continue;
-                    uint32_t bb[KC::KS_PER_CHUNK][2];
-                    KC::unpack(kw[c], bb);
+                for (int nt = 0; nt < NT; nt++) d[nt][0] = d[nt][1] = d[nt][2] = d[nt][3] = 0;
 #pragma unroll
-                    for (int u = 0; u < KC::KS_PER_CHUNK; u++)
-                        mma16816(acc, aq[c * KC::KS_PER_CHUNK + u], bb[u][0], bb[u][1]);
+                for (int kq = 0; kq < KC::KQ; kq++) {
+                    if (KC::group_of_kq(kq) != gi) continue;
+                    uint32_t a[4];
+                    KC::afrag(kw, kw8, kq, a);
+#pragma unroll
+                    for (int nt = 0; nt < NT; nt++) imma16832(d[nt], a, qb[nt][kq][0], qb[nt][kq][1]);
                 }
-                s0 = fmaf(sk[2 * nt][gi], acc[0] + acc[2], s0);
-                s1 = fmaf(sk[2 * nt + 1][gi], acc[1] + acc[3], s1);
-            }
-            sc[2 * nt] = s0;
-            sc[2 * nt + 1] = s1;
-        }
-        if (nvalid < kPageTokens || !page_ok) {
+                const float sk_r = h2f_bits(*reinterpret_cast<const uint16_t *>(meta_r + 2 * gi));
+                const float sk_r8 = h2f_bits(*reinterpret_cast<const uint16_t *>(meta_r8 + 2 * gi));
 #pragma unroll
-            for (int q = 0; q < 4; q++)
-                if (tk[q] >= nvalid || !page_ok) sc[q] = -INFINITY;
+                for (int t = 0; t < NH; t++) {
+                    // digits of head j + 4t: (d1, d2, d3) for row r (c0/c1) and r+8 (c2/c3)
+                    const int n12 = G8 ? t : 0, n3 = G8 ? 2 : 1, c3 = G8 ? t : 0;
+                    float v_r, v_r8;
+                    if constexpr (KF == KVQ_INT8_SYM) {
+                        v_r = fmaf(__int2float_rn(d[n12][0]), 16384.f,
+                                   fmaf(__int2float_rn(d[n12][1]), 128.f, __int2float_rn(d[n3][c3])));
+                        v_r8 = fmaf(__int2float_rn(d[n12][2]), 16384.f,
+                                    fmaf(__int2float_rn(d[n12][3]), 128.f, __int2float_rn(d[n3][2 + c3])));
+                    } else {
+                        v_r = __int2float_rn(d[n12][0] * 16384 + d[n12][1] * 128 + d[n3][c3]);
+                        v_r8 = __int2float_rn(d[n12][2] * 16384 + d[n12][3] * 128 + d[n3][2 + c3]);
+                    }
+                    acc_r[t] = fmaf(sk_r, v_r, acc_r[t]);
+                    acc_r8[t] = fmaf(sk_r8, v_r8, acc_r8[t]);
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < NH; t++) {
+                s_r[t] = fmaf(acc_r[t], qinv[t], zr[t]);
+                s_r8[t] = fmaf(acc_r8[t], qinv[t], zr8[t]);
+                if (ragged) {
+                    if (r >= nvalid || !page_ok) s_r[t] = -INFINITY;
+                    if (r + 8 >= nvalid || !page_ok) s_r8[t] = -INFINITY;
+                }
+            }
         }
 
         // ---------------- online softmax (log2 domain) ----------------
-        float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-        const bool need = mx > m_run + 8.0f;
-        if (__any_sync(kFull, need)) {
-            const float m_new = need ? mx : m_run;
-            const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
-            m_run = m_new;
-            l_part *= alpha;
-            const float a0 = __shfl_sync(kFull, alpha, 8 * j), a1 = __shfl_sync(kFull, alpha, 8 * j + 4);
+        float p_r[NH], p_r8[NH];
+        {
+            float mx[NH];
+            bool need = false;
 #pragma unroll
-            for (int mt = 0; mt < C::MT; mt++) {
-                oacc[mt][0] *= a0;
-                oacc[mt][1] *= a1;
-                oacc[mt][2] *= a0;
-                oacc[mt][3] *= a1;
+            for (int t = 0; t < NH; t++) {
+                float m = fmaxf(s_r[t], s_r8[t]);
+                m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
+                m = fmaxf(m, __shfl_xor_sync(kFull, m, 8));
+                m = fmaxf(m, __shfl_xor_sync(kFull, m, 16));
+                mx[t] = m;
+                need |= m > m_run[t] + 8.0f;
             }
-            oz[0] *= a0;
-            oz[1] *= a1;
-            oz[2] *= a0;
-            oz[3] *= a1;
-        }
-        float pr[4];
+            if (__any_sync(kFull, need)) {
 #pragma unroll
-        for (int q = 0; q < 4; q++) {
-            pr[q] = (m_run == -INFINITY) ? 0.f : exp2f(sc[q] - m_run);
-            l_part += pr[q];
+                for (int t = 0; t < NH; t++) {
+                    const float m_new = mx[t] > m_run[t] + 8.0f ? mx[t] : m_run[t];
+                    const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_run[t] - m_new);
+                    m_run[t] = m_new;
+                    l_part[t] *= alpha;
+#pragma unroll
+                    for (int mt = 0; mt < C::MT; mt++) {
+                        oacc[t][mt][0] *= alpha;
+                        oacc[t][mt][1] *= alpha;
+                        oacc[t][mt][2] *= alpha;
+                        oacc[t][mt][3] *= alpha;
+                    }
+                    oz[t][0] *= alpha;
+                    oz[t][1] *= alpha;
+                    oz[t][2] *= alpha;
+                    oz[t][3] *= alpha;
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < NH; t++) {
+                const bool live = m_run[t] != -INFINITY;
+                p_r[t] = live ? ex2(s_r[t] - m_run[t]) : 0.f;
+                p_r8[t] = live ? ex2(s_r8[t] - m_run[t]) : 0.f;
+                l_part[t] += p_r[t] + p_r8[t];
+            }
         }
 
         // ---------------- PV ----------------
-        float sv[4][VC::NG];
-        uint16_t zv[4];
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-            const unsigned char *mrow = sp + C::V_META + tk[q] * VC::ROW_META;
-            const bool valid = page_ok && tk[q] < nvalid;
-#pragma unroll
-            for (int gi = 0; gi < VC::NG; gi++)
-                sv[q][gi] = valid ? h2f_bits(*reinterpret_cast<const uint16_t *>(mrow + 2 * gi)) : 0.f;
-            zv[q] = (valid && r < VC::NG) ? *reinterpret_cast<const uint16_t *>(mrow + 2 * VC::NG + 2 * r) : 0;
-        }
-        // p and p*scale enter the MMAs as fp16 hi + lo pairs (two MMAs each),
-        // so the weights carry ~22 bits instead of fp16's 11
         {
-            uint32_t ph[2], pl[2];
-            split_pair(pr[0], pr[1], ph[0], pl[0]);
-            split_pair(pr[2], pr[3], ph[1], pl[1]);
-            const uint32_t az[4] = {uint32_t(zv[0]) | (uint32_t(zv[1]) << 16), 0u,
-                                    uint32_t(zv[2]) | (uint32_t(zv[3]) << 16), 0u};
-            mma16816(oz, az, ph[0], ph[1]);
-            mma16816(oz, az, pl[0], pl[1]);
-        }
-        uint32_t wh[VC::NG][2], wl[VC::NG][2];
+            const unsigned char *vmeta_r = sp + C::V_META + r * VC::ROW_META;
+            const unsigned char *vmeta_r8 = sp + C::V_META + (r + 8) * VC::ROW_META;
+            float sv_r[VC::NG], sv_r8[VC::NG];
 #pragma unroll
-        for (int gi = 0; gi < VC::NG; gi++) {
-            split_pair(pr[0] * sv[0][gi], pr[1] * sv[1][gi], wh[gi][0], wl[gi][0]);
-            split_pair(pr[2] * sv[2][gi], pr[3] * sv[3][gi], wh[gi][1], wl[gi][1]);
-        }
-        uint32_t vA[VC::NCH], vB[VC::NCH];
-        ld_rows_t<VC::NCH>(sb + C::V_CODES, lane, vA, vB);
+            for (int gi = 0; gi < VC::NG; gi++) {
+                sv_r[gi] = h2f_bits(*reinterpret_cast<const uint16_t *>(vmeta_r + 2 * gi));
+                sv_r8[gi] = h2f_bits(*reinterpret_cast<const uint16_t *>(vmeta_r8 + 2 * gi));
+            }
+            if (ragged) {
+                const bool v_r = page_ok && r < nvalid, v_r8 = page_ok && r + 8 < nvalid;
 #pragma unroll
-        for (int c = 0; c < VC::NCH; c++) {
+                for (int gi = 0; gi < VC::NG; gi++) {
+                    sv_r[gi] = v_r ? sv_r[gi] : 0.f;
+                    sv_r8[gi] = v_r8 ? sv_r8[gi] : 0.f;
+                }
+            }
+            // zero term: A = zeros^T (group r, tokens 2j, 2j+1 | 2j+8, 2j+9)
+            uint32_t az[4] = {0u, 0u, 0u, 0u};
+            if (r < VC::NG) {
+                const unsigned char *zrow = sp + C::V_META + 2 * VC::NG + 2 * r;
+                uint32_t z0 = *reinterpret_cast<const uint16_t *>(zrow + (2 * j) * VC::ROW_META);
+                uint32_t z1 = *reinterpret_cast<const uint16_t *>(zrow + (2 * j + 1) * VC::ROW_META);
+                uint32_t z2 = *reinterpret_cast<const uint16_t *>(zrow + (2 * j + 8) * VC::ROW_META);
+                uint32_t z3 = *reinterpret_cast<const uint16_t *>(zrow + (2 * j + 9) * VC::ROW_META);
+                if (ragged) {
+                    if (!page_ok || 2 * j >= nvalid) z0 = 0;
+                    if (!page_ok || 2 * j + 1 >= nvalid) z1 = 0;
+                    if (!page_ok || 2 * j + 8 >= nvalid) z2 = 0;
+                    if (!page_ok || 2 * j + 9 >= nvalid) z3 = 0;
+                }
+                az[0] = z0 | (z1 << 16);
+                az[2] = z2 | (z3 << 16);
+            }
+            uint32_t vA[VC::NCH], vB[VC::NCH];
+            ld_vrows_t<VC::NCH>(sb + C::V_CODES, lane, vA, vB);
 #pragma unroll
-            for (int u = 0; u < VC::MT_PER_CHUNK; u++) {
-                const int mt = c * VC::MT_PER_CHUNK + u;
-                uint32_t a[4];
-                VC::afrag(vA[c], vB[c], u, a);
-                const int gi = VC::group_of_mt(mt);
-                mma16816(oacc[mt], a, wh[gi][0], wh[gi][1]);
-                mma16816(oacc[mt], a, wl[gi][0], wl[gi][1]);
+            for (int t = 0; t < NH; t++) {
+                // p as (hi, lo) columns, transposed into B layout
+                const uint32_t bz0 = movm_t(hilo(p_r[t])), bz1 = movm_t(hilo(p_r8[t]));
+                mma16816(oz[t], az, bz0, bz1);
+                uint32_t wb[VC::NG][2];
+#pragma unroll
+                for (int gi = 0; gi < VC::NG; gi++) {
+                    wb[gi][0] = movm_t(hilo(p_r[t] * sv_r[gi]));
+                    wb[gi][1] = movm_t(hilo(p_r8[t] * sv_r8[gi]));
+                }
+#pragma unroll
+                for (int c = 0; c < VC::NCH; c++) {
+#pragma unroll
+                    for (int u = 0; u < VC::MT_PER_CHUNK; u++) {
+                        const int mt = c * VC::MT_PER_CHUNK + u;
+                        uint32_t a[4];
+                        VC::afrag(vA[c], vB[c], u, a);
+                        const int gi = VC::group_of_mt(mt);
+                        mma16816(oacc[t][mt], a, wb[gi][0], wb[gi][1]);
+                    }
+                }
             }
         }
 
@@ -607,29 +723,32 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
     }
 
     // ---- warp state -> shared memory, CTA merge ----
-    l_part += __shfl_xor_sync(kFull, l_part, 1);
-    l_part += __shfl_xor_sync(kFull, l_part, 2);
+#pragma unroll
+    for (int t = 0; t < NH; t++) {
+        l_part[t] += __shfl_xor_sync(kFull, l_part[t], 4);
+        l_part[t] += __shfl_xor_sync(kFull, l_part[t], 8);
+        l_part[t] += __shfl_xor_sync(kFull, l_part[t], 16);
+    }
     __syncthreads();  // every warp is done with the stage ring
     float *macc = reinterpret_cast<float *>(smem + C::MERGE_ACC);
     float *mz = reinterpret_cast<float *>(smem + C::MERGE_Z);
     float *mm = reinterpret_cast<float *>(smem + C::MERGE_M);
     float *ml = reinterpret_cast<float *>(smem + C::MERGE_L);
 #pragma unroll
-    for (int mt = 0; mt < C::MT; mt++) {
+    for (int t = 0; t < NH; t++) {
+        const int head = j + 4 * t;
+        if (head < g) {
 #pragma unroll
-        for (int q = 0; q < 4; q++) {
-            const int row = r + 8 * (q >> 1), col = 2 * j + (q & 1);
-            if (col < g) macc[(warp * kMaxGqa + col) * D + VC::chan(mt, row)] = oacc[mt][q];
+            for (int mt = 0; mt < C::MT; mt++) {
+                macc[(warp * kMaxGqa + head) * D + VC::chan(mt, r)] = oacc[t][mt][0] + oacc[t][mt][1];
+                macc[(warp * kMaxGqa + head) * D + VC::chan(mt, r + 8)] = oacc[t][mt][2] + oacc[t][mt][3];
+            }
+            if (r < VC::NG) mz[(warp * 4 + r) * kMaxGqa + head] = oz[t][0] + oz[t][1];
+            if (r == 0) {
+                mm[warp * kMaxGqa + head] = m_run[t];
+                ml[warp * kMaxGqa + head] = l_part[t];
+            }
         }
-    }
-#pragma unroll
-    for (int q = 0; q < 2; q++) {
-        const int col = 2 * j + q;
-        if (r < VC::NG && col < g) mz[(warp * 4 + r) * kMaxGqa + col] = oz[q];
-    }
-    if (j == 0 && r < g) {
-        mm[warp * kMaxGqa + r] = m_run;
-        ml[warp * kMaxGqa + r] = l_part;
     }
     __syncthreads();
 
@@ -645,7 +764,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
 #pragma unroll
             for (int w = 0; w < kDecodeWarps; w++) {
                 const float mw = mm[w * kMaxGqa + h];
-                const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+                const float f = (mw == -INFINITY) ? 0.f : ex2(mw - M);
                 acc += f * (macc[(w * kMaxGqa + h) * D + ch] + mz[(w * 4 + VC::group_of_chan(ch)) * kMaxGqa + h]);
                 Lsum += f * ml[w * kMaxGqa + h];
             }
@@ -670,37 +789,71 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
     __threadfence();
     if (tid == 0) p.counters[b * L.hkv + kvh] = 0u;
 
+    // scratch in the ring: pw[n*g] split weights, po[g][D] merged output, pL[g]
+    float *pw = reinterpret_cast<float *>(smem);
+    float *po = pw + n_active * g;
+    float *pL = po + g * D;
+    // (1) per head: max over splits, weights e^(m - M), total sum L
     for (int h = warp; h < g; h += kDecodeWarps) {
         float M = -INFINITY;
-        for (int s = lane; s < n_active; s += 32) M = fmaxf(M, __ldcg(part_base + ((long long)s * g + h) * (D + 4) + D));
+        for (int s = lane; s < n_active; s += 32)
+            M = fmaxf(M, __ldcg(part_base + ((long long)s * g + h) * (D + 4) + D));
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, m));
-        float o[E];
+        float Ls = 0.f;
+        for (int s = lane; s < n_active; s += 32) {
+            const float *src = part_base + ((long long)s * g + h) * (D + 4);
+            const float ms = __ldcg(src + D), ls = __ldcg(src + D + 1);
+            const float f = (ms == -INFINITY || M == -INFINITY) ? 0.f : ex2(ms - M);
+            pw[s * g + h] = f;
+            Ls += f * ls;
+        }
 #pragma unroll
-        for (int e = 0; e < E; e++) o[e] = 0.f;
-        float Lsum = 0.f;
-        if (M != -INFINITY) {
-            for (int s = 0; s < n_active; s++) {
-                const float *src = part_base + ((long long)s * g + h) * (D + 4);
-                const float ms = __ldcg(src + D), ls = __ldcg(src + D + 1);
-                const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-                Lsum += f * ls;
-                if constexpr (E == 4) {
-                    const float4 v = __ldcg(reinterpret_cast<const float4 *>(src) + lane);
-                    o[0] += f * v.x;
-                    o[1] += f * v.y;
-                    o[2] += f * v.z;
-                    o[3] += f * v.w;
-                } else {
-                    const float2 v = __ldcg(reinterpret_cast<const float2 *>(src) + lane);
-                    o[0] += f * v.x;
-                    o[1] += f * v.y;
+        for (int m = 16; m >= 1; m >>= 1) Ls += __shfl_xor_sync(kFull, Ls, m);
+        if (lane == 0) pL[h] = Ls;
+    }
+    for (int idx = tid; idx < g * D; idx += kDecodeThreads) po[idx] = 0.f;
+    __syncthreads();
+    // (2) weighted sum of the split accumulators: every (split, head, float4)
+    //     is an independent load, 8 in flight per thread
+    {
+        constexpr int QUADS = D / 4;
+        const int items = n_active * g * QUADS;
+        for (int base = tid; base < items; base += 8 * kDecodeThreads) {
+            float4 v[8];
+            float f[8];
+            int dsti[8];
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const int it = base + u * kDecodeThreads;
+                f[u] = 0.f;
+                dsti[u] = -1;
+                if (it < items) {
+                    const int qd = it % QUADS, sh = it / QUADS, h = sh % g, s = sh / g;
+                    v[u] = __ldcg(reinterpret_cast<const float4 *>(part_base + ((long long)s * g + h) * (D + 4)) + qd);
+                    f[u] = pw[s * g + h];
+                    dsti[u] = h * D + 4 * qd;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                if (dsti[u] >= 0 && f[u] != 0.f) {
+                    atomicAdd(po + dsti[u] + 0, f[u] * v[u].x);
+                    atomicAdd(po + dsti[u] + 1, f[u] * v[u].y);
+                    atomicAdd(po + dsti[u] + 2, f[u] * v[u].z);
+                    atomicAdd(po + dsti[u] + 3, f[u] * v[u].w);
                 }
             }
         }
-        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    }
+    __syncthreads();
+    // (3) normalise, inverse rotation, store
+    for (int h = warp; h < g; h += kDecodeWarps) {
+        const float Ls = pL[h];
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+        float o[E];
 #pragma unroll
-        for (int e = 0; e < E; e++) o[e] *= inv;
+        for (int e = 0; e < E; e++) o[e] = po[h * D + lane * E + e] * inv;
         if (p.rotate) {
             fwht_warp<D>(o, lane);
 #pragma unroll
@@ -715,19 +868,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const __grid_
     }
 }
 
-template <int D, int KF, int VF>
+template <int D, int KF, int VF, bool G8>
 cudaError_t launch_t(const DecodeParams &p, dim3 grid, cudaStream_t s)
 {
-    using C = Cfg<KF, VF, D>;
+    using C = Cfg<KF, VF, D, G8>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, KF, VF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, KF, VF, G8>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    decode_kernel<D, KF, VF><<<grid, kDecodeThreads, C::SMEM, s>>>(p);
+    decode_kernel<D, KF, VF, G8><<<grid, kDecodeThreads, C::SMEM, s>>>(p);
     return cudaGetLastError();
+}
+
+template <int D, int KF, int VF>
+cudaError_t launch_g(const DecodeParams &p, dim3 grid, cudaStream_t s)
+{
+    return p.L.g > 4 ? launch_t<D, KF, VF, true>(p, grid, s) : launch_t<D, KF, VF, false>(p, grid, s);
 }
 
 }  // namespace
@@ -740,21 +899,29 @@ bool decode_supported(const Layout &L)
     return L.d == 128;
 }
 
+int decode_max_splits(const Layout &L)
+{
+    // the final merge keeps n*g weights, g*d outputs and g sums (fp32) in the
+    // smallest ring of any instantiation (8 warps x 4 stages x 1152 bytes)
+    const int ring_floats = kDecodeWarps * 4 * 1152 / 4;
+    return (ring_floats - L.g * L.d - L.g) / L.g;
+}
+
 cudaError_t launch_decode(const DecodeParams &p, dim3 grid, cudaStream_t s)
 {
     const Layout &L = p.L;
-    if (L.d == 64) return launch_t<64, KVQ_INT4_ASYM, KVQ_INT4_ASYM>(p, grid, s);
+    if (L.d == 64) return launch_g<64, KVQ_INT4_ASYM, KVQ_INT4_ASYM>(p, grid, s);
     if (L.v_fmt == KVQ_INT4_ASYM) {
         switch (L.k_fmt) {
-        case KVQ_INT4_ASYM: return launch_t<128, KVQ_INT4_ASYM, KVQ_INT4_ASYM>(p, grid, s);
-        case KVQ_INT8_SYM: return launch_t<128, KVQ_INT8_SYM, KVQ_INT4_ASYM>(p, grid, s);
-        default: return launch_t<128, KVQ_INT2_ASYM, KVQ_INT4_ASYM>(p, grid, s);
+        case KVQ_INT4_ASYM: return launch_g<128, KVQ_INT4_ASYM, KVQ_INT4_ASYM>(p, grid, s);
+        case KVQ_INT8_SYM: return launch_g<128, KVQ_INT8_SYM, KVQ_INT4_ASYM>(p, grid, s);
+        default: return launch_g<128, KVQ_INT2_ASYM, KVQ_INT4_ASYM>(p, grid, s);
         }
     }
     switch (L.k_fmt) {
-    case KVQ_INT4_ASYM: return launch_t<128, KVQ_INT4_ASYM, KVQ_INT2_ASYM>(p, grid, s);
-    case KVQ_INT8_SYM: return launch_t<128, KVQ_INT8_SYM, KVQ_INT2_ASYM>(p, grid, s);
-    default: return launch_t<128, KVQ_INT2_ASYM, KVQ_INT2_ASYM>(p, grid, s);
+    case KVQ_INT4_ASYM: return launch_g<128, KVQ_INT4_ASYM, KVQ_INT2_ASYM>(p, grid, s);
+    case KVQ_INT8_SYM: return launch_g<128, KVQ_INT8_SYM, KVQ_INT2_ASYM>(p, grid, s);
+    default: return launch_g<128, KVQ_INT2_ASYM, KVQ_INT2_ASYM>(p, grid, s);
     }
 }
 

@@ -132,6 +132,7 @@ cudaError_t launch_decode(const DecodeParams &p, dim3 grid, cudaStream_t s);
 cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
 cudaError_t launch_reset_pages(unsigned char *pool, Layout L, const int32_t *pages, int n, cudaStream_t s);
 bool decode_supported(const Layout &L);
+int decode_max_splits(const Layout &L);
 constexpr int kDecodeWarps = 8;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
 
