@@ -124,6 +124,12 @@ template <int D> struct KCodec<KVQ_INT4_ASYM, D> {
     static constexpr int ROW_META = 4 * NG;
     __device__ static int chan(int kq, int k) { return 32 * kq + 8 * ((k & 15) >> 2) + 2 * (k & 3) + (k >> 4); }
     __device__ static int group_of_kq(int kq) { return kq; }
+    __device__ static void inv_chan(int ch, int &kq, int &k)
+    {
+        const int c = ch & 31;
+        kq = ch >> 5;
+        k = 16 * (c & 1) + 4 * (c >> 3) + ((c >> 1) & 3);
+    }
     // w[c] / w8[c]: word j of chunk c for tokens r / r+8
     __device__ static void afrag(const uint32_t (&w)[NCH], const uint32_t (&w8)[NCH], int kq, uint32_t (&a)[4])
     {
@@ -142,6 +148,11 @@ template <int D> struct KCodec<KVQ_INT8_SYM, D> {
     static constexpr int ROW_META = 2;
     __device__ static int chan(int kq, int k) { return 32 * kq + k; }
     __device__ static int group_of_kq(int) { return 0; }
+    __device__ static void inv_chan(int ch, int &kq, int &k)
+    {
+        kq = ch >> 5;
+        k = ch & 31;
+    }
     __device__ static void afrag(const uint32_t (&w)[NCH], const uint32_t (&w8)[NCH], int kq, uint32_t (&a)[4])
     {
         a[0] = w[2 * kq];
@@ -162,6 +173,12 @@ template <int D> struct KCodec<KVQ_INT2_ASYM, D> {
         return 64 * (kq >> 1) + 16 * ((k & 15) >> 2) + 4 * (k & 3) + 2 * (kq & 1) + (k >> 4);
     }
     __device__ static int group_of_kq(int) { return 0; }
+    __device__ static void inv_chan(int ch, int &kq, int &k)
+    {
+        const int rem = ch & 63;
+        kq = 2 * (ch >> 6) + ((rem >> 1) & 1);
+        k = 16 * (rem & 1) + 4 * (rem >> 4) + ((rem >> 2) & 3);
+    }
     __device__ static void afrag(const uint32_t (&w)[NCH], const uint32_t (&w8)[NCH], int kq, uint32_t (&a)[4])
     {
         const int c = kq >> 1, s = 2 * (kq & 1);
@@ -230,8 +247,7 @@ template <int KF, int VF, int D, bool G8> struct Cfg {
     static constexpr int E = D / 32;   // elements per lane in warp-wide vectors
     // shared memory map
     static constexpr int RING = kDecodeWarps * NST * STAGE;
-    static constexpr int OFF_QF = RING;                             // f32 [8][D]
-    static constexpr int OFF_QV = OFF_QF + kMaxGqa * D * 4;          // s8 [NT][KQ][8][32]
+    static constexpr int OFF_QV = RING;                              // s8 [NT][KQ][8][32]
     static constexpr int OFF_QSUM = OFF_QV + NT * K::KQ * 8 * 32;    // f32 [8][4]
     static constexpr int OFF_QEXP = OFF_QSUM + kMaxGqa * 4 * 4;      // i32 [8]
     static constexpr int OFF_BAR = OFF_QEXP + kMaxGqa * 4;
@@ -327,6 +343,25 @@ __device__ __forceinline__ void col_src(int nt, int n, int &head, int &digit)
     }
 }
 
+// Column (n-tile, col) holding digit dg of head h (the inverse of col_src).
+template <bool G8>
+__device__ __forceinline__ void digit_col(int h, int dg, int &nt, int &col)
+{
+    if (!G8) {
+        nt = dg == 2 ? 1 : 0;
+        col = 2 * h + (dg == 1 ? 1 : 0);
+    } else {
+        const int hh = h & 3, hi = h >> 2;
+        if (dg < 2) {
+            nt = hi;
+            col = 2 * hh + dg;
+        } else {
+            nt = 2;
+            col = 2 * hh + hi;
+        }
+    }
+}
+
 template <int D, int KF, int VF, bool G8>
 __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(const __grid_constant__ DecodeParams p)
 {
@@ -354,7 +389,6 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     if (split >= n_active) return;
 
     extern __shared__ __align__(128) unsigned char smem[];
-    float *qf = reinterpret_cast<float *>(smem + C::OFF_QF);
     int8_t *qv = reinterpret_cast<int8_t *>(smem + C::OFF_QV);
     float *qsum = reinterpret_cast<float *>(smem + C::OFF_QSUM);
     int *qexp = reinterpret_cast<int *>(smem + C::OFF_QEXP);
@@ -363,82 +397,18 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     const uint32_t stage0 = smem_u32(smem) + warp * NST * C::STAGE;
     const unsigned char *stage0_ptr = smem + warp * NST * C::STAGE;
 
-    // ---- query: rotate, pre-scale, digit exponent, group sums (warp h) ----
-    for (int h = warp; h < g; h += kDecodeWarps) {
-        const __half *qh = p.q + ((long long)b * L.hq + kvh * g + h) * D + lane * E;
-        float x[E];
-        if constexpr (E == 4) {
-            const uint2 u = *reinterpret_cast<const uint2 *>(qh);
-            const float2 f0 = __half22float2(bits_h2(u.x)), f1 = __half22float2(bits_h2(u.y));
-            x[0] = f0.x;
-            x[1] = f0.y;
-            x[2] = f1.x;
-            x[3] = f1.y;
-        } else {
-            const float2 f0 = __half22float2(bits_h2(*reinterpret_cast<const uint32_t *>(qh)));
-            x[0] = f0.x;
-            x[1] = f0.y;
-        }
-        float sc = p.qscale;
-        if (p.rotate) {
-#pragma unroll
-            for (int e = 0; e < E; e++) x[e] *= p.signs[lane * E + e];
-            fwht_warp<D>(x, lane);
-            sc *= p.rot_scale;
-        }
-        float amax = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; e++) {
-            x[e] *= sc;
-            qf[h * D + lane * E + e] = x[e];
-            amax = fmaxf(amax, fabsf(x[e]));
-        }
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, m));
-        if (lane == 0) {
-            int ex = 0;
-            if (amax > 0.f) frexpf(amax, &ex);  // amax < 2^ex
-            qexp[h] = 20 - ex;                  // |q * 2^E| < 2^20
-        }
-        if constexpr (KC::ZERO) {
-            float s = 0.f;
-#pragma unroll
-            for (int e = 0; e < E; e++) s += x[e];
-            constexpr int LANES = (KF == KVQ_INT4_ASYM) ? 32 / E : 32;
-#pragma unroll
-            for (int m = 1; m < LANES; m <<= 1) s += __shfl_xor_sync(kFull, s, m);
-            if ((lane % LANES) == 0) qsum[h * 4 + (lane * E) / (KF == KVQ_INT4_ASYM ? 32 : D)] = s;
-        }
-    }
-    if (lane == 0) {
-        for (int s = 0; s < NST; s++) mbar_init(bar0 + 8 * s, 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    // signed 7-bit digits of q*2^E in the virtual channel order of the codes
-    for (int idx = tid; idx < NT * KC::KQ * 8 * 32; idx += kDecodeThreads) {
-        const int k = idx & 31, col = (idx >> 5) & 7, kq = (idx >> 8) % KC::KQ, nt = (idx >> 8) / KC::KQ;
-        int head, digit;
-        col_src<G8>(nt, col, head, digit);
-        int v = 0;
-        if (digit >= 0 && head < g) {
-            const int Q = __float2int_rn(ldexpf(qf[head * D + KC::chan(kq, k)], qexp[head]));
-            const int d3 = ((Q + 64) & 127) - 64;
-            const int R = (Q - d3) >> 7;
-            const int d2 = ((R + 64) & 127) - 64;
-            const int d1 = (R - d2) >> 7;
-            v = digit == 0 ? d1 : digit == 1 ? d2 : d3;
-        }
-        qv[idx] = (int8_t)v;
-    }
-    __syncthreads();
-
-    // ---- this warp's pages ----
+    // ---- this warp's pages: barriers and the first copies go out before
+    //      any query work, so the page data is in flight during it ----
     const int p_begin = split * p.pages_per_split + warp * p.pages_per_warp;
     const int p_end = min(p_begin + p.pages_per_warp, n_pages);
     const int npg = max(0, p_end - p_begin);
     const int32_t *bt = p.block_table + (long long)b * p.max_pages;
     const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
+    if (lane == 0) {
+        for (int s = 0; s < NST; s++) mbar_init(bar0 + 8 * s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
 
     auto fetch_ids = [&](int i0) -> int {
         const int i = i0 + lane;
@@ -467,6 +437,84 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         }
     };
     for (int i = 0; i < NST && i < npg; i++) issue(i);
+
+    // ---- query (warp h): rotate, pre-scale, group sums, and the three signed
+    //      7-bit digits of q * 2^E written straight into the B layout ----
+    for (int h = warp; h < g; h += kDecodeWarps) {
+        const __half *qh = p.q + ((long long)b * L.hq + kvh * g + h) * D + lane * E;
+        float x[E];
+        if constexpr (E == 4) {
+            const uint2 u = *reinterpret_cast<const uint2 *>(qh);
+            const float2 f0 = __half22float2(bits_h2(u.x)), f1 = __half22float2(bits_h2(u.y));
+            x[0] = f0.x;
+            x[1] = f0.y;
+            x[2] = f1.x;
+            x[3] = f1.y;
+        } else {
+            const float2 f0 = __half22float2(bits_h2(*reinterpret_cast<const uint32_t *>(qh)));
+            x[0] = f0.x;
+            x[1] = f0.y;
+        }
+        float sc = p.qscale;
+        if (p.rotate) {
+#pragma unroll
+            for (int e = 0; e < E; e++) x[e] *= p.signs[lane * E + e];
+            fwht_warp<D>(x, lane);
+            sc *= p.rot_scale;
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            x[e] *= sc;
+            amax = fmaxf(amax, fabsf(x[e]));
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, m));
+        // amax < 2^ex with ex = biased exponent - 126; E = 20 - ex keeps
+        // |q * 2^E| < 2^20, so the leading digit stays within +-64
+        const int ex = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFF) - 126 : 20;
+        const int Eh = max(-126, min(127, 20 - ex));
+        if (lane == 0) qexp[h] = Eh;
+        const float pw2 = __int_as_float((127 + Eh) << 23);
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            const int ch = lane * E + e;
+            const int Q = __float2int_rn(x[e] * pw2);
+            const int d3 = ((Q + 64) & 127) - 64;
+            const int R = (Q - d3) >> 7;
+            const int d2 = ((R + 64) & 127) - 64;
+            const int d1 = (R - d2) >> 7;
+            int kq, k;
+            KC::inv_chan(ch, kq, k);
+            const int dig[3] = {d1, d2, d3};
+#pragma unroll
+            for (int dg = 0; dg < 3; dg++) {
+                int nt, col;
+                digit_col<G8>(h, dg, nt, col);
+                qv[((nt * KC::KQ + kq) * 8 + col) * 32 + k] = (int8_t)dig[dg];
+            }
+        }
+        if constexpr (KC::ZERO) {
+            float sm = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; e++) sm += x[e];
+            constexpr int LANES = (KF == KVQ_INT4_ASYM) ? 32 / E : 32;
+#pragma unroll
+            for (int m = 1; m < LANES; m <<= 1) sm += __shfl_xor_sync(kFull, sm, m);
+            if ((lane % LANES) == 0) qsum[h * 4 + (lane * E) / (KF == KVQ_INT4_ASYM ? 32 : D)] = sm;
+        }
+    }
+    // warps without a head clear the digit columns no head writes
+    if (warp >= g) {
+        uint32_t *qv32 = reinterpret_cast<uint32_t *>(qv);
+        for (int idx = (warp - g) * 32 + lane; idx < NT * KC::KQ * 8 * 8; idx += (kDecodeWarps - g) * 32) {
+            const int col = (idx >> 3) & 7, nt = (idx >> 6) / KC::KQ;
+            int head, digit;
+            col_src<G8>(nt, col, head, digit);
+            if (digit < 0 || head >= g) qv32[idx] = 0u;
+        }
+    }
+    __syncthreads();
 
     // ---- per-lane constants: query digit B fragments, zero-term B fragments ----
     uint32_t qb[NT][KC::KQ][2];
@@ -498,7 +546,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     }
     float qinv[NH];
 #pragma unroll
-    for (int t = 0; t < NH; t++) qinv[t] = (j + 4 * t < g) ? ldexpf(1.f, -qexp[j + 4 * t]) : 0.f;
+    for (int t = 0; t < NH; t++) qinv[t] = (j + 4 * t < g) ? __int_as_float((127 - qexp[j + 4 * t]) << 23) : 0.f;
 
     float oacc[NH][C::MT][4];
     float oz[NH][4];
@@ -789,71 +837,69 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     __threadfence();
     if (tid == 0) p.counters[b * L.hkv + kvh] = 0u;
 
-    // scratch in the ring: pw[n*g] split weights, po[g][D] merged output, pL[g]
+    // scratch in the ring: pw[n*g] split max then weight, pl[n*g] split sums,
+    // pL[8] totals, po[nhalf][g][D] partial outputs
+    constexpr int QUADS = D / 4;
     float *pw = reinterpret_cast<float *>(smem);
-    float *po = pw + n_active * g;
-    float *pL = po + g * D;
-    // (1) per head: max over splits, weights e^(m - M), total sum L
+    float *pl = pw + n_active * g;
+    float *pL = pl + n_active * g;
+    float *po = pL + kMaxGqa;
+    // (1) warp h: one load round for every split's (m, l), then the weights
     for (int h = warp; h < g; h += kDecodeWarps) {
         float M = -INFINITY;
-        for (int s = lane; s < n_active; s += 32)
-            M = fmaxf(M, __ldcg(part_base + ((long long)s * g + h) * (D + 4) + D));
+        for (int s = lane; s < n_active; s += 32) {
+            const float *src = part_base + ((long long)s * g + h) * (D + 4);
+            const float ms = __ldcg(src + D), ls = __ldcg(src + D + 1);
+            pw[s * g + h] = ms;
+            pl[s * g + h] = ls;
+            M = fmaxf(M, ms);
+        }
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, m));
         float Ls = 0.f;
         for (int s = lane; s < n_active; s += 32) {
-            const float *src = part_base + ((long long)s * g + h) * (D + 4);
-            const float ms = __ldcg(src + D), ls = __ldcg(src + D + 1);
+            const float ms = pw[s * g + h];
             const float f = (ms == -INFINITY || M == -INFINITY) ? 0.f : ex2(ms - M);
             pw[s * g + h] = f;
-            Ls += f * ls;
+            Ls += f * pl[s * g + h];
         }
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) Ls += __shfl_xor_sync(kFull, Ls, m);
         if (lane == 0) pL[h] = Ls;
     }
-    for (int idx = tid; idx < g * D; idx += kDecodeThreads) po[idx] = 0.f;
     __syncthreads();
-    // (2) weighted sum of the split accumulators: every (split, head, float4)
-    //     is an independent load, 8 in flight per thread
-    {
-        constexpr int QUADS = D / 4;
-        const int items = n_active * g * QUADS;
-        for (int base = tid; base < items; base += 8 * kDecodeThreads) {
-            float4 v[8];
-            float f[8];
-            int dsti[8];
-#pragma unroll
-            for (int u = 0; u < 8; u++) {
-                const int it = base + u * kDecodeThreads;
-                f[u] = 0.f;
-                dsti[u] = -1;
-                if (it < items) {
-                    const int qd = it % QUADS, sh = it / QUADS, h = sh % g, s = sh / g;
-                    v[u] = __ldcg(reinterpret_cast<const float4 *>(part_base + ((long long)s * g + h) * (D + 4)) + qd);
-                    f[u] = pw[s * g + h];
-                    dsti[u] = h * D + 4 * qd;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 8; u++) {
-                if (dsti[u] >= 0 && f[u] != 0.f) {
-                    atomicAdd(po + dsti[u] + 0, f[u] * v[u].x);
-                    atomicAdd(po + dsti[u] + 1, f[u] * v[u].y);
-                    atomicAdd(po + dsti[u] + 2, f[u] * v[u].z);
-                    atomicAdd(po + dsti[u] + 3, f[u] * v[u].w);
-                }
-            }
+    // (2) each thread owns one (head, float4) of the output and a stride of
+    //     the splits; the loads are independent, unrolled 8 deep
+    const int items = g * QUADS;
+    const int nhalf = max(1, kDecodeThreads / items);
+    if (tid < items * nhalf) {
+        const int it = tid % items, half = tid / items;
+        const int h = it / QUADS, qd = it % QUADS;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int s = half; s < n_active; s += nhalf) {
+            const float f = pw[s * g + h];
+            const float4 v =
+                __ldcg(reinterpret_cast<const float4 *>(part_base + ((long long)s * g + h) * (D + 4)) + qd);
+            acc.x = fmaf(f, v.x, acc.x);
+            acc.y = fmaf(f, v.y, acc.y);
+            acc.z = fmaf(f, v.z, acc.z);
+            acc.w = fmaf(f, v.w, acc.w);
         }
+        *reinterpret_cast<float4 *>(po + (half * g + h) * D + 4 * qd) = acc;
     }
     __syncthreads();
-    // (3) normalise, inverse rotation, store
+    // (3) sum the strides, normalise, inverse rotation, store
     for (int h = warp; h < g; h += kDecodeWarps) {
         const float Ls = pL[h];
         const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
         float o[E];
 #pragma unroll
-        for (int e = 0; e < E; e++) o[e] = po[h * D + lane * E + e] * inv;
+        for (int e = 0; e < E; e++) {
+            float v = 0.f;
+            for (int hf = 0; hf < nhalf; hf++) v += po[(hf * g + h) * D + lane * E + e];
+            o[e] = v * inv;
+        }
         if (p.rotate) {
             fwht_warp<D>(o, lane);
 #pragma unroll
@@ -901,10 +947,10 @@ bool decode_supported(const Layout &L)
 
 int decode_max_splits(const Layout &L)
 {
-    // the final merge keeps n*g weights, g*d outputs and g sums (fp32) in the
-    // smallest ring of any instantiation (8 warps x 4 stages x 1152 bytes)
+    // the final merge keeps 2*n*g split values, 8 sums and up to 256*4 output
+    // floats in the smallest ring of any instantiation (8 warps x 4 x 1152 B)
     const int ring_floats = kDecodeWarps * 4 * 1152 / 4;
-    return (ring_floats - L.g * L.d - L.g) / L.g;
+    return (ring_floats - kMaxGqa - kDecodeThreads * 4) / (2 * L.g);
 }
 
 cudaError_t launch_decode(const DecodeParams &p, dim3 grid, cudaStream_t s)
