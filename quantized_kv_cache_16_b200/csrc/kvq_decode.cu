@@ -843,7 +843,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     float *pw = reinterpret_cast<float *>(smem);
     float *pl = pw + n_active * g;
     float *pL = pl + n_active * g;
-    float *po = pL + kMaxGqa;
+    float *po = pw + ((2 * n_active * g + kMaxGqa + 3) & ~3);  // 16-byte aligned for float4
     // (1) warp h: one load round for every split's (m, l), then the weights
     for (int h = warp; h < g; h += kDecodeWarps) {
         float M = -INFINITY;
