@@ -38,6 +38,7 @@ namespace kvq {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
+constexpr int kCombineSplits = 40;  // split records the last CTA can stage
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per stage wait
 
 // fp16x2 constants (bit patterns)
@@ -251,8 +252,12 @@ template <int KF, int VF, int D, bool G8> struct Cfg {
     static constexpr int OFF_QSUM = OFF_QV + NT * K::KQ * 8 * 32;    // f32 [8][4]
     static constexpr int OFF_QEXP = OFF_QSUM + kMaxGqa * 4 * 4;      // i32 [8]
     static constexpr int OFF_BAR = OFF_QEXP + kMaxGqa * 4;
-    static constexpr int OFF_FLAG = OFF_BAR + kDecodeWarps * NST * 8;
-    static constexpr int SMEM = OFF_FLAG + 16;
+    // the last CTA stages up to kCombineSplits split records per head there
+    static constexpr int GM = G8 ? kMaxGqa : 4;
+    static constexpr int COMB = kCombineSplits * GM * ((D + 4) * 4 + 4) + GM * D * 4 + kMaxGqa * 4;
+    static constexpr int END = OFF_BAR + kDecodeWarps * NST * 8;
+    static constexpr int OFF_FLAG = ((END > COMB ? END : COMB) + 7) / 8 * 8;
+    static constexpr int SMEM = OFF_FLAG + 16;  // flag (int) + the staging mbarrier
     // merge scratch (aliases the ring after the page loop)
     static constexpr int MERGE_ACC = 0;                                         // [W][8][D]
     static constexpr int MERGE_Z = MERGE_ACC + kDecodeWarps * kMaxGqa * D * 4;    // [W][4][8]
@@ -379,7 +384,18 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     const int r = lane >> 2, j = lane & 3;
     const int g = L.g;
 
+    // independent loads first: the context length, this warp's first 32
+    // block-table entries (speculative) and the query row all go out together
     int T = p.ctx_lens[b];
+    const int p_begin = split * p.pages_per_split + warp * p.pages_per_warp;
+    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
+    const int id_raw = (lane < p.pages_per_warp && p_begin + lane < p.max_pages) ? bt[p_begin + lane] : -1;
+    uint2 q_raw = make_uint2(0u, 0u);
+    if (warp < g) {
+        const __half *qh = p.q + ((long long)b * L.hq + kvh * g + warp) * D + lane * E;
+        if constexpr (E == 4) q_raw = *reinterpret_cast<const uint2 *>(qh);
+        else q_raw.x = *reinterpret_cast<const uint32_t *>(qh);
+    }
     if (T < 0 || T > p.max_pages * kPageTokens) {
         if (split == 0 && tid == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
         T = T < 0 ? 0 : p.max_pages * kPageTokens;
@@ -399,10 +415,8 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
 
     // ---- this warp's pages: barriers and the first copies go out before
     //      any query work, so the page data is in flight during it ----
-    const int p_begin = split * p.pages_per_split + warp * p.pages_per_warp;
     const int p_end = min(p_begin + p.pages_per_warp, n_pages);
     const int npg = max(0, p_end - p_begin);
-    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
     const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
     if (lane == 0) {
         for (int s = 0; s < NST; s++) mbar_init(bar0 + 8 * s, 1);
@@ -422,7 +436,14 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         }
         return pg;
     };
-    int ids = fetch_ids(0);  // page ids of the issue window [32k, 32k+32)
+    int ids = -1;  // page ids of the issue window [32k, 32k+32)
+    if (lane < npg) {
+        ids = id_raw;
+        if (ids < 0 || ids >= L.num_pages) {
+            set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
+            ids = -1;
+        }
+    }
     uint32_t vbits = 0;      // bit s: stage s holds a valid page
     auto issue = [&](int i) {  // every lane calls this
         const int pg = __shfl_sync(kFull, ids, i & 31);
@@ -440,18 +461,18 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
 
     // ---- query (warp h): rotate, pre-scale, group sums, and the three signed
     //      7-bit digits of q * 2^E written straight into the B layout ----
-    for (int h = warp; h < g; h += kDecodeWarps) {
-        const __half *qh = p.q + ((long long)b * L.hq + kvh * g + h) * D + lane * E;
+    if (warp < g) {
+        const int h = warp;
         float x[E];
         if constexpr (E == 4) {
-            const uint2 u = *reinterpret_cast<const uint2 *>(qh);
+            const uint2 u = q_raw;
             const float2 f0 = __half22float2(bits_h2(u.x)), f1 = __half22float2(bits_h2(u.y));
             x[0] = f0.x;
             x[1] = f0.y;
             x[2] = f1.x;
             x[3] = f1.y;
         } else {
-            const float2 f0 = __half22float2(bits_h2(*reinterpret_cast<const uint32_t *>(qh)));
+            const float2 f0 = __half22float2(bits_h2(q_raw.x));
             x[0] = f0.x;
             x[1] = f0.y;
         }
@@ -837,69 +858,57 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     __threadfence();
     if (tid == 0) p.counters[b * L.hkv + kvh] = 0u;
 
-    // scratch in the ring: pw[n*g] split max then weight, pl[n*g] split sums,
-    // pL[8] totals, po[nhalf][g][D] partial outputs
-    constexpr int QUADS = D / 4;
-    float *pw = reinterpret_cast<float *>(smem);
-    float *pl = pw + n_active * g;
-    float *pL = pl + n_active * g;
-    float *po = pw + ((2 * n_active * g + kMaxGqa + 3) & ~3);  // 16-byte aligned for float4
-    // (1) warp h: one load round for every split's (m, l), then the weights
+    // stage every split's partial record of this (sequence, kv head) in
+    // shared memory with one bulk copy (the records are contiguous), then
+    // merge from there: one global round trip instead of one per phase
+    constexpr int REC = D + 4;
+    const int nrec = n_active * g;
+    float *stage = reinterpret_cast<float *>(smem);
+    float *pw = stage + nrec * REC;
+    float *po = pw + nrec;
+    float *pL = po + g * D;
+    const uint32_t cbar = smem_u32(smem + C::OFF_FLAG + 8);
+    if (tid == 0) {
+        mbar_init(cbar, 1);
+        fence_mbar_init();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        bulk_load(smem_u32(stage), part_base, (uint32_t)(nrec * REC * 4), cbar);
+    }
+    __syncthreads();
+    if (!mbar_wait_bounded(cbar, 0, kWaitLimitNs)) set_status(p.pool, KVQ_ERR_TIMEOUT);
+    // (1) warp h: the max over splits, the weights e^(m - M) and the total sum
     for (int h = warp; h < g; h += kDecodeWarps) {
         float M = -INFINITY;
-        for (int s = lane; s < n_active; s += 32) {
-            const float *src = part_base + ((long long)s * g + h) * (D + 4);
-            const float ms = __ldcg(src + D), ls = __ldcg(src + D + 1);
-            pw[s * g + h] = ms;
-            pl[s * g + h] = ls;
-            M = fmaxf(M, ms);
-        }
+        for (int s = lane; s < n_active; s += 32) M = fmaxf(M, stage[(s * g + h) * REC + D]);
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, m));
         float Ls = 0.f;
         for (int s = lane; s < n_active; s += 32) {
-            const float ms = pw[s * g + h];
+            const float ms = stage[(s * g + h) * REC + D];
             const float f = (ms == -INFINITY || M == -INFINITY) ? 0.f : ex2(ms - M);
             pw[s * g + h] = f;
-            Ls += f * pl[s * g + h];
+            Ls += f * stage[(s * g + h) * REC + D + 1];
         }
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) Ls += __shfl_xor_sync(kFull, Ls, m);
         if (lane == 0) pL[h] = Ls;
     }
     __syncthreads();
-    // (2) each thread owns one (head, float4) of the output and a stride of
-    //     the splits; the loads are independent, unrolled 8 deep
-    const int items = g * QUADS;
-    const int nhalf = max(1, kDecodeThreads / items);
-    if (tid < items * nhalf) {
-        const int it = tid % items, half = tid / items;
-        const int h = it / QUADS, qd = it % QUADS;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int s = half; s < n_active; s += nhalf) {
-            const float f = pw[s * g + h];
-            const float4 v =
-                __ldcg(reinterpret_cast<const float4 *>(part_base + ((long long)s * g + h) * (D + 4)) + qd);
-            acc.x = fmaf(f, v.x, acc.x);
-            acc.y = fmaf(f, v.y, acc.y);
-            acc.z = fmaf(f, v.z, acc.z);
-            acc.w = fmaf(f, v.w, acc.w);
-        }
-        *reinterpret_cast<float4 *>(po + (half * g + h) * D + 4 * qd) = acc;
+    // (2) weighted sum over the splits
+    for (int idx = tid; idx < g * D; idx += kDecodeThreads) {
+        const int h = idx / D, ch = idx - h * D;
+        float o = 0.f;
+        for (int s = 0; s < n_active; s++) o = fmaf(pw[s * g + h], stage[(s * g + h) * REC + ch], o);
+        po[idx] = o;
     }
     __syncthreads();
-    // (3) sum the strides, normalise, inverse rotation, store
+    // (3) normalise, inverse rotation, store
     for (int h = warp; h < g; h += kDecodeWarps) {
         const float Ls = pL[h];
         const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
         float o[E];
 #pragma unroll
-        for (int e = 0; e < E; e++) {
-            float v = 0.f;
-            for (int hf = 0; hf < nhalf; hf++) v += po[(hf * g + h) * D + lane * E + e];
-            o[e] = v * inv;
-        }
+        for (int e = 0; e < E; e++) o[e] = po[h * D + lane * E + e] * inv;
         if (p.rotate) {
             fwht_warp<D>(o, lane);
 #pragma unroll
@@ -945,13 +954,7 @@ bool decode_supported(const Layout &L)
     return L.d == 128;
 }
 
-int decode_max_splits(const Layout &L)
-{
-    // the final merge keeps 2*n*g split values, 8 sums and up to 256*4 output
-    // floats in the smallest ring of any instantiation (8 warps x 4 x 1152 B)
-    const int ring_floats = kDecodeWarps * 4 * 1152 / 4;
-    return (ring_floats - kMaxGqa - kDecodeThreads * 4) / (2 * L.g);
-}
+int decode_max_splits(const Layout &) { return kCombineSplits; }
 
 cudaError_t launch_decode(const DecodeParams &p, dim3 grid, cudaStream_t s)
 {
