@@ -147,6 +147,20 @@ kvq_status kvq_decode_attn(kvq_cache *cache, const void *q, const int32_t *block
                            const int32_t *ctx_lens, int32_t batch, float softmax_scale, const kvq_tier2 *tier2,
                            void *workspace, size_t ws_bytes, void *out, int32_t *promoted_out, void *stream);
 
+/* One decode step: quantise-on-append of each sequence's new token followed
+ * by decode attention over the grown context, in one launch.  k_new, v_new:
+ * fp16 [batch][Hkv][d] (16-byte aligned), the token at position
+ * ctx_lens[b] - 1; slot_mapping[b] must be that position's slot, i.e.
+ * block_table[b][(ctx_lens[b]-1)/16]*16 + (ctx_lens[b]-1)%16 (otherwise the
+ * token is not stored and KVQ_ERR_OUT_OF_RANGE is recorded).  The stored
+ * codes are byte-identical to kvq_append's and the output equals kvq_append
+ * followed by kvq_decode_attn.  Other arguments as kvq_decode_attn (no
+ * certified mode). */
+kvq_status kvq_decode_step(kvq_cache *cache, const void *k_new, const void *v_new, const int32_t *slot_mapping,
+                           const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
+                           const int32_t *ctx_lens, int32_t batch, float softmax_scale, void *workspace,
+                           size_t ws_bytes, void *out, void *stream);
+
 /* Read back n stored rows (slots[0..n), int32 device) per kv head:
  *   k_out, v_out: fp32 [n][Hkv][d] rotated-domain dequantised values
  *                 (code*scale + zero, one rounding), may be NULL;

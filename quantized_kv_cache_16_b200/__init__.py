@@ -24,7 +24,7 @@ PAGE_TOKENS = 16
 # Every symbol include/kvq.h declares (checked by the ABI test).
 EXPORTS = (
     "kvq_pool_bytes", "kvq_create_cache", "kvq_destroy_cache", "kvq_append", "kvq_reset_pages",
-    "kvq_decode_workspace_bytes", "kvq_decode_attn", "kvq_dequant_debug", "kvq_sync_status",
+    "kvq_decode_workspace_bytes", "kvq_decode_attn", "kvq_decode_step", "kvq_dequant_debug", "kvq_sync_status",
     "kvq_status_string",
 )
 
@@ -70,6 +70,7 @@ def lib() -> C.CDLL:
             "kvq_reset_pages": (i32, [P, P, i32, P]),
             "kvq_decode_workspace_bytes": (sz, [P, i32, i32]),
             "kvq_decode_attn": (i32, [P, P, P, i32, P, i32, C.c_float, C.POINTER(kvq_tier2), P, sz, P, P, P]),
+            "kvq_decode_step": (i32, [P, P, P, P, P, P, i32, P, i32, C.c_float, P, sz, P, P]),
             "kvq_dequant_debug": (i32, [P, P, i32, P, P, P, P, P]),
             "kvq_sync_status": (i32, [P]),
             "kvq_status_string": (C.c_char_p, [i32]),
@@ -150,6 +151,14 @@ def kvq_decode_attn(cache, q, block_table, max_pages_per_seq: int, ctx_lens, bat
                                  _stream(stream)))
 
 
+def kvq_decode_step(cache, k_new, v_new, slot_mapping, q, block_table, max_pages_per_seq: int, ctx_lens,
+                    batch: int, softmax_scale: float, workspace, ws_bytes: int, out, stream=None) -> None:
+    _check("kvq_decode_step",
+           lib().kvq_decode_step(cache, _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(q), _ptr(block_table),
+                                 max_pages_per_seq, _ptr(ctx_lens), batch, softmax_scale, _ptr(workspace), ws_bytes,
+                                 _ptr(out), _stream(stream)))
+
+
 def kvq_dequant_debug(cache, slots, n: int | None = None, k_out=None, v_out=None, codes_out=None, meta_out=None,
                       stream=None) -> None:
     n = slots.shape[0] if n is None else n
@@ -214,6 +223,18 @@ class Cache:
         ws = self.workspace_for(batch, max_pages)
         kvq_decode_attn(self.handle, q, block_table, max_pages, ctx_lens, batch, softmax_scale, tier2, ws,
                         ws.numel(), out, promoted_out, stream)
+        return out
+
+    def step(self, k_new, v_new, slot_mapping, q, block_table, ctx_lens, out=None, softmax_scale: float = 0.0,
+             stream=None):
+        """Append one token per sequence and decode, in one launch."""
+        import torch
+        batch, max_pages = block_table.shape
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        ws = self.workspace_for(batch, max_pages)
+        kvq_decode_step(self.handle, k_new, v_new, slot_mapping, q, block_table, max_pages, ctx_lens, batch,
+                        softmax_scale, ws, ws.numel(), out, stream)
         return out
 
     def dequant(self, slots):

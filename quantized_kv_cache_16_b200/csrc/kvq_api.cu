@@ -184,15 +184,21 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *c, int32_t batch, int32_t max
     return counters_bytes(batch, c->L.hkv) + part;
 }
 
-kvq_status kvq_decode_attn(kvq_cache *c, const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
-                           const int32_t *ctx_lens, int32_t batch, float softmax_scale, const kvq_tier2 *tier2,
-                           void *workspace, size_t ws_bytes, void *out, int32_t *promoted_out, void *stream)
+}  // extern "C"
+
+namespace {
+
+kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const int32_t *slot_mapping,
+                       const void *q, const int32_t *block_table, int32_t max_pages_per_seq, const int32_t *ctx_lens,
+                       int32_t batch, float softmax_scale, const kvq_tier2 *tier2, void *workspace, size_t ws_bytes,
+                       void *out, int32_t *promoted_out, void *stream)
 {
     (void)promoted_out;
     if (!c || batch < 0 || max_pages_per_seq < 1) return KVQ_ERR_INVALID_ARG;
     if (batch == 0) return KVQ_OK;
     if (!q || !block_table || !ctx_lens || !out || !workspace) return KVQ_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
+    if (k_new && (!v_new || !slot_mapping || !aligned(k_new, 16) || !aligned(v_new, 16))) return KVQ_ERR_INVALID_ARG;
     if (!decode_supported(c->L)) return KVQ_ERR_UNSUPPORTED;
     if (tier2) return KVQ_ERR_UNSUPPORTED;
     if (ws_bytes < kvq_decode_workspace_bytes(c, batch, max_pages_per_seq)) return KVQ_ERR_CAPACITY;
@@ -216,9 +222,35 @@ kvq_status kvq_decode_attn(kvq_cache *c, const void *q, const int32_t *block_tab
     p.counters = static_cast<unsigned int *>(workspace);
     p.part = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + counters_bytes(batch, c->L.hkv));
     p.out = static_cast<float *>(out);
+    p.new_k = static_cast<const __half *>(k_new);
+    p.new_v = static_cast<const __half *>(v_new);
+    p.new_slots = slot_mapping;
+    p.clip = c->cfg.clip_ratio;
     c->last_stream = stream;
     const dim3 grid(s.n_splits, c->L.hkv, batch);
     return cuda_status(launch_decode(p, grid, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_decode_attn(kvq_cache *c, const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
+                           const int32_t *ctx_lens, int32_t batch, float softmax_scale, const kvq_tier2 *tier2,
+                           void *workspace, size_t ws_bytes, void *out, int32_t *promoted_out, void *stream)
+{
+    return decode_impl(c, nullptr, nullptr, nullptr, q, block_table, max_pages_per_seq, ctx_lens, batch,
+                       softmax_scale, tier2, workspace, ws_bytes, out, promoted_out, stream);
+}
+
+kvq_status kvq_decode_step(kvq_cache *c, const void *k_new, const void *v_new, const int32_t *slot_mapping,
+                           const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
+                           const int32_t *ctx_lens, int32_t batch, float softmax_scale, void *workspace,
+                           size_t ws_bytes, void *out, void *stream)
+{
+    if (!k_new) return KVQ_ERR_INVALID_ARG;
+    return decode_impl(c, k_new, v_new, slot_mapping, q, block_table, max_pages_per_seq, ctx_lens, batch,
+                       softmax_scale, nullptr, workspace, ws_bytes, out, nullptr, stream);
 }
 
 kvq_status kvq_dequant_debug(kvq_cache *c, const int32_t *slots, int32_t n, float *k_out, float *v_out,

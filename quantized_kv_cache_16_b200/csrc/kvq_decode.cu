@@ -109,6 +109,160 @@ __device__ __forceinline__ void imma16832(int *d, const uint32_t (&a)[4], uint32
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+
+// ------------------------------------------------------------ fused append ---
+// Quantise-on-append of one K or V row by a whole warp: lane l holds elements
+// [l*E, l*E+E).  Same fp32 operations in the same order as the append kernel
+// (sign, butterflies h = 1, 2, 4, ..., d/2 as (a+b, a-b), times c_d; group
+// statistics; fp16 scale/zero; rounding), so the stored bytes are identical.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint32_t round_code(float v, float lo, float hi)
+{
+    v = fminf(fmaxf(v, lo), hi);
+    return __float_as_uint(__fadd_rn(v, kRoundMagic)) & 0xFFu;
+}
+
+__device__ __forceinline__ float code_value(uint32_t c, bool is_signed)
+{
+    return (float)(is_signed ? (int)(int8_t)c : (int)c);
+}
+
+template <int LANES> __device__ __forceinline__ float group_min(float v)
+{
+#pragma unroll
+    for (int m = 1; m < LANES; m <<= 1) v = fminf(v, __shfl_xor_sync(kFull, v, m));
+    return v;
+}
+template <int LANES> __device__ __forceinline__ float group_max(float v)
+{
+#pragma unroll
+    for (int m = 1; m < LANES; m <<= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, m));
+    return v;
+}
+
+template <int D, int FMT>
+__device__ __forceinline__ void warp_append_row(const __half *src, const float *signs, int rotate, float rot_scale,
+                                                float clip, unsigned char *codes, unsigned char *meta_row, int tok,
+                                                unsigned int *desc, int tensor, int lane)
+{
+    constexpr int E = D / 32;
+    float x[E];
+    if constexpr (E == 4) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(src + lane * E);
+        const float2 f0 = __half22float2(bits_h2(u.x)), f1 = __half22float2(bits_h2(u.y));
+        x[0] = f0.x;
+        x[1] = f0.y;
+        x[2] = f1.x;
+        x[3] = f1.y;
+    } else {
+        const float2 f0 = __half22float2(bits_h2(*reinterpret_cast<const uint32_t *>(src + lane * E)));
+        x[0] = f0.x;
+        x[1] = f0.y;
+    }
+    if (rotate) {
+#pragma unroll
+        for (int e = 0; e < E; e++) x[e] = __fmul_rn(x[e], signs[lane * E + e]);
+#pragma unroll
+        for (int h = 1; h < E; h <<= 1)
+#pragma unroll
+            for (int e = 0; e < E; e++)
+                if (!(e & h)) {
+                    const float a = x[e], b = x[e + h];
+                    x[e] = __fadd_rn(a, b);
+                    x[e + h] = __fsub_rn(a, b);
+                }
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+            const float sg = (lane & m) ? -1.0f : 1.0f;  // upper partner: a - b
+#pragma unroll
+            for (int e = 0; e < E; e++) x[e] = __fmaf_rn(sg, x[e], __shfl_xor_sync(kFull, x[e], m));
+        }
+#pragma unroll
+        for (int e = 0; e < E; e++) x[e] = __fmul_rn(x[e], rot_scale);
+    }
+    const bool want_desc = desc != nullptr;
+    float emax = 0.f, amax = 0.f;
+    if constexpr (FMT == KVQ_INT8_SYM) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; e++) a = fmaxf(a, fabsf(x[e]));
+        a = group_max<32>(a);
+        const __half shh = __float2half_ru(__fdiv_rn(a, 127.0f));
+        const float sf = __half2float(shh);
+        const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
+        amax = a;
+        uint32_t packed = 0;
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            const uint32_t c = round_code(__fmul_rn(x[e], inv), -127.0f, 127.0f);
+            packed |= c << (8 * e);
+            emax = fmaxf(emax, fabsf(__fsub_rn(x[e], __fmul_rn(code_value(c, true), sf))));
+        }
+        const int byte0 = lane * E;  // stream byte
+        unsigned char *dst = codes + ((byte0 / 16) * 16 + tok) * 16 + byte0 % 16;
+        if constexpr (E == 4) *reinterpret_cast<uint32_t *>(dst) = packed;
+        else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)packed;
+        if (lane == 0) *reinterpret_cast<uint16_t *>(meta_row) = __half_as_ushort(shh);
+    } else {
+        constexpr bool I4 = FMT == KVQ_INT4_ASYM;
+        constexpr int GL = I4 ? 32 / E : 32;  // lanes per group
+        constexpr int NG = I4 ? D / 32 : 1;
+        constexpr float QMAX = I4 ? 15.0f : 3.0f;
+        float lo = x[0], hi = x[0];
+#pragma unroll
+        for (int e = 1; e < E; e++) {
+            lo = fminf(lo, x[e]);
+            hi = fmaxf(hi, x[e]);
+        }
+        lo = group_min<GL>(lo);
+        hi = group_max<GL>(hi);
+        if (clip < 1.0f) {
+            lo = __fmul_rn(lo, clip);
+            hi = __fmul_rn(hi, clip);
+        }
+        const __half shh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), QMAX));
+        const __half zhh = __float2half_rn(lo);
+        const float sf = __half2float(shh), zf = __half2float(zhh);
+        const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
+        uint32_t packed = 0;
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            const uint32_t c = round_code(__fmul_rn(__fsub_rn(x[e], zf), inv), 0.0f, QMAX);
+            packed |= c << ((I4 ? 4 : 2) * e);
+            emax = fmaxf(emax, fabsf(__fsub_rn(x[e], __fadd_rn(__fmul_rn(code_value(c, false), sf), zf))));
+            amax = fmaxf(amax, fabsf(x[e]));
+        }
+        if constexpr (I4) {
+            const int gi = lane / GL, q = lane % GL;  // q-th run of E codes in group gi
+            unsigned char *dst = codes + (gi * 16 + tok) * 16 + (q * E) / 2;
+            if constexpr (E == 4) *reinterpret_cast<uint16_t *>(dst) = (uint16_t)packed;
+            else *dst = (unsigned char)packed;
+            if (q == 0) {
+                reinterpret_cast<uint16_t *>(meta_row)[gi] = __half_as_ushort(shh);
+                reinterpret_cast<uint16_t *>(meta_row)[NG + gi] = __half_as_ushort(zhh);
+            }
+        } else {
+            static_assert(I4 || E == 4, "2-bit fused append needs head_dim 128");
+            codes[((lane / 16) * 16 + tok) * 16 + lane % 16] = (unsigned char)packed;  // stream byte = lane
+            if (lane == 0)
+                *reinterpret_cast<uint32_t *>(meta_row) = __half_as_ushort(shh) | (uint32_t(__half_as_ushort(zhh)) << 16);
+        }
+    }
+    if (want_desc) {
+        emax = group_max<32>(emax);
+        amax = group_max<32>(amax);
+        if (lane == 0) {
+            if (tensor == 0) {
+                atomicMax(desc + 0, __float_as_uint(emax));
+            } else {
+                atomicMax(desc + 1, __float_as_uint(emax));
+                atomicMax(desc + 2, __float_as_uint(amax));
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------ key codecs ---
 // A operand of the QK IMMA: thread (r, j) holds, for k-step kq (32 virtual
 // channels), 4 bytes at virtual k = 4j..4j+3 and 4j+16..4j+19 of tokens r and
@@ -457,6 +611,29 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
                 asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar0 + 8 * st) : "memory");
         }
     };
+    // fused append: the warp that owns the page of position T-1 quantises
+    // the new token's K and V rows into it before any copy of that page
+    if (p.new_k != nullptr && T > 0 && n_pages - 1 >= p_begin && n_pages - 1 < p_end) {
+        const int pg = bt[n_pages - 1];
+        const int slot = p.new_slots[b];
+        const int tok = (T - 1) % kPageTokens;
+        if (pg < 0 || pg >= L.num_pages || slot != pg * kPageTokens + tok) {
+            if (lane == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
+        } else {
+            unsigned char *chunk = const_cast<unsigned char *>(kv_base) + (long long)pg * L.page_bytes;
+            unsigned int *desc = L.desc_off ? reinterpret_cast<unsigned int *>(const_cast<unsigned char *>(p.pool) +
+                                                                                L.desc_off + ((long long)pg * L.hkv + kvh) * 16)
+                                            : nullptr;
+            const long long row = ((long long)b * L.hkv + kvh) * D;
+            warp_append_row<D, KF>(p.new_k + row, p.signs, p.rotate, p.rot_scale, p.clip, chunk + L.k_codes,
+                                   chunk + L.k_meta + tok * L.k_row_meta, tok, desc, 0, lane);
+            warp_append_row<D, VF>(p.new_v + row, p.signs, p.rotate, p.rot_scale, p.clip, chunk + L.v_codes,
+                                   chunk + L.v_meta + tok * L.v_row_meta, tok, desc, 1, lane);
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+    }
     for (int i = 0; i < NST && i < npg; i++) issue(i);
 
     // ---- query (warp h): rotate, pre-scale, group sums, and the three signed

@@ -113,6 +113,11 @@ struct DecodeParams {
     float *part;              // [B][Hkv][n_splits][g][d + 4]
     unsigned int *counters;   // [B][Hkv]
     float *out;
+    // fused append of one token per sequence before attending (null = off)
+    const __half *new_k;      // [B][Hkv][d]
+    const __half *new_v;
+    const int32_t *new_slots; // [B]: the slot of position ctx_lens[b] - 1
+    float clip;
 };
 
 struct DequantParams {

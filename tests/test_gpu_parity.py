@@ -147,3 +147,50 @@ def test_full_size_workloads(name, make):
     diff = np.nonzero(gpu[256:] != pair.opool[256:])[0]
     assert diff.size == 0, f"{diff.size} bytes differ, first at {256 + diff[0]}"
     _decode_check(pair)
+
+
+STEP_CASES = [
+    ("tiny", W.scaled(W.tiny(), [255])),
+    ("llama-ragged", W.scaled(W.llama(), [1000, 31, 16])),
+    ("int8k-descriptors", W.scaled(W.certified(), [700])),
+    ("int2-B2", W.scaled(W.int2(), [301, 64])),
+]
+
+
+@pytest.mark.parametrize("name,wl", STEP_CASES, ids=[s[0] for s in STEP_CASES])
+def test_decode_step_fuses_append_and_decode(name, wl):
+    """kvq_decode_step stores exactly the bytes kvq_append stores and returns
+    exactly what kvq_append followed by kvq_decode_attn returns."""
+    import torch
+    fused = build_pair(wl, extra_tokens=2)
+    split = build_pair(wl, extra_tokens=2, oracle=False)
+    for step in range(2):
+        k, v = W.step_kv(wl, step)
+        slots = np.array([fused.pages.slot(b, wl.ctx[b] + step) for b in range(wl.B)], np.int32)
+        q = torch.from_numpy(W.queries(wl, step)).cuda()
+        kd, vd, sd = torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(), torch.from_numpy(slots).cuda()
+        out_f = fused.cache.step(kd, vd, sd, q, fused.block_table(), fused.ctx(step + 1))
+        split.cache.append(kd, vd, sd)
+        out_s = split.cache.decode(q, split.block_table(), split.ctx(step + 1))
+        assert O.append(fused.ocfg, fused.opool, k, v, slots) == 0
+        assert fused.cache.sync_status() == 0
+        gpu = fused.cache.pool.cpu().numpy()
+        assert np.array_equal(gpu[256:], fused.opool[256:])
+        assert np.array_equal(out_f.cpu().numpy(), out_s.cpu().numpy())
+        want = O.decode(fused.ocfg, fused.opool, W.queries(wl, step), fused.pages.block_table,
+                        [t + step + 1 for t in wl.ctx])
+        max_abs, rel = attn_errors(out_f.cpu().numpy(), want)
+        assert max_abs <= TOL_MAX_ABS and rel <= TOL_REL_L2, f"max_abs={max_abs:.3e} rel={rel:.3e}"
+
+
+def test_decode_step_rejects_a_slot_off_the_last_position():
+    import torch
+    wl = W.scaled(W.llama(), [40])
+    pair = build_pair(wl, extra_tokens=1)
+    before = pair.cache.pool.cpu().numpy().copy()
+    k, v = W.step_kv(wl, 0)
+    bad = np.array([pair.pages.slot(0, 3)], np.int32)  # not position 40
+    pair.cache.step(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(), torch.from_numpy(bad).cuda(),
+                    torch.from_numpy(W.queries(wl, 0)).cuda(), pair.block_table(), pair.ctx(1))
+    assert pair.cache.sync_status() == 4  # KVQ_ERR_OUT_OF_RANGE
+    assert np.array_equal(pair.cache.pool.cpu().numpy()[256:], before[256:])
