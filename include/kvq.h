@@ -161,6 +161,29 @@ kvq_status kvq_decode_step(kvq_cache *cache, const void *k_new, const void *v_ne
                            const int32_t *ctx_lens, int32_t batch, float softmax_scale, void *workspace,
                            size_t ws_bytes, void *out, void *stream);
 
+/* Decode attention that allocates nothing and takes no workspace, for
+ * callers that cannot allocate device memory: an engine that reserves all of
+ * the GPU's memory up front for its own pools (so any later cudaMalloc fails
+ * or would steal from the KV pool), or code that must not allocate once it is
+ * serving (allocation can block and synchronise the device).  The pages have
+ * no counterpart of this call; it exists for such integrations.
+ *
+ * Same arguments and result as kvq_decode_attn without the workspace and
+ * certified-mode arguments.  The workspace is a 4 MiB array in the library's
+ * own device memory (one per GPU that loads the library, held until process
+ * exit); a call whose kvq_decode_workspace_bytes(cache, batch,
+ * max_pages_per_seq) exceeds 4 MiB returns KVQ_ERR_CAPACITY and launches
+ * nothing.  The cache's device must be current.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress), so make that
+ * first call before any stream capture.  Each call clears the array's split
+ * counters on `stream` (cudaMemsetAsync) and then launches the decode; every
+ * call shares the one array and it keeps the last call's contents, so calls
+ * that can overlap on the GPU (different streams, or concurrent host threads)
+ * race on it and must be serialised by the caller. */
+kvq_status kvq_decode_attn_static(kvq_cache *cache, const void *q, const int32_t *block_table,
+                                  int32_t max_pages_per_seq, const int32_t *ctx_lens, int32_t batch,
+                                  float softmax_scale, void *out, void *stream);
+
 /* Read back n stored rows (slots[0..n), int32 device) per kv head:
  *   k_out, v_out: fp32 [n][Hkv][d] rotated-domain dequantised values
  *                 (code*scale + zero, one rounding), may be NULL;

@@ -24,7 +24,8 @@ PAGE_TOKENS = 16
 # Every symbol include/kvq.h declares (checked by the ABI test).
 EXPORTS = (
     "kvq_pool_bytes", "kvq_create_cache", "kvq_destroy_cache", "kvq_append", "kvq_reset_pages",
-    "kvq_decode_workspace_bytes", "kvq_decode_attn", "kvq_decode_step", "kvq_dequant_debug", "kvq_sync_status",
+    "kvq_decode_workspace_bytes", "kvq_decode_attn", "kvq_decode_step", "kvq_decode_attn_static",
+    "kvq_dequant_debug", "kvq_sync_status",
     "kvq_status_string",
 )
 
@@ -71,6 +72,7 @@ def lib() -> C.CDLL:
             "kvq_decode_workspace_bytes": (sz, [P, i32, i32]),
             "kvq_decode_attn": (i32, [P, P, P, i32, P, i32, C.c_float, C.POINTER(kvq_tier2), P, sz, P, P, P]),
             "kvq_decode_step": (i32, [P, P, P, P, P, P, i32, P, i32, C.c_float, P, sz, P, P]),
+            "kvq_decode_attn_static": (i32, [P, P, P, i32, P, i32, C.c_float, P, P]),
             "kvq_dequant_debug": (i32, [P, P, i32, P, P, P, P, P]),
             "kvq_sync_status": (i32, [P]),
             "kvq_status_string": (C.c_char_p, [i32]),
@@ -157,6 +159,13 @@ def kvq_decode_step(cache, k_new, v_new, slot_mapping, q, block_table, max_pages
            lib().kvq_decode_step(cache, _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(q), _ptr(block_table),
                                  max_pages_per_seq, _ptr(ctx_lens), batch, softmax_scale, _ptr(workspace), ws_bytes,
                                  _ptr(out), _stream(stream)))
+
+
+def kvq_decode_attn_static(cache, q, block_table, max_pages_per_seq: int, ctx_lens, batch: int,
+                           softmax_scale: float, out, stream=None) -> None:
+    _check("kvq_decode_attn_static",
+           lib().kvq_decode_attn_static(cache, _ptr(q), _ptr(block_table), max_pages_per_seq, _ptr(ctx_lens),
+                                        batch, softmax_scale, _ptr(out), _stream(stream)))
 
 
 def kvq_dequant_debug(cache, slots, n: int | None = None, k_out=None, v_out=None, codes_out=None, meta_out=None,
