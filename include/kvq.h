@@ -76,10 +76,13 @@ typedef struct {
 
 typedef struct kvq_cache kvq_cache; /* opaque; owned by the library */
 
-/* Tier-2 store of the certified mode: the original fp16 K and V rows indexed
- * by slot, [num_pages*16][Hkv][d] each, in pinned host memory mapped into the
- * device address space (the pointers given must be device-accessible, e.g.
- * from cudaHostGetDevicePointer).  The caller keeps it current (it is the
+/* Tier-2 store of the certified mode ["Runtime-Certified Bounded-Error
+ * Quantized Attention", Methodology 1]: the original fp16 K and V rows (not
+ * rotated) indexed by slot, [num_pages*16][Hkv][d] each, 16-byte aligned.
+ * Pinned host memory (cudaHostAlloc / cudaMallocHost / cudaHostRegister) is
+ * read by the kernels through its device mapping, as the pages place it;
+ * device memory is accepted as well.  Pageable host memory is rejected with
+ * KVQ_ERR_INVALID_ARG.  The caller keeps the rows current (they are the
  * ground truth the pages call tier 2). */
 typedef struct {
     const void *k_host;
@@ -121,8 +124,10 @@ kvq_status kvq_append(kvq_cache *cache, const void *k, const void *v, const int3
 kvq_status kvq_reset_pages(kvq_cache *cache, const int32_t *page_ids, int32_t n, void *stream);
 
 /* Workspace bytes kvq_decode_attn needs for `batch` sequences with block
- * tables of max_pages_per_seq entries.  The workspace must be zero-filled
- * before its first use; every decode call leaves it ready for the next one. */
+ * tables of max_pages_per_seq entries (with bound blocks configured, this
+ * includes the certified mode's page statistics, promoted-block lists and
+ * partials).  The workspace must be zero-filled before its first use; every
+ * decode call leaves it ready for the next one. */
 size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int32_t batch, int32_t max_pages_per_seq);
 
 /* Decode attention ["OSCAR", 2.2b]: for each sequence b and query head h,
@@ -133,7 +138,18 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int32_t batch, int32_t
  *   block_table: int32 [batch][max_pages_per_seq] (device)
  *   ctx_lens:    int32 [batch] (device), 0 <= ctx_lens[b] <= 16*max_pages_per_seq
  *   softmax_scale: <= 0 means 1/sqrt(d)
- *   tier2:       NULL, or the certified-mode store (needs bound_block_tokens)
+ *   tier2:       NULL, or the certified-mode store (needs bound_block_tokens
+ *                and a block count 16*max_pages_per_seq/bound_block_tokens of
+ *                at most 16384, else KVQ_ERR_UNSUPPORTED; promote_frac in
+ *                [0, 1]).  The quantised decode then records per-page
+ *                softmax statistics; per (sequence, kv head) a bound is formed
+ *                for every block [Methodology 2: a key term from the score
+ *                perturbation, a value term from the value error, weighted by
+ *                the block's softmax mass], the ceil(promote_frac * n_blocks)
+ *                highest blocks (ties: lower block first) are recomputed from
+ *                the tier-2 rows, and their quantised contribution to the
+ *                output is replaced by the exact one [Methodology 3].  Three
+ *                launches on `stream`.
  *   workspace:   >= kvq_decode_workspace_bytes, zero-filled before first use;
  *                one workspace must not serve two decode calls that overlap
  *   out:         fp32 [batch][Hq][d] (device, 16-byte aligned); fp32 so the

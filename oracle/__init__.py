@@ -100,7 +100,7 @@ def lib():
             "kvqo_decode": (i32, [cfgp, P, P, P, i32, P, i32, f64, i32, P, P]),
             "kvqo_decode_fp16": (i32, [cfgp, P, P, P, P, i32, P, i32, f64, P, P]),
             "kvqo_promote_count": (i32, [f64, i32]),
-            "kvqo_decode_certified": (i32, [cfgp, P, P, P, P, P, i32, P, i32, f64, f64, P, P, P, i32, P, i32, P]),
+            "kvqo_decode_certified": (i32, [cfgp, P, P, P, P, P, i32, P, i32, f64, f64, P, P, P, i32, P, i32, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -298,9 +298,10 @@ def promote_count(frac: float, n_blocks: int) -> int:
 
 
 def decode_certified(cfg: Config, pool: np.ndarray, k_slots, v_slots, q, block_table, ctx_lens, frac: float,
-                     scale: float = 0.0, sel=None):
+                     scale: float = 0.0, sel=None, forced=None):
     """Returns (out [B,Hq,d], promoted [B,Hkv,kmax], scores [B,Hkv,nblk_max],
-    bound_sums [B,Hq])."""
+    bound_sums [B,Hq]).  forced [B,Hkv,kmax] (-1 padded): promote exactly
+    these blocks instead of the top scores."""
     k = _c(k_slots, np.float16).view(np.uint16)
     v = _c(v_slots, np.float16).view(np.uint16)
     q = _c(q, np.float16).view(np.uint16)
@@ -311,12 +312,17 @@ def decode_certified(cfg: Config, pool: np.ndarray, k_slots, v_slots, q, block_t
     nbmax = max(1, int((int(cl.max()) + blk - 1) // blk)) if B else 1
     kmax = max(1, promote_count(frac, nbmax))
     sel = None if sel is None else _c(sel, np.int32)
+    if forced is not None:
+        forced = _c(forced, np.int32)
+        kmax = forced.shape[2]
+        assert forced.shape == (B, cfg.num_kv_heads, kmax)
     out = np.zeros((B, cfg.num_q_heads, cfg.head_dim), np.float64)
     prom = np.full((B, cfg.num_kv_heads, kmax), -1, np.int32)
     scores = np.zeros((B, cfg.num_kv_heads, nbmax), np.float64)
     bsum = np.zeros((B, cfg.num_q_heads), np.float64)
     rc = lib().kvqo_decode_certified(C.byref(cfg), _p(pool), _p(k), _p(v), _p(q), _p(bt), bt.shape[1], _p(cl), B,
-                                     scale, frac, _p(sel), _p(out), _p(prom), kmax, _p(scores), nbmax, _p(bsum))
+                                     scale, frac, _p(sel), _p(out), _p(prom), kmax, _p(scores), nbmax, _p(bsum),
+                                     _p(forced))
     if rc != 0:
         raise ValueError(f"oracle certified decode rejected its arguments (rc={rc})")
     return out, prom, scores, bsum

@@ -746,14 +746,17 @@ static void block_bounds_one_head(const double *phat, int T, int block, const do
  * (rotated in fp64), and run attention with promoted blocks exact and all
  * others dequantised.  k_slots/v_slots: tier-2 fp16 rows [num_slots][Hkv][d].
  * promoted (optional): [B][Hkv][max_promote] block indices in descending score
- * order, -1 padded.  score_out (optional): [B][Hkv][max_blocks].
+ * order, -1 padded.  forced (optional, same shape): promote exactly these
+ * blocks (entries < 0 or >= n_blocks ignored) instead of the top scores --
+ * for checking an implementation whose selection legitimately differs on a
+ * near-tie; bounds and scores are computed as usual.  score_out (optional): [B][Hkv][max_blocks].
  * bound_sum_out (optional): [B][Hq], sum_b bound_b of each head (all blocks
  * quantised).  quant_out (optional): [B][Hq][d] the plain quantised output. */
 int kvqo_decode_certified(const kvqo_config *c, const uint8_t *pool, const uint16_t *k_slots,
                           const uint16_t *v_slots, const uint16_t *q, const int32_t *block_table, int max_pages,
                           const int32_t *ctx_lens, int B, double scale, double frac, const int32_t *sel,
                           double *out, int32_t *promoted, int max_promote, double *score_out, int max_blocks,
-                          double *bound_sum_out)
+                          double *bound_sum_out, const int32_t *forced)
 {
     if (!kvqo_config_ok(c) || c->bound_block_tokens <= 0) return -2;
     if (!decode_args_ok(c, block_table, max_pages, ctx_lens, B)) return -1;
@@ -819,6 +822,14 @@ int kvqo_decode_certified(const kvqo_config *c, const uint8_t *pool, const uint1
             /* selection: top k by score, ties to the lower index */
             int k = kvqo_promote_count(frac, nb);
             char *taken = (char *)calloc((size_t)nb + 1, 1);
+            if (forced) {
+                const int32_t *f = forced + ((size_t)b * hkv + kvh) * max_promote;
+                for (int r = 0; r < max_promote; r++) {
+                    if (f[r] >= 0 && f[r] < nb) taken[f[r]] = 1;
+                    if (promoted) promoted[((size_t)b * hkv + kvh) * max_promote + r] = f[r];
+                }
+                k = 0;
+            }
             for (int r = 0; r < k; r++) {
                 int best = -1;
                 for (int bb = 0; bb < nb; bb++)
@@ -826,7 +837,7 @@ int kvqo_decode_certified(const kvqo_config *c, const uint8_t *pool, const uint1
                 taken[best] = 1;
                 if (promoted && r < max_promote) promoted[((size_t)b * hkv + kvh) * max_promote + r] = best;
             }
-            if (promoted)
+            if (promoted && !forced)
                 for (int r = k; r < max_promote; r++) promoted[((size_t)b * hkv + kvh) * max_promote + r] = -1;
             /* promoted blocks use the exact rotated fp16 originals */
             for (int t = 0; t < T; t++) {

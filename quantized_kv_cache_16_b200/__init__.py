@@ -234,6 +234,14 @@ class Cache:
                         ws.numel(), out, promoted_out, stream)
         return out
 
+    def decode_certified(self, q, block_table, ctx_lens, k_tier2, v_tier2, promote_frac: float,
+                         promoted_out=None, out=None, softmax_scale: float = 0.0, stream=None):
+        """Certified decode: k_tier2 / v_tier2 are the exact fp16 rows
+        [num_pages*16, Hkv, d] by slot, in pinned host memory (or on the
+        device); promoted_out (optional) int32 [B, Hkv, kmax] on the device."""
+        t2 = kvq_tier2(k_tier2.data_ptr(), v_tier2.data_ptr(), promote_frac)
+        return self.decode(q, block_table, ctx_lens, out, softmax_scale, t2, promoted_out, stream)
+
     def step(self, k_new, v_new, slot_mapping, q, block_table, ctx_lens, out=None, softmax_scale: float = 0.0,
              stream=None):
         """Append one token per sequence and decode, in one launch."""

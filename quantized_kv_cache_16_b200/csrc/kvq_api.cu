@@ -82,6 +82,75 @@ SplitPlan plan_splits(const kvq_cache *c, int batch, int max_pages)
 
 size_t counters_bytes(int batch, int hkv) { return ((size_t)batch * hkv * 4 + 255) / 256 * 256; }
 
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+// Bound blocks a sequence of max_pages pages can hold, and the power of two
+// the selection sorts.
+int cert_blocks(const kvq_cache *c, int max_pages)
+{
+    const long long blk = c->L.bound_block;
+    return blk > 0 ? (int)(((long long)max_pages * kPageTokens + blk - 1) / blk) : 0;
+}
+
+int pow2_at_least(int n)
+{
+    int p = 1;
+    while (p < n) p <<= 1;
+    return p;
+}
+
+// ceil(frac * n_blocks) in fp64 with a 1e-9 guard, clamped to [0, n_blocks]
+int promote_count(float frac, int n_blocks)
+{
+    if (!(frac > 0.0f) || n_blocks <= 0) return 0;
+    int k = (int)ceil((double)frac * (double)n_blocks - 1e-9);
+    return k < 0 ? 0 : (k > n_blocks ? n_blocks : k);
+}
+
+// Certified-mode workspace, after the decode partials: page statistics,
+// per-head totals, promoted-block lists and counts, promote partials and
+// the promote counters (zero between calls).
+struct CertWs {
+    size_t page_stats, head_ml, prom, prom_count, cpart, ccount, bytes;
+};
+
+CertWs cert_ws(const kvq_cache *c, int batch, int max_pages)
+{
+    CertWs w{};
+    if (c->L.bound_block <= 0) return w;
+    const size_t bk = (size_t)batch * c->L.hkv, g = c->L.g;
+    const size_t cap = (size_t)pow2_at_least(cert_blocks(c, max_pages));
+    size_t off = 0;
+    w.page_stats = off;
+    off += round256(bk * max_pages * g * 8);
+    w.head_ml = off;
+    off += round256(bk * g * 8);
+    w.prom = off;
+    off += round256(bk * cap * 4);
+    w.prom_count = off;
+    off += round256(bk * 4);
+    w.cpart = off;
+    off += round256(bk * kCertChunks * g * 2 * (c->L.d + 4) * 4);
+    w.ccount = off;
+    off += round256(bk * 4);
+    w.bytes = off;
+    return w;
+}
+
+// A device-accessible address for `p`: device or managed memory as is; pinned
+// host memory through its device mapping.  Null for unregistered host memory.
+const void *device_view(const void *p)
+{
+    cudaPointerAttributes a;
+    if (!p || cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return p;
+    if (a.type == cudaMemoryTypeHost) return a.devicePointer;
+    return nullptr;
+}
+
 kvq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
 
 }  // namespace
@@ -181,7 +250,7 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *c, int32_t batch, int32_t max
     if (!c || batch < 0 || max_pages_per_seq < 1) return 0;
     const SplitPlan s = plan_splits(c, batch, max_pages_per_seq);
     const size_t part = (size_t)batch * c->L.hkv * s.n_splits * c->L.g * (c->L.d + 4) * sizeof(float);
-    return counters_bytes(batch, c->L.hkv) + part;
+    return counters_bytes(batch, c->L.hkv) + round256(part) + cert_ws(c, batch, max_pages_per_seq).bytes;
 }
 
 }  // extern "C"
@@ -193,14 +262,27 @@ kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const
                        int32_t batch, float softmax_scale, const kvq_tier2 *tier2, void *workspace, size_t ws_bytes,
                        void *out, int32_t *promoted_out, void *stream)
 {
-    (void)promoted_out;
     if (!c || batch < 0 || max_pages_per_seq < 1) return KVQ_ERR_INVALID_ARG;
     if (batch == 0) return KVQ_OK;
     if (!q || !block_table || !ctx_lens || !out || !workspace) return KVQ_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
     if (k_new && (!v_new || !slot_mapping || !aligned(k_new, 16) || !aligned(v_new, 16))) return KVQ_ERR_INVALID_ARG;
     if (!decode_supported(c->L)) return KVQ_ERR_UNSUPPORTED;
-    if (tier2) return KVQ_ERR_UNSUPPORTED;
+    // certified mode: checks and the tier-2 device view
+    int kmax = 0;
+    const void *k2 = nullptr, *v2 = nullptr;
+    if (tier2) {
+        if (k_new || c->L.bound_block <= 0) return KVQ_ERR_INVALID_ARG;
+        if (!(tier2->promote_frac >= 0.0f && tier2->promote_frac <= 1.0f)) return KVQ_ERR_INVALID_ARG;
+        const int nb_max = cert_blocks(c, max_pages_per_seq);
+        if (nb_max > kCertMaxBlocks) return KVQ_ERR_UNSUPPORTED;
+        kmax = promote_count(tier2->promote_frac, nb_max);
+        if (kmax > 0) {
+            k2 = device_view(tier2->k_host);
+            v2 = device_view(tier2->v_host);
+            if (!k2 || !v2 || !aligned(k2, 16) || !aligned(v2, 16)) return KVQ_ERR_INVALID_ARG;
+        }
+    }
     if (ws_bytes < kvq_decode_workspace_bytes(c, batch, max_pages_per_seq)) return KVQ_ERR_CAPACITY;
     const SplitPlan s = plan_splits(c, batch, max_pages_per_seq);
     DecodeParams p{};
@@ -228,7 +310,43 @@ kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const
     p.clip = c->cfg.clip_ratio;
     c->last_stream = stream;
     const dim3 grid(s.n_splits, c->L.hkv, batch);
-    return cuda_status(launch_decode(p, grid, static_cast<cudaStream_t>(stream)));
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned char *cert_base = static_cast<unsigned char *>(workspace) + counters_bytes(batch, c->L.hkv) +
+                               round256((size_t)batch * c->L.hkv * s.n_splits * c->L.g * (c->L.d + 4) * 4);
+    const CertWs w = cert_ws(c, batch, max_pages_per_seq);
+    if (kmax > 0) p.page_stats = reinterpret_cast<float2 *>(cert_base + w.page_stats);
+    kvq_status rc = cuda_status(launch_decode(p, grid, st));
+    if (rc != KVQ_OK || kmax == 0) return rc;
+
+    CertParams cp{};
+    cp.pool = c->pool;
+    cp.q = p.q;
+    cp.block_table = block_table;
+    cp.ctx_lens = ctx_lens;
+    cp.max_pages = max_pages_per_seq;
+    cp.L = c->L;
+    cp.scale = scale;
+    cp.qscale = p.qscale;
+    cp.rot_scale = c->rot_scale;
+    cp.rotate = c->cfg.rotate;
+    memcpy(cp.signs, c->signs, sizeof(cp.signs));
+    cp.frac = tier2->promote_frac;
+    cp.sort_cap = pow2_at_least(cert_blocks(c, max_pages_per_seq));
+    cp.kmax_out = kmax;
+    cp.n_chunks = kmax < kCertChunks ? kmax : kCertChunks;
+    cp.page_stats = p.page_stats;
+    cp.head_ml = reinterpret_cast<float2 *>(cert_base + w.head_ml);
+    cp.prom = reinterpret_cast<int32_t *>(cert_base + w.prom);
+    cp.prom_count = reinterpret_cast<int32_t *>(cert_base + w.prom_count);
+    cp.promoted_out = promoted_out;
+    cp.k2 = static_cast<const __half *>(k2);
+    cp.v2 = static_cast<const __half *>(v2);
+    cp.cpart = reinterpret_cast<float *>(cert_base + w.cpart);
+    cp.ccount = reinterpret_cast<unsigned int *>(cert_base + w.ccount);
+    cp.out = p.out;
+    rc = cuda_status(launch_cert_select(cp, batch, st));
+    if (rc != KVQ_OK) return rc;
+    return cuda_status(launch_cert_promote(cp, batch, st));
 }
 
 }  // namespace

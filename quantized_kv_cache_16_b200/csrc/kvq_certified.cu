@@ -1,0 +1,558 @@
+// kvq_certified.cu -- the certified decode mode ["Runtime-Certified
+// Bounded-Error Quantized Attention", Methodology 1-3].
+//
+// The quantised decode kernel runs first and, besides its output, records
+// for every page and query head the pair (m, l): its running max and the sum
+// of 2^(s - m) over the page's tokens (log2 units).  Then:
+//
+//   select  (one CTA per sequence and kv head) per query head: the totals
+//           M, L of the quantised softmax, the mass P_b of every bound block,
+//           and with the block descriptors (eps: max key error, eta: max
+//           value error, nu: max |value|, all in the rotated domain)
+//             Delta_b = scale * ||q_r||_1 * eps_b
+//             A       = ln sum_b P_b e^(Delta_b)
+//             bound_b = P_b * ((e^(Delta_b + A) - 1) * nu_b + eta_b);
+//           a block's score is the largest bound over the group's heads; the
+//           top ceil(frac * n_blocks) blocks (ties: lower block first) are
+//           promoted.  The pages give the key term as a total-variation bound
+//           on the softmax shift and the value term as the mass-weighted
+//           value error, without a formula; this is the rigorous reading.
+//   promote (up to kCertChunks CTAs per sequence and kv head) reads the
+//           promoted blocks' exact fp16 rows from tier 2 (pinned host memory
+//           mapped into the device's address space), rotates them, and forms
+//           two partials per head over those tokens: with the exact rows and
+//           with the dequantised rows.  The last CTA replaces the quantised
+//           contribution of the promoted blocks by the exact one:
+//             o = (L 2^(M-R) o_q + R^T(acc_e 2^(m_e-R) - acc_q 2^(m_q-R)))
+//                 / (L 2^(M-R) + l_e 2^(m_e-R) - l_q 2^(m_q-R)).
+#include <math.h>
+
+#include "kvq_internal.cuh"
+#include "kvq_warp.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kSelThreads = 1024;  // 32 warps: one reduction slot per lane
+constexpr int kPromWarps = 8;
+constexpr int kPromThreads = kPromWarps * 32;
+constexpr int kTokBatch = 4;       // exact rows a warp has in flight per lane
+
+__device__ __forceinline__ int clamp_ctx(int T, int max_pages)
+{
+    return T < 0 ? 0 : (T > max_pages * kPageTokens ? max_pages * kPageTokens : T);
+}
+
+struct MaxOp {
+    __device__ float operator()(float a, float b) const { return fmaxf(a, b); }
+};
+struct SumOp {
+    __device__ double operator()(double a, double b) const { return a + b; }
+};
+
+// Reduce kMaxGqa values per thread over the whole CTA (32 warps); every
+// thread gets the results.  red: 32 * kMaxGqa elements of shared memory.
+template <typename T, typename Op>
+__device__ __forceinline__ void cta_reduce(T (&v)[kMaxGqa], T *red, Op op)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int h = 0; h < kMaxGqa; h++)
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) v[h] = op(v[h], __shfl_xor_sync(kFull, v[h], m));
+    __syncthreads();
+    if (lane == 0)
+#pragma unroll
+        for (int h = 0; h < kMaxGqa; h++) red[warp * kMaxGqa + h] = v[h];
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < kMaxGqa; h++) {
+        T x = red[lane * kMaxGqa + h];
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) x = op(x, __shfl_xor_sync(kFull, x, m));
+        v[h] = x;
+    }
+}
+
+// The rotated query row of head (b, head) in lane order: element lane*E + e.
+template <int D>
+__device__ __forceinline__ void rotated_query(const CertParams &p, int b, int head, int lane, float (&x)[D / 32])
+{
+    constexpr int E = D / 32;
+    const __half *qh = p.q + ((long long)b * p.L.hq + head) * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; e++) x[e] = __half2float(qh[e]);
+    if (p.rotate) {
+#pragma unroll
+        for (int e = 0; e < E; e++) x[e] *= p.signs[lane * E + e];
+        fwht_warp<D>(x, lane);
+#pragma unroll
+        for (int e = 0; e < E; e++) x[e] *= p.rot_scale;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_constant__ CertParams p)
+{
+    constexpr int E = D / 32;
+    const Layout &L = p.L;
+    const int kvh = blockIdx.x, b = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = L.g;
+    extern __shared__ unsigned long long keys[];
+    __shared__ double red_d[32 * kMaxGqa];
+    __shared__ float red_f[32 * kMaxGqa];
+    __shared__ float qn1[kMaxGqa];
+
+    const int T = clamp_ctx(p.ctx_lens[b], p.max_pages);
+    const int n_pages = (T + kPageTokens - 1) / kPageTokens;
+    const int block = L.bound_block, ppb = block / kPageTokens;
+    const int nb = (T + block - 1) / block;
+    const long long bk = (long long)b * L.hkv + kvh;
+    const float2 *ps = p.page_stats + bk * p.max_pages * g;
+    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
+
+    // ||q_r||_1 of each head (rotated query, softmax scale not applied)
+    if (warp < g) {
+        float x[E];
+        rotated_query<D>(p, b, kvh * g + warp, lane, x);
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; e++) a += fabsf(x[e]);
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) a += __shfl_xor_sync(kFull, a, m);
+        if (lane == 0) qn1[warp] = a;
+    }
+
+    // totals of the quantised softmax per head: M = max page max, L = sum l 2^(m - M)
+    float mh[kMaxGqa];
+#pragma unroll
+    for (int h = 0; h < kMaxGqa; h++) mh[h] = -INFINITY;
+    for (int i = tid; i < n_pages; i += kSelThreads)
+#pragma unroll
+        for (int h = 0; h < kMaxGqa; h++)
+            if (h < g) {
+                const float2 s = ps[(long long)i * g + h];
+                if (s.y > 0.f) mh[h] = fmaxf(mh[h], s.x);
+            }
+    cta_reduce(mh, red_f, MaxOp());
+    double lh[kMaxGqa];
+#pragma unroll
+    for (int h = 0; h < kMaxGqa; h++) lh[h] = 0.0;
+    for (int i = tid; i < n_pages; i += kSelThreads)
+#pragma unroll
+        for (int h = 0; h < kMaxGqa; h++)
+            if (h < g) {
+                const float2 s = ps[(long long)i * g + h];
+                if (s.y > 0.f) lh[h] += (double)s.y * exp2((double)s.x - (double)mh[h]);
+            }
+    cta_reduce(lh, red_d, SumOp());
+
+    // block descriptors (max over the block's pages) and masses P_b per head
+    auto block_desc = [&](int bb, float &eps, float &eta, float &nu) {
+        eps = eta = nu = 0.f;
+        const int p1 = min(bb * ppb + ppb, n_pages);
+        for (int i = bb * ppb; i < p1; i++) {
+            const int pg = bt[i];
+            if (pg < 0 || pg >= L.num_pages) continue;  // recorded by the decode kernel
+            const float4 dsc =
+                *reinterpret_cast<const float4 *>(p.pool + L.desc_off + ((long long)pg * L.hkv + kvh) * 16);
+            eps = fmaxf(eps, dsc.x);
+            eta = fmaxf(eta, dsc.y);
+            nu = fmaxf(nu, dsc.z);
+        }
+    };
+    auto block_mass = [&](int bb, double (&P)[kMaxGqa]) {
+#pragma unroll
+        for (int h = 0; h < kMaxGqa; h++) P[h] = 0.0;
+        const int p1 = min(bb * ppb + ppb, n_pages);
+        for (int i = bb * ppb; i < p1; i++)
+#pragma unroll
+            for (int h = 0; h < kMaxGqa; h++)
+                if (h < g) {
+                    const float2 s = ps[(long long)i * g + h];
+                    if (s.y > 0.f) P[h] += (double)s.y * exp2((double)s.x - (double)mh[h]);
+                }
+#pragma unroll
+        for (int h = 0; h < kMaxGqa; h++) P[h] = lh[h] > 0.0 ? P[h] / lh[h] : 0.0;
+    };
+    __syncthreads();  // qn1
+    const double scale = p.scale;
+
+    // A = ln sum_b P_b e^(Delta_b) per head
+    double sh[kMaxGqa];
+#pragma unroll
+    for (int h = 0; h < kMaxGqa; h++) sh[h] = 0.0;
+    for (int bb = tid; bb < nb; bb += kSelThreads) {
+        float eps, eta, nu;
+        block_desc(bb, eps, eta, nu);
+        double P[kMaxGqa];
+        block_mass(bb, P);
+#pragma unroll
+        for (int h = 0; h < kMaxGqa; h++)
+            if (h < g) sh[h] += P[h] * exp(scale * (double)qn1[h] * (double)eps);
+    }
+    cta_reduce(sh, red_d, SumOp());
+
+    // score of every block -> sort key (score bits, then the complement of
+    // the index so that equal scores order the lower block first)
+    int np2 = 1;
+    while (np2 < nb) np2 <<= 1;
+    for (int bb = tid; bb < np2; bb += kSelThreads) {
+        unsigned long long key = 0ull;
+        if (bb < nb) {
+            float eps, eta, nu;
+            block_desc(bb, eps, eta, nu);
+            double P[kMaxGqa];
+            block_mass(bb, P);
+            double sc = 0.0;
+#pragma unroll
+            for (int h = 0; h < kMaxGqa; h++)
+                if (h < g && P[h] > 0.0) {
+                    const double Db = scale * (double)qn1[h] * (double)eps;
+                    const double bound = P[h] * ((exp(Db + log(sh[h])) - 1.0) * (double)nu + (double)eta);
+                    sc = fmax(sc, bound);
+                }
+            float scf = (float)sc;
+            if (!(scf >= 0.f)) scf = 0.f;
+            key = ((unsigned long long)__float_as_uint(scf) << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)bb);
+        }
+        keys[bb] = key;
+    }
+    __syncthreads();
+
+    // bitonic sort of the keys, descending
+    for (int k = 2; k <= np2; k <<= 1)
+        for (int jj = k >> 1; jj > 0; jj >>= 1) {
+            for (int i = tid; i < np2; i += kSelThreads) {
+                const int ixj = i ^ jj;
+                if (ixj > i) {
+                    const unsigned long long a = keys[i], c = keys[ixj];
+                    const bool desc = (i & k) == 0;
+                    if (desc ? (a < c) : (a > c)) {
+                        keys[i] = c;
+                        keys[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+
+    // the top ceil(frac * nb) blocks (fp64, guarded so an exact product is not bumped up)
+    int kp = 0;
+    if (p.frac > 0.f && nb > 0) {
+        kp = (int)ceil((double)p.frac * (double)nb - 1e-9);
+        kp = kp < 0 ? 0 : (kp > nb ? nb : kp);
+    }
+    int32_t *prom = p.prom + bk * p.sort_cap;
+    for (int r = tid; r < kp; r += kSelThreads) prom[r] = (int)(0xFFFFFFFFu - (unsigned)(keys[r] & 0xFFFFFFFFull));
+    if (p.promoted_out)
+        for (int r = tid; r < p.kmax_out; r += kSelThreads)
+            p.promoted_out[bk * p.kmax_out + r] =
+                r < kp ? (int)(0xFFFFFFFFu - (unsigned)(keys[r] & 0xFFFFFFFFull)) : -1;
+    if (tid == 0) p.prom_count[bk] = kp;
+#pragma unroll
+    for (int h = 0; h < kMaxGqa; h++)
+        if (tid == h && h < g) p.head_ml[bk * g + h] = make_float2(mh[h], (float)lh[h]);
+}
+
+// Dequantised values of channels lane*E .. lane*E+E-1 of token `tok` in a
+// chunk (the same arithmetic as the stored codec: code*scale + zero, one
+// rounding; int8: code*scale).
+template <int E>
+__device__ __forceinline__ void dequant_lane(const unsigned char *chunk, int codes_off, int meta_off, int row_meta,
+                                             int fmt, int tok, int lane, float (&x)[E])
+{
+    const unsigned char *codes = chunk + codes_off;
+    const uint16_t *meta = reinterpret_cast<const uint16_t *>(chunk + meta_off + tok * row_meta);
+    const int bits = fmt_bits(fmt);
+    const int ng = row_meta / 4;  // asymmetric formats: scales then zeros
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        const int ch = lane * E + e;
+        const int bit = ch * bits, byte = bit >> 3;
+        const unsigned bv = codes[((byte >> 4) * 16 + tok) * 16 + (byte & 15)];
+        const int raw = (int)((bv >> (bit & 7)) & ((1u << bits) - 1u));
+        if (fmt == KVQ_INT8_SYM) {
+            x[e] = __fmul_rn((float)(int)(int8_t)raw, __half2float(__ushort_as_half(meta[0])));
+        } else {
+            const int gi = fmt == KVQ_INT4_ASYM ? ch / 32 : 0;
+            x[e] = __fmaf_rn((float)raw, __half2float(__ushort_as_half(meta[gi])),
+                             __half2float(__ushort_as_half(meta[ng + gi])));
+        }
+    }
+}
+
+template <int E>
+__device__ __forceinline__ void online_update(float &m, float &l, float (&a)[E], float s, const float (&v)[E])
+{
+    const float mn = fmaxf(m, s);
+    const float al = (m == -INFINITY) ? 0.f : ex2(m - mn);
+    const float pe = ex2(s - mn);
+    l = fmaf(l, al, pe);
+#pragma unroll
+    for (int e = 0; e < E; e++) a[e] = fmaf(a[e], al, pe * v[e]);
+    m = mn;
+}
+
+template <int E>
+__device__ __forceinline__ void load_row(const __half *src, float (&x)[E])
+{
+    if constexpr (E == 4) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(src);
+        const float2 a = __half22float2(bits_h2(u.x)), c = __half22float2(bits_h2(u.y));
+        x[0] = a.x;
+        x[1] = a.y;
+        x[2] = c.x;
+        x[3] = c.y;
+    } else {
+        const float2 a = __half22float2(bits_h2(*reinterpret_cast<const uint32_t *>(src)));
+        x[0] = a.x;
+        x[1] = a.y;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid_constant__ CertParams p)
+{
+    constexpr int E = D / 32;
+    const Layout &L = p.L;
+    const int chunk_id = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = L.g;
+    const long long bk = (long long)b * L.hkv + kvh;
+    const int kp = p.prom_count[bk];
+    const int n_act = min(kp, p.n_chunks);
+    if (chunk_id >= n_act) return;
+
+    extern __shared__ float wacc[];  // [kPromWarps][g][2][D]
+    __shared__ float sq[kMaxGqa * kMaxD];
+    __shared__ float wm[kPromWarps * kMaxGqa * 2], wl[kPromWarps * kMaxGqa * 2];
+    __shared__ int sflag;
+
+    const int T = clamp_ctx(p.ctx_lens[b], p.max_pages);
+    const int block = L.bound_block;
+    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
+    const int32_t *prom = p.prom + bk * p.sort_cap;
+
+    // rotated query of each head, pre-scaled into log2 units
+    if (warp < g) {
+        float x[E];
+        rotated_query<D>(p, b, kvh * g + warp, lane, x);
+#pragma unroll
+        for (int e = 0; e < E; e++) sq[warp * D + lane * E + e] = x[e] * p.qscale;
+    }
+    __syncthreads();
+    float qr[kMaxGqa][E];
+#pragma unroll
+    for (int h = 0; h < kMaxGqa; h++)
+#pragma unroll
+        for (int e = 0; e < E; e++) qr[h][e] = h < g ? sq[h * D + lane * E + e] : 0.f;
+
+    // (m, l, acc) over this CTA's promoted tokens: [0] exact rows, [1] dequantised rows
+    float m[kMaxGqa][2], l[kMaxGqa][2], acc[kMaxGqa][2][E];
+#pragma unroll
+    for (int h = 0; h < kMaxGqa; h++)
+#pragma unroll
+        for (int w = 0; w < 2; w++) {
+            m[h][w] = -INFINITY;
+            l[h][w] = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; e++) acc[h][w][e] = 0.f;
+        }
+
+    for (int r = chunk_id; r < kp; r += n_act) {
+        const int t0 = prom[r] * block, t1 = min(t0 + block, T);
+        for (int tb = t0 + warp * kTokBatch; tb < t1; tb += kPromWarps * kTokBatch) {
+            // issue the batch's exact-row loads (host link) before any math
+            float ke[kTokBatch][E], ve[kTokBatch][E];
+            int pgs[kTokBatch];
+#pragma unroll
+            for (int u = 0; u < kTokBatch; u++) {
+                const int t = tb + u;
+                int pg = -1;
+                if (t < t1) {
+                    pg = bt[t / kPageTokens];
+                    if (pg >= L.num_pages) pg = -1;
+                }
+                pgs[u] = pg;
+                if (pg >= 0) {
+                    const long long row = ((long long)(pg * kPageTokens + t % kPageTokens) * L.hkv + kvh) * D + lane * E;
+                    load_row<E>(p.k2 + row, ke[u]);
+                    load_row<E>(p.v2 + row, ve[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kTokBatch; u++) {
+                if (pgs[u] < 0) continue;  // warp-uniform
+                const int tok = (tb + u) % kPageTokens;
+                if (p.rotate) {
+#pragma unroll
+                    for (int e = 0; e < E; e++) {
+                        ke[u][e] *= p.signs[lane * E + e];
+                        ve[u][e] *= p.signs[lane * E + e];
+                    }
+                    fwht_warp<D>(ke[u], lane);
+                    fwht_warp<D>(ve[u], lane);
+#pragma unroll
+                    for (int e = 0; e < E; e++) {
+                        ke[u][e] *= p.rot_scale;
+                        ve[u][e] *= p.rot_scale;
+                    }
+                }
+                const unsigned char *chunk =
+                    p.pool + kHeaderBytes + (long long)pgs[u] * L.page_bytes + (long long)kvh * L.chunk_bytes;
+                float kq[E], vq[E];
+                dequant_lane<E>(chunk, L.k_codes, L.k_meta, L.k_row_meta, L.k_fmt, tok, lane, kq);
+                dequant_lane<E>(chunk, L.v_codes, L.v_meta, L.v_row_meta, L.v_fmt, tok, lane, vq);
+#pragma unroll
+                for (int h = 0; h < kMaxGqa; h++) {
+                    if (h >= g) break;
+                    float se = 0.f, sqv = 0.f;
+#pragma unroll
+                    for (int e = 0; e < E; e++) {
+                        se = fmaf(qr[h][e], ke[u][e], se);
+                        sqv = fmaf(qr[h][e], kq[e], sqv);
+                    }
+#pragma unroll
+                    for (int mm = 16; mm >= 1; mm >>= 1) {
+                        se += __shfl_xor_sync(kFull, se, mm);
+                        sqv += __shfl_xor_sync(kFull, sqv, mm);
+                    }
+                    online_update<E>(m[h][0], l[h][0], acc[h][0], se, ve[u]);
+                    online_update<E>(m[h][1], l[h][1], acc[h][1], sqv, vq);
+                }
+            }
+        }
+    }
+
+    // warps -> shared memory -> one partial per (head, exact|quantised)
+#pragma unroll
+    for (int h = 0; h < kMaxGqa; h++)
+        if (h < g)
+#pragma unroll
+            for (int w = 0; w < 2; w++) {
+#pragma unroll
+                for (int e = 0; e < E; e++) wacc[((warp * g + h) * 2 + w) * D + lane * E + e] = acc[h][w][e];
+                if (lane == 0) {
+                    wm[(warp * kMaxGqa + h) * 2 + w] = m[h][w];
+                    wl[(warp * kMaxGqa + h) * 2 + w] = l[h][w];
+                }
+            }
+    __syncthreads();
+    constexpr int REC = D + 4;
+    float *cp = p.cpart + (bk * p.n_chunks + chunk_id) * (long long)g * 2 * REC;
+    for (int idx = tid; idx < g * 2 * D; idx += kPromThreads) {
+        const int hw = idx / D, ch = idx - hw * D;  // hw = h * 2 + w
+        const int h = hw >> 1, w = hw & 1;
+        float M = -INFINITY;
+#pragma unroll
+        for (int ww = 0; ww < kPromWarps; ww++) M = fmaxf(M, wm[(ww * kMaxGqa + h) * 2 + w]);
+        float a = 0.f, Ls = 0.f;
+        if (M != -INFINITY)
+#pragma unroll
+            for (int ww = 0; ww < kPromWarps; ww++) {
+                const float mw = wm[(ww * kMaxGqa + h) * 2 + w];
+                const float f = mw == -INFINITY ? 0.f : ex2(mw - M);
+                a = fmaf(f, wacc[((ww * g + h) * 2 + w) * D + ch], a);
+                Ls = fmaf(f, wl[(ww * kMaxGqa + h) * 2 + w], Ls);
+            }
+        cp[hw * REC + ch] = a;
+        if (ch == 0) {
+            cp[hw * REC + D] = M;
+            cp[hw * REC + D + 1] = Ls;
+        }
+    }
+
+    // the last CTA of this (sequence, kv head) applies the correction
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(p.ccount + bk, 1u);
+        sflag = prev == (unsigned)(n_act - 1);
+    }
+    __syncthreads();
+    if (!sflag) return;
+    __threadfence();
+    if (tid == 0) p.ccount[bk] = 0u;
+    const float *cbase = p.cpart + bk * p.n_chunks * (long long)g * 2 * REC;
+    for (int h = warp; h < g; h += kPromWarps) {
+        float Mx[2] = {-INFINITY, -INFINITY}, Ls[2] = {0.f, 0.f}, a[2][E];
+#pragma unroll
+        for (int w = 0; w < 2; w++) {
+#pragma unroll
+            for (int e = 0; e < E; e++) a[w][e] = 0.f;
+            for (int c = 0; c < n_act; c++) Mx[w] = fmaxf(Mx[w], __ldcg(cbase + ((c * g + h) * 2 + w) * REC + D));
+            if (Mx[w] == -INFINITY) continue;
+            for (int c = 0; c < n_act; c++) {
+                const float *rec = cbase + ((c * g + h) * 2 + w) * REC;
+                const float mc = __ldcg(rec + D);
+                const float f = mc == -INFINITY ? 0.f : ex2(mc - Mx[w]);
+                Ls[w] = fmaf(f, __ldcg(rec + D + 1), Ls[w]);
+#pragma unroll
+                for (int e = 0; e < E; e++) a[w][e] = fmaf(f, __ldcg(rec + lane * E + e), a[w][e]);
+            }
+        }
+        const float2 ml = p.head_ml[bk * g + h];  // the quantised pass: (M, L)
+        float R = fmaxf(Mx[0], Mx[1]);
+        if (ml.y > 0.f) R = fmaxf(R, ml.x);
+        const float f0 = ml.y > 0.f ? ml.y * ex2(ml.x - R) : 0.f;
+        const float fe = Mx[0] == -INFINITY ? 0.f : ex2(Mx[0] - R);
+        const float fq = Mx[1] == -INFINITY ? 0.f : ex2(Mx[1] - R);
+        const float den = f0 + Ls[0] * fe - Ls[1] * fq;
+        float dlt[E];
+#pragma unroll
+        for (int e = 0; e < E; e++) dlt[e] = a[0][e] * fe - a[1][e] * fq;
+        if (p.rotate) {
+            fwht_warp<D>(dlt, lane);
+#pragma unroll
+            for (int e = 0; e < E; e++) dlt[e] *= p.rot_scale * p.signs[lane * E + e];
+        }
+        float *o = p.out + ((long long)b * L.hq + kvh * g + h) * D + lane * E;
+#pragma unroll
+        for (int e = 0; e < E; e++) o[e] = den > 0.f ? (f0 * o[e] + dlt[e]) / den : 0.f;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_cert_select(const CertParams &p, int batch, cudaStream_t s)
+{
+    static bool configured[2] = {false, false};
+    const int di = p.L.d == 64 ? 0 : 1;
+    const size_t smem = (size_t)p.sort_cap * sizeof(unsigned long long);
+    if (!configured[di]) {
+        const cudaError_t e =
+            di ? cudaFuncSetAttribute(cert_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kCertMaxBlocks * (int)sizeof(unsigned long long))
+               : cudaFuncSetAttribute(cert_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kCertMaxBlocks * (int)sizeof(unsigned long long));
+        if (e != cudaSuccess) return e;
+        configured[di] = true;
+    }
+    const dim3 grid(p.L.hkv, batch);
+    if (di) cert_select_kernel<128><<<grid, kSelThreads, smem, s>>>(p);
+    else cert_select_kernel<64><<<grid, kSelThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cert_promote(const CertParams &p, int batch, cudaStream_t s)
+{
+    static bool configured[2] = {false, false};
+    const int di = p.L.d == 64 ? 0 : 1;
+    const size_t smem = (size_t)kPromWarps * p.L.g * 2 * p.L.d * sizeof(float);
+    if (!configured[di]) {
+        const int cap = kPromWarps * kMaxGqa * 2 * kMaxD * (int)sizeof(float);
+        const cudaError_t e =
+            di ? cudaFuncSetAttribute(cert_promote_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, cap)
+               : cudaFuncSetAttribute(cert_promote_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
+        if (e != cudaSuccess) return e;
+        configured[di] = true;
+    }
+    const dim3 grid(p.n_chunks, p.L.hkv, batch);
+    if (di) cert_promote_kernel<128><<<grid, kPromThreads, smem, s>>>(p);
+    else cert_promote_kernel<64><<<grid, kPromThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace kvq

@@ -33,13 +33,12 @@
 #include <math.h>
 
 #include "kvq_internal.cuh"
+#include "kvq_warp.cuh"
 
 namespace kvq {
 namespace {
 
-constexpr unsigned kFull = 0xffffffffu;
 constexpr int kCombineSplits = 40;  // split records the last CTA can stage
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per stage wait
 
 // fp16x2 constants (bit patterns)
 constexpr uint32_t kH1024 = 0x64006400u;  // (1024, 1024)
@@ -84,13 +83,6 @@ __device__ __forceinline__ uint32_t hilo(float x)
 {
     const float hf = __half2float(__float2half_rn(x));
     return pack_h2(x, x - hf);
-}
-
-__device__ __forceinline__ float ex2(float x)
-{
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
 }
 
 __device__ __forceinline__ uint32_t movm_t(uint32_t x)
@@ -457,29 +449,6 @@ __device__ __forceinline__ void ld_vrows_t(uint32_t base, int lane, uint32_t (&w
         uint32_t d0, d1;
         ldsm_x4_t(base + tok * 16, wA[0], wB[0], d0, d1);
     }
-}
-
-// Walsh-Hadamard transform of a warp-wide vector (element lane*E + e), fp32.
-template <int D>
-__device__ __forceinline__ void fwht_warp(float (&x)[D / 32], int lane)
-{
-    constexpr int E = D / 32;
-#pragma unroll
-    for (int h = 1; h < E; h <<= 1)
-#pragma unroll
-        for (int e = 0; e < E; e++)
-            if (!(e & h)) {
-                const float a = x[e], b = x[e + h];
-                x[e] = a + b;
-                x[e + h] = a - b;
-            }
-#pragma unroll
-    for (int m = 1; m < 32; m <<= 1)
-#pragma unroll
-        for (int e = 0; e < E; e++) {
-            const float o = __shfl_xor_sync(kFull, x[e], m);
-            x[e] = (lane & m) ? (o - x[e]) : (x[e] + o);
-        }
 }
 
 __device__ __forceinline__ float h2f_bits(uint16_t u) { return __half2float(__ushort_as_half(u)); }
@@ -894,6 +863,17 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
                 p_r[t] = live ? ex2(s_r[t] - m_run[t]) : 0.f;
                 p_r8[t] = live ? ex2(s_r8[t] - m_run[t]) : 0.f;
                 l_part[t] += p_r[t] + p_r8[t];
+            }
+            if (p.page_stats != nullptr) {  // certified mode: this page's (m, l) per head
+                float2 *ps = p.page_stats + (((long long)b * L.hkv + kvh) * p.max_pages + p_begin + i) * g;
+#pragma unroll
+                for (int t = 0; t < NH; t++) {
+                    float l = p_r[t] + p_r8[t];
+                    l += __shfl_xor_sync(kFull, l, 4);
+                    l += __shfl_xor_sync(kFull, l, 8);
+                    l += __shfl_xor_sync(kFull, l, 16);
+                    if (r == 0 && j + 4 * t < g) ps[j + 4 * t] = make_float2(m_run[t], l);
+                }
             }
         }
 

@@ -118,6 +118,9 @@ struct DecodeParams {
     const __half *new_v;
     const int32_t *new_slots; // [B]: the slot of position ctx_lens[b] - 1
     float clip;
+    // certified mode: per page and head (m, l) = (running max, sum of
+    // 2^(s - m) over the page's tokens), log2 units; null = off
+    float2 *page_stats;       // [B][Hkv][max_pages][g]
 };
 
 struct DequantParams {
@@ -131,11 +134,50 @@ struct DequantParams {
     uint16_t *meta_out;
 };
 
+// Certified mode ["Runtime-Certified Bounded-Error Quantized Attention",
+// Methodology 1-3]: after the quantised decode (which records page_stats),
+// one CTA per (sequence, kv head) turns the page statistics and the block
+// descriptors into per-block error bounds and picks the top blocks; then up
+// to kCertChunks CTAs per (sequence, kv head) recompute those blocks from the
+// exact fp16 rows (tier 2) and correct the output in place.
+constexpr int kCertChunks = 16;       // promote CTAs per (sequence, kv head)
+constexpr int kCertMaxBlocks = 16384; // bound blocks per sequence the selection can sort
+
+struct CertParams {
+    const unsigned char *pool;
+    const __half *q;
+    const int32_t *block_table;
+    const int32_t *ctx_lens;
+    int max_pages;
+    Layout L;
+    float scale;   // softmax scale (natural units)
+    float qscale;  // scale * log2(e)
+    float rot_scale;
+    int rotate;
+    float signs[kMaxD];
+    float frac;        // promoted fraction of each (sequence, kv head)'s blocks
+    int sort_cap;      // power of two >= every sequence's block count
+    int kmax_out;      // columns of promoted_out
+    int n_chunks;      // promote CTAs per (sequence, kv head)
+    const float2 *page_stats;  // [B][Hkv][max_pages][g] from the decode kernel
+    float2 *head_ml;           // [B][Hkv][g]: (M, L) of the quantised pass, log2 units
+    int32_t *prom;             // [B][Hkv][sort_cap]: promoted blocks, highest bound first
+    int32_t *prom_count;       // [B][Hkv]
+    int32_t *promoted_out;     // optional [B][Hkv][kmax_out], -1 padded
+    const __half *k2;          // tier 2: exact rows [num_pages*16][Hkv][d] fp16, device-accessible
+    const __half *v2;
+    float *cpart;              // [B][Hkv][n_chunks][g][2][d + 4]: exact / quantised block partials
+    unsigned int *ccount;      // [B][Hkv], zero between calls
+    float *out;                // [B][Hq][d]
+};
+
 // launchers (return cudaGetLastError() of the launch)
 cudaError_t launch_append(const AppendParams &p, int k_group, int v_group, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, dim3 grid, cudaStream_t s);
 cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
 cudaError_t launch_reset_pages(unsigned char *pool, Layout L, const int32_t *pages, int n, cudaStream_t s);
+cudaError_t launch_cert_select(const CertParams &p, int batch, cudaStream_t s);
+cudaError_t launch_cert_promote(const CertParams &p, int batch, cudaStream_t s);
 bool decode_supported(const Layout &L);
 int decode_max_splits(const Layout &L);
 constexpr int kDecodeWarps = 8;

@@ -492,3 +492,21 @@ def test_certified_promotes_top_scores_and_reduces_error():
         order = sorted(range(nb), key=lambda b: (-scores[0, kvh, b], b))[:k]
         assert sel.tolist() == order
     assert np.linalg.norm(out - exact) <= np.linalg.norm(quant - exact)
+
+
+def test_certified_forced_selection():
+    """Forcing the oracle's own top-k reproduces its output exactly; forcing
+    every block gives fp16 attention; forcing none gives quantised attention."""
+    wl, cfg, pool, pages, ks, vs = _cert_case(T=900)
+    q = W.queries(wl, 1)
+    bt, ctx = pages.block_table, wl.ctx
+    nb = (ctx[0] + 127) // 128
+    out, prom, _, _ = O.decode_certified(cfg, pool, ks, vs, q, bt, ctx, 0.3)
+    out_f, prom_f, _, _ = O.decode_certified(cfg, pool, ks, vs, q, bt, ctx, 0.3, forced=prom)
+    assert np.array_equal(out, out_f) and np.array_equal(prom, prom_f)
+    every = np.tile(np.arange(nb, dtype=np.int32), (1, wl.Hkv, 1))
+    out_all, _, _, _ = O.decode_certified(cfg, pool, ks, vs, q, bt, ctx, 0.0, forced=every)
+    assert np.allclose(out_all, O.decode_fp16(cfg, ks, vs, q, bt, ctx), rtol=0, atol=1e-10)
+    none = np.full((1, wl.Hkv, 3), -1, np.int32)
+    out_none, _, _, _ = O.decode_certified(cfg, pool, ks, vs, q, bt, ctx, 0.5, forced=none)
+    assert np.allclose(out_none, O.decode(cfg, pool, q, bt, ctx), rtol=0, atol=1e-12)
