@@ -35,6 +35,29 @@ METRIC = "int4-KV decode attn: KV-bytes GB/s as % of HBM peak; µs/step; append 
 NOMINAL_HBM_GBS = 8000.0
 
 
+# DRAM bytes (read + write) per launch of the dominant kernel from the ncu
+# capture summarised under profiles/ (decode_kernel_llama3-8b-layer-T32768.md).
+# Reported as roofline.traffic only while the decode kernel's sources hash to
+# the digest they had when the counters were taken; null otherwise.
+PROFILED_DECODE = {"sources_sha256": None, "dram_bytes_per_launch": None}
+DECODE_SOURCES = ("kvq_decode.cu", "kvq_internal.cuh", "kvq_warp.cuh")
+
+
+def decode_sources_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "quantized_kv_cache_16_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic():
+    if PROFILED_DECODE["sources_sha256"] and PROFILED_DECODE["sources_sha256"] == decode_sources_digest():
+        return PROFILED_DECODE["dram_bytes_per_launch"]
+    return None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -338,7 +361,7 @@ def run_ours(args, dist: Dist):
         "pct_hbm_peak": value / dist.world / peak, "peak_gbs": peak, "peak_kind": peak_kind,
         "pct_hbm_nominal_8tbs": value / dist.world / NOMINAL_HBM_GBS,
         "roofline": {"bound": "hbm", "kernel": "decode_kernel<128,int4,int4> (fused append + decode step)", "achieved": round(achieved, 1),
-                     "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": profiled_traffic(),
                      "bytes_per_launch": alg, "launch_us": dec_mean * 1e3,
                      "note": f"peak of {peak_kind}"},
         "gpu_launches": K,
@@ -347,6 +370,7 @@ def run_ours(args, dist: Dist):
     if not args.no_extras:
         result["e2e"] = e2e_leg(wk, K, stream, dist)
         result["append"] = append_leg()
+        result["certified"] = certified_leg(min(K, 200))
     if dist.rank == 0:
         if not args.no_extras:
             result["cpu_baseline"] = cpu_leg(wk, args.cpu_steps)
@@ -442,6 +466,86 @@ def append_leg():
     return {"workload": "prefill append 65536 x 8 x 128 K and V, 2-bit g128 clip 0.9, rotated",
             "GB/s": round(gbs, 1), "us": us, "bytes": in_bytes + out_bytes, "pct_hbm_peak": gbs / peak,
             "peak_kind": kind, "inputs_exceed_l2": True}
+
+
+def certified_leg(steps: int):
+    """Certified decode at its own configuration: batch 1, context 131072,
+    int8 K / int4 g32 V, 128-token bound blocks, top 1% of each kv head's
+    blocks promoted from exact fp16 rows in pinned host memory.  Timed per
+    call (three launches) in a CUDA graph over two cache copies (440 MB >
+    3x L2), beside the plain quantised decode of the same cache."""
+    import torch
+
+    import quantized_kv_cache_16_b200 as K
+    import workloads as W
+    wl = W.certified()
+    T, frac, copies = wl.ctx[0], 0.01, 2
+    dev = torch.device("cuda", torch.cuda.current_device())
+    tabs = W.page_table(wl, copies=copies)
+    cfg = K.make_config(wl.Hq, wl.Hkv, wl.d, wl.k_fmt, wl.v_fmt, wl.k_group, wl.v_group, wl.clip, wl.rotation_seed,
+                        num_pages=tabs[0].num_pages, bound_block_tokens=wl.bound_block)
+    cache = K.Cache(cfg)
+    kd, vd = W.prefix_kv_device(wl, 0, dev)
+    rows = tabs[0].num_pages * 16
+    k2 = torch.empty((rows, wl.Hkv, wl.d), dtype=torch.float16).pin_memory()
+    v2 = torch.empty_like(k2).pin_memory()
+    kh, vh = kd.cpu(), vd.cpu()
+    for c in range(copies):
+        sl = torch.from_numpy(tabs[c].slots(0, 0, T)).long()
+        cache.append(kd, vd, sl.int().to(dev))
+        k2[sl], v2[sl] = kh, vh
+    del kd, vd, kh, vh
+    nq = 8
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed)
+    qs = torch.randn((nq, 1, wl.Hq, wl.d), generator=gen, device=dev).half()
+    bts = [torch.from_numpy(t.block_table).to(dev) for t in tabs]
+    max_pages = bts[0].shape[1]
+    ctx = torch.tensor([T], dtype=torch.int32, device=dev)
+    ws = cache.workspace_for(1, max_pages)
+    out = torch.empty((1, wl.Hq, wl.d), dtype=torch.float32, device=dev)
+    nb = (T + wl.bound_block - 1) // wl.bound_block
+    kmax = math.ceil(frac * nb - 1e-9)
+    prom = torch.empty((1, wl.Hkv, kmax), dtype=torch.int32, device=dev)
+    t2 = K.kvq_tier2(k2.data_ptr(), v2.data_ptr(), frac)
+    stream = torch.cuda.Stream()
+    rt = Cudart()
+
+    def call(s, tier2):
+        K.kvq_decode_attn(cache.handle, qs[s % nq], bts[s % copies], max_pages, ctx, 1, 0.0, tier2, ws, ws.numel(),
+                          out, prom if tier2 is not None else None, stream)
+
+    res = {}
+    for name, tier2 in (("quantised_only", None), ("certified", t2)):
+        with torch.cuda.stream(stream):
+            for s in range(4):
+                call(s, tier2)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        evs = [(rt.event(), rt.event()) for _ in range(steps)]
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+            for s in range(steps):
+                rt.record_external(evs[s][0], stream.cuda_stream)
+                call(s, tier2)
+                rt.record_external(evs[s][1], stream.cuda_stream)
+        g.replay()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        res[name] = statistics.mean(rt.elapsed_ms(a, b) for a, b in evs) * 1e3
+        del g
+    assert cache.sync_status() == 0
+    hbm = T * wl.Hkv * (wl.d + 2 + wl.d // 2 + 4 * (wl.d // 32))
+    link = wl.Hkv * kmax * wl.bound_block * wl.d * 2 * 2
+    peak, kind = measured_peaks()
+    return {"workload": "certified decode: B=1, 32/8 heads, d=128, context 131072, int8 K / int4 g32 V, "
+                        "128-token bound blocks, top 1% promoted from pinned host fp16 rows",
+            "us": round(res["certified"], 2), "quantised_only_us": round(res["quantised_only"], 2),
+            "overhead_x": round(res["certified"] / res["quantised_only"], 2),
+            "hbm_bytes": hbm, "host_link_bytes": link, "promoted_blocks_per_kv_head": kmax,
+            "quantised_only_GB/s": round(hbm / (res["quantised_only"] * 1e-6) / 1e9, 1),
+            "quantised_only_pct_hbm_peak": hbm / (res["quantised_only"] * 1e-6) / 1e9 / peak, "peak_kind": kind,
+            "l2_policy": "2 cache copies (440 MB) alternate", "steps": steps}
 
 
 def cpu_leg(wk: Workload, n_steps: int):

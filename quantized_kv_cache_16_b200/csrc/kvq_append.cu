@@ -6,14 +6,17 @@
 // Certified Bounded-Error Quantized Attention", Methodology 1: INT8 keys,
 // INT4 values, per-block error descriptors; "OSCAR", 2.2: INT2 with clipping].
 //
-// A row of d elements is spread over d/32 consecutive lanes, one 32-element
-// slice each.  Butterfly stages h = 1..16 stay inside a slice (registers);
-// stages h = 32 and 64 pair slice s with s^1 and s^2 (one shuffle and one
-// exact fma(+-1, x, partner) per element), in the same stage order as a plain
-// fp32 statement of the transform.  For int4 a slice is one quantisation
-// group; int2/int8 row statistics reduce over the row's lanes.  Every codec
-// operation is an explicitly rounded intrinsic so the integer codes match
-// that plain statement bit for bit.
+// A row of d elements is spread over d/64 consecutive lanes (one lane for
+// d = 64, two for d = 128), 64 elements each, held as 32 fp32 pairs.  The
+// butterfly stage h = 1 pairs the two halves of a register pair (scalar
+// add/sub); stages h = 2..32 pair register pairs (packed f32x2 add / fma);
+// stage h = 64 pairs the row's two lanes (one shuffle per element and a
+// packed exact fma(+-1, x, partner)).  The stages run in the order h = 1, 2,
+// 4, ... of a plain fp32 statement of the transform, each result rounded to
+// nearest, and every codec operation is an explicitly rounded operation, so
+// the integer codes match that plain statement bit for bit.  For int4 a lane
+// holds two quantisation groups; int2/int8 row statistics reduce over the
+// row's lanes.
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -21,13 +24,6 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer (ties to even)
-
-// code (as the low bits of x + magic), clamped to [lo, hi] before rounding
-__device__ __forceinline__ uint32_t round_code(float v, float lo, float hi)
-{
-    v = fminf(fmaxf(v, lo), hi);
-    return __float_as_uint(__fadd_rn(v, kRoundMagic));
-}
 
 __device__ __forceinline__ float code_value(uint32_t cw) { return __fsub_rn(__uint_as_float(cw), kRoundMagic); }
 
@@ -38,7 +34,37 @@ __device__ __forceinline__ uint32_t pack4bytes(uint32_t b0, uint32_t b1, uint32_
     return __byte_perm(t01, t23, 0x5410);
 }
 
-// min/max/sum over the `lanes` consecutive lanes that hold one row
+__device__ __forceinline__ float min3(float a, float b, float c)
+{
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// a - b, rounded once: fma(b, -1, a)
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
+
+// codes of a pair: clamp(rint((y - z) * inv), lo, hi) as the low bits of
+// (value + magic); the clamp comes before the rounding, which gives the same
+// integer
+__device__ __forceinline__ void quant_pair(float2 y, float2 z2, float2 inv2, float lo, float hi, uint32_t &c0,
+                                           uint32_t &c1)
+{
+    float2 t = __fmul2_rn(sub2(y, z2), inv2);
+    t.x = fminf(fmaxf(t.x, lo), hi);
+    t.y = fminf(fmaxf(t.y, lo), hi);
+    t = __fadd2_rn(t, make_float2(kRoundMagic, kRoundMagic));
+    c0 = __float_as_uint(t.x);
+    c1 = __float_as_uint(t.y);
+}
+
 template <int LANES> __device__ __forceinline__ float row_min(float v)
 {
 #pragma unroll
@@ -52,54 +78,85 @@ template <int LANES> __device__ __forceinline__ float row_max(float v)
     return v;
 }
 
-template <int D, int FMT>
-__device__ __forceinline__ void slice_row(const AppendParams &p, const uint32_t *sign_xor, const __half *src,
-                                          unsigned char *chunk, int tok, int tensor, int s, bool active,
-                                          unsigned int *desc)
+// min and max of y[i0 .. i0+n) (pairs), 3-input min/max
+template <int N>
+__device__ __forceinline__ void pair_minmax(const float2 *y, float &lo, float &hi)
 {
-    constexpr int LANES = D / 32;
-    const Layout &L = p.L;
-    // ---- load 32 fp16, flip signs (exact), widen ----
-    float y[32];
-    {
-        const uint4 *s4 = reinterpret_cast<const uint4 *>(src + 32 * s);
+    lo = fminf(y[0].x, y[0].y);
+    hi = fmaxf(y[0].x, y[0].y);
 #pragma unroll
-        for (int i = 0; i < 4; i++) {
-            uint4 w = active ? __ldg(s4 + i) : make_uint4(0, 0, 0, 0);
-            uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    for (int i = 1; i < N; i++) {
+        lo = min3(lo, y[i].x, y[i].y);
+        hi = max3(hi, y[i].x, y[i].y);
+    }
+}
+
+// Dequantisation error and magnitude of a pair (descriptors): the stored
+// value is code * scale + zero, each step rounded.
+__device__ __forceinline__ void pair_err(float2 y, uint32_t c0, uint32_t c1, float2 s2, float2 z2, float &emax,
+                                         float &amax)
+{
+    float2 yh = make_float2(code_value(c0), code_value(c1));
+    yh = __fadd2_rn(__fmul2_rn(yh, s2), z2);
+    const float2 e = sub2(y, yh);
+    emax = max3(emax, fabsf(e.x), fabsf(e.y));
+    amax = max3(amax, fabsf(y.x), fabsf(y.y));
+}
+
+template <int D, int FMT>
+__device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *sign_xor, const __half *src,
+                                         unsigned char *chunk, int tok, int tensor, int s, bool active,
+                                         unsigned int *desc)
+{
+    constexpr int LANES = D / 64;
+    const Layout &L = p.L;
+    // ---- load 64 fp16, flip signs (exact), widen to 32 pairs ----
+    float2 y[32];
+    {
+        const uint4 *s4 = reinterpret_cast<const uint4 *>(src + 64 * s);
+        uint4 w[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) w[i] = active ? __ldg(s4 + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            uint32_t ww[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
 #pragma unroll
             for (int e = 0; e < 4; e++) {
                 uint32_t x = ww[e];
-                if (p.rotate) x ^= sign_xor[16 * s + 4 * i + e];
-                const float2 f = __half22float2(bits_h2(x));
-                y[8 * i + 2 * e] = f.x;
-                y[8 * i + 2 * e + 1] = f.y;
+                if (p.rotate) x ^= sign_xor[32 * s + 4 * i + e];
+                y[4 * i + e] = __half22float2(bits_h2(x));
             }
         }
     }
-    // ---- butterflies: h = 1..16 in the slice, h = 32, 64 across slices ----
+    // ---- butterflies: h = 1 inside a pair, h = 2..32 across pairs, h = 64 across lanes ----
     if (p.rotate) {
 #pragma unroll
-        for (int h = 1; h < 32; h <<= 1)
-#pragma unroll
-            for (int jj = 0; jj < 32; jj++)
-                if (!(jj & h)) {
-                    const float a = y[jj], b = y[jj + h];
-                    y[jj] = __fadd_rn(a, b);
-                    y[jj + h] = __fsub_rn(a, b);
-                }
-#pragma unroll
-        for (int m = 1; m < LANES; m <<= 1) {
-            // lower slice: a + b; upper slice: a - b with a = the lower's value
-            const float sg = (s & m) ? -1.0f : 1.0f;
-#pragma unroll
-            for (int jj = 0; jj < 32; jj++) {
-                const float o = __shfl_xor_sync(kFull, y[jj], m);
-                y[jj] = __fmaf_rn(sg, y[jj], o);
-            }
+        for (int i = 0; i < 32; i++) {
+            const float a = y[i].x, b = y[i].y;
+            y[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
         }
 #pragma unroll
-        for (int jj = 0; jj < 32; jj++) y[jj] = __fmul_rn(y[jj], p.rot_scale);
+        for (int hh = 1; hh < 32; hh <<= 1)
+#pragma unroll
+            for (int i = 0; i < 32; i++)
+                if (!(i & hh)) {
+                    const float2 a = y[i], b = y[i + hh];
+                    y[i] = __fadd2_rn(a, b);
+                    y[i + hh] = sub2(a, b);
+                }
+        if constexpr (LANES == 2) {
+            // lower lane: a + b; upper lane: a - b with a = the lower lane's value
+            const float sg = s ? -1.0f : 1.0f;
+            const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+            for (int i = 0; i < 32; i++) {
+                const float2 o = make_float2(__shfl_xor_sync(kFull, y[i].x, 1), __shfl_xor_sync(kFull, y[i].y, 1));
+                y[i] = __ffma2_rn(sg2, y[i], o);
+            }
+        }
+        const float2 c2 = make_float2(p.rot_scale, p.rot_scale);
+#pragma unroll
+        for (int i = 0; i < 32; i++) y[i] = __fmul2_rn(y[i], c2);
     }
 
     unsigned char *codes = chunk + (tensor ? L.v_codes : L.k_codes);
@@ -108,55 +165,48 @@ __device__ __forceinline__ void slice_row(const AppendParams &p, const uint32_t 
     float emax = 0.0f, amax = 0.0f;
 
     if (FMT == KVQ_INT4_ASYM) {
-        // one group per slice, 16 bytes = one chunk
-        float lo = y[0], hi = y[0];
+        // two groups of 32 per lane (16 pairs each), one 16-byte chunk each
+        uint32_t sz[2][2];  // [scale|zero][group] fp16 bits
 #pragma unroll
-        for (int i = 1; i < 32; i++) {
-            lo = fminf(lo, y[i]);
-            hi = fmaxf(hi, y[i]);
-        }
-        if (p.clip < 1.0f) {
-            lo = __fmul_rn(lo, p.clip);
-            hi = __fmul_rn(hi, p.clip);
-        }
-        const __half shh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
-        const __half zhh = __float2half_rn(lo);
-        const float sf = __half2float(shh), zf = __half2float(zhh);
-        const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
-        uint32_t w[4];
-#pragma unroll
-        for (int m = 0; m < 4; m++) {
-            uint32_t bb[4];
-#pragma unroll
-            for (int k = 0; k < 4; k++) {
-                uint32_t cw[2];
-#pragma unroll
-                for (int e = 0; e < 2; e++) {
-                    const float yi = y[8 * m + 2 * k + e];
-                    cw[e] = round_code(__fmul_rn(__fsub_rn(yi, zf), inv), 0.0f, 15.0f);
-                    if (want_desc) {
-                        const float yhat = __fadd_rn(__fmul_rn(code_value(cw[e]), sf), zf);
-                        emax = fmaxf(emax, fabsf(__fsub_rn(yi, yhat)));
-                        amax = fmaxf(amax, fabsf(yi));
-                    }
-                }
-                bb[k] = cw[0] + (cw[1] << 4);
+        for (int gq = 0; gq < 2; gq++) {
+            const float2 *yg = y + 16 * gq;
+            float lo, hi;
+            pair_minmax<16>(yg, lo, hi);
+            if (p.clip < 1.0f) {
+                lo = __fmul_rn(lo, p.clip);
+                hi = __fmul_rn(hi, p.clip);
             }
-            w[m] = pack4bytes(bb[0], bb[1], bb[2], bb[3]);
+            const __half shh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
+            const __half zhh = __float2half_rn(lo);
+            const float sf = __half2float(shh), zf = __half2float(zhh);
+            const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
+            const float2 z2 = make_float2(zf, zf), inv2 = make_float2(inv, inv), s2 = make_float2(sf, sf);
+            uint32_t w[4];
+#pragma unroll
+            for (int m = 0; m < 4; m++) {
+                uint32_t bb[4];
+#pragma unroll
+                for (int k = 0; k < 4; k++) {
+                    uint32_t c0, c1;
+                    quant_pair(yg[4 * m + k], z2, inv2, 0.0f, 15.0f, c0, c1);
+                    if (want_desc) pair_err(yg[4 * m + k], c0, c1, s2, z2, emax, amax);
+                    bb[k] = c0 + (c1 << 4);
+                }
+                w[m] = pack4bytes(bb[0], bb[1], bb[2], bb[3]);
+            }
+            if (active) *reinterpret_cast<uint4 *>(codes + ((2 * s + gq) * 16 + tok) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+            sz[0][gq] = __half_as_ushort(shh);
+            sz[1][gq] = __half_as_ushort(zhh);
         }
         if (active) {
-            *reinterpret_cast<uint4 *>(codes + (s * 16 + tok) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-            reinterpret_cast<uint16_t *>(meta)[s] = __half_as_ushort(shh);
-            reinterpret_cast<uint16_t *>(meta)[LANES + s] = __half_as_ushort(zhh);
+            constexpr int NG = D / 32;
+            *reinterpret_cast<uint32_t *>(meta + 4 * s) = sz[0][0] | (sz[0][1] << 16);
+            *reinterpret_cast<uint32_t *>(meta + 2 * NG + 4 * s) = sz[1][0] | (sz[1][1] << 16);
         }
     } else if (FMT == KVQ_INT2_ASYM) {
-        // one group over the row; this slice's 32 codes are bytes [8s, 8s+8)
-        float lo = y[0], hi = y[0];
-#pragma unroll
-        for (int i = 1; i < 32; i++) {
-            lo = fminf(lo, y[i]);
-            hi = fmaxf(hi, y[i]);
-        }
+        // one group over the row; this lane's 64 codes are stream bytes [16s, 16s+16)
+        float lo, hi;
+        pair_minmax<32>(y, lo, hi);
         lo = row_min<LANES>(lo);
         hi = row_max<LANES>(hi);
         if (p.clip < 1.0f) {
@@ -167,64 +217,58 @@ __device__ __forceinline__ void slice_row(const AppendParams &p, const uint32_t 
         const __half zhh = __float2half_rn(lo);
         const float sf = __half2float(shh), zf = __half2float(zhh);
         const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
-        uint32_t w[2];
+        const float2 z2 = make_float2(zf, zf), inv2 = make_float2(inv, inv), s2 = make_float2(sf, sf);
+        uint32_t w[4];
 #pragma unroll
-        for (int m = 0; m < 2; m++) {
+        for (int m = 0; m < 4; m++) {
             uint32_t bb[4];
 #pragma unroll
             for (int k = 0; k < 4; k++) {
-                uint32_t cw[4];
-#pragma unroll
-                for (int e = 0; e < 4; e++) {
-                    const float yi = y[16 * m + 4 * k + e];
-                    cw[e] = round_code(__fmul_rn(__fsub_rn(yi, zf), inv), 0.0f, 3.0f);
-                    if (want_desc) {
-                        const float yhat = __fadd_rn(__fmul_rn(code_value(cw[e]), sf), zf);
-                        emax = fmaxf(emax, fabsf(__fsub_rn(yi, yhat)));
-                        amax = fmaxf(amax, fabsf(yi));
-                    }
+                uint32_t c[4];
+                quant_pair(y[8 * m + 2 * k], z2, inv2, 0.0f, 3.0f, c[0], c[1]);
+                quant_pair(y[8 * m + 2 * k + 1], z2, inv2, 0.0f, 3.0f, c[2], c[3]);
+                if (want_desc) {
+                    pair_err(y[8 * m + 2 * k], c[0], c[1], s2, z2, emax, amax);
+                    pair_err(y[8 * m + 2 * k + 1], c[2], c[3], s2, z2, emax, amax);
                 }
-                bb[k] = cw[0] + (cw[1] << 2) + (cw[2] << 4) + (cw[3] << 6);
+                bb[k] = c[0] + (c[1] << 2) + (c[2] << 4) + (c[3] << 6);
             }
             w[m] = pack4bytes(bb[0], bb[1], bb[2], bb[3]);
         }
         if (active) {
-            const int byte0 = 8 * s;  // stream byte of this slice
-            *reinterpret_cast<uint2 *>(codes + ((byte0 / 16) * 16 + tok) * 16 + byte0 % 16) = make_uint2(w[0], w[1]);
+            *reinterpret_cast<uint4 *>(codes + (s * 16 + tok) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
             if (s == 0)
-                *reinterpret_cast<uint32_t *>(meta) =
-                    __half_as_ushort(shh) | (uint32_t(__half_as_ushort(zhh)) << 16);
+                *reinterpret_cast<uint32_t *>(meta) = __half_as_ushort(shh) | (uint32_t(__half_as_ushort(zhh)) << 16);
         }
     } else {
-        // symmetric int8, one fp16 scale (rounded up) per row; 32 bytes per slice
-        float a = 0.0f;
+        // symmetric int8, one fp16 scale (rounded up) per row; 64 bytes per lane
+        float a = fmaxf(fabsf(y[0].x), fabsf(y[0].y));
 #pragma unroll
-        for (int i = 0; i < 32; i++) a = fmaxf(a, fabsf(y[i]));
+        for (int i = 1; i < 32; i++) a = max3(a, fabsf(y[i].x), fabsf(y[i].y));
         a = row_max<LANES>(a);
         const __half shh = __float2half_ru(__fdiv_rn(a, 127.0f));
         const float sf = __half2float(shh);
         const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
         if (want_desc) amax = a;
-        uint32_t w[8];
+        const float2 inv2 = make_float2(inv, inv), s2 = make_float2(sf, sf), z2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int m = 0; m < 8; m++) {
-            uint32_t cw[4];
+        for (int c = 0; c < 4; c++) {
+            uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 4; e++) {
-                const float yi = y[4 * m + e];
-                cw[e] = round_code(__fmul_rn(yi, inv), -127.0f, 127.0f);
+            for (int m = 0; m < 4; m++) {
+                uint32_t cw[4];
+                quant_pair(y[8 * c + 2 * m], z2, inv2, -127.0f, 127.0f, cw[0], cw[1]);
+                quant_pair(y[8 * c + 2 * m + 1], z2, inv2, -127.0f, 127.0f, cw[2], cw[3]);
                 if (want_desc) {
-                    const float yhat = __fmul_rn(code_value(cw[e]), sf);
-                    emax = fmaxf(emax, fabsf(__fsub_rn(yi, yhat)));
+                    float unused = 0.0f;
+                    pair_err(y[8 * c + 2 * m], cw[0], cw[1], s2, z2, emax, unused);
+                    pair_err(y[8 * c + 2 * m + 1], cw[2], cw[3], s2, z2, emax, unused);
                 }
+                w[m] = pack4bytes(cw[0], cw[1], cw[2], cw[3]);
             }
-            w[m] = pack4bytes(cw[0], cw[1], cw[2], cw[3]);
+            if (active) *reinterpret_cast<uint4 *>(codes + ((4 * s + c) * 16 + tok) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        if (active) {
-            *reinterpret_cast<uint4 *>(codes + ((2 * s) * 16 + tok) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<uint4 *>(codes + ((2 * s + 1) * 16 + tok) * 16) = make_uint4(w[4], w[5], w[6], w[7]);
-            if (s == 0) *reinterpret_cast<uint16_t *>(meta) = __half_as_ushort(shh);
-        }
+        if (active && s == 0) *reinterpret_cast<uint16_t *>(meta) = __half_as_ushort(shh);
     }
     if (want_desc) {
         emax = row_max<LANES>(emax);
@@ -244,7 +288,7 @@ __device__ __forceinline__ void slice_row(const AppendParams &p, const uint32_t 
 template <int D, int KF, int VF>
 __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ AppendParams p)
 {
-    constexpr int LANES = D / 32;
+    constexpr int LANES = D / 64;
     __shared__ uint32_t sign_xor[kMaxD / 2];
     if (threadIdx.x < D / 2) sign_xor[threadIdx.x] = p.sign_xor[threadIdx.x];
     __syncthreads();
@@ -252,17 +296,18 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
     // K rows take the first k_threads threads, V rows start on the next warp
     // boundary: every warp runs one format path, so the full-warp shuffles
     // below are always executed by all 32 lanes together
-    const long long rows_per_tensor = (long long)p.n_tok * p.L.hkv;
-    const long long k_threads = (rows_per_tensor * LANES + 31) / 32 * 32;
-    const long long gthread = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const unsigned rows_per_tensor = (unsigned)p.n_tok * (unsigned)p.L.hkv;
+    const unsigned k_threads = (rows_per_tensor * LANES + 31u) / 32u * 32u;
+    const unsigned gthread = blockIdx.x * blockDim.x + threadIdx.x;
     const int tensor = gthread >= k_threads;
-    const long long row = (gthread - tensor * k_threads) / LANES;
+    const unsigned row = (gthread - (tensor ? k_threads : 0u)) / LANES;
     const int s = (int)(gthread % LANES);
     // lanes past the last row still run the butterflies (partners stay inside
     // the row's lane group) but store nothing
     bool active = row < rows_per_tensor;
-    const long long rem = active ? row : 0;
-    const int n = (int)(rem / p.L.hkv), kvh = (int)(rem % p.L.hkv);
+    const unsigned rem = active ? row : 0u;
+    const unsigned hkv = (unsigned)p.L.hkv;
+    const int n = (int)(rem / hkv), kvh = (int)(rem - (unsigned)n * hkv);
     const int slot = p.slots[n];
     if (slot < 0) active = false;
     if (active && slot >= p.L.num_pages * kPageTokens) {
@@ -274,9 +319,9 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
     unsigned int *desc =
         p.L.desc_off ? reinterpret_cast<unsigned int *>(p.pool + p.L.desc_off + ((long long)page * p.L.hkv + kvh) * 16)
                      : nullptr;
-    const __half *src = (tensor ? p.v : p.k) + rem * D;
-    if (tensor == 0) slice_row<D, KF>(p, sign_xor, src, chunk, tok, 0, s, active, desc);
-    else slice_row<D, VF>(p, sign_xor, src, chunk, tok, 1, s, active, desc);
+    const __half *src = (tensor ? p.v : p.k) + (long long)rem * D;
+    if (tensor == 0) half_row<D, KF>(p, sign_xor, src, chunk, tok, 0, s, active, desc);
+    else half_row<D, VF>(p, sign_xor, src, chunk, tok, 1, s, active, desc);
 }
 
 template <int D, int KF>
@@ -306,7 +351,8 @@ cudaError_t launch_append(const AppendParams &p, int, int, cudaStream_t st)
 {
     const long long rows_per_tensor = (long long)p.n_tok * p.L.hkv;
     if (rows_per_tensor == 0) return cudaSuccess;
-    const long long threads = 2 * ((rows_per_tensor * (p.L.d / 32) + 31) / 32 * 32);
+    const long long threads = 2 * ((rows_per_tensor * (p.L.d / 64) + 31) / 32 * 32);
+    if (threads > 0xFFFFFFFFll) return cudaErrorInvalidValue;  // 32-bit thread indexing
     const dim3 grid((unsigned)((threads + 255) / 256));
     return p.L.d == 64 ? launch_d<64>(p, grid, st) : launch_d<128>(p, grid, st);
 }

@@ -193,3 +193,35 @@ def page_table(wl: Workload, extra_tokens: int = 0, copies: int = 1, shuffle: bo
             pos += n
         out.append(Pages(total, bt, [n * PAGE_TOKENS for n in need]))
     return out
+
+
+# --- device-side draws for timing runs --------------------------------------
+
+def prefix_kv_device(wl: Workload, b: int, device):
+    """fp16 K, V [ctx_b, Hkv, d] of sequence b drawn on the device with the
+    same recipe as prefix_kv (same distributions and outlier channels, a
+    torch generator instead of numpy's streams, so not the same numbers).
+    For timing runs whose inputs are too large to draw on the host quickly;
+    parity tests use prefix_kv."""
+    import torch
+    T = wl.ctx[b]
+    shape = (T, wl.Hkv, wl.d)
+    out = []
+    for tensor, stream in ((0, _S_K), (1, _S_V)):
+        gen = torch.Generator(device=device)
+        gen.manual_seed((wl.seed * 1000003 + stream * 1009 + b) & 0x7FFFFFFFFFFFFFFF)
+        if wl.dist == "laplace":
+            u = torch.rand(shape, generator=gen, device=device, dtype=torch.float32) - 0.5
+            x = -torch.sign(u) * torch.log1p(-2.0 * u.abs())
+            mask = torch.rand(shape, generator=gen, device=device) < 0.01
+            x = torch.where(mask, x * 30.0, x)
+        elif wl.dist == "tiny" or tensor == 0:
+            x = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+            n, factor = (2, 20.0) if wl.dist == "tiny" else (4, 15.0)
+            ch = torch.from_numpy(_outlier_channels(wl, n)).to(device)
+            for h in range(wl.Hkv):
+                x[:, h, ch[h]] *= factor
+        else:
+            x = torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * 0.5
+        out.append(x.to(torch.float16))
+    return out[0], out[1]
