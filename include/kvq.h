@@ -139,9 +139,9 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int32_t batch, int32_t
  *   ctx_lens:    int32 [batch] (device), 0 <= ctx_lens[b] <= 16*max_pages_per_seq
  *   softmax_scale: <= 0 means 1/sqrt(d)
  *   tier2:       NULL, or the certified-mode store (needs bound_block_tokens
- *                and a block count 16*max_pages_per_seq/bound_block_tokens of
- *                at most 16384, else KVQ_ERR_UNSUPPORTED; promote_frac in
- *                [0, 1]).  The quantised decode then records per-page
+ *                of 16 * 2^k tokens, at most 512, and a block count
+ *                16*max_pages_per_seq/bound_block_tokens of at most 16384,
+ *                else KVQ_ERR_UNSUPPORTED; promote_frac in [0, 1]).  The quantised decode then records per-page
  *                softmax statistics; per (sequence, kv head) a bound is formed
  *                for every block [Methodology 2: a key term from the score
  *                perturbation, a value term from the value error, weighted by

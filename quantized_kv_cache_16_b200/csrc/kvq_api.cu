@@ -107,11 +107,14 @@ int promote_count(float frac, int n_blocks)
     return k < 0 ? 0 : (k > n_blocks ? n_blocks : k);
 }
 
+// Page chunks of the certified blocks kernel (256 pages each).
+size_t cert_chunks(int max_pages) { return ((size_t)max_pages + 255) / 256; }
+
 // Certified-mode workspace, after the decode partials: page statistics,
 // per-head totals, promoted-block lists and counts, promote partials and
 // the promote counters (zero between calls).
 struct CertWs {
-    size_t page_stats, head_ml, prom, prom_count, cpart, ccount, bytes;
+    size_t page_stats, head_ml, blk, spart, dq, prom, prom_count, cpart, ccount, bytes;
 };
 
 CertWs cert_ws(const kvq_cache *c, int batch, int max_pages)
@@ -125,6 +128,12 @@ CertWs cert_ws(const kvq_cache *c, int batch, int max_pages)
     off += round256(bk * max_pages * g * 8);
     w.head_ml = off;
     off += round256(bk * g * 8);
+    w.blk = off;
+    off += round256(bk * cap * 12 * 4);
+    w.spart = off;
+    off += round256(bk * g * cert_chunks(max_pages) * 4);
+    w.dq = off;
+    off += round256(bk * g * 4);
     w.prom = off;
     off += round256(bk * cap * 4);
     w.prom_count = off;
@@ -234,7 +243,7 @@ kvq_status kvq_append(kvq_cache *c, const void *k, const void *v, const int32_t 
     p.rotate = c->cfg.rotate;
     memcpy(p.sign_xor, c->sign_xor, sizeof(p.sign_xor));
     c->last_stream = stream;
-    return cuda_status(launch_append(p, c->cfg.k_group, c->cfg.v_group, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_append(p, c->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
 kvq_status kvq_reset_pages(kvq_cache *c, const int32_t *page_ids, int32_t n, void *stream)
@@ -276,6 +285,8 @@ kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const
         if (!(tier2->promote_frac >= 0.0f && tier2->promote_frac <= 1.0f)) return KVQ_ERR_INVALID_ARG;
         const int nb_max = cert_blocks(c, max_pages_per_seq);
         if (nb_max > kCertMaxBlocks) return KVQ_ERR_UNSUPPORTED;
+        const int ppb = c->L.bound_block / kPageTokens;  // pages per block: a power of two <= 32
+        if (ppb > 32 || (ppb & (ppb - 1))) return KVQ_ERR_UNSUPPORTED;
         kmax = promote_count(tier2->promote_frac, nb_max);
         if (kmax > 0) {
             k2 = device_view(tier2->k_host);
@@ -314,7 +325,10 @@ kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const
     unsigned char *cert_base = static_cast<unsigned char *>(workspace) + counters_bytes(batch, c->L.hkv) +
                                round256((size_t)batch * c->L.hkv * s.n_splits * c->L.g * (c->L.d + 4) * 4);
     const CertWs w = cert_ws(c, batch, max_pages_per_seq);
-    if (kmax > 0) p.page_stats = reinterpret_cast<float2 *>(cert_base + w.page_stats);
+    if (kmax > 0) {
+        p.page_stats = reinterpret_cast<float2 *>(cert_base + w.page_stats);
+        p.head_ml = reinterpret_cast<float2 *>(cert_base + w.head_ml);
+    }
     kvq_status rc = cuda_status(launch_decode(p, grid, st));
     if (rc != KVQ_OK || kmax == 0) return rc;
 
@@ -335,7 +349,11 @@ kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const
     cp.kmax_out = kmax;
     cp.n_chunks = kmax < kCertChunks ? kmax : kCertChunks;
     cp.page_stats = p.page_stats;
-    cp.head_ml = reinterpret_cast<float2 *>(cert_base + w.head_ml);
+    cp.head_ml = p.head_ml;
+    cp.blk = reinterpret_cast<float *>(cert_base + w.blk);
+    cp.spart = reinterpret_cast<float *>(cert_base + w.spart);
+    cp.dq = reinterpret_cast<float *>(cert_base + w.dq);
+    cp.n_chunk_cap = (int)cert_chunks(max_pages_per_seq);
     cp.prom = reinterpret_cast<int32_t *>(cert_base + w.prom);
     cp.prom_count = reinterpret_cast<int32_t *>(cert_base + w.prom_count);
     cp.promoted_out = promoted_out;

@@ -24,6 +24,7 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer (ties to even)
+constexpr unsigned long long kAppendWaitNs = 1000000000ull;  // 1 s per bounded wait
 
 __device__ __forceinline__ float code_value(uint32_t cw) { return __fsub_rn(__uint_as_float(cw), kRoundMagic); }
 
@@ -65,16 +66,15 @@ __device__ __forceinline__ void quant_pair(float2 y, float2 z2, float2 inv2, flo
     c1 = __float_as_uint(t.y);
 }
 
+// min / max over the row's lanes (lane and lane ^ 16 for d = 128)
 template <int LANES> __device__ __forceinline__ float row_min(float v)
 {
-#pragma unroll
-    for (int m = 1; m < LANES; m <<= 1) v = fminf(v, __shfl_xor_sync(kFull, v, m));
+    if constexpr (LANES == 2) v = fminf(v, __shfl_xor_sync(kFull, v, 16));
     return v;
 }
 template <int LANES> __device__ __forceinline__ float row_max(float v)
 {
-#pragma unroll
-    for (int m = 1; m < LANES; m <<= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, m));
+    if constexpr (LANES == 2) v = fmaxf(v, __shfl_xor_sync(kFull, v, 16));
     return v;
 }
 
@@ -104,19 +104,20 @@ __device__ __forceinline__ void pair_err(float2 y, uint32_t c0, uint32_t c1, flo
 }
 
 template <int D, int FMT>
-__device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *sign_xor, const __half *src,
+__device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *sign_xor, const unsigned char *src,
                                          unsigned char *chunk, int tok, int tensor, int s, bool active,
                                          unsigned int *desc)
 {
     constexpr int LANES = D / 64;
+    constexpr unsigned PARTNER = 16;  // the row's other lane (d = 128)
     const Layout &L = p.L;
-    // ---- load 64 fp16, flip signs (exact), widen to 32 pairs ----
+    // ---- 64 fp16 from the staged row (shared memory), flip signs (exact), widen to 32 pairs ----
     float2 y[32];
     {
-        const uint4 *s4 = reinterpret_cast<const uint4 *>(src + 64 * s);
+        const uint4 *s4 = reinterpret_cast<const uint4 *>(src + 128 * s);
         uint4 w[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) w[i] = active ? __ldg(s4 + i) : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 8; i++) w[i] = s4[i];
 #pragma unroll
         for (int i = 0; i < 8; i++) {
             uint32_t ww[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
@@ -150,7 +151,8 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
             const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
             for (int i = 0; i < 32; i++) {
-                const float2 o = make_float2(__shfl_xor_sync(kFull, y[i].x, 1), __shfl_xor_sync(kFull, y[i].y, 1));
+                const float2 o = make_float2(__shfl_xor_sync(kFull, y[i].x, PARTNER),
+                                             __shfl_xor_sync(kFull, y[i].y, PARTNER));
                 y[i] = __ffma2_rn(sg2, y[i], o);
             }
         }
@@ -285,76 +287,156 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
     }
 }
 
+// Rows are processed in groups of 32/LANES consecutive rows of one tensor per
+// warp (16 rows for d = 128).  Each group is staged in shared memory by one
+// bulk copy per row (whole 256-byte rows: full DRAM sectors), double-buffered
+// so the next group streams in while this one is computed; rows sit at a
+// stride of 2d+16 bytes and lane (row = lane & 15, half = lane >> 4) reads its
+// half-row with conflict-free 16-byte loads.  Persistent grid: each warp
+// takes groups g, g + all warps, ...
+constexpr int kAppendWarps = 8;
+
+template <int D> struct AppendSmem {
+    static constexpr int LANES = D / 64;
+    static constexpr int ROWS = 32 / LANES;       // rows per group
+    static constexpr int ROW_BYTES = 2 * D;
+    static constexpr int STRIDE = ROW_BYTES + 16;
+    static constexpr int BUF = ROWS * STRIDE;
+    static constexpr int BYTES = kAppendWarps * 2 * BUF + kAppendWarps * 2 * 8;  // buffers + mbarriers
+};
+
 template <int D, int KF, int VF>
-__global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ AppendParams p)
+__global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(const __grid_constant__ AppendParams p)
 {
-    constexpr int LANES = D / 64;
+    using S = AppendSmem<D>;
+    constexpr int LANES = S::LANES, ROWS = S::ROWS;
     __shared__ uint32_t sign_xor[kMaxD / 2];
+    extern __shared__ __align__(128) unsigned char smem[];
     if (threadIdx.x < D / 2) sign_xor[threadIdx.x] = p.sign_xor[threadIdx.x];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = lane % ROWS, s = lane / ROWS;  // row in the group, half of the row
+    unsigned char *buf0 = smem + warp * 2 * S::BUF;
+    const uint32_t bar0 = smem_u32(smem + kAppendWarps * 2 * S::BUF) + warp * 16;
+    if (lane == 0) {
+        mbar_init(bar0, 1);
+        mbar_init(bar0 + 8, 1);
+        fence_mbar_init();
+    }
     __syncthreads();
 
-    // K rows take the first k_threads threads, V rows start on the next warp
-    // boundary: every warp runs one format path, so the full-warp shuffles
-    // below are always executed by all 32 lanes together
-    const unsigned rows_per_tensor = (unsigned)p.n_tok * (unsigned)p.L.hkv;
-    const unsigned k_threads = (rows_per_tensor * LANES + 31u) / 32u * 32u;
-    const unsigned gthread = blockIdx.x * blockDim.x + threadIdx.x;
-    const int tensor = gthread >= k_threads;
-    const unsigned row = (gthread - (tensor ? k_threads : 0u)) / LANES;
-    const int s = (int)(gthread % LANES);
-    // lanes past the last row still run the butterflies (partners stay inside
-    // the row's lane group) but store nothing
-    bool active = row < rows_per_tensor;
-    const unsigned rem = active ? row : 0u;
-    const unsigned hkv = (unsigned)p.L.hkv;
-    const int n = (int)(rem / hkv), kvh = (int)(rem - (unsigned)n * hkv);
-    const int slot = p.slots[n];
-    if (slot < 0) active = false;
-    if (active && slot >= p.L.num_pages * kPageTokens) {
-        if (s == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
-        active = false;
+    const int rows_per_tensor = p.n_tok * p.L.hkv;
+    const int groups_per_tensor = (rows_per_tensor + ROWS - 1) / ROWS;
+    const int n_groups = 2 * groups_per_tensor;
+    const int stride = gridDim.x * kAppendWarps;
+    const int g0 = blockIdx.x * kAppendWarps + warp;
+
+    // start the copies of group gi into buffer bsel (lanes 0..ROWS-1 one row each)
+    auto issue = [&](int gi, int bsel) {
+        const int tensor = gi >= groups_per_tensor;
+        const int row0 = (gi - tensor * groups_per_tensor) * ROWS;
+        const int nrows = min(ROWS, rows_per_tensor - row0);
+        const uint32_t bar = bar0 + 8 * bsel;
+        if (lane == 0) {
+            fence_proxy_async();
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+                         "r"((uint32_t)(nrows * S::ROW_BYTES))
+                         : "memory");
+        }
+        __syncwarp();
+        if (lane < nrows) {
+            const __half *src = (tensor ? p.v : p.k) + (long long)(row0 + lane) * D;
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                    smem_u32(buf0 + bsel * S::BUF + lane * S::STRIDE)),
+                "l"(src), "r"((uint32_t)S::ROW_BYTES), "r"(bar)
+                : "memory");
+        }
+    };
+
+    if (g0 < n_groups) issue(g0, 0);
+    int it = 0;
+    for (int gi = g0; gi < n_groups; gi += stride, it++) {
+        const int bsel = it & 1;
+        if (gi + stride < n_groups) issue(gi + stride, bsel ^ 1);
+        // this group's row: slot, page, chunk (independent of the staged data)
+        const int tensor = gi >= groups_per_tensor;
+        const int row = (gi - tensor * groups_per_tensor) * ROWS + r;
+        bool active = row < rows_per_tensor;
+        const int rem = active ? row : 0;
+        const int n = rem / p.L.hkv, kvh = rem - n * p.L.hkv;
+        const int slot = p.slots[n];
+        if (slot < 0) active = false;
+        if (active && slot >= p.L.num_pages * kPageTokens) {
+            if (s == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
+            active = false;
+        }
+        const int page = active ? slot / kPageTokens : 0, tok = active ? slot % kPageTokens : 0;
+        unsigned char *chunk =
+            p.pool + kHeaderBytes + (long long)page * p.L.page_bytes + (long long)kvh * p.L.chunk_bytes;
+        unsigned int *desc = p.L.desc_off ? reinterpret_cast<unsigned int *>(p.pool + p.L.desc_off +
+                                                                             ((long long)page * p.L.hkv + kvh) * 16)
+                                          : nullptr;
+        if (!mbar_wait_bounded(bar0 + 8 * bsel, (it >> 1) & 1, kAppendWaitNs)) {
+            if (lane == 0) set_status(p.pool, KVQ_ERR_TIMEOUT);
+            // the other buffer may still have copies in flight: wait for them (bounded) and stop
+            if (gi + stride < n_groups) (void)mbar_wait_bounded(bar0 + 8 * (bsel ^ 1), ((it + 1) >> 1) & 1, kAppendWaitNs);
+            break;
+        }
+        const unsigned char *src = buf0 + bsel * S::BUF + r * S::STRIDE;
+        if (tensor == 0) half_row<D, KF>(p, sign_xor, src, chunk, tok, 0, s, active, desc);
+        else half_row<D, VF>(p, sign_xor, src, chunk, tok, 1, s, active, desc);
+        __syncwarp();  // every lane is done with this buffer before it is refilled
     }
-    const int page = active ? slot / kPageTokens : 0, tok = active ? slot % kPageTokens : 0;
-    unsigned char *chunk = p.pool + kHeaderBytes + (long long)page * p.L.page_bytes + (long long)kvh * p.L.chunk_bytes;
-    unsigned int *desc =
-        p.L.desc_off ? reinterpret_cast<unsigned int *>(p.pool + p.L.desc_off + ((long long)page * p.L.hkv + kvh) * 16)
-                     : nullptr;
-    const __half *src = (tensor ? p.v : p.k) + (long long)rem * D;
-    if (tensor == 0) half_row<D, KF>(p, sign_xor, src, chunk, tok, 0, s, active, desc);
-    else half_row<D, VF>(p, sign_xor, src, chunk, tok, 1, s, active, desc);
+    (void)LANES;
 }
 
-template <int D, int KF>
-cudaError_t launch_d_k(const AppendParams &p, int vf, dim3 grid, cudaStream_t st)
+template <int D, int KF, int VF>
+cudaError_t launch_one(const AppendParams &p, int blocks, cudaStream_t st)
 {
-    switch (vf) {
-    case KVQ_INT4_ASYM: append_kernel<D, KF, KVQ_INT4_ASYM><<<grid, 256, 0, st>>>(p); break;
-    case KVQ_INT8_SYM: append_kernel<D, KF, KVQ_INT8_SYM><<<grid, 256, 0, st>>>(p); break;
-    default: append_kernel<D, KF, KVQ_INT2_ASYM><<<grid, 256, 0, st>>>(p); break;
+    static bool configured = false;
+    if (!configured) {
+        const cudaError_t e = cudaFuncSetAttribute(append_kernel<D, KF, VF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   AppendSmem<D>::BYTES);
+        if (e != cudaSuccess) return e;
+        configured = true;
     }
+    append_kernel<D, KF, VF><<<blocks, kAppendWarps * 32, AppendSmem<D>::BYTES, st>>>(p);
     return cudaGetLastError();
 }
 
+template <int D, int KF>
+cudaError_t launch_d_k(const AppendParams &p, int blocks, cudaStream_t st)
+{
+    switch (p.L.v_fmt) {
+    case KVQ_INT4_ASYM: return launch_one<D, KF, KVQ_INT4_ASYM>(p, blocks, st);
+    case KVQ_INT8_SYM: return launch_one<D, KF, KVQ_INT8_SYM>(p, blocks, st);
+    default: return launch_one<D, KF, KVQ_INT2_ASYM>(p, blocks, st);
+    }
+}
+
 template <int D>
-cudaError_t launch_d(const AppendParams &p, dim3 grid, cudaStream_t st)
+cudaError_t launch_d(const AppendParams &p, int blocks, cudaStream_t st)
 {
     switch (p.L.k_fmt) {
-    case KVQ_INT4_ASYM: return launch_d_k<D, KVQ_INT4_ASYM>(p, p.L.v_fmt, grid, st);
-    case KVQ_INT8_SYM: return launch_d_k<D, KVQ_INT8_SYM>(p, p.L.v_fmt, grid, st);
-    default: return launch_d_k<D, KVQ_INT2_ASYM>(p, p.L.v_fmt, grid, st);
+    case KVQ_INT4_ASYM: return launch_d_k<D, KVQ_INT4_ASYM>(p, blocks, st);
+    case KVQ_INT8_SYM: return launch_d_k<D, KVQ_INT8_SYM>(p, blocks, st);
+    default: return launch_d_k<D, KVQ_INT2_ASYM>(p, blocks, st);
     }
 }
 
 }  // namespace
 
-cudaError_t launch_append(const AppendParams &p, int, int, cudaStream_t st)
+cudaError_t launch_append(const AppendParams &p, int num_sms, cudaStream_t st)
 {
     const long long rows_per_tensor = (long long)p.n_tok * p.L.hkv;
     if (rows_per_tensor == 0) return cudaSuccess;
-    const long long threads = 2 * ((rows_per_tensor * (p.L.d / 64) + 31) / 32 * 32);
-    if (threads > 0xFFFFFFFFll) return cudaErrorInvalidValue;  // 32-bit thread indexing
-    const dim3 grid((unsigned)((threads + 255) / 256));
-    return p.L.d == 64 ? launch_d<64>(p, grid, st) : launch_d<128>(p, grid, st);
+    if (rows_per_tensor > (1ll << 30)) return cudaErrorInvalidValue;  // 32-bit row indexing
+    const int rows = p.L.d == 64 ? 32 : 16;
+    const long long groups = 2 * ((rows_per_tensor + rows - 1) / rows);
+    const long long want = (groups + kAppendWarps - 1) / kAppendWarps;
+    const int blocks = (int)(want < 2LL * num_sms ? want : 2LL * num_sms);  // two CTAs per SM stay resident
+    return p.L.d == 64 ? launch_d<64>(p, blocks, st) : launch_d<128>(p, blocks, st);
 }
 
 }  // namespace kvq

@@ -5,8 +5,10 @@
 // for every page and query head the pair (m, l): its running max and the sum
 // of 2^(s - m) over the page's tokens (log2 units).  Then:
 //
-//   select  (one CTA per sequence and kv head) per query head: the totals
-//           M, L of the quantised softmax, the mass P_b of every bound block,
+//   blocks  (one thread per page and query head, many CTAs) and
+//   select  (one CTA per sequence and kv head) per query head, from the
+//           totals M, L of the quantised softmax (written by the decode
+//           kernel's final merge): the mass P_b of every bound block,
 //           and with the block descriptors (eps: max key error, eta: max
 //           value error, nu: max |value|, all in the rotated domain)
 //             Delta_b = scale * ||q_r||_1 * eps_b
@@ -33,7 +35,9 @@
 namespace kvq {
 namespace {
 
-constexpr int kSelThreads = 1024;  // 32 warps: one reduction slot per lane
+constexpr int kSelThreads = 512;
+constexpr int kBlkThreads = 256;  // pages per CTA of the blocks kernel
+constexpr int kBlkRec = 12;   // block record: P[8], eps, eta, nu, pad
 constexpr int kPromWarps = 8;
 constexpr int kPromThreads = kPromWarps * 32;
 constexpr int kTokBatch = 4;       // exact rows a warp has in flight per lane
@@ -41,37 +45,6 @@ constexpr int kTokBatch = 4;       // exact rows a warp has in flight per lane
 __device__ __forceinline__ int clamp_ctx(int T, int max_pages)
 {
     return T < 0 ? 0 : (T > max_pages * kPageTokens ? max_pages * kPageTokens : T);
-}
-
-struct MaxOp {
-    __device__ float operator()(float a, float b) const { return fmaxf(a, b); }
-};
-struct SumOp {
-    __device__ double operator()(double a, double b) const { return a + b; }
-};
-
-// Reduce kMaxGqa values per thread over the whole CTA (32 warps); every
-// thread gets the results.  red: 32 * kMaxGqa elements of shared memory.
-template <typename T, typename Op>
-__device__ __forceinline__ void cta_reduce(T (&v)[kMaxGqa], T *red, Op op)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int h = 0; h < kMaxGqa; h++)
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) v[h] = op(v[h], __shfl_xor_sync(kFull, v[h], m));
-    __syncthreads();
-    if (lane == 0)
-#pragma unroll
-        for (int h = 0; h < kMaxGqa; h++) red[warp * kMaxGqa + h] = v[h];
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < kMaxGqa; h++) {
-        T x = red[lane * kMaxGqa + h];
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) x = op(x, __shfl_xor_sync(kFull, x, m));
-        v[h] = x;
-    }
 }
 
 // The rotated query row of head (b, head) in lane order: element lane*E + e.
@@ -91,131 +64,130 @@ __device__ __forceinline__ void rotated_query(const CertParams &p, int b, int he
     }
 }
 
+// Pass 1, one thread per (page, query head), pages of a bound block in
+// consecutive lanes: the page's softmax mass l 2^(m - M) / L and its
+// descriptor, reduced over the block's ppb lanes (ppb a power of two <= 32);
+// the block's first lane stores the head's mass (head 0 also the block's
+// descriptors) and P_b e^(Delta_b); the CTA's sum of those goes to spart.
 template <int D>
-__global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_constant__ CertParams p)
+__global__ void __launch_bounds__(kBlkThreads) cert_blocks_kernel(const __grid_constant__ CertParams p)
 {
     constexpr int E = D / 32;
     const Layout &L = p.L;
-    const int kvh = blockIdx.x, b = blockIdx.y;
+    const int chunk = blockIdx.x, b = blockIdx.z;
+    const int g = L.g, kvh = blockIdx.y / g, h = blockIdx.y - kvh * g;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = L.g;
-    extern __shared__ unsigned long long keys[];
-    __shared__ double red_d[32 * kMaxGqa];
-    __shared__ float red_f[32 * kMaxGqa];
-    __shared__ float qn1[kMaxGqa];
+    __shared__ float dq_s;
+    __shared__ float red[kBlkThreads / 32];
 
     const int T = clamp_ctx(p.ctx_lens[b], p.max_pages);
     const int n_pages = (T + kPageTokens - 1) / kPageTokens;
-    const int block = L.bound_block, ppb = block / kPageTokens;
-    const int nb = (T + block - 1) / block;
+    if (chunk * kBlkThreads >= n_pages) return;  // the whole CTA lies past the context
+    const int ppb = L.bound_block / kPageTokens;
     const long long bk = (long long)b * L.hkv + kvh;
-    const float2 *ps = p.page_stats + bk * p.max_pages * g;
-    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
-
-    // ||q_r||_1 of each head (rotated query, softmax scale not applied)
-    if (warp < g) {
+    if (warp == 0) {  // scale * ||q_r||_1 of this head: Delta_b = dq * eps_b
         float x[E];
-        rotated_query<D>(p, b, kvh * g + warp, lane, x);
+        rotated_query<D>(p, b, kvh * g + h, lane, x);
         float a = 0.f;
 #pragma unroll
         for (int e = 0; e < E; e++) a += fabsf(x[e]);
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) a += __shfl_xor_sync(kFull, a, m);
-        if (lane == 0) qn1[warp] = a;
+        if (lane == 0) {
+            dq_s = p.scale * a;
+            if (chunk == 0) p.dq[bk * g + h] = p.scale * a;
+        }
     }
-
-    // totals of the quantised softmax per head: M = max page max, L = sum l 2^(m - M)
-    float mh[kMaxGqa];
-#pragma unroll
-    for (int h = 0; h < kMaxGqa; h++) mh[h] = -INFINITY;
-    for (int i = tid; i < n_pages; i += kSelThreads)
-#pragma unroll
-        for (int h = 0; h < kMaxGqa; h++)
-            if (h < g) {
-                const float2 s = ps[(long long)i * g + h];
-                if (s.y > 0.f) mh[h] = fmaxf(mh[h], s.x);
-            }
-    cta_reduce(mh, red_f, MaxOp());
-    double lh[kMaxGqa];
-#pragma unroll
-    for (int h = 0; h < kMaxGqa; h++) lh[h] = 0.0;
-    for (int i = tid; i < n_pages; i += kSelThreads)
-#pragma unroll
-        for (int h = 0; h < kMaxGqa; h++)
-            if (h < g) {
-                const float2 s = ps[(long long)i * g + h];
-                if (s.y > 0.f) lh[h] += (double)s.y * exp2((double)s.x - (double)mh[h]);
-            }
-    cta_reduce(lh, red_d, SumOp());
-
-    // block descriptors (max over the block's pages) and masses P_b per head
-    auto block_desc = [&](int bb, float &eps, float &eta, float &nu) {
-        eps = eta = nu = 0.f;
-        const int p1 = min(bb * ppb + ppb, n_pages);
-        for (int i = bb * ppb; i < p1; i++) {
-            const int pg = bt[i];
-            if (pg < 0 || pg >= L.num_pages) continue;  // recorded by the decode kernel
+    const int pi = chunk * kBlkThreads + tid;
+    const float2 ml = p.head_ml[bk * g + h];
+    float P = 0.f, eps = 0.f, eta = 0.f, nu = 0.f;
+    if (pi < n_pages) {
+        const int pg = p.block_table[(long long)b * p.max_pages + pi];
+        const float2 s = p.page_stats[(bk * p.max_pages + pi) * g + h];
+        if (pg >= 0 && pg < L.num_pages) {  // others were recorded by the decode kernel
             const float4 dsc =
                 *reinterpret_cast<const float4 *>(p.pool + L.desc_off + ((long long)pg * L.hkv + kvh) * 16);
-            eps = fmaxf(eps, dsc.x);
-            eta = fmaxf(eta, dsc.y);
-            nu = fmaxf(nu, dsc.z);
+            eps = dsc.x;
+            eta = dsc.y;
+            nu = dsc.z;
         }
-    };
-    auto block_mass = [&](int bb, double (&P)[kMaxGqa]) {
-#pragma unroll
-        for (int h = 0; h < kMaxGqa; h++) P[h] = 0.0;
-        const int p1 = min(bb * ppb + ppb, n_pages);
-        for (int i = bb * ppb; i < p1; i++)
-#pragma unroll
-            for (int h = 0; h < kMaxGqa; h++)
-                if (h < g) {
-                    const float2 s = ps[(long long)i * g + h];
-                    if (s.y > 0.f) P[h] += (double)s.y * exp2((double)s.x - (double)mh[h]);
-                }
-#pragma unroll
-        for (int h = 0; h < kMaxGqa; h++) P[h] = lh[h] > 0.0 ? P[h] / lh[h] : 0.0;
-    };
-    __syncthreads();  // qn1
-    const double scale = p.scale;
-
-    // A = ln sum_b P_b e^(Delta_b) per head
-    double sh[kMaxGqa];
-#pragma unroll
-    for (int h = 0; h < kMaxGqa; h++) sh[h] = 0.0;
-    for (int bb = tid; bb < nb; bb += kSelThreads) {
-        float eps, eta, nu;
-        block_desc(bb, eps, eta, nu);
-        double P[kMaxGqa];
-        block_mass(bb, P);
-#pragma unroll
-        for (int h = 0; h < kMaxGqa; h++)
-            if (h < g) sh[h] += P[h] * exp(scale * (double)qn1[h] * (double)eps);
+        if (s.y > 0.f && ml.y > 0.f) P = s.y * ex2(s.x - ml.x) / ml.y;
     }
-    cta_reduce(sh, red_d, SumOp());
+    for (int m = 1; m < ppb; m <<= 1) {  // uniform trip count
+        P += __shfl_xor_sync(kFull, P, m);
+        eps = fmaxf(eps, __shfl_xor_sync(kFull, eps, m));
+        eta = fmaxf(eta, __shfl_xor_sync(kFull, eta, m));
+        nu = fmaxf(nu, __shfl_xor_sync(kFull, nu, m));
+    }
+    __syncthreads();  // dq_s
+    float contrib = 0.f;
+    if (pi < n_pages && (pi & (ppb - 1)) == 0) {
+        float *rec = p.blk + (bk * p.sort_cap + pi / ppb) * kBlkRec;
+        rec[h] = P;
+        if (h == 0) {
+            rec[8] = eps;
+            rec[9] = eta;
+            rec[10] = nu;
+        }
+        contrib = P * expf(dq_s * eps);
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) contrib += __shfl_xor_sync(kFull, contrib, m);
+    if (lane == 0) red[warp] = contrib;
+    __syncthreads();
+    if (tid == 0) {
+        float sum = 0.f;
+        for (int w = 0; w < kBlkThreads / 32; w++) sum += red[w];
+        p.spart[(bk * g + h) * p.n_chunk_cap + chunk] = sum;
+    }
+}
 
-    // score of every block -> sort key (score bits, then the complement of
-    // the index so that equal scores order the lower block first)
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_constant__ CertParams p)
+{
+    const Layout &L = p.L;
+    const int kvh = blockIdx.x, b = blockIdx.y;
+    const int tid = threadIdx.x;
+    const int g = L.g;
+    extern __shared__ unsigned long long keys[];
+    __shared__ float dq[kMaxGqa];  // scale * ||q_r||_1: Delta_b = dq * eps_b
+    __shared__ float A[kMaxGqa];
+
+    const int T = clamp_ctx(p.ctx_lens[b], p.max_pages);
+    const int n_pages = (T + kPageTokens - 1) / kPageTokens;
+    const int block = L.bound_block;
+    const int nb = (T + block - 1) / block;
+    const long long bk = (long long)b * L.hkv + kvh;
+
+    // A = ln sum_b P_b e^(Delta_b) per head: the blocks kernel's chunk sums,
+    // added in a fixed order
+    const int n_chunks = (n_pages + kBlkThreads - 1) / kBlkThreads;
+    if (tid < g) {
+        float sum = 0.f;
+        for (int ch = 0; ch < n_chunks; ch++) sum += p.spart[(bk * g + tid) * p.n_chunk_cap + ch];
+        A[tid] = sum > 0.f ? logf(sum) : 0.f;
+        dq[tid] = nb > 0 ? p.dq[bk * g + tid] : 0.f;
+    }
+    __syncthreads();
+    const float *blk = p.blk + bk * (long long)p.sort_cap * kBlkRec;
+
+    // pass 2, one thread per block: score -> sort key (score bits, then the
+    // complement of the index so that equal scores order the lower block first)
     int np2 = 1;
     while (np2 < nb) np2 <<= 1;
     for (int bb = tid; bb < np2; bb += kSelThreads) {
         unsigned long long key = 0ull;
         if (bb < nb) {
-            float eps, eta, nu;
-            block_desc(bb, eps, eta, nu);
-            double P[kMaxGqa];
-            block_mass(bb, P);
-            double sc = 0.0;
+            const float *rec = blk + (long long)bb * kBlkRec;
+            const float4 p0 = *reinterpret_cast<const float4 *>(rec), p1 = *reinterpret_cast<const float4 *>(rec + 4);
+            const float4 d = *reinterpret_cast<const float4 *>(rec + 8);
+            const float P[kMaxGqa] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            float sc = 0.f;
 #pragma unroll
             for (int h = 0; h < kMaxGqa; h++)
-                if (h < g && P[h] > 0.0) {
-                    const double Db = scale * (double)qn1[h] * (double)eps;
-                    const double bound = P[h] * ((exp(Db + log(sh[h])) - 1.0) * (double)nu + (double)eta);
-                    sc = fmax(sc, bound);
-                }
-            float scf = (float)sc;
-            if (!(scf >= 0.f)) scf = 0.f;
-            key = ((unsigned long long)__float_as_uint(scf) << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)bb);
+                if (h < g && P[h] > 0.f) sc = fmaxf(sc, P[h] * fmaf(expm1f(fmaf(dq[h], d.x, A[h])), d.z, d.y));
+            if (!(sc >= 0.f)) sc = 0.f;
+            key = ((unsigned long long)__float_as_uint(sc) << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)bb);
         }
         keys[bb] = key;
     }
@@ -251,9 +223,6 @@ __global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_c
             p.promoted_out[bk * p.kmax_out + r] =
                 r < kp ? (int)(0xFFFFFFFFu - (unsigned)(keys[r] & 0xFFFFFFFFull)) : -1;
     if (tid == 0) p.prom_count[bk] = kp;
-#pragma unroll
-    for (int h = 0; h < kMaxGqa; h++)
-        if (tid == h && h < g) p.head_ml[bk * g + h] = make_float2(mh[h], (float)lh[h]);
 }
 
 // Dequantised values of channels lane*E .. lane*E+E-1 of token `tok` in a
@@ -530,6 +499,11 @@ cudaError_t launch_cert_select(const CertParams &p, int batch, cudaStream_t s)
         if (e != cudaSuccess) return e;
         configured[di] = true;
     }
+    const dim3 bgrid(p.n_chunk_cap, p.L.hkv * p.L.g, batch);
+    if (di) cert_blocks_kernel<128><<<bgrid, kBlkThreads, 0, s>>>(p);
+    else cert_blocks_kernel<64><<<bgrid, kBlkThreads, 0, s>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     const dim3 grid(p.L.hkv, batch);
     if (di) cert_select_kernel<128><<<grid, kSelThreads, smem, s>>>(p);
     else cert_select_kernel<64><<<grid, kSelThreads, smem, s>>>(p);

@@ -38,7 +38,8 @@
 namespace kvq {
 namespace {
 
-constexpr int kCombineSplits = 40;  // split records the last CTA can stage
+constexpr int kCombineSplits = 40;  // most splits per (sequence, kv head)
+constexpr int kMergeBatch = 10;     // split records a merging warp loads at once
 
 // fp16x2 constants (bit patterns)
 constexpr uint32_t kH1024 = 0x64006400u;  // (1024, 1024)
@@ -398,12 +399,9 @@ template <int KF, int VF, int D, bool G8> struct Cfg {
     static constexpr int OFF_QSUM = OFF_QV + NT * K::KQ * 8 * 32;    // f32 [8][4]
     static constexpr int OFF_QEXP = OFF_QSUM + kMaxGqa * 4 * 4;      // i32 [8]
     static constexpr int OFF_BAR = OFF_QEXP + kMaxGqa * 4;
-    // the last CTA stages up to kCombineSplits split records per head there
-    static constexpr int GM = G8 ? kMaxGqa : 4;
-    static constexpr int COMB = kCombineSplits * GM * ((D + 4) * 4 + 4) + GM * D * 4 + kMaxGqa * 4;
     static constexpr int END = OFF_BAR + kDecodeWarps * NST * 8;
-    static constexpr int OFF_FLAG = ((END > COMB ? END : COMB) + 7) / 8 * 8;
-    static constexpr int SMEM = OFF_FLAG + 16;  // flag (int) + the staging mbarrier
+    static constexpr int OFF_FLAG = (END + 7) / 8 * 8;
+    static constexpr int SMEM = OFF_FLAG + 16;  // the last-CTA flag (int)
     // merge scratch (aliases the ring after the page loop)
     static constexpr int MERGE_ACC = 0;                                         // [W][8][D]
     static constexpr int MERGE_Z = MERGE_ACC + kDecodeWarps * kMaxGqa * D * 4;    // [W][4][8]
@@ -1015,57 +1013,96 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     __threadfence();
     if (tid == 0) p.counters[b * L.hkv + kvh] = 0u;
 
-    // stage every split's partial record of this (sequence, kv head) in
-    // shared memory with one bulk copy (the records are contiguous), then
-    // merge from there: one global round trip instead of one per phase
+    // merge the splits' records straight from L2.  kDecodeWarps / g warps per
+    // head split the records between them; a warp first issues the loads of
+    // all its accumulator rows (lane l: channels l*E .. l*E+E-1), its lanes
+    // load the records' (max, sum) pairs in parallel, then the weighted sum
+    // runs from registers.  The parts meet in shared memory; warp h
+    // normalises head h, applies the inverse rotation and stores.
     constexpr int REC = D + 4;
-    const int nrec = n_active * g;
-    float *stage = reinterpret_cast<float *>(smem);
-    float *pw = stage + nrec * REC;
-    float *po = pw + nrec;
-    float *pL = po + g * D;
-    const uint32_t cbar = smem_u32(smem + C::OFF_FLAG + 8);
-    if (tid == 0) {
-        mbar_init(cbar, 1);
-        fence_mbar_init();
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        bulk_load(smem_u32(stage), part_base, (uint32_t)(nrec * REC * 4), cbar);
-    }
-    __syncthreads();
-    if (!mbar_wait_bounded(cbar, 0, kWaitLimitNs)) set_status(p.pool, KVQ_ERR_TIMEOUT);
-    // (1) warp h: the max over splits, the weights e^(m - M) and the total sum
-    for (int h = warp; h < g; h += kDecodeWarps) {
-        float M = -INFINITY;
-        for (int s = lane; s < n_active; s += 32) M = fmaxf(M, stage[(s * g + h) * REC + D]);
+    constexpr int MB = kMergeBatch;
+    const int parts = kDecodeWarps / g;  // >= 1
+    float *wacc = reinterpret_cast<float *>(smem);            // [warp][D]
+    float *wml = wacc + kDecodeWarps * D;                      // [warp][2]
+    if (warp < parts * g) {
+        const int h = warp % g, part = warp / g;
+        const int nmine = (n_active - part + parts - 1) / parts;  // records part, part + parts, ...
+        const float *rec0 = part_base + (long long)h * REC;
+        const long long rstride = (long long)parts * g * REC;     // between this warp's records
+        float M = -INFINITY, Ls = 0.f, o[E];
 #pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, m));
-        float Ls = 0.f;
-        for (int s = lane; s < n_active; s += 32) {
-            const float ms = stage[(s * g + h) * REC + D];
-            const float f = (ms == -INFINITY || M == -INFINITY) ? 0.f : ex2(ms - M);
-            pw[s * g + h] = f;
-            Ls += f * stage[(s * g + h) * REC + D + 1];
+        for (int e = 0; e < E; e++) o[e] = 0.f;
+        for (int i0 = 0; i0 < nmine; i0 += MB) {
+            const float *rb = rec0 + (part + (long long)i0 * parts) * g * REC;
+            float a[MB][E];
+#pragma unroll
+            for (int i = 0; i < MB; i++) {  // every load of the batch goes out first
+                if (i0 + i < nmine) {
+                    if constexpr (E == 4) {
+                        const float4 v = __ldcg(reinterpret_cast<const float4 *>(rb + i * rstride + lane * E));
+                        a[i][0] = v.x;
+                        a[i][1] = v.y;
+                        a[i][2] = v.z;
+                        a[i][3] = v.w;
+                    } else {
+                        const float2 v = __ldcg(reinterpret_cast<const float2 *>(rb + i * rstride + lane * E));
+                        a[i][0] = v.x;
+                        a[i][1] = v.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < E; e++) a[i][e] = 0.f;
+                }
+            }
+            // lane i: (max, sum) of record i0 + i; the running max moves to
+            // the batch's, rescaling what came before (online merge)
+            float2 ml = make_float2(-INFINITY, 0.f);
+            if (lane < MB && i0 + lane < nmine) ml = __ldcg(reinterpret_cast<const float2 *>(rb + lane * rstride + D));
+            float Mb = ml.x;
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) Mb = fmaxf(Mb, __shfl_xor_sync(kFull, Mb, m));
+            const float Mn = fmaxf(M, Mb);
+            const float sc = (M == -INFINITY) ? 0.f : ex2(M - Mn);
+            M = Mn;
+            Ls *= sc;
+#pragma unroll
+            for (int e = 0; e < E; e++) o[e] *= sc;
+            const float f = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M);
+            Ls = fmaf(f, ml.y, Ls);
+#pragma unroll
+            for (int i = 0; i < MB; i++) {
+                const float fi = __shfl_sync(kFull, f, i);
+#pragma unroll
+                for (int e = 0; e < E; e++) o[e] = fmaf(fi, a[i][e], o[e]);
+            }
         }
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) Ls += __shfl_xor_sync(kFull, Ls, m);
-        if (lane == 0) pL[h] = Ls;
-    }
-    __syncthreads();
-    // (2) weighted sum over the splits
-    for (int idx = tid; idx < g * D; idx += kDecodeThreads) {
-        const int h = idx / D, ch = idx - h * D;
-        float o = 0.f;
-        for (int s = 0; s < n_active; s++) o = fmaf(pw[s * g + h], stage[(s * g + h) * REC + ch], o);
-        po[idx] = o;
-    }
-    __syncthreads();
-    // (3) normalise, inverse rotation, store
-    for (int h = warp; h < g; h += kDecodeWarps) {
-        const float Ls = pL[h];
-        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-        float o[E];
 #pragma unroll
-        for (int e = 0; e < E; e++) o[e] = po[h * D + lane * E + e] * inv;
+        for (int e = 0; e < E; e++) wacc[warp * D + lane * E + e] = o[e];
+        if (lane == 0) {
+            wml[2 * warp] = M;
+            wml[2 * warp + 1] = Ls;
+        }
+    }
+    __syncthreads();
+    for (int h = warp; h < g; h += kDecodeWarps) {
+        float M = -INFINITY;
+        for (int pt = 0; pt < parts; pt++) M = fmaxf(M, wml[2 * (pt * g + h)]);
+        float Ls = 0.f, o[E];
+#pragma unroll
+        for (int e = 0; e < E; e++) o[e] = 0.f;
+        for (int pt = 0; pt < parts; pt++) {
+            const int w = pt * g + h;
+            const float f = (wml[2 * w] == -INFINITY) ? 0.f : ex2(wml[2 * w] - M);
+            Ls = fmaf(f, wml[2 * w + 1], Ls);
+#pragma unroll
+            for (int e = 0; e < E; e++) o[e] = fmaf(f, wacc[w * D + lane * E + e], o[e]);
+        }
+        if (lane == 0 && p.head_ml) p.head_ml[((long long)b * L.hkv + kvh) * g + h] = make_float2(M, Ls);
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+#pragma unroll
+        for (int e = 0; e < E; e++) o[e] *= inv;
         if (p.rotate) {
             fwht_warp<D>(o, lane);
 #pragma unroll

@@ -121,6 +121,7 @@ struct DecodeParams {
     // certified mode: per page and head (m, l) = (running max, sum of
     // 2^(s - m) over the page's tokens), log2 units; null = off
     float2 *page_stats;       // [B][Hkv][max_pages][g]
+    float2 *head_ml;          // [B][Hkv][g]: totals (M, L) of the softmax, certified mode only
 };
 
 struct DequantParams {
@@ -160,7 +161,11 @@ struct CertParams {
     int kmax_out;      // columns of promoted_out
     int n_chunks;      // promote CTAs per (sequence, kv head)
     const float2 *page_stats;  // [B][Hkv][max_pages][g] from the decode kernel
-    float2 *head_ml;           // [B][Hkv][g]: (M, L) of the quantised pass, log2 units
+    const float2 *head_ml;     // [B][Hkv][g]: (M, L) of the quantised pass, log2 units (decode kernel)
+    float *blk;                // [B][Hkv][sort_cap][12]: per-block masses and descriptors
+    float *spart;              // [B][Hkv][g][n_chunk_cap]: per-chunk sums of P_b e^(Delta_b)
+    float *dq;                 // [B][Hkv][g]: scale * ||q_r||_1
+    int n_chunk_cap;           // page chunks of the blocks kernel: ceil(max_pages / 256)
     int32_t *prom;             // [B][Hkv][sort_cap]: promoted blocks, highest bound first
     int32_t *prom_count;       // [B][Hkv]
     int32_t *promoted_out;     // optional [B][Hkv][kmax_out], -1 padded
@@ -172,7 +177,7 @@ struct CertParams {
 };
 
 // launchers (return cudaGetLastError() of the launch)
-cudaError_t launch_append(const AppendParams &p, int k_group, int v_group, cudaStream_t s);
+cudaError_t launch_append(const AppendParams &p, int num_sms, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, dim3 grid, cudaStream_t s);
 cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
 cudaError_t launch_reset_pages(unsigned char *pool, Layout L, const int32_t *pages, int n, cudaStream_t s);
