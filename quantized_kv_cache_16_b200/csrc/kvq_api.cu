@@ -80,7 +80,7 @@ SplitPlan plan_splits(const kvq_cache *c, int batch, int max_pages)
     return s;
 }
 
-size_t counters_bytes(int batch, int hkv) { return ((size_t)batch * hkv * 4 + 255) / 256 * 256; }
+size_t counters_bytes(int batch, int hkv) { return decode_counter_bytes(batch, hkv); }
 
 size_t round256(size_t n) { return (n + 255) / 256 * 256; }
 

@@ -517,6 +517,12 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         if constexpr (E == 4) q_raw = *reinterpret_cast<const uint2 *>(qh);
         else q_raw.x = *reinterpret_cast<const uint32_t *>(qh);
     }
+    extern __shared__ __align__(128) unsigned char smem[];
+    const uint32_t bar0 = smem_u32(smem + C::OFF_BAR) + warp * NST * 8;
+    if (lane == 0) {  // the ring's barriers, while the loads above are in flight
+        for (int s = 0; s < NST; s++) mbar_init(bar0 + 8 * s, 1);
+        fence_mbar_init();
+    }
     if (T < 0 || T > p.max_pages * kPageTokens) {
         if (split == 0 && tid == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
         T = T < 0 ? 0 : p.max_pages * kPageTokens;
@@ -525,12 +531,10 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     const int n_active = max(1, (n_pages + p.pages_per_split - 1) / p.pages_per_split);
     if (split >= n_active) return;
 
-    extern __shared__ __align__(128) unsigned char smem[];
     int8_t *qv = reinterpret_cast<int8_t *>(smem + C::OFF_QV);
     float *qsum = reinterpret_cast<float *>(smem + C::OFF_QSUM);
     int *qexp = reinterpret_cast<int *>(smem + C::OFF_QEXP);
     int *sflag = reinterpret_cast<int *>(smem + C::OFF_FLAG);
-    const uint32_t bar0 = smem_u32(smem + C::OFF_BAR) + warp * NST * 8;
     const uint32_t stage0 = smem_u32(smem) + warp * NST * C::STAGE;
     const unsigned char *stage0_ptr = smem + warp * NST * C::STAGE;
 
@@ -539,10 +543,6 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     const int p_end = min(p_begin + p.pages_per_warp, n_pages);
     const int npg = max(0, p_end - p_begin);
     const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
-    if (lane == 0) {
-        for (int s = 0; s < NST; s++) mbar_init(bar0 + 8 * s, 1);
-        fence_mbar_init();
-    }
     __syncwarp();
 
     auto fetch_ids = [&](int i0) -> int {
@@ -570,12 +570,14 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         const int pg = __shfl_sync(kFull, ids, i & 31);
         const int st = i % NST;
         vbits = (vbits & ~(1u << st)) | ((pg >= 0 ? 1u : 0u) << st);
+        // (a stage was last read by this warp's ldmatrix loads, complete before
+        // the __syncwarp that precedes every refill; no generic-proxy write to
+        // the ring precedes the copy, so no proxy fence)
         if (lane == 0) {
-            fence_proxy_async();
             if (pg >= 0)
                 bulk_load(stage0 + st * C::STAGE, kv_base + (long long)pg * L.page_bytes, C::CHUNK, bar0 + 8 * st);
             else
-                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar0 + 8 * st) : "memory");
+                asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar0 + 8 * st) : "memory");
         }
     };
     // fused append: the warp that owns the page of position T-1 quantises
@@ -1004,13 +1006,17 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     // ---- last CTA of this (sequence, kv head) merges the splits ----
     __syncthreads();
     if (tid == 0) {
-        __threadfence();
-        const unsigned prev = atomicAdd(p.counters + (b * L.hkv + kvh), 1u);
+        // release: this CTA's record (ordered by the barrier above) is visible
+        // before the count; acquire: the last CTA then sees every record
+        unsigned prev;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                     : "=r"(prev)
+                     : "l"(p.counters + (b * L.hkv + kvh))
+                     : "memory");
         *sflag = (prev == (unsigned)(n_active - 1));
     }
     __syncthreads();
     if (!*sflag) return;
-    __threadfence();
     if (tid == 0) p.counters[b * L.hkv + kvh] = 0u;
 
     // merge the splits' records straight from L2.  kDecodeWarps / g warps per

@@ -111,7 +111,7 @@ struct DecodeParams {
     int pages_per_warp;
     int n_splits;
     float *part;              // [B][Hkv][n_splits][g][d + 4]
-    unsigned int *counters;   // [B][Hkv]
+    unsigned int *counters;   // [B][Hkv] finished CTAs, zero between calls
     float *out;
     // fused append of one token per sequence before attending (null = off)
     const __half *new_k;      // [B][Hkv][d]
@@ -186,6 +186,13 @@ cudaError_t launch_cert_promote(const CertParams &p, int batch, cudaStream_t s);
 bool decode_supported(const Layout &L);
 int decode_max_splits(const Layout &L);
 constexpr int kDecodeWarps = 8;
+
+// Decode workspace head: the finished-CTA counters [B][Hkv], rounded to 256
+// bytes.  Zero before the first call; every call leaves them zero.
+inline size_t decode_counter_bytes(int batch, int hkv)
+{
+    return ((size_t)batch * hkv * 4 + 255) / 256 * 256;
+}
 constexpr int kDecodeThreads = kDecodeWarps * 32;
 
 // ------------------------------------------------------------- device util ---
@@ -218,9 +225,14 @@ __device__ __forceinline__ void fence_proxy_async()
 
 // Arm the barrier for `bytes` and start a bulk global->shared copy that
 // completes the transaction on it.  src/dst 16-byte aligned, bytes % 16 == 0.
+// The arrive is relaxed: the copy's completion publishes the data to the
+// waiting consumer, and the issuing thread has nothing of its own to publish,
+// so its earlier memory operations (e.g. an atomic in flight) need not finish
+// first.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
 {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+    asm volatile("mbarrier.arrive.expect_tx.relaxed.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
         "l"(src), "r"(bytes), "r"(bar)

@@ -6,6 +6,8 @@
 
 #include "kvq_internal.cuh"
 
+using kvq::decode_counter_bytes;
+
 namespace {
 
 // Decode workspace (split counters + split partials) for every call of
@@ -52,8 +54,8 @@ extern "C" kvq_status kvq_decode_attn_static(kvq_cache *c, const void *q, const 
     void *ws = nullptr;
     const kvq_status st = scratch_for_current_device(&ws);
     if (st != KVQ_OK) return st;
-    // the split counters must start at zero; the partials need no clearing
-    const size_t counters = ((size_t)batch * c->L.hkv * 4 + 255) / 256 * 256;
+    // the counters must start at zero; the partials need no clearing
+    const size_t counters = decode_counter_bytes(batch, c->L.hkv);
     if (cudaMemsetAsync(ws, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess) return KVQ_ERR_CUDA;
     return kvq_decode_attn(c, q, block_table, max_pages_per_seq, ctx_lens, batch, softmax_scale, nullptr, ws,
                            kStaticScratchBytes, out, nullptr, stream);
