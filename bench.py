@@ -87,6 +87,7 @@ class Dist:
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.device = "cpu"
 
     def init(self, backend):
         if self.world > 1:
@@ -94,6 +95,7 @@ class Dist:
             import torch.distributed as td
             td.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
             self.pg = True
+            self.device = "cuda" if backend == "nccl" else "cpu"
 
     def barrier(self):
         if self.pg:
@@ -105,7 +107,7 @@ class Dist:
             return x
         import torch
         import torch.distributed as td
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
         td.all_reduce(t, op=td.ReduceOp.MAX)
         return float(t.item())
 

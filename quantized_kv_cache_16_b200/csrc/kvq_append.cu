@@ -78,17 +78,27 @@ template <int LANES> __device__ __forceinline__ float row_max(float v)
     return v;
 }
 
-// min and max of y[i0 .. i0+n) (pairs), 3-input min/max
+// min and max of the N pairs y[0 .. N), 3-input min/max in four independent
+// chains (short dependency chains; min/max are exact in any order)
 template <int N>
 __device__ __forceinline__ void pair_minmax(const float2 *y, float &lo, float &hi)
 {
-    lo = fminf(y[0].x, y[0].y);
-    hi = fmaxf(y[0].x, y[0].y);
+    static_assert(N % 4 == 0, "four chains");
+    float l[4], h[4];
 #pragma unroll
-    for (int i = 1; i < N; i++) {
-        lo = min3(lo, y[i].x, y[i].y);
-        hi = max3(hi, y[i].x, y[i].y);
+    for (int c = 0; c < 4; c++) {
+        l[c] = fminf(y[c].x, y[c].y);
+        h[c] = fmaxf(y[c].x, y[c].y);
     }
+#pragma unroll
+    for (int i = 4; i < N; i += 4)
+#pragma unroll
+        for (int c = 0; c < 4; c++) {
+            l[c] = min3(l[c], y[i + c].x, y[i + c].y);
+            h[c] = max3(h[c], y[i + c].x, y[i + c].y);
+        }
+    lo = fminf(min3(l[0], l[1], l[2]), l[3]);
+    hi = fmaxf(max3(h[0], h[1], h[2]), h[3]);
 }
 
 // Dequantisation error and magnitude of a pair (descriptors): the stored
@@ -118,15 +128,19 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
         uint4 w[8];
 #pragma unroll
         for (int i = 0; i < 8; i++) w[i] = s4[i];
+        const uint4 *sx4 = reinterpret_cast<const uint4 *>(sign_xor + 32 * s);
 #pragma unroll
         for (int i = 0; i < 8; i++) {
             uint32_t ww[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
-#pragma unroll
-            for (int e = 0; e < 4; e++) {
-                uint32_t x = ww[e];
-                if (p.rotate) x ^= sign_xor[32 * s + 4 * i + e];
-                y[4 * i + e] = __half22float2(bits_h2(x));
+            if (p.rotate) {
+                const uint4 m = sx4[i];
+                ww[0] ^= m.x;
+                ww[1] ^= m.y;
+                ww[2] ^= m.z;
+                ww[3] ^= m.w;
             }
+#pragma unroll
+            for (int e = 0; e < 4; e++) y[4 * i + e] = __half22float2(bits_h2(ww[e]));
         }
     }
     // ---- butterflies: h = 1 inside a pair, h = 2..32 across pairs, h = 64 across lanes ----
@@ -244,9 +258,14 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
         }
     } else {
         // symmetric int8, one fp16 scale (rounded up) per row; 64 bytes per lane
-        float a = fmaxf(fabsf(y[0].x), fabsf(y[0].y));
+        float am[4];
 #pragma unroll
-        for (int i = 1; i < 32; i++) a = max3(a, fabsf(y[i].x), fabsf(y[i].y));
+        for (int c = 0; c < 4; c++) am[c] = fmaxf(fabsf(y[c].x), fabsf(y[c].y));
+#pragma unroll
+        for (int i = 4; i < 32; i += 4)
+#pragma unroll
+            for (int c = 0; c < 4; c++) am[c] = max3(am[c], fabsf(y[i + c].x), fabsf(y[i + c].y));
+        float a = fmaxf(max3(am[0], am[1], am[2]), am[3]);
         a = row_max<LANES>(a);
         const __half shh = __float2half_ru(__fdiv_rn(a, 127.0f));
         const float sf = __half2float(shh);
@@ -310,7 +329,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(const __grid_
 {
     using S = AppendSmem<D>;
     constexpr int LANES = S::LANES, ROWS = S::ROWS;
-    __shared__ uint32_t sign_xor[kMaxD / 2];
+    __shared__ __align__(16) uint32_t sign_xor[kMaxD / 2];
     extern __shared__ __align__(128) unsigned char smem[];
     if (threadIdx.x < D / 2) sign_xor[threadIdx.x] = p.sign_xor[threadIdx.x];
 
@@ -329,6 +348,8 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(const __grid_
     const int groups_per_tensor = (rows_per_tensor + ROWS - 1) / ROWS;
     const int n_groups = 2 * groups_per_tensor;
     const int stride = gridDim.x * kAppendWarps;
+    const bool hkv_pow2 = (p.L.hkv & (p.L.hkv - 1)) == 0;
+    const int hkv_shift = __ffs(p.L.hkv) - 1;
     const int g0 = blockIdx.x * kAppendWarps + warp;
 
     // start the copies of group gi into buffer bsel (lanes 0..ROWS-1 one row each)
@@ -364,7 +385,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(const __grid_
         const int row = (gi - tensor * groups_per_tensor) * ROWS + r;
         bool active = row < rows_per_tensor;
         const int rem = active ? row : 0;
-        const int n = rem / p.L.hkv, kvh = rem - n * p.L.hkv;
+        const int n = hkv_pow2 ? (rem >> hkv_shift) : rem / p.L.hkv, kvh = rem - n * p.L.hkv;
         const int slot = p.slots[n];
         if (slot < 0) active = false;
         if (active && slot >= p.L.num_pages * kPageTokens) {
