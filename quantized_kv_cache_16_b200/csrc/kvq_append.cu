@@ -358,12 +358,14 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(const __grid_
         const int row0 = (gi - tensor * groups_per_tensor) * ROWS;
         const int nrows = min(ROWS, rows_per_tensor - row0);
         const uint32_t bar = bar0 + 8 * bsel;
-        if (lane == 0) {
-            fence_proxy_async();
-            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+        // relaxed arm, no proxy fence: the buffer was last read (generic
+        // loads, complete before the __syncwarp ending its group) and the
+        // copy's completion is what publishes the data; a release arrive
+        // would wait for this lane's code stores of the previous group
+        if (lane == 0)
+            asm volatile("mbarrier.arrive.expect_tx.relaxed.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
                          "r"((uint32_t)(nrows * S::ROW_BYTES))
                          : "memory");
-        }
         __syncwarp();
         if (lane < nrows) {
             const __half *src = (tensor ? p.v : p.k) + (long long)(row0 + lane) * D;

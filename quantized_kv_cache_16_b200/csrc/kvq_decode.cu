@@ -79,11 +79,37 @@ __device__ __forceinline__ uint32_t fld2(uint32_t w, int f)
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) { return h2_bits(__floats2half2_rn(lo, hi)); }
 
-// x ~= hi + lo, returned as the fp16 pair (hi, lo).
-__device__ __forceinline__ uint32_t hilo(float x)
+
+// x ~= hi + lo as the fp16 pair (hi, lo) = (fp16(x), fp16(x - hi)), for two
+// values at once (one packed conversion each way): rx for x, ry for y
+__device__ __forceinline__ void hilo_pair(float x, float y, uint32_t &rx, uint32_t &ry)
 {
-    const float hf = __half2float(__float2half_rn(x));
-    return pack_h2(x, x - hf);
+    const __half2 h = __floats2half2_rn(x, y);
+    const float2 hf = __half22float2(h);
+    const uint32_t hb = h2_bits(h), lb = h2_bits(__floats2half2_rn(x - hf.x, y - hf.y));
+    rx = __byte_perm(hb, lb, 0x5410);
+    ry = __byte_perm(hb, lb, 0x7632);
+}
+
+// NG fp16 values stored consecutively (4-byte aligned for NG >= 2) as fp32
+template <int NG>
+__device__ __forceinline__ void load_h(const unsigned char *p, float (&s)[NG])
+{
+    if constexpr (NG == 4) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p);
+        const float2 a = __half22float2(bits_h2(u.x)), b = __half22float2(bits_h2(u.y));
+        s[0] = a.x;
+        s[1] = a.y;
+        s[2] = b.x;
+        s[3] = b.y;
+    } else if constexpr (NG == 2) {
+        const float2 a = __half22float2(bits_h2(*reinterpret_cast<const uint32_t *>(p)));
+        s[0] = a.x;
+        s[1] = a.y;
+    } else {
+        static_assert(NG == 1, "1, 2 or 4 groups");
+        s[0] = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(p)));
+    }
 }
 
 __device__ __forceinline__ uint32_t movm_t(uint32_t x)
@@ -449,7 +475,6 @@ __device__ __forceinline__ void ld_vrows_t(uint32_t base, int lane, uint32_t (&w
     }
 }
 
-__device__ __forceinline__ float h2f_bits(uint16_t u) { return __half2float(__ushort_as_half(u)); }
 
 // Which (head, digit) a query-digit column holds; digit -1 = unused column.
 template <bool G8>
@@ -779,6 +804,9 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             float acc_r[NH], acc_r8[NH];
 #pragma unroll
             for (int t = 0; t < NH; t++) acc_r[t] = acc_r8[t] = 0.f;
+            float skr[KC::NG], skr8[KC::NG];  // the rows' group scales
+            load_h<KC::NG>(meta_r, skr);
+            load_h<KC::NG>(meta_r8, skr8);
 #pragma unroll
             for (int gi = 0; gi < KC::NG; gi++) {
                 int d[NT][4];
@@ -792,8 +820,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
 #pragma unroll
                     for (int nt = 0; nt < NT; nt++) imma16832(d[nt], a, qb[nt][kq][0], qb[nt][kq][1]);
                 }
-                const float sk_r = h2f_bits(*reinterpret_cast<const uint16_t *>(meta_r + 2 * gi));
-                const float sk_r8 = h2f_bits(*reinterpret_cast<const uint16_t *>(meta_r8 + 2 * gi));
+                const float sk_r = skr[gi], sk_r8 = skr8[gi];
 #pragma unroll
                 for (int t = 0; t < NH; t++) {
                     // digits of head j + 4t: (d1, d2, d3) for row r (c0/c1) and r+8 (c2/c3)
@@ -882,11 +909,8 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             const unsigned char *vmeta_r = sp + C::V_META + r * VC::ROW_META;
             const unsigned char *vmeta_r8 = sp + C::V_META + (r + 8) * VC::ROW_META;
             float sv_r[VC::NG], sv_r8[VC::NG];
-#pragma unroll
-            for (int gi = 0; gi < VC::NG; gi++) {
-                sv_r[gi] = h2f_bits(*reinterpret_cast<const uint16_t *>(vmeta_r + 2 * gi));
-                sv_r8[gi] = h2f_bits(*reinterpret_cast<const uint16_t *>(vmeta_r8 + 2 * gi));
-            }
+            load_h<VC::NG>(vmeta_r, sv_r);
+            load_h<VC::NG>(vmeta_r8, sv_r8);
             if (ragged) {
                 const bool v_r = page_ok && r < nvalid, v_r8 = page_ok && r + 8 < nvalid;
 #pragma unroll
@@ -917,13 +941,15 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
 #pragma unroll
             for (int t = 0; t < NH; t++) {
                 // p as (hi, lo) columns, transposed into B layout
-                const uint32_t bz0 = movm_t(hilo(p_r[t])), bz1 = movm_t(hilo(p_r8[t]));
-                mma16816(oz[t], az, bz0, bz1);
+                uint32_t h0, h1;
+                hilo_pair(p_r[t], p_r8[t], h0, h1);
+                mma16816(oz[t], az, movm_t(h0), movm_t(h1));
                 uint32_t wb[VC::NG][2];
 #pragma unroll
                 for (int gi = 0; gi < VC::NG; gi++) {
-                    wb[gi][0] = movm_t(hilo(p_r[t] * sv_r[gi]));
-                    wb[gi][1] = movm_t(hilo(p_r8[t] * sv_r8[gi]));
+                    hilo_pair(p_r[t] * sv_r[gi], p_r8[t] * sv_r8[gi], h0, h1);
+                    wb[gi][0] = movm_t(h0);
+                    wb[gi][1] = movm_t(h1);
                 }
 #pragma unroll
                 for (int c = 0; c < VC::NCH; c++) {
