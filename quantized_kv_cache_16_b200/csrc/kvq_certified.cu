@@ -40,7 +40,7 @@ constexpr int kBlkThreads = 256;  // pages per CTA of the blocks kernel
 constexpr int kBlkRec = 12;   // block record: P[8], eps, eta, nu, pad
 constexpr int kPromWarps = 8;
 constexpr int kPromThreads = kPromWarps * 32;
-constexpr int kTokBatch = 4;       // exact rows a warp has in flight per lane
+constexpr int kTokBatch = 8;       // tokens whose exact rows a warp has in flight
 
 __device__ __forceinline__ int clamp_ctx(int T, int max_pages)
 {
@@ -227,7 +227,9 @@ __global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_c
 
 // Dequantised values of channels lane*E .. lane*E+E-1 of token `tok` in a
 // chunk (the same arithmetic as the stored codec: code*scale + zero, one
-// rounding; int8: code*scale).
+// rounding; int8: code*scale).  The lane's codes are E*bits consecutive bits
+// of the token's stream (4, 8, 16 or 32 bits, aligned to their size, inside
+// one 16-byte chunk): one load, then shifts.
 template <int E>
 __device__ __forceinline__ void dequant_lane(const unsigned char *chunk, int codes_off, int meta_off, int row_meta,
                                              int fmt, int tok, int lane, float (&x)[E])
@@ -235,20 +237,24 @@ __device__ __forceinline__ void dequant_lane(const unsigned char *chunk, int cod
     const unsigned char *codes = chunk + codes_off;
     const uint16_t *meta = reinterpret_cast<const uint16_t *>(chunk + meta_off + tok * row_meta);
     const int bits = fmt_bits(fmt);
-    const int ng = row_meta / 4;  // asymmetric formats: scales then zeros
+    const int bit0 = lane * E * bits, byte0 = bit0 >> 3;
+    const unsigned char *src = codes + ((byte0 >> 4) * 16 + tok) * 16 + (byte0 & 15);
+    const int nbits = E * bits;
+    uint32_t w;
+    if (nbits == 32) w = *reinterpret_cast<const uint32_t *>(src);
+    else if (nbits == 16) w = *reinterpret_cast<const uint16_t *>(src);
+    else w = *src >> (bit0 & 7);
+    const uint32_t mask = (1u << bits) - 1u;
+    if (fmt == KVQ_INT8_SYM) {
+        const float s = __half2float(__ushort_as_half(meta[0]));
 #pragma unroll
-    for (int e = 0; e < E; e++) {
-        const int ch = lane * E + e;
-        const int bit = ch * bits, byte = bit >> 3;
-        const unsigned bv = codes[((byte >> 4) * 16 + tok) * 16 + (byte & 15)];
-        const int raw = (int)((bv >> (bit & 7)) & ((1u << bits) - 1u));
-        if (fmt == KVQ_INT8_SYM) {
-            x[e] = __fmul_rn((float)(int)(int8_t)raw, __half2float(__ushort_as_half(meta[0])));
-        } else {
-            const int gi = fmt == KVQ_INT4_ASYM ? ch / 32 : 0;
-            x[e] = __fmaf_rn((float)raw, __half2float(__ushort_as_half(meta[gi])),
-                             __half2float(__ushort_as_half(meta[ng + gi])));
-        }
+        for (int e = 0; e < E; e++) x[e] = __fmul_rn((float)(int)(int8_t)((w >> (8 * e)) & 0xFFu), s);
+    } else {
+        const int ng = row_meta / 4;  // asymmetric formats: scales then zeros
+        const int gi = fmt == KVQ_INT4_ASYM ? (lane * E) / 32 : 0;
+        const float s = __half2float(__ushort_as_half(meta[gi])), z = __half2float(__ushort_as_half(meta[ng + gi]));
+#pragma unroll
+        for (int e = 0; e < E; e++) x[e] = __fmaf_rn((float)((w >> (bits * e)) & mask), s, z);
     }
 }
 
@@ -264,22 +270,31 @@ __device__ __forceinline__ void online_update(float &m, float &l, float (&a)[E],
     m = mn;
 }
 
-template <int E>
-__device__ __forceinline__ void load_row(const __half *src, float (&x)[E])
-{
-    if constexpr (E == 4) {
-        const uint2 u = *reinterpret_cast<const uint2 *>(src);
+// A lane's E fp16 values of a row, kept raw (the loads stay in flight in
+// half the registers) and widened when used.
+template <int E> struct RawRow;
+template <> struct RawRow<4> {
+    uint2 u;
+    __device__ void load(const __half *src) { u = *reinterpret_cast<const uint2 *>(src); }
+    __device__ void widen(float (&x)[4]) const
+    {
         const float2 a = __half22float2(bits_h2(u.x)), c = __half22float2(bits_h2(u.y));
         x[0] = a.x;
         x[1] = a.y;
         x[2] = c.x;
         x[3] = c.y;
-    } else {
-        const float2 a = __half22float2(bits_h2(*reinterpret_cast<const uint32_t *>(src)));
+    }
+};
+template <> struct RawRow<2> {
+    uint32_t u;
+    __device__ void load(const __half *src) { u = *reinterpret_cast<const uint32_t *>(src); }
+    __device__ void widen(float (&x)[2]) const
+    {
+        const float2 a = __half22float2(bits_h2(u));
         x[0] = a.x;
         x[1] = a.y;
     }
-}
+};
 
 template <int D>
 __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid_constant__ CertParams p)
@@ -334,7 +349,7 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
         const int t0 = prom[r] * block, t1 = min(t0 + block, T);
         for (int tb = t0 + warp * kTokBatch; tb < t1; tb += kPromWarps * kTokBatch) {
             // issue the batch's exact-row loads (host link) before any math
-            float ke[kTokBatch][E], ve[kTokBatch][E];
+            RawRow<E> kraw[kTokBatch], vraw[kTokBatch];
             int pgs[kTokBatch];
 #pragma unroll
             for (int u = 0; u < kTokBatch; u++) {
@@ -347,26 +362,29 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
                 pgs[u] = pg;
                 if (pg >= 0) {
                     const long long row = ((long long)(pg * kPageTokens + t % kPageTokens) * L.hkv + kvh) * D + lane * E;
-                    load_row<E>(p.k2 + row, ke[u]);
-                    load_row<E>(p.v2 + row, ve[u]);
+                    kraw[u].load(p.k2 + row);
+                    vraw[u].load(p.v2 + row);
                 }
             }
 #pragma unroll
             for (int u = 0; u < kTokBatch; u++) {
                 if (pgs[u] < 0) continue;  // warp-uniform
                 const int tok = (tb + u) % kPageTokens;
+                float ke[E], ve[E];
+                kraw[u].widen(ke);
+                vraw[u].widen(ve);
                 if (p.rotate) {
 #pragma unroll
                     for (int e = 0; e < E; e++) {
-                        ke[u][e] *= p.signs[lane * E + e];
-                        ve[u][e] *= p.signs[lane * E + e];
+                        ke[e] *= p.signs[lane * E + e];
+                        ve[e] *= p.signs[lane * E + e];
                     }
-                    fwht_warp<D>(ke[u], lane);
-                    fwht_warp<D>(ve[u], lane);
+                    fwht_warp<D>(ke, lane);
+                    fwht_warp<D>(ve, lane);
 #pragma unroll
                     for (int e = 0; e < E; e++) {
-                        ke[u][e] *= p.rot_scale;
-                        ve[u][e] *= p.rot_scale;
+                        ke[e] *= p.rot_scale;
+                        ve[e] *= p.rot_scale;
                     }
                 }
                 const unsigned char *chunk =
@@ -380,7 +398,7 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
                     float se = 0.f, sqv = 0.f;
 #pragma unroll
                     for (int e = 0; e < E; e++) {
-                        se = fmaf(qr[h][e], ke[u][e], se);
+                        se = fmaf(qr[h][e], ke[e], se);
                         sqv = fmaf(qr[h][e], kq[e], sqv);
                     }
 #pragma unroll
@@ -388,7 +406,7 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
                         se += __shfl_xor_sync(kFull, se, mm);
                         sqv += __shfl_xor_sync(kFull, sqv, mm);
                     }
-                    online_update<E>(m[h][0], l[h][0], acc[h][0], se, ve[u]);
+                    online_update<E>(m[h][0], l[h][0], acc[h][0], se, ve);
                     online_update<E>(m[h][1], l[h][1], acc[h][1], sqv, vq);
                 }
             }
