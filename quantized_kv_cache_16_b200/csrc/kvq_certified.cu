@@ -42,6 +42,31 @@ constexpr int kPromWarps = 8;
 constexpr int kPromThreads = kPromWarps * 32;
 constexpr int kTokBatch = 8;       // tokens whose exact rows a warp has in flight
 
+// Programmatic dependent launch: wait for the stream's previous grid to
+// complete (its writes visible) before any memory access, then allow the next
+// grid to be set up; only launch latency is hidden, no work overlaps.
+__device__ __forceinline__ void pdl_enter()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename Kern>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, int threads, size_t smem, cudaStream_t s, const CertParams &p)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 __device__ __forceinline__ int clamp_ctx(int T, int max_pages)
 {
     return T < 0 ? 0 : (T > max_pages * kPageTokens ? max_pages * kPageTokens : T);
@@ -72,6 +97,7 @@ __device__ __forceinline__ void rotated_query(const CertParams &p, int b, int he
 template <int D>
 __global__ void __launch_bounds__(kBlkThreads) cert_blocks_kernel(const __grid_constant__ CertParams p)
 {
+    pdl_enter();
     constexpr int E = D / 32;
     const Layout &L = p.L;
     const int chunk = blockIdx.x, b = blockIdx.z;
@@ -145,6 +171,7 @@ __global__ void __launch_bounds__(kBlkThreads) cert_blocks_kernel(const __grid_c
 template <int D>
 __global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_constant__ CertParams p)
 {
+    pdl_enter();
     const Layout &L = p.L;
     const int kvh = blockIdx.x, b = blockIdx.y;
     const int tid = threadIdx.x;
@@ -299,6 +326,7 @@ template <> struct RawRow<2> {
 template <int D>
 __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid_constant__ CertParams p)
 {
+    pdl_enter();
     constexpr int E = D / 32;
     const Layout &L = p.L;
     const int chunk_id = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -518,14 +546,12 @@ cudaError_t launch_cert_select(const CertParams &p, int batch, cudaStream_t s)
         configured[di] = true;
     }
     const dim3 bgrid(p.n_chunk_cap, p.L.hkv * p.L.g, batch);
-    if (di) cert_blocks_kernel<128><<<bgrid, kBlkThreads, 0, s>>>(p);
-    else cert_blocks_kernel<64><<<bgrid, kBlkThreads, 0, s>>>(p);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = di ? launch_pdl(cert_blocks_kernel<128>, bgrid, kBlkThreads, 0, s, p)
+                             : launch_pdl(cert_blocks_kernel<64>, bgrid, kBlkThreads, 0, s, p);
     if (e != cudaSuccess) return e;
     const dim3 grid(p.L.hkv, batch);
-    if (di) cert_select_kernel<128><<<grid, kSelThreads, smem, s>>>(p);
-    else cert_select_kernel<64><<<grid, kSelThreads, smem, s>>>(p);
-    return cudaGetLastError();
+    return di ? launch_pdl(cert_select_kernel<128>, grid, kSelThreads, smem, s, p)
+              : launch_pdl(cert_select_kernel<64>, grid, kSelThreads, smem, s, p);
 }
 
 cudaError_t launch_cert_promote(const CertParams &p, int batch, cudaStream_t s)
@@ -542,9 +568,8 @@ cudaError_t launch_cert_promote(const CertParams &p, int batch, cudaStream_t s)
         configured[di] = true;
     }
     const dim3 grid(p.n_chunks, p.L.hkv, batch);
-    if (di) cert_promote_kernel<128><<<grid, kPromThreads, smem, s>>>(p);
-    else cert_promote_kernel<64><<<grid, kPromThreads, smem, s>>>(p);
-    return cudaGetLastError();
+    return di ? launch_pdl(cert_promote_kernel<128>, grid, kPromThreads, smem, s, p)
+              : launch_pdl(cert_promote_kernel<64>, grid, kPromThreads, smem, s, p);
 }
 
 }  // namespace kvq

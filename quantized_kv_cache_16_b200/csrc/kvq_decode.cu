@@ -524,6 +524,13 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     constexpr int NH = C::NH;
     constexpr int NT = C::NT;
 
+    // Launched as a programmatic dependent of the stream's previous kernel:
+    // wait for that grid to complete (its writes visible) before touching
+    // memory, then let the next dependent grid be set up early.  No work of
+    // this grid overlaps the previous one; only the launch latency is hidden.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
     const Layout &L = p.L;
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1160,8 +1167,17 @@ cudaError_t launch_t(const DecodeParams &p, dim3 grid, cudaStream_t s)
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    decode_kernel<D, KF, VF, G8><<<grid, kDecodeThreads, C::SMEM, s>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<D, KF, VF, G8>, p);
 }
 
 template <int D, int KF, int VF>
