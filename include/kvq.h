@@ -158,7 +158,11 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int32_t batch, int32_t
  *   promoted_out (certified mode, optional): int32 [batch][Hkv][kmax] block
  *                indices promoted, highest bound first, -1 padded, where
  *                kmax = ceil(promote_frac * ceil(16*max_pages_per_seq / block)).
- * An empty context gives a zero output row. */
+ * An empty context gives a zero output row.
+ * Kernels of this call (and of kvq_decode_step) are launched as programmatic
+ * dependents of the stream's previous kernel: each waits for that kernel to
+ * complete, with its writes visible, before touching memory, so stream order
+ * holds as for a plain launch; only the launch latency is overlapped. */
 kvq_status kvq_decode_attn(kvq_cache *cache, const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
                            const int32_t *ctx_lens, int32_t batch, float softmax_scale, const kvq_tier2 *tier2,
                            void *workspace, size_t ws_bytes, void *out, int32_t *promoted_out, void *stream);
