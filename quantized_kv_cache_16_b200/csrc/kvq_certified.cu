@@ -188,12 +188,21 @@ __global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_c
 
     // A = ln sum_b P_b e^(Delta_b) per head: the blocks kernel's chunk sums,
     // added in a fixed order
+    // (warp h: lanes over the chunks, then a fixed-order tree)
     const int n_chunks = (n_pages + kBlkThreads - 1) / kBlkThreads;
-    if (tid < g) {
-        float sum = 0.f;
-        for (int ch = 0; ch < n_chunks; ch++) sum += p.spart[(bk * g + tid) * p.n_chunk_cap + ch];
-        A[tid] = sum > 0.f ? logf(sum) : 0.f;
-        dq[tid] = nb > 0 ? p.dq[bk * g + tid] : 0.f;
+    {
+        const int warp = tid >> 5, lane = tid & 31;
+        if (warp < g) {
+            const float *sp = p.spart + (bk * g + warp) * p.n_chunk_cap;
+            float sum = 0.f;
+            for (int ch = lane; ch < n_chunks; ch += 32) sum += sp[ch];
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) sum += __shfl_xor_sync(kFull, sum, m);
+            if (lane == 0) {
+                A[warp] = sum > 0.f ? logf(sum) : 0.f;
+                dq[warp] = nb > 0 ? p.dq[bk * g + warp] : 0.f;
+            }
+        }
     }
     __syncthreads();
     const float *blk = p.blk + bk * (long long)p.sort_cap * kBlkRec;
@@ -495,17 +504,32 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
         float Mx[2] = {-INFINITY, -INFINITY}, Ls[2] = {0.f, 0.f}, a[2][E];
 #pragma unroll
         for (int w = 0; w < 2; w++) {
+            // lane c: (max, sum) of chunk c's record, loaded in parallel; the
+            // accumulator rows of every chunk go out together (unrolled)
+            float2 mlc = make_float2(-INFINITY, 0.f);
+            if (lane < n_act) mlc = __ldcg(reinterpret_cast<const float2 *>(cbase + ((lane * g + h) * 2 + w) * REC + D));
+            float M = mlc.x;
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, m));
+            Mx[w] = M;
+            const float f = (mlc.x == -INFINITY || M == -INFINITY) ? 0.f : ex2(mlc.x - M);
+            float l = f * mlc.y;
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) l += __shfl_xor_sync(kFull, l, m);
+            Ls[w] = l;
+            float rows[kCertChunks][E];
+#pragma unroll
+            for (int c = 0; c < kCertChunks; c++)
+#pragma unroll
+                for (int e = 0; e < E; e++)
+                    rows[c][e] = c < n_act ? __ldcg(cbase + ((c * g + h) * 2 + w) * REC + lane * E + e) : 0.f;
 #pragma unroll
             for (int e = 0; e < E; e++) a[w][e] = 0.f;
-            for (int c = 0; c < n_act; c++) Mx[w] = fmaxf(Mx[w], __ldcg(cbase + ((c * g + h) * 2 + w) * REC + D));
-            if (Mx[w] == -INFINITY) continue;
-            for (int c = 0; c < n_act; c++) {
-                const float *rec = cbase + ((c * g + h) * 2 + w) * REC;
-                const float mc = __ldcg(rec + D);
-                const float f = mc == -INFINITY ? 0.f : ex2(mc - Mx[w]);
-                Ls[w] = fmaf(f, __ldcg(rec + D + 1), Ls[w]);
 #pragma unroll
-                for (int e = 0; e < E; e++) a[w][e] = fmaf(f, __ldcg(rec + lane * E + e), a[w][e]);
+            for (int c = 0; c < kCertChunks; c++) {
+                const float fc = __shfl_sync(kFull, f, c);
+#pragma unroll
+                for (int e = 0; e < E; e++) a[w][e] = fmaf(fc, rows[c][e], a[w][e]);
             }
         }
         const float2 ml = p.head_ml[bk * g + h];  // the quantised pass: (M, L)
