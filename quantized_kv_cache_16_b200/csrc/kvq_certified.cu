@@ -230,21 +230,58 @@ __global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_c
     __syncthreads();
 
     // bitonic sort of the keys, descending
-    for (int k = 2; k <= np2; k <<= 1)
-        for (int jj = k >> 1; jj > 0; jj >>= 1) {
-            for (int i = tid; i < np2; i += kSelThreads) {
-                const int ixj = i ^ jj;
-                if (ixj > i) {
-                    const unsigned long long a = keys[i], c = keys[ixj];
-                    const bool desc = (i & k) == 0;
-                    if (desc ? (a < c) : (a > c)) {
-                        keys[i] = c;
-                        keys[ixj] = a;
-                    }
+    if (np2 <= 2 * kSelThreads) {
+        // keys tid and tid + kSelThreads in registers: stages whose partner is
+        // under 32 keys away are warp shuffles, the others go through shared
+        // memory (indices >= np2 only ever meet each other)
+        unsigned long long v[2];
+#pragma unroll
+        for (int c = 0; c < 2; c++) v[c] = tid + c * kSelThreads < np2 ? keys[tid + c * kSelThreads] : 0ull;
+        for (int k = 2; k <= np2; k <<= 1)
+            for (int jj = k >> 1; jj > 0; jj >>= 1) {
+                unsigned long long o[2];
+                if (jj >= 32) {
+                    __syncthreads();  // the last stage's reads are done
+#pragma unroll
+                    for (int c = 0; c < 2; c++)
+                        if (tid + c * kSelThreads < np2) keys[tid + c * kSelThreads] = v[c];
+                    __syncthreads();
+#pragma unroll
+                    for (int c = 0; c < 2; c++) o[c] = tid + c * kSelThreads < np2 ? keys[(tid + c * kSelThreads) ^ jj] : 0ull;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 2; c++) o[c] = __shfl_xor_sync(kFull, v[c], jj);
+                }
+#pragma unroll
+                for (int c = 0; c < 2; c++) {
+                    const int i = tid + c * kSelThreads;
+                    const bool lower = (i & jj) == 0, desc = (i & k) == 0;
+                    const unsigned long long hi = v[c] > o[c] ? v[c] : o[c], lo = v[c] > o[c] ? o[c] : v[c];
+                    v[c] = (lower == desc) ? hi : lo;
                 }
             }
-            __syncthreads();
-        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < 2; c++)
+            if (tid + c * kSelThreads < np2) keys[tid + c * kSelThreads] = v[c];
+        __syncthreads();
+    } else {
+        for (int k = 2; k <= np2; k <<= 1)
+            for (int jj = k >> 1; jj > 0; jj >>= 1) {
+                for (int i = tid; i < np2; i += kSelThreads) {
+                    const int ixj = i ^ jj;
+                    if (ixj > i) {
+                        const unsigned long long a = keys[i], c = keys[ixj];
+                        const bool desc = (i & k) == 0;
+                        if (desc ? (a < c) : (a > c)) {
+                            keys[i] = c;
+                            keys[ixj] = a;
+                        }
+                    }
+                }
+                __syncthreads();
+            }
+    }
 
     // the top ceil(frac * nb) blocks (fp64, guarded so an exact product is not bumped up)
     int kp = 0;

@@ -110,6 +110,14 @@ def test_certified_matches_oracle(name, wl, frac):
     _check(build_pair(wl), frac)
 
 
+def test_certified_many_blocks_sorted_in_shared_memory():
+    """1250 bound blocks of 16 tokens: more than the selection's register sort
+    holds, so the shared-memory sort runs."""
+    import dataclasses
+    wl = dataclasses.replace(W.scaled(W.certified(), [20000]), bound_block=16)
+    _check(build_pair(wl), 0.01)
+
+
 def test_certified_tier2_on_the_device():
     _check(build_pair(W.scaled(W.certified(), [1200])), 0.3, pinned=False)
 
