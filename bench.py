@@ -39,8 +39,8 @@ NOMINAL_HBM_GBS = 8000.0
 # capture summarised under profiles/ (decode_kernel_llama3-8b-layer-T32768.md).
 # Reported as roofline.traffic only while the decode kernel's sources hash to
 # the digest they had when the counters were taken; null otherwise.
-PROFILED_DECODE = {"sources_sha256": "b489770acc9e1c03901c0a4bc748519ac18bf211cc665585a7c18659f20d4c05",
-                   "dram_bytes_per_launch": 42164352}
+PROFILED_DECODE = {"sources_sha256": "6aeb408ca39736939021e873beb39d0c1d62850781346d41c57dcaf757be5ce1",
+                   "dram_bytes_per_launch": 42130176}
 DECODE_SOURCES = ("kvq_decode.cu", "kvq_internal.cuh", "kvq_warp.cuh")
 
 
