@@ -58,6 +58,26 @@ class Config(C.Structure):
     ]
 
 
+class Ladder(C.Structure):
+    """Mirror of the oracle's ladder policy."""
+
+    _fields_ = [(n, C.c_double) for n in ("tau_cov", "max_frac", "key_tol", "v_tol", "rank_tol", "cert_tol",
+                                           "layer_frac")]
+
+
+class LadderOut(C.Structure):
+    """Mirror of the oracle's ladder output pointers."""
+
+    _fields_ = [("out", C.c_void_p), ("mixed", C.c_void_p), ("dense", C.c_void_p), ("err", C.c_void_p),
+                ("bound", C.c_void_p), ("status", C.c_void_p), ("k_star", C.c_void_p), ("k_cov", C.c_void_p),
+                ("k_key", C.c_void_p), ("flags", C.c_void_p), ("rscore", C.c_void_p), ("cov", C.c_void_p),
+                ("ekey", C.c_void_p), ("max_blocks", C.c_int32)]
+
+
+LADDER_EXPANDED, LADDER_CAPPED, LADDER_VALUES = 1, 2, 4
+LADDER_RANK_FAIL, LADDER_BOUND_FAIL, LADDER_HEAD_DENSE, LADDER_LAYER_DENSE = 8, 16, 32, 64
+
+
 def make_config(num_q_heads, num_kv_heads, head_dim, k_fmt=INT4_ASYM, v_fmt=INT4_ASYM, k_group=32, v_group=32,
                 clip_ratio=1.0, rotation_seed=0, rotate=1, num_pages=1, bound_block_tokens=0) -> Config:
     return Config(num_q_heads, num_kv_heads, head_dim, k_fmt, v_fmt, k_group, v_group, clip_ratio,
@@ -101,6 +121,8 @@ def lib():
             "kvqo_decode_fp16": (i32, [cfgp, P, P, P, P, i32, P, i32, f64, P, P]),
             "kvqo_promote_count": (i32, [f64, i32]),
             "kvqo_decode_certified": (i32, [cfgp, P, P, P, P, P, i32, P, i32, f64, f64, P, P, P, i32, P, i32, P, P]),
+            "kvqo_decode_ladder": (i32, [cfgp, P, P, P, P, P, i32, P, i32, f64, C.POINTER(Ladder), P, P,
+                                         C.POINTER(LadderOut)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -326,3 +348,45 @@ def decode_certified(cfg: Config, pool: np.ndarray, k_slots, v_slots, q, block_t
     if rc != 0:
         raise ValueError(f"oracle certified decode rejected its arguments (rc={rc})")
     return out, prom, scores, bsum
+
+
+def decode_ladder(cfg: Config, pool: np.ndarray, k_slots, v_slots, q, block_table, ctx_lens, policy: dict,
+                  scale: float = 0.0, max_blocks: int = 0, forced_flags=None, forced_fallback=None) -> dict:
+    """Certified decode with the adaptive ladder.  policy: tau_cov, max_frac,
+    key_tol, v_tol, rank_tol, cert_tol, layer_frac (missing entries: the rung
+    is off -- tau 0, budget 1, tolerances inf, layer_frac 1).  Returns a dict
+    of numpy arrays: out, mixed, dense [B,Hq,d]; err, bound, status [B,Hq];
+    k_star, k_cov, k_key [B,Hkv]; flags, rscore [B,Hkv,max_blocks]; cov, ekey
+    [B,Hkv,max_blocks+1]."""
+    k = _c(k_slots, np.float16).view(np.uint16)
+    v = _c(v_slots, np.float16).view(np.uint16)
+    q = _c(q, np.float16).view(np.uint16)
+    bt = _c(block_table, np.int32)
+    cl = _c(ctx_lens, np.int32)
+    B, hq, hkv, d = cl.shape[0], cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim
+    blk = cfg.bound_block_tokens
+    mb = max_blocks or max(1, int((int(cl.max()) + blk - 1) // blk) if B else 1)
+    pol = dict(tau_cov=0.0, max_frac=1.0, key_tol=np.inf, v_tol=np.inf, rank_tol=np.inf, cert_tol=np.inf,
+               layer_frac=1.0)
+    pol.update(policy)
+    r = {
+        "out": np.zeros((B, hq, d)), "mixed": np.zeros((B, hq, d)), "dense": np.zeros((B, hq, d)),
+        "err": np.zeros((B, hq)), "bound": np.zeros((B, hq)), "status": np.zeros((B, hq), np.int32),
+        "k_star": np.zeros((B, hkv), np.int32), "k_cov": np.zeros((B, hkv), np.int32),
+        "k_key": np.zeros((B, hkv), np.int32), "flags": np.zeros((B, hkv, mb), np.uint8),
+        "rscore": np.zeros((B, hkv, mb)), "cov": np.zeros((B, hkv, mb + 1)), "ekey": np.zeros((B, hkv, mb + 1)),
+    }
+    o = LadderOut(*[r[n].ctypes.data for n in ("out", "mixed", "dense", "err", "bound", "status", "k_star", "k_cov",
+                                                "k_key", "flags", "rscore", "cov", "ekey")], mb)
+    ff = None if forced_flags is None else _c(forced_flags, np.uint8)
+    if ff is not None:
+        assert ff.shape == (B, hkv, mb)
+    fb = None if forced_fallback is None else _c(forced_fallback, np.int32)
+    if fb is not None:
+        assert fb.shape == (B, hq)
+    lp = Ladder(**{f[0]: float(pol[f[0]]) for f in Ladder._fields_})
+    rc = lib().kvqo_decode_ladder(C.byref(cfg), _p(pool), _p(k), _p(v), _p(q), _p(bt), bt.shape[1], _p(cl), B,
+                                  scale, C.byref(lp), _p(ff), _p(fb), C.byref(o))
+    if rc != 0:
+        raise ValueError(f"oracle ladder decode rejected its arguments (rc={rc})")
+    return r

@@ -874,6 +874,383 @@ int kvqo_decode_certified(const kvqo_config *c, const uint8_t *pool, const uint1
 }
 
 /* ------------------------------------------------------------------------- */
+/* Certified decode with the adaptive ladder ([CERT] Methodology 3)          */
+/* ------------------------------------------------------------------------- */
+
+/* Policy of the ladder.  Readings of [CERT] Methodology 3 ("adaptive Top-K",
+ * "ranking-consistency check", "four-rung fallback ladder"), which name the
+ * steps but print no formula:
+ *   tau_cov    coverage target of the estimated block mass (e.g. 0.995);
+ *   max_frac   budget: at most ceil(max_frac * n_blocks) key-promoted blocks;
+ *   key_tol    rung 1 target for the predicted key term (inf: rung 1 off);
+ *   v_tol      rung 2 threshold on a block's estimated value error
+ *              contribution max_h Phat_h(b) * eta_b (inf: rung 2 off);
+ *   rank_tol   relative slack rho of the ranking-consistency check (inf: off);
+ *   cert_tol   a head whose certified bound exceeds it falls back (rung 3);
+ *   layer_frac rung 4: every head of the call falls back when more than
+ *              layer_frac * B * Hq heads fall back on their own. */
+typedef struct {
+    double tau_cov, max_frac, key_tol, v_tol, rank_tol, cert_tol, layer_frac;
+} kvqo_ladder;
+
+/* Outputs (every pointer but out optional).  [B][Hq][d]: out (final), mixed
+ * (before any fallback), dense (fp16 attention).  [B][Hq]: err (measured
+ * rotated-domain inf-norm error of mixed against exact attention), bound,
+ * status (bits below).  [B][Hkv]: k_star, k_cov, k_key.  [B][Hkv][max_blocks]:
+ * flags (bit 0 key exact, bit 1 value exact), rscore (the ranking score r).
+ * [B][Hkv][max_blocks + 1]: cov (min over the group's heads of the coverage of
+ * the first K ranked blocks), ekey (max over the heads of the predicted key
+ * term with the first K ranked blocks' keys exact). */
+typedef struct {
+    double *out, *mixed, *dense, *err, *bound;
+    int32_t *status, *k_star, *k_cov, *k_key;
+    uint8_t *flags;
+    double *rscore, *cov, *ekey;
+    int32_t max_blocks;
+} kvqo_ladder_out;
+
+#define KVQO_LADDER_EXPANDED 1    /* rung 1 added blocks beyond the coverage set */
+#define KVQO_LADDER_CAPPED 2      /* the budget stopped coverage or rung 1     */
+#define KVQO_LADDER_VALUES 4      /* rung 2 promoted values in this group      */
+#define KVQO_LADDER_RANK_FAIL 8   /* ranking-consistency check failed          */
+#define KVQO_LADDER_BOUND_FAIL 16 /* certified bound above cert_tol            */
+#define KVQO_LADDER_HEAD_DENSE 32 /* rung 3: this head recomputed in fp16      */
+#define KVQO_LADDER_LAYER_DENSE 64 /* rung 4: every head recomputed in fp16    */
+
+typedef struct {
+    double r;
+    int idx;
+} kvqo_ranked;
+
+/* descending r, then ascending block index */
+static int ranked_cmp(const void *a, const void *b)
+{
+    const kvqo_ranked *x = (const kvqo_ranked *)a, *y = (const kvqo_ranked *)b;
+    if (x->r > y->r) return -1;
+    if (x->r < y->r) return 1;
+    return (x->idx > y->idx) - (x->idx < y->idx);
+}
+
+/* Block masses of a softmax over scores sc[0..T): P[b] = sum_{t in b} p_t. */
+static void block_masses(const double *sc, int T, int block, double *P)
+{
+    int nb = (T + block - 1) / block;
+    double mx = -INFINITY, L = 0.0;
+    for (int b = 0; b < nb; b++) P[b] = 0.0;
+    for (int t = 0; t < T; t++) mx = fmax(mx, sc[t]);
+    for (int t = 0; t < T; t++) L += exp(sc[t] - mx);
+    for (int t = 0; t < T; t++) P[t / block] += exp(sc[t] - mx) / L;
+}
+
+/* Key term of the bound for one head with the blocks flagged in `exact`
+ * having exact keys (their score perturbation is zero):
+ *   A = ln sum_b P_b e^{D_b},  E = sum_b P_b nu_b (e^{D_b + A} - 1),
+ * D_b = 0 for exact blocks, Delta_b otherwise.  P are the masses of the
+ * distribution the output is formed from. */
+static double key_term(const double *P, const double *Dl, const double *nu, const char *exact, int nb)
+{
+    double s = 0.0, E = 0.0;
+    for (int b = 0; b < nb; b++) s += P[b] * exp(exact[b] ? 0.0 : Dl[b]);
+    double A = s > 0.0 ? log(s) : 0.0;
+    for (int b = 0; b < nb; b++) E += P[b] * nu[b] * (exp((exact[b] ? 0.0 : Dl[b]) + A) - 1.0);
+    return E;
+}
+
+/* Certified decode with the adaptive ladder.  Per (sequence, kv head), with
+ * Phat_h(b) the block masses under the quantised scores of query head h,
+ * Delta_h(b) = scale * ||q_r,h||_1 * eps_b and eta_b, nu_b the block's value
+ * error and largest |value| (all as in kvqo_decode_certified):
+ *  1. rank the blocks by r(b) = max_h Phat_h(b), descending, ties to the
+ *     lower block index;
+ *  2. K_cov = the fewest leading blocks whose estimated mass reaches tau_cov
+ *     for every head of the group (0 if tau_cov <= 0);
+ *  3. rung 1: K_key = the fewest leading blocks whose exact keys bring the
+ *     predicted key term (key_term over Phat) of every head to key_tol or
+ *     below; K* = min(ceil(max_frac * n_blocks), max(K_cov, K_key)); the
+ *     first K* ranked blocks get their exact keys from tier 2;
+ *  4. rung 2: blocks with max_h Phat_h(b) * eta_b > v_tol get their exact
+ *     values from tier 2;
+ *  5. attention with those keys/values exact and the rest dequantised (the
+ *     mixed output);
+ *  6. ranking-consistency check per head: order the key-promoted blocks by
+ *     Phat_h; the check fails when a block placed lower has an exact mass
+ *     above (1 + rank_tol) times that of a block placed higher;
+ *  7. certified bound per head of the mixed output, from its own block masses
+ *     P': key_term(P', Delta with zeros for exact-key blocks) plus
+ *     sum over blocks with quantised values of P'(b) * eta_b.  It bounds
+ *     ||o_r,exact - o_r,mixed||_inf (the distribution the output uses is the
+ *     reference of the total-variation argument, as in the plain bound);
+ *  8. rung 3: a head falls back to fp16 attention over its tier-2 rows when
+ *     its ranking check fails or its bound exceeds cert_tol;
+ *  9. rung 4: when more than layer_frac * B * Hq heads fall back, all do.
+ * forced_flags ([B][Hkv][max_blocks], optional) replaces steps 1-4 by the
+ * given key/value flags; forced_fallback ([B][Hq], optional) replaces the
+ * decisions of steps 8-9 -- both for checking an implementation whose fp32
+ * decisions legitimately differ on a near-tie.  Returns 0, -1 (bad table or
+ * length), -2 (bad config) or -3 (a sequence has more than max_blocks). */
+int kvqo_decode_ladder(const kvqo_config *c, const uint8_t *pool, const uint16_t *k_slots, const uint16_t *v_slots,
+                       const uint16_t *q, const int32_t *block_table, int max_pages, const int32_t *ctx_lens, int B,
+                       double scale, const kvqo_ladder *pol, const uint8_t *forced_flags,
+                       const int32_t *forced_fallback, const kvqo_ladder_out *o)
+{
+    if (!kvqo_config_ok(c) || c->bound_block_tokens <= 0) return -2;
+    if (!decode_args_ok(c, block_table, max_pages, ctx_lens, B)) return -1;
+    int d = c->head_dim, hq = c->num_q_heads, hkv = c->num_kv_heads, g = hq / hkv;
+    int block = c->bound_block_tokens, MB = o->max_blocks;
+    for (int b = 0; b < B; b++)
+        if ((ctx_lens[b] + block - 1) / block > MB) return -3;
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    float s[KVQO_MAXD];
+    kvqo_signs(c->rotation_seed, d, s);
+    size_t nout = (size_t)B * hq * d;
+    double *mixed = o->mixed ? o->mixed : (double *)calloc(nout + 1, sizeof(double));
+    double *dense = o->dense ? o->dense : (double *)calloc(nout + 1, sizeof(double));
+    int32_t *fall = (int32_t *)calloc((size_t)B * hq + 1, sizeof(int32_t));
+    int32_t *stat = (int32_t *)calloc((size_t)B * hq + 1, sizeof(int32_t));
+    for (size_t i = 0; i < nout; i++) mixed[i] = 0.0;
+
+    for (int b = 0; b < B; b++) {
+        int T = ctx_lens[b];
+        int nb = (T + block - 1) / block;
+        for (int kvh = 0; kvh < hkv; kvh++) {
+            size_t n = (size_t)T * d + 1, bk = (size_t)b * hkv + kvh;
+            double *Kq = (double *)malloc(sizeof(double) * n), *Vq = (double *)malloc(sizeof(double) * n);
+            double *Ke = (double *)malloc(sizeof(double) * n), *Ve = (double *)malloc(sizeof(double) * n);
+            double *eps = (double *)calloc((size_t)nb + 1, sizeof(double));
+            double *eta = (double *)calloc((size_t)nb + 1, sizeof(double));
+            double *nu = (double *)calloc((size_t)nb + 1, sizeof(double));
+            double *Ph = (double *)calloc((size_t)g * nb + 1, sizeof(double));
+            double *Pe = (double *)calloc((size_t)g * nb + 1, sizeof(double));
+            double *Pm = (double *)calloc((size_t)nb + 1, sizeof(double));
+            double *Dl = (double *)calloc((size_t)g * nb + 1, sizeof(double));
+            double *scq = (double *)malloc(sizeof(double) * ((size_t)g * T + 1));
+            double *sce = (double *)malloc(sizeof(double) * ((size_t)g * T + 1));
+            double *sm = (double *)malloc(sizeof(double) * ((size_t)T + 1));
+            double *cov = (double *)calloc((size_t)nb + 2, sizeof(double));
+            double *run = (double *)calloc((size_t)g + 1, sizeof(double));
+            kvqo_ranked *rk = (kvqo_ranked *)malloc(sizeof(kvqo_ranked) * ((size_t)nb + 1));
+            char *kx = (char *)calloc((size_t)nb + 1, 1), *vx = (char *)calloc((size_t)nb + 1, 1);
+            char *tmp = (char *)calloc((size_t)nb + 1, 1);
+            double qr[16][KVQO_MAXD];
+
+            /* quantised rows, exact rotated rows, block descriptors */
+            for (int t = 0; t < T; t++) {
+                int slot = slot_of(block_table, max_pages, b, t);
+                size_t row = ((size_t)slot * hkv + kvh) * d;
+                double xk[KVQO_MAXD], xv[KVQO_MAXD];
+                kvqo_dequant_row(c, pool, slot, kvh, 0, Kq + (size_t)t * d);
+                kvqo_dequant_row(c, pool, slot, kvh, 1, Vq + (size_t)t * d);
+                for (int i = 0; i < d; i++) {
+                    xk[i] = kvqo_h2f(k_slots[row + i]);
+                    xv[i] = kvqo_h2f(v_slots[row + i]);
+                }
+                kvqo_rotate_f64(xk, s, d, c->rotate, Ke + (size_t)t * d);
+                kvqo_rotate_f64(xv, s, d, c->rotate, Ve + (size_t)t * d);
+            }
+            for (int p = 0; p < (T + KVQO_PAGE_TOKENS - 1) / KVQO_PAGE_TOKENS; p++) {
+                int pg = block_table[(size_t)b * max_pages + p];
+                const float *desc = (const float *)(pool + kvqo_desc_offset(c) + ((size_t)pg * hkv + kvh) * 16);
+                int blk = p * KVQO_PAGE_TOKENS / block;
+                eps[blk] = fmax(eps[blk], (double)desc[0]);
+                eta[blk] = fmax(eta[blk], (double)desc[1]);
+                nu[blk] = fmax(nu[blk], (double)desc[2]);
+            }
+            /* per head: rotated query, scores, block masses, Delta */
+            for (int hh = 0; hh < g; hh++) {
+                int h = kvh * g + hh;
+                double qx[KVQO_MAXD], qn = 0.0;
+                for (int i = 0; i < d; i++) qx[i] = (double)kvqo_h2f(q[((size_t)b * hq + h) * d + i]);
+                kvqo_rotate_f64(qx, s, d, c->rotate, qr[hh]);
+                for (int i = 0; i < d; i++) qn += fabs(qr[hh][i]);
+                for (int t = 0; t < T; t++) {
+                    double dq = 0.0, de = 0.0;
+                    for (int i = 0; i < d; i++) {
+                        dq += qr[hh][i] * Kq[(size_t)t * d + i];
+                        de += qr[hh][i] * Ke[(size_t)t * d + i];
+                    }
+                    scq[(size_t)hh * T + t] = scale * dq;
+                    sce[(size_t)hh * T + t] = scale * de;
+                }
+                block_masses(scq + (size_t)hh * T, T, block, Ph + (size_t)hh * nb);
+                block_masses(sce + (size_t)hh * T, T, block, Pe + (size_t)hh * nb);
+                for (int bb = 0; bb < nb; bb++) Dl[(size_t)hh * nb + bb] = scale * qn * eps[bb];
+            }
+            /* 1. ranking */
+            for (int bb = 0; bb < nb; bb++) {
+                double r = 0.0;
+                for (int hh = 0; hh < g; hh++) r = fmax(r, Ph[(size_t)hh * nb + bb]);
+                rk[bb].r = r;
+                rk[bb].idx = bb;
+                if (o->rscore) o->rscore[bk * MB + bb] = r;
+            }
+            qsort(rk, (size_t)nb, sizeof(kvqo_ranked), ranked_cmp);
+            /* 2. coverage of the first K ranked blocks, every head */
+            for (int K = 0; K <= nb; K++) {
+                if (K > 0)
+                    for (int hh = 0; hh < g; hh++) run[hh] += Ph[(size_t)hh * nb + rk[K - 1].idx];
+                double m = INFINITY;
+                for (int hh = 0; hh < g; hh++) m = fmin(m, run[hh]);
+                cov[K] = g > 0 ? m : 0.0;
+                if (o->cov) o->cov[bk * (MB + 1) + K] = cov[K];
+            }
+            int k_cov = 0;
+            if (pol->tau_cov > 0.0) {
+                k_cov = nb;
+                for (int K = 0; K <= nb; K++)
+                    if (cov[K] >= pol->tau_cov) {
+                        k_cov = K;
+                        break;
+                    }
+            }
+            /* 3. rung 1: predicted key term with the first K ranked keys exact */
+            int k_key = -1;
+            for (int K = 0; K <= nb; K++) {
+                memset(tmp, 0, (size_t)nb + 1);
+                for (int r = 0; r < K; r++) tmp[rk[r].idx] = 1;
+                double E = 0.0;
+                for (int hh = 0; hh < g; hh++)
+                    E = fmax(E, key_term(Ph + (size_t)hh * nb, Dl + (size_t)hh * nb, nu, tmp, nb));
+                if (o->ekey) o->ekey[bk * (MB + 1) + K] = E;
+                if (k_key < 0 && E <= pol->key_tol) k_key = K;
+            }
+            if (k_key < 0) k_key = nb;
+            int k_cap = kvqo_promote_count(pol->max_frac, nb);
+            int want = k_cov > k_key ? k_cov : k_key;
+            int k_star = want < k_cap ? want : k_cap;
+            /* 4. rung 2 and the flags */
+            for (int r = 0; r < k_star; r++) kx[rk[r].idx] = 1;
+            for (int bb = 0; bb < nb; bb++) {
+                double w = 0.0;
+                for (int hh = 0; hh < g; hh++) w = fmax(w, Ph[(size_t)hh * nb + bb] * eta[bb]);
+                vx[bb] = w > pol->v_tol;
+            }
+            if (forced_flags) {
+                k_star = 0;
+                for (int bb = 0; bb < nb; bb++) {
+                    uint8_t f = forced_flags[bk * MB + bb];
+                    kx[bb] = f & 1;
+                    vx[bb] = (f >> 1) & 1;
+                    k_star += kx[bb];
+                }
+            }
+            int gstat = 0;
+            if (!forced_flags && k_star > k_cov) gstat |= KVQO_LADDER_EXPANDED;
+            if (want > k_cap) gstat |= KVQO_LADDER_CAPPED;
+            for (int bb = 0; bb < nb; bb++)
+                if (vx[bb]) gstat |= KVQO_LADDER_VALUES;
+            if (o->flags)
+                for (int bb = 0; bb < MB; bb++) o->flags[bk * MB + bb] = bb < nb ? (uint8_t)(kx[bb] | (vx[bb] << 1)) : 0;
+            if (o->k_star) o->k_star[bk] = k_star;
+            if (o->k_cov) o->k_cov[bk] = k_cov;
+            if (o->k_key) o->k_key[bk] = k_key;
+
+            for (int hh = 0; hh < g; hh++) {
+                int h = kvh * g + hh;
+                const double *sq = scq + (size_t)hh * T, *se = sce + (size_t)hh * T;
+                /* 5. mixed attention and exact attention (rotated domain) */
+                double om[KVQO_MAXD], oe[KVQO_MAXD];
+                for (int t = 0; t < T; t++) sm[t] = kx[t / block] ? se[t] : sq[t];
+                double mm = -INFINITY, me = -INFINITY, lm = 0.0, le = 0.0;
+                for (int i = 0; i < d; i++) om[i] = oe[i] = 0.0;
+                for (int t = 0; t < T; t++) {
+                    mm = fmax(mm, sm[t]);
+                    me = fmax(me, se[t]);
+                }
+                for (int t = 0; t < T; t++) {
+                    double pm = exp(sm[t] - mm), pe = exp(se[t] - me);
+                    const double *vm = (vx[t / block] ? Ve : Vq) + (size_t)t * d, *ve = Ve + (size_t)t * d;
+                    lm += pm;
+                    le += pe;
+                    for (int i = 0; i < d; i++) {
+                        om[i] += pm * vm[i];
+                        oe[i] += pe * ve[i];
+                    }
+                }
+                double err = 0.0;
+                for (int i = 0; i < d; i++) {
+                    om[i] = T > 0 ? om[i] / lm : 0.0;
+                    oe[i] = T > 0 ? oe[i] / le : 0.0;
+                    err = fmax(err, fabs(oe[i] - om[i]));
+                }
+                kvqo_inv_rotate_f64(om, s, d, c->rotate, mixed + ((size_t)b * hq + h) * d);
+                /* 6. ranking-consistency check over the key-promoted blocks */
+                int fail_rank = 0;
+                if (!isinf(pol->rank_tol)) {
+                    int nS = 0;
+                    for (int bb = 0; bb < nb; bb++)
+                        if (kx[bb]) {
+                            rk[nS].r = Ph[(size_t)hh * nb + bb];
+                            rk[nS].idx = bb;
+                            nS++;
+                        }
+                    qsort(rk, (size_t)nS, sizeof(kvqo_ranked), ranked_cmp);
+                    for (int i = 0; i < nS && !fail_rank; i++)
+                        for (int j = i + 1; j < nS; j++)
+                            if (Pe[(size_t)hh * nb + rk[j].idx] > (1.0 + pol->rank_tol) * Pe[(size_t)hh * nb + rk[i].idx]) {
+                                fail_rank = 1;
+                                break;
+                            }
+                }
+                /* 7. certified bound of the mixed output */
+                block_masses(sm, T, block, Pm);
+                double bnd = key_term(Pm, Dl + (size_t)hh * nb, nu, kx, nb);
+                for (int bb = 0; bb < nb; bb++)
+                    if (!vx[bb]) bnd += Pm[bb] * eta[bb];
+                int fail_bound = bnd > pol->cert_tol;
+                int st = gstat | (fail_rank ? KVQO_LADDER_RANK_FAIL : 0) | (fail_bound ? KVQO_LADDER_BOUND_FAIL : 0);
+                stat[(size_t)b * hq + h] = st;
+                fall[(size_t)b * hq + h] = fail_rank || fail_bound;
+                if (o->err) o->err[(size_t)b * hq + h] = err;
+                if (o->bound) o->bound[(size_t)b * hq + h] = bnd;
+            }
+            free(Kq);
+            free(Vq);
+            free(Ke);
+            free(Ve);
+            free(eps);
+            free(eta);
+            free(nu);
+            free(Ph);
+            free(Pe);
+            free(Pm);
+            free(Dl);
+            free(scq);
+            free(sce);
+            free(sm);
+            free(cov);
+            free(run);
+            free(rk);
+            free(kx);
+            free(vx);
+            free(tmp);
+        }
+    }
+    /* 8-9. fallbacks: fp16 attention over the tier-2 rows */
+    long long count = 0;
+    for (size_t i = 0; i < (size_t)B * hq; i++) count += fall[i];
+    int layer = (double)count > pol->layer_frac * (double)B * (double)hq;
+    int rc = kvqo_decode_fp16(c, k_slots, v_slots, q, block_table, max_pages, ctx_lens, B, scale, NULL, dense);
+    for (size_t i = 0; i < (size_t)B * hq && rc == 0; i++) {
+        int fb;
+        if (forced_fallback) {
+            fb = forced_fallback[i] != 0;
+            if (fb) stat[i] |= KVQO_LADDER_HEAD_DENSE;
+        } else {
+            fb = fall[i] || layer;
+            if (fall[i]) stat[i] |= KVQO_LADDER_HEAD_DENSE;
+            if (layer) stat[i] |= KVQO_LADDER_LAYER_DENSE;
+        }
+        if (o->status) o->status[i] = stat[i];
+        for (int k = 0; k < d; k++) o->out[i * d + k] = fb ? dense[i * d + k] : mixed[i * d + k];
+    }
+    if (!o->mixed) free(mixed);
+    if (!o->dense) free(dense);
+    free(fall);
+    free(stat);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Array helpers for the tests                                               */
 /* ------------------------------------------------------------------------- */
 

@@ -17,10 +17,17 @@ Recipes (numpy ``default_rng``; every stream is keyed by (seed, stream id)):
   certified   B=1, 32/8, d=128, T=131072; llama's distributions; K int8
               symmetric per token-head, V int4 g32; 128-token bound blocks;
               top 1% of blocks promoted from the fp16 copy.
+  ladder      certified's geometry and formats with concentrated attention
+              (a stand-in for the needle-retrieval workloads the pages
+              measure): llama's K/V, plus per kv head a seeded unit direction
+              u; the keys of "hot" tokens -- the first 16 (sink), six needle
+              spans of 64 tokens at seeded positions, the last 128 -- get
+              a*u added with a ~ U[10, 14] (then rounded to fp16); queries are
+              N(0,1) + 10*u of their kv head.
   int2        prefill of 65536 tokens x 8 kv heads x d=128 per sequence, K and
               V ~ Laplace(0,1) with 1% of elements x30; 2-bit g128, clip 0.9;
               decode B=4, Hq=32, T=65536 (four independent prefills).
-  q           ~ N(0,1), drawn anew for every step.
+  q           ~ N(0,1), drawn anew for every step (ladder: plus its pull).
 """
 from __future__ import annotations
 
@@ -33,7 +40,9 @@ INT4_ASYM, INT8_SYM, INT2_ASYM = 0, 1, 2
 PAGE_TOKENS = 16
 
 # stream ids
-_S_K, _S_V, _S_Q, _S_LEN, _S_PERM, _S_OUT, _S_NEWK, _S_NEWV = range(8)
+_S_K, _S_V, _S_Q, _S_LEN, _S_PERM, _S_OUT, _S_NEWK, _S_NEWV, _S_DIR, _S_HOT = range(10)
+
+NEEDLES, NEEDLE_LEN, SINK_LEN, RECENT_LEN, QUERY_PULL = 6, 64, 16, 128, 10.0
 
 
 @dataclass
@@ -51,7 +60,7 @@ class Workload:
     clip: float = 1.0
     bound_block: int = 0
     promote_frac: float = 0.0
-    dist: str = "llama"  # tiny | llama | laplace
+    dist: str = "llama"  # tiny | llama | laplace | needle
     seed: int = 0
     rotation_seed: int = 0x5EED
     steps: int = 1  # decode steps (each appends one token per sequence first)
@@ -89,6 +98,14 @@ def certified(T: int = 131072) -> Workload:
                                 "128-token bound blocks, top 1% promoted from pinned fp16")
 
 
+def ladder(T: int = 131072) -> Workload:
+    return Workload(f"int8k-int4v-ladder-T{T}", 1, 32, 8, 128, [T], k_fmt=INT8_SYM, k_group=128,
+                    bound_block=128, dist="needle", seed=5, steps=1,
+                    description="batch 1, 32/8 heads, head_dim 128, K int8 symmetric per token-head, V int4 g32, "
+                                "128-token bound blocks, attention concentrated on a sink, six needles and the "
+                                "recent window; adaptive certified ladder over pinned fp16")
+
+
 def int2(B: int = 4, T: int = 65536) -> Workload:
     return Workload(f"int2-g128-clip0.9-B{B}-T{T}", B, 32, 8, 128, [T] * B, k_fmt=INT2_ASYM, v_fmt=INT2_ASYM,
                     k_group=128, v_group=128, clip=0.9, dist="laplace", seed=4, steps=1,
@@ -96,7 +113,7 @@ def int2(B: int = 4, T: int = 65536) -> Workload:
                                 "g128 clip 0.9; decode batch 4, 32 q heads, context 65536")
 
 
-ALL = {"tiny": tiny, "llama": llama, "paged": paged, "certified": certified, "int2": int2}
+ALL = {"tiny": tiny, "llama": llama, "paged": paged, "certified": certified, "ladder": ladder, "int2": int2}
 
 
 def scaled(wl: Workload, ctx, steps: int = 1) -> Workload:
@@ -128,7 +145,7 @@ def _rows(wl: Workload, b: int, stream: int, n: int, t0: int, tensor: int) -> np
         ch = _outlier_channels(wl, 2)
         for h in range(wl.Hkv):
             x[:, h, ch[h]] *= 20.0
-    else:  # llama
+    else:  # llama (and the needle recipe's base rows)
         if tensor == 0:
             x = rng.standard_normal(size=shape)
             ch = _outlier_channels(wl, 4)
@@ -139,10 +156,36 @@ def _rows(wl: Workload, b: int, stream: int, n: int, t0: int, tensor: int) -> np
     return x.astype(np.float16)
 
 
+def needle_directions(wl: Workload) -> np.ndarray:
+    """Unit directions u [Hkv, d] (float64) of the needle recipe."""
+    rng = np.random.default_rng([wl.seed, _S_DIR])
+    u = rng.standard_normal(size=(wl.Hkv, wl.d))
+    return u / np.linalg.norm(u, axis=1, keepdims=True)
+
+
+def hot_tokens(wl: Workload, b: int):
+    """(positions int64 [n], amplitudes float64 [n]) of sequence b's hot
+    tokens in the needle recipe: sink, needle spans, recent window (clipped to
+    the prefix; overlaps keep one entry)."""
+    T = wl.ctx[b]
+    rng = np.random.default_rng([wl.seed, _S_HOT, b])
+    starts = rng.integers(0, max(1, T - NEEDLE_LEN), size=NEEDLES)
+    pos = [np.arange(0, min(SINK_LEN, T)), np.arange(max(0, T - RECENT_LEN), T)]
+    pos += [np.arange(s, min(s + NEEDLE_LEN, T)) for s in starts]
+    pos = np.unique(np.concatenate(pos)).astype(np.int64)
+    amp = rng.uniform(10.0, 14.0, size=pos.shape[0])
+    return pos, amp
+
+
 def prefix_kv(wl: Workload, b: int):
     """fp16 K, V [ctx_b, Hkv, d] of sequence b's prefix."""
     T = wl.ctx[b]
-    return _rows(wl, b, _S_K, T, 0, 0), _rows(wl, b, _S_V, T, 0, 1)
+    k, v = _rows(wl, b, _S_K, T, 0, 0), _rows(wl, b, _S_V, T, 0, 1)
+    if wl.dist == "needle" and T > 0:
+        pos, amp = hot_tokens(wl, b)
+        u = needle_directions(wl)
+        k[pos] = (k[pos].astype(np.float64) + amp[:, None, None] * u[None]).astype(np.float16)
+    return k, v
 
 
 def step_kv(wl: Workload, step: int):
@@ -154,7 +197,10 @@ def step_kv(wl: Workload, step: int):
 
 def queries(wl: Workload, step: int) -> np.ndarray:
     rng = np.random.default_rng([wl.seed, _S_Q, step])
-    return rng.standard_normal(size=(wl.B, wl.Hq, wl.d)).astype(np.float16)
+    q = rng.standard_normal(size=(wl.B, wl.Hq, wl.d))
+    if wl.dist == "needle":
+        q = q + QUERY_PULL * np.repeat(needle_directions(wl), wl.g, axis=0)[None]
+    return q.astype(np.float16)
 
 
 # --- page tables --------------------------------------------------------------
@@ -224,4 +270,10 @@ def prefix_kv_device(wl: Workload, b: int, device):
         else:
             x = torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * 0.5
         out.append(x.to(torch.float16))
+    if wl.dist == "needle" and T > 0:
+        pos, amp = hot_tokens(wl, b)
+        u = torch.from_numpy(needle_directions(wl)).to(device)
+        p = torch.from_numpy(pos).to(device)
+        a = torch.from_numpy(amp).to(device)
+        out[0][p] = (out[0][p].double() + a[:, None, None] * u[None]).to(torch.float16)
     return out[0], out[1]
