@@ -391,6 +391,7 @@ def run_ours(args, dist: Dist):
         result["e2e"] = e2e_leg(wk, K, stream, dist)
         result["append"] = append_leg()
         result["certified"] = certified_leg(min(K, 200))
+        result["ladder"] = ladder_leg(min(K, 100))
     if dist.rank == 0:
         if not args.no_extras:
             result["cpu_baseline"] = cpu_leg(wk, args.cpu_steps)
@@ -495,19 +496,15 @@ def append_leg():
             "peak_kind": kind, "inputs_exceed_l2": True}
 
 
-def certified_leg(steps: int):
-    """Certified decode at its own configuration: batch 1, context 131072,
-    int8 K / int4 g32 V, 128-token bound blocks, top 1% of each kv head's
-    blocks promoted from exact fp16 rows in pinned host memory.  Calls (three
-    launches each) replayed in a CUDA graph over two cache copies (440 MB >
-    3x L2) and timed as a whole, beside the plain quantised decode of the
-    same cache."""
+def _tier2_cache(wl, copies: int):
+    """A certified-mode cache of `copies` independent copies of sequence 0 of
+    `wl` (drawn on the device), with the exact fp16 rows in pinned host memory
+    as tier 2."""
     import torch
 
     import quantized_kv_cache_16_b200 as K
     import workloads as W
-    wl = W.certified()
-    T, frac, copies = wl.ctx[0], 0.01, 2
+    T = wl.ctx[0]
     dev = torch.device("cuda", torch.cuda.current_device())
     tabs = W.page_table(wl, copies=copies)
     cfg = K.make_config(wl.Hq, wl.Hkv, wl.d, wl.k_fmt, wl.v_fmt, wl.k_group, wl.v_group, wl.clip, wl.rotation_seed,
@@ -523,13 +520,57 @@ def certified_leg(steps: int):
         cache.append(kd, vd, sl.int().to(dev))
         k2[sl], v2[sl] = kh, vh
     del kd, vd, kh, vh
+    bts = [torch.from_numpy(t.block_table).to(dev) for t in tabs]
+    ctx = torch.tensor([T], dtype=torch.int32, device=dev)
+    return cache, k2, v2, bts, ctx
+
+
+def _graph_time(call, steps: int, stream) -> float:
+    """Mean microseconds of call(s) for s in range(steps), replayed as one
+    CUDA graph after four eager warm-up calls and one warm-up replay."""
+    import torch
+    with torch.cuda.stream(stream):
+        for s in range(4):
+            call(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        for s in range(steps):
+            call(s)
+    g.replay()
+    torch.cuda.synchronize()
+    rt = Cudart()
+    e0, e1 = rt.event(), rt.event()
+    rt.record(e0, stream.cuda_stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+    rt.record(e1, stream.cuda_stream)
+    torch.cuda.synchronize()
+    us = rt.elapsed_ms(e0, e1) * 1e3 / steps
+    del g
+    return us
+
+
+def certified_leg(steps: int):
+    """Certified decode at its own configuration: batch 1, context 131072,
+    int8 K / int4 g32 V, 128-token bound blocks, top 1% of each kv head's
+    blocks promoted from exact fp16 rows in pinned host memory.  Calls (four
+    launches each) replayed in a CUDA graph over two cache copies (440 MB >
+    3x L2) and timed as a whole, beside the plain quantised decode of the
+    same cache."""
+    import torch
+
+    import quantized_kv_cache_16_b200 as K
+    import workloads as W
+    wl = W.certified()
+    T, frac, copies = wl.ctx[0], 0.01, 2
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cache, k2, v2, bts, ctx = _tier2_cache(wl, copies)
     nq = 8
     gen = torch.Generator(device=dev)
     gen.manual_seed(wl.seed)
     qs = torch.randn((nq, 1, wl.Hq, wl.d), generator=gen, device=dev).half()
-    bts = [torch.from_numpy(t.block_table).to(dev) for t in tabs]
     max_pages = bts[0].shape[1]
-    ctx = torch.tensor([T], dtype=torch.int32, device=dev)
     ws = cache.workspace_for(1, max_pages)
     out = torch.empty((1, wl.Hq, wl.d), dtype=torch.float32, device=dev)
     nb = (T + wl.bound_block - 1) // wl.bound_block
@@ -537,32 +578,15 @@ def certified_leg(steps: int):
     prom = torch.empty((1, wl.Hkv, kmax), dtype=torch.int32, device=dev)
     t2 = K.kvq_tier2(k2.data_ptr(), v2.data_ptr(), frac)
     stream = torch.cuda.Stream()
-    rt = Cudart()
 
-    def call(s, tier2):
-        K.kvq_decode_attn(cache.handle, qs[s % nq], bts[s % copies], max_pages, ctx, 1, 0.0, tier2, ws, ws.numel(),
-                          out, prom if tier2 is not None else None, stream)
+    def caller(tier2):
+        def call(s):
+            K.kvq_decode_attn(cache.handle, qs[s % nq], bts[s % copies], max_pages, ctx, 1, 0.0, tier2, ws,
+                              ws.numel(), out, prom if tier2 is not None else None, stream)
+        return call
 
-    res = {}
-    for name, tier2 in (("quantised_only", None), ("certified", t2)):
-        with torch.cuda.stream(stream):
-            for s in range(4):
-                call(s, tier2)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
-            for s in range(steps):
-                call(s, tier2)
-        g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = rt.event(), rt.event()
-        rt.record(e0, stream.cuda_stream)
-        with torch.cuda.stream(stream):
-            g.replay()
-        rt.record(e1, stream.cuda_stream)
-        torch.cuda.synchronize()
-        res[name] = rt.elapsed_ms(e0, e1) * 1e3 / steps
-        del g
+    res = {name: _graph_time(caller(tier2), steps, stream) for name, tier2 in (("quantised_only", None),
+                                                                                ("certified", t2))}
     assert cache.sync_status() == 0
     hbm = T * wl.Hkv * (wl.d + 2 + wl.d // 2 + 4 * (wl.d // 32))
     link = wl.Hkv * kmax * wl.bound_block * wl.d * 2 * 2
@@ -575,6 +599,97 @@ def certified_leg(steps: int):
             "quantised_only_GB/s": round(hbm / (res["quantised_only"] * 1e-6) / 1e9, 1),
             "quantised_only_pct_hbm_peak": hbm / (res["quantised_only"] * 1e-6) / 1e9 / peak, "peak_kind": kind,
             "l2_policy": "2 cache copies (440 MB) alternate", "steps": steps}
+
+
+LADDER_POLICY = dict(tau_cov=0.995, max_frac=0.05, key_tol=0.02, v_tol=1e-3, rank_tol=0.05, cert_tol=0.02,
+                     layer_frac=0.5)
+
+
+def ladder_leg(steps: int):
+    """Certified decode with the adaptive ladder (kvq_decode_certified, six
+    launches) at context 131072 on the needle workload (attention
+    concentrated on a sink, six needles and the recent window), replayed in
+    a CUDA graph over two cache copies; beside it the quantised decode of the
+    same cache, and the whole-call fp16 fallback (rung 4, every head
+    recomputed from pinned host rows) timed eagerly over a few calls."""
+    import numpy as np
+    import torch
+
+    import quantized_kv_cache_16_b200 as K
+    import workloads as W
+    wl = W.ladder()
+    T, copies = wl.ctx[0], 2
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cache, k2, v2, bts, ctx = _tier2_cache(wl, copies)
+    nq = 8
+    qs = torch.from_numpy(np.stack([W.queries(wl, s) for s in range(nq)])).to(dev)
+    max_pages = bts[0].shape[1]
+    ws = cache.workspace_for(1, max_pages)
+    out = torch.empty((1, wl.Hq, wl.d), dtype=torch.float32, device=dev)
+    nb = (T + wl.bound_block - 1) // wl.bound_block
+    rep_t = {"k_star": torch.zeros((1, wl.Hkv), dtype=torch.int32, device=dev),
+             "flags": torch.zeros((1, wl.Hkv, nb), dtype=torch.uint8, device=dev),
+             "bound": torch.zeros((1, wl.Hq), dtype=torch.float32, device=dev),
+             "status": torch.zeros((1, wl.Hq), dtype=torch.int32, device=dev)}
+    rep = K.kvq_ladder_report(rep_t["k_star"].data_ptr(), rep_t["flags"].data_ptr(), nb, rep_t["bound"].data_ptr(),
+                              rep_t["status"].data_ptr())
+    stream = torch.cuda.Stream()
+
+    def caller(pol):
+        names = ("tau_cov", "max_frac", "key_tol", "v_tol", "rank_tol", "cert_tol", "layer_frac")
+        lp = None if pol is None else K.kvq_ladder(*[pol[n] for n in names])
+
+        def call(s):
+            if pol is None:
+                K.kvq_decode_attn(cache.handle, qs[s % nq], bts[s % copies], max_pages, ctx, 1, 0.0, None, ws,
+                                  ws.numel(), out, None, stream)
+            else:
+                K.kvq_decode_certified(cache.handle, qs[s % nq], bts[s % copies], max_pages, ctx, 1, 0.0, k2, v2, lp,
+                                       ws, ws.numel(), out, rep, stream)
+        return call
+
+    quant_us = _graph_time(caller(None), steps, stream)
+    ladder_us = _graph_time(caller(LADDER_POLICY), steps, stream)
+    # rungs 1-2 alone: no ranking check, no bound fallback
+    rungs12_us = _graph_time(caller(dict(LADDER_POLICY, rank_tol=math.inf, cert_tol=math.inf)), steps, stream)
+    # what the ladder did on each of the nq queries
+    kstar, nval, dense = [], [], []
+    for s in range(nq):
+        caller(LADDER_POLICY)(s)
+        torch.cuda.synchronize()
+        fl = rep_t["flags"].cpu().numpy()
+        kstar.append(rep_t["k_star"].cpu().numpy().mean())
+        nval.append(((fl >> 1) & 1).sum(axis=2).mean())
+        dense.append(int(((rep_t["status"].cpu().numpy() & K.KVQ_LADDER_HEAD_DENSE) != 0).sum()))
+    # rung 4: every head recomputed from the host rows
+    layer_pol = dict(LADDER_POLICY, cert_tol=0.0)
+    call = caller(layer_pol)
+    with torch.cuda.stream(stream):
+        call(0)
+    torch.cuda.synchronize()
+    rt = Cudart()
+    e0, e1 = rt.event(), rt.event()
+    n_layer = 3
+    rt.record(e0, stream.cuda_stream)
+    for s in range(n_layer):
+        call(s)
+    rt.record(e1, stream.cuda_stream)
+    torch.cuda.synchronize()
+    layer_us = rt.elapsed_ms(e0, e1) * 1e3 / n_layer
+    assert int((rep_t["status"].cpu().numpy() & K.KVQ_LADDER_LAYER_DENSE != 0).sum()) == wl.Hq
+    assert cache.sync_status() == 0
+    row = wl.bound_block * wl.d * 2
+    link = int(round((np.mean(kstar) + np.mean(nval)) * wl.Hkv * row))
+    return {"workload": "certified ladder: B=1, 32/8 heads, d=128, context 131072, int8 K / int4 g32 V, 128-token "
+                        "blocks, needle attention (sink, six needles, recent window); pinned host fp16 tier 2",
+            "policy": LADDER_POLICY, "us": round(ladder_us, 2), "quantised_only_us": round(quant_us, 2),
+            "overhead_x": round(ladder_us / quant_us, 2), "no_fallback_us": round(rungs12_us, 2),
+            "no_fallback_overhead_x": round(rungs12_us / quant_us, 2),
+            "mean_key_blocks_per_kv_head": round(float(np.mean(kstar)), 2),
+            "mean_value_blocks_per_kv_head": round(float(np.mean(nval)), 2),
+            "mean_heads_dense": round(float(np.mean(dense)), 2), "host_link_bytes": link,
+            "layer_fallback_us": round(layer_us, 1), "layer_fallback_host_bytes": T * wl.Hkv * wl.d * 2 * 2,
+            "steps": steps, "queries": nq}
 
 
 def cpu_leg(wk: Workload, n_steps: int):

@@ -18,7 +18,9 @@
  *    log-sum-exp rule, inverse-rotated ["OSCAR", 2.2b (fused kernel: unpack,
  *    dequantise, inverse rotation, attention over a paged cache)].
  *  - Certified mode: per-block key/value error bounds, top-fraction promotion
- *    of blocks to their fp16 originals held in pinned host memory
+ *    of blocks to their fp16 originals held in pinned host memory, and the
+ *    adaptive ladder (coverage-driven key promotion, value promotion, the
+ *    ranking-consistency check, per-head and whole-call fp16 fallbacks)
  *    ["Runtime-Certified Bounded-Error Quantized Attention", Methodology 1-3].
  *
  * Conventions for every call:
@@ -166,6 +168,81 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int32_t batch, int32_t
 kvq_status kvq_decode_attn(kvq_cache *cache, const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
                            const int32_t *ctx_lens, int32_t batch, float softmax_scale, const kvq_tier2 *tier2,
                            void *workspace, size_t ws_bytes, void *out, int32_t *promoted_out, void *stream);
+
+/* Policy of the certified ladder ["Runtime-Certified Bounded-Error Quantized
+ * Attention", Methodology 3: adaptive Top-K, ranking-consistency check,
+ * four-rung fallback ladder].  Tolerances may be +INFINITY (that rung or
+ * check off); NaN or a value outside its range is KVQ_ERR_INVALID_ARG. */
+typedef struct {
+    float tau_cov;    /* [0, 1]: estimated block mass the exact keys must cover, for every head   */
+    float max_frac;   /* [0, 1]: budget, at most ceil(max_frac * n_blocks) key-promoted blocks     */
+    float key_tol;    /* >= 0: rung 1 grows the key set until the predicted key term is <= key_tol */
+    float v_tol;      /* >= 0: rung 2 promotes values of blocks with max_h Phat_h(b)*eta_b > v_tol */
+    float rank_tol;   /* >= 0: slack of the ranking-consistency check                              */
+    float cert_tol;   /* >= 0: heads whose certified bound exceeds it fall back to fp16 (rung 3)   */
+    float layer_frac; /* [0, 1]: every head falls back when more than layer_frac*batch*Hq do (rung 4) */
+} kvq_ladder;
+
+/* Status bits of a head (kvq_ladder_report.status). */
+enum {
+    KVQ_LADDER_EXPANDED = 1,    /* rung 1 added blocks beyond the coverage set (group-wide)   */
+    KVQ_LADDER_CAPPED = 2,      /* the budget cut the key set short (group-wide)              */
+    KVQ_LADDER_VALUES = 4,      /* rung 2 promoted values in this kv head's group             */
+    KVQ_LADDER_RANK_FAIL = 8,   /* the ranking-consistency check failed for this head         */
+    KVQ_LADDER_BOUND_FAIL = 16, /* the certified bound exceeded cert_tol                      */
+    KVQ_LADDER_HEAD_DENSE = 32, /* rung 3: this head was recomputed as fp16 attention         */
+    KVQ_LADDER_LAYER_DENSE = 64 /* rung 4: every head of the call was recomputed in fp16      */
+};
+
+/* Optional device outputs of kvq_decode_certified (any pointer may be NULL). */
+typedef struct {
+    int32_t *k_star;      /* [batch][Hkv]: key-promoted blocks                              */
+    uint8_t *block_flags; /* [batch][Hkv][flags_cols]: bit 0 key exact, bit 1 value exact;
+                             flags_cols >= ceil(16*max_pages_per_seq / bound_block_tokens) */
+    int32_t flags_cols;
+    float *bound;         /* [batch][Hq]: certified bound of the mixed output (before any
+                             fallback), an upper bound on the inf-norm of its error in the
+                             rotated domain                                                 */
+    int32_t *status;      /* [batch][Hq]: KVQ_LADDER_* bits                                 */
+} kvq_ladder_report;
+
+/* Certified decode with the adaptive ladder ["Runtime-Certified Bounded-Error
+ * Quantized Attention", Methodology 1-3].  Per sequence and kv head, with
+ * Phat_h(b) the softmax mass of bound block b under the quantised scores of
+ * query head h, Delta_h(b) = scale*||R q_h||_1*eps_b the largest score error
+ * of the block, and eta_b, nu_b its largest value error and |value| (the
+ * descriptors):
+ *  1. blocks are ranked by max_h Phat_h(b) (ties: lower block first);
+ *  2. K_cov = the fewest leading blocks whose Phat reaches tau_cov for every
+ *     head of the group;
+ *  3. rung 1: K_key = the fewest leading blocks whose exact keys bring every
+ *     head's predicted key term sum_b Phat nu_b (e^{D_b + A} - 1), A = ln
+ *     sum_b Phat e^{D_b} (D = 0 for exact-key blocks, Delta otherwise) to
+ *     key_tol; the first K* = min(budget, max(K_cov, K_key)) blocks are
+ *     recomputed with their tier-2 keys;
+ *  4. rung 2: blocks with max_h Phat_h(b)*eta_b > v_tol use their tier-2 values;
+ *  5. the output is attention with those keys/values exact, the rest dequantised;
+ *  6. per head, the key-promoted blocks ordered by Phat_h fail the ranking
+ *     check when a later one has an exact mass above (1 + rank_tol) times an
+ *     earlier one's;
+ *  7. per head, the certified bound of that output is the key term and the
+ *     mass-weighted value error of the blocks with quantised values, both
+ *     over the output's own softmax masses;
+ *  8. rung 3: a head whose check fails or whose bound exceeds cert_tol is
+ *     recomputed as fp16 attention over its tier-2 rows;
+ *  9. rung 4: if more than layer_frac*batch*Hq heads fall back, all do.
+ * Decisions are taken in fp32 from the quantised pass's statistics.
+ *   k_tier2, v_tier2: the tier-2 store as for kvq_tier2 (pinned host or
+ *                device memory, [num_pages*16][Hkv][d] fp16, 16-byte aligned;
+ *                pageable host memory: KVQ_ERR_INVALID_ARG)
+ *   Other arguments as kvq_decode_attn, with the certified-mode limits on
+ *   the bound blocks (KVQ_ERR_UNSUPPORTED beyond them).  Six launches on
+ *   `stream`; the fp16 fallback kernel exits at once when no head needs it. */
+kvq_status kvq_decode_certified(kvq_cache *cache, const void *q, const int32_t *block_table,
+                                int32_t max_pages_per_seq, const int32_t *ctx_lens, int32_t batch,
+                                float softmax_scale, const void *k_tier2, const void *v_tier2,
+                                const kvq_ladder *policy, void *workspace, size_t ws_bytes, void *out,
+                                const kvq_ladder_report *report, void *stream);
 
 /* One decode step: quantise-on-append of each sequence's new token followed
  * by decode attention over the grown context, in one launch.  k_new, v_new:

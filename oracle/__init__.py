@@ -71,7 +71,7 @@ class LadderOut(C.Structure):
     _fields_ = [("out", C.c_void_p), ("mixed", C.c_void_p), ("dense", C.c_void_p), ("err", C.c_void_p),
                 ("bound", C.c_void_p), ("status", C.c_void_p), ("k_star", C.c_void_p), ("k_cov", C.c_void_p),
                 ("k_key", C.c_void_p), ("flags", C.c_void_p), ("rscore", C.c_void_p), ("cov", C.c_void_p),
-                ("ekey", C.c_void_p), ("max_blocks", C.c_int32)]
+                ("ekey", C.c_void_p), ("max_blocks", C.c_int32), ("rank_margin", C.c_void_p)]
 
 
 LADDER_EXPANDED, LADDER_CAPPED, LADDER_VALUES = 1, 2, 4
@@ -357,7 +357,7 @@ def decode_ladder(cfg: Config, pool: np.ndarray, k_slots, v_slots, q, block_tabl
     is off -- tau 0, budget 1, tolerances inf, layer_frac 1).  Returns a dict
     of numpy arrays: out, mixed, dense [B,Hq,d]; err, bound, status [B,Hq];
     k_star, k_cov, k_key [B,Hkv]; flags, rscore [B,Hkv,max_blocks]; cov, ekey
-    [B,Hkv,max_blocks+1]."""
+    [B,Hkv,max_blocks+1]; rank_margin [B,Hq]."""
     k = _c(k_slots, np.float16).view(np.uint16)
     v = _c(v_slots, np.float16).view(np.uint16)
     q = _c(q, np.float16).view(np.uint16)
@@ -375,9 +375,11 @@ def decode_ladder(cfg: Config, pool: np.ndarray, k_slots, v_slots, q, block_tabl
         "k_star": np.zeros((B, hkv), np.int32), "k_cov": np.zeros((B, hkv), np.int32),
         "k_key": np.zeros((B, hkv), np.int32), "flags": np.zeros((B, hkv, mb), np.uint8),
         "rscore": np.zeros((B, hkv, mb)), "cov": np.zeros((B, hkv, mb + 1)), "ekey": np.zeros((B, hkv, mb + 1)),
+        "rank_margin": np.zeros((B, hq)),
     }
     o = LadderOut(*[r[n].ctypes.data for n in ("out", "mixed", "dense", "err", "bound", "status", "k_star", "k_cov",
-                                                "k_key", "flags", "rscore", "cov", "ekey")], mb)
+                                                "k_key", "flags", "rscore", "cov", "ekey")], mb,
+                  r["rank_margin"].ctypes.data)
     ff = None if forced_flags is None else _c(forced_flags, np.uint8)
     if ff is not None:
         assert ff.shape == (B, hkv, mb)

@@ -897,7 +897,10 @@ typedef struct {
  * (before any fallback), dense (fp16 attention).  [B][Hq]: err (measured
  * rotated-domain inf-norm error of mixed against exact attention), bound,
  * status (bits below).  [B][Hkv]: k_star, k_cov, k_key.  [B][Hkv][max_blocks]:
- * flags (bit 0 key exact, bit 1 value exact), rscore (the ranking score r).
+ * flags (bit 0 key exact, bit 1 value exact), rscore (the ranking score r);
+ * rank_margin [B][Hq]: max over ordered pairs of (later exact mass / earlier
+ * exact mass) - 1 (0 with fewer than two key-promoted blocks, inf when an
+ * earlier block has zero exact mass and a later one does not).
  * [B][Hkv][max_blocks + 1]: cov (min over the group's heads of the coverage of
  * the first K ranked blocks), ekey (max over the heads of the predicted key
  * term with the first K ranked blocks' keys exact). */
@@ -907,6 +910,7 @@ typedef struct {
     uint8_t *flags;
     double *rscore, *cov, *ekey;
     int32_t max_blocks;
+    double *rank_margin; /* [B][Hq]: the smallest rank_tol the head's check passes with */
 } kvqo_ladder_out;
 
 #define KVQO_LADDER_EXPANDED 1    /* rung 1 added blocks beyond the coverage set */
@@ -1175,22 +1179,23 @@ int kvqo_decode_ladder(const kvqo_config *c, const uint8_t *pool, const uint16_t
                 kvqo_inv_rotate_f64(om, s, d, c->rotate, mixed + ((size_t)b * hq + h) * d);
                 /* 6. ranking-consistency check over the key-promoted blocks */
                 int fail_rank = 0;
-                if (!isinf(pol->rank_tol)) {
-                    int nS = 0;
-                    for (int bb = 0; bb < nb; bb++)
-                        if (kx[bb]) {
-                            rk[nS].r = Ph[(size_t)hh * nb + bb];
-                            rk[nS].idx = bb;
-                            nS++;
-                        }
-                    qsort(rk, (size_t)nS, sizeof(kvqo_ranked), ranked_cmp);
-                    for (int i = 0; i < nS && !fail_rank; i++)
-                        for (int j = i + 1; j < nS; j++)
-                            if (Pe[(size_t)hh * nb + rk[j].idx] > (1.0 + pol->rank_tol) * Pe[(size_t)hh * nb + rk[i].idx]) {
-                                fail_rank = 1;
-                                break;
-                            }
-                }
+                double margin = 0.0;
+                int nS = 0;
+                for (int bb = 0; bb < nb; bb++)
+                    if (kx[bb]) {
+                        rk[nS].r = Ph[(size_t)hh * nb + bb];
+                        rk[nS].idx = bb;
+                        nS++;
+                    }
+                qsort(rk, (size_t)nS, sizeof(kvqo_ranked), ranked_cmp);
+                for (int i = 0; i < nS; i++)
+                    for (int j = i + 1; j < nS; j++) {
+                        double ei = Pe[(size_t)hh * nb + rk[i].idx], ej = Pe[(size_t)hh * nb + rk[j].idx];
+                        if (!isinf(pol->rank_tol) && ej > (1.0 + pol->rank_tol) * ei) fail_rank = 1;
+                        if (ei > 0.0) margin = fmax(margin, ej / ei - 1.0);
+                        else if (ej > 0.0) margin = INFINITY;
+                    }
+                if (o->rank_margin) o->rank_margin[(size_t)b * hq + h] = margin;
                 /* 7. certified bound of the mixed output */
                 block_masses(sm, T, block, Pm);
                 double bnd = key_term(Pm, Dl + (size_t)hh * nb, nu, kx, nb);

@@ -24,8 +24,8 @@ PAGE_TOKENS = 16
 # Every symbol include/kvq.h declares (checked by the ABI test).
 EXPORTS = (
     "kvq_pool_bytes", "kvq_create_cache", "kvq_destroy_cache", "kvq_append", "kvq_reset_pages",
-    "kvq_decode_workspace_bytes", "kvq_decode_attn", "kvq_decode_step", "kvq_decode_attn_static",
-    "kvq_dequant_debug", "kvq_sync_status",
+    "kvq_decode_workspace_bytes", "kvq_decode_attn", "kvq_decode_certified", "kvq_decode_step",
+    "kvq_decode_attn_static", "kvq_dequant_debug", "kvq_sync_status",
     "kvq_status_string",
 )
 
@@ -49,6 +49,19 @@ class kvq_tier2(C.Structure):
     _fields_ = [("k_host", C.c_void_p), ("v_host", C.c_void_p), ("promote_frac", C.c_float)]
 
 
+class kvq_ladder(C.Structure):
+    _fields_ = [(n, C.c_float) for n in ("tau_cov", "max_frac", "key_tol", "v_tol", "rank_tol", "cert_tol",
+                                          "layer_frac")]
+
+
+class kvq_ladder_report(C.Structure):
+    _fields_ = [("k_star", C.c_void_p), ("block_flags", C.c_void_p), ("flags_cols", C.c_int32),
+                ("bound", C.c_void_p), ("status", C.c_void_p)]
+
+
+KVQ_LADDER_EXPANDED, KVQ_LADDER_CAPPED, KVQ_LADDER_VALUES = 1, 2, 4
+KVQ_LADDER_RANK_FAIL, KVQ_LADDER_BOUND_FAIL, KVQ_LADDER_HEAD_DENSE, KVQ_LADDER_LAYER_DENSE = 8, 16, 32, 64
+
 _lib = None
 
 
@@ -71,6 +84,8 @@ def lib() -> C.CDLL:
             "kvq_reset_pages": (i32, [P, P, i32, P]),
             "kvq_decode_workspace_bytes": (sz, [P, i32, i32]),
             "kvq_decode_attn": (i32, [P, P, P, i32, P, i32, C.c_float, C.POINTER(kvq_tier2), P, sz, P, P, P]),
+            "kvq_decode_certified": (i32, [P, P, P, i32, P, i32, C.c_float, P, P, C.POINTER(kvq_ladder), P, sz,
+                                           P, C.POINTER(kvq_ladder_report), P]),
             "kvq_decode_step": (i32, [P, P, P, P, P, P, i32, P, i32, C.c_float, P, sz, P, P]),
             "kvq_decode_attn_static": (i32, [P, P, P, i32, P, i32, C.c_float, P, P]),
             "kvq_dequant_debug": (i32, [P, P, i32, P, P, P, P, P]),
@@ -151,6 +166,16 @@ def kvq_decode_attn(cache, q, block_table, max_pages_per_seq: int, ctx_lens, bat
            lib().kvq_decode_attn(cache, _ptr(q), _ptr(block_table), max_pages_per_seq, _ptr(ctx_lens), batch,
                                  softmax_scale, t2, _ptr(workspace), ws_bytes, _ptr(out), _ptr(promoted_out),
                                  _stream(stream)))
+
+
+def kvq_decode_certified(cache, q, block_table, max_pages_per_seq: int, ctx_lens, batch: int,
+                         softmax_scale: float, k_tier2, v_tier2, policy: kvq_ladder, workspace, ws_bytes: int, out,
+                         report: kvq_ladder_report | None = None, stream=None) -> None:
+    rep = C.byref(report) if report is not None else None
+    _check("kvq_decode_certified",
+           lib().kvq_decode_certified(cache, _ptr(q), _ptr(block_table), max_pages_per_seq, _ptr(ctx_lens), batch,
+                                      softmax_scale, _ptr(k_tier2), _ptr(v_tier2), C.byref(policy), _ptr(workspace),
+                                      ws_bytes, _ptr(out), rep, _stream(stream)))
 
 
 def kvq_decode_step(cache, k_new, v_new, slot_mapping, q, block_table, max_pages_per_seq: int, ctx_lens,
@@ -241,6 +266,35 @@ class Cache:
         device); promoted_out (optional) int32 [B, Hkv, kmax] on the device."""
         t2 = kvq_tier2(k_tier2.data_ptr(), v_tier2.data_ptr(), promote_frac)
         return self.decode(q, block_table, ctx_lens, out, softmax_scale, t2, promoted_out, stream)
+
+    def decode_ladder(self, q, block_table, ctx_lens, k_tier2, v_tier2, tau_cov: float = 0.995,
+                      max_frac: float = 1.0, key_tol: float = float("inf"), v_tol: float = float("inf"),
+                      rank_tol: float = float("inf"), cert_tol: float = float("inf"), layer_frac: float = 1.0,
+                      out=None, report: bool = False, softmax_scale: float = 0.0, stream=None):
+        """Certified decode with the adaptive ladder (kvq_decode_certified).
+        Returns out, or (out, dict of device tensors k_star [B,Hkv],
+        flags [B,Hkv,nb], bound [B,Hq], status [B,Hq]) with report=True."""
+        import torch
+        batch, max_pages = block_table.shape
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        ws = self.workspace_for(batch, max_pages)
+        pol = kvq_ladder(tau_cov, max_frac, key_tol, v_tol, rank_tol, cert_tol, layer_frac)
+        rep, rd = None, None
+        if report:
+            blk = self.cfg.bound_block_tokens
+            nb = max(1, (max_pages * PAGE_TOKENS + blk - 1) // blk)
+            dev = q.device
+            hkv, hq = self.cfg.num_kv_heads, self.cfg.num_q_heads
+            rd = {"k_star": torch.full((batch, hkv), -1, dtype=torch.int32, device=dev),
+                  "flags": torch.full((batch, hkv, nb), 255, dtype=torch.uint8, device=dev),
+                  "bound": torch.full((batch, hq), -1.0, dtype=torch.float32, device=dev),
+                  "status": torch.full((batch, hq), -1, dtype=torch.int32, device=dev)}
+            rep = kvq_ladder_report(rd["k_star"].data_ptr(), rd["flags"].data_ptr(), nb, rd["bound"].data_ptr(),
+                                    rd["status"].data_ptr())
+        kvq_decode_certified(self.handle, q, block_table, max_pages, ctx_lens, batch, softmax_scale, k_tier2,
+                             v_tier2, pol, ws, ws.numel(), out, rep, stream)
+        return (out, rd) if report else out
 
     def step(self, k_new, v_new, slot_mapping, q, block_table, ctx_lens, out=None, softmax_scale: float = 0.0,
              stream=None):

@@ -114,7 +114,9 @@ size_t cert_chunks(int max_pages) { return ((size_t)max_pages + 255) / 256; }
 // per-head totals, promoted-block lists and counts, promote partials and
 // the promote counters (zero between calls).
 struct CertWs {
-    size_t page_stats, head_ml, blk, spart, dq, prom, prom_count, cpart, ccount, bytes;
+    size_t page_stats, head_ml, blk, spart, dq, prom, prom_count, cpart, ccount;
+    size_t flags, bml, mix, gstat, status, bound, nfall, dpart, dcount;  // the ladder
+    size_t bytes;
 };
 
 CertWs cert_ws(const kvq_cache *c, int batch, int max_pages)
@@ -142,8 +144,40 @@ CertWs cert_ws(const kvq_cache *c, int batch, int max_pages)
     off += round256(bk * kCertChunks * g * 2 * (c->L.d + 4) * 4);
     w.ccount = off;
     off += round256(bk * 4);
+    w.flags = off;
+    off += round256(bk * cap);
+    w.bml = off;
+    off += round256(bk * cap * g * 8);
+    w.mix = off;
+    off += round256(bk * g * 8);
+    w.gstat = off;
+    off += round256(bk * 4);
+    w.status = off;
+    off += round256(bk * g * 4);
+    w.bound = off;
+    off += round256(bk * g * 4);
+    w.nfall = off;
+    off += 256;
+    w.dpart = off;
+    off += round256(bk * kDenseSplitsMax * g * (c->L.d + 4) * 4);
+    w.dcount = off;
+    off += round256(bk * 4);
     w.bytes = off;
     return w;
+}
+
+// Dense-fallback split: at most kDenseSplitsMax splits of >= 1024 tokens
+// (a multiple of 64) per (sequence, kv head).
+void dense_split(int max_pages, int *n_split, int *tokens)
+{
+    const long long T = (long long)max_pages * kPageTokens;
+    long long n = (T + 1023) / 1024;
+    if (n > kDenseSplitsMax) n = kDenseSplitsMax;
+    if (n < 1) n = 1;
+    long long per = (T + n - 1) / n;
+    per = (per + 63) / 64 * 64;
+    *n_split = (int)((T + per - 1) / per);
+    *tokens = (int)per;
 }
 
 // A device-accessible address for `p`: device or managed memory as is; pinned
@@ -266,6 +300,82 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *c, int32_t batch, int32_t max
 
 namespace {
 
+DecodeParams decode_params(kvq_cache *c, const SplitPlan &s, const void *q, const int32_t *block_table,
+                           int32_t max_pages, const int32_t *ctx_lens, int32_t batch, float scale, void *workspace,
+                           void *out)
+{
+    DecodeParams p{};
+    p.pool = c->pool;
+    p.q = static_cast<const __half *>(q);
+    p.block_table = block_table;
+    p.ctx_lens = ctx_lens;
+    p.max_pages = max_pages;
+    p.batch = batch;
+    p.L = c->L;
+    p.qscale = scale * 1.4426950408889634f;  // log2(e)
+    p.rot_scale = c->rot_scale;
+    p.rotate = c->cfg.rotate;
+    memcpy(p.signs, c->signs, sizeof(p.signs));
+    p.pages_per_split = s.pages_per_split;
+    p.pages_per_warp = s.pages_per_warp;
+    p.n_splits = s.n_splits;
+    p.counters = static_cast<unsigned int *>(workspace);
+    p.part = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + counters_bytes(batch, c->L.hkv));
+    p.out = static_cast<float *>(out);
+    p.clip = c->cfg.clip_ratio;
+    return p;
+}
+
+// The certified-mode workspace regions start after the decode partials.
+unsigned char *cert_base(const kvq_cache *c, const SplitPlan &s, int batch, void *workspace)
+{
+    return static_cast<unsigned char *>(workspace) + counters_bytes(batch, c->L.hkv) +
+           round256((size_t)batch * c->L.hkv * s.n_splits * c->L.g * (c->L.d + 4) * 4);
+}
+
+CertParams cert_params(const kvq_cache *c, const DecodeParams &p, int max_pages, float scale, unsigned char *base,
+                       const CertWs &w, const void *k2, const void *v2)
+{
+    CertParams cp{};
+    cp.pool = c->pool;
+    cp.q = p.q;
+    cp.block_table = p.block_table;
+    cp.ctx_lens = p.ctx_lens;
+    cp.max_pages = max_pages;
+    cp.L = c->L;
+    cp.scale = scale;
+    cp.qscale = p.qscale;
+    cp.rot_scale = c->rot_scale;
+    cp.rotate = c->cfg.rotate;
+    memcpy(cp.signs, c->signs, sizeof(cp.signs));
+    cp.sort_cap = pow2_at_least(cert_blocks(c, max_pages));
+    cp.page_stats = p.page_stats;
+    cp.head_ml = p.head_ml;
+    cp.blk = reinterpret_cast<float *>(base + w.blk);
+    cp.spart = reinterpret_cast<float *>(base + w.spart);
+    cp.dq = reinterpret_cast<float *>(base + w.dq);
+    cp.n_chunk_cap = (int)cert_chunks(max_pages);
+    cp.prom = reinterpret_cast<int32_t *>(base + w.prom);
+    cp.prom_count = reinterpret_cast<int32_t *>(base + w.prom_count);
+    cp.k2 = static_cast<const __half *>(k2);
+    cp.v2 = static_cast<const __half *>(v2);
+    cp.cpart = reinterpret_cast<float *>(base + w.cpart);
+    cp.ccount = reinterpret_cast<unsigned int *>(base + w.ccount);
+    cp.out = p.out;
+    return cp;
+}
+
+// Certified-mode limits shared by both modes: bound blocks of 16 * 2^k <= 512
+// tokens, at most kCertMaxBlocks per sequence.
+kvq_status cert_shape_ok(const kvq_cache *c, int max_pages)
+{
+    if (c->L.bound_block <= 0) return KVQ_ERR_INVALID_ARG;
+    if (cert_blocks(c, max_pages) > kCertMaxBlocks) return KVQ_ERR_UNSUPPORTED;
+    const int ppb = c->L.bound_block / kPageTokens;  // pages per block: a power of two <= 32
+    if (ppb > 32 || (ppb & (ppb - 1))) return KVQ_ERR_UNSUPPORTED;
+    return KVQ_OK;
+}
+
 kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const int32_t *slot_mapping,
                        const void *q, const int32_t *block_table, int32_t max_pages_per_seq, const int32_t *ctx_lens,
                        int32_t batch, float softmax_scale, const kvq_tier2 *tier2, void *workspace, size_t ws_bytes,
@@ -283,11 +393,9 @@ kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const
     if (tier2) {
         if (k_new || c->L.bound_block <= 0) return KVQ_ERR_INVALID_ARG;
         if (!(tier2->promote_frac >= 0.0f && tier2->promote_frac <= 1.0f)) return KVQ_ERR_INVALID_ARG;
-        const int nb_max = cert_blocks(c, max_pages_per_seq);
-        if (nb_max > kCertMaxBlocks) return KVQ_ERR_UNSUPPORTED;
-        const int ppb = c->L.bound_block / kPageTokens;  // pages per block: a power of two <= 32
-        if (ppb > 32 || (ppb & (ppb - 1))) return KVQ_ERR_UNSUPPORTED;
-        kmax = promote_count(tier2->promote_frac, nb_max);
+        const kvq_status sh = cert_shape_ok(c, max_pages_per_seq);
+        if (sh != KVQ_OK) return sh;
+        kmax = promote_count(tier2->promote_frac, cert_blocks(c, max_pages_per_seq));
         if (kmax > 0) {
             k2 = device_view(tier2->k_host);
             v2 = device_view(tier2->v_host);
@@ -296,80 +404,119 @@ kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const
     }
     if (ws_bytes < kvq_decode_workspace_bytes(c, batch, max_pages_per_seq)) return KVQ_ERR_CAPACITY;
     const SplitPlan s = plan_splits(c, batch, max_pages_per_seq);
-    DecodeParams p{};
-    p.pool = c->pool;
-    p.q = static_cast<const __half *>(q);
-    p.block_table = block_table;
-    p.ctx_lens = ctx_lens;
-    p.max_pages = max_pages_per_seq;
-    p.batch = batch;
-    p.L = c->L;
     const float scale = softmax_scale > 0.0f ? softmax_scale : (float)(1.0 / sqrt((double)c->L.d));
-    p.qscale = scale * 1.4426950408889634f;  // log2(e)
-    p.rot_scale = c->rot_scale;
-    p.rotate = c->cfg.rotate;
-    memcpy(p.signs, c->signs, sizeof(p.signs));
-    p.pages_per_split = s.pages_per_split;
-    p.pages_per_warp = s.pages_per_warp;
-    p.n_splits = s.n_splits;
-    p.counters = static_cast<unsigned int *>(workspace);
-    p.part = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + counters_bytes(batch, c->L.hkv));
-    p.out = static_cast<float *>(out);
+    DecodeParams p = decode_params(c, s, q, block_table, max_pages_per_seq, ctx_lens, batch, scale, workspace, out);
     p.new_k = static_cast<const __half *>(k_new);
     p.new_v = static_cast<const __half *>(v_new);
     p.new_slots = slot_mapping;
-    p.clip = c->cfg.clip_ratio;
     c->last_stream = stream;
     const dim3 grid(s.n_splits, c->L.hkv, batch);
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
-    unsigned char *cert_base = static_cast<unsigned char *>(workspace) + counters_bytes(batch, c->L.hkv) +
-                               round256((size_t)batch * c->L.hkv * s.n_splits * c->L.g * (c->L.d + 4) * 4);
+    unsigned char *base = cert_base(c, s, batch, workspace);
     const CertWs w = cert_ws(c, batch, max_pages_per_seq);
     if (kmax > 0) {
-        p.page_stats = reinterpret_cast<float2 *>(cert_base + w.page_stats);
-        p.head_ml = reinterpret_cast<float2 *>(cert_base + w.head_ml);
+        p.page_stats = reinterpret_cast<float2 *>(base + w.page_stats);
+        p.head_ml = reinterpret_cast<float2 *>(base + w.head_ml);
     }
     kvq_status rc = cuda_status(launch_decode(p, grid, st));
     if (rc != KVQ_OK || kmax == 0) return rc;
 
-    CertParams cp{};
-    cp.pool = c->pool;
-    cp.q = p.q;
-    cp.block_table = block_table;
-    cp.ctx_lens = ctx_lens;
-    cp.max_pages = max_pages_per_seq;
-    cp.L = c->L;
-    cp.scale = scale;
-    cp.qscale = p.qscale;
-    cp.rot_scale = c->rot_scale;
-    cp.rotate = c->cfg.rotate;
-    memcpy(cp.signs, c->signs, sizeof(cp.signs));
+    CertParams cp = cert_params(c, p, max_pages_per_seq, scale, base, w, k2, v2);
     cp.frac = tier2->promote_frac;
-    cp.sort_cap = pow2_at_least(cert_blocks(c, max_pages_per_seq));
     cp.kmax_out = kmax;
     cp.n_chunks = kmax < kCertChunks ? kmax : kCertChunks;
-    cp.page_stats = p.page_stats;
-    cp.head_ml = p.head_ml;
-    cp.blk = reinterpret_cast<float *>(cert_base + w.blk);
-    cp.spart = reinterpret_cast<float *>(cert_base + w.spart);
-    cp.dq = reinterpret_cast<float *>(cert_base + w.dq);
-    cp.n_chunk_cap = (int)cert_chunks(max_pages_per_seq);
-    cp.prom = reinterpret_cast<int32_t *>(cert_base + w.prom);
-    cp.prom_count = reinterpret_cast<int32_t *>(cert_base + w.prom_count);
     cp.promoted_out = promoted_out;
-    cp.k2 = static_cast<const __half *>(k2);
-    cp.v2 = static_cast<const __half *>(v2);
-    cp.cpart = reinterpret_cast<float *>(cert_base + w.cpart);
-    cp.ccount = reinterpret_cast<unsigned int *>(cert_base + w.ccount);
-    cp.out = p.out;
+    rc = cuda_status(launch_cert_blocks(cp, batch, st));
+    if (rc != KVQ_OK) return rc;
     rc = cuda_status(launch_cert_select(cp, batch, st));
     if (rc != KVQ_OK) return rc;
     return cuda_status(launch_cert_promote(cp, batch, st));
 }
 
+bool in_unit(float x) { return x >= 0.0f && x <= 1.0f; }  // false for NaN
+bool non_negative(float x) { return x >= 0.0f; }          // +inf allowed, NaN not
+
+kvq_status ladder_impl(kvq_cache *c, const void *q, const int32_t *block_table, int32_t max_pages,
+                       const int32_t *ctx_lens, int32_t batch, float softmax_scale, const void *k_tier2,
+                       const void *v_tier2, const kvq_ladder *pol, void *workspace, size_t ws_bytes, void *out,
+                       const kvq_ladder_report *rep, void *stream)
+{
+    if (!c || batch < 0 || max_pages < 1 || !pol) return KVQ_ERR_INVALID_ARG;
+    if (batch == 0) return KVQ_OK;
+    if (!q || !block_table || !ctx_lens || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
+    if (!decode_supported(c->L)) return KVQ_ERR_UNSUPPORTED;
+    const kvq_status sh = cert_shape_ok(c, max_pages);
+    if (sh != KVQ_OK) return sh;
+    if (!in_unit(pol->tau_cov) || !in_unit(pol->max_frac) || !in_unit(pol->layer_frac) ||
+        !non_negative(pol->key_tol) || !non_negative(pol->v_tol) || !non_negative(pol->rank_tol) ||
+        !non_negative(pol->cert_tol))
+        return KVQ_ERR_INVALID_ARG;
+    const int nb_max = cert_blocks(c, max_pages);
+    if (rep && rep->block_flags && rep->flags_cols < nb_max) return KVQ_ERR_INVALID_ARG;
+    const void *k2 = device_view(k_tier2), *v2 = device_view(v_tier2);
+    if (!k2 || !v2 || !aligned(k2, 16) || !aligned(v2, 16)) return KVQ_ERR_INVALID_ARG;
+    if (ws_bytes < kvq_decode_workspace_bytes(c, batch, max_pages)) return KVQ_ERR_CAPACITY;
+
+    const SplitPlan s = plan_splits(c, batch, max_pages);
+    const float scale = softmax_scale > 0.0f ? softmax_scale : (float)(1.0 / sqrt((double)c->L.d));
+    DecodeParams p = decode_params(c, s, q, block_table, max_pages, ctx_lens, batch, scale, workspace, out);
+    unsigned char *base = cert_base(c, s, batch, workspace);
+    const CertWs w = cert_ws(c, batch, max_pages);
+    p.page_stats = reinterpret_cast<float2 *>(base + w.page_stats);
+    p.head_ml = reinterpret_cast<float2 *>(base + w.head_ml);
+    c->last_stream = stream;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    kvq_status rc = cuda_status(launch_decode(p, dim3(s.n_splits, c->L.hkv, batch), st));
+    if (rc != KVQ_OK) return rc;
+
+    CertParams cp = cert_params(c, p, max_pages, scale, base, w, k2, v2);
+    cp.ladder = 1;
+    cp.frac = pol->max_frac;
+    cp.n_chunks = kCertChunks;
+    cp.tau_cov = pol->tau_cov;
+    cp.key_tol = pol->key_tol;
+    cp.v_tol = pol->v_tol;
+    cp.rank_tol = pol->rank_tol;
+    cp.cert_tol = pol->cert_tol;
+    // more than layer_frac * batch * Hq heads <=> more than its floor (an integer count)
+    cp.layer_thresh = (int)floor((double)pol->layer_frac * (double)batch * (double)c->L.hq);
+    cp.flags = base + w.flags;
+    cp.bml = reinterpret_cast<float2 *>(base + w.bml);
+    cp.mix = reinterpret_cast<float2 *>(base + w.mix);
+    cp.gstat = reinterpret_cast<int32_t *>(base + w.gstat);
+    cp.status = reinterpret_cast<int32_t *>(base + w.status);
+    cp.bound = reinterpret_cast<float *>(base + w.bound);
+    cp.nfall = reinterpret_cast<unsigned int *>(base + w.nfall);
+    if (rep) {
+        cp.k_star_out = rep->k_star;
+        cp.flags_out = rep->block_flags;
+        cp.nb_out = rep->block_flags ? rep->flags_cols : 0;
+        cp.bound_out = rep->bound;
+        cp.status_out = rep->status;
+    }
+    dense_split(max_pages, &cp.n_dsplit, &cp.dsplit_tokens);
+    cp.dpart = reinterpret_cast<float *>(base + w.dpart);
+    cp.dcount = reinterpret_cast<unsigned int *>(base + w.dcount);
+    rc = cuda_status(launch_cert_blocks(cp, batch, st));
+    if (rc == KVQ_OK) rc = cuda_status(launch_ladder_select(cp, batch, st));
+    if (rc == KVQ_OK) rc = cuda_status(launch_cert_promote(cp, batch, st));
+    if (rc == KVQ_OK) rc = cuda_status(launch_ladder_finish(cp, batch, st));
+    return rc;
+}
+
 }  // namespace
 
 extern "C" {
+
+kvq_status kvq_decode_certified(kvq_cache *c, const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
+                                const int32_t *ctx_lens, int32_t batch, float softmax_scale, const void *k_tier2,
+                                const void *v_tier2, const kvq_ladder *policy, void *workspace, size_t ws_bytes,
+                                void *out, const kvq_ladder_report *report, void *stream)
+{
+    return ladder_impl(c, q, block_table, max_pages_per_seq, ctx_lens, batch, softmax_scale, k_tier2, v_tier2, policy,
+                       workspace, ws_bytes, out, report, stream);
+}
 
 kvq_status kvq_decode_attn(kvq_cache *c, const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
                            const int32_t *ctx_lens, int32_t batch, float softmax_scale, const kvq_tier2 *tier2,

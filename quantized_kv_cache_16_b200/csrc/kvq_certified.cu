@@ -29,65 +29,14 @@
 //                 / (L 2^(M-R) + l_e 2^(m_e-R) - l_q 2^(m_q-R)).
 #include <math.h>
 
-#include "kvq_internal.cuh"
-#include "kvq_warp.cuh"
+#include "kvq_cert.cuh"
 
 namespace kvq {
 namespace {
 
-constexpr int kSelThreads = 512;
+using namespace cert;
+
 constexpr int kBlkThreads = 256;  // pages per CTA of the blocks kernel
-constexpr int kBlkRec = 12;   // block record: P[8], eps, eta, nu, pad
-constexpr int kPromWarps = 8;
-constexpr int kPromThreads = kPromWarps * 32;
-constexpr int kTokBatch = 8;       // tokens whose exact rows a warp has in flight
-
-// Programmatic dependent launch: wait for the stream's previous grid to
-// complete (its writes visible) before any memory access, then allow the next
-// grid to be set up; only launch latency is hidden, no work overlaps.
-__device__ __forceinline__ void pdl_enter()
-{
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-template <typename Kern>
-cudaError_t launch_pdl(Kern kernel, dim3 grid, int threads, size_t smem, cudaStream_t s, const CertParams &p)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, p);
-}
-
-__device__ __forceinline__ int clamp_ctx(int T, int max_pages)
-{
-    return T < 0 ? 0 : (T > max_pages * kPageTokens ? max_pages * kPageTokens : T);
-}
-
-// The rotated query row of head (b, head) in lane order: element lane*E + e.
-template <int D>
-__device__ __forceinline__ void rotated_query(const CertParams &p, int b, int head, int lane, float (&x)[D / 32])
-{
-    constexpr int E = D / 32;
-    const __half *qh = p.q + ((long long)b * p.L.hq + head) * D + lane * E;
-#pragma unroll
-    for (int e = 0; e < E; e++) x[e] = __half2float(qh[e]);
-    if (p.rotate) {
-#pragma unroll
-        for (int e = 0; e < E; e++) x[e] *= p.signs[lane * E + e];
-        fwht_warp<D>(x, lane);
-#pragma unroll
-        for (int e = 0; e < E; e++) x[e] *= p.rot_scale;
-    }
-}
 
 // Pass 1, one thread per (page, query head), pages of a bound block in
 // consecutive lanes: the page's softmax mass l 2^(m - M) / L and its
@@ -222,66 +171,11 @@ __global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_c
 #pragma unroll
             for (int h = 0; h < kMaxGqa; h++)
                 if (h < g && P[h] > 0.f) sc = fmaxf(sc, P[h] * fmaf(expm1f(fmaf(dq[h], d.x, A[h])), d.z, d.y));
-            if (!(sc >= 0.f)) sc = 0.f;
-            key = ((unsigned long long)__float_as_uint(sc) << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)bb);
+            key = sort_key(sc, bb);
         }
         keys[bb] = key;
     }
-    __syncthreads();
-
-    // bitonic sort of the keys, descending
-    if (np2 <= 2 * kSelThreads) {
-        // keys tid and tid + kSelThreads in registers: stages whose partner is
-        // under 32 keys away are warp shuffles, the others go through shared
-        // memory (indices >= np2 only ever meet each other)
-        unsigned long long v[2];
-#pragma unroll
-        for (int c = 0; c < 2; c++) v[c] = tid + c * kSelThreads < np2 ? keys[tid + c * kSelThreads] : 0ull;
-        for (int k = 2; k <= np2; k <<= 1)
-            for (int jj = k >> 1; jj > 0; jj >>= 1) {
-                unsigned long long o[2];
-                if (jj >= 32) {
-                    __syncthreads();  // the last stage's reads are done
-#pragma unroll
-                    for (int c = 0; c < 2; c++)
-                        if (tid + c * kSelThreads < np2) keys[tid + c * kSelThreads] = v[c];
-                    __syncthreads();
-#pragma unroll
-                    for (int c = 0; c < 2; c++) o[c] = tid + c * kSelThreads < np2 ? keys[(tid + c * kSelThreads) ^ jj] : 0ull;
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 2; c++) o[c] = __shfl_xor_sync(kFull, v[c], jj);
-                }
-#pragma unroll
-                for (int c = 0; c < 2; c++) {
-                    const int i = tid + c * kSelThreads;
-                    const bool lower = (i & jj) == 0, desc = (i & k) == 0;
-                    const unsigned long long hi = v[c] > o[c] ? v[c] : o[c], lo = v[c] > o[c] ? o[c] : v[c];
-                    v[c] = (lower == desc) ? hi : lo;
-                }
-            }
-        __syncthreads();
-#pragma unroll
-        for (int c = 0; c < 2; c++)
-            if (tid + c * kSelThreads < np2) keys[tid + c * kSelThreads] = v[c];
-        __syncthreads();
-    } else {
-        for (int k = 2; k <= np2; k <<= 1)
-            for (int jj = k >> 1; jj > 0; jj >>= 1) {
-                for (int i = tid; i < np2; i += kSelThreads) {
-                    const int ixj = i ^ jj;
-                    if (ixj > i) {
-                        const unsigned long long a = keys[i], c = keys[ixj];
-                        const bool desc = (i & k) == 0;
-                        if (desc ? (a < c) : (a > c)) {
-                            keys[i] = c;
-                            keys[ixj] = a;
-                        }
-                    }
-                }
-                __syncthreads();
-            }
-    }
+    sort_keys_desc<kSelThreads>(keys, np2, tid);
 
     // the top ceil(frac * nb) blocks (fp64, guarded so an exact product is not bumped up)
     int kp = 0;
@@ -290,84 +184,12 @@ __global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_c
         kp = kp < 0 ? 0 : (kp > nb ? nb : kp);
     }
     int32_t *prom = p.prom + bk * p.sort_cap;
-    for (int r = tid; r < kp; r += kSelThreads) prom[r] = (int)(0xFFFFFFFFu - (unsigned)(keys[r] & 0xFFFFFFFFull));
+    for (int r = tid; r < kp; r += kSelThreads) prom[r] = key_index(keys[r]) | kPromKey | kPromVal;
     if (p.promoted_out)
         for (int r = tid; r < p.kmax_out; r += kSelThreads)
-            p.promoted_out[bk * p.kmax_out + r] =
-                r < kp ? (int)(0xFFFFFFFFu - (unsigned)(keys[r] & 0xFFFFFFFFull)) : -1;
+            p.promoted_out[bk * p.kmax_out + r] = r < kp ? key_index(keys[r]) : -1;
     if (tid == 0) p.prom_count[bk] = kp;
 }
-
-// Dequantised values of channels lane*E .. lane*E+E-1 of token `tok` in a
-// chunk (the same arithmetic as the stored codec: code*scale + zero, one
-// rounding; int8: code*scale).  The lane's codes are E*bits consecutive bits
-// of the token's stream (4, 8, 16 or 32 bits, aligned to their size, inside
-// one 16-byte chunk): one load, then shifts.
-template <int E>
-__device__ __forceinline__ void dequant_lane(const unsigned char *chunk, int codes_off, int meta_off, int row_meta,
-                                             int fmt, int tok, int lane, float (&x)[E])
-{
-    const unsigned char *codes = chunk + codes_off;
-    const uint16_t *meta = reinterpret_cast<const uint16_t *>(chunk + meta_off + tok * row_meta);
-    const int bits = fmt_bits(fmt);
-    const int bit0 = lane * E * bits, byte0 = bit0 >> 3;
-    const unsigned char *src = codes + ((byte0 >> 4) * 16 + tok) * 16 + (byte0 & 15);
-    const int nbits = E * bits;
-    uint32_t w;
-    if (nbits == 32) w = *reinterpret_cast<const uint32_t *>(src);
-    else if (nbits == 16) w = *reinterpret_cast<const uint16_t *>(src);
-    else w = *src >> (bit0 & 7);
-    const uint32_t mask = (1u << bits) - 1u;
-    if (fmt == KVQ_INT8_SYM) {
-        const float s = __half2float(__ushort_as_half(meta[0]));
-#pragma unroll
-        for (int e = 0; e < E; e++) x[e] = __fmul_rn((float)(int)(int8_t)((w >> (8 * e)) & 0xFFu), s);
-    } else {
-        const int ng = row_meta / 4;  // asymmetric formats: scales then zeros
-        const int gi = fmt == KVQ_INT4_ASYM ? (lane * E) / 32 : 0;
-        const float s = __half2float(__ushort_as_half(meta[gi])), z = __half2float(__ushort_as_half(meta[ng + gi]));
-#pragma unroll
-        for (int e = 0; e < E; e++) x[e] = __fmaf_rn((float)((w >> (bits * e)) & mask), s, z);
-    }
-}
-
-template <int E>
-__device__ __forceinline__ void online_update(float &m, float &l, float (&a)[E], float s, const float (&v)[E])
-{
-    const float mn = fmaxf(m, s);
-    const float al = (m == -INFINITY) ? 0.f : ex2(m - mn);
-    const float pe = ex2(s - mn);
-    l = fmaf(l, al, pe);
-#pragma unroll
-    for (int e = 0; e < E; e++) a[e] = fmaf(a[e], al, pe * v[e]);
-    m = mn;
-}
-
-// A lane's E fp16 values of a row, kept raw (the loads stay in flight in
-// half the registers) and widened when used.
-template <int E> struct RawRow;
-template <> struct RawRow<4> {
-    uint2 u;
-    __device__ void load(const __half *src) { u = *reinterpret_cast<const uint2 *>(src); }
-    __device__ void widen(float (&x)[4]) const
-    {
-        const float2 a = __half22float2(bits_h2(u.x)), c = __half22float2(bits_h2(u.y));
-        x[0] = a.x;
-        x[1] = a.y;
-        x[2] = c.x;
-        x[3] = c.y;
-    }
-};
-template <> struct RawRow<2> {
-    uint32_t u;
-    __device__ void load(const __half *src) { u = *reinterpret_cast<const uint32_t *>(src); }
-    __device__ void widen(float (&x)[2]) const
-    {
-        const float2 a = __half22float2(bits_h2(u));
-        x[0] = a.x;
-        x[1] = a.y;
-    }
-};
 
 template <int D>
 __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid_constant__ CertParams p)
@@ -419,8 +241,22 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
             for (int e = 0; e < E; e++) acc[h][w][e] = 0.f;
         }
 
-    for (int r = chunk_id; r < kp; r += n_act) {
-        const int t0 = prom[r] * block, t1 = min(t0 + block, T);
+    // per warp and head, (m, l) of a key-promoted block's exact scores over
+    // the warp's share of its tokens (the ladder's ranking check); two
+    // buffers, a barrier every block
+    __shared__ float2 bsm[2][kPromWarps][kMaxGqa];
+    int parity = 0;
+    for (int r = chunk_id; r < kp; r += n_act, parity ^= 1) {
+        const int ent = prom[r];
+        const int blk_id = ent & kPromIdx;
+        const bool kx = (ent & kPromKey) != 0, vx = (ent & kPromVal) != 0;
+        const int t0 = blk_id * block, t1 = min(t0 + block, T);
+        float bm[kMaxGqa], bl[kMaxGqa];
+#pragma unroll
+        for (int h = 0; h < kMaxGqa; h++) {
+            bm[h] = -INFINITY;
+            bl[h] = 0.f;
+        }
         for (int tb = t0 + warp * kTokBatch; tb < t1; tb += kPromWarps * kTokBatch) {
             // issue the batch's exact-row loads (host link) before any math
             RawRow<E> kraw[kTokBatch], vraw[kTokBatch];
@@ -436,53 +272,82 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
                 pgs[u] = pg;
                 if (pg >= 0) {
                     const long long row = ((long long)(pg * kPageTokens + t % kPageTokens) * L.hkv + kvh) * D + lane * E;
-                    kraw[u].load(p.k2 + row);
-                    vraw[u].load(p.v2 + row);
+                    if (kx) kraw[u].load(p.k2 + row);
+                    if (vx) vraw[u].load(p.v2 + row);
                 }
             }
 #pragma unroll
             for (int u = 0; u < kTokBatch; u++) {
                 if (pgs[u] < 0) continue;  // warp-uniform
                 const int tok = (tb + u) % kPageTokens;
-                float ke[E], ve[E];
-                kraw[u].widen(ke);
-                vraw[u].widen(ve);
+                const unsigned char *chunk =
+                    p.pool + kHeaderBytes + (long long)pgs[u] * L.page_bytes + (long long)kvh * L.chunk_bytes;
+                float kq[E], vq[E], ke[E] = {}, ve[E] = {};
+                // exact rows, rotated (both together when both are exact)
+                if (kx) kraw[u].widen(ke);
+                if (vx) vraw[u].widen(ve);
                 if (p.rotate) {
 #pragma unroll
                     for (int e = 0; e < E; e++) {
                         ke[e] *= p.signs[lane * E + e];
                         ve[e] *= p.signs[lane * E + e];
                     }
-                    fwht_warp<D>(ke, lane);
-                    fwht_warp<D>(ve, lane);
+                    if (kx && vx) fwht_warp2<D>(ke, ve, lane);
+                    else if (kx) fwht_warp<D>(ke, lane);
+                    else if (vx) fwht_warp<D>(ve, lane);
 #pragma unroll
                     for (int e = 0; e < E; e++) {
                         ke[e] *= p.rot_scale;
                         ve[e] *= p.rot_scale;
                     }
                 }
-                const unsigned char *chunk =
-                    p.pool + kHeaderBytes + (long long)pgs[u] * L.page_bytes + (long long)kvh * L.chunk_bytes;
-                float kq[E], vq[E];
                 dequant_lane<E>(chunk, L.k_codes, L.k_meta, L.k_row_meta, L.k_fmt, tok, lane, kq);
                 dequant_lane<E>(chunk, L.v_codes, L.v_meta, L.v_row_meta, L.v_fmt, tok, lane, vq);
+                if (!vx)
+#pragma unroll
+                    for (int e = 0; e < E; e++) ve[e] = vq[e];
 #pragma unroll
                 for (int h = 0; h < kMaxGqa; h++) {
                     if (h >= g) break;
                     float se = 0.f, sqv = 0.f;
 #pragma unroll
-                    for (int e = 0; e < E; e++) {
-                        se = fmaf(qr[h][e], ke[e], se);
-                        sqv = fmaf(qr[h][e], kq[e], sqv);
+                    for (int e = 0; e < E; e++) sqv = fmaf(qr[h][e], kq[e], sqv);
+                    if (kx) {
+#pragma unroll
+                        for (int e = 0; e < E; e++) se = fmaf(qr[h][e], ke[e], se);
                     }
 #pragma unroll
                     for (int mm = 16; mm >= 1; mm >>= 1) {
-                        se += __shfl_xor_sync(kFull, se, mm);
                         sqv += __shfl_xor_sync(kFull, sqv, mm);
+                        if (kx) se += __shfl_xor_sync(kFull, se, mm);
                     }
+                    if (!kx) se = sqv;
                     online_update<E>(m[h][0], l[h][0], acc[h][0], se, ve);
                     online_update<E>(m[h][1], l[h][1], acc[h][1], sqv, vq);
+                    if (p.ladder && kx) {
+                        const float mn = fmaxf(bm[h], se);
+                        bl[h] = fmaf(bl[h], ex2(bm[h] - mn), ex2(se - mn));
+                        bm[h] = mn;
+                    }
                 }
+            }
+        }
+        if (p.ladder) {  // CTA-uniform
+            if (kx && lane == 0)
+#pragma unroll
+                for (int h = 0; h < kMaxGqa; h++)
+                    if (h < g) bsm[parity][warp][h] = make_float2(bm[h], bl[h]);
+            __syncthreads();
+            if (kx && warp == 0 && lane < g) {
+                float M = -INFINITY, Ls = 0.f;
+#pragma unroll
+                for (int w = 0; w < kPromWarps; w++) M = fmaxf(M, bsm[parity][w][lane].x);
+#pragma unroll
+                for (int w = 0; w < kPromWarps; w++) {
+                    const float2 v = bsm[parity][w][lane];
+                    if (v.x != -INFINITY) Ls = fmaf(v.y, ex2(v.x - M), Ls);
+                }
+                p.bml[((long long)bk * p.sort_cap + blk_id) * g + lane] = make_float2(M, Ls);
             }
         }
     }
@@ -576,6 +441,7 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
         const float fe = Mx[0] == -INFINITY ? 0.f : ex2(Mx[0] - R);
         const float fq = Mx[1] == -INFINITY ? 0.f : ex2(Mx[1] - R);
         const float den = f0 + Ls[0] * fe - Ls[1] * fq;
+        if (p.ladder && lane == 0) p.mix[bk * g + h] = make_float2(R, den);
         float dlt[E];
 #pragma unroll
         for (int e = 0; e < E; e++) dlt[e] = a[0][e] * fe - a[1][e] * fq;
@@ -592,6 +458,13 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
 
 }  // namespace
 
+cudaError_t launch_cert_blocks(const CertParams &p, int batch, cudaStream_t s)
+{
+    const dim3 bgrid(p.n_chunk_cap, p.L.hkv * p.L.g, batch);
+    return p.L.d == 128 ? launch_pdl(cert_blocks_kernel<128>, bgrid, kBlkThreads, 0, s, p)
+                        : launch_pdl(cert_blocks_kernel<64>, bgrid, kBlkThreads, 0, s, p);
+}
+
 cudaError_t launch_cert_select(const CertParams &p, int batch, cudaStream_t s)
 {
     static bool configured[2] = {false, false};
@@ -606,10 +479,6 @@ cudaError_t launch_cert_select(const CertParams &p, int batch, cudaStream_t s)
         if (e != cudaSuccess) return e;
         configured[di] = true;
     }
-    const dim3 bgrid(p.n_chunk_cap, p.L.hkv * p.L.g, batch);
-    const cudaError_t e = di ? launch_pdl(cert_blocks_kernel<128>, bgrid, kBlkThreads, 0, s, p)
-                             : launch_pdl(cert_blocks_kernel<64>, bgrid, kBlkThreads, 0, s, p);
-    if (e != cudaSuccess) return e;
     const dim3 grid(p.L.hkv, batch);
     return di ? launch_pdl(cert_select_kernel<128>, grid, kSelThreads, smem, s, p)
               : launch_pdl(cert_select_kernel<64>, grid, kSelThreads, smem, s, p);

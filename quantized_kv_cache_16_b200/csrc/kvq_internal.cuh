@@ -174,15 +174,47 @@ struct CertParams {
     float *cpart;              // [B][Hkv][n_chunks][g][2][d + 4]: exact / quantised block partials
     unsigned int *ccount;      // [B][Hkv], zero between calls
     float *out;                // [B][Hq][d]
+
+    // adaptive ladder ["Runtime-Certified...", Methodology 3]; frac is then
+    // the budget of key-promoted blocks.  prom entries carry flags in bits
+    // 24-25 (kPromKey, kPromVal); the fixed-fraction mode promotes both.
+    int ladder;
+    float tau_cov, key_tol, v_tol, rank_tol, cert_tol;
+    int layer_thresh;          // every head falls back when more than this many do on their own
+    unsigned char *flags;      // [B][Hkv][sort_cap]: bit 0 key exact, bit 1 value exact
+    float2 *bml;               // [B][Hkv][sort_cap][g]: (m, l) of key-promoted blocks' exact scores, log2 units
+    float2 *mix;               // [B][Hkv][g]: (R, den) of the mixed output's softmax (promote's merge)
+    int32_t *gstat;            // [B][Hkv]: group status bits and K* (bits 16+)
+    int32_t *status;           // [B][Hq]: status bits of each head
+    float *bound;              // [B][Hq]: certified bound of each head's mixed output
+    unsigned int *nfall;       // heads that fell back on their own (one counter)
+    int32_t *k_star_out;       // optional [B][Hkv]
+    unsigned char *flags_out;  // optional [B][Hkv][nb_out]
+    int nb_out;
+    float *bound_out;          // optional [B][Hq]
+    int32_t *status_out;       // optional [B][Hq]
+    int n_dsplit, dsplit_tokens;  // dense fallback: splits per (sequence, kv head) and tokens per split
+    float *dpart;              // [B][Hkv][n_dsplit][g][d + 4]
+    unsigned int *dcount;      // [B][Hkv], zero between calls
 };
+
+constexpr int kPromKey = 1 << 24, kPromVal = 1 << 25, kPromIdx = (1 << 24) - 1;
+constexpr int kDenseSplitsMax = 64;
+
+// ladder status bits (kvq.h: KVQ_LADDER_*)
+constexpr int kStExpanded = 1, kStCapped = 2, kStValues = 4, kStRankFail = 8, kStBoundFail = 16,
+              kStHeadDense = 32, kStLayerDense = 64;
 
 // launchers (return cudaGetLastError() of the launch)
 cudaError_t launch_append(const AppendParams &p, int num_sms, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, dim3 grid, cudaStream_t s);
 cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
 cudaError_t launch_reset_pages(unsigned char *pool, Layout L, const int32_t *pages, int n, cudaStream_t s);
+cudaError_t launch_cert_blocks(const CertParams &p, int batch, cudaStream_t s);
 cudaError_t launch_cert_select(const CertParams &p, int batch, cudaStream_t s);
 cudaError_t launch_cert_promote(const CertParams &p, int batch, cudaStream_t s);
+cudaError_t launch_ladder_select(const CertParams &p, int batch, cudaStream_t s);
+cudaError_t launch_ladder_finish(const CertParams &p, int batch, cudaStream_t s);
 bool decode_supported(const Layout &L);
 int decode_max_splits(const Layout &L);
 constexpr int kDecodeWarps = 8;

@@ -41,4 +41,30 @@ __device__ __forceinline__ void fwht_warp(float (&x)[D / 32], int lane)
         }
 }
 
+// Two vectors transformed together (independent shuffle chains interleave).
+template <int D>
+__device__ __forceinline__ void fwht_warp2(float (&x)[D / 32], float (&y)[D / 32], int lane)
+{
+    constexpr int E = D / 32;
+#pragma unroll
+    for (int h = 1; h < E; h <<= 1)
+#pragma unroll
+        for (int e = 0; e < E; e++)
+            if (!(e & h)) {
+                const float a = x[e], b = x[e + h], c = y[e], d = y[e + h];
+                x[e] = a + b;
+                x[e + h] = a - b;
+                y[e] = c + d;
+                y[e + h] = c - d;
+            }
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1)
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            const float o = __shfl_xor_sync(kFull, x[e], m), q = __shfl_xor_sync(kFull, y[e], m);
+            x[e] = (lane & m) ? (o - x[e]) : (x[e] + o);
+            y[e] = (lane & m) ? (q - y[e]) : (y[e] + q);
+        }
+}
+
 }  // namespace kvq

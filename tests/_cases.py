@@ -41,7 +41,7 @@ class Pair:
         return torch.tensor([t + extra for t in self.wl.ctx], dtype=torch.int32, device="cuda")
 
 
-def build_pair(wl: W.Workload, extra_tokens: int = 0, rotate: int = 1, oracle: bool = True) -> Pair:
+def build_pair(wl: W.Workload, extra_tokens: int = 0, rotate: int = 1, oracle: bool = True, kv_rows=None) -> Pair:
     import torch
     import quantized_kv_cache_16_b200 as K
     pages = W.page_table(wl, extra_tokens=extra_tokens)[0]
@@ -50,7 +50,7 @@ def build_pair(wl: W.Workload, extra_tokens: int = 0, rotate: int = 1, oracle: b
     opool = O.new_pool(ocfg) if oracle else None
     kv = []
     for b in range(wl.B):
-        k, v = W.prefix_kv(wl, b)
+        k, v = W.prefix_kv(wl, b) if kv_rows is None else kv_rows[b]
         slots = pages.slots(b, 0, wl.ctx[b])
         if len(slots):
             cache.append(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(), torch.from_numpy(slots).cuda())

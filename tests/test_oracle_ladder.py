@@ -278,6 +278,10 @@ def test_ranking_check_catches_a_tampered_tier2_store():
     assert np.all(loose["status"] & O.LADDER_RANK_FAIL == 0)
     tight = _run(wl, cfg, pool, pages, bad, vs, q, tau_cov=1.0, rank_tol=ratio * 0.999 - 1.0)
     assert np.all(tight["status"] & O.LADDER_RANK_FAIL)
+    # the margin is that ratio (the swap is the only inversion); with the true
+    # store every promoted block keeps its place
+    assert np.allclose(r["rank_margin"], ratio - 1.0, rtol=1e-12, atol=0)
+    assert np.all(clean["rank_margin"] == 0.0)
     # outside the promoted set the check sees nothing: promote only block 3 (the heaviest)
     one = _run(wl, cfg, pool, pages, bad, vs, q, tau_cov=0.01, rank_tol=0.0)
     assert np.all(one["k_star"] == 1) and np.all(one["status"] & O.LADDER_RANK_FAIL == 0)

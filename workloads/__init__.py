@@ -23,7 +23,7 @@ Recipes (numpy ``default_rng``; every stream is keyed by (seed, stream id)):
               u; the keys of "hot" tokens -- the first 16 (sink), six needle
               spans of 64 tokens at seeded positions, the last 128 -- get
               a*u added with a ~ U[10, 14] (then rounded to fp16); queries are
-              N(0,1) + 10*u of their kv head.
+              N(0,1) + 14*u of their kv head.
   int2        prefill of 65536 tokens x 8 kv heads x d=128 per sequence, K and
               V ~ Laplace(0,1) with 1% of elements x30; 2-bit g128, clip 0.9;
               decode B=4, Hq=32, T=65536 (four independent prefills).
@@ -42,7 +42,7 @@ PAGE_TOKENS = 16
 # stream ids
 _S_K, _S_V, _S_Q, _S_LEN, _S_PERM, _S_OUT, _S_NEWK, _S_NEWV, _S_DIR, _S_HOT = range(10)
 
-NEEDLES, NEEDLE_LEN, SINK_LEN, RECENT_LEN, QUERY_PULL = 6, 64, 16, 128, 10.0
+NEEDLES, NEEDLE_LEN, SINK_LEN, RECENT_LEN, QUERY_PULL = 6, 64, 16, 128, 14.0
 
 
 @dataclass
