@@ -141,7 +141,7 @@ CertWs cert_ws(const kvq_cache *c, int batch, int max_pages)
     w.prom_count = off;
     off += round256(bk * 4);
     w.cpart = off;
-    off += round256(bk * kCertChunks * g * 2 * (c->L.d + 4) * 4);
+    off += round256(bk * kCertChunks * g * (3 * c->L.d + 4) * 4);
     w.ccount = off;
     off += round256(bk * 4);
     w.flags = off;
@@ -496,6 +496,8 @@ kvq_status ladder_impl(kvq_cache *c, const void *q, const int32_t *block_table, 
         cp.status_out = rep->status;
     }
     dense_split(max_pages, &cp.n_dsplit, &cp.dsplit_tokens);
+    cp.batch = batch;
+    cp.dense_ctas = c->num_sms;  // one 256-thread CTA per SM fits the kernel's registers
     cp.dpart = reinterpret_cast<float *>(base + w.dpart);
     cp.dcount = reinterpret_cast<unsigned int *>(base + w.dcount);
     rc = cuda_status(launch_cert_blocks(cp, batch, st));

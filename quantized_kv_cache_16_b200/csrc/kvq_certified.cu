@@ -191,7 +191,12 @@ __global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_c
     if (tid == 0) p.prom_count[bk] = kp;
 }
 
-template <int D>
+// Recomputation of the promoted blocks, up to n_chunks CTAs per (sequence,
+// kv head), G >= the GQA group (a power of two).  Exact rows stay in the
+// original domain: an exact key's score is q.k there (equal to (Rq).(Rk),
+// R orthogonal) and exact values are summed unrotated; only the dequantised
+// rows live in the rotated domain.
+template <int D, int G>
 __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid_constant__ CertParams p)
 {
     pdl_enter();
@@ -205,9 +210,13 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
     const int n_act = min(kp, p.n_chunks);
     if (chunk_id >= n_act) return;
 
-    extern __shared__ float wacc[];  // [kPromWarps][g][2][D]
-    __shared__ float sq[kMaxGqa * kMaxD];
-    __shared__ float wm[kPromWarps * kMaxGqa * 2], wl[kPromWarps * kMaxGqa * 2];
+    extern __shared__ float wacc[];  // [kPromWarps][g][3][D]
+    __shared__ float sq[G * kMaxD], so[G * kMaxD];
+    __shared__ float wm[kPromWarps * G * 2], wl[kPromWarps * G * 2];
+    // per warp and head, (m, l) of a key-promoted block's exact scores over
+    // the warp's share of its tokens (the ladder's ranking check); two
+    // buffers, a barrier every block
+    __shared__ float2 bsm[2][kPromWarps][G];
     __shared__ int sflag;
 
     const int T = clamp_ctx(p.ctx_lens[b], p.max_pages);
@@ -215,45 +224,50 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
     const int32_t *bt = p.block_table + (long long)b * p.max_pages;
     const int32_t *prom = p.prom + bk * p.sort_cap;
 
-    // rotated query of each head, pre-scaled into log2 units
+    // queries in log2 units: rotated (against dequantised keys) and original
+    // (against exact keys)
     if (warp < g) {
         float x[E];
         rotated_query<D>(p, b, kvh * g + warp, lane, x);
+        const __half *qh = p.q + ((long long)b * L.hq + kvh * g + warp) * D + lane * E;
 #pragma unroll
-        for (int e = 0; e < E; e++) sq[warp * D + lane * E + e] = x[e] * p.qscale;
+        for (int e = 0; e < E; e++) {
+            sq[warp * D + lane * E + e] = x[e] * p.qscale;
+            so[warp * D + lane * E + e] = __half2float(qh[e]) * p.qscale;
+        }
     }
     __syncthreads();
-    float qr[kMaxGqa][E];
+    float qr[G][E];  // the original-domain query stays in shared memory (one vector load per use)
 #pragma unroll
-    for (int h = 0; h < kMaxGqa; h++)
+    for (int h = 0; h < G; h++)
 #pragma unroll
         for (int e = 0; e < E; e++) qr[h][e] = h < g ? sq[h * D + lane * E + e] : 0.f;
 
-    // (m, l, acc) over this CTA's promoted tokens: [0] exact rows, [1] dequantised rows
-    float m[kMaxGqa][2], l[kMaxGqa][2], acc[kMaxGqa][2][E];
+    // partials over this CTA's promoted tokens: [0] the mixed softmax (exact
+    // keys and values where promoted), [1] the quantised one.  The mixed
+    // side sums exact values (original domain, ae) and dequantised ones
+    // (rotated domain, ar) apart; aq is the quantised side's sum.
+    float m[G][2], l[G][2], ae[G][E], ar[G][E], aq[G][E];
 #pragma unroll
-    for (int h = 0; h < kMaxGqa; h++)
+    for (int h = 0; h < G; h++) {
 #pragma unroll
         for (int w = 0; w < 2; w++) {
             m[h][w] = -INFINITY;
             l[h][w] = 0.f;
-#pragma unroll
-            for (int e = 0; e < E; e++) acc[h][w][e] = 0.f;
         }
+#pragma unroll
+        for (int e = 0; e < E; e++) ae[h][e] = ar[h][e] = aq[h][e] = 0.f;
+    }
 
-    // per warp and head, (m, l) of a key-promoted block's exact scores over
-    // the warp's share of its tokens (the ladder's ranking check); two
-    // buffers, a barrier every block
-    __shared__ float2 bsm[2][kPromWarps][kMaxGqa];
     int parity = 0;
     for (int r = chunk_id; r < kp; r += n_act, parity ^= 1) {
         const int ent = prom[r];
         const int blk_id = ent & kPromIdx;
         const bool kx = (ent & kPromKey) != 0, vx = (ent & kPromVal) != 0;
         const int t0 = blk_id * block, t1 = min(t0 + block, T);
-        float bm[kMaxGqa], bl[kMaxGqa];
+        float bm[G], bl[G];
 #pragma unroll
-        for (int h = 0; h < kMaxGqa; h++) {
+        for (int h = 0; h < G; h++) {
             bm[h] = -INFINITY;
             bl[h] = 0.f;
         }
@@ -283,38 +297,29 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
                 const unsigned char *chunk =
                     p.pool + kHeaderBytes + (long long)pgs[u] * L.page_bytes + (long long)kvh * L.chunk_bytes;
                 float kq[E], vq[E], ke[E] = {}, ve[E] = {};
-                // exact rows, rotated (both together when both are exact)
-                if (kx) kraw[u].widen(ke);
-                if (vx) vraw[u].widen(ve);
-                if (p.rotate) {
-#pragma unroll
-                    for (int e = 0; e < E; e++) {
-                        ke[e] *= p.signs[lane * E + e];
-                        ve[e] *= p.signs[lane * E + e];
-                    }
-                    if (kx && vx) fwht_warp2<D>(ke, ve, lane);
-                    else if (kx) fwht_warp<D>(ke, lane);
-                    else if (vx) fwht_warp<D>(ve, lane);
-#pragma unroll
-                    for (int e = 0; e < E; e++) {
-                        ke[e] *= p.rot_scale;
-                        ve[e] *= p.rot_scale;
-                    }
-                }
                 dequant_lane<E>(chunk, L.k_codes, L.k_meta, L.k_row_meta, L.k_fmt, tok, lane, kq);
                 dequant_lane<E>(chunk, L.v_codes, L.v_meta, L.v_row_meta, L.v_fmt, tok, lane, vq);
-                if (!vx)
+                if (kx) kraw[u].widen(ke);
+                if (vx) vraw[u].widen(ve);
 #pragma unroll
-                    for (int e = 0; e < E; e++) ve[e] = vq[e];
-#pragma unroll
-                for (int h = 0; h < kMaxGqa; h++) {
+                for (int h = 0; h < G; h++) {
                     if (h >= g) break;
-                    float se = 0.f, sqv = 0.f;
+                    float qo[E];
+                    if (E == 4) {
+                        const float4 v4 = *reinterpret_cast<const float4 *>(so + h * D + lane * E);
+                        qo[0] = v4.x;
+                        qo[E > 1 ? 1 : 0] = v4.y;
+                        qo[E > 2 ? 2 : 0] = v4.z;
+                        qo[E > 3 ? 3 : 0] = v4.w;
+                    } else {
 #pragma unroll
-                    for (int e = 0; e < E; e++) sqv = fmaf(qr[h][e], kq[e], sqv);
-                    if (kx) {
+                        for (int e = 0; e < E; e++) qo[e] = so[h * D + lane * E + e];
+                    }
+                    float sqv = 0.f, se = 0.f;
 #pragma unroll
-                        for (int e = 0; e < E; e++) se = fmaf(qr[h][e], ke[e], se);
+                    for (int e = 0; e < E; e++) {
+                        sqv = fmaf(qr[h][e], kq[e], sqv);
+                        se = fmaf(qo[e], ke[e], se);
                     }
 #pragma unroll
                     for (int mm = 16; mm >= 1; mm >>= 1) {
@@ -322,8 +327,20 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
                         if (kx) se += __shfl_xor_sync(kFull, se, mm);
                     }
                     if (!kx) se = sqv;
-                    online_update<E>(m[h][0], l[h][0], acc[h][0], se, ve);
-                    online_update<E>(m[h][1], l[h][1], acc[h][1], sqv, vq);
+                    online_update<E>(m[h][1], l[h][1], aq[h], sqv, vq);
+                    {  // the mixed side: one (m, l), two sums
+                        const float mn = fmaxf(m[h][0], se);
+                        const float al = (m[h][0] == -INFINITY) ? 0.f : ex2(m[h][0] - mn);
+                        const float pe = ex2(se - mn);
+                        l[h][0] = fmaf(l[h][0], al, pe);
+                        const float pv = vx ? pe : 0.f, pq = vx ? 0.f : pe;
+#pragma unroll
+                        for (int e = 0; e < E; e++) {
+                            ae[h][e] = fmaf(ae[h][e], al, pv * ve[e]);
+                            ar[h][e] = fmaf(ar[h][e], al, pq * vq[e]);
+                        }
+                        m[h][0] = mn;
+                    }
                     if (p.ladder && kx) {
                         const float mn = fmaxf(bm[h], se);
                         bl[h] = fmaf(bl[h], ex2(bm[h] - mn), ex2(se - mn));
@@ -335,7 +352,7 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
         if (p.ladder) {  // CTA-uniform
             if (kx && lane == 0)
 #pragma unroll
-                for (int h = 0; h < kMaxGqa; h++)
+                for (int h = 0; h < G; h++)
                     if (h < g) bsm[parity][warp][h] = make_float2(bm[h], bl[h]);
             __syncthreads();
             if (kx && warp == 0 && lane < g) {
@@ -352,41 +369,47 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
         }
     }
 
-    // warps -> shared memory -> one partial per (head, exact|quantised)
+    // warps -> shared memory -> one partial per head: rows ae, ar, aq, then
+    // (m, l) of the mixed and of the quantised side
 #pragma unroll
-    for (int h = 0; h < kMaxGqa; h++)
-        if (h < g)
+    for (int h = 0; h < G; h++)
+        if (h < g) {
 #pragma unroll
-            for (int w = 0; w < 2; w++) {
-#pragma unroll
-                for (int e = 0; e < E; e++) wacc[((warp * g + h) * 2 + w) * D + lane * E + e] = acc[h][w][e];
-                if (lane == 0) {
-                    wm[(warp * kMaxGqa + h) * 2 + w] = m[h][w];
-                    wl[(warp * kMaxGqa + h) * 2 + w] = l[h][w];
-                }
+            for (int e = 0; e < E; e++) {
+                wacc[((warp * g + h) * 3 + 0) * D + lane * E + e] = ae[h][e];
+                wacc[((warp * g + h) * 3 + 1) * D + lane * E + e] = ar[h][e];
+                wacc[((warp * g + h) * 3 + 2) * D + lane * E + e] = aq[h][e];
             }
+            if (lane == 0)
+#pragma unroll
+                for (int w = 0; w < 2; w++) {
+                    wm[(warp * G + h) * 2 + w] = m[h][w];
+                    wl[(warp * G + h) * 2 + w] = l[h][w];
+                }
+        }
     __syncthreads();
-    constexpr int REC = D + 4;
-    float *cp = p.cpart + (bk * p.n_chunks + chunk_id) * (long long)g * 2 * REC;
-    for (int idx = tid; idx < g * 2 * D; idx += kPromThreads) {
-        const int hw = idx / D, ch = idx - hw * D;  // hw = h * 2 + w
-        const int h = hw >> 1, w = hw & 1;
+    constexpr int REC = 3 * D + 4;
+    float *cp = p.cpart + (bk * p.n_chunks + chunk_id) * (long long)g * REC;
+    for (int idx = tid; idx < g * 3 * D; idx += kPromThreads) {
+        const int h = idx / (3 * D), rem = idx - h * 3 * D;
+        const int row = rem / D, ch = rem - row * D;
+        const int w = row == 2 ? 1 : 0;  // rows 0, 1: the mixed side; row 2: the quantised side
         float M = -INFINITY;
 #pragma unroll
-        for (int ww = 0; ww < kPromWarps; ww++) M = fmaxf(M, wm[(ww * kMaxGqa + h) * 2 + w]);
+        for (int ww = 0; ww < kPromWarps; ww++) M = fmaxf(M, wm[(ww * G + h) * 2 + w]);
         float a = 0.f, Ls = 0.f;
         if (M != -INFINITY)
 #pragma unroll
             for (int ww = 0; ww < kPromWarps; ww++) {
-                const float mw = wm[(ww * kMaxGqa + h) * 2 + w];
+                const float mw = wm[(ww * G + h) * 2 + w];
                 const float f = mw == -INFINITY ? 0.f : ex2(mw - M);
-                a = fmaf(f, wacc[((ww * g + h) * 2 + w) * D + ch], a);
-                Ls = fmaf(f, wl[(ww * kMaxGqa + h) * 2 + w], Ls);
+                a = fmaf(f, wacc[((ww * g + h) * 3 + row) * D + ch], a);
+                Ls = fmaf(f, wl[(ww * G + h) * 2 + w], Ls);
             }
-        cp[hw * REC + ch] = a;
-        if (ch == 0) {
-            cp[hw * REC + D] = M;
-            cp[hw * REC + D + 1] = Ls;
+        cp[h * REC + row * D + ch] = a;
+        if (ch == 0 && row != 1) {
+            cp[h * REC + 3 * D + 2 * w] = M;
+            cp[h * REC + 3 * D + 2 * w + 1] = Ls;
         }
     }
 
@@ -401,37 +424,42 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
     if (!sflag) return;
     __threadfence();
     if (tid == 0) p.ccount[bk] = 0u;
-    const float *cbase = p.cpart + bk * p.n_chunks * (long long)g * 2 * REC;
+    const float *cbase = p.cpart + bk * p.n_chunks * (long long)g * REC;
     for (int h = warp; h < g; h += kPromWarps) {
-        float Mx[2] = {-INFINITY, -INFINITY}, Ls[2] = {0.f, 0.f}, a[2][E];
+        // lane c: (max, sum) of chunk c's two sides, loaded in parallel
+        float Mx[2], Ls[2], fch[2];
 #pragma unroll
         for (int w = 0; w < 2; w++) {
-            // lane c: (max, sum) of chunk c's record, loaded in parallel; the
-            // accumulator rows of every chunk go out together (unrolled)
             float2 mlc = make_float2(-INFINITY, 0.f);
-            if (lane < n_act) mlc = __ldcg(reinterpret_cast<const float2 *>(cbase + ((lane * g + h) * 2 + w) * REC + D));
+            if (lane < n_act) mlc = __ldcg(reinterpret_cast<const float2 *>(cbase + (lane * g + h) * REC + 3 * D + 2 * w));
             float M = mlc.x;
 #pragma unroll
-            for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, m));
+            for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
             Mx[w] = M;
-            const float f = (mlc.x == -INFINITY || M == -INFINITY) ? 0.f : ex2(mlc.x - M);
-            float l = f * mlc.y;
+            fch[w] = (mlc.x == -INFINITY || M == -INFINITY) ? 0.f : ex2(mlc.x - M);
+            float lsum = fch[w] * mlc.y;
 #pragma unroll
-            for (int m = 16; m >= 1; m >>= 1) l += __shfl_xor_sync(kFull, l, m);
-            Ls[w] = l;
+            for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(kFull, lsum, o);
+            Ls[w] = lsum;
+        }
+        // the three sums over the chunks, one row at a time (loads unrolled)
+        float a[3][E];
+#pragma unroll
+        for (int row = 0; row < 3; row++) {
+            const int w = row == 2 ? 1 : 0;
             float rows[kCertChunks][E];
 #pragma unroll
             for (int c = 0; c < kCertChunks; c++)
 #pragma unroll
                 for (int e = 0; e < E; e++)
-                    rows[c][e] = c < n_act ? __ldcg(cbase + ((c * g + h) * 2 + w) * REC + lane * E + e) : 0.f;
+                    rows[c][e] = c < n_act ? __ldcg(cbase + (c * g + h) * REC + row * D + lane * E + e) : 0.f;
 #pragma unroll
-            for (int e = 0; e < E; e++) a[w][e] = 0.f;
+            for (int e = 0; e < E; e++) a[row][e] = 0.f;
 #pragma unroll
             for (int c = 0; c < kCertChunks; c++) {
-                const float fc = __shfl_sync(kFull, f, c);
+                const float fc = __shfl_sync(kFull, fch[w], c);
 #pragma unroll
-                for (int e = 0; e < E; e++) a[w][e] = fmaf(fc, rows[c][e], a[w][e]);
+                for (int e = 0; e < E; e++) a[row][e] = fmaf(fc, rows[c][e], a[row][e]);
             }
         }
         const float2 ml = p.head_ml[bk * g + h];  // the quantised pass: (M, L)
@@ -442,9 +470,10 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
         const float fq = Mx[1] == -INFINITY ? 0.f : ex2(Mx[1] - R);
         const float den = f0 + Ls[0] * fe - Ls[1] * fq;
         if (p.ladder && lane == 0) p.mix[bk * g + h] = make_float2(R, den);
+        // dequantised sums (rotated domain) back to the original domain
         float dlt[E];
 #pragma unroll
-        for (int e = 0; e < E; e++) dlt[e] = a[0][e] * fe - a[1][e] * fq;
+        for (int e = 0; e < E; e++) dlt[e] = a[1][e] * fe - a[2][e] * fq;
         if (p.rotate) {
             fwht_warp<D>(dlt, lane);
 #pragma unroll
@@ -452,7 +481,7 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
         }
         float *o = p.out + ((long long)b * L.hq + kvh * g + h) * D + lane * E;
 #pragma unroll
-        for (int e = 0; e < E; e++) o[e] = den > 0.f ? (f0 * o[e] + dlt[e]) / den : 0.f;
+        for (int e = 0; e < E; e++) o[e] = den > 0.f ? (f0 * o[e] + a[0][e] * fe + dlt[e]) / den : 0.f;
     }
 }
 
@@ -484,22 +513,35 @@ cudaError_t launch_cert_select(const CertParams &p, int batch, cudaStream_t s)
               : launch_pdl(cert_select_kernel<64>, grid, kSelThreads, smem, s, p);
 }
 
+template <int D, int G>
+cudaError_t launch_promote_t(const CertParams &p, int batch, cudaStream_t s)
+{
+    static bool configured = false;
+    if (!configured) {
+        const int cap = kPromWarps * G * 3 * D * (int)sizeof(float);
+        const cudaError_t e =
+            cudaFuncSetAttribute(cert_promote_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const size_t smem = (size_t)kPromWarps * p.L.g * 3 * D * sizeof(float);
+    const dim3 grid(p.n_chunks, p.L.hkv, batch);
+    return launch_pdl(cert_promote_kernel<D, G>, grid, kPromThreads, smem, s, p);
+}
+
+template <int D>
+cudaError_t launch_promote_d(const CertParams &p, int batch, cudaStream_t s)
+{
+    const int g = p.L.g;
+    if (g <= 1) return launch_promote_t<D, 1>(p, batch, s);
+    if (g <= 2) return launch_promote_t<D, 2>(p, batch, s);
+    if (g <= 4) return launch_promote_t<D, 4>(p, batch, s);
+    return launch_promote_t<D, 8>(p, batch, s);
+}
+
 cudaError_t launch_cert_promote(const CertParams &p, int batch, cudaStream_t s)
 {
-    static bool configured[2] = {false, false};
-    const int di = p.L.d == 64 ? 0 : 1;
-    const size_t smem = (size_t)kPromWarps * p.L.g * 2 * p.L.d * sizeof(float);
-    if (!configured[di]) {
-        const int cap = kPromWarps * kMaxGqa * 2 * kMaxD * (int)sizeof(float);
-        const cudaError_t e =
-            di ? cudaFuncSetAttribute(cert_promote_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, cap)
-               : cudaFuncSetAttribute(cert_promote_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
-        if (e != cudaSuccess) return e;
-        configured[di] = true;
-    }
-    const dim3 grid(p.n_chunks, p.L.hkv, batch);
-    return di ? launch_pdl(cert_promote_kernel<128>, grid, kPromThreads, smem, s, p)
-              : launch_pdl(cert_promote_kernel<64>, grid, kPromThreads, smem, s, p);
+    return p.L.d == 128 ? launch_promote_d<128>(p, batch, s) : launch_promote_d<64>(p, batch, s);
 }
 
 }  // namespace kvq

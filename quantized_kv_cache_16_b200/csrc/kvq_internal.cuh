@@ -171,7 +171,8 @@ struct CertParams {
     int32_t *promoted_out;     // optional [B][Hkv][kmax_out], -1 padded
     const __half *k2;          // tier 2: exact rows [num_pages*16][Hkv][d] fp16, device-accessible
     const __half *v2;
-    float *cpart;              // [B][Hkv][n_chunks][g][2][d + 4]: exact / quantised block partials
+    float *cpart;              // [B][Hkv][n_chunks][g][3d + 4]: sums of the mixed (exact values, dequantised
+                               // values) and quantised sides, then (m, l) of each side
     unsigned int *ccount;      // [B][Hkv], zero between calls
     float *out;                // [B][Hq][d]
 
@@ -194,6 +195,7 @@ struct CertParams {
     float *bound_out;          // optional [B][Hq]
     int32_t *status_out;       // optional [B][Hq]
     int n_dsplit, dsplit_tokens;  // dense fallback: splits per (sequence, kv head) and tokens per split
+    int batch, dense_ctas;        // the persistent dense-fallback grid
     float *dpart;              // [B][Hkv][n_dsplit][g][d + 4]
     unsigned int *dcount;      // [B][Hkv], zero between calls
 };

@@ -347,27 +347,18 @@ __global__ void __launch_bounds__(kSelThreads) ladder_finish_kernel(const __grid
 }
 
 // fp16 attention over the tier-2 rows (original domain, no rotation) for the
-// heads that fell back, one context split per CTA, merged by the last CTA.
+// heads that fell back.  Work items (context split, kv head, sequence) are
+// handed out over a persistent grid; a group's splits are merged by the CTA
+// that finishes its last one.
 template <int D>
-__global__ void __launch_bounds__(kPromThreads) ladder_dense_kernel(const __grid_constant__ CertParams p)
+__device__ __forceinline__ void dense_item(const CertParams &p, int split, int kvh, int b, unsigned mask, bool layer,
+                                           float *wacc, float *wm, float *wl, int *sflag)
 {
-    pdl_enter();
     constexpr int E = D / 32;
     const Layout &L = p.L;
-    const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = L.g;
     const long long bk = (long long)b * L.hkv + kvh;
-    const bool layer = __ldcg(p.nfall) > (unsigned)p.layer_thresh;
-    unsigned mask = 0;
-    for (int h = 0; h < g; h++)
-        if (layer || (__ldcg(p.status + (long long)b * L.hq + kvh * g + h) & kStHeadDense)) mask |= 1u << h;
-    if (!mask) return;  // uniform over the (sequence, kv head)'s CTAs
-
-    extern __shared__ float wacc[];  // [kPromWarps][g][D]
-    __shared__ float wm[kPromWarps * kMaxGqa], wl[kPromWarps * kMaxGqa];
-    __shared__ int sflag;
-
     const int T = clamp_ctx(p.ctx_lens[b], p.max_pages);
     const int t0 = split * p.dsplit_tokens, t1 = min(T, t0 + p.dsplit_tokens);
     const int32_t *bt = p.block_table + (long long)b * p.max_pages;
@@ -424,6 +415,7 @@ __global__ void __launch_bounds__(kPromThreads) ladder_dense_kernel(const __grid
     }
 
     // warps -> one partial per head
+    __syncthreads();  // the previous item's shared-memory reads are done
 #pragma unroll
     for (int h = 0; h < kMaxGqa; h++)
         if (h < g) {
@@ -458,15 +450,15 @@ __global__ void __launch_bounds__(kPromThreads) ladder_dense_kernel(const __grid
         }
     }
 
-    // the last CTA of this (sequence, kv head) merges the splits
+    // the CTA that finishes the group's last split merges them
     __syncthreads();
     if (tid == 0) {
         __threadfence();
         const unsigned prev = atomicAdd(p.dcount + bk, 1u);
-        sflag = prev == (unsigned)(p.n_dsplit - 1);
+        *sflag = prev == (unsigned)(p.n_dsplit - 1);
     }
     __syncthreads();
-    if (!sflag) return;
+    if (!*sflag) return;
     __threadfence();
     if (tid == 0) p.dcount[bk] = 0u;
     const float *base = p.dpart + bk * p.n_dsplit * (long long)g * REC;
@@ -494,6 +486,29 @@ __global__ void __launch_bounds__(kPromThreads) ladder_dense_kernel(const __grid
             p.status[head] |= kStLayerDense;
             if (p.status_out) p.status_out[head] |= kStLayerDense;
         }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPromThreads) ladder_dense_kernel(const __grid_constant__ CertParams p)
+{
+    pdl_enter();
+    const Layout &L = p.L;
+    extern __shared__ float wacc[];  // [kPromWarps][g][D]
+    __shared__ float wm[kPromWarps * kMaxGqa], wl[kPromWarps * kMaxGqa];
+    __shared__ int sflag;
+    const unsigned nfall = __ldcg(p.nfall);
+    if (nfall == 0u) return;  // no head fell back (the common case)
+    const bool layer = nfall > (unsigned)p.layer_thresh;
+    const int per_b = p.n_dsplit * L.hkv;
+    const int n_items = per_b * p.batch;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {  // uniform over the CTA
+        const int b = it / per_b, r = it - b * per_b;
+        const int kvh = r / p.n_dsplit, split = r - kvh * p.n_dsplit;
+        unsigned mask = 0;
+        for (int h = 0; h < L.g; h++)
+            if (layer || (__ldcg(p.status + (long long)b * L.hq + kvh * L.g + h) & kStHeadDense)) mask |= 1u << h;
+        if (mask) dense_item<D>(p, split, kvh, b, mask, layer, wacc, wm, wl, &sflag);
     }
 }
 
@@ -539,7 +554,8 @@ cudaError_t launch_ladder_finish(const CertParams &p, int batch, cudaStream_t s)
                        : launch_pdl(ladder_finish_kernel<64>, grid, kSelThreads, smem, s, p);
     if (e != cudaSuccess) return e;
     const size_t dsmem = (size_t)kPromWarps * p.L.g * p.L.d * sizeof(float);
-    const dim3 dgrid(p.n_dsplit, p.L.hkv, batch);
+    const int items = p.n_dsplit * p.L.hkv * batch;
+    const dim3 dgrid(items < p.dense_ctas ? items : p.dense_ctas);
     return di ? launch_pdl(ladder_dense_kernel<128>, dgrid, kPromThreads, dsmem, s, p)
               : launch_pdl(ladder_dense_kernel<64>, dgrid, kPromThreads, dsmem, s, p);
 }
