@@ -76,6 +76,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-steps", type=int, default=4, help="oracle steps in the CPU baseline sample")
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, append and CPU legs")
+    ap.add_argument("--leg", choices=["certified", "ladder"],
+                    help="run only this leg (one GPU, --steps calls) and print its JSON")
+    ap.add_argument("--ctx", type=int, default=0, help="context length of --leg (default: its workload's)")
     return ap.parse_args()
 
 
@@ -551,7 +554,7 @@ def _graph_time(call, steps: int, stream) -> float:
     return us
 
 
-def certified_leg(steps: int):
+def certified_leg(steps: int, T: int = 0):
     """Certified decode at its own configuration: batch 1, context 131072,
     int8 K / int4 g32 V, 128-token bound blocks, top 1% of each kv head's
     blocks promoted from exact fp16 rows in pinned host memory.  Calls (four
@@ -562,7 +565,7 @@ def certified_leg(steps: int):
 
     import quantized_kv_cache_16_b200 as K
     import workloads as W
-    wl = W.certified()
+    wl = W.certified(T) if T else W.certified()
     T, frac, copies = wl.ctx[0], 0.01, 2
     dev = torch.device("cuda", torch.cuda.current_device())
     cache, k2, v2, bts, ctx = _tier2_cache(wl, copies)
@@ -591,7 +594,7 @@ def certified_leg(steps: int):
     hbm = T * wl.Hkv * (wl.d + 2 + wl.d // 2 + 4 * (wl.d // 32))
     link = wl.Hkv * kmax * wl.bound_block * wl.d * 2 * 2
     peak, kind = measured_peaks()
-    return {"workload": "certified decode: B=1, 32/8 heads, d=128, context 131072, int8 K / int4 g32 V, "
+    return {"workload": f"certified decode: B=1, 32/8 heads, d=128, context {T}, int8 K / int4 g32 V, "
                         "128-token bound blocks, top 1% promoted from pinned host fp16 rows",
             "us": round(res["certified"], 2), "quantised_only_us": round(res["quantised_only"], 2),
             "overhead_x": round(res["certified"] / res["quantised_only"], 2),
@@ -605,7 +608,7 @@ LADDER_POLICY = dict(tau_cov=0.995, max_frac=0.05, key_tol=0.02, v_tol=1e-3, ran
                      layer_frac=0.5)
 
 
-def ladder_leg(steps: int):
+def ladder_leg(steps: int, T: int = 0):
     """Certified decode with the adaptive ladder (kvq_decode_certified, six
     launches) at context 131072 on the needle workload (attention
     concentrated on a sink, six needles and the recent window), replayed in
@@ -617,7 +620,7 @@ def ladder_leg(steps: int):
 
     import quantized_kv_cache_16_b200 as K
     import workloads as W
-    wl = W.ladder()
+    wl = W.ladder(T) if T else W.ladder()
     T, copies = wl.ctx[0], 2
     dev = torch.device("cuda", torch.cuda.current_device())
     cache, k2, v2, bts, ctx = _tier2_cache(wl, copies)
@@ -680,7 +683,7 @@ def ladder_leg(steps: int):
     assert cache.sync_status() == 0
     row = wl.bound_block * wl.d * 2
     link = int(round((np.mean(kstar) + np.mean(nval)) * wl.Hkv * row))
-    return {"workload": "certified ladder: B=1, 32/8 heads, d=128, context 131072, int8 K / int4 g32 V, 128-token "
+    return {"workload": f"certified ladder: B=1, 32/8 heads, d=128, context {T}, int8 K / int4 g32 V, 128-token "
                         "blocks, needle attention (sink, six needles, recent window); pinned host fp16 tier 2",
             "policy": LADDER_POLICY, "us": round(ladder_us, 2), "quantised_only_us": round(quant_us, 2),
             "overhead_x": round(ladder_us / quant_us, 2), "no_fallback_us": round(rungs12_us, 2),
@@ -763,6 +766,12 @@ def run_reference(args, dist: Dist):
 def main():
     args = parse()
     dist = Dist()
+    if args.leg:
+        import torch
+        torch.cuda.set_device(0)
+        leg = certified_leg if args.leg == "certified" else ladder_leg
+        print(json.dumps(leg(args.steps, args.ctx)), flush=True)
+        return
     if args.impl == "reference":
         run_reference(args, dist)
     else:
