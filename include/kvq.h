@@ -74,6 +74,7 @@ typedef struct {
     int32_t page_tokens;        /* tokens per page; must be 16                        */
     int32_t num_pages;          /* pages in the pool                                  */
     int32_t bound_block_tokens; /* 0 = no error descriptors; else a multiple of 16    */
+    int32_t scale_search;       /* 1 = ScaleSearch of each scale (see kvq_append)     */
 } kvq_config;
 
 typedef struct kvq_cache kvq_cache; /* opaque; owned by the library */
@@ -118,7 +119,15 @@ kvq_status kvq_destroy_cache(kvq_cache *cache);
  * slot skips the token; a slot >= num_pages*16 is skipped and recorded as
  * KVQ_ERR_OUT_OF_RANGE in the status word.  With descriptors on, each row's
  * max |k - khat|, max |v - vhat| and max |v| are max-reduced into its page's
- * descriptor (reset a page with kvq_reset_pages before reusing it). */
+ * descriptor (reset a page with kvq_reset_pages before reusing it).
+ * With cfg.scale_search = 1 each group's fp16 scale is searched
+ * ["Search Your Block Floating Point Scales!", ScaleSearch]: the scales whose
+ * bit patterns are the default scale's plus f, f in [-2, 6] (positive finite
+ * only), each quantise the group and the one with the least squared
+ * reconstruction error is stored (fp32 sums: per run of 64 consecutive
+ * elements, even and odd elements apart in element order, then added, the
+ * runs added in order; candidates tried as 0, -1, 1, -2, 2, 3, 4, 5, 6, a
+ * later one kept only if strictly better); the zero is unchanged. */
 kvq_status kvq_append(kvq_cache *cache, const void *k, const void *v, const int32_t *slot_mapping, int32_t n_tok,
                       void *stream);
 
@@ -252,7 +261,8 @@ kvq_status kvq_decode_certified(kvq_cache *cache, const void *q, const int32_t *
  * token is not stored and KVQ_ERR_OUT_OF_RANGE is recorded).  The stored
  * codes are byte-identical to kvq_append's and the output equals kvq_append
  * followed by kvq_decode_attn.  Other arguments as kvq_decode_attn (no
- * certified mode). */
+ * certified mode).  A cache configured with scale_search returns
+ * KVQ_ERR_UNSUPPORTED (use kvq_append, then kvq_decode_attn). */
 kvq_status kvq_decode_step(kvq_cache *cache, const void *k_new, const void *v_new, const int32_t *slot_mapping,
                            const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
                            const int32_t *ctx_lens, int32_t batch, float softmax_scale, void *workspace,

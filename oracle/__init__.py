@@ -55,6 +55,7 @@ class Config(C.Structure):
         ("page_tokens", C.c_int32),
         ("num_pages", C.c_int32),
         ("bound_block_tokens", C.c_int32),
+        ("scale_search", C.c_int32),
     ]
 
 
@@ -79,9 +80,10 @@ LADDER_RANK_FAIL, LADDER_BOUND_FAIL, LADDER_HEAD_DENSE, LADDER_LAYER_DENSE = 8, 
 
 
 def make_config(num_q_heads, num_kv_heads, head_dim, k_fmt=INT4_ASYM, v_fmt=INT4_ASYM, k_group=32, v_group=32,
-                clip_ratio=1.0, rotation_seed=0, rotate=1, num_pages=1, bound_block_tokens=0) -> Config:
+                clip_ratio=1.0, rotation_seed=0, rotate=1, num_pages=1, bound_block_tokens=0,
+                scale_search=0) -> Config:
     return Config(num_q_heads, num_kv_heads, head_dim, k_fmt, v_fmt, k_group, v_group, clip_ratio,
-                  rotation_seed, rotate, PAGE_TOKENS, num_pages, bound_block_tokens)
+                  rotation_seed, rotate, PAGE_TOKENS, num_pages, bound_block_tokens, scale_search)
 
 
 _lib = None
@@ -107,7 +109,7 @@ def lib():
             "kvqo_rotate_f32": (None, [P, P, i32, i32, P]),
             "kvqo_rotate_f64": (None, [P, P, i32, i32, P]),
             "kvqo_inv_rotate_f64": (None, [P, P, i32, i32, P]),
-            "kvqo_quantize_rows": (None, [i32, i32, C.c_float, P, i32, i32, P, P, P, P, P]),
+            "kvqo_quantize_rows": (None, [i32, i32, C.c_float, P, i32, i32, P, P, P, P, P, i32]),
             "kvqo_config_ok": (i32, [cfgp]),
             "kvqo_page_bytes": (sz, [cfgp]),
             "kvqo_desc_offset": (sz, [cfgp]),
@@ -208,9 +210,9 @@ def inv_rotate_f64(x, seed: int, rotate: int = 1) -> np.ndarray:
     return _rot64(lib().kvqo_inv_rotate_f64, x, seed, rotate)
 
 
-def quantize_rows(fmt: int, group: int, clip: float, y):
+def quantize_rows(fmt: int, group: int, clip: float, y, search: int = 0):
     """Quantise rotated fp32 rows y[n, d]; returns codes, scales, zeros (fp16
-    bits), max |y - yhat| and max |y| per row."""
+    bits), max |y - yhat| and max |y| per row.  search=1: ScaleSearch."""
     y = _c(y, np.float32)
     n, d = y.shape
     ng = 1 if fmt == INT8_SYM else d // group
@@ -219,7 +221,7 @@ def quantize_rows(fmt: int, group: int, clip: float, y):
     zh = np.empty((n, ng), np.uint16)
     em = np.empty(n, np.float32)
     am = np.empty(n, np.float32)
-    lib().kvqo_quantize_rows(fmt, group, clip, _p(y), n, d, _p(code), _p(sh), _p(zh), _p(em), _p(am))
+    lib().kvqo_quantize_rows(fmt, group, clip, _p(y), n, d, _p(code), _p(sh), _p(zh), _p(em), _p(am), search)
     return code, sh, zh, em, am
 
 

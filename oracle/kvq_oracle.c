@@ -61,6 +61,7 @@ typedef struct {
     int32_t page_tokens;
     int32_t num_pages;
     int32_t bound_block_tokens;
+    int32_t scale_search; /* 1: ScaleSearch over the scale's fp16 bit pattern */
 } kvqo_config;
 
 /* ------------------------------------------------------------------------- */
@@ -263,7 +264,63 @@ static int fmt_bits(int fmt) { return fmt == KVQO_INT4_ASYM ? 4 : fmt == KVQO_IN
  * Outputs: code[d], scale_h[ng], zero_h[ng] (zero unused for int8), and the
  * fp32 descriptors max|y - yhat| and max|y| with yhat = float(code)*scale
  * (+ zero), each operation rounded on its own. */
-static void quantize_row(int fmt, int group, float clip, const float *y, int d, int16_t *code,
+/* ScaleSearch ["Search Your Block Floating Point Scales!", ScaleSearch]: the
+ * page searches integer offsets f in [-2, 6] on the bit pattern of the
+ * default block scale and keeps the scale of least squared error.  Here the
+ * scale is the codec's fp16 scale: candidate f has the bits of the default
+ * scale plus f (only positive finite fp16 values), the zero stays.  Each
+ * candidate quantises the group as the codec does and sums the squared
+ * reconstruction errors in fp32, in a fixed order: the group is cut into
+ * runs of 64 consecutive elements (one run if it is shorter); in a run, the
+ * even and the odd elements are summed apart, in element order, and the
+ * two added; the runs' sums are added in order.  Candidates are tried in
+ * the order 0, -1, 1, -2, 2, 3, 4, 5, 6 and one replaces the best so far
+ * only with a strictly smaller error, so ties keep the one nearer the
+ * default.  Returns the chosen scale bits. */
+static const int kvqo_search_order[9] = {0, -1, 1, -2, 2, 3, 4, 5, 6};
+
+static float group_sq_error(const float *yg, int n, float sf, float zf, float lo_code, float hi_code)
+{
+    float inv = (sf == 0.0f) ? 0.0f : 1.0f / sf;
+    int run = n < 64 ? n : 64;
+    float total = 0.0f;
+    for (int r0 = 0; r0 < n; r0 += run) {
+        float ev = 0.0f, od = 0.0f;
+        for (int i = r0; i < r0 + run; i++) {
+            float v = (yg[i] - zf) * inv;
+            float c = rintf(v);
+            if (c < lo_code) c = lo_code;
+            if (c > hi_code) c = hi_code;
+            float yhat = c * sf + zf;
+            float e = yg[i] - yhat;
+            float e2 = e * e;
+            if ((i - r0) % 2 == 0) ev = ev + e2;
+            else od = od + e2;
+        }
+        float rs = ev + od;
+        total = (r0 == 0) ? rs : total + rs;
+    }
+    return total;
+}
+
+static uint16_t search_scale(const float *yg, int n, uint16_t sh0, float zf, float lo_code, float hi_code)
+{
+    if (sh0 == 0 || sh0 >= 0x7C00u) return sh0;
+    uint16_t best = sh0;
+    float best_err = 0.0f;
+    for (int k = 0; k < 9; k++) {
+        int bits = (int)sh0 + kvqo_search_order[k];
+        if (bits <= 0 || bits >= 0x7C00) continue;
+        float err = group_sq_error(yg, n, kvqo_h2f((uint16_t)bits), zf, lo_code, hi_code);
+        if (k == 0 || err < best_err) {
+            best = (uint16_t)bits;
+            best_err = err;
+        }
+    }
+    return best;
+}
+
+static void quantize_row(int fmt, int group, float clip, int search, const float *y, int d, int16_t *code,
                          uint16_t *scale_h, uint16_t *zero_h, float *err_max, float *abs_max)
 {
     float emax = 0.0f, amax = 0.0f;
@@ -272,6 +329,7 @@ static void quantize_row(int fmt, int group, float clip, const float *y, int d, 
         for (int i = 0; i < d; i++) a = fmaxf(a, fabsf(y[i]));
         float sf_raw = a / 127.0f;
         uint16_t sh = kvqo_f2h_ru(sf_raw);
+        if (search) sh = search_scale(y, d, sh, 0.0f, -127.0f, 127.0f);
         float sf = kvqo_h2f(sh);
         float inv = (sf == 0.0f) ? 0.0f : 1.0f / sf;
         for (int i = 0; i < d; i++) {
@@ -304,6 +362,7 @@ static void quantize_row(int fmt, int group, float clip, const float *y, int d, 
             float sf_raw = (hi - lo) / qmax;
             uint16_t sh = kvqo_f2h_rn(sf_raw);
             uint16_t zh = kvqo_f2h_rn(lo);
+            if (search) sh = search_scale(yg, group, sh, kvqo_h2f(zh), 0.0f, qmax);
             float sf = kvqo_h2f(sh), zf = kvqo_h2f(zh);
             float inv = (sf == 0.0f) ? 0.0f : 1.0f / sf;
             for (int i = 0; i < group; i++) {
@@ -478,6 +537,7 @@ int kvqo_config_ok(const kvqo_config *c)
     if (!fmt_ok(c->k_fmt, c->k_group, d) || !fmt_ok(c->v_fmt, c->v_group, d)) return 0;
     if (!(c->clip_ratio > 0.0f && c->clip_ratio <= 1.0f)) return 0;
     if (c->bound_block_tokens < 0 || c->bound_block_tokens % KVQO_PAGE_TOKENS) return 0;
+    if (c->scale_search != 0 && c->scale_search != 1) return 0;
     return 1;
 }
 
@@ -516,7 +576,8 @@ int kvqo_append(const kvqo_config *c, uint8_t *pool, const uint16_t *k, const ui
                 int16_t code[KVQO_MAXD];
                 uint16_t sh[KVQO_MAXD], zh[KVQO_MAXD];
                 float emax, amax;
-                quantize_row(fmt, group, fmt == KVQO_INT8_SYM ? 1.0f : c->clip_ratio, y, d, code, sh, zh, &emax,
+                quantize_row(fmt, group, fmt == KVQO_INT8_SYM ? 1.0f : c->clip_ratio, c->scale_search, y, d, code, sh,
+                             zh, &emax,
                              &amax);
                 pack_row(c, pool, page, tok, kvh, tensor, code, sh, zh);
                 if (c->bound_block_tokens > 0) {
@@ -1275,12 +1336,13 @@ void kvqo_h2f_n(const uint16_t *h, float *x, size_t n)
 }
 
 /* Quantise already-rotated rows y[n][d] on their own (no pool): codes
- * [n][d], scales/zeros [n][d/group] (int8: one scale per row). */
+ * [n][d], scales/zeros [n][d/group] (int8: one scale per row); search = 1
+ * applies ScaleSearch. */
 void kvqo_quantize_rows(int fmt, int group, float clip, const float *y, int n, int d, int16_t *code,
-                        uint16_t *scale_h, uint16_t *zero_h, float *err_max, float *abs_max)
+                        uint16_t *scale_h, uint16_t *zero_h, float *err_max, float *abs_max, int search)
 {
     int ng = (fmt == KVQO_INT8_SYM) ? 1 : d / group;
     for (int r = 0; r < n; r++)
-        quantize_row(fmt, group, fmt == KVQO_INT8_SYM ? 1.0f : clip, y + (size_t)r * d, d, code + (size_t)r * d,
-                     scale_h + (size_t)r * ng, zero_h + (size_t)r * ng, err_max + r, abs_max + r);
+        quantize_row(fmt, group, fmt == KVQO_INT8_SYM ? 1.0f : clip, search, y + (size_t)r * d, d,
+                     code + (size_t)r * d, scale_h + (size_t)r * ng, zero_h + (size_t)r * ng, err_max + r, abs_max + r);
 }

@@ -42,6 +42,7 @@ class kvq_config(C.Structure):
         ("k_fmt", C.c_int32), ("v_fmt", C.c_int32), ("k_group", C.c_int32), ("v_group", C.c_int32),
         ("clip_ratio", C.c_float), ("rotation_seed", C.c_uint64), ("rotate", C.c_int32),
         ("page_tokens", C.c_int32), ("num_pages", C.c_int32), ("bound_block_tokens", C.c_int32),
+        ("scale_search", C.c_int32),
     ]
 
 
@@ -123,9 +124,10 @@ def _check(fn, status):
 
 
 def make_config(num_q_heads, num_kv_heads, head_dim, k_fmt=KVQ_INT4_ASYM, v_fmt=KVQ_INT4_ASYM, k_group=32,
-                v_group=32, clip_ratio=1.0, rotation_seed=0, rotate=1, num_pages=1, bound_block_tokens=0):
+                v_group=32, clip_ratio=1.0, rotation_seed=0, rotate=1, num_pages=1, bound_block_tokens=0,
+                scale_search=0):
     return kvq_config(num_q_heads, num_kv_heads, head_dim, k_fmt, v_fmt, k_group, v_group, clip_ratio,
-                      rotation_seed, rotate, PAGE_TOKENS, num_pages, bound_block_tokens)
+                      rotation_seed, rotate, PAGE_TOKENS, num_pages, bound_block_tokens, scale_search)
 
 
 # ------------------------------------------------------------ C entry points --

@@ -51,6 +51,7 @@ kvq_status check_config(const kvq_config *c)
     if (!(c->clip_ratio > 0.0f && c->clip_ratio <= 1.0f)) return KVQ_ERR_INVALID_ARG;
     if (c->bound_block_tokens < 0 || c->bound_block_tokens % kPageTokens) return KVQ_ERR_INVALID_ARG;
     if (c->rotate != 0 && c->rotate != 1) return KVQ_ERR_INVALID_ARG;
+    if (c->scale_search != 0 && c->scale_search != 1) return KVQ_ERR_INVALID_ARG;
     return KVQ_OK;
 }
 
@@ -275,6 +276,7 @@ kvq_status kvq_append(kvq_cache *c, const void *k, const void *v, const int32_t 
     p.clip = c->cfg.clip_ratio;
     p.rot_scale = c->rot_scale;
     p.rotate = c->cfg.rotate;
+    p.scale_search = c->cfg.scale_search;
     memcpy(p.sign_xor, c->sign_xor, sizeof(p.sign_xor));
     c->last_stream = stream;
     return cuda_status(launch_append(p, c->num_sms, static_cast<cudaStream_t>(stream)));
@@ -534,6 +536,7 @@ kvq_status kvq_decode_step(kvq_cache *c, const void *k_new, const void *v_new, c
                            size_t ws_bytes, void *out, void *stream)
 {
     if (!k_new) return KVQ_ERR_INVALID_ARG;
+    if (c && c->cfg.scale_search) return KVQ_ERR_UNSUPPORTED;  // the fused append does not search scales
     return decode_impl(c, k_new, v_new, slot_mapping, q, block_table, max_pages_per_seq, ctx_lens, batch,
                        softmax_scale, nullptr, workspace, ws_bytes, out, nullptr, stream);
 }

@@ -113,7 +113,63 @@ __device__ __forceinline__ void pair_err(float2 y, uint32_t c0, uint32_t c1, flo
     amax = max3(amax, fabsf(y.x), fabsf(y.y));
 }
 
-template <int D, int FMT>
+// Squared reconstruction error of NP pairs quantised with scale sf and zero
+// z (the codec's arithmetic), summed in fp32 with the even and the odd
+// elements apart, in order, then added.  The reconstruction and the sums use
+// the scalar _rn operations, which are never fused into a multiply-add (a
+// fused square-and-add rounds once instead of twice and was seen to move a
+// near-tie decision).
+template <int NP>
+__device__ __forceinline__ float run_sq_error(const float2 *y, float2 z2, float sf, float lo, float hi)
+{
+    const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
+    const float2 inv2 = make_float2(inv, inv);
+    float ev = 0.0f, od = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NP; i++) {
+        uint32_t c0, c1;
+        quant_pair(y[i], z2, inv2, lo, hi, c0, c1);
+        const float h0 = __fadd_rn(__fmul_rn(code_value(c0), sf), z2.x);
+        const float h1 = __fadd_rn(__fmul_rn(code_value(c1), sf), z2.x);
+        const float e0 = __fsub_rn(y[i].x, h0), e1 = __fsub_rn(y[i].y, h1);
+        ev = __fadd_rn(ev, __fmul_rn(e0, e0));
+        od = __fadd_rn(od, __fmul_rn(e1, e1));
+    }
+    return __fadd_rn(ev, od);
+}
+
+// ScaleSearch ["Search Your Block Floating Point Scales!", ScaleSearch] on
+// the fp16 scale: the candidates' bit patterns are the default's plus f,
+// tried as f = 0, -1, 1, -2, 2, 3, 4, 5, 6 (positive finite ones only); the
+// least squared error wins, a later candidate only if strictly better.  A
+// group spread over the row's two lanes adds the two lanes' sums (each lane
+// holds a run of 64 consecutive elements).  Every lane of the warp runs every
+// candidate, so the shuffle never diverges.
+template <int NP, int LANES>
+__device__ __forceinline__ __half search_scale(const float2 *y, __half sh0, float zf, float lo, float hi)
+{
+    const int b0 = __half_as_ushort(sh0);
+    const bool searchable = b0 != 0 && b0 < 0x7C00;
+    const float2 z2 = make_float2(zf, zf);
+    int best = b0;
+    float best_err = 0.0f;
+#pragma unroll 1
+    for (int k = 0; k < 9; k++) {
+        const int f = k == 0 ? 0 : k == 1 ? -1 : k == 2 ? 1 : k == 3 ? -2 : k - 2;
+        const int bits = b0 + f;
+        const bool valid = searchable && bits > 0 && bits < 0x7C00;
+        const float sf = valid ? __half2float(__ushort_as_half((unsigned short)bits)) : 0.0f;
+        float err = run_sq_error<NP>(y, z2, sf, lo, hi);
+        if constexpr (LANES == 2) err = __fadd_rn(err, __shfl_xor_sync(kFull, err, 16));
+        if (valid && (k == 0 || err < best_err)) {
+            best = bits;
+            best_err = err;
+        }
+    }
+    return __ushort_as_half((unsigned short)best);
+}
+
+template <int D, int FMT, bool SEARCH>
 __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *sign_xor, const unsigned char *src,
                                          unsigned char *chunk, int tok, int tensor, int s, bool active,
                                          unsigned int *desc)
@@ -192,8 +248,9 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
                 lo = __fmul_rn(lo, p.clip);
                 hi = __fmul_rn(hi, p.clip);
             }
-            const __half shh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
+            __half shh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
             const __half zhh = __float2half_rn(lo);
+            if constexpr (SEARCH) shh = search_scale<16, 1>(yg, shh, __half2float(zhh), 0.0f, 15.0f);
             const float sf = __half2float(shh), zf = __half2float(zhh);
             const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
             const float2 z2 = make_float2(zf, zf), inv2 = make_float2(inv, inv), s2 = make_float2(sf, sf);
@@ -229,8 +286,9 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
             lo = __fmul_rn(lo, p.clip);
             hi = __fmul_rn(hi, p.clip);
         }
-        const __half shh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 3.0f));
+        __half shh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 3.0f));
         const __half zhh = __float2half_rn(lo);
+        if constexpr (SEARCH) shh = search_scale<32, LANES>(y, shh, __half2float(zhh), 0.0f, 3.0f);
         const float sf = __half2float(shh), zf = __half2float(zhh);
         const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
         const float2 z2 = make_float2(zf, zf), inv2 = make_float2(inv, inv), s2 = make_float2(sf, sf);
@@ -267,7 +325,8 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
             for (int c = 0; c < 4; c++) am[c] = max3(am[c], fabsf(y[i + c].x), fabsf(y[i + c].y));
         float a = fmaxf(max3(am[0], am[1], am[2]), am[3]);
         a = row_max<LANES>(a);
-        const __half shh = __float2half_ru(__fdiv_rn(a, 127.0f));
+        __half shh = __float2half_ru(__fdiv_rn(a, 127.0f));
+        if constexpr (SEARCH) shh = search_scale<32, LANES>(y, shh, 0.0f, -127.0f, 127.0f);
         const float sf = __half2float(shh);
         const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
         if (want_desc) amax = a;
@@ -324,7 +383,7 @@ template <int D> struct AppendSmem {
     static constexpr int BYTES = kAppendWarps * 2 * BUF + kAppendWarps * 2 * 8;  // buffers + mbarriers
 };
 
-template <int D, int KF, int VF>
+template <int D, int KF, int VF, bool SEARCH>
 __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(const __grid_constant__ AppendParams p)
 {
     using S = AppendSmem<D>;
@@ -407,44 +466,61 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(const __grid_
             break;
         }
         const unsigned char *src = buf0 + bsel * S::BUF + r * S::STRIDE;
-        if (tensor == 0) half_row<D, KF>(p, sign_xor, src, chunk, tok, 0, s, active, desc);
-        else half_row<D, VF>(p, sign_xor, src, chunk, tok, 1, s, active, desc);
+        if (tensor == 0) half_row<D, KF, SEARCH>(p, sign_xor, src, chunk, tok, 0, s, active, desc);
+        else half_row<D, VF, SEARCH>(p, sign_xor, src, chunk, tok, 1, s, active, desc);
         __syncwarp();  // every lane is done with this buffer before it is refilled
     }
     (void)LANES;
 }
 
-template <int D, int KF, int VF>
-cudaError_t launch_one(const AppendParams &p, int blocks, cudaStream_t st)
+// Persistent grid: as many CTAs as stay resident (the instantiation's own
+// occupancy), at most one per eight groups of work.
+template <int D, int KF, int VF, bool SEARCH>
+cudaError_t launch_one_s(const AppendParams &p, long long want, int num_sms, cudaStream_t st)
 {
-    static bool configured = false;
-    if (!configured) {
-        const cudaError_t e = cudaFuncSetAttribute(append_kernel<D, KF, VF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   AppendSmem<D>::BYTES);
+    static int resident = 0;
+    if (resident == 0) {
+        cudaError_t e = cudaFuncSetAttribute(append_kernel<D, KF, VF, SEARCH>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, AppendSmem<D>::BYTES);
         if (e != cudaSuccess) return e;
-        configured = true;
+        int n = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, append_kernel<D, KF, VF, SEARCH>, kAppendWarps * 32,
+                                                          AppendSmem<D>::BYTES);
+        if (e != cudaSuccess) return e;
+        resident = n < 1 ? 1 : (n > 2 ? 2 : n);
     }
-    append_kernel<D, KF, VF><<<blocks, kAppendWarps * 32, AppendSmem<D>::BYTES, st>>>(p);
+    const long long cap = (long long)resident * num_sms;
+    const int blocks = (int)(want < cap ? want : cap);
+    append_kernel<D, KF, VF, SEARCH><<<blocks, kAppendWarps * 32, AppendSmem<D>::BYTES, st>>>(p);
     return cudaGetLastError();
 }
 
+// The scale search is its own instantiation so that the kernel without it
+// keeps its register budget (two CTAs per SM).
+template <int D, int KF, int VF>
+cudaError_t launch_one(const AppendParams &p, long long want, int num_sms, cudaStream_t st)
+{
+    return p.scale_search ? launch_one_s<D, KF, VF, true>(p, want, num_sms, st)
+                          : launch_one_s<D, KF, VF, false>(p, want, num_sms, st);
+}
+
 template <int D, int KF>
-cudaError_t launch_d_k(const AppendParams &p, int blocks, cudaStream_t st)
+cudaError_t launch_d_k(const AppendParams &p, long long want, int num_sms, cudaStream_t st)
 {
     switch (p.L.v_fmt) {
-    case KVQ_INT4_ASYM: return launch_one<D, KF, KVQ_INT4_ASYM>(p, blocks, st);
-    case KVQ_INT8_SYM: return launch_one<D, KF, KVQ_INT8_SYM>(p, blocks, st);
-    default: return launch_one<D, KF, KVQ_INT2_ASYM>(p, blocks, st);
+    case KVQ_INT4_ASYM: return launch_one<D, KF, KVQ_INT4_ASYM>(p, want, num_sms, st);
+    case KVQ_INT8_SYM: return launch_one<D, KF, KVQ_INT8_SYM>(p, want, num_sms, st);
+    default: return launch_one<D, KF, KVQ_INT2_ASYM>(p, want, num_sms, st);
     }
 }
 
 template <int D>
-cudaError_t launch_d(const AppendParams &p, int blocks, cudaStream_t st)
+cudaError_t launch_d(const AppendParams &p, long long want, int num_sms, cudaStream_t st)
 {
     switch (p.L.k_fmt) {
-    case KVQ_INT4_ASYM: return launch_d_k<D, KVQ_INT4_ASYM>(p, blocks, st);
-    case KVQ_INT8_SYM: return launch_d_k<D, KVQ_INT8_SYM>(p, blocks, st);
-    default: return launch_d_k<D, KVQ_INT2_ASYM>(p, blocks, st);
+    case KVQ_INT4_ASYM: return launch_d_k<D, KVQ_INT4_ASYM>(p, want, num_sms, st);
+    case KVQ_INT8_SYM: return launch_d_k<D, KVQ_INT8_SYM>(p, want, num_sms, st);
+    default: return launch_d_k<D, KVQ_INT2_ASYM>(p, want, num_sms, st);
     }
 }
 
@@ -458,8 +534,7 @@ cudaError_t launch_append(const AppendParams &p, int num_sms, cudaStream_t st)
     const int rows = p.L.d == 64 ? 32 : 16;
     const long long groups = 2 * ((rows_per_tensor + rows - 1) / rows);
     const long long want = (groups + kAppendWarps - 1) / kAppendWarps;
-    const int blocks = (int)(want < 2LL * num_sms ? want : 2LL * num_sms);  // two CTAs per SM stay resident
-    return p.L.d == 64 ? launch_d<64>(p, blocks, st) : launch_d<128>(p, blocks, st);
+    return p.L.d == 64 ? launch_d<64>(p, want, num_sms, st) : launch_d<128>(p, want, num_sms, st);
 }
 
 }  // namespace kvq

@@ -92,6 +92,7 @@ struct AppendParams {
     float clip;
     float rot_scale;
     int rotate;
+    int scale_search;
     uint32_t sign_xor[kMaxD / 2];
 };
 

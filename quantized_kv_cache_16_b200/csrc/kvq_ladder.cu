@@ -284,7 +284,32 @@ __global__ void __launch_bounds__(kSelThreads) ladder_finish_kernel(const __grid
     block_scan<kSelThreads, 5 * kMaxGqa, false, SumOp>(S, tot, scan_sm, tid, 5 * g);
 
     // ranking-consistency check per head over the key-promoted blocks
-    if (isfinite(p.rank_tol) && k_star >= 2) {
+    if (isfinite(p.rank_tol) && k_star >= 2 && k_star <= 32) {
+        // few blocks: one warp per head, lane i holds the i-th block and
+        // compares it with every block placed after it in the Phat order
+        const int32_t *prom = p.prom + bk * p.sort_cap;
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int h = warp; h < g; h += kSelThreads / 32) {
+            float ph = 0.f, pe = 0.f;
+            int bb = 0;
+            if (lane < k_star) {
+                bb = prom[lane] & kPromIdx;
+                ph = blk[(long long)bb * kBlkRec + h];
+                const float2 v = bml[(long long)bb * g + h];
+                pe = v.y * ex2(v.x - Rs[h]);
+            }
+            int fail = 0;
+            for (int j = 0; j < k_star; j++) {
+                const float phj = __shfl_sync(kFull, ph, j), pej = __shfl_sync(kFull, pe, j);
+                const int bj = __shfl_sync(kFull, bb, j);
+                const bool after = phj < ph || (phj == ph && bj > bb);
+                if (lane < k_star && after && pej > (1.f + p.rank_tol) * pe) fail = 1;
+            }
+            fail = __any_sync(kFull, fail);
+            if (lane == 0) fail_s[h] = fail;
+        }
+        __syncthreads();
+    } else if (isfinite(p.rank_tol) && k_star >= 2) {
         int np2 = 1;
         while (np2 < k_star) np2 <<= 1;
         const int32_t *prom = p.prom + bk * p.sort_cap;

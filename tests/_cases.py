@@ -19,7 +19,7 @@ def configs(wl: W.Workload, num_pages: int, rotate: int = 1):
     import quantized_kv_cache_16_b200 as K
     kw = dict(num_q_heads=wl.Hq, num_kv_heads=wl.Hkv, head_dim=wl.d, k_fmt=wl.k_fmt, v_fmt=wl.v_fmt,
               k_group=wl.k_group, v_group=wl.v_group, clip_ratio=wl.clip, rotation_seed=wl.rotation_seed,
-              rotate=rotate, num_pages=num_pages, bound_block_tokens=wl.bound_block)
+              rotate=rotate, num_pages=num_pages, bound_block_tokens=wl.bound_block, scale_search=wl.scale_search)
     return K.make_config(**kw), O.make_config(**kw)
 
 

@@ -60,6 +60,7 @@ class Workload:
     clip: float = 1.0
     bound_block: int = 0
     promote_frac: float = 0.0
+    scale_search: int = 0  # 1: the codec searches each scale (ScaleSearch)
     dist: str = "llama"  # tiny | llama | laplace | needle
     seed: int = 0
     rotation_seed: int = 0x5EED
