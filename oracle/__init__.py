@@ -123,6 +123,7 @@ def lib():
             "kvqo_decode_fp16": (i32, [cfgp, P, P, P, P, i32, P, i32, f64, P, P]),
             "kvqo_promote_count": (i32, [f64, i32]),
             "kvqo_decode_certified": (i32, [cfgp, P, P, P, P, P, i32, P, i32, f64, f64, P, P, P, i32, P, i32, P, P]),
+            "kvqo_decode_windows": (i32, [cfgp, P, P, P, i32, i32, P, P, i32, P, i32, f64, P]),
             "kvqo_decode_ladder": (i32, [cfgp, P, P, P, P, P, i32, P, i32, f64, C.POINTER(Ladder), P, P,
                                          C.POINTER(LadderOut)]),
         }
@@ -394,3 +395,22 @@ def decode_ladder(cfg: Config, pool: np.ndarray, k_slots, v_slots, q, block_tabl
     if rc != 0:
         raise ValueError(f"oracle ladder decode rejected its arguments (rc={rc})")
     return r
+
+
+def decode_windows(cfg: Config, pool: np.ndarray, win_k, win_v, sink: int, recent: int, q, block_table, ctx_lens,
+                   scale: float = 0.0) -> np.ndarray:
+    """Decode with each sequence's first `sink` and last `recent` tokens exact
+    (fp16 rows from the window store win_k/win_v [B, sink + recent, Hkv, d]:
+    row t for t < sink, row sink + t % recent for recent tokens)."""
+    wk = _c(win_k, np.float16).view(np.uint16)
+    wv = _c(win_v, np.float16).view(np.uint16)
+    q = _c(q, np.float16).view(np.uint16)
+    bt = _c(block_table, np.int32)
+    cl = _c(ctx_lens, np.int32)
+    B = cl.shape[0]
+    out = np.zeros((B, cfg.num_q_heads, cfg.head_dim), np.float64)
+    rc = lib().kvqo_decode_windows(C.byref(cfg), _p(pool), _p(wk), _p(wv), sink, recent, _p(q), _p(bt), bt.shape[1],
+                                   _p(cl), B, scale, _p(out))
+    if rc != 0:
+        raise ValueError(f"oracle window decode rejected its arguments (rc={rc})")
+    return out

@@ -1317,6 +1317,70 @@ int kvqo_decode_ladder(const kvqo_config *c, const uint8_t *pool, const uint16_t
 }
 
 /* ------------------------------------------------------------------------- */
+/* Sink and recent windows at 16-bit precision ([OSCAR] 2.2b)                */
+/* ------------------------------------------------------------------------- */
+
+/* Decode where each sequence's first `sink` tokens and last `recent` tokens
+ * attend with their fp16 rows and the tokens between with the quantised
+ * cache: the page keeps the sink and recent tokens at full precision and the
+ * middle history low-bit ([OSCAR] 2.2b, mixed-precision layout).  Window
+ * rows come from a compact store win_k/win_v, fp16 [B][sink + recent][Hkv][d]:
+ * row t for t < sink, row sink + t % recent for a recent token t (a ring
+ * the caller keeps current).  Windows overlap when T < sink + recent; a token
+ * is exact when it is in either.  Attention in fp64 in the rotated domain,
+ * output inverse-rotated.  Returns 0, -1 (bad table or length), -2 (bad
+ * config) or -3 (negative window sizes). */
+int kvqo_decode_windows(const kvqo_config *c, const uint8_t *pool, const uint16_t *win_k, const uint16_t *win_v,
+                        int sink, int recent, const uint16_t *q, const int32_t *block_table, int max_pages,
+                        const int32_t *ctx_lens, int B, double scale, double *out)
+{
+    if (!kvqo_config_ok(c)) return -2;
+    if (sink < 0 || recent < 0) return -3;
+    if (!decode_args_ok(c, block_table, max_pages, ctx_lens, B)) return -1;
+    int d = c->head_dim, hq = c->num_q_heads, hkv = c->num_kv_heads, g = hq / hkv;
+    int W = sink + recent;
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    float s[KVQO_MAXD];
+    kvqo_signs(c->rotation_seed, d, s);
+    for (int b = 0; b < B; b++) {
+        int T = ctx_lens[b];
+        for (int kvh = 0; kvh < hkv; kvh++) {
+            double *K = (double *)malloc(sizeof(double) * ((size_t)T * d + 1));
+            double *V = (double *)malloc(sizeof(double) * ((size_t)T * d + 1));
+            for (int t = 0; t < T; t++) {
+                int in_sink = t < sink, in_recent = recent > 0 && t >= T - recent;
+                if (in_sink || in_recent) {
+                    int row = in_sink ? t : sink + t % recent;
+                    size_t off = (((size_t)b * W + row) * hkv + kvh) * d;
+                    double xk[KVQO_MAXD], xv[KVQO_MAXD];
+                    for (int i = 0; i < d; i++) {
+                        xk[i] = kvqo_h2f(win_k[off + i]);
+                        xv[i] = kvqo_h2f(win_v[off + i]);
+                    }
+                    kvqo_rotate_f64(xk, s, d, c->rotate, K + (size_t)t * d);
+                    kvqo_rotate_f64(xv, s, d, c->rotate, V + (size_t)t * d);
+                } else {
+                    int slot = slot_of(block_table, max_pages, b, t);
+                    kvqo_dequant_row(c, pool, slot, kvh, 0, K + (size_t)t * d);
+                    kvqo_dequant_row(c, pool, slot, kvh, 1, V + (size_t)t * d);
+                }
+            }
+            for (int hh = 0; hh < g; hh++) {
+                int h = kvh * g + hh;
+                double qx[KVQO_MAXD], qr[KVQO_MAXD], orot[KVQO_MAXD];
+                for (int i = 0; i < d; i++) qx[i] = (double)kvqo_h2f(q[((size_t)b * hq + h) * d + i]);
+                kvqo_rotate_f64(qx, s, d, c->rotate, qr);
+                kvqo_attend(qr, K, V, T, d, scale, 1, orot);
+                kvqo_inv_rotate_f64(orot, s, d, c->rotate, out + ((size_t)b * hq + h) * d);
+            }
+            free(K);
+            free(V);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Array helpers for the tests                                               */
 /* ------------------------------------------------------------------------- */
 
