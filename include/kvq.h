@@ -17,6 +17,8 @@
  *    cache, dequantised in registers, merged across context splits by the
  *    log-sum-exp rule, inverse-rotated ["OSCAR", 2.2b (fused kernel: unpack,
  *    dequantise, inverse rotation, attention over a paged cache)].
+ *  - Sink and recent windows: the first and the latest tokens at fp16, the
+ *    middle history quantised ["OSCAR", 2.2b, mixed-precision layout].
  *  - Certified mode: per-block key/value error bounds, top-fraction promotion
  *    of blocks to their fp16 originals held in pinned host memory, and the
  *    adaptive ladder (coverage-driven key promotion, value promotion, the
@@ -177,6 +179,32 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int32_t batch, int32_t
 kvq_status kvq_decode_attn(kvq_cache *cache, const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
                            const int32_t *ctx_lens, int32_t batch, float softmax_scale, const kvq_tier2 *tier2,
                            void *workspace, size_t ws_bytes, void *out, int32_t *promoted_out, void *stream);
+
+/* Workspace bytes kvq_decode_windows needs (zero-filled before first use;
+ * every call leaves it ready for the next). */
+size_t kvq_decode_windows_workspace_bytes(const kvq_cache *cache, int32_t batch, int32_t max_pages_per_seq);
+
+/* Decode with 16-bit sink and recent windows ["OSCAR", 2.2b: the paged cache
+ * keeps the first (sink) and the most recent tokens at full precision and
+ * the middle history low-bit]: as kvq_decode_attn, except that each
+ * sequence's first `sink` tokens and last `recent` tokens attend with their
+ * fp16 rows from a compact window store, the rest with the quantised cache.
+ *   k_win, v_win: fp16 [batch][sink + recent][Hkv][d] (not rotated; device
+ *                 memory or pinned host memory, 16-byte aligned): row t holds
+ *                 token t for t < sink; row sink + t % recent holds token t
+ *                 of the recent window.  The caller keeps the store current
+ *                 (write each new token's row at sink + t % recent when it is
+ *                 appended; rows of tokens outside both windows are not read).
+ *   sink, recent: >= 0; a token in both windows is read from its sink row.
+ * The quantised decode runs first over the tokens between the windows (the
+ * window tokens are in the pool too, but masked out of that pass); then up
+ * to 16 CTAs per (sequence, kv head) attend over the window rows and merge
+ * their partial into the output by the log-sum-exp rule.  Two launches; one
+ * when both windows are empty.  Workspace: kvq_decode_windows_workspace_bytes. */
+kvq_status kvq_decode_windows(kvq_cache *cache, const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
+                              const int32_t *ctx_lens, int32_t batch, float softmax_scale, const void *k_win,
+                              const void *v_win, int32_t sink, int32_t recent, void *workspace, size_t ws_bytes,
+                              void *out, void *stream);
 
 /* Policy of the certified ladder ["Runtime-Certified Bounded-Error Quantized
  * Attention", Methodology 3: adaptive Top-K, ranking-consistency check,

@@ -24,7 +24,8 @@ PAGE_TOKENS = 16
 # Every symbol include/kvq.h declares (checked by the ABI test).
 EXPORTS = (
     "kvq_pool_bytes", "kvq_create_cache", "kvq_destroy_cache", "kvq_append", "kvq_reset_pages",
-    "kvq_decode_workspace_bytes", "kvq_decode_attn", "kvq_decode_certified", "kvq_decode_step",
+    "kvq_decode_workspace_bytes", "kvq_decode_attn", "kvq_decode_certified", "kvq_decode_windows",
+    "kvq_decode_windows_workspace_bytes", "kvq_decode_step",
     "kvq_decode_attn_static", "kvq_dequant_debug", "kvq_sync_status",
     "kvq_status_string",
 )
@@ -87,6 +88,8 @@ def lib() -> C.CDLL:
             "kvq_decode_attn": (i32, [P, P, P, i32, P, i32, C.c_float, C.POINTER(kvq_tier2), P, sz, P, P, P]),
             "kvq_decode_certified": (i32, [P, P, P, i32, P, i32, C.c_float, P, P, C.POINTER(kvq_ladder), P, sz,
                                            P, C.POINTER(kvq_ladder_report), P]),
+            "kvq_decode_windows": (i32, [P, P, P, i32, P, i32, C.c_float, P, P, i32, i32, P, sz, P, P]),
+            "kvq_decode_windows_workspace_bytes": (sz, [P, i32, i32]),
             "kvq_decode_step": (i32, [P, P, P, P, P, P, i32, P, i32, C.c_float, P, sz, P, P]),
             "kvq_decode_attn_static": (i32, [P, P, P, i32, P, i32, C.c_float, P, P]),
             "kvq_dequant_debug": (i32, [P, P, i32, P, P, P, P, P]),
@@ -180,6 +183,18 @@ def kvq_decode_certified(cache, q, block_table, max_pages_per_seq: int, ctx_lens
                                       ws_bytes, _ptr(out), rep, _stream(stream)))
 
 
+def kvq_decode_windows_workspace_bytes(cache, batch: int, max_pages_per_seq: int) -> int:
+    return int(lib().kvq_decode_windows_workspace_bytes(cache, batch, max_pages_per_seq))
+
+
+def kvq_decode_windows(cache, q, block_table, max_pages_per_seq: int, ctx_lens, batch: int, softmax_scale: float,
+                       k_win, v_win, sink: int, recent: int, workspace, ws_bytes: int, out, stream=None) -> None:
+    _check("kvq_decode_windows",
+           lib().kvq_decode_windows(cache, _ptr(q), _ptr(block_table), max_pages_per_seq, _ptr(ctx_lens), batch,
+                                    softmax_scale, _ptr(k_win), _ptr(v_win), sink, recent, _ptr(workspace), ws_bytes,
+                                    _ptr(out), _stream(stream)))
+
+
 def kvq_decode_step(cache, k_new, v_new, slot_mapping, q, block_table, max_pages_per_seq: int, ctx_lens,
                     batch: int, softmax_scale: float, workspace, ws_bytes: int, out, stream=None) -> None:
     _check("kvq_decode_step",
@@ -245,7 +260,8 @@ class Cache:
 
     def workspace_for(self, batch: int, max_pages: int):
         import torch
-        need = kvq_decode_workspace_bytes(self.handle, batch, max_pages)
+        need = max(kvq_decode_workspace_bytes(self.handle, batch, max_pages),
+                   kvq_decode_windows_workspace_bytes(self.handle, batch, max_pages))
         if self.workspace is None or self.workspace.numel() < need:
             self.workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=self.pool.device)
         return self.workspace
@@ -297,6 +313,20 @@ class Cache:
         kvq_decode_certified(self.handle, q, block_table, max_pages, ctx_lens, batch, softmax_scale, k_tier2,
                              v_tier2, pol, ws, ws.numel(), out, rep, stream)
         return (out, rd) if report else out
+
+    def decode_windows(self, q, block_table, ctx_lens, k_win, v_win, sink: int, recent: int, out=None,
+                       softmax_scale: float = 0.0, stream=None):
+        """Decode with each sequence's first `sink` and last `recent` tokens
+        at fp16 from the window store k_win / v_win [B, sink + recent, Hkv, d]
+        (row t for t < sink, row sink + t % recent for recent tokens)."""
+        import torch
+        batch, max_pages = block_table.shape
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        ws = self.workspace_for(batch, max_pages)
+        kvq_decode_windows(self.handle, q, block_table, max_pages, ctx_lens, batch, softmax_scale, k_win, v_win, sink,
+                           recent, ws, ws.numel(), out, stream)
+        return out
 
     def step(self, k_new, v_new, slot_mapping, q, block_table, ctx_lens, out=None, softmax_scale: float = 0.0,
              stream=None):

@@ -167,6 +167,28 @@ CertWs cert_ws(const kvq_cache *c, int batch, int max_pages)
     return w;
 }
 
+// Window-decode workspace, after the decode partials and the certified-mode
+// regions: per-head softmax totals, the correction partials and their
+// counters (zero between calls).
+struct WinWs {
+    size_t head_ml, cpart, ccount, bytes;
+};
+
+WinWs win_ws(const kvq_cache *c, int batch)
+{
+    WinWs w{};
+    const size_t bk = (size_t)batch * c->L.hkv, g = c->L.g;
+    size_t off = 0;
+    w.head_ml = off;
+    off += round256(bk * g * 8);
+    w.cpart = off;
+    off += round256(bk * kCertChunks * g * (3 * c->L.d + 4) * 4);
+    w.ccount = off;
+    off += round256(bk * 4);
+    w.bytes = off;
+    return w;
+}
+
 // Dense-fallback split: at most kDenseSplitsMax splits of >= 1024 tokens
 // (a multiple of 64) per (sequence, kv head).
 void dense_split(int max_pages, int *n_split, int *tokens)
@@ -288,6 +310,15 @@ kvq_status kvq_reset_pages(kvq_cache *c, const int32_t *page_ids, int32_t n, voi
     if (n == 0 || c->L.desc_off == 0) return KVQ_OK;
     c->last_stream = stream;
     return cuda_status(launch_reset_pages(c->pool, c->L, page_ids, n, static_cast<cudaStream_t>(stream)));
+}
+
+size_t kvq_decode_windows_workspace_bytes(const kvq_cache *c, int32_t batch, int32_t max_pages_per_seq)
+{
+    if (!c || batch < 0 || max_pages_per_seq < 1) return 0;
+    const SplitPlan s = plan_splits(c, batch, max_pages_per_seq);
+    const size_t part = (size_t)batch * c->L.hkv * s.n_splits * c->L.g * (c->L.d + 4) * sizeof(float);
+    return counters_bytes(batch, c->L.hkv) + round256(part) + cert_ws(c, batch, max_pages_per_seq).bytes +
+           win_ws(c, batch).bytes;
 }
 
 size_t kvq_decode_workspace_bytes(const kvq_cache *c, int32_t batch, int32_t max_pages_per_seq)
@@ -512,6 +543,63 @@ kvq_status ladder_impl(kvq_cache *c, const void *q, const int32_t *block_table, 
 }  // namespace
 
 extern "C" {
+
+kvq_status kvq_decode_windows(kvq_cache *c, const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
+                              const int32_t *ctx_lens, int32_t batch, float softmax_scale, const void *k_win,
+                              const void *v_win, int32_t sink, int32_t recent, void *workspace, size_t ws_bytes,
+                              void *out, void *stream)
+{
+    if (!c || batch < 0 || max_pages_per_seq < 1 || sink < 0 || recent < 0) return KVQ_ERR_INVALID_ARG;
+    if (batch == 0) return KVQ_OK;
+    if (!q || !block_table || !ctx_lens || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
+    if (!decode_supported(c->L)) return KVQ_ERR_UNSUPPORTED;
+    const void *k2 = nullptr, *v2 = nullptr;
+    if (sink + recent > 0) {
+        k2 = device_view(k_win);
+        v2 = device_view(v_win);
+        if (!k2 || !v2 || !aligned(k2, 16) || !aligned(v2, 16)) return KVQ_ERR_INVALID_ARG;
+    }
+    if (ws_bytes < kvq_decode_windows_workspace_bytes(c, batch, max_pages_per_seq)) return KVQ_ERR_CAPACITY;
+    const SplitPlan s = plan_splits(c, batch, max_pages_per_seq);
+    const float scale = softmax_scale > 0.0f ? softmax_scale : (float)(1.0 / sqrt((double)c->L.d));
+    DecodeParams p = decode_params(c, s, q, block_table, max_pages_per_seq, ctx_lens, batch, scale, workspace, out);
+    // the window regions follow every certified-mode region, so calls of the
+    // two kinds can share one workspace (each leaves its own counters zero)
+    unsigned char *base = cert_base(c, s, batch, workspace) + cert_ws(c, batch, max_pages_per_seq).bytes;
+    const WinWs w = win_ws(c, batch);
+    if (sink + recent > 0) {
+        p.head_ml = reinterpret_cast<float2 *>(base + w.head_ml);
+        p.win_sink = sink;  // the quantised pass leaves the window tokens out
+        p.win_recent = recent;
+    }
+    c->last_stream = stream;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    kvq_status rc = cuda_status(launch_decode(p, dim3(s.n_splits, c->L.hkv, batch), st));
+    if (rc != KVQ_OK || sink + recent == 0) return rc;
+    CertParams cp{};
+    cp.pool = c->pool;
+    cp.q = p.q;
+    cp.block_table = block_table;
+    cp.ctx_lens = ctx_lens;
+    cp.max_pages = max_pages_per_seq;
+    cp.L = c->L;
+    cp.scale = scale;
+    cp.qscale = p.qscale;
+    cp.rot_scale = c->rot_scale;
+    cp.rotate = c->cfg.rotate;
+    memcpy(cp.signs, c->signs, sizeof(cp.signs));
+    cp.head_ml = p.head_ml;
+    cp.n_chunks = kCertChunks;
+    cp.k2 = static_cast<const __half *>(k2);
+    cp.v2 = static_cast<const __half *>(v2);
+    cp.sink = sink;
+    cp.recent = recent;
+    cp.cpart = reinterpret_cast<float *>(base + w.cpart);
+    cp.ccount = reinterpret_cast<unsigned int *>(base + w.ccount);
+    cp.out = p.out;
+    return cuda_status(launch_windows(cp, batch, st));
+}
 
 kvq_status kvq_decode_certified(kvq_cache *c, const void *q, const int32_t *block_table, int32_t max_pages_per_seq,
                                 const int32_t *ctx_lens, int32_t batch, float softmax_scale, const void *k_tier2,

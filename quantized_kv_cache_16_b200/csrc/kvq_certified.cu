@@ -196,7 +196,14 @@ __global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_c
 // original domain: an exact key's score is q.k there (equal to (Rq).(Rk),
 // R orthogonal) and exact values are summed unrotated; only the dequantised
 // rows live in the rotated domain.
-template <int D, int G>
+// WIN: the exact tokens are a sequence's sink and recent windows instead of
+// promoted blocks; their fp16 rows come from the compact window store (row
+// t for t < sink, row sink + t % recent for a recent token), and each CTA
+// takes a contiguous share of the window tokens.  The quantised pass left
+// those tokens out, so there is no quantised side to take away: the merge
+// adds the exact partial to the quantised one (a plain log-sum-exp merge;
+// the quantised side's mass is 0).
+template <int D, int G, bool WIN>
 __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid_constant__ CertParams p)
 {
     pdl_enter();
@@ -206,7 +213,20 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = L.g;
     const long long bk = (long long)b * L.hkv + kvh;
-    const int kp = p.prom_count[bk];
+    const int T = clamp_ctx(p.ctx_lens[b], p.max_pages);
+    // window tokens: [0, ns) and [lo_r, T), nwin in all, `per` a CTA
+    int kp, ns = 0, lo_r = 0, nwin = 0, per = 0;
+    if constexpr (WIN) {
+        ns = min(p.sink, T);
+        lo_r = p.recent > 0 ? max(p.sink, T - p.recent) : T;
+        lo_r = min(lo_r, T);
+        nwin = ns + (T - lo_r);
+        constexpr int span = kPromWarps * kTokBatch;
+        kp = min(p.n_chunks, (nwin + span - 1) / span);
+        per = kp > 0 ? (nwin + kp - 1) / kp : 0;
+    } else {
+        kp = p.prom_count[bk];
+    }
     const int n_act = min(kp, p.n_chunks);
     if (chunk_id >= n_act) return;
 
@@ -219,10 +239,9 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
     __shared__ float2 bsm[2][kPromWarps][G];
     __shared__ int sflag;
 
-    const int T = clamp_ctx(p.ctx_lens[b], p.max_pages);
     const int block = L.bound_block;
     const int32_t *bt = p.block_table + (long long)b * p.max_pages;
-    const int32_t *prom = p.prom + bk * p.sort_cap;
+    const int32_t *prom = WIN ? nullptr : p.prom + bk * p.sort_cap;
 
     // queries in log2 units: rotated (against dequantised keys) and original
     // (against exact keys)
@@ -261,10 +280,20 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
 
     int parity = 0;
     for (int r = chunk_id; r < kp; r += n_act, parity ^= 1) {
-        const int ent = prom[r];
-        const int blk_id = ent & kPromIdx;
-        const bool kx = (ent & kPromKey) != 0, vx = (ent & kPromVal) != 0;
-        const int t0 = blk_id * block, t1 = min(t0 + block, T);
+        // this segment: positions (WIN: window indices) [t0, t1)
+        int blk_id = 0, t0, t1;
+        bool kx = true, vx = true;
+        if constexpr (WIN) {
+            t0 = r * per;
+            t1 = min(nwin, t0 + per);
+        } else {
+            const int ent = prom[r];
+            blk_id = ent & kPromIdx;
+            kx = (ent & kPromKey) != 0;
+            vx = (ent & kPromVal) != 0;
+            t0 = blk_id * block;
+            t1 = min(t0 + block, T);
+        }
         float bm[G], bl[G];
 #pragma unroll
         for (int h = 0; h < G; h++) {
@@ -274,18 +303,26 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
         for (int tb = t0 + warp * kTokBatch; tb < t1; tb += kPromWarps * kTokBatch) {
             // issue the batch's exact-row loads (host link) before any math
             RawRow<E> kraw[kTokBatch], vraw[kTokBatch];
-            int pgs[kTokBatch];
+            int pgs[kTokBatch], toks[kTokBatch];
 #pragma unroll
             for (int u = 0; u < kTokBatch; u++) {
-                const int t = tb + u;
-                int pg = -1;
-                if (t < t1) {
+                int t = -1, pg = -1;
+                if (tb + u < t1) {
+                    t = tb + u;
+                    if constexpr (WIN) t = t < ns ? t : lo_r + (t - ns);
                     pg = bt[t / kPageTokens];
                     if (pg >= L.num_pages) pg = -1;
                 }
                 pgs[u] = pg;
+                toks[u] = t % kPageTokens;
                 if (pg >= 0) {
-                    const long long row = ((long long)(pg * kPageTokens + t % kPageTokens) * L.hkv + kvh) * D + lane * E;
+                    long long row;
+                    if constexpr (WIN) {
+                        const int wrow = t < p.sink ? t : p.sink + t % p.recent;
+                        row = (((long long)b * (p.sink + p.recent) + wrow) * L.hkv + kvh) * D + lane * E;
+                    } else {
+                        row = ((long long)(pg * kPageTokens + t % kPageTokens) * L.hkv + kvh) * D + lane * E;
+                    }
                     if (kx) kraw[u].load(p.k2 + row);
                     if (vx) vraw[u].load(p.v2 + row);
                 }
@@ -293,12 +330,14 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
 #pragma unroll
             for (int u = 0; u < kTokBatch; u++) {
                 if (pgs[u] < 0) continue;  // warp-uniform
-                const int tok = (tb + u) % kPageTokens;
+                const int tok = toks[u];
                 const unsigned char *chunk =
                     p.pool + kHeaderBytes + (long long)pgs[u] * L.page_bytes + (long long)kvh * L.chunk_bytes;
-                float kq[E], vq[E], ke[E] = {}, ve[E] = {};
-                dequant_lane<E>(chunk, L.k_codes, L.k_meta, L.k_row_meta, L.k_fmt, tok, lane, kq);
-                dequant_lane<E>(chunk, L.v_codes, L.v_meta, L.v_row_meta, L.v_fmt, tok, lane, vq);
+                float kq[E] = {}, vq[E] = {}, ke[E] = {}, ve[E] = {};
+                if constexpr (!WIN) {  // windows: the quantised pass left these tokens out
+                    dequant_lane<E>(chunk, L.k_codes, L.k_meta, L.k_row_meta, L.k_fmt, tok, lane, kq);
+                    dequant_lane<E>(chunk, L.v_codes, L.v_meta, L.v_row_meta, L.v_fmt, tok, lane, vq);
+                }
                 if (kx) kraw[u].widen(ke);
                 if (vx) vraw[u].widen(ve);
 #pragma unroll
@@ -318,16 +357,16 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
                     float sqv = 0.f, se = 0.f;
 #pragma unroll
                     for (int e = 0; e < E; e++) {
-                        sqv = fmaf(qr[h][e], kq[e], sqv);
+                        if constexpr (!WIN) sqv = fmaf(qr[h][e], kq[e], sqv);
                         se = fmaf(qo[e], ke[e], se);
                     }
 #pragma unroll
                     for (int mm = 16; mm >= 1; mm >>= 1) {
-                        sqv += __shfl_xor_sync(kFull, sqv, mm);
+                        if constexpr (!WIN) sqv += __shfl_xor_sync(kFull, sqv, mm);
                         if (kx) se += __shfl_xor_sync(kFull, se, mm);
                     }
                     if (!kx) se = sqv;
-                    online_update<E>(m[h][1], l[h][1], aq[h], sqv, vq);
+                    if constexpr (!WIN) online_update<E>(m[h][1], l[h][1], aq[h], sqv, vq);
                     {  // the mixed side: one (m, l), two sums
                         const float mn = fmaxf(m[h][0], se);
                         const float al = (m[h][0] == -INFINITY) ? 0.f : ex2(m[h][0] - mn);
@@ -513,35 +552,40 @@ cudaError_t launch_cert_select(const CertParams &p, int batch, cudaStream_t s)
               : launch_pdl(cert_select_kernel<64>, grid, kSelThreads, smem, s, p);
 }
 
-template <int D, int G>
+template <int D, int G, bool WIN>
 cudaError_t launch_promote_t(const CertParams &p, int batch, cudaStream_t s)
 {
     static bool configured = false;
     if (!configured) {
         const int cap = kPromWarps * G * 3 * D * (int)sizeof(float);
         const cudaError_t e =
-            cudaFuncSetAttribute(cert_promote_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
+            cudaFuncSetAttribute(cert_promote_kernel<D, G, WIN>, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
         if (e != cudaSuccess) return e;
         configured = true;
     }
     const size_t smem = (size_t)kPromWarps * p.L.g * 3 * D * sizeof(float);
     const dim3 grid(p.n_chunks, p.L.hkv, batch);
-    return launch_pdl(cert_promote_kernel<D, G>, grid, kPromThreads, smem, s, p);
+    return launch_pdl(cert_promote_kernel<D, G, WIN>, grid, kPromThreads, smem, s, p);
 }
 
-template <int D>
+template <int D, bool WIN>
 cudaError_t launch_promote_d(const CertParams &p, int batch, cudaStream_t s)
 {
     const int g = p.L.g;
-    if (g <= 1) return launch_promote_t<D, 1>(p, batch, s);
-    if (g <= 2) return launch_promote_t<D, 2>(p, batch, s);
-    if (g <= 4) return launch_promote_t<D, 4>(p, batch, s);
-    return launch_promote_t<D, 8>(p, batch, s);
+    if (g <= 1) return launch_promote_t<D, 1, WIN>(p, batch, s);
+    if (g <= 2) return launch_promote_t<D, 2, WIN>(p, batch, s);
+    if (g <= 4) return launch_promote_t<D, 4, WIN>(p, batch, s);
+    return launch_promote_t<D, 8, WIN>(p, batch, s);
 }
 
 cudaError_t launch_cert_promote(const CertParams &p, int batch, cudaStream_t s)
 {
-    return p.L.d == 128 ? launch_promote_d<128>(p, batch, s) : launch_promote_d<64>(p, batch, s);
+    return p.L.d == 128 ? launch_promote_d<128, false>(p, batch, s) : launch_promote_d<64, false>(p, batch, s);
+}
+
+cudaError_t launch_windows(const CertParams &p, int batch, cudaStream_t s)
+{
+    return p.L.d == 128 ? launch_promote_d<128, true>(p, batch, s) : launch_promote_d<64, true>(p, batch, s);
 }
 
 }  // namespace kvq

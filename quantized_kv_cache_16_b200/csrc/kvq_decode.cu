@@ -562,6 +562,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     const int n_pages = (T + kPageTokens - 1) / kPageTokens;
     const int n_active = max(1, (n_pages + p.pages_per_split - 1) / p.pages_per_split);
     if (split >= n_active) return;
+    const int q_lo = min(p.win_sink, T), q_hi = max(q_lo, T - p.win_recent);  // tokens attended here
 
     int8_t *qv = reinterpret_cast<int8_t *>(smem + C::OFF_QV);
     float *qsum = reinterpret_cast<float *>(smem + C::OFF_QSUM);
@@ -771,11 +772,13 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             break;
         }
         const int t0 = (p_begin + i) * kPageTokens;
-        const int nvalid = min(kPageTokens, T - t0);
+        // valid tokens of the page: [vlo, vhi) (the tail, and windows attended elsewhere)
+        const int vlo = min(max(q_lo - t0, 0), kPageTokens);
+        const int vhi = min(max(q_hi - t0, 0), kPageTokens);
         const uint32_t sb = stage0 + st * C::STAGE;
         const unsigned char *sp = stage0_ptr + st * C::STAGE;
         const bool page_ok = (vbits >> st) & 1u;
-        const bool ragged = nvalid < kPageTokens || !page_ok;
+        const bool ragged = vlo > 0 || vhi < kPageTokens || !page_ok;
 
         // ---------------- QK: scores of tokens r, r+8 for the lane's heads ----
         float s_r[NH], s_r8[NH];
@@ -851,8 +854,8 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
                 s_r[t] = fmaf(acc_r[t], qinv[t], zr[t]);
                 s_r8[t] = fmaf(acc_r8[t], qinv[t], zr8[t]);
                 if (ragged) {
-                    if (r >= nvalid || !page_ok) s_r[t] = -INFINITY;
-                    if (r + 8 >= nvalid || !page_ok) s_r8[t] = -INFINITY;
+                    if (r < vlo || r >= vhi || !page_ok) s_r[t] = -INFINITY;
+                    if (r + 8 < vlo || r + 8 >= vhi || !page_ok) s_r8[t] = -INFINITY;
                 }
             }
         }
@@ -919,7 +922,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             load_h<VC::NG>(vmeta_r, sv_r);
             load_h<VC::NG>(vmeta_r8, sv_r8);
             if (ragged) {
-                const bool v_r = page_ok && r < nvalid, v_r8 = page_ok && r + 8 < nvalid;
+                const bool v_r = page_ok && r >= vlo && r < vhi, v_r8 = page_ok && r + 8 >= vlo && r + 8 < vhi;
 #pragma unroll
                 for (int gi = 0; gi < VC::NG; gi++) {
                     sv_r[gi] = v_r ? sv_r[gi] : 0.f;
@@ -935,10 +938,10 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
                 uint32_t z2 = *reinterpret_cast<const uint16_t *>(zrow + (2 * j + 8) * VC::ROW_META);
                 uint32_t z3 = *reinterpret_cast<const uint16_t *>(zrow + (2 * j + 9) * VC::ROW_META);
                 if (ragged) {
-                    if (!page_ok || 2 * j >= nvalid) z0 = 0;
-                    if (!page_ok || 2 * j + 1 >= nvalid) z1 = 0;
-                    if (!page_ok || 2 * j + 8 >= nvalid) z2 = 0;
-                    if (!page_ok || 2 * j + 9 >= nvalid) z3 = 0;
+                    if (!page_ok || 2 * j < vlo || 2 * j >= vhi) z0 = 0;
+                    if (!page_ok || 2 * j + 1 < vlo || 2 * j + 1 >= vhi) z1 = 0;
+                    if (!page_ok || 2 * j + 8 < vlo || 2 * j + 8 >= vhi) z2 = 0;
+                    if (!page_ok || 2 * j + 9 < vlo || 2 * j + 9 >= vhi) z3 = 0;
                 }
                 az[0] = z0 | (z1 << 16);
                 az[2] = z2 | (z3 << 16);

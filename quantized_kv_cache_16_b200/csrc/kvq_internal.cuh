@@ -122,6 +122,9 @@ struct DecodeParams {
     // certified mode: per page and head (m, l) = (running max, sum of
     // 2^(s - m) over the page's tokens), log2 units; null = off
     float2 *page_stats;       // [B][Hkv][max_pages][g]
+    // sink and recent windows attended elsewhere (0, 0 = none): only tokens
+    // [min(sink, T), max(that, T - recent)) are attended here
+    int win_sink, win_recent;
     float2 *head_ml;          // [B][Hkv][g]: totals (M, L) of the softmax, certified mode only
 };
 
@@ -195,6 +198,7 @@ struct CertParams {
     int nb_out;
     float *bound_out;          // optional [B][Hq]
     int32_t *status_out;       // optional [B][Hq]
+    int sink, recent;             // window decode: the store's sink rows and recent ring length (k2/v2 = the store)
     int n_dsplit, dsplit_tokens;  // dense fallback: splits per (sequence, kv head) and tokens per split
     int batch, dense_ctas;        // the persistent dense-fallback grid
     float *dpart;              // [B][Hkv][n_dsplit][g][d + 4]
@@ -218,6 +222,7 @@ cudaError_t launch_cert_select(const CertParams &p, int batch, cudaStream_t s);
 cudaError_t launch_cert_promote(const CertParams &p, int batch, cudaStream_t s);
 cudaError_t launch_ladder_select(const CertParams &p, int batch, cudaStream_t s);
 cudaError_t launch_ladder_finish(const CertParams &p, int batch, cudaStream_t s);
+cudaError_t launch_windows(const CertParams &p, int batch, cudaStream_t s);
 bool decode_supported(const Layout &L);
 int decode_max_splits(const Layout &L);
 constexpr int kDecodeWarps = 8;
