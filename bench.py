@@ -39,8 +39,8 @@ NOMINAL_HBM_GBS = 8000.0
 # capture summarised under profiles/ (decode_kernel_llama3-8b-layer-T32768.md).
 # Reported as roofline.traffic only while the decode kernel's sources hash to
 # the digest they had when the counters were taken; null otherwise.
-PROFILED_DECODE = {"sources_sha256": "6aeb408ca39736939021e873beb39d0c1d62850781346d41c57dcaf757be5ce1",
-                   "dram_bytes_per_launch": 42130176}
+PROFILED_DECODE = {"sources_sha256": "473c0c7612212fb4025186ee5fc5a2d1c1bd87c9da5b2832a5836b9cf77575d1",
+                   "dram_bytes_per_launch": 42148224}
 DECODE_SOURCES = ("kvq_decode.cu", "kvq_internal.cuh", "kvq_warp.cuh")
 
 
@@ -76,7 +76,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-steps", type=int, default=4, help="oracle steps in the CPU baseline sample")
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, append and CPU legs")
-    ap.add_argument("--leg", choices=["certified", "ladder"],
+    ap.add_argument("--leg", choices=["certified", "ladder", "windows"],
                     help="run only this leg (one GPU, --steps calls) and print its JSON")
     ap.add_argument("--ctx", type=int, default=0, help="context length of --leg (default: its workload's)")
     return ap.parse_args()
@@ -395,6 +395,7 @@ def run_ours(args, dist: Dist):
         result["append"] = append_leg()
         result["certified"] = certified_leg(min(K, 200))
         result["ladder"] = ladder_leg(min(K, 100))
+        result["windows"] = windows_leg(min(K, 200))
     if dist.rank == 0:
         if not args.no_extras:
             result["cpu_baseline"] = cpu_leg(wk, args.cpu_steps)
@@ -610,6 +611,65 @@ def certified_leg(steps: int, T: int = 0):
             "l2_policy": "2 cache copies (440 MB) alternate", "steps": steps}
 
 
+def windows_leg(steps: int, T: int = 0, sink: int = 128, recent: int = 1024):
+    """Decode with fp16 sink and recent windows over the 2-bit cache (batch 4,
+    32/8 heads, context 65536, 2-bit g128 clip 0.9): the first 128 and the
+    last 1024 tokens of each sequence from a device window store, the rest
+    quantised; CUDA graph over two cache copies, beside the plain quantised
+    decode of the same cache."""
+    import torch
+
+    import quantized_kv_cache_16_b200 as K
+    import workloads as W
+    wl = W.int2() if not T else W.int2(T=T)
+    copies = 2
+    dev = torch.device("cuda", torch.cuda.current_device())
+    tabs = W.page_table(wl, copies=copies)
+    cfg = K.make_config(wl.Hq, wl.Hkv, wl.d, wl.k_fmt, wl.v_fmt, wl.k_group, wl.v_group, wl.clip, wl.rotation_seed,
+                        num_pages=tabs[0].num_pages)
+    cache = K.Cache(cfg)
+    Wn = sink + recent
+    wk = torch.empty((wl.B, Wn, wl.Hkv, wl.d), dtype=torch.float16, device=dev)
+    wv = torch.empty_like(wk)
+    for b in range(wl.B):
+        kd, vd = W.prefix_kv_device(wl, b, dev)
+        Tb = wl.ctx[b]
+        for c in range(copies):
+            cache.append(kd, vd, torch.from_numpy(tabs[c].slots(b, 0, Tb)).to(dev))
+        wk[b, :sink], wv[b, :sink] = kd[:sink], vd[:sink]
+        pos = torch.arange(Tb - recent, Tb, device=dev)
+        wk[b, sink + pos % recent], wv[b, sink + pos % recent] = kd[pos], vd[pos]
+        del kd, vd
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed)
+    nq = 8
+    qs = torch.randn((nq, wl.B, wl.Hq, wl.d), generator=gen, device=dev).half()
+    bts = [torch.from_numpy(t.block_table).to(dev) for t in tabs]
+    max_pages = bts[0].shape[1]
+    ctx = torch.tensor(wl.ctx, dtype=torch.int32, device=dev)
+    ws = cache.workspace_for(wl.B, max_pages)
+    out = torch.empty((wl.B, wl.Hq, wl.d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream()
+
+    def quant(s):
+        K.kvq_decode_attn(cache.handle, qs[s % nq], bts[s % copies], max_pages, ctx, wl.B, 0.0, None, ws, ws.numel(),
+                          out, None, stream)
+
+    def win(s):
+        K.kvq_decode_windows(cache.handle, qs[s % nq], bts[s % copies], max_pages, ctx, wl.B, 0.0, wk, wv, sink,
+                             recent, ws, ws.numel(), out, stream)
+
+    q_us = _graph_time(quant, steps, stream)
+    w_us = _graph_time(win, steps, stream)
+    assert cache.sync_status() == 0
+    kv_bytes = sum(wl.ctx) * wl.Hkv * 2 * (wl.d // 4 + 4)
+    win_bytes = wl.B * Wn * wl.Hkv * wl.d * 2 * 2
+    return {"workload": f"2-bit g128 cache, B={wl.B}, 32/8 heads, d=128, context {wl.ctx[0]}, fp16 sink {sink} + "
+                        f"recent {recent} tokens per sequence from a device store",
+            "us": round(w_us, 2), "quantised_only_us": round(q_us, 2), "overhead_x": round(w_us / q_us, 3),
+            "cache_bytes": kv_bytes, "window_bytes": win_bytes, "steps": steps}
+
+
 LADDER_POLICY = dict(tau_cov=0.995, max_frac=0.05, key_tol=0.02, v_tol=1e-3, rank_tol=0.05, cert_tol=0.02,
                      layer_frac=0.5)
 
@@ -775,7 +835,7 @@ def main():
     if args.leg:
         import torch
         torch.cuda.set_device(0)
-        leg = certified_leg if args.leg == "certified" else ladder_leg
+        leg = {"certified": certified_leg, "ladder": ladder_leg, "windows": windows_leg}[args.leg]
         print(json.dumps(leg(args.steps, args.ctx)), flush=True)
         return
     if args.impl == "reference":

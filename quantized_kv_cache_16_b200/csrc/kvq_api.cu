@@ -590,7 +590,11 @@ kvq_status kvq_decode_windows(kvq_cache *c, const void *q, const int32_t *block_
     cp.rotate = c->cfg.rotate;
     memcpy(cp.signs, c->signs, sizeof(cp.signs));
     cp.head_ml = p.head_ml;
-    cp.n_chunks = kCertChunks;
+    {  // one wave: about one CTA per SM over all (sequence, kv head) pairs
+        const long long groups = (long long)batch * c->L.hkv;
+        long long n = (c->num_sms + groups - 1) / groups;
+        cp.n_chunks = (int)(n < 1 ? 1 : (n > kCertChunks ? kCertChunks : n));
+    }
     cp.k2 = static_cast<const __half *>(k2);
     cp.v2 = static_cast<const __half *>(v2);
     cp.sink = sink;
