@@ -137,6 +137,42 @@ template <> struct RawRow<2> {
     }
 };
 
+// Transpose-reduce: each lane holds 32 partial sums v[0..31] (index i); after
+// five halving exchanges lane j holds the warp-wide total of index j.  At the
+// step with offset o a lane keeps the half whose index bit log2(o) equals its
+// own lane bit and adds the partner's copy of that half: 31 shuffles for 32
+// totals (instead of 32 five-step butterflies).
+__device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane)
+{
+#pragma unroll
+    for (int k = 0; k < 16; k++) {
+        const bool up = lane & 16;
+        const float send = up ? v[k] : v[k + 16], keep = up ? v[k + 16] : v[k];
+        v[k] = keep + __shfl_xor_sync(kFull, send, 16);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        const bool up = lane & 8;
+        const float send = up ? v[k] : v[k + 8], keep = up ? v[k + 8] : v[k];
+        v[k] = keep + __shfl_xor_sync(kFull, send, 8);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const bool up = lane & 4;
+        const float send = up ? v[k] : v[k + 4], keep = up ? v[k + 4] : v[k];
+        v[k] = keep + __shfl_xor_sync(kFull, send, 4);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; k++) {
+        const bool up = lane & 2;
+        const float send = up ? v[k] : v[k + 2], keep = up ? v[k + 2] : v[k];
+        v[k] = keep + __shfl_xor_sync(kFull, send, 2);
+    }
+    const bool up = lane & 1;
+    const float send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
+    return keep + __shfl_xor_sync(kFull, send, 1);
+}
+
 // Sort keys[0..np2) (np2 a power of two) in descending order with NT
 // threads; keys past the live entries must be 0.  Up to 2*NT keys stay in
 // registers (two per thread, warp shuffles for the stages whose partner is

@@ -327,63 +327,141 @@ __global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid
                     if (vx) vraw[u].load(p.v2 + row);
                 }
             }
+            unsigned vmask = 0;  // tokens of the batch that are there
 #pragma unroll
-            for (int u = 0; u < kTokBatch; u++) {
-                if (pgs[u] < 0) continue;  // warp-uniform
-                const int tok = toks[u];
-                const unsigned char *chunk =
-                    p.pool + kHeaderBytes + (long long)pgs[u] * L.page_bytes + (long long)kvh * L.chunk_bytes;
-                float kq[E] = {}, vq[E] = {}, ke[E] = {}, ve[E] = {};
-                if constexpr (!WIN) {  // windows: the quantised pass left these tokens out
-                    dequant_lane<E>(chunk, L.k_codes, L.k_meta, L.k_row_meta, L.k_fmt, tok, lane, kq);
-                    dequant_lane<E>(chunk, L.v_codes, L.v_meta, L.v_row_meta, L.v_fmt, tok, lane, vq);
-                }
-                if (kx) kraw[u].widen(ke);
-                if (vx) vraw[u].widen(ve);
+            for (int u = 0; u < kTokBatch; u++) vmask |= (pgs[u] >= 0 ? 1u : 0u) << u;
+            static_assert(kTokBatch == 8, "a batch of 8 tokens x 4 heads fills one transpose-reduce");
+            // heads in groups of four (a group past g holds zeros); lane j of
+            // a reduction holds token j >> 2, head 4 hg + (j & 3)
+            constexpr int NHG = G > 4 ? G / 4 : 1;
+            const int uj = lane >> 2, hlj = lane & 3;
 #pragma unroll
-                for (int h = 0; h < G; h++) {
-                    if (h >= g) break;
-                    float qo[E];
-                    if (E == 4) {
-                        const float4 v4 = *reinterpret_cast<const float4 *>(so + h * D + lane * E);
-                        qo[0] = v4.x;
-                        qo[E > 1 ? 1 : 0] = v4.y;
-                        qo[E > 2 ? 2 : 0] = v4.z;
-                        qo[E > 3 ? 3 : 0] = v4.w;
-                    } else {
+            for (int hg = 0; hg < NHG; hg++) {
+                // 1. partial dot products, index u * 4 + head: [0] the mixed
+                // side (exact keys where promoted), [1] the quantised side
+                float d0[32], d1[32];
 #pragma unroll
-                        for (int e = 0; e < E; e++) qo[e] = so[h * D + lane * E + e];
-                    }
-                    float sqv = 0.f, se = 0.f;
+                for (int i = 0; i < 32; i++) d0[i] = d1[i] = 0.f;
 #pragma unroll
-                    for (int e = 0; e < E; e++) {
-                        if constexpr (!WIN) sqv = fmaf(qr[h][e], kq[e], sqv);
-                        se = fmaf(qo[e], ke[e], se);
+                for (int u = 0; u < kTokBatch; u++) {
+                    if (!((vmask >> u) & 1u)) continue;  // warp-uniform
+                    float ke[E] = {}, kq[E] = {};
+                    if (kx) kraw[u].widen(ke);
+                    if constexpr (!WIN) {
+                        const unsigned char *chunk =
+                            p.pool + kHeaderBytes + (long long)pgs[u] * L.page_bytes + (long long)kvh * L.chunk_bytes;
+                        dequant_lane<E>(chunk, L.k_codes, L.k_meta, L.k_row_meta, L.k_fmt, toks[u], lane, kq);
                     }
 #pragma unroll
-                    for (int mm = 16; mm >= 1; mm >>= 1) {
-                        if constexpr (!WIN) sqv += __shfl_xor_sync(kFull, sqv, mm);
-                        if (kx) se += __shfl_xor_sync(kFull, se, mm);
-                    }
-                    if (!kx) se = sqv;
-                    if constexpr (!WIN) online_update<E>(m[h][1], l[h][1], aq[h], sqv, vq);
-                    {  // the mixed side: one (m, l), two sums
-                        const float mn = fmaxf(m[h][0], se);
-                        const float al = (m[h][0] == -INFINITY) ? 0.f : ex2(m[h][0] - mn);
-                        const float pe = ex2(se - mn);
-                        l[h][0] = fmaf(l[h][0], al, pe);
-                        const float pv = vx ? pe : 0.f, pq = vx ? 0.f : pe;
+                    for (int hl = 0; hl < 4; hl++) {
+                        const int h = hg * 4 + hl;
+                        if (h >= g) break;
+                        float qo[E];
+                        if constexpr (E == 4) {
+                            const float4 v4 = *reinterpret_cast<const float4 *>(so + h * D + lane * E);
+                            qo[0] = v4.x;
+                            qo[E > 1 ? 1 : 0] = v4.y;
+                            qo[E > 2 ? 2 : 0] = v4.z;
+                            qo[E > 3 ? 3 : 0] = v4.w;
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < E; e++) qo[e] = so[h * D + lane * E + e];
+                        }
+                        float a0 = 0.f, a1 = 0.f;
 #pragma unroll
                         for (int e = 0; e < E; e++) {
-                            ae[h][e] = fmaf(ae[h][e], al, pv * ve[e]);
-                            ar[h][e] = fmaf(ar[h][e], al, pq * vq[e]);
+                            a0 = fmaf(qo[e], ke[e], a0);
+                            if constexpr (!WIN) a1 = fmaf(qr[h][e], kq[e], a1);
                         }
-                        m[h][0] = mn;
+                        d0[u * 4 + hl] = a0;
+                        d1[u * 4 + hl] = a1;
                     }
-                    if (p.ladder && kx) {
-                        const float mn = fmaxf(bm[h], se);
-                        bl[h] = fmaf(bl[h], ex2(bm[h] - mn), ex2(se - mn));
-                        bm[h] = mn;
+                }
+                // 2. the totals, one (token, head) per lane
+                const bool live = ((vmask >> uj) & 1u) && hg * 4 + hlj < g;
+                float s1 = -INFINITY;
+                if constexpr (!WIN) {
+                    s1 = transpose_reduce32(d1, lane);
+                    if (!live) s1 = -INFINITY;
+                }
+                float s0 = s1;
+                if (kx) {
+                    s0 = transpose_reduce32(d0, lane);
+                    if (!live) s0 = -INFINITY;
+                }
+                // 3. per side and head: the batch max, the weights relative to
+                // the new running max, the batch sum; then rescale (m, l, sums)
+                float pw[2] = {0.f, 0.f};
+#pragma unroll
+                for (int w = 0; w < 2; w++) {
+                    if (WIN && w == 1) break;
+                    const float sw = w ? s1 : s0;
+                    float bmax = sw;
+#pragma unroll
+                    for (int o = 4; o < 32; o <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
+                    float mo = m[hg * 4][w];
+#pragma unroll
+                    for (int k = 1; k < 4; k++)
+                        if (hg * 4 + k < G && hlj == k) mo = m[hg * 4 + k][w];
+                    const float mnew = fmaxf(mo, bmax);
+                    const float pj = sw == -INFINITY ? 0.f : ex2(sw - mnew);
+                    float psum = pj;
+#pragma unroll
+                    for (int o = 4; o < 32; o <<= 1) psum += __shfl_xor_sync(kFull, psum, o);
+                    pw[w] = pj;
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {  // lane k holds head 4 hg + k's figures
+                        const int h = hg * 4 + k;
+                        if (h >= g) break;
+                        const float mn = __shfl_sync(kFull, mnew, k), ps = __shfl_sync(kFull, psum, k);
+                        const float al = m[h][w] == -INFINITY ? 0.f : ex2(m[h][w] - mn);
+                        l[h][w] = fmaf(l[h][w], al, ps);
+#pragma unroll
+                        for (int e = 0; e < E; e++) {
+                            if (w == 0) {
+                                ae[h][e] *= al;
+                                ar[h][e] *= al;
+                            } else {
+                                aq[h][e] *= al;
+                            }
+                        }
+                        if (p.ladder && kx && w == 0) {  // the block's own (max, sum) for the check
+                            const float bmx = __shfl_sync(kFull, bmax, k);
+                            if (bmx != -INFINITY) {
+                                const float nbm = fmaxf(bm[h], bmx);
+                                bl[h] = fmaf(bl[h], ex2(bm[h] - nbm), ps * ex2(mn - nbm));
+                                bm[h] = nbm;
+                            }
+                        }
+                        m[h][w] = mn;
+                    }
+                }
+                // 4. values: every lane takes each (token, head) weight in turn
+#pragma unroll
+                for (int u = 0; u < kTokBatch; u++) {
+                    if (!((vmask >> u) & 1u)) continue;  // warp-uniform
+                    float ve[E] = {}, vq[E] = {};
+                    if (vx) vraw[u].widen(ve);
+                    if (!WIN || !vx) {
+                        const unsigned char *chunk =
+                            p.pool + kHeaderBytes + (long long)pgs[u] * L.page_bytes + (long long)kvh * L.chunk_bytes;
+                        dequant_lane<E>(chunk, L.v_codes, L.v_meta, L.v_row_meta, L.v_fmt, toks[u], lane, vq);
+                    }
+#pragma unroll
+                    for (int hl = 0; hl < 4; hl++) {
+                        const int h = hg * 4 + hl;
+                        if (h >= g) break;
+                        const float w0 = __shfl_sync(kFull, pw[0], u * 4 + hl);
+#pragma unroll
+                        for (int e = 0; e < E; e++) {
+                            if (vx) ae[h][e] = fmaf(w0, ve[e], ae[h][e]);
+                            else ar[h][e] = fmaf(w0, vq[e], ar[h][e]);
+                        }
+                        if constexpr (!WIN) {
+                            const float w1 = __shfl_sync(kFull, pw[1], u * 4 + hl);
+#pragma unroll
+                            for (int e = 0; e < E; e++) aq[h][e] = fmaf(w1, vq[e], aq[h][e]);
+                        }
                     }
                 }
             }
