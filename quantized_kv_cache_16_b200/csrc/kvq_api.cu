@@ -590,9 +590,9 @@ kvq_status kvq_decode_windows(kvq_cache *c, const void *q, const int32_t *block_
     cp.rotate = c->cfg.rotate;
     memcpy(cp.signs, c->signs, sizeof(cp.signs));
     cp.head_ml = p.head_ml;
-    {  // one wave: at most one CTA per SM over all (sequence, kv head) pairs
+    {  // one wave over all (sequence, kv head) pairs
         const long long groups = (long long)batch * c->L.hkv;
-        long long n = c->num_sms / groups;
+        long long n = 2LL * c->num_sms / groups;  // the window instantiation keeps two CTAs per SM
         cp.n_chunks = (int)(n < 1 ? 1 : (n > kCertChunks ? kCertChunks : n));
     }
     cp.k2 = static_cast<const __half *>(k2);

@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(kSelThreads) cert_select_kernel(const __grid_c
 // adds the exact partial to the quantised one (a plain log-sum-exp merge;
 // the quantised side's mass is 0).
 template <int D, int G, bool WIN>
-__global__ void __launch_bounds__(kPromThreads) cert_promote_kernel(const __grid_constant__ CertParams p)
+__global__ void __launch_bounds__(kPromThreads, WIN ? 2 : 1) cert_promote_kernel(const __grid_constant__ CertParams p)
 {
     pdl_enter();
     constexpr int E = D / 32;
