@@ -21,7 +21,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "kvq_oracle.c")
 _LIB = os.path.join(_HERE, "_liboracle.so")
 
-INT4_ASYM, INT8_SYM, INT2_ASYM = 0, 1, 2
+INT4_ASYM, INT8_SYM, INT2_ASYM, HQMQ = 0, 1, 2, 3
+HQMQ_NS, HQMQ_NO = 1024, 2
 PAGE_TOKENS = 16
 
 
@@ -123,6 +124,13 @@ def lib():
             "kvqo_decode_fp16": (i32, [cfgp, P, P, P, P, i32, P, i32, f64, P, P]),
             "kvqo_promote_count": (i32, [f64, i32]),
             "kvqo_decode_certified": (i32, [cfgp, P, P, P, P, P, i32, P, i32, f64, f64, P, P, P, i32, P, i32, P, P]),
+            "kvqo_init_pool": (None, [cfgp, P]),
+            "kvqo_hqmq_table_offset": (sz, [cfgp]),
+            "kvqo_hqmq_unit": (None, [i32, P]),
+            "kvqo_hqmq_codebook": (None, [u64, i32, i32, P]),
+            "kvqo_hqmq_quantize_rows": (None, [P, i32, i32, P, P, P, P, P]),
+            "kvqo_hqmq_encode_dirs": (None, [P, i32, P, P]),
+            "kvqo_hqmq_read_row": (None, [cfgp, P, i32, i32, i32, P, P, P, P]),
             "kvqo_decode_windows": (i32, [cfgp, P, P, P, i32, i32, P, P, i32, P, i32, f64, P]),
             "kvqo_decode_ladder": (i32, [cfgp, P, P, P, P, P, i32, P, i32, f64, C.POINTER(Ladder), P, P,
                                          C.POINTER(LadderOut)]),
@@ -245,7 +253,11 @@ def config_ok(cfg: Config) -> bool:
 
 
 def new_pool(cfg: Config) -> np.ndarray:
-    return np.zeros(pool_bytes(cfg), np.uint8)
+    """A zeroed pool of the config's size (with the HQMQ codebooks written,
+    as kvq_create_cache does)."""
+    pool = np.zeros(pool_bytes(cfg), np.uint8)
+    lib().kvqo_init_pool(C.byref(cfg), _p(pool))
+    return pool
 
 
 def append(cfg: Config, pool: np.ndarray, k, v, slot_mapping, want_rotated: bool = False):
@@ -414,3 +426,49 @@ def decode_windows(cfg: Config, pool: np.ndarray, win_k, win_v, sink: int, recen
     if rc != 0:
         raise ValueError(f"oracle window decode rejected its arguments (rc={rc})")
     return out
+
+
+# --- HQMQ ([HQMQ] Hurwitz quaternion multiplicative quantisation) ------------
+
+def hqmq_unit(p: int) -> np.ndarray:
+    q = np.zeros(4, np.float32)
+    lib().kvqo_hqmq_unit(p, _p(q))
+    return q
+
+
+def hqmq_codebook(seed: int, kvh: int, tensor: int) -> np.ndarray:
+    S = np.zeros((HQMQ_NS, 4), np.float32)
+    lib().kvqo_hqmq_codebook(seed, kvh, tensor, _p(S))
+    return S
+
+
+def hqmq_quantize_rows(y, S):
+    """Encode rotated rows y [n, d]: fields [n, d/4] (15-bit index, 5-bit radius
+    code), step (fp16 bits) [n], outlier mask [n], outlier slots [n, NO, 4]."""
+    y = _c(y, np.float32)
+    S = _c(S, np.float32)
+    n, d = y.shape
+    field = np.zeros((n, d // 4), np.uint32)
+    step = np.zeros(n, np.uint16)
+    mask = np.zeros(n, np.uint32)
+    outl = np.zeros((n, HQMQ_NO, 4), np.uint16)
+    lib().kvqo_hqmq_quantize_rows(_p(y), n, d, _p(S), _p(field), _p(step), _p(mask), _p(outl))
+    return field, step, mask, outl
+
+
+def hqmq_encode_dirs(u, S) -> np.ndarray:
+    u = _c(u, np.float32)
+    S = _c(S, np.float32)
+    idx = np.zeros(u.shape[0], np.int32)
+    lib().kvqo_hqmq_encode_dirs(_p(u), u.shape[0], _p(S), _p(idx))
+    return idx
+
+
+def hqmq_read_row(cfg: Config, pool: np.ndarray, slot: int, kvh: int, tensor: int):
+    d = cfg.head_dim
+    field = np.zeros(d // 4, np.uint32)
+    step = np.zeros(1, np.uint16)
+    mask = np.zeros(1, np.uint32)
+    outl = np.zeros((HQMQ_NO, 4), np.uint16)
+    lib().kvqo_hqmq_read_row(C.byref(cfg), _p(pool), slot, kvh, tensor, _p(field), _p(step), _p(mask), _p(outl))
+    return field, int(step[0]), int(mask[0]), outl

@@ -42,6 +42,9 @@
 #define KVQO_INT4_ASYM 0
 #define KVQO_INT8_SYM 1
 #define KVQO_INT2_ASYM 2
+#define KVQO_HQMQ 3        /* Hurwitz-quaternion multiplicative VQ of 4-element blocks */
+#define KVQO_HQMQ_NS 1024  /* secondary codebook size per (kv head, K|V) */
+#define KVQO_HQMQ_NO 2     /* fp16 outlier blocks a row can keep (Med3x) */
 
 #define KVQO_PAGE_TOKENS 16
 #define KVQO_HEADER_BYTES 256
@@ -385,6 +388,185 @@ static void quantize_row(int fmt, int group, float clip, int search, const float
 }
 
 /* ------------------------------------------------------------------------- */
+/* HQMQ: Hurwitz quaternion multiplicative quantisation ([HQMQ] 1-3)          */
+/* ------------------------------------------------------------------------- */
+
+/* The 24 unit Hurwitz quaternions (the binary tetrahedral group 2T) in code
+ * order: p = 0..7 are +1, -1, +i, -i, +j, -j, +k, -k; p = 8..23 are
+ * (+-1 +-i +-j +-k)/2 with component c negative iff bit c of p - 8 is set. */
+void kvqo_hqmq_unit(int p, float q[4])
+{
+    for (int i = 0; i < 4; i++) q[i] = 0.0f;
+    if (p < 8) {
+        q[p / 2] = (p & 1) ? -1.0f : 1.0f;
+    } else {
+        for (int i = 0; i < 4; i++) q[i] = (((p - 8) >> i) & 1) ? -0.5f : 0.5f;
+    }
+}
+
+/* Hamilton product r = a b, each component's products rounded and summed
+ * left to right in fp32 (the order the kernels use). */
+static void qmul_f32(const float a[4], const float b[4], float r[4])
+{
+    r[0] = a[0] * b[0] - a[1] * b[1] - a[2] * b[2] - a[3] * b[3];
+    r[1] = a[0] * b[1] + a[1] * b[0] + a[2] * b[3] - a[3] * b[2];
+    r[2] = a[0] * b[2] - a[1] * b[3] + a[2] * b[0] + a[3] * b[1];
+    r[3] = a[0] * b[3] + a[1] * b[2] - a[2] * b[1] + a[3] * b[0];
+}
+
+/* Secondary codebook S of (kv head, tensor): NS unit quaternions drawn
+ * without calibration ([HQMQ] 1: random unit quaternions per layer, head
+ * and role).  SplitMix64 stream of state seed ^ ((2 kvh + tensor + 1) *
+ * 0xD1B54A32D192ED03); a candidate takes four outputs, component =
+ * (out >> 40) / 2^23 - 1 (exact in fp32, in [-1, 1)), and is kept when
+ * 1e-4 < |a|^2 <= 1 (squares summed in order), divided by sqrt(|a|^2). */
+void kvqo_hqmq_codebook(uint64_t seed, int kvh, int tensor, float *S)
+{
+    uint64_t st = seed ^ ((uint64_t)(2 * kvh + tensor + 1) * 0xD1B54A32D192ED03ULL);
+    int n = 0;
+    while (n < KVQO_HQMQ_NS) {
+        float a[4];
+        for (int i = 0; i < 4; i++) a[i] = (float)(splitmix64_next(&st) >> 40) / 8388608.0f - 1.0f;
+        float n2 = a[0] * a[0] + a[1] * a[1] + a[2] * a[2] + a[3] * a[3];
+        if (!(n2 > 1e-4f && n2 <= 1.0f)) continue;
+        float r = sqrtf(n2);
+        for (int i = 0; i < 4; i++) S[4 * n + i] = a[i] / r;
+        n++;
+    }
+}
+
+/* Codeword index of a unit direction u ([HQMQ] 1: the codeword of largest
+ * inner product in C = {q_p q_s}).  <u, q_p q_s> = <u conj(q_s), q_p>, so for
+ * each s, w = u conj(q_s) and the best unit of 2T is closed-form: an axis
+ * unit scores max_i |w_i| (first i on ties, sign of w_i), a half unit
+ * (((|w0| + |w1|) + |w2|) + |w3|) / 2 (signs of w); the half unit wins only
+ * when strictly higher, and over s the first highest score wins.
+ * Index = 24 s + p. */
+static int hqmq_encode_dir(const float u[4], const float *S)
+{
+    int best = 0;
+    float best_sc = -INFINITY;
+    for (int si = 0; si < KVQO_HQMQ_NS; si++) {
+        const float cb[4] = {S[4 * si], -S[4 * si + 1], -S[4 * si + 2], -S[4 * si + 3]};
+        float w[4], aw[4];
+        qmul_f32(u, cb, w);
+        for (int i = 0; i < 4; i++) aw[i] = fabsf(w[i]);
+        int ia = 0;
+        float ma = aw[0];
+        for (int i = 1; i < 4; i++)
+            if (aw[i] > ma) {
+                ma = aw[i];
+                ia = i;
+            }
+        float mh = (aw[0] + aw[1] + aw[2] + aw[3]) * 0.5f;
+        int pp;
+        float sc;
+        if (mh > ma) {
+            sc = mh;
+            pp = 8 + (w[0] < 0.0f) + 2 * (w[1] < 0.0f) + 4 * (w[2] < 0.0f) + 8 * (w[3] < 0.0f);
+        } else {
+            sc = ma;
+            pp = 2 * ia + (w[ia] < 0.0f);
+        }
+        if (sc > best_sc) {
+            best_sc = sc;
+            best = 24 * si + pp;
+        }
+    }
+    return best;
+}
+
+/* One HQMQ row (d/4 blocks) with Med3x outlier extraction ([HQMQ] 1 and 3):
+ *   r_b = sqrt(((x0^2 + x1^2) + x2^2) + x3^2), fp32;
+ *   r_med = the lower median of the row's radii, tau = 3 r_med (the page's
+ *     C = 3; the "batch" is read as the row, the unit quantised at once);
+ *   outliers: up to KVQO_HQMQ_NO blocks with r_b > tau, largest first (lower
+ *     block on ties), kept as fp16 with their mask bit set;
+ *   radius step = fp16 rounded up of tau / 31; radius code = min(31,
+ *     rint(r_b / step)) (0 when the step is 0);
+ *   direction code = hqmq_encode_dir(x_b / r_b) (0 when r_b = 0).
+ * field[b] = index | code << 15.  The page quantises the radius without
+ * saying how; a uniform 5-bit code on [0, tau] with the outliers cut off is
+ * the plainest reading that gives its ~5 bits per element (15 + 5 bits per
+ * 4 elements). */
+static void hqmq_quantize_row(const float *y, int d, const float *S, uint32_t *field, uint16_t *step_h,
+                              uint32_t *mask, uint16_t outl[KVQO_HQMQ_NO][4])
+{
+    int nb = d / 4;
+    float r[64], srt[64];
+    for (int b = 0; b < nb; b++) {
+        const float *x = y + 4 * b;
+        r[b] = sqrtf(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
+        srt[b] = r[b];
+    }
+    for (int i = 1; i < nb; i++)
+        for (int j = i; j > 0 && srt[j - 1] > srt[j]; j--) {
+            float t = srt[j];
+            srt[j] = srt[j - 1];
+            srt[j - 1] = t;
+        }
+    float tau = 3.0f * srt[(nb - 1) / 2];
+    uint32_t m = 0;
+    for (int k = 0; k < KVQO_HQMQ_NO; k++) {
+        int pick = -1;
+        for (int b = 0; b < nb; b++)
+            if (!((m >> b) & 1u) && r[b] > tau && (pick < 0 || r[b] > r[pick])) pick = b;
+        if (pick >= 0) m |= 1u << pick;
+    }
+    uint16_t sh = kvqo_f2h_ru(tau / 31.0f);
+    float sf = kvqo_h2f(sh);
+    int slot = 0;
+    for (int k = 0; k < KVQO_HQMQ_NO; k++)
+        for (int i = 0; i < 4; i++) outl[k][i] = 0;
+    for (int b = 0; b < nb; b++) {
+        const float *x = y + 4 * b;
+        if ((m >> b) & 1u) {
+            for (int i = 0; i < 4; i++) outl[slot][i] = kvqo_f2h_rn(x[i]);
+            slot++;
+            field[b] = 0;
+            continue;
+        }
+        unsigned rc = 0;
+        if (sf > 0.0f) {
+            float v = rintf(r[b] / sf);
+            rc = v > 31.0f ? 31u : (unsigned)v;
+        }
+        int idx = 0;
+        if (r[b] > 0.0f) {
+            float u[4];
+            for (int i = 0; i < 4; i++) u[i] = x[i] / r[b];
+            idx = hqmq_encode_dir(u, S);
+        }
+        field[b] = (uint32_t)idx | (rc << 15);
+    }
+    *step_h = sh;
+    *mask = m;
+}
+
+/* Reconstruction of block b of an HQMQ row in fp64: the outlier's fp16
+ * values, or (radius code x step) times the codeword q_p q_s. */
+static void hqmq_dequant_block(uint32_t field, int is_outlier, const uint16_t *outl4, const float *S, double step,
+                               double out[4])
+{
+    if (is_outlier) {
+        for (int i = 0; i < 4; i++) out[i] = kvqo_h2f(outl4[i]);
+        return;
+    }
+    int idx = (int)(field & 0x7FFFu), rc = (int)(field >> 15);
+    int si = idx / 24, pp = idx % 24;
+    float qp[4];
+    kvqo_hqmq_unit(pp, qp);
+    const float *b = S + 4 * si;
+    double a[4] = {qp[0], qp[1], qp[2], qp[3]}, c[4];
+    c[0] = a[0] * b[0] - a[1] * b[1] - a[2] * b[2] - a[3] * b[3];
+    c[1] = a[0] * b[1] + a[1] * b[0] + a[2] * b[3] - a[3] * b[2];
+    c[2] = a[0] * b[2] - a[1] * b[3] + a[2] * b[0] + a[3] * b[1];
+    c[3] = a[0] * b[3] + a[1] * b[2] - a[2] * b[1] + a[3] * b[0];
+    double rh = (double)rc * step;
+    for (int i = 0; i < 4; i++) out[i] = rh * c[i];
+}
+
+/* ------------------------------------------------------------------------- */
 /* Paged pool layout (restated here from the written layout definition)      */
 /* ------------------------------------------------------------------------- */
 /* pool  = [header: 256 B][pages: num_pages x page_bytes][descriptors]
@@ -400,8 +582,16 @@ static void quantize_row(int fmt, int group, float clip, int search, const float
  * descriptors (only when bound blocks are on): per (page, kv head) four fp32
  *         {max key error, max value error, max |value|, 0} over the page. */
 
-static int row_code_bytes(int fmt, int d) { return d * fmt_bits(fmt) / 8; }
-static int row_meta_bytes(int fmt, int d, int group) { return fmt == KVQO_INT8_SYM ? 2 : 4 * (d / group); }
+/* HQMQ rows: d/4 blocks x 20 bits (15-bit codeword index, then a 5-bit
+ * radius code) as one little-endian bit stream; meta = fp16 radius step,
+ * 2 zero bytes, the 32-bit outlier mask, KVQO_HQMQ_NO outlier slots of four
+ * fp16 values (in block order). */
+static int row_code_bytes(int fmt, int d) { return fmt == KVQO_HQMQ ? d * 5 / 8 : d * fmt_bits(fmt) / 8; }
+static int row_meta_bytes(int fmt, int d, int group)
+{
+    if (fmt == KVQO_HQMQ) return 8 + 8 * KVQO_HQMQ_NO;
+    return fmt == KVQO_INT8_SYM ? 2 : 4 * (d / group);
+}
 static size_t region_code_bytes(int fmt, int d) { return (size_t)KVQO_PAGE_TOKENS * row_code_bytes(fmt, d); }
 static size_t region_meta_bytes(int fmt, int d, int g) { return (size_t)KVQO_PAGE_TOKENS * row_meta_bytes(fmt, d, g); }
 
@@ -419,10 +609,19 @@ size_t kvqo_desc_offset(const kvqo_config *c)
     return KVQO_HEADER_BYTES + (size_t)c->num_pages * kvqo_page_bytes(c);
 }
 
-size_t kvqo_pool_bytes(const kvqo_config *c)
+/* HQMQ secondary codebooks follow the descriptors: [Hkv][2][NS] unit
+ * quaternions, fp32 x 4. */
+size_t kvqo_hqmq_table_offset(const kvqo_config *c)
 {
     size_t n = kvqo_desc_offset(c);
     if (c->bound_block_tokens > 0) n += (size_t)c->num_pages * c->num_kv_heads * 16;
+    return n;
+}
+
+size_t kvqo_pool_bytes(const kvqo_config *c)
+{
+    size_t n = kvqo_hqmq_table_offset(c);
+    if (c->k_fmt == KVQO_HQMQ) n += (size_t)c->num_kv_heads * 2 * KVQO_HQMQ_NS * 16;
     return n;
 }
 
@@ -464,6 +663,60 @@ static void pack_row(const kvqo_config *c, uint8_t *pool, int page, int tok, int
     }
 }
 
+/* The HQMQ secondary codebook of (kv head, tensor) in the pool. */
+static const float *hqmq_table(const kvqo_config *c, const uint8_t *pool, int kvh, int tensor)
+{
+    return (const float *)(pool + kvqo_hqmq_table_offset(c)) + ((size_t)kvh * 2 + tensor) * KVQO_HQMQ_NS * 4;
+}
+
+/* Write the HQMQ secondary codebooks into a new pool (every (kv head,
+ * tensor) pair); nothing for the other formats. */
+void kvqo_init_pool(const kvqo_config *c, uint8_t *pool)
+{
+    if (c->k_fmt != KVQO_HQMQ) return;
+    for (int kvh = 0; kvh < c->num_kv_heads; kvh++)
+        for (int tensor = 0; tensor < 2; tensor++)
+            kvqo_hqmq_codebook(c->rotation_seed, kvh, tensor, (float *)(void *)hqmq_table(c, pool, kvh, tensor));
+}
+
+/* HQMQ rows are stored token-major: the 20-bit fields as one little-endian
+ * bit stream, then the meta row (see row_meta_bytes). */
+static void hqmq_pack_row(const kvqo_config *c, uint8_t *pool, int page, int tok, int kvh, int tensor,
+                          const uint32_t *field, uint16_t step, uint32_t mask, uint16_t outl[KVQO_HQMQ_NO][4])
+{
+    int d = c->head_dim, nb = d / 4, rb = row_code_bytes(KVQO_HQMQ, d);
+    uint8_t stream[KVQO_MAXD];
+    memset(stream, 0, sizeof(stream));
+    for (int b = 0; b < nb; b++)
+        for (int bit = 0; bit < 20; bit++)
+            if ((field[b] >> bit) & 1u) stream[(20 * b + bit) / 8] |= (uint8_t)(1u << ((20 * b + bit) % 8));
+    memcpy(pool + region_base(c, page, kvh, tensor, 0) + (size_t)tok * rb, stream, (size_t)rb);
+    uint8_t *meta = pool + region_base(c, page, kvh, tensor, 1) + (size_t)tok * row_meta_bytes(KVQO_HQMQ, d, 4);
+    memset(meta, 0, (size_t)row_meta_bytes(KVQO_HQMQ, d, 4));
+    memcpy(meta, &step, 2);
+    memcpy(meta + 4, &mask, 4);
+    for (int k = 0; k < KVQO_HQMQ_NO; k++) memcpy(meta + 8 + 8 * k, outl[k], 8);
+}
+
+/* Read an HQMQ row back: fields, step, mask, outlier slots. */
+void kvqo_hqmq_read_row(const kvqo_config *c, const uint8_t *pool, int slot, int kvh, int tensor, uint32_t *field,
+                        uint16_t *step, uint32_t *mask, uint16_t *outl)
+{
+    int d = c->head_dim, nb = d / 4, rb = row_code_bytes(KVQO_HQMQ, d);
+    int page = slot / KVQO_PAGE_TOKENS, tok = slot % KVQO_PAGE_TOKENS;
+    const uint8_t *stream = pool + region_base(c, page, kvh, tensor, 0) + (size_t)tok * rb;
+    for (int b = 0; b < nb; b++) {
+        uint32_t f = 0;
+        for (int bit = 0; bit < 20; bit++)
+            f |= (uint32_t)((stream[(20 * b + bit) / 8] >> ((20 * b + bit) % 8)) & 1u) << bit;
+        field[b] = f;
+    }
+    const uint8_t *meta = pool + region_base(c, page, kvh, tensor, 1) + (size_t)tok * row_meta_bytes(KVQO_HQMQ, d, 4);
+    memcpy(step, meta, 2);
+    memcpy(mask, meta + 4, 4);
+    memcpy(outl, meta + 8, 8 * KVQO_HQMQ_NO);
+}
+
 /* Read back the codes, scales and zeros of one stored row (inverse of
  * pack_row). */
 void kvqo_read_row(const kvqo_config *c, const uint8_t *pool, int slot, int kvh, int tensor, int16_t *code,
@@ -503,6 +756,19 @@ void kvqo_dequant_row(const kvqo_config *c, const uint8_t *pool, int slot, int k
     int d = c->head_dim;
     int fmt = tensor ? c->v_fmt : c->k_fmt;
     int group = tensor ? c->v_group : c->k_group;
+    if (fmt == KVQO_HQMQ) {
+        uint32_t field[64], mask;
+        uint16_t step, outl[KVQO_HQMQ_NO][4];
+        kvqo_hqmq_read_row(c, pool, slot, kvh, tensor, field, &step, &mask, &outl[0][0]);
+        const float *S = hqmq_table(c, pool, kvh, tensor);
+        int k = 0;
+        for (int b = 0; b < d / 4; b++) {
+            int is_out = (mask >> b) & 1u;
+            hqmq_dequant_block(field[b], is_out, is_out ? outl[k] : NULL, S, (double)kvqo_h2f(step), out + 4 * b);
+            k += is_out;
+        }
+        return;
+    }
     int16_t code[KVQO_MAXD];
     uint16_t sh[KVQO_MAXD], zh[KVQO_MAXD];
     kvqo_read_row(c, pool, slot, kvh, tensor, code, sh, zh);
@@ -523,6 +789,7 @@ void kvqo_dequant_row(const kvqo_config *c, const uint8_t *pool, int slot, int k
 static int fmt_ok(int fmt, int group, int d)
 {
     if (fmt == KVQO_INT8_SYM) return 1;
+    if (fmt == KVQO_HQMQ) return group == 4 && d == 128;
     if (fmt != KVQO_INT4_ASYM && fmt != KVQO_INT2_ASYM) return 0;
     if (group <= 0 || d % group) return 0;
     return 1;
@@ -538,6 +805,8 @@ int kvqo_config_ok(const kvqo_config *c)
     if (!(c->clip_ratio > 0.0f && c->clip_ratio <= 1.0f)) return 0;
     if (c->bound_block_tokens < 0 || c->bound_block_tokens % KVQO_PAGE_TOKENS) return 0;
     if (c->scale_search != 0 && c->scale_search != 1) return 0;
+    if ((c->k_fmt == KVQO_HQMQ) != (c->v_fmt == KVQO_HQMQ)) return 0;  /* both or neither */
+    if (c->k_fmt == KVQO_HQMQ && (c->bound_block_tokens != 0 || c->scale_search)) return 0;
     return 1;
 }
 
@@ -573,6 +842,13 @@ int kvqo_append(const kvqo_config *c, uint8_t *pool, const uint16_t *k, const ui
                 for (int i = 0; i < d; i++) x[i] = kvqo_h2f(src[i]);
                 kvqo_rotate_f32(x, s, d, c->rotate, y);
                 if (y_out) memcpy(y_out + (((size_t)n * hkv + kvh) * 2 + tensor) * d, y, sizeof(float) * d);
+                if (fmt == KVQO_HQMQ) {
+                    uint32_t field[64], mask;
+                    uint16_t step, outl[KVQO_HQMQ_NO][4];
+                    hqmq_quantize_row(y, d, hqmq_table(c, pool, kvh, tensor), field, &step, &mask, outl);
+                    hqmq_pack_row(c, pool, page, tok, kvh, tensor, field, step, mask, outl);
+                    continue;
+                }
                 int16_t code[KVQO_MAXD];
                 uint16_t sh[KVQO_MAXD], zh[KVQO_MAXD];
                 float emax, amax;
@@ -1383,6 +1659,22 @@ int kvqo_decode_windows(const kvqo_config *c, const uint8_t *pool, const uint16_
 /* ------------------------------------------------------------------------- */
 /* Array helpers for the tests                                               */
 /* ------------------------------------------------------------------------- */
+
+/* HQMQ on its own: encode rotated rows y[n][d] (fields [n][d/4], step [n],
+ * mask [n], outliers [n][NO][4]) with the codebook S [NS][4]; and the
+ * codeword index of single unit directions u[n][4]. */
+void kvqo_hqmq_quantize_rows(const float *y, int n, int d, const float *S, uint32_t *field, uint16_t *step,
+                             uint32_t *mask, uint16_t *outl)
+{
+    for (int r = 0; r < n; r++)
+        hqmq_quantize_row(y + (size_t)r * d, d, S, field + (size_t)r * (d / 4), step + r, mask + r,
+                          (uint16_t(*)[4])(outl + (size_t)r * KVQO_HQMQ_NO * 4));
+}
+
+void kvqo_hqmq_encode_dirs(const float *u, int n, const float *S, int32_t *idx)
+{
+    for (int i = 0; i < n; i++) idx[i] = hqmq_encode_dir(u + 4 * i, S);
+}
 
 void kvqo_f2h_rn_n(const float *x, uint16_t *h, size_t n)
 {

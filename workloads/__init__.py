@@ -24,6 +24,8 @@ Recipes (numpy ``default_rng``; every stream is keyed by (seed, stream id)):
               spans of 64 tokens at seeded positions, the last 128 -- get
               a*u added with a ~ U[10, 14] (then rounded to fp16); queries are
               N(0,1) + 14*u of their kv head.
+  hqmq        llama's geometry, distributions and context with the HQMQ codec
+              for K and V.
   int2        prefill of 65536 tokens x 8 kv heads x d=128 per sequence, K and
               V ~ Laplace(0,1) with 1% of elements x30; 2-bit g128, clip 0.9;
               decode B=4, Hq=32, T=65536 (four independent prefills).
@@ -36,7 +38,7 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-INT4_ASYM, INT8_SYM, INT2_ASYM = 0, 1, 2
+INT4_ASYM, INT8_SYM, INT2_ASYM, HQMQ_FMT = 0, 1, 2, 3
 PAGE_TOKENS = 16
 
 # stream ids
@@ -107,6 +109,13 @@ def ladder(T: int = 131072) -> Workload:
                                 "recent window; adaptive certified ladder over pinned fp16")
 
 
+def hqmq(T: int = 32768) -> Workload:
+    return Workload(f"hqmq-llama3-8b-layer-T{T}", 1, 32, 8, 128, [T], k_fmt=HQMQ_FMT, v_fmt=HQMQ_FMT, k_group=4,
+                    v_group=4, dist="llama", seed=6, steps=1,
+                    description="batch 1, 32/8 heads, head_dim 128, llama's K/V, HQMQ K and V (4-element quaternion "
+                                "blocks, 24 x 1024 codewords, 5-bit radii, Med3x fp16 outliers)")
+
+
 def int2(B: int = 4, T: int = 65536) -> Workload:
     return Workload(f"int2-g128-clip0.9-B{B}-T{T}", B, 32, 8, 128, [T] * B, k_fmt=INT2_ASYM, v_fmt=INT2_ASYM,
                     k_group=128, v_group=128, clip=0.9, dist="laplace", seed=4, steps=1,
@@ -114,7 +123,8 @@ def int2(B: int = 4, T: int = 65536) -> Workload:
                                 "g128 clip 0.9; decode batch 4, 32 q heads, context 65536")
 
 
-ALL = {"tiny": tiny, "llama": llama, "paged": paged, "certified": certified, "ladder": ladder, "int2": int2}
+ALL = {"tiny": tiny, "llama": llama, "paged": paged, "certified": certified, "ladder": ladder, "int2": int2,
+       "hqmq": hqmq}
 
 
 def scaled(wl: Workload, ctx, steps: int = 1) -> Workload:
