@@ -76,7 +76,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-steps", type=int, default=4, help="oracle steps in the CPU baseline sample")
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, append and CPU legs")
-    ap.add_argument("--leg", choices=["certified", "ladder", "windows"],
+    ap.add_argument("--leg", choices=["certified", "ladder", "windows", "hqmq"],
                     help="run only this leg (one GPU, --steps calls) and print its JSON")
     ap.add_argument("--ctx", type=int, default=0, help="context length of --leg (default: its workload's)")
     return ap.parse_args()
@@ -396,6 +396,7 @@ def run_ours(args, dist: Dist):
         result["certified"] = certified_leg(min(K, 200))
         result["ladder"] = ladder_leg(min(K, 100))
         result["windows"] = windows_leg(min(K, 200))
+        result["hqmq"] = hqmq_leg(min(K, 200))
     if dist.rank == 0:
         if not args.no_extras:
             result["cpu_baseline"] = cpu_leg(wk, args.cpu_steps)
@@ -670,6 +671,79 @@ def windows_leg(steps: int, T: int = 0, sink: int = 128, recent: int = 1024):
             "cache_bytes": kv_bytes, "window_bytes": win_bytes, "steps": steps}
 
 
+def hqmq_leg(steps: int, T: int = 0):
+    """The HQMQ codec at Llama-3-8B layer shape (batch 1, 32/8 heads, d=128,
+    context 32768, K and V coded from the raw rows): the bulk append of the
+    whole context and a one-token append (8 kv heads, the CTA per row), timed
+    with events; the decode replayed in a CUDA graph over four cache copies
+    (218 MB, above L2)."""
+    import torch
+
+    import quantized_kv_cache_16_b200 as K
+    import workloads as W
+    wl = W.hqmq(T) if T else W.hqmq()
+    T, copies = wl.ctx[0], 4
+    dev = torch.device("cuda", torch.cuda.current_device())
+    tabs = W.page_table(wl, copies=copies, extra_tokens=8)
+    cfg = K.make_config(wl.Hq, wl.Hkv, wl.d, wl.k_fmt, wl.v_fmt, wl.k_group, wl.v_group, wl.clip, wl.rotation_seed,
+                        rotate=wl.rotate, num_pages=tabs[0].num_pages)
+    cache = K.Cache(cfg)
+    kd, vd = W.prefix_kv_device(wl, 0, dev)
+    rt = Cudart()
+    stream = torch.cuda.Stream()
+    slots = [torch.from_numpy(t.slots(0, 0, T)).to(dev) for t in tabs]
+    e0, e1 = rt.event(), rt.event()
+    bulk_ms = []
+    for c in range(copies):
+        rt.record(e0, stream.cuda_stream)
+        with torch.cuda.stream(stream):
+            cache.append(kd, vd, slots[c], stream=stream)
+        rt.record(e1, stream.cuda_stream)
+        torch.cuda.synchronize()
+        bulk_ms.append(rt.elapsed_ms(e0, e1))
+    del kd, vd
+    # one token (all kv heads) per call, into spare slots of copy 0
+    kn, vn = (torch.from_numpy(x).to(dev) for x in W.step_kv(wl, 0))
+    tok_slots = [torch.from_numpy(tabs[0].slots(0, T + i, T + i + 1)).to(dev) for i in range(8)]
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            cache.append(kn, vn, tok_slots[i], stream=stream)
+    torch.cuda.synchronize()
+    n_tok_calls = 50
+    rt.record(e0, stream.cuda_stream)
+    with torch.cuda.stream(stream):
+        for i in range(n_tok_calls):
+            cache.append(kn, vn, tok_slots[i % 8], stream=stream)
+    rt.record(e1, stream.cuda_stream)
+    torch.cuda.synchronize()
+    tok_us = rt.elapsed_ms(e0, e1) * 1e3 / n_tok_calls
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed)
+    nq = 8
+    qs = torch.randn((nq, wl.B, wl.Hq, wl.d), generator=gen, device=dev).half()
+    bts = [torch.from_numpy(t.block_table).to(dev) for t in tabs]
+    max_pages = bts[0].shape[1]
+    ctx = torch.tensor(wl.ctx, dtype=torch.int32, device=dev)
+    ws = cache.workspace_for(wl.B, max_pages)
+    out = torch.empty((wl.B, wl.Hq, wl.d), dtype=torch.float32, device=dev)
+
+    def dec(s):
+        K.kvq_decode_attn(cache.handle, qs[s % nq], bts[s % copies], max_pages, ctx, wl.B, 0.0, None, ws, ws.numel(),
+                          out, None, stream)
+
+    d_us = _graph_time(dec, steps, stream)
+    assert cache.sync_status() == 0
+    row_bytes = wl.d * 5 // 8 + 24  # 20-bit fields + step, mask and two fp16 outlier blocks
+    kv_bytes = T * wl.Hkv * 2 * row_bytes
+    rows = 2 * T * wl.Hkv
+    bulk = min(bulk_ms)
+    return {"workload": f"HQMQ K/V, B=1, 32/8 heads, d=128, context {T}, raw rows (no rotation)",
+            "decode_us": round(d_us, 2), "decode_gbs": round(kv_bytes / d_us / 1e3, 1), "cache_bytes": kv_bytes,
+            "bits_per_element": row_bytes * 8 / wl.d, "bulk_append_ms": round(bulk, 3),
+            "bulk_append_rows_per_s": round(rows / bulk * 1e3, 1), "token_append_us": round(tok_us, 2),
+            "steps": steps}
+
+
 LADDER_POLICY = dict(tau_cov=0.995, max_frac=0.05, key_tol=0.02, v_tol=1e-3, rank_tol=0.05, cert_tol=0.02,
                      layer_frac=0.5)
 
@@ -835,7 +909,7 @@ def main():
     if args.leg:
         import torch
         torch.cuda.set_device(0)
-        leg = {"certified": certified_leg, "ladder": ladder_leg, "windows": windows_leg}[args.leg]
+        leg = {"certified": certified_leg, "ladder": ladder_leg, "windows": windows_leg, "hqmq": hqmq_leg}[args.leg]
         print(json.dumps(leg(args.steps, args.ctx)), flush=True)
         return
     if args.impl == "reference":

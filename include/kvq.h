@@ -61,15 +61,54 @@ typedef enum {
 typedef enum {
     KVQ_INT4_ASYM = 0, /* 4-bit codes, group 32, fp16 scale + fp16 zero         */
     KVQ_INT8_SYM = 1,  /* 8-bit signed codes, one fp16 scale per token-head     */
-    KVQ_INT2_ASYM = 2  /* 2-bit codes, group = head_dim, fp16 scale + fp16 zero */
+    KVQ_INT2_ASYM = 2, /* 2-bit codes, group = head_dim, fp16 scale + fp16 zero */
+    KVQ_HQMQ = 3       /* Hurwitz-quaternion codes of 4-element blocks (group 4,
+                          head_dim 128, keys and values both), see below       */
 } kvq_fmt;
+
+/* HQMQ ["Hurwitz Quaternion Multiplicative Quantization for KV Cache
+ * Compression", 1-3].  A rotated row is cut into d/4 blocks x (a quaternion);
+ * a block is coded as radius x direction, the direction as the codeword of
+ * largest inner product among the 24 x 1024 products q_p q_s of a unit
+ * Hurwitz quaternion q_p (the binary tetrahedral group, p = 0..23) and a
+ * secondary unit quaternion q_s (s = 0..1023, drawn per kv head and K|V, no
+ * calibration).  Blocks whose radius exceeds tau = 3 x the row's lower median
+ * radius are outliers (Med3x): the two largest keep their four fp16 values;
+ * further ones are coded with a clipped radius.
+ *   units: p = 0..7 are +1, -1, +i, -i, +j, -j, +k, -k; p = 8..23 are
+ *     (+-1 +-i +-j +-k)/2, component c negative iff bit c of p - 8 is set;
+ *   codebook S of (kv head h, tensor t in {0 = K, 1 = V}): SplitMix64 from
+ *     state rotation_seed ^ ((2h + t + 1) * 0xD1B54A32D192ED03); a candidate
+ *     takes four outputs, component = (out >> 40) / 2^23 - 1 (fp32), and is
+ *     kept when 1e-4 < |a|^2 <= 1 (fp32, squares summed in order), then
+ *     divided by fp32 sqrt(|a|^2); the first 1024 kept are S[0..1024);
+ *   row (fp32, each operation rounded, in this order): r_b = sqrt(((x0^2 +
+ *     x1^2) + x2^2) + x3^2); tau = 3 x the 16th smallest r_b; outliers: up to
+ *     two blocks with r_b > tau, largest first (lower block on ties); step =
+ *     fp16 rounded up of tau / 31; radius code = min(31, rint(r_b / step)) (0
+ *     when step = 0); direction u = x / r_b; for each s in order, w = u
+ *     conj(q_s) (Hamilton product, each component's four products summed
+ *     left to right) scores max_i |w_i| (first i, sign of w_i) or, when
+ *     strictly larger, (((|w0| + |w1|) + |w2|) + |w3|) / 2 (signs of w); the
+ *     first s of highest score wins; index = 24 s + p (0 when r_b = 0);
+ *   storage: a token's code row is d/4 fields of 20 bits (index | radius code
+ *     << 15) as one little-endian bit stream (80 bytes at d = 128), 16 rows
+ *     per region, token-major; meta row (24 bytes) = fp16 step, 2 zero bytes,
+ *     the 32-bit outlier mask (bit b = block b), two outlier slots of four
+ *     fp16 values in block order (unused slots zero).  The codebooks sit in
+ *     the pool after the pages (and descriptors): [Hkv][2][1024] x 4 fp32.
+ * A block decodes to (radius code x step) x q_p q_s, an outlier to its fp16
+ * values.  HQMQ caches have no descriptors and no scale search; kvq_append
+ * and kvq_decode_attn (without tier 2) serve them, the other decode calls
+ * return KVQ_ERR_UNSUPPORTED. */
 
 typedef struct {
     int32_t num_q_heads;        /* Hq; Hq / Hkv (the GQA group) must be 1..8          */
     int32_t num_kv_heads;       /* Hkv                                                */
     int32_t head_dim;           /* d: 64 or 128                                       */
-    int32_t k_fmt, v_fmt;       /* kvq_fmt of keys / values (values: int4 or int2)    */
-    int32_t k_group, v_group;   /* int4: 32; int2: head_dim; int8: head_dim           */
+    int32_t k_fmt, v_fmt;       /* kvq_fmt of keys / values (values: int4, int2, or
+                                   HQMQ with HQMQ keys)                              */
+    int32_t k_group, v_group;   /* int4: 32; int2: head_dim; int8: head_dim; HQMQ: 4  */
     float clip_ratio;           /* (0, 1]; scales both ends of int2/int4 groups       */
     uint64_t rotation_seed;     /* SplitMix64 state that draws the sign vector        */
     int32_t rotate;             /* 1 = sign + Hadamard rotation, 0 = identity         */
@@ -104,12 +143,14 @@ typedef struct {
  * token t at (c*16 + t)*16, so one 16-byte load is a whole int4 group.  Meta
  * rows are fp16 scales then fp16 zeros (int8: one scale).  Descriptors (when
  * bound_block_tokens > 0): per (page, kv head) four fp32 {max key error, max
- * value error, max |value|, 0}. */
+ * value error, max |value|, 0}.  HQMQ pools add the codebooks (see
+ * KVQ_HQMQ). */
 size_t kvq_pool_bytes(const kvq_config *cfg);
 
 /* Create a cache over caller-owned device memory `pool_dev` of `pool_bytes`
- * (>= kvq_pool_bytes, 256-byte aligned).  Zero-fills the pool (synchronous)
- * and draws the sign vector from rotation_seed.  *out receives the handle. */
+ * (>= kvq_pool_bytes, 256-byte aligned).  Zero-fills the pool (synchronous),
+ * draws the sign vector from rotation_seed and, for HQMQ, writes the
+ * codebooks.  *out receives the handle. */
 kvq_status kvq_create_cache(const kvq_config *cfg, void *pool_dev, size_t pool_bytes, kvq_cache **out);
 
 /* Release the handle (the pool memory stays the caller's). */
@@ -129,7 +170,9 @@ kvq_status kvq_destroy_cache(kvq_cache *cache);
  * reconstruction error is stored (fp32 sums: per run of 64 consecutive
  * elements, even and odd elements apart in element order, then added, the
  * runs added in order; candidates tried as 0, -1, 1, -2, 2, 3, 4, 5, 6, a
- * later one kept only if strictly better); the zero is unchanged. */
+ * later one kept only if strictly better); the zero is unchanged.
+ * HQMQ caches code each row as KVQ_HQMQ states (a search over 24,576
+ * codewords per block: compute-bound, about 1.5 M fp32 operations a row). */
 kvq_status kvq_append(kvq_cache *cache, const void *k, const void *v, const int32_t *slot_mapping, int32_t n_tok,
                       void *stream);
 

@@ -24,6 +24,35 @@ uint64_t splitmix64_next(uint64_t &state)
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// HQMQ secondary codebook of (kv head h, tensor t) ["Hurwitz Quaternion
+// Multiplicative Quantization for KV Cache Compression", 1: random unit
+// quaternions per head and role, no calibration]: candidates of four
+// SplitMix64 draws mapped to [-1, 1) by (out >> 40) / 2^23 - 1, rejected
+// unless 1e-4 < |a|^2 <= 1, then normalised, all in fp32 (kvq.h states the
+// exact recipe; the host computes it, the pool stores it).
+void hqmq_codebook(uint64_t seed, int h, int t, float *S)
+{
+    uint64_t state = seed ^ ((uint64_t)(2 * h + t + 1) * 0xD1B54A32D192ED03ULL);
+    for (int n = 0; n < kHqmqNS;) {
+        float a[4];
+        for (int i = 0; i < 4; i++) {
+            const float m = (float)(splitmix64_next(state) >> 40);  // < 2^24: exact
+            a[i] = m * (1.0f / 8388608.0f) - 1.0f;
+        }
+        // each square and each sum rounded to fp32, in order (the stores
+        // through volatile keep a product from fusing into the next add)
+        volatile float sq[4];
+        for (int i = 0; i < 4; i++) sq[i] = a[i] * a[i];
+        volatile float n2 = sq[0];
+        for (int i = 1; i < 4; i++) n2 = n2 + sq[i];
+        const float q = n2;
+        if (!(q > 1e-4f && q <= 1.0f)) continue;
+        const float r = sqrtf(q);
+        for (int i = 0; i < 4; i++) S[4 * n + i] = a[i] / r;
+        n++;
+    }
+}
+
 kvq_status check_config(const kvq_config *c)
 {
     if (!c) return KVQ_ERR_INVALID_ARG;
@@ -45,9 +74,15 @@ kvq_status check_config(const kvq_config *c)
             if (t == 1) return KVQ_ERR_UNSUPPORTED;  // values: int4 or int2
             if (groups[t] != c->head_dim) return KVQ_ERR_UNSUPPORTED;
             break;
+        case KVQ_HQMQ:
+            if (groups[t] != 4 || c->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+            break;
         default: return KVQ_ERR_INVALID_ARG;
         }
     }
+    const bool hq = c->k_fmt == KVQ_HQMQ;
+    if (hq != (c->v_fmt == KVQ_HQMQ)) return KVQ_ERR_UNSUPPORTED;  // HQMQ keys and values, or neither
+    if (hq && (c->bound_block_tokens != 0 || c->scale_search != 0)) return KVQ_ERR_UNSUPPORTED;
     if (!(c->clip_ratio > 0.0f && c->clip_ratio <= 1.0f)) return KVQ_ERR_INVALID_ARG;
     if (c->bound_block_tokens < 0 || c->bound_block_tokens % kPageTokens) return KVQ_ERR_INVALID_ARG;
     if (c->rotate != 0 && c->rotate != 1) return KVQ_ERR_INVALID_ARG;
@@ -229,6 +264,7 @@ size_t kvq_pool_bytes(const kvq_config *cfg)
     const Layout L = make_layout(*cfg);
     size_t n = kHeaderBytes + (size_t)cfg->num_pages * L.page_bytes;
     if (cfg->bound_block_tokens > 0) n += (size_t)cfg->num_pages * cfg->num_kv_heads * 16;
+    if (cfg->k_fmt == KVQ_HQMQ) n += (size_t)cfg->num_kv_heads * 2 * kHqmqNS * 16;
     return n;
 }
 
@@ -270,6 +306,22 @@ kvq_status kvq_create_cache(const kvq_config *cfg, void *pool_dev, size_t pool_b
         delete c;
         return KVQ_ERR_CUDA;
     }
+    if (c->L.hq_tab) {
+        const size_t n = (size_t)cfg->num_kv_heads * 2 * kHqmqNS * 4;
+        float *tab = static_cast<float *>(malloc(n * sizeof(float)));
+        if (!tab) {
+            delete c;
+            return KVQ_ERR_CUDA;
+        }
+        for (int h = 0; h < cfg->num_kv_heads; h++)
+            for (int t = 0; t < 2; t++) hqmq_codebook(cfg->rotation_seed, h, t, tab + ((size_t)h * 2 + t) * kHqmqNS * 4);
+        const cudaError_t e = cudaMemcpy(c->pool + c->L.hq_tab, tab, n * sizeof(float), cudaMemcpyHostToDevice);
+        free(tab);
+        if (e != cudaSuccess) {
+            delete c;
+            return KVQ_ERR_CUDA;
+        }
+    }
     *out = c;
     return KVQ_OK;
 }
@@ -301,6 +353,7 @@ kvq_status kvq_append(kvq_cache *c, const void *k, const void *v, const int32_t 
     p.scale_search = c->cfg.scale_search;
     memcpy(p.sign_xor, c->sign_xor, sizeof(p.sign_xor));
     c->last_stream = stream;
+    if (c->L.hq_tab) return cuda_status(launch_hqmq_append(p, c->num_sms, static_cast<cudaStream_t>(stream)));
     return cuda_status(launch_append(p, c->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
@@ -419,6 +472,17 @@ kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const
     if (!q || !block_table || !ctx_lens || !out || !workspace) return KVQ_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
     if (k_new && (!v_new || !slot_mapping || !aligned(k_new, 16) || !aligned(v_new, 16))) return KVQ_ERR_INVALID_ARG;
+    if (c->L.hq_tab) {  // HQMQ: its own decode kernel, no fused append, no tier 2
+        if (k_new || tier2) return KVQ_ERR_UNSUPPORTED;
+        if (ws_bytes < kvq_decode_workspace_bytes(c, batch, max_pages_per_seq)) return KVQ_ERR_CAPACITY;
+        const SplitPlan s = plan_splits(c, batch, max_pages_per_seq);
+        const float scale = softmax_scale > 0.0f ? softmax_scale : (float)(1.0 / sqrt((double)c->L.d));
+        const DecodeParams p =
+            decode_params(c, s, q, block_table, max_pages_per_seq, ctx_lens, batch, scale, workspace, out);
+        c->last_stream = stream;
+        return cuda_status(
+            launch_hqmq_decode(p, dim3(s.n_splits, c->L.hkv, batch), static_cast<cudaStream_t>(stream)));
+    }
     if (!decode_supported(c->L)) return KVQ_ERR_UNSUPPORTED;
     // certified mode: checks and the tier-2 device view
     int kmax = 0;
@@ -637,6 +701,7 @@ kvq_status kvq_dequant_debug(kvq_cache *c, const int32_t *slots, int32_t n, floa
                              uint8_t *codes_out, uint16_t *meta_out, void *stream)
 {
     if (!c || n < 0) return KVQ_ERR_INVALID_ARG;
+    if (c->L.hq_tab) return KVQ_ERR_UNSUPPORTED;  // integer formats only
     if (n == 0) return KVQ_OK;
     if (!slots) return KVQ_ERR_INVALID_ARG;
     DequantParams p{};

@@ -1,0 +1,619 @@
+// kvq_hqmq.cu -- the HQMQ codec ["Hurwitz Quaternion Multiplicative
+// Quantization for KV Cache Compression", 1-3] on the paged pool:
+// quantise-on-append of K/V rows into 20-bit quaternion codes with Med3x
+// fp16 outliers, and split-K decode attention over those codes.
+//
+// Append.  A warp holds one rotated row of 128 elements, lane b owning the
+// quaternion block b (elements 4b..4b+3), so the row statistics (radii, the
+// lower median by a bitonic sort across lanes, the two largest outliers by
+// warp max-reductions) are shuffles and the code of block b is lane b's.
+// The codeword search dominates: for each of the 1024 secondary quaternions
+// q_s, w = u conj(q_s) and the best of the 24 Hurwitz units is closed-form
+// (largest |w_i| or half the sum of |w_i|), 16 multiplies, 12 adds and a
+// handful of max/compare operations per candidate; conj(q_s) comes from
+// shared memory as one broadcast 16-byte load.  Every operation that decides
+// a code is an explicitly rounded fp32 operation in the order kvq.h states,
+// so codes match a plain fp32 statement bit for bit.  When there are few rows
+// (a decode step appends one token), the 1024 candidates of a row are split
+// over the CTA's 8 warps and the per-block winners combined (highest score,
+// lowest candidate on ties, which is the sequential rule).
+//
+// Decode.  CTAs take contiguous token ranges of one (sequence, kv head) and
+// hold that head's two codebooks in shared memory (32 KB); a warp decodes 8
+// tokens at a time, lane b rebuilding block b of K and V as (radius code x
+// step) x q_p q_s (or the fp16 outlier), then partial dot products for 8
+// tokens x 4 heads reduce in one transpose-reduce and the online softmax
+// runs per head.  Split partials merge in the last CTA of each (sequence, kv
+// head), which also applies the inverse rotation.  The path is bound by the
+// fp32 pipe (about 80 operations a block per token for K and V together),
+// not by HBM: 208 bytes a token-head against ~2.5 K operations.
+#include <math.h>
+
+#include "kvq_cert.cuh"
+#include "kvq_internal.cuh"
+#include "kvq_warp.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kHqWarps = 8;
+constexpr int kHqThreads = kHqWarps * 32;
+constexpr int kHqD = 128;          // head_dim of HQMQ caches
+constexpr int kHqRowCode = 80;     // 32 blocks x 20 bits
+constexpr int kHqTok = 8;          // tokens a decode warp has in flight
+constexpr unsigned kHqFieldMask = 0xFFFFFu;
+
+// ------------------------------------------------------------------ append --
+
+// Score of unit direction u against codeword conj(q_s) = c, exactly as kvq.h
+// states: w = u c (Hamilton product, products summed left to right), the
+// best axis unit max_i |w_i| or the best half unit (sum |w_i|) / 2.
+__device__ __forceinline__ void hamilton_rn(const float (&u)[4], float4 c, float (&w)[4])
+{
+    w[0] = __fsub_rn(__fsub_rn(__fsub_rn(__fmul_rn(u[0], c.x), __fmul_rn(u[1], c.y)), __fmul_rn(u[2], c.z)),
+                     __fmul_rn(u[3], c.w));
+    w[1] = __fsub_rn(__fadd_rn(__fadd_rn(__fmul_rn(u[0], c.y), __fmul_rn(u[1], c.x)), __fmul_rn(u[2], c.w)),
+                     __fmul_rn(u[3], c.z));
+    w[2] = __fadd_rn(__fadd_rn(__fsub_rn(__fmul_rn(u[0], c.z), __fmul_rn(u[1], c.w)), __fmul_rn(u[2], c.x)),
+                     __fmul_rn(u[3], c.y));
+    w[3] = __fadd_rn(__fsub_rn(__fadd_rn(__fmul_rn(u[0], c.w), __fmul_rn(u[1], c.z)), __fmul_rn(u[2], c.y)),
+                     __fmul_rn(u[3], c.x));
+}
+
+__device__ __forceinline__ float score_only(const float (&u)[4], float4 c)
+{
+    float w[4];
+    hamilton_rn(u, c, w);
+    const float a0 = fabsf(w[0]), a1 = fabsf(w[1]), a2 = fabsf(w[2]), a3 = fabsf(w[3]);
+    const float ma = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+    const float mh = __fmul_rn(__fadd_rn(__fadd_rn(__fadd_rn(a0, a1), a2), a3), 0.5f);
+    return mh > ma ? mh : ma;
+}
+
+__device__ __forceinline__ int unit_of(const float (&u)[4], float4 c)
+{
+    float w[4];
+    hamilton_rn(u, c, w);
+    float aw[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) aw[i] = fabsf(w[i]);
+    int ia = 0;
+    float ma = aw[0];
+#pragma unroll
+    for (int i = 1; i < 4; i++)
+        if (aw[i] > ma) {
+            ma = aw[i];
+            ia = i;
+        }
+    const float mh = __fmul_rn(__fadd_rn(__fadd_rn(__fadd_rn(aw[0], aw[1]), aw[2]), aw[3]), 0.5f);
+    if (mh > ma) return 8 + (w[0] < 0.f) + 2 * (w[1] < 0.f) + 4 * (w[2] < 0.f) + 8 * (w[3] < 0.f);
+    return 2 * ia + (w[ia] < 0.f);
+}
+
+// ascending bitonic sort of one float per lane across the warp
+__device__ __forceinline__ float warp_sort_asc(float v, int lane)
+{
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const float o = __shfl_xor_sync(kFull, v, j);
+            const bool up = (lane & k) == 0 || k == 32;
+            const bool low = (lane & j) == 0;
+            v = (low == up) ? fminf(v, o) : fmaxf(v, o);
+        }
+    return v;
+}
+
+// One row's statistics and codes, every lane of the warp (lane = block).
+struct HqRow {
+    float x[4];      // rotated values of the lane's block
+    float u[4];      // unit direction (r > 0)
+    float r;         // radius
+    unsigned rc;     // radius code
+    uint32_t mask;   // outlier blocks
+    __half step;
+};
+
+__device__ __forceinline__ void hq_prepare(const AppendParams &p, const __half *src, int lane, HqRow &R)
+{
+    uint2 raw = *reinterpret_cast<const uint2 *>(src + 4 * lane);
+    if (p.rotate) {
+        raw.x ^= p.sign_xor[2 * lane];
+        raw.y ^= p.sign_xor[2 * lane + 1];
+    }
+    const float2 a = __half22float2(bits_h2(raw.x)), b = __half22float2(bits_h2(raw.y));
+    float x[4] = {a.x, a.y, b.x, b.y};
+    if (p.rotate) {
+        fwht_warp<kHqD>(x, lane);  // butterfly stages h = 1, 2, ..., 64, each add rounded
+#pragma unroll
+        for (int e = 0; e < 4; e++) x[e] = __fmul_rn(x[e], p.rot_scale);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; e++) R.x[e] = x[e];
+    const float r = __fsqrt_rn(__fadd_rn(__fadd_rn(__fadd_rn(__fmul_rn(x[0], x[0]), __fmul_rn(x[1], x[1])),
+                                                   __fmul_rn(x[2], x[2])),
+                                         __fmul_rn(x[3], x[3])));
+    R.r = r;
+    // Med3x: tau = 3 x the lower median radius (the 16th smallest of 32)
+    const float med = __shfl_sync(kFull, warp_sort_asc(r, lane), 15);
+    const float tau = __fmul_rn(3.0f, med);
+    // outliers: the largest radius above tau, then the next (lowest block on ties);
+    // radii above tau are positive, so their bit patterns order like the values
+    const bool over = r > tau;
+    const unsigned rb = __float_as_uint(r);
+    const unsigned m1 = __reduce_max_sync(kFull, over ? rb : 0u);
+    const unsigned b1 = __ballot_sync(kFull, over && rb == m1);
+    const int pick1 = b1 ? __ffs(b1) - 1 : -1;
+    const bool over2 = over && lane != pick1;
+    const unsigned m2 = __reduce_max_sync(kFull, over2 ? rb : 0u);
+    const unsigned b2 = __ballot_sync(kFull, over2 && rb == m2);
+    const int pick2 = b2 ? __ffs(b2) - 1 : -1;
+    R.mask = (pick1 >= 0 ? 1u << pick1 : 0u) | (pick2 >= 0 ? 1u << pick2 : 0u);
+    // radius step and code
+    R.step = __float2half_ru(__fdiv_rn(tau, 31.0f));
+    const float sf = __half2float(R.step);
+    unsigned rc = 0;
+    if (sf > 0.0f) {
+        const float v = rintf(__fdiv_rn(r, sf));
+        rc = v > 31.0f ? 31u : (unsigned)v;
+    }
+    R.rc = min(rc, 31u);  // (a NaN radius must not spill into the next field)
+#pragma unroll
+    for (int e = 0; e < 4; e++) R.u[e] = r > 0.0f ? __fdiv_rn(x[e], r) : 0.0f;
+}
+
+// Best candidate of s in [s0, s1): strictly higher score wins, so the first
+// of equal scores stays.
+__device__ __forceinline__ void hq_search(const float (&u)[4], const float4 *cb, int s0, int s1, float &best, int &bs)
+{
+    best = -INFINITY;
+    bs = s0;
+#pragma unroll 4
+    for (int s = s0; s < s1; s++) {
+        const float sc = score_only(u, cb[s]);
+        if (sc > best) {
+            best = sc;
+            bs = s;
+        }
+    }
+}
+
+// Pack and store a coded row: fields as one little-endian 20-bit stream
+// (lane k < 20 writes 32-bit word k), then the meta row.
+__device__ __forceinline__ void hq_store(unsigned char *codes, unsigned char *meta, uint32_t field, const HqRow &R,
+                                         int lane)
+{
+    const int blo = (32 * lane) / 20, sh = 32 * lane - 20 * blo;
+    const uint32_t f0 = __shfl_sync(kFull, field, min(blo, 31));
+    const uint32_t f1 = __shfl_sync(kFull, field, min(blo + 1, 31));
+    const uint32_t f2 = __shfl_sync(kFull, field, min(blo + 2, 31));
+    const unsigned long long v = (unsigned long long)f0 | ((unsigned long long)(blo + 1 <= 31 ? f1 : 0u) << 20) |
+                                 ((unsigned long long)(blo + 2 <= 31 ? f2 : 0u) << 40);
+    if (lane < kHqRowCode / 4) reinterpret_cast<uint32_t *>(codes)[lane] = (uint32_t)(v >> sh);
+    const int nout = __popc(R.mask);
+    if (lane == 0) reinterpret_cast<uint32_t *>(meta)[0] = (uint32_t)__half_as_ushort(R.step);
+    if (lane == 1) reinterpret_cast<uint32_t *>(meta)[1] = R.mask;
+    if ((R.mask >> lane) & 1u) {
+        const int slot = __popc(R.mask & ((1u << lane) - 1u));
+        const __half2 h01 = __floats2half2_rn(R.x[0], R.x[1]), h23 = __floats2half2_rn(R.x[2], R.x[3]);
+        reinterpret_cast<uint2 *>(meta + 8)[slot] = make_uint2(h2_bits(h01), h2_bits(h23));
+    }
+    if (lane >= 2 && lane < 2 + kHqmqOut && lane - 2 >= nout)
+        reinterpret_cast<uint2 *>(meta + 8)[lane - 2] = make_uint2(0u, 0u);
+}
+
+// Grid (CTAs per (kv head, tensor), 2 Hkv): the CTA loads conj(S) of its
+// (kv head, tensor) once, then codes rows of tokens n = its own, stride all
+// of its column.  WPR warps share a row (1: a warp a row; 8: the CTA a row).
+template <int WPR>
+__global__ void __launch_bounds__(kHqThreads) hqmq_append_kernel(const __grid_constant__ AppendParams p)
+{
+    constexpr int RPC = kHqWarps / WPR;  // rows per CTA pass
+    constexpr int SPAN = kHqmqNS / WPR;  // candidates per warp
+    __shared__ float4 cb[kHqmqNS];
+    __shared__ float wsc[WPR > 1 ? 2 : 1][kHqWarps][32];
+    __shared__ int wsi[WPR > 1 ? 2 : 1][kHqWarps][32];
+    const int pair = blockIdx.y, kvh = pair >> 1, tensor = pair & 1;
+    const Layout &L = p.L;
+    {
+        const float4 *S = reinterpret_cast<const float4 *>(p.pool + L.hq_tab) + (long long)pair * kHqmqNS;
+        for (int i = threadIdx.x; i < kHqmqNS; i += kHqThreads) {
+            const float4 s = S[i];
+            cb[i] = make_float4(s.x, -s.y, -s.z, -s.w);  // exact sign flips
+        }
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rgrp = warp / WPR, slice = warp % WPR;
+    const int stride = gridDim.x * RPC;
+    int par = 0;
+    for (int base = blockIdx.x * RPC; base < p.n_tok; base += stride, par ^= 1) {
+        const int n = base + rgrp;
+        bool active = n < p.n_tok;
+        int slot = active ? p.slots[n] : -1;
+        if (slot < 0) active = false;
+        if (active && slot >= L.num_pages * kPageTokens) {
+            if (lane == 0 && slice == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
+            active = false;
+        }
+        float best = -INFINITY;
+        int bs = 0;
+        HqRow R{};
+        if (active) {  // warp-uniform
+            const __half *src = (tensor ? p.v : p.k) + ((long long)n * L.hkv + kvh) * kHqD;
+            hq_prepare(p, src, lane, R);
+            hq_search(R.u, cb, slice * SPAN, slice * SPAN + SPAN, best, bs);
+        }
+        if constexpr (WPR > 1) {
+            wsc[par][warp][lane] = best;
+            wsi[par][warp][lane] = bs;
+            __syncthreads();  // (two buffers: the next pass writes the other one)
+            if (slice == 0) {
+#pragma unroll
+                for (int w = 1; w < WPR; w++) {
+                    const float o = wsc[par][rgrp * WPR + w][lane];
+                    if (o > best) {
+                        best = o;
+                        bs = wsi[par][rgrp * WPR + w][lane];
+                    }
+                }
+            }
+        }
+        if (active && slice == 0) {
+            const bool outl = (R.mask >> lane) & 1u;
+            uint32_t field = 0;
+            if (!outl) {
+                const uint32_t idx = R.r > 0.0f ? (uint32_t)(24 * bs + unit_of(R.u, cb[bs])) : 0u;
+                field = idx | (R.rc << 15);
+            }
+            const int page = slot / kPageTokens, tok = slot % kPageTokens;
+            unsigned char *chunk =
+                p.pool + kHeaderBytes + (long long)page * L.page_bytes + (long long)kvh * L.chunk_bytes;
+            unsigned char *codes = chunk + (tensor ? L.v_codes : L.k_codes) + tok * kHqRowCode;
+            unsigned char *meta = chunk + (tensor ? L.v_meta : L.k_meta) + tok * kHqmqRowMeta;
+            hq_store(codes, meta, field, R, lane);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ decode --
+
+// The 20-bit field of block `lane` in a token's code row.
+__device__ __forceinline__ uint32_t hq_field(const unsigned char *row, int lane)
+{
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(row);
+    const int bit = 20 * lane, w0 = bit >> 5, sh = bit & 31;
+    const uint32_t lo = __ldg(w + w0);
+    const uint32_t hi = sh > 12 ? __ldg(w + w0 + 1) : 0u;  // word 20 is never needed
+    return __funnelshift_r(lo, hi, sh) & kHqFieldMask;
+}
+
+// Block `lane` of a row: (radius code x step) x q_p q_s with q_s from the
+// codebook in shared memory, or the fp16 outlier values.  meta = (step | 0,
+// outlier mask) of the row; outl = its outlier slots.
+__device__ __forceinline__ void hq_block(uint32_t f, uint2 meta, const unsigned char *outl, const float4 *S, int lane,
+                                         float (&c)[4])
+{
+    if ((meta.y >> lane) & 1u) {
+        const int slot = min(__popc(meta.y & ((1u << lane) - 1u)), kHqmqOut - 1);
+        const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(outl) + slot);
+        const float2 a = __half22float2(bits_h2(raw.x)), b = __half22float2(bits_h2(raw.y));
+        c[0] = a.x;
+        c[1] = a.y;
+        c[2] = b.x;
+        c[3] = b.y;
+        return;
+    }
+    const uint32_t idx = f & 0x7FFFu, s = min(idx / 24u, (uint32_t)kHqmqNS - 1u), pp = idx - 24u * (idx / 24u);
+    const float4 q = S[s];
+    const float rad = (float)(f >> 15) * __half2float(__ushort_as_half((unsigned short)(meta.x & 0xFFFFu)));
+    // q_p: an axis unit (+-1 on component pp/2) or a half unit (+-1/2, bit i of pp - 8 = sign of component i)
+    float a[4];
+    const bool half = pp >= 8u;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const float hv = ((pp - 8u) >> i) & 1u ? -0.5f : 0.5f;
+        const float av = (pp >> 1) == (uint32_t)i ? ((pp & 1u) ? -1.0f : 1.0f) : 0.0f;
+        a[i] = (half ? hv : av) * rad;
+    }
+    c[0] = a[0] * q.x - a[1] * q.y - a[2] * q.z - a[3] * q.w;
+    c[1] = a[0] * q.y + a[1] * q.x + a[2] * q.w - a[3] * q.z;
+    c[2] = a[0] * q.z - a[1] * q.w + a[2] * q.x + a[3] * q.y;
+    c[3] = a[0] * q.w + a[1] * q.z - a[2] * q.y + a[3] * q.x;
+}
+
+// Grid (splits, Hkv, B); split `blockIdx.x` attends tokens [x * tps, +tps) of
+// its sequence (tps = pages_per_split * 16).  Partials [g][d + 4] (sums, max,
+// sum of weights) go to p.part; the last CTA merges them.
+template <int G>
+__global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid_constant__ DecodeParams p)
+{
+    const Layout &L = p.L;
+    const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = L.g;
+    __shared__ __align__(16) float4 tab[2 * kHqmqNS];  // K then V codebook; the warps' sums after the loop
+    __shared__ __align__(16) float sq[G * kHqD];
+    __shared__ float wm[kHqWarps][G], wl[kHqWarps][G];
+    __shared__ int sflag;
+
+    int T = p.ctx_lens[b];
+    if (T < 0 || T > p.max_pages * kPageTokens) {
+        if (split == 0 && tid == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
+        T = T < 0 ? 0 : p.max_pages * kPageTokens;
+    }
+    const int tps = p.pages_per_split * kPageTokens;
+    const int n_act = max(1, (T + tps - 1) / tps);
+    if (split >= n_act) return;
+    const int t_begin = split * tps, t_end = min(T, t_begin + tps);
+
+    {
+        const float4 *S = reinterpret_cast<const float4 *>(p.pool + L.hq_tab) + (long long)kvh * 2 * kHqmqNS;
+        for (int i = tid; i < 2 * kHqmqNS; i += kHqThreads) tab[i] = __ldg(S + i);
+    }
+    if (warp < g) {  // the rotated query in log2 units
+        const __half *qh = p.q + ((long long)b * L.hq + kvh * g + warp) * kHqD + lane * 4;
+        const uint2 raw = *reinterpret_cast<const uint2 *>(qh);
+        const float2 a = __half22float2(bits_h2(raw.x)), c = __half22float2(bits_h2(raw.y));
+        float x[4] = {a.x, a.y, c.x, c.y};
+        if (p.rotate) {
+#pragma unroll
+            for (int e = 0; e < 4; e++) x[e] *= p.signs[lane * 4 + e];
+            fwht_warp<kHqD>(x, lane);
+#pragma unroll
+            for (int e = 0; e < 4; e++) x[e] *= p.rot_scale;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; e++) sq[warp * kHqD + lane * 4 + e] = x[e] * p.qscale;
+    }
+    __syncthreads();
+    const float4 *SK = tab, *SV = tab + kHqmqNS;
+    float qr[G][4];
+#pragma unroll
+    for (int h = 0; h < G; h++)
+#pragma unroll
+        for (int e = 0; e < 4; e++) qr[h][e] = h < g ? sq[h * kHqD + lane * 4 + e] : 0.f;
+
+    float m[G], l[G], acc[G][4];
+#pragma unroll
+    for (int h = 0; h < G; h++) {
+        m[h] = -INFINITY;
+        l[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; e++) acc[h][e] = 0.f;
+    }
+    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
+    const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
+    constexpr int NHG = G > 4 ? G / 4 : 1;
+    const int uj = lane >> 2, hlj = lane & 3;
+
+    for (int tb = t_begin + warp * kHqTok; tb < t_end; tb += kHqWarps * kHqTok) {
+        // the batch's fields and meta rows, all loads issued before any math
+        // the batch's token rows (chunk offsets), fields and meta rows, all
+        // loads issued before any math; a batch never leaves its page
+        uint32_t kf[kHqTok], vf[kHqTok];
+        uint2 km[kHqTok], vm[kHqTok];
+        unsigned vmask = 0;
+        long long cofs = 0;  // the batch's chunk, from kv_base
+        {
+            const int pg = tb < t_end ? bt[tb / kPageTokens] : -1;
+            if (tb < t_end && (pg < 0 || pg >= L.num_pages)) {
+                if (lane == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
+            } else if (tb < t_end) {
+                cofs = (long long)pg * L.page_bytes;
+                vmask = (1u << min(kHqTok, t_end - tb)) - 1u;
+            }
+        }
+        const unsigned char *chunk = kv_base + cofs;
+        const int tok0 = tb % kPageTokens;
+#pragma unroll
+        for (int u = 0; u < kHqTok; u++) {
+            kf[u] = vf[u] = 0u;
+            km[u] = vm[u] = make_uint2(0u, 0u);
+            if ((vmask >> u) & 1u) {
+                const int tok = tok0 + u;
+                kf[u] = hq_field(chunk + L.k_codes + tok * kHqRowCode, lane);
+                vf[u] = hq_field(chunk + L.v_codes + tok * kHqRowCode, lane);
+                km[u] = __ldg(reinterpret_cast<const uint2 *>(chunk + L.k_meta + tok * kHqmqRowMeta));
+                vm[u] = __ldg(reinterpret_cast<const uint2 *>(chunk + L.v_meta + tok * kHqmqRowMeta));
+            }
+        }
+        // keys: per head group, rebuild each block and take the partial dots
+        // (one group of four heads rebuilds once), then totals and softmax
+        float pw[NHG];
+#pragma unroll
+        for (int hg = 0; hg < NHG; hg++) {
+            float d[32];
+#pragma unroll
+            for (int u = 0; u < kHqTok; u++) {
+                float kc[4] = {0.f, 0.f, 0.f, 0.f};
+                if ((vmask >> u) & 1u)
+                    hq_block(kf[u], km[u], chunk + L.k_meta + (tok0 + u) * kHqmqRowMeta + 8, SK, lane, kc);
+#pragma unroll
+                for (int hl = 0; hl < 4; hl++) {
+                    const int h = hg * 4 + hl;
+                    float a = 0.f;
+                    if (h < G) {
+#pragma unroll
+                        for (int e = 0; e < 4; e++) a = fmaf(qr[h][e], kc[e], a);
+                    }
+                    d[u * 4 + hl] = a;
+                }
+            }
+            float sc = cert::transpose_reduce32(d, lane);  // lane: token uj, head 4 hg + hlj
+            const bool live = ((vmask >> uj) & 1u) && hg * 4 + hlj < g;
+            if (!live) sc = -INFINITY;
+            float bmax = sc;
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
+            float mo = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 4; k++)
+                if (hg * 4 + k < G && hlj == k) mo = m[hg * 4 + k];
+            const float mnew = fmaxf(mo, bmax);
+            const float pj = sc == -INFINITY ? 0.f : ex2(sc - mnew);
+            float psum = pj;
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) psum += __shfl_xor_sync(kFull, psum, o);
+            pw[hg] = pj;
+#pragma unroll
+            for (int k = 0; k < 4; k++) {  // lane k holds head 4 hg + k's figures
+                const int h = hg * 4 + k;
+                if (h >= G || h >= g) break;
+                const float mn = __shfl_sync(kFull, mnew, k), ps = __shfl_sync(kFull, psum, k);
+                const float al = m[h] == -INFINITY ? 0.f : ex2(m[h] - mn);
+                l[h] = fmaf(l[h], al, ps);
+#pragma unroll
+                for (int e = 0; e < 4; e++) acc[h][e] *= al;
+                m[h] = mn;
+            }
+        }
+        // values: rebuild each token's block once, every head takes its weight
+#pragma unroll
+        for (int u = 0; u < kHqTok; u++) {
+            if (!((vmask >> u) & 1u)) continue;  // warp-uniform
+            float vc[4];
+            hq_block(vf[u], vm[u], chunk + L.v_meta + (tok0 + u) * kHqmqRowMeta + 8, SV, lane, vc);
+#pragma unroll
+            for (int h = 0; h < G; h++) {
+                if (h >= g) break;
+                const float w = __shfl_sync(kFull, pw[h >> 2], u * 4 + (h & 3));
+#pragma unroll
+                for (int e = 0; e < 4; e++) acc[h][e] = fmaf(w, vc[e], acc[h][e]);
+            }
+        }
+    }
+
+    // warps -> one partial per head: sums, then (max, sum of weights)
+    __syncthreads();  // every warp is done with the codebooks
+    float *wacc = reinterpret_cast<float *>(tab);  // [kHqWarps][G][128]
+#pragma unroll
+    for (int h = 0; h < G; h++)
+        if (h < g) {
+            *reinterpret_cast<float4 *>(wacc + (warp * G + h) * kHqD + lane * 4) =
+                make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+            if (lane == 0) {
+                wm[warp][h] = m[h];
+                wl[warp][h] = l[h];
+            }
+        }
+    __syncthreads();
+    constexpr int REC = kHqD + 4;
+    const long long bk = (long long)b * L.hkv + kvh;
+    float *part = p.part + (bk * p.n_splits + split) * (long long)g * REC;
+    for (int idx = tid; idx < g * kHqD; idx += kHqThreads) {
+        const int h = idx / kHqD, ch = idx - h * kHqD;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kHqWarps; w++) M = fmaxf(M, wm[w][h]);
+        float a = 0.f, Ls = 0.f;
+        if (M != -INFINITY)
+#pragma unroll
+            for (int w = 0; w < kHqWarps; w++) {
+                const float f = wm[w][h] == -INFINITY ? 0.f : ex2(wm[w][h] - M);
+                a = fmaf(f, wacc[(w * G + h) * kHqD + ch], a);
+                Ls = fmaf(f, wl[w][h], Ls);
+            }
+        part[h * REC + ch] = a;
+        if (ch == 0) {
+            part[h * REC + kHqD] = M;
+            part[h * REC + kHqD + 1] = Ls;
+        }
+    }
+
+    // the last CTA of this (sequence, kv head) merges the splits
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(p.counters + bk, 1u);
+        sflag = prev == (unsigned)(n_act - 1);
+    }
+    __syncthreads();
+    if (!sflag) return;
+    __threadfence();
+    if (tid == 0) p.counters[bk] = 0u;
+    const float *pb = p.part + bk * p.n_splits * (long long)g * REC;
+    for (int h = warp; h < g; h += kHqWarps) {
+        float M = -INFINITY;
+        for (int c = lane; c < n_act; c += 32) M = fmaxf(M, __ldcg(pb + (c * g + h) * REC + kHqD));
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+        float Ls = 0.f;
+        for (int c = lane; c < n_act; c += 32) {
+            const float mc = __ldcg(pb + (c * g + h) * REC + kHqD), lc = __ldcg(pb + (c * g + h) * REC + kHqD + 1);
+            if (mc != -INFINITY) Ls = fmaf(lc, ex2(mc - M), Ls);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) Ls += __shfl_xor_sync(kFull, Ls, o);
+        float o4[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c = 0; c < n_act; c++) {
+            const float mc = __ldcg(pb + (c * g + h) * REC + kHqD);
+            const float f = mc == -INFINITY ? 0.f : ex2(mc - M);
+            const float4 r = __ldcg(reinterpret_cast<const float4 *>(pb + (c * g + h) * REC + lane * 4));
+            o4[0] = fmaf(f, r.x, o4[0]);
+            o4[1] = fmaf(f, r.y, o4[1]);
+            o4[2] = fmaf(f, r.z, o4[2]);
+            o4[3] = fmaf(f, r.w, o4[3]);
+        }
+        if (p.rotate) {  // back to the original domain: diag(s) H c
+            fwht_warp<kHqD>(o4, lane);
+#pragma unroll
+            for (int e = 0; e < 4; e++) o4[e] *= p.rot_scale * p.signs[lane * 4 + e];
+        }
+        float *out = p.out + ((long long)b * L.hq + kvh * g + h) * kHqD + lane * 4;
+        *reinterpret_cast<float4 *>(out) = Ls > 0.f ? make_float4(o4[0] / Ls, o4[1] / Ls, o4[2] / Ls, o4[3] / Ls)
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+template <int G>
+cudaError_t launch_hq_decode_g(const DecodeParams &p, dim3 grid, cudaStream_t s)
+{
+    hqmq_decode_kernel<G><<<grid, kHqThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+// CTAs per (kv head, tensor) column: what stays resident in one wave (the
+// instantiation's own occupancy), no more than the tokens need (8 / WPR rows a pass).
+template <int WPR>
+cudaError_t launch_hq_append_w(const AppendParams &p, int num_sms, cudaStream_t st)
+{
+    static int resident = 0;
+    if (resident == 0) {
+        int n = 0;
+        const cudaError_t e =
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, hqmq_append_kernel<WPR>, kHqThreads, 0);
+        if (e != cudaSuccess) return e;
+        resident = n < 1 ? 1 : n;
+    }
+    const int pairs = 2 * p.L.hkv;
+    const long long wave = (long long)resident * num_sms / pairs;
+    const long long need = (p.n_tok + kHqWarps / WPR - 1) / (kHqWarps / WPR);
+    const int per = (int)(wave < 1 ? 1 : (wave < need ? wave : need));
+    hqmq_append_kernel<WPR><<<dim3(per, pairs), kHqThreads, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_hqmq_append(const AppendParams &p, int num_sms, cudaStream_t st)
+{
+    if (p.n_tok == 0) return cudaSuccess;
+    if ((long long)p.n_tok * p.L.hkv > (1ll << 30)) return cudaErrorInvalidValue;  // 32-bit row indexing
+    // few rows (a decode step): the CTA shares each row; many: a warp a row
+    const long long rows = 2LL * p.n_tok * p.L.hkv;
+    if (rows < 2LL * num_sms * kHqWarps) return launch_hq_append_w<8>(p, num_sms, st);
+    return launch_hq_append_w<1>(p, num_sms, st);
+}
+
+cudaError_t launch_hqmq_decode(const DecodeParams &p, dim3 grid, cudaStream_t s)
+{
+    const int g = p.L.g;
+    if (g <= 1) return launch_hq_decode_g<1>(p, grid, s);
+    if (g <= 2) return launch_hq_decode_g<2>(p, grid, s);
+    if (g <= 4) return launch_hq_decode_g<4>(p, grid, s);
+    return launch_hq_decode_g<8>(p, grid, s);
+}
+
+}  // namespace kvq

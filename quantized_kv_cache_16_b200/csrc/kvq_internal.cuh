@@ -22,7 +22,16 @@ struct PoolHeader {
     unsigned int pad[63];
 };
 
-inline __host__ __device__ int fmt_bits(int fmt) { return fmt == KVQ_INT4_ASYM ? 4 : fmt == KVQ_INT8_SYM ? 8 : 2; }
+// HQMQ: 1024 secondary codewords per (kv head, K|V); two fp16 outlier blocks
+// per row; 20 bits per 4-element block (5 bits an element); 24 meta bytes.
+constexpr int kHqmqNS = 1024;
+constexpr int kHqmqOut = 2;
+constexpr int kHqmqRowMeta = 8 + 8 * kHqmqOut;
+
+inline __host__ __device__ int fmt_bits(int fmt)
+{
+    return fmt == KVQ_INT4_ASYM ? 4 : fmt == KVQ_INT8_SYM ? 8 : fmt == KVQ_HQMQ ? 5 : 2;
+}
 
 // Byte layout of the pool (see kvq_pool_bytes in kvq.h).
 struct Layout {
@@ -36,6 +45,7 @@ struct Layout {
     int num_pages;
     long long desc_off;  // from the pool start; 0 when descriptors are off
     int bound_block;
+    long long hq_tab;    // HQMQ codebooks [Hkv][2][1024] float4 from the pool start; 0 otherwise
 };
 
 inline __host__ Layout make_layout(const kvq_config &c)
@@ -49,8 +59,8 @@ inline __host__ Layout make_layout(const kvq_config &c)
     L.v_fmt = c.v_fmt;
     L.k_row_code = L.d * fmt_bits(c.k_fmt) / 8;
     L.v_row_code = L.d * fmt_bits(c.v_fmt) / 8;
-    L.k_row_meta = c.k_fmt == KVQ_INT8_SYM ? 2 : 4 * (L.d / c.k_group);
-    L.v_row_meta = c.v_fmt == KVQ_INT8_SYM ? 2 : 4 * (L.d / c.v_group);
+    L.k_row_meta = c.k_fmt == KVQ_HQMQ ? kHqmqRowMeta : c.k_fmt == KVQ_INT8_SYM ? 2 : 4 * (L.d / c.k_group);
+    L.v_row_meta = c.v_fmt == KVQ_HQMQ ? kHqmqRowMeta : c.v_fmt == KVQ_INT8_SYM ? 2 : 4 * (L.d / c.v_group);
     L.k_codes = 0;
     L.k_meta = kPageTokens * L.k_row_code;
     L.v_codes = L.k_meta + kPageTokens * L.k_row_meta;
@@ -60,6 +70,10 @@ inline __host__ Layout make_layout(const kvq_config &c)
     L.num_pages = c.num_pages;
     L.bound_block = c.bound_block_tokens;
     L.desc_off = c.bound_block_tokens > 0 ? kHeaderBytes + (long long)c.num_pages * L.page_bytes : 0;
+    L.hq_tab = 0;
+    if (c.k_fmt == KVQ_HQMQ)
+        L.hq_tab = kHeaderBytes + (long long)c.num_pages * L.page_bytes +
+                   (c.bound_block_tokens > 0 ? (long long)c.num_pages * L.hkv * 16 : 0);
     return L;
 }
 
@@ -223,6 +237,8 @@ cudaError_t launch_cert_promote(const CertParams &p, int batch, cudaStream_t s);
 cudaError_t launch_ladder_select(const CertParams &p, int batch, cudaStream_t s);
 cudaError_t launch_ladder_finish(const CertParams &p, int batch, cudaStream_t s);
 cudaError_t launch_windows(const CertParams &p, int batch, cudaStream_t s);
+cudaError_t launch_hqmq_append(const AppendParams &p, int num_sms, cudaStream_t s);
+cudaError_t launch_hqmq_decode(const DecodeParams &p, dim3 grid, cudaStream_t s);
 bool decode_supported(const Layout &L);
 int decode_max_splits(const Layout &L);
 constexpr int kDecodeWarps = 8;

@@ -15,7 +15,8 @@ TOL_MAX_ABS = 2e-3  # attention vs the oracle's fp64 attention (same dequantised
 TOL_REL_L2 = 1e-3
 
 
-def configs(wl: W.Workload, num_pages: int, rotate: int = 1):
+def configs(wl: W.Workload, num_pages: int, rotate=None):
+    rotate = wl.rotate if rotate is None else rotate
     import quantized_kv_cache_16_b200 as K
     kw = dict(num_q_heads=wl.Hq, num_kv_heads=wl.Hkv, head_dim=wl.d, k_fmt=wl.k_fmt, v_fmt=wl.v_fmt,
               k_group=wl.k_group, v_group=wl.v_group, clip_ratio=wl.clip, rotation_seed=wl.rotation_seed,
@@ -41,7 +42,7 @@ class Pair:
         return torch.tensor([t + extra for t in self.wl.ctx], dtype=torch.int32, device="cuda")
 
 
-def build_pair(wl: W.Workload, extra_tokens: int = 0, rotate: int = 1, oracle: bool = True, kv_rows=None) -> Pair:
+def build_pair(wl: W.Workload, extra_tokens: int = 0, rotate=None, oracle: bool = True, kv_rows=None) -> Pair:
     import torch
     import quantized_kv_cache_16_b200 as K
     pages = W.page_table(wl, extra_tokens=extra_tokens)[0]

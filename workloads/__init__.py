@@ -67,6 +67,7 @@ class Workload:
     seed: int = 0
     rotation_seed: int = 0x5EED
     steps: int = 1  # decode steps (each appends one token per sequence first)
+    rotate: int = 1  # 1: sign + Hadamard rotation before coding; 0: the raw rows
     description: str = ""
     extra: dict = field(default_factory=dict)
 
@@ -111,9 +112,10 @@ def ladder(T: int = 131072) -> Workload:
 
 def hqmq(T: int = 32768) -> Workload:
     return Workload(f"hqmq-llama3-8b-layer-T{T}", 1, 32, 8, 128, [T], k_fmt=HQMQ_FMT, v_fmt=HQMQ_FMT, k_group=4,
-                    v_group=4, dist="llama", seed=6, steps=1,
-                    description="batch 1, 32/8 heads, head_dim 128, llama's K/V, HQMQ K and V (4-element quaternion "
-                                "blocks, 24 x 1024 codewords, 5-bit radii, Med3x fp16 outliers)")
+                    v_group=4, dist="llama", seed=6, steps=1, rotate=0,
+                    description="batch 1, 32/8 heads, head_dim 128, llama's K/V (outlier key channels x15), HQMQ K "
+                                "and V of the raw rows (4-element quaternion blocks, 24 x 1024 codewords, 5-bit "
+                                "radii, Med3x fp16 outliers)")
 
 
 def int2(B: int = 4, T: int = 65536) -> Workload:
