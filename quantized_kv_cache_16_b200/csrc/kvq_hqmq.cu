@@ -279,25 +279,37 @@ __global__ void __launch_bounds__(kHqThreads) hqmq_append_kernel(const __grid_co
 
 // ------------------------------------------------------------------ decode --
 
-// The 20-bit field of block `lane` in a token's code row.
+// A (page, kv head) chunk of an HQMQ pool: K codes, K meta, V codes, V meta
+// of 16 tokens; the decode copies it whole into shared memory.
+constexpr int kHqChunk = 2 * kPageTokens * (kHqRowCode + kHqmqRowMeta);  // 3328 bytes
+constexpr int kHqStages = 2;                                                // per warp
+constexpr int kHqTabBytes = 2 * kHqmqNS * 16;
+constexpr int kHqOffStage = kHqTabBytes;
+constexpr int kHqOffBar = kHqOffStage + kHqWarps * kHqStages * kHqChunk;
+constexpr int kHqSmem = kHqOffBar + kHqWarps * kHqStages * 8;
+static_assert(kHqChunk % 16 == 0 && kHqOffStage % 16 == 0 && kHqOffBar % 8 == 0, "bulk copy alignment");
+constexpr int kHqMaxSplits = 64;  // the merge holds one weight per split in registers (two per lane)
+
+// The 20-bit field of block `lane` in a token's code row (shared memory).
 __device__ __forceinline__ uint32_t hq_field(const unsigned char *row, int lane)
 {
     const uint32_t *w = reinterpret_cast<const uint32_t *>(row);
     const int bit = 20 * lane, w0 = bit >> 5, sh = bit & 31;
-    const uint32_t lo = __ldg(w + w0);
-    const uint32_t hi = sh > 12 ? __ldg(w + w0 + 1) : 0u;  // word 20 is never needed
+    const uint32_t lo = w[w0];
+    const uint32_t hi = sh > 12 ? w[w0 + 1] : 0u;  // word 20 is never needed
     return __funnelshift_r(lo, hi, sh) & kHqFieldMask;
 }
 
 // Block `lane` of a row: (radius code x step) x q_p q_s with q_s from the
-// codebook in shared memory, or the fp16 outlier values.  meta = (step | 0,
-// outlier mask) of the row; outl = its outlier slots.
-__device__ __forceinline__ void hq_block(uint32_t f, uint2 meta, const unsigned char *outl, const float4 *S, int lane,
+// codebook in shared memory, or the fp16 outlier values.  meta = the row's
+// meta (shared memory): step | 0, outlier mask, two outlier slots.
+__device__ __forceinline__ void hq_block(uint32_t f, const unsigned char *meta, const float4 *S, int lane,
                                          float (&c)[4])
 {
-    if ((meta.y >> lane) & 1u) {
-        const int slot = min(__popc(meta.y & ((1u << lane) - 1u)), kHqmqOut - 1);
-        const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(outl) + slot);
+    const uint2 mm = *reinterpret_cast<const uint2 *>(meta);
+    if ((mm.y >> lane) & 1u) {
+        const int slot = min(__popc(mm.y & ((1u << lane) - 1u)), kHqmqOut - 1);
+        const uint2 raw = reinterpret_cast<const uint2 *>(meta + 8)[slot];
         const float2 a = __half22float2(bits_h2(raw.x)), b = __half22float2(bits_h2(raw.y));
         c[0] = a.x;
         c[1] = a.y;
@@ -305,17 +317,19 @@ __device__ __forceinline__ void hq_block(uint32_t f, uint2 meta, const unsigned 
         c[3] = b.y;
         return;
     }
-    const uint32_t idx = f & 0x7FFFu, s = min(idx / 24u, (uint32_t)kHqmqNS - 1u), pp = idx - 24u * (idx / 24u);
-    const float4 q = S[s];
-    const float rad = (float)(f >> 15) * __half2float(__ushort_as_half((unsigned short)(meta.x & 0xFFFFu)));
-    // q_p: an axis unit (+-1 on component pp/2) or a half unit (+-1/2, bit i of pp - 8 = sign of component i)
-    float a[4];
+    const uint32_t idx = f & 0x7FFFu, sq = idx / 24u, pp = idx - 24u * sq;
+    const float4 q = S[min(sq, (uint32_t)kHqmqNS - 1u)];
+    const float rad = (float)(f >> 15) * __half2float(__ushort_as_half((unsigned short)(mm.x & 0xFFFFu)));
+    // q_p x rad: an axis unit (+-1 on component pp/2) or a half unit (+-1/2,
+    // bit i of pp - 8 = the sign of component i), built from bit patterns
     const bool half = pp >= 8u;
+    const uint32_t hb = __float_as_uint(0.5f * rad), ab = __float_as_uint(rad);
+    float a[4];
 #pragma unroll
     for (int i = 0; i < 4; i++) {
-        const float hv = ((pp - 8u) >> i) & 1u ? -0.5f : 0.5f;
-        const float av = (pp >> 1) == (uint32_t)i ? ((pp & 1u) ? -1.0f : 1.0f) : 0.0f;
-        a[i] = (half ? hv : av) * rad;
+        const uint32_t hv = hb | ((((pp - 8u) >> i) & 1u) << 31);
+        const uint32_t av = (pp >> 1) == (uint32_t)i ? (ab | ((pp & 1u) << 31)) : 0u;
+        a[i] = __uint_as_float(half ? hv : av);
     }
     c[0] = a[0] * q.x - a[1] * q.y - a[2] * q.z - a[3] * q.w;
     c[1] = a[0] * q.y + a[1] * q.x + a[2] * q.w - a[3] * q.z;
@@ -323,9 +337,11 @@ __device__ __forceinline__ void hq_block(uint32_t f, uint2 meta, const unsigned 
     c[3] = a[0] * q.w + a[1] * q.z - a[2] * q.y + a[3] * q.x;
 }
 
-// Grid (splits, Hkv, B); split `blockIdx.x` attends tokens [x * tps, +tps) of
-// its sequence (tps = pages_per_split * 16).  Partials [g][d + 4] (sums, max,
-// sum of weights) go to p.part; the last CTA merges them.
+// Grid (splits, Hkv, B); split `blockIdx.x` attends pages [x * pps, +pps) of
+// its sequence, warp w pages [x * pps + w * ppw, +ppw) (pps = 8 ppw), each
+// page copied whole into the warp's two-stage ring by one bulk copy.
+// Partials [g][d + 4] (sums, max, sum of weights) go to p.part; the last CTA
+// merges them.
 template <int G>
 __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid_constant__ DecodeParams p)
 {
@@ -333,7 +349,8 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = L.g;
-    __shared__ __align__(16) float4 tab[2 * kHqmqNS];  // K then V codebook; the warps' sums after the loop
+    extern __shared__ __align__(128) unsigned char smem[];
+    float4 *tab = reinterpret_cast<float4 *>(smem);  // K then V codebook; the warps' sums after the loop
     __shared__ __align__(16) float sq[G * kHqD];
     __shared__ float wm[kHqWarps][G], wl[kHqWarps][G];
     __shared__ int sflag;
@@ -343,10 +360,42 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
         if (split == 0 && tid == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
         T = T < 0 ? 0 : p.max_pages * kPageTokens;
     }
-    const int tps = p.pages_per_split * kPageTokens;
-    const int n_act = max(1, (T + tps - 1) / tps);
+    const int n_pages = (T + kPageTokens - 1) / kPageTokens;
+    const int n_act = max(1, (n_pages + p.pages_per_split - 1) / p.pages_per_split);
     if (split >= n_act) return;
-    const int t_begin = split * tps, t_end = min(T, t_begin + tps);
+
+    // this warp's pages and its ring; the first copies go out first
+    const int p_begin = split * p.pages_per_split + warp * p.pages_per_warp;
+    const int npg = max(0, min(p_begin + p.pages_per_warp, n_pages) - p_begin);
+    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
+    const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
+    const uint32_t stage0 = smem_u32(smem + kHqOffStage) + warp * kHqStages * kHqChunk;
+    const unsigned char *stage0_ptr = smem + kHqOffStage + warp * kHqStages * kHqChunk;
+    const uint32_t bar0 = smem_u32(smem + kHqOffBar) + warp * kHqStages * 8;
+    if (lane == 0) {
+        for (int st = 0; st < kHqStages; st++) mbar_init(bar0 + 8 * st, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    uint32_t vbits = 0;  // bit st: stage st holds a valid page
+    auto issue = [&](int i) {  // every lane calls this
+        const int st = i % kHqStages;
+        int pg = 0;
+        if (lane == 0) {
+            pg = bt[p_begin + i];
+            if (pg < 0 || pg >= L.num_pages) {
+                set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
+                pg = -1;
+            }
+            if (pg >= 0)
+                bulk_load(stage0 + st * kHqChunk, kv_base + (long long)pg * L.page_bytes, kHqChunk, bar0 + 8 * st);
+            else
+                asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar0 + 8 * st) : "memory");
+        }
+        pg = __shfl_sync(kFull, pg, 0);
+        vbits = (vbits & ~(1u << st)) | ((pg >= 0 ? 1u : 0u) << st);
+    };
+    for (int i = 0; i < kHqStages && i < npg; i++) issue(i);
 
     {
         const float4 *S = reinterpret_cast<const float4 *>(p.pool + L.hq_tab) + (long long)kvh * 2 * kHqmqNS;
@@ -383,106 +432,100 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
 #pragma unroll
         for (int e = 0; e < 4; e++) acc[h][e] = 0.f;
     }
-    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
-    const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
     constexpr int NHG = G > 4 ? G / 4 : 1;
     const int uj = lane >> 2, hlj = lane & 3;
 
-    for (int tb = t_begin + warp * kHqTok; tb < t_end; tb += kHqWarps * kHqTok) {
-        // the batch's fields and meta rows, all loads issued before any math
-        // the batch's token rows (chunk offsets), fields and meta rows, all
-        // loads issued before any math; a batch never leaves its page
-        uint32_t kf[kHqTok], vf[kHqTok];
-        uint2 km[kHqTok], vm[kHqTok];
-        unsigned vmask = 0;
-        long long cofs = 0;  // the batch's chunk, from kv_base
-        {
-            const int pg = tb < t_end ? bt[tb / kPageTokens] : -1;
-            if (tb < t_end && (pg < 0 || pg >= L.num_pages)) {
-                if (lane == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
-            } else if (tb < t_end) {
-                cofs = (long long)pg * L.page_bytes;
-                vmask = (1u << min(kHqTok, t_end - tb)) - 1u;
-            }
+    for (int i = 0; i < npg; i++) {
+        const int st = i % kHqStages;
+        const bool ok = mbar_wait_bounded(bar0 + 8 * st, (i / kHqStages) & 1, kWaitLimitNs);
+        if (!__all_sync(kFull, ok)) {
+            // record it, then wait (bounded) for the copies still in flight
+            if (lane == 0) set_status(p.pool, KVQ_ERR_TIMEOUT);
+            for (int k = i; k < npg && k < i + kHqStages; k++)
+                (void)mbar_wait_bounded(bar0 + 8 * (k % kHqStages), (k / kHqStages) & 1, kWaitLimitNs);
+            break;
         }
-        const unsigned char *chunk = kv_base + cofs;
-        const int tok0 = tb % kPageTokens;
+        const unsigned char *chunk = stage0_ptr + st * kHqChunk;
+        const int t_page = (p_begin + i) * kPageTokens;
+        const int nvalid = ((vbits >> st) & 1u) ? min(kPageTokens, T - t_page) : 0;
+#pragma unroll 1
+        for (int half = 0; half < 2; half++) {
+            const int tok0 = half * kHqTok;
+            const unsigned vmask = (1u << max(0, min(kHqTok, nvalid - tok0))) - 1u;
+            if (vmask == 0) break;  // warp-uniform
+            // keys: per head group, rebuild each block and take the partial dots
+            // (one group of four heads rebuilds once), then totals and softmax
+            float pw[NHG];
 #pragma unroll
-        for (int u = 0; u < kHqTok; u++) {
-            kf[u] = vf[u] = 0u;
-            km[u] = vm[u] = make_uint2(0u, 0u);
-            if ((vmask >> u) & 1u) {
-                const int tok = tok0 + u;
-                kf[u] = hq_field(chunk + L.k_codes + tok * kHqRowCode, lane);
-                vf[u] = hq_field(chunk + L.v_codes + tok * kHqRowCode, lane);
-                km[u] = __ldg(reinterpret_cast<const uint2 *>(chunk + L.k_meta + tok * kHqmqRowMeta));
-                vm[u] = __ldg(reinterpret_cast<const uint2 *>(chunk + L.v_meta + tok * kHqmqRowMeta));
-            }
-        }
-        // keys: per head group, rebuild each block and take the partial dots
-        // (one group of four heads rebuilds once), then totals and softmax
-        float pw[NHG];
+            for (int hg = 0; hg < NHG; hg++) {
+                float d[32];
 #pragma unroll
-        for (int hg = 0; hg < NHG; hg++) {
-            float d[32];
-#pragma unroll
-            for (int u = 0; u < kHqTok; u++) {
-                float kc[4] = {0.f, 0.f, 0.f, 0.f};
-                if ((vmask >> u) & 1u)
-                    hq_block(kf[u], km[u], chunk + L.k_meta + (tok0 + u) * kHqmqRowMeta + 8, SK, lane, kc);
-#pragma unroll
-                for (int hl = 0; hl < 4; hl++) {
-                    const int h = hg * 4 + hl;
-                    float a = 0.f;
-                    if (h < G) {
-#pragma unroll
-                        for (int e = 0; e < 4; e++) a = fmaf(qr[h][e], kc[e], a);
+                for (int u = 0; u < kHqTok; u++) {
+                    float kc[4] = {0.f, 0.f, 0.f, 0.f};
+                    if ((vmask >> u) & 1u) {
+                        const int tok = tok0 + u;
+                        hq_block(hq_field(chunk + L.k_codes + tok * kHqRowCode, lane),
+                                 chunk + L.k_meta + tok * kHqmqRowMeta, SK, lane, kc);
                     }
-                    d[u * 4 + hl] = a;
+#pragma unroll
+                    for (int hl = 0; hl < 4; hl++) {
+                        const int h = hg * 4 + hl;
+                        float a = 0.f;
+                        if (h < G) {
+#pragma unroll
+                            for (int e = 0; e < 4; e++) a = fmaf(qr[h][e], kc[e], a);
+                        }
+                        d[u * 4 + hl] = a;
+                    }
+                }
+                float sc = cert::transpose_reduce32(d, lane);  // lane: token uj, head 4 hg + hlj
+                const bool live = ((vmask >> uj) & 1u) && hg * 4 + hlj < g;
+                if (!live) sc = -INFINITY;
+                float bmax = sc;
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
+                float mo = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 4; k++)
+                    if (hg * 4 + k < G && hlj == k) mo = m[hg * 4 + k];
+                const float mnew = fmaxf(mo, bmax);
+                const float pj = sc == -INFINITY ? 0.f : ex2(sc - mnew);
+                float psum = pj;
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) psum += __shfl_xor_sync(kFull, psum, o);
+                pw[hg] = pj;
+#pragma unroll
+                for (int k = 0; k < 4; k++) {  // lane k holds head 4 hg + k's figures
+                    const int h = hg * 4 + k;
+                    if (h >= G || h >= g) break;
+                    const float mn = __shfl_sync(kFull, mnew, k), ps = __shfl_sync(kFull, psum, k);
+                    const float al = m[h] == -INFINITY ? 0.f : ex2(m[h] - mn);
+                    l[h] = fmaf(l[h], al, ps);
+#pragma unroll
+                    for (int e = 0; e < 4; e++) acc[h][e] *= al;
+                    m[h] = mn;
                 }
             }
-            float sc = cert::transpose_reduce32(d, lane);  // lane: token uj, head 4 hg + hlj
-            const bool live = ((vmask >> uj) & 1u) && hg * 4 + hlj < g;
-            if (!live) sc = -INFINITY;
-            float bmax = sc;
+            // values: rebuild each token's block once, every head takes its weight
 #pragma unroll
-            for (int o = 4; o < 32; o <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
-            float mo = -INFINITY;
+            for (int u = 0; u < kHqTok; u++) {
+                if (!((vmask >> u) & 1u)) continue;  // warp-uniform
+                const int tok = tok0 + u;
+                float vc[4];
+                hq_block(hq_field(chunk + L.v_codes + tok * kHqRowCode, lane), chunk + L.v_meta + tok * kHqmqRowMeta,
+                         SV, lane, vc);
 #pragma unroll
-            for (int k = 0; k < 4; k++)
-                if (hg * 4 + k < G && hlj == k) mo = m[hg * 4 + k];
-            const float mnew = fmaxf(mo, bmax);
-            const float pj = sc == -INFINITY ? 0.f : ex2(sc - mnew);
-            float psum = pj;
+                for (int h = 0; h < G; h++) {
+                    if (h >= g) break;
+                    const float w = __shfl_sync(kFull, pw[h >> 2], u * 4 + (h & 3));
 #pragma unroll
-            for (int o = 4; o < 32; o <<= 1) psum += __shfl_xor_sync(kFull, psum, o);
-            pw[hg] = pj;
-#pragma unroll
-            for (int k = 0; k < 4; k++) {  // lane k holds head 4 hg + k's figures
-                const int h = hg * 4 + k;
-                if (h >= G || h >= g) break;
-                const float mn = __shfl_sync(kFull, mnew, k), ps = __shfl_sync(kFull, psum, k);
-                const float al = m[h] == -INFINITY ? 0.f : ex2(m[h] - mn);
-                l[h] = fmaf(l[h], al, ps);
-#pragma unroll
-                for (int e = 0; e < 4; e++) acc[h][e] *= al;
-                m[h] = mn;
+                    for (int e = 0; e < 4; e++) acc[h][e] = fmaf(w, vc[e], acc[h][e]);
+                }
             }
         }
-        // values: rebuild each token's block once, every head takes its weight
-#pragma unroll
-        for (int u = 0; u < kHqTok; u++) {
-            if (!((vmask >> u) & 1u)) continue;  // warp-uniform
-            float vc[4];
-            hq_block(vf[u], vm[u], chunk + L.v_meta + (tok0 + u) * kHqmqRowMeta + 8, SV, lane, vc);
-#pragma unroll
-            for (int h = 0; h < G; h++) {
-                if (h >= g) break;
-                const float w = __shfl_sync(kFull, pw[h >> 2], u * 4 + (h & 3));
-#pragma unroll
-                for (int e = 0; e < 4; e++) acc[h][e] = fmaf(w, vc[e], acc[h][e]);
-            }
-        }
+        // refill this stage (every lane is done reading it)
+        __syncwarp();
+        if (i + kHqStages < npg) issue(i + kHqStages);
     }
 
     // warps -> one partial per head: sums, then (max, sum of weights)
@@ -535,26 +578,35 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
     if (tid == 0) p.counters[bk] = 0u;
     const float *pb = p.part + bk * p.n_splits * (long long)g * REC;
     for (int h = warp; h < g; h += kHqWarps) {
-        float M = -INFINITY;
-        for (int c = lane; c < n_act; c += 32) M = fmaxf(M, __ldcg(pb + (c * g + h) * REC + kHqD));
+        // lane c: the weights of splits c and c + 32, then every split's row
+        // loaded before any is summed (one round trip)
+        float mc[2], lc[2];
+#pragma unroll
+        for (int k = 0; k < 2; k++) {
+            const int c = lane + 32 * k;
+            mc[k] = c < n_act ? __ldcg(pb + (c * g + h) * REC + kHqD) : -INFINITY;
+            lc[k] = c < n_act ? __ldcg(pb + (c * g + h) * REC + kHqD + 1) : 0.f;
+        }
+        float M = fmaxf(mc[0], mc[1]);
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-        float Ls = 0.f;
-        for (int c = lane; c < n_act; c += 32) {
-            const float mc = __ldcg(pb + (c * g + h) * REC + kHqD), lc = __ldcg(pb + (c * g + h) * REC + kHqD + 1);
-            if (mc != -INFINITY) Ls = fmaf(lc, ex2(mc - M), Ls);
+        float f[2], Ls = 0.f;
+#pragma unroll
+        for (int k = 0; k < 2; k++) {
+            f[k] = mc[k] == -INFINITY ? 0.f : ex2(mc[k] - M);
+            Ls = fmaf(lc[k], f[k], Ls);
         }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) Ls += __shfl_xor_sync(kFull, Ls, o);
         float o4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
         for (int c = 0; c < n_act; c++) {
-            const float mc = __ldcg(pb + (c * g + h) * REC + kHqD);
-            const float f = mc == -INFINITY ? 0.f : ex2(mc - M);
+            const float fc = __shfl_sync(kFull, c < 32 ? f[0] : f[1], c & 31);
             const float4 r = __ldcg(reinterpret_cast<const float4 *>(pb + (c * g + h) * REC + lane * 4));
-            o4[0] = fmaf(f, r.x, o4[0]);
-            o4[1] = fmaf(f, r.y, o4[1]);
-            o4[2] = fmaf(f, r.z, o4[2]);
-            o4[3] = fmaf(f, r.w, o4[3]);
+            o4[0] = fmaf(fc, r.x, o4[0]);
+            o4[1] = fmaf(fc, r.y, o4[1]);
+            o4[2] = fmaf(fc, r.z, o4[2]);
+            o4[3] = fmaf(fc, r.w, o4[3]);
         }
         if (p.rotate) {  // back to the original domain: diag(s) H c
             fwht_warp<kHqD>(o4, lane);
@@ -570,7 +622,15 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
 template <int G>
 cudaError_t launch_hq_decode_g(const DecodeParams &p, dim3 grid, cudaStream_t s)
 {
-    hqmq_decode_kernel<G><<<grid, kHqThreads, 0, s>>>(p);
+    static bool configured = false;
+    if (!configured) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(hqmq_decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHqSmem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    if (p.n_splits > kHqMaxSplits || p.L.chunk_bytes != kHqChunk) return cudaErrorInvalidValue;
+    hqmq_decode_kernel<G><<<grid, kHqThreads, kHqSmem, s>>>(p);
     return cudaGetLastError();
 }
 
