@@ -301,10 +301,13 @@ __device__ __forceinline__ uint32_t hq_field(const unsigned char *row, int lane)
 }
 
 // Block `lane` of a row: (radius code x step) x q_p q_s with q_s from the
-// codebook in shared memory, or the fp16 outlier values.  meta = the row's
-// meta (shared memory): step | 0, outlier mask, two outlier slots.
-__device__ __forceinline__ void hq_block(uint32_t f, const unsigned char *meta, const float4 *S, int lane,
-                                         float (&c)[4])
+// codebook and q_p from the unit table (both in shared memory), or the fp16
+// outlier values.  meta = the row's meta (shared memory): step | 0, outlier
+// mask, two outlier slots.  The unit table holds 8 copies of the 24 units,
+// copy r of unit p at p * 8 + r: lane reads copy lane % 8, so the eight
+// lanes of each 16-byte load phase hit eight different bank groups.
+__device__ __forceinline__ void hq_block(uint32_t f, const unsigned char *meta, const float4 *S, const float4 *units,
+                                         int lane, float (&c)[4])
 {
     const uint2 mm = *reinterpret_cast<const uint2 *>(meta);
     if ((mm.y >> lane) & 1u) {
@@ -320,17 +323,8 @@ __device__ __forceinline__ void hq_block(uint32_t f, const unsigned char *meta, 
     const uint32_t idx = f & 0x7FFFu, sq = idx / 24u, pp = idx - 24u * sq;
     const float4 q = S[min(sq, (uint32_t)kHqmqNS - 1u)];
     const float rad = (float)(f >> 15) * __half2float(__ushort_as_half((unsigned short)(mm.x & 0xFFFFu)));
-    // q_p x rad: an axis unit (+-1 on component pp/2) or a half unit (+-1/2,
-    // bit i of pp - 8 = the sign of component i), built from bit patterns
-    const bool half = pp >= 8u;
-    const uint32_t hb = __float_as_uint(0.5f * rad), ab = __float_as_uint(rad);
-    float a[4];
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        const uint32_t hv = hb | ((((pp - 8u) >> i) & 1u) << 31);
-        const uint32_t av = (pp >> 1) == (uint32_t)i ? (ab | ((pp & 1u) << 31)) : 0u;
-        a[i] = __uint_as_float(half ? hv : av);
-    }
+    const float4 qp = units[min(pp, 23u) * 8 + (lane & 7)];
+    const float a[4] = {qp.x * rad, qp.y * rad, qp.z * rad, qp.w * rad};
     c[0] = a[0] * q.x - a[1] * q.y - a[2] * q.z - a[3] * q.w;
     c[1] = a[0] * q.y + a[1] * q.x + a[2] * q.w - a[3] * q.z;
     c[2] = a[0] * q.z - a[1] * q.w + a[2] * q.x + a[3] * q.y;
@@ -352,6 +346,7 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
     extern __shared__ __align__(128) unsigned char smem[];
     float4 *tab = reinterpret_cast<float4 *>(smem);  // K then V codebook; the warps' sums after the loop
     __shared__ __align__(16) float sq[G * kHqD];
+    __shared__ __align__(16) float4 units[24 * 8];
     __shared__ float wm[kHqWarps][G], wl[kHqWarps][G];
     __shared__ int sflag;
 
@@ -400,6 +395,16 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
     {
         const float4 *S = reinterpret_cast<const float4 *>(p.pool + L.hq_tab) + (long long)kvh * 2 * kHqmqNS;
         for (int i = tid; i < 2 * kHqmqNS; i += kHqThreads) tab[i] = __ldg(S + i);
+        // the 24 unit Hurwitz quaternions: p < 8 are +-1, +-i, +-j, +-k; p >= 8
+        // are (+-1 +-i +-j +-k)/2 with component c negative iff bit c of p - 8
+        if (tid < 24 * 8) {
+            const int pu = tid >> 3;
+            float u4[4];
+#pragma unroll
+            for (int c = 0; c < 4; c++)
+                u4[c] = pu < 8 ? (pu / 2 == c ? ((pu & 1) ? -1.f : 1.f) : 0.f) : ((((pu - 8) >> c) & 1) ? -0.5f : 0.5f);
+            units[tid] = make_float4(u4[0], u4[1], u4[2], u4[3]);
+        }
     }
     if (warp < g) {  // the rotated query in log2 units
         const __half *qh = p.q + ((long long)b * L.hq + kvh * g + warp) * kHqD + lane * 4;
@@ -465,7 +470,7 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
                     if ((vmask >> u) & 1u) {
                         const int tok = tok0 + u;
                         hq_block(hq_field(chunk + L.k_codes + tok * kHqRowCode, lane),
-                                 chunk + L.k_meta + tok * kHqmqRowMeta, SK, lane, kc);
+                                 chunk + L.k_meta + tok * kHqmqRowMeta, SK, units, lane, kc);
                     }
 #pragma unroll
                     for (int hl = 0; hl < 4; hl++) {
@@ -513,7 +518,7 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
                 const int tok = tok0 + u;
                 float vc[4];
                 hq_block(hq_field(chunk + L.v_codes + tok * kHqRowCode, lane), chunk + L.v_meta + tok * kHqmqRowMeta,
-                         SV, lane, vc);
+                         SV, units, lane, vc);
 #pragma unroll
                 for (int h = 0; h < G; h++) {
                     if (h >= g) break;
