@@ -87,8 +87,10 @@ typedef enum {
  *     two blocks with r_b > tau, largest first (lower block on ties); step =
  *     fp16 rounded up of tau / 31; radius code = min(31, rint(r_b / step)) (0
  *     when step = 0); direction u = x / r_b; for each s in order, w = u
- *     conj(q_s) (Hamilton product, each component's four products summed
- *     left to right) scores max_i |w_i| (first i, sign of w_i) or, when
+ *     conj(q_s) (Hamilton product; each component is its first product,
+ *     rounded, then the other three added in order by fused multiply-adds,
+ *     a subtracted product as one with its first factor negated) scores
+ *     max_i |w_i| (first i, sign of w_i) or, when
  *     strictly larger, (((|w0| + |w1|) + |w2|) + |w3|) / 2 (signs of w); the
  *     first s of highest score wins; index = 24 s + p (0 when r_b = 0);
  *   storage: a token's code row is d/4 fields of 20 bits (index | radius code

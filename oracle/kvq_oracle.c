@@ -404,14 +404,16 @@ void kvqo_hqmq_unit(int p, float q[4])
     }
 }
 
-/* Hamilton product r = a b, each component's products rounded and summed
- * left to right in fp32 (the order the kernels use). */
+/* Hamilton product r = a b in fp32 as fused multiply-add chains: each
+ * component starts from its first product (rounded) and adds the other three
+ * products in order, each with one rounding (fmaf); a subtracted product is
+ * added with its first factor negated. */
 static void qmul_f32(const float a[4], const float b[4], float r[4])
 {
-    r[0] = a[0] * b[0] - a[1] * b[1] - a[2] * b[2] - a[3] * b[3];
-    r[1] = a[0] * b[1] + a[1] * b[0] + a[2] * b[3] - a[3] * b[2];
-    r[2] = a[0] * b[2] - a[1] * b[3] + a[2] * b[0] + a[3] * b[1];
-    r[3] = a[0] * b[3] + a[1] * b[2] - a[2] * b[1] + a[3] * b[0];
+    r[0] = fmaf(-a[3], b[3], fmaf(-a[2], b[2], fmaf(-a[1], b[1], a[0] * b[0])));
+    r[1] = fmaf(-a[3], b[2], fmaf(a[2], b[3], fmaf(a[1], b[0], a[0] * b[1])));
+    r[2] = fmaf(a[3], b[1], fmaf(a[2], b[0], fmaf(-a[1], b[3], a[0] * b[2])));
+    r[3] = fmaf(a[3], b[0], fmaf(-a[2], b[1], fmaf(a[1], b[2], a[0] * b[3])));
 }
 
 /* Secondary codebook S of (kv head, tensor): NS unit quaternions drawn

@@ -45,29 +45,16 @@ constexpr unsigned kHqFieldMask = 0xFFFFFu;
 
 // ------------------------------------------------------------------ append --
 
-// Score of unit direction u against codeword conj(q_s) = c, exactly as kvq.h
-// states: w = u c (Hamilton product, products summed left to right), the
-// best axis unit max_i |w_i| or the best half unit (sum |w_i|) / 2.
+// w = u c for unit direction u and codeword conj(q_s) = c, exactly as kvq.h
+// states: each component is its first product, rounded, then the other three
+// products added in order by fused multiply-adds (a subtracted product as
+// one with its first factor negated).
 __device__ __forceinline__ void hamilton_rn(const float (&u)[4], float4 c, float (&w)[4])
 {
-    w[0] = __fsub_rn(__fsub_rn(__fsub_rn(__fmul_rn(u[0], c.x), __fmul_rn(u[1], c.y)), __fmul_rn(u[2], c.z)),
-                     __fmul_rn(u[3], c.w));
-    w[1] = __fsub_rn(__fadd_rn(__fadd_rn(__fmul_rn(u[0], c.y), __fmul_rn(u[1], c.x)), __fmul_rn(u[2], c.w)),
-                     __fmul_rn(u[3], c.z));
-    w[2] = __fadd_rn(__fadd_rn(__fsub_rn(__fmul_rn(u[0], c.z), __fmul_rn(u[1], c.w)), __fmul_rn(u[2], c.x)),
-                     __fmul_rn(u[3], c.y));
-    w[3] = __fadd_rn(__fsub_rn(__fadd_rn(__fmul_rn(u[0], c.w), __fmul_rn(u[1], c.z)), __fmul_rn(u[2], c.y)),
-                     __fmul_rn(u[3], c.x));
-}
-
-__device__ __forceinline__ float score_only(const float (&u)[4], float4 c)
-{
-    float w[4];
-    hamilton_rn(u, c, w);
-    const float a0 = fabsf(w[0]), a1 = fabsf(w[1]), a2 = fabsf(w[2]), a3 = fabsf(w[3]);
-    const float ma = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
-    const float mh = __fmul_rn(__fadd_rn(__fadd_rn(__fadd_rn(a0, a1), a2), a3), 0.5f);
-    return mh > ma ? mh : ma;
+    w[0] = __fmaf_rn(-u[3], c.w, __fmaf_rn(-u[2], c.z, __fmaf_rn(-u[1], c.y, __fmul_rn(u[0], c.x))));
+    w[1] = __fmaf_rn(-u[3], c.z, __fmaf_rn(u[2], c.w, __fmaf_rn(u[1], c.x, __fmul_rn(u[0], c.y))));
+    w[2] = __fmaf_rn(u[3], c.y, __fmaf_rn(u[2], c.x, __fmaf_rn(-u[1], c.w, __fmul_rn(u[0], c.z))));
+    w[3] = __fmaf_rn(u[3], c.x, __fmaf_rn(-u[2], c.y, __fmaf_rn(u[1], c.z, __fmul_rn(u[0], c.w))));
 }
 
 __device__ __forceinline__ int unit_of(const float (&u)[4], float4 c)
@@ -163,20 +150,82 @@ __device__ __forceinline__ void hq_prepare(const AppendParams &p, const __half *
     for (int e = 0; e < 4; e++) R.u[e] = r > 0.0f ? __fdiv_rn(x[e], r) : 0.0f;
 }
 
-// Best candidate of s in [s0, s1): strictly higher score wins, so the first
-// of equal scores stays.
-__device__ __forceinline__ void hq_search(const float (&u)[4], const float4 *cb, int s0, int s1, float &best, int &bs)
+// Best candidate of s in [s0, s1) (s0, s1 even): strictly higher score
+// wins, so the first of equal scores stays.  Two candidates per step with
+// packed f32x2 products and fused multiply-adds (four products and twelve
+// multiply-adds per pair instead of 28 scalar operations per candidate).
+// Table entries 2j, 2j + 1 hold candidates 2j and 2j + 1 interleaved:
+// (c0(2j), c0(2j+1), c1(2j), c1(2j+1)), (c2(2j), c2(2j+1), c3(2j), c3(2j+1)).
+__device__ __forceinline__ float pair_score(float2 w0, float2 w1, float2 w2, float2 w3, bool hi)
 {
+    const float a0 = fabsf(hi ? w0.y : w0.x), a1 = fabsf(hi ? w1.y : w1.x), a2 = fabsf(hi ? w2.y : w2.x),
+                a3 = fabsf(hi ? w3.y : w3.x);
+    const float ma = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+    const float mh = __fmul_rn(__fadd_rn(__fadd_rn(__fadd_rn(a0, a1), a2), a3), 0.5f);
+    return mh > ma ? mh : ma;
+}
+
+// Packed f32x2 multiply and fused multiply-add (each lane rounds as the
+// scalar operation does).
+__device__ __forceinline__ unsigned long long pk(float2 v)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+    return r;
+}
+__device__ __forceinline__ float2 upk(unsigned long long r)
+{
+    float2 v;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+    return v;
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b)
+{
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ void hq_search(const float (&u)[4], const float4 *cb2, int s0, int s1, float &best, int &bs)
+{
+    const unsigned long long U0 = pk(make_float2(u[0], u[0])), U1 = pk(make_float2(u[1], u[1])),
+                             U2 = pk(make_float2(u[2], u[2])), U3 = pk(make_float2(u[3], u[3]));
+    const unsigned long long N1 = pk(make_float2(-u[1], -u[1])), N2 = pk(make_float2(-u[2], -u[2])),
+                             N3 = pk(make_float2(-u[3], -u[3]));
     best = -INFINITY;
     bs = s0;
-#pragma unroll 4
-    for (int s = s0; s < s1; s++) {
-        const float sc = score_only(u, cb[s]);
-        if (sc > best) {
-            best = sc;
+#pragma unroll 2
+    for (int s = s0; s < s1; s += 2) {
+        const float4 a = cb2[s], b = cb2[s + 1];  // (pair s/2 occupies entries s and s + 1)
+        const unsigned long long C0 = pk(make_float2(a.x, a.y)), C1 = pk(make_float2(a.z, a.w)),
+                                 C2 = pk(make_float2(b.x, b.y)), C3 = pk(make_float2(b.z, b.w));
+        const float2 w0 = upk(fma2(N3, C3, fma2(N2, C2, fma2(N1, C1, mul2(U0, C0)))));
+        const float2 w1 = upk(fma2(N3, C2, fma2(U2, C3, fma2(U1, C0, mul2(U0, C1)))));
+        const float2 w2 = upk(fma2(U3, C1, fma2(U2, C0, fma2(N1, C3, mul2(U0, C2)))));
+        const float2 w3 = upk(fma2(U3, C0, fma2(N2, C1, fma2(U1, C2, mul2(U0, C3)))));
+        const float sa = pair_score(w0, w1, w2, w3, false), sb = pair_score(w0, w1, w2, w3, true);
+        if (sa > best) {
+            best = sa;
             bs = s;
         }
+        if (sb > best) {
+            best = sb;
+            bs = s + 1;
+        }
     }
+}
+
+// Candidate s of the interleaved table as conj(q_s).
+__device__ __forceinline__ float4 cand(const float4 *cb2, int s)
+{
+    const float4 a = cb2[s & ~1], b = cb2[s | 1];
+    return (s & 1) ? make_float4(a.y, a.w, b.y, b.w) : make_float4(a.x, a.z, b.x, b.z);
 }
 
 // Pack and store a coded row: fields as one little-endian 20-bit stream
@@ -211,16 +260,17 @@ __global__ void __launch_bounds__(kHqThreads) hqmq_append_kernel(const __grid_co
 {
     constexpr int RPC = kHqWarps / WPR;  // rows per CTA pass
     constexpr int SPAN = kHqmqNS / WPR;  // candidates per warp
-    __shared__ float4 cb[kHqmqNS];
+    __shared__ float4 cb2[kHqmqNS];  // conj(S), candidates interleaved in pairs (see hq_search)
     __shared__ float wsc[WPR > 1 ? 2 : 1][kHqWarps][32];
     __shared__ int wsi[WPR > 1 ? 2 : 1][kHqWarps][32];
     const int pair = blockIdx.y, kvh = pair >> 1, tensor = pair & 1;
     const Layout &L = p.L;
     {
         const float4 *S = reinterpret_cast<const float4 *>(p.pool + L.hq_tab) + (long long)pair * kHqmqNS;
-        for (int i = threadIdx.x; i < kHqmqNS; i += kHqThreads) {
-            const float4 s = S[i];
-            cb[i] = make_float4(s.x, -s.y, -s.z, -s.w);  // exact sign flips
+        for (int j = threadIdx.x; j < kHqmqNS / 2; j += kHqThreads) {
+            const float4 a = S[2 * j], b = S[2 * j + 1];  // conj: exact sign flips
+            cb2[2 * j] = make_float4(a.x, b.x, -a.y, -b.y);
+            cb2[2 * j + 1] = make_float4(-a.z, -b.z, -a.w, -b.w);
         }
     }
     __syncthreads();
@@ -243,7 +293,7 @@ __global__ void __launch_bounds__(kHqThreads) hqmq_append_kernel(const __grid_co
         if (active) {  // warp-uniform
             const __half *src = (tensor ? p.v : p.k) + ((long long)n * L.hkv + kvh) * kHqD;
             hq_prepare(p, src, lane, R);
-            hq_search(R.u, cb, slice * SPAN, slice * SPAN + SPAN, best, bs);
+            hq_search(R.u, cb2, slice * SPAN, slice * SPAN + SPAN, best, bs);
         }
         if constexpr (WPR > 1) {
             wsc[par][warp][lane] = best;
@@ -264,7 +314,7 @@ __global__ void __launch_bounds__(kHqThreads) hqmq_append_kernel(const __grid_co
             const bool outl = (R.mask >> lane) & 1u;
             uint32_t field = 0;
             if (!outl) {
-                const uint32_t idx = R.r > 0.0f ? (uint32_t)(24 * bs + unit_of(R.u, cb[bs])) : 0u;
+                const uint32_t idx = R.r > 0.0f ? (uint32_t)(24 * bs + unit_of(R.u, cand(cb2, bs))) : 0u;
                 field = idx | (R.rc << 15);
             }
             const int page = slot / kPageTokens, tok = slot % kPageTokens;
