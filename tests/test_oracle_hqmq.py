@@ -130,3 +130,42 @@ def test_pool_round_trip_and_reconstruction():
     # relative reconstruction error of the whole cache is small (~5 bits per element)
     yk = yrot[:, :, 0].reshape(40, -1)
     assert np.linalg.norm(yk - kd.reshape(40, -1)) / np.linalg.norm(yk) < 0.15
+
+
+def test_tie_rules_of_the_codeword_choice():
+    """Exact ties, built with a codebook of identical entries: the first s
+    wins; an axis unit wins a tie against a half unit; the first component
+    wins among equal |w_i|."""
+    S = np.tile(np.array([1.0, 0.0, 0.0, 0.0], np.float32), (O.HQMQ_NS, 1))
+    h = np.float32(1.0) / np.sqrt(np.float32(2.0))
+    u = np.array([[h, h, 0, 0],        # max |w_i| = half-sum exactly: axis unit p = 0
+                  [0, -h, h, 0],       # axis -i (p = 3) beats +j on the component tie
+                  [0.5, -0.5, 0.5, 0.5],  # a half unit exactly: p = 8 + 2 = 10
+                  [0, 0, 0, -1]], np.float32)  # -k: p = 7
+    idx = O.hqmq_encode_dirs(u, S)
+    assert idx.tolist() == [0, 3, 10, 7]  # every s ties: s = 0
+
+
+def test_tie_rules_of_med3x():
+    """A block exactly at tau = 3 x median is not an outlier (strictly
+    greater); among equal radii above tau the lowest blocks are kept."""
+    y = np.zeros((1, 128), np.float32)
+    y[0, 0::4] = 1.0                   # every block radius 1: median 1, tau 3
+    y[0, 4 * 2] = 3.0                  # exactly tau: coded, not kept
+    for b in (5, 9, 20):
+        y[0, 4 * b] = 5.0              # three equal radii above tau: blocks 5, 9 kept
+    S = O.hqmq_codebook(1, 0, 0)
+    field, step, mask, outl = O.hqmq_quantize_rows(y, S)
+    assert int(mask[0]) == (1 << 5) | (1 << 9)
+    assert np.all(np.asarray(outl[0]).view(np.float16).astype(np.float32)[:, 0] == 5.0)
+    st = float(np.array(step[0], np.uint16).view(np.float16))
+    q = np.float32(3.0) / np.float32(31.0)       # the step: fp16 rounded up of tau / 31
+    up = np.float16(q) if float(np.float16(q)) >= q else np.nextafter(np.float16(q), np.float16(np.inf))
+    assert st == float(up)
+    assert (int(field[0, 20]) >> 15) == 31   # the third one: clipped radius
+    assert (int(field[0, 2]) >> 15) == int(np.rint(3.0 / st))
+    # one block above tau and one exactly at it: only the first is kept
+    y2 = np.zeros((1, 128), np.float32)
+    y2[0, 0::4] = 1.0
+    y2[0, 4 * 2], y2[0, 4 * 7] = 3.0, 5.0
+    assert int(O.hqmq_quantize_rows(y2, S)[2][0]) == 1 << 7
