@@ -39,8 +39,8 @@ NOMINAL_HBM_GBS = 8000.0
 # capture summarised under profiles/ (decode_kernel_llama3-8b-layer-T32768.md).
 # Reported as roofline.traffic only while the decode kernel's sources hash to
 # the digest they had when the counters were taken; null otherwise.
-PROFILED_DECODE = {"sources_sha256": "473c0c7612212fb4025186ee5fc5a2d1c1bd87c9da5b2832a5836b9cf77575d1",
-                   "dram_bytes_per_launch": 42148224}
+PROFILED_DECODE = {"sources_sha256": "4f2686c25844259234cdd81d4fac3484f962ce661750f6a10d1b6afab05f5edb",
+                   "dram_bytes_per_launch": 42147456}
 DECODE_SOURCES = ("kvq_decode.cu", "kvq_internal.cuh", "kvq_warp.cuh")
 
 
