@@ -360,16 +360,6 @@ __device__ __forceinline__ void hq_block(uint32_t f, const unsigned char *meta, 
                                          int lane, float (&c)[4])
 {
     const uint2 mm = *reinterpret_cast<const uint2 *>(meta);
-    if ((mm.y >> lane) & 1u) {
-        const int slot = min(__popc(mm.y & ((1u << lane) - 1u)), kHqmqOut - 1);
-        const uint2 raw = reinterpret_cast<const uint2 *>(meta + 8)[slot];
-        const float2 a = __half22float2(bits_h2(raw.x)), b = __half22float2(bits_h2(raw.y));
-        c[0] = a.x;
-        c[1] = a.y;
-        c[2] = b.x;
-        c[3] = b.y;
-        return;
-    }
     const uint32_t idx = f & 0x7FFFu, sq = idx / 24u, pp = idx - 24u * sq;
     const float4 q = S[min(sq, (uint32_t)kHqmqNS - 1u)];
     const float rad = (float)(f >> 15) * __half2float(__ushort_as_half((unsigned short)(mm.x & 0xFFFFu)));
@@ -379,6 +369,16 @@ __device__ __forceinline__ void hq_block(uint32_t f, const unsigned char *meta, 
     c[1] = a[0] * q.y + a[1] * q.x + a[2] * q.w - a[3] * q.z;
     c[2] = a[0] * q.z - a[1] * q.w + a[2] * q.x + a[3] * q.y;
     c[3] = a[0] * q.w + a[1] * q.z - a[2] * q.y + a[3] * q.x;
+    if (mm.y != 0u) {  // the row has outliers (uniform across the warp): select, no divergent branch
+        const int slot = min(__popc(mm.y & ((1u << lane) - 1u)), kHqmqOut - 1);
+        const uint2 raw = reinterpret_cast<const uint2 *>(meta + 8)[slot];
+        const float2 lo = __half22float2(bits_h2(raw.x)), hi = __half22float2(bits_h2(raw.y));
+        const bool mine = (mm.y >> lane) & 1u;
+        c[0] = mine ? lo.x : c[0];
+        c[1] = mine ? lo.y : c[1];
+        c[2] = mine ? hi.x : c[2];
+        c[3] = mine ? hi.y : c[3];
+    }
 }
 
 // Grid (splits, Hkv, B); split `blockIdx.x` attends pages [x * pps, +pps) of
