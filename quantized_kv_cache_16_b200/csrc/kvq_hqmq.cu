@@ -18,15 +18,19 @@
 // over the CTA's 8 warps and the per-block winners combined (highest score,
 // lowest candidate on ties, which is the sequential rule).
 //
-// Decode.  CTAs take contiguous token ranges of one (sequence, kv head) and
-// hold that head's two codebooks in shared memory (32 KB); a warp decodes 8
-// tokens at a time, lane b rebuilding block b of K and V as (radius code x
-// step) x q_p q_s (or the fp16 outlier), then partial dot products for 8
-// tokens x 4 heads reduce in one transpose-reduce and the online softmax
-// runs per head.  Split partials merge in the last CTA of each (sequence, kv
-// head), which also applies the inverse rotation.  The path is bound by the
-// fp32 pipe (about 80 operations a block per token for K and V together),
-// not by HBM: 208 bytes a token-head against ~2.5 K operations.
+// Decode.  CTAs take contiguous page ranges of one (sequence, kv head) and
+// hold that head's two codebooks in shared memory (32 KB); each warp streams
+// whole 16-token pages into a shared-memory ring by bulk copy.  Lanes rebuild
+// K and V blocks as (radius code x step) x q_p q_s (or the fp16 outlier)
+// straight into fp16 tensor-core fragments (K, V, the query and the weights
+// as hi + lo fp16 pairs, ~22 bits each): scores as K Q^T and the output as V^T P^T
+// (m16n8k16, M = tokens or dims, N = 8 heads), with the block-to-
+// fragment assignment chosen (a permutation of the contraction index and of
+// the output rows) so that every lane rebuilds whole blocks and the score
+// fragments become P^T by two 8x8 transposes.  Split partials merge in the
+// last CTA of each (sequence, kv head), which also applies the inverse
+// rotation.  Rebuilding blocks (lookups and a 16-term quaternion product)
+// dominates: the path is bound by instruction issue, not by HBM.
 #include <math.h>
 
 #include "kvq_cert.cuh"
@@ -340,11 +344,11 @@ constexpr int kHqSmem = kHqOffBar + kHqWarps * kHqStages * 8;
 static_assert(kHqChunk % 16 == 0 && kHqOffStage % 16 == 0 && kHqOffBar % 8 == 0, "bulk copy alignment");
 constexpr int kHqMaxSplits = 64;  // the merge holds one weight per split in registers (two per lane)
 
-// The 20-bit field of block `lane` in a token's code row (shared memory).
-__device__ __forceinline__ uint32_t hq_field(const unsigned char *row, int lane)
+// The 20-bit field of block `blk` in a token's code row (shared memory).
+__device__ __forceinline__ uint32_t hq_field(const unsigned char *row, int blk)
 {
     const uint32_t *w = reinterpret_cast<const uint32_t *>(row);
-    const int bit = 20 * lane, w0 = bit >> 5, sh = bit & 31;
+    const int bit = 20 * blk, w0 = bit >> 5, sh = bit & 31;
     const uint32_t lo = w[w0];
     const uint32_t hi = sh > 12 ? w[w0 + 1] : 0u;  // word 20 is never needed
     return __funnelshift_r(lo, hi, sh) & kHqFieldMask;
@@ -357,28 +361,38 @@ __device__ __forceinline__ uint32_t hq_field(const unsigned char *row, int lane)
 // copy r of unit p at p * 8 + r: lane reads copy lane % 8, so the eight
 // lanes of each 16-byte load phase hit eight different bank groups.
 __device__ __forceinline__ void hq_block(uint32_t f, const unsigned char *meta, const float4 *S, const float4 *units,
-                                         int lane, float (&c)[4])
+                                         int blk, int cpy, float (&c)[4])
 {
     const uint2 mm = *reinterpret_cast<const uint2 *>(meta);
     const uint32_t idx = f & 0x7FFFu, sq = idx / 24u, pp = idx - 24u * sq;
     const float4 q = S[min(sq, (uint32_t)kHqmqNS - 1u)];
     const float rad = (float)(f >> 15) * __half2float(__ushort_as_half((unsigned short)(mm.x & 0xFFFFu)));
-    const float4 qp = units[min(pp, 23u) * 8 + (lane & 7)];
+    const float4 qp = units[min(pp, 23u) * 8 + cpy];
     const float a[4] = {qp.x * rad, qp.y * rad, qp.z * rad, qp.w * rad};
     c[0] = a[0] * q.x - a[1] * q.y - a[2] * q.z - a[3] * q.w;
     c[1] = a[0] * q.y + a[1] * q.x + a[2] * q.w - a[3] * q.z;
     c[2] = a[0] * q.z - a[1] * q.w + a[2] * q.x + a[3] * q.y;
     c[3] = a[0] * q.w + a[1] * q.z - a[2] * q.y + a[3] * q.x;
     if (mm.y != 0u) {  // the row has outliers (uniform across the warp): select, no divergent branch
-        const int slot = min(__popc(mm.y & ((1u << lane) - 1u)), kHqmqOut - 1);
+        const int slot = min(__popc(mm.y & ((1u << blk) - 1u)), kHqmqOut - 1);
         const uint2 raw = reinterpret_cast<const uint2 *>(meta + 8)[slot];
         const float2 lo = __half22float2(bits_h2(raw.x)), hi = __half22float2(bits_h2(raw.y));
-        const bool mine = (mm.y >> lane) & 1u;
+        const bool mine = (mm.y >> blk) & 1u;
         c[0] = mine ? lo.x : c[0];
         c[1] = mine ? lo.y : c[1];
         c[2] = mine ? hi.x : c[2];
         c[3] = mine ? hi.y : c[3];
     }
+}
+
+// A float pair as two fp16 pairs, hi = fp16(x) and lo = fp16(x - hi): the
+// tensor-core products keep ~22 bits of each operand.
+__device__ __forceinline__ void split_h2(float x0, float x1, uint32_t &hi, uint32_t &lo)
+{
+    const __half2 h = __floats2half2_rn(x0, x1);
+    const float2 b = __half22float2(h);
+    hi = h2_bits(h);
+    lo = h2_bits(__floats2half2_rn(x0 - b.x, x1 - b.y));
 }
 
 // Grid (splits, Hkv, B); split `blockIdx.x` attends pages [x * pps, +pps) of
@@ -473,22 +487,31 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
     }
     __syncthreads();
     const float4 *SK = tab, *SV = tab + kHqmqNS;
-    float qr[G][4];
+    // Fragment roles (mma m16n8k16, fp16 in, fp32 out; r = lane / 4, j = lane % 4):
+    //   scores S^T [16 tokens x 8 heads] = K [16 x 128] Q^T: k-slice ks holds
+    //     blocks 4 ks .. 4 ks + 3, slice position {2j, 2j+1, 2j+8, 2j+9} = dims
+    //     0..3 of block 4 ks + j, so lane rebuilds block 4 ks + j of tokens r
+    //     and r + 8 and holds the query's block 4 ks + j of head r;
+    //   the scores land as tokens r, r + 8 x heads 2j, 2j + 1;
+    //   O^T [128 dims x 8 heads] += V^T [128 x 16 tokens] P^T: m-tiles 2i and
+    //     2i + 1 hold, in rows r / r + 8, dims 0 / 1 and 2 / 3 of block 8i + r,
+    //     so lane rebuilds block 8i + r of tokens 2j, 2j+1, 2j+8, 2j+9; P^T
+    //     comes from the score fragments by two 8x8 transposes (movmatrix).
+    const int r = lane >> 2, j = lane & 3, cpy = lane & 7;
+    uint32_t qb[8][2], ql[8][2];  // the query's hi and lo fp16 parts
 #pragma unroll
-    for (int h = 0; h < G; h++)
-#pragma unroll
-        for (int e = 0; e < 4; e++) qr[h][e] = h < g ? sq[h * kHqD + lane * 4 + e] : 0.f;
-
-    float m[G], l[G], acc[G][4];
-#pragma unroll
-    for (int h = 0; h < G; h++) {
-        m[h] = -INFINITY;
-        l[h] = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; e++) acc[h][e] = 0.f;
+    for (int ks = 0; ks < 8; ks++) {
+        qb[ks][0] = qb[ks][1] = ql[ks][0] = ql[ks][1] = 0u;
+        if (r < g) {  // (sq holds g heads)
+            const float4 q4 = *reinterpret_cast<const float4 *>(sq + r * kHqD + 4 * (4 * ks + j));
+            split_h2(q4.x, q4.y, qb[ks][0], ql[ks][0]);
+            split_h2(q4.z, q4.w, qb[ks][1], ql[ks][1]);
+        }
     }
-    constexpr int NHG = G > 4 ? G / 4 : 1;
-    const int uj = lane >> 2, hlj = lane & 3;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2j, 2j + 1
+    float acc[8][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; mt++) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
 
     for (int i = 0; i < npg; i++) {
         const int st = i % kHqStages;
@@ -503,78 +526,98 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
         const unsigned char *chunk = stage0_ptr + st * kHqChunk;
         const int t_page = (p_begin + i) * kPageTokens;
         const int nvalid = ((vbits >> st) & 1u) ? min(kPageTokens, T - t_page) : 0;
-#pragma unroll 1
-        for (int half = 0; half < 2; half++) {
-            const int tok0 = half * kHqTok;
-            const unsigned vmask = (1u << max(0, min(kHqTok, nvalid - tok0))) - 1u;
-            if (vmask == 0) break;  // warp-uniform
-            // keys: per head group, rebuild each block and take the partial dots
-            // (one group of four heads rebuilds once), then totals and softmax
-            float pw[NHG];
+
+        // ---- scores of tokens r, r + 8 for heads 2j, 2j + 1 ----
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            const bool va = r < nvalid, vb = r + 8 < nvalid;
+            const unsigned char *ra = chunk + L.k_codes + r * kHqRowCode, *rb = ra + 8 * kHqRowCode;
+            const unsigned char *ma = chunk + L.k_meta + r * kHqmqRowMeta, *mb = ma + 8 * kHqmqRowMeta;
 #pragma unroll
-            for (int hg = 0; hg < NHG; hg++) {
-                float d[32];
-#pragma unroll
-                for (int u = 0; u < kHqTok; u++) {
-                    float kc[4] = {0.f, 0.f, 0.f, 0.f};
-                    if ((vmask >> u) & 1u) {
-                        const int tok = tok0 + u;
-                        hq_block(hq_field(chunk + L.k_codes + tok * kHqRowCode, lane),
-                                 chunk + L.k_meta + tok * kHqmqRowMeta, SK, units, lane, kc);
-                    }
-#pragma unroll
-                    for (int hl = 0; hl < 4; hl++) {
-                        const int h = hg * 4 + hl;
-                        float a = 0.f;
-                        if (h < G) {
-#pragma unroll
-                            for (int e = 0; e < 4; e++) a = fmaf(qr[h][e], kc[e], a);
-                        }
-                        d[u * 4 + hl] = a;
-                    }
-                }
-                float sc = cert::transpose_reduce32(d, lane);  // lane: token uj, head 4 hg + hlj
-                const bool live = ((vmask >> uj) & 1u) && hg * 4 + hlj < g;
-                if (!live) sc = -INFINITY;
-                float bmax = sc;
-#pragma unroll
-                for (int o = 4; o < 32; o <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
-                float mo = -INFINITY;
-#pragma unroll
-                for (int k = 0; k < 4; k++)
-                    if (hg * 4 + k < G && hlj == k) mo = m[hg * 4 + k];
-                const float mnew = fmaxf(mo, bmax);
-                const float pj = sc == -INFINITY ? 0.f : ex2(sc - mnew);
-                float psum = pj;
-#pragma unroll
-                for (int o = 4; o < 32; o <<= 1) psum += __shfl_xor_sync(kFull, psum, o);
-                pw[hg] = pj;
-#pragma unroll
-                for (int k = 0; k < 4; k++) {  // lane k holds head 4 hg + k's figures
-                    const int h = hg * 4 + k;
-                    if (h >= G || h >= g) break;
-                    const float mn = __shfl_sync(kFull, mnew, k), ps = __shfl_sync(kFull, psum, k);
-                    const float al = m[h] == -INFINITY ? 0.f : ex2(m[h] - mn);
-                    l[h] = fmaf(l[h], al, ps);
-#pragma unroll
-                    for (int e = 0; e < 4; e++) acc[h][e] *= al;
-                    m[h] = mn;
-                }
+            for (int ks = 0; ks < 8; ks++) {
+                const int blk = 4 * ks + j;
+                float ka[4], kb[4];
+                hq_block(hq_field(ra, blk), ma, SK, units, blk, cpy, ka);
+                hq_block(hq_field(rb, blk), mb, SK, units, blk, cpy, kb);
+                if (!va) ka[0] = ka[1] = ka[2] = ka[3] = 0.f;
+                if (!vb) kb[0] = kb[1] = kb[2] = kb[3] = 0.f;
+                uint32_t ah[4], al[4];
+                split_h2(ka[0], ka[1], ah[0], al[0]);
+                split_h2(kb[0], kb[1], ah[1], al[1]);
+                split_h2(ka[2], ka[3], ah[2], al[2]);
+                split_h2(kb[2], kb[3], ah[3], al[3]);
+                // (K_hi + K_lo)(q_hi + q_lo) without the lo x lo term
+                mma16816(sc, ah, qb[ks][0], qb[ks][1]);
+                mma16816(sc, al, qb[ks][0], qb[ks][1]);
+                mma16816(sc, ah, ql[ks][0], ql[ks][1]);
             }
-            // values: rebuild each token's block once, every head takes its weight
+            if (!va) sc[0] = sc[1] = -INFINITY;
+            if (!vb) sc[2] = sc[3] = -INFINITY;
+        }
+        // ---- online softmax per head over the page's 16 tokens ----
+        float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
 #pragma unroll
-            for (int u = 0; u < kHqTok; u++) {
-                if (!((vmask >> u) & 1u)) continue;  // warp-uniform
-                const int tok = tok0 + u;
-                float vc[4];
-                hq_block(hq_field(chunk + L.v_codes + tok * kHqRowCode, lane), chunk + L.v_meta + tok * kHqmqRowMeta,
-                         SV, units, lane, vc);
+        for (int o = 4; o < 32; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o));
+        }
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float al0 = m0 == -INFINITY ? 0.f : ex2(m0 - mn0), al1 = m1 == -INFINITY ? 0.f : ex2(m1 - mn1);
+        const float p0 = sc[0] == -INFINITY ? 0.f : ex2(sc[0] - mn0), p1 = sc[1] == -INFINITY ? 0.f : ex2(sc[1] - mn1);
+        const float p2 = sc[2] == -INFINITY ? 0.f : ex2(sc[2] - mn0), p3 = sc[3] == -INFINITY ? 0.f : ex2(sc[3] - mn1);
+        float ps0 = p0 + p2, ps1 = p1 + p3;
 #pragma unroll
-                for (int h = 0; h < G; h++) {
-                    if (h >= g) break;
-                    const float w = __shfl_sync(kFull, pw[h >> 2], u * 4 + (h & 3));
+        for (int o = 4; o < 32; o <<= 1) {
+            ps0 += __shfl_xor_sync(kFull, ps0, o);
+            ps1 += __shfl_xor_sync(kFull, ps1, o);
+        }
+        l0 = fmaf(l0, al0, ps0);
+        l1 = fmaf(l1, al1, ps1);
+        m0 = mn0;
+        m1 = mn1;
 #pragma unroll
-                    for (int e = 0; e < 4; e++) acc[h][e] = fmaf(w, vc[e], acc[h][e]);
+        for (int mt = 0; mt < 8; mt++) {
+            acc[mt][0] *= al0;
+            acc[mt][1] *= al1;
+            acc[mt][2] *= al0;
+            acc[mt][3] *= al1;
+        }
+        // P^T fragments (hi and lo): tokens 2j, 2j+1 (b0) and 2j+8, 2j+9 (b1) of head r
+        uint32_t pb[2][2];
+        {
+            uint32_t t[2][2];
+            split_h2(p0, p1, t[0][0], t[1][0]);
+            split_h2(p2, p3, t[0][1], t[1][1]);
+#pragma unroll
+            for (int hl = 0; hl < 2; hl++)
+#pragma unroll
+                for (int k = 0; k < 2; k++)
+                    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(pb[hl][k]) : "r"(t[hl][k]));
+        }
+        // ---- values: block 8i + r of tokens 2j, 2j+1, 2j+8, 2j+9 ----
+        {
+            const int tk[4] = {2 * j, 2 * j + 1, 2 * j + 8, 2 * j + 9};
+#pragma unroll
+            for (int ib = 0; ib < 4; ib++) {
+                const int blk = 8 * ib + r;
+                float v[4][4];
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    hq_block(hq_field(chunk + L.v_codes + tk[u] * kHqRowCode, blk),
+                             chunk + L.v_meta + tk[u] * kHqmqRowMeta, SV, units, blk, cpy, v[u]);
+                    if (tk[u] >= nvalid) v[u][0] = v[u][1] = v[u][2] = v[u][3] = 0.f;
+                }
+#pragma unroll
+                for (int hf = 0; hf < 2; hf++) {  // tile 2 ib + hf: dims 2 hf (rows r), 2 hf + 1 (rows r + 8)
+                    uint32_t ah[4], al[4];
+                    split_h2(v[0][2 * hf], v[1][2 * hf], ah[0], al[0]);
+                    split_h2(v[0][2 * hf + 1], v[1][2 * hf + 1], ah[1], al[1]);
+                    split_h2(v[2][2 * hf], v[3][2 * hf], ah[2], al[2]);
+                    split_h2(v[2][2 * hf + 1], v[3][2 * hf + 1], ah[3], al[3]);
+                    // (V_hi + V_lo)(P_hi + P_lo) without the lo x lo term
+                    mma16816(acc[2 * ib + hf], ah, pb[0][0], pb[0][1]);
+                    mma16816(acc[2 * ib + hf], ah, pb[1][0], pb[1][1]);
+                    mma16816(acc[2 * ib + hf], al, pb[0][0], pb[0][1]);
                 }
             }
         }
@@ -587,15 +630,21 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
     __syncthreads();  // every warp is done with the codebooks
     float *wacc = reinterpret_cast<float *>(tab);  // [kHqWarps][G][128]
 #pragma unroll
-    for (int h = 0; h < G; h++)
+    for (int hh = 0; hh < 2; hh++) {
+        const int h = 2 * j + hh;
         if (h < g) {
-            *reinterpret_cast<float4 *>(wacc + (warp * G + h) * kHqD + lane * 4) =
-                make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
-            if (lane == 0) {
-                wm[warp][h] = m[h];
-                wl[warp][h] = l[h];
+#pragma unroll
+            for (int ib = 0; ib < 4; ib++) {
+                const int blk = 8 * ib + r;
+                *reinterpret_cast<float4 *>(wacc + (warp * G + h) * kHqD + 4 * blk) =
+                    make_float4(acc[2 * ib][hh], acc[2 * ib][2 + hh], acc[2 * ib + 1][hh], acc[2 * ib + 1][2 + hh]);
+            }
+            if (r == 0) {
+                wm[warp][h] = hh ? m1 : m0;
+                wl[warp][h] = hh ? l1 : l0;
             }
         }
+    }
     __syncthreads();
     constexpr int REC = kHqD + 4;
     const long long bk = (long long)b * L.hkv + kvh;
