@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "kvq_oracle.c")
 _LIB = os.path.join(_HERE, "_liboracle.so")
 
-INT4_ASYM, INT8_SYM, INT2_ASYM, HQMQ = 0, 1, 2, 3
+INT4_ASYM, INT8_SYM, INT2_ASYM, HQMQ, NVFP4 = 0, 1, 2, 3, 4
 HQMQ_NS, HQMQ_NO = 1024, 2
 PAGE_TOKENS = 16
 
@@ -131,6 +131,11 @@ def lib():
             "kvqo_hqmq_quantize_rows": (None, [P, i32, i32, P, P, P, P, P]),
             "kvqo_hqmq_encode_dirs": (None, [P, i32, P, P]),
             "kvqo_hqmq_read_row": (None, [cfgp, P, i32, i32, i32, P, P, P, P]),
+            "kvqo_e4m3_value": (f64, [C.c_uint8]),
+            "kvqo_e4m3_rn_sat_n": (None, [P, P, sz]),
+            "kvqo_e2m1_rn_n": (None, [P, P, sz]),
+            "kvqo_nvfp4_quantize_rows": (None, [P, i32, i32, i32, P, P]),
+            "kvqo_nvfp4_read_row": (None, [cfgp, P, i32, i32, i32, P, P]),
             "kvqo_decode_windows": (i32, [cfgp, P, P, P, i32, i32, P, P, i32, P, i32, f64, P]),
             "kvqo_decode_ladder": (i32, [cfgp, P, P, P, P, P, i32, P, i32, f64, C.POINTER(Ladder), P, P,
                                          C.POINTER(LadderOut)]),
@@ -462,6 +467,46 @@ def hqmq_encode_dirs(u, S) -> np.ndarray:
     idx = np.zeros(u.shape[0], np.int32)
     lib().kvqo_hqmq_encode_dirs(_p(u), u.shape[0], _p(S), _p(idx))
     return idx
+
+
+def e4m3_value(b: int) -> float:
+    """Value of an E4M3 byte (NaN for S.1111.111)."""
+    return float(lib().kvqo_e4m3_value(int(b) & 0xFF))
+
+
+def e4m3_rn(x) -> np.ndarray:
+    """Non-negative fp32 values to E4M3 bytes (nearest, ties to even, saturating at 448)."""
+    x = _c(np.atleast_1d(x), np.float32)
+    out = np.zeros(x.shape, np.uint8)
+    lib().kvqo_e4m3_rn_sat_n(_p(x), _p(out), x.size)
+    return out
+
+
+def e2m1_rn(v) -> np.ndarray:
+    """fp32 values to 4-bit e2m1 codes (nearest, ties to the even magnitude, saturating at 6)."""
+    v = _c(np.atleast_1d(v), np.float32)
+    out = np.zeros(v.shape, np.uint8)
+    lib().kvqo_e2m1_rn_n(_p(v), _p(out), v.size)
+    return out
+
+
+def nvfp4_quantize_rows(y, search: int = 0):
+    """NVFP4 codes [n, d] (uint8, one per element) and E4M3 scale bytes [n, d/16]
+    of fp32 rows [n, d] (the codec the append applies)."""
+    y = _c(y, np.float32)
+    n, d = y.shape
+    code = np.zeros((n, d), np.uint8)
+    scale = np.zeros((n, d // 16), np.uint8)
+    lib().kvqo_nvfp4_quantize_rows(_p(y), n, d, int(search), _p(code), _p(scale))
+    return code, scale
+
+
+def nvfp4_read_row(cfg: Config, pool: np.ndarray, slot: int, kvh: int, tensor: int):
+    d = cfg.head_dim
+    code = np.zeros(d, np.uint8)
+    scale = np.zeros(d // 16, np.uint8)
+    lib().kvqo_nvfp4_read_row(C.byref(cfg), _p(pool), slot, kvh, tensor, _p(code), _p(scale))
+    return code, scale
 
 
 def hqmq_read_row(cfg: Config, pool: np.ndarray, slot: int, kvh: int, tensor: int):

@@ -43,6 +43,7 @@
 #define KVQO_INT8_SYM 1
 #define KVQO_INT2_ASYM 2
 #define KVQO_HQMQ 3        /* Hurwitz-quaternion multiplicative VQ of 4-element blocks */
+#define KVQO_NVFP4 4       /* e2m1 codes, one E4M3 scale per 16 elements */
 #define KVQO_HQMQ_NS 1024  /* secondary codebook size per (kv head, K|V) */
 #define KVQO_HQMQ_NO 2     /* fp16 outlier blocks a row can keep (Med3x) */
 
@@ -569,6 +570,122 @@ static void hqmq_dequant_block(uint32_t field, int is_outlier, const uint16_t *o
 }
 
 /* ------------------------------------------------------------------------- */
+/* NVFP4 ([ScaleSearch] NVFP4 and ScaleSearch: e2m1 values, an E4M3 scale    */
+/* per block of 16, default scale = round(max|x| / 6) in E4M3)               */
+/* ------------------------------------------------------------------------- */
+
+/* Value of an E4M3 byte (OCP FP8 E4M3FN: bias 7, no infinities, S.1111.111
+ * is NaN, subnormals m * 2^-9). */
+double kvqo_e4m3_value(uint8_t b)
+{
+    int e = (b >> 3) & 15, m = b & 7;
+    double sg = (b & 0x80) ? -1.0 : 1.0;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) return sg * ldexp((double)m, -9);
+    return sg * ldexp(1.0 + m / 8.0, e - 7);
+}
+
+/* Non-negative x to E4M3: the nearest finite code, ties to the even code,
+ * anything above the largest finite value (448) to 448; NaN to NaN. */
+uint8_t kvqo_e4m3_rn_sat(float x)
+{
+    if (isnan(x)) return 0x7F;
+    int best = 0;
+    double bd = INFINITY;
+    for (int b = 0; b <= 0x7E; b++) {
+        double dd = fabs((double)x - kvqo_e4m3_value((uint8_t)b));
+        if (dd < bd || (dd == bd && !(b & 1))) {
+            bd = dd;
+            best = b;
+        }
+    }
+    return (uint8_t)best;
+}
+
+static const double e2m1_mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+/* v to a 4-bit e2m1 code: the nearest of +-{0, 0.5, 1, 1.5, 2, 3, 4, 6},
+ * ties to the even magnitude index, beyond 6 to 6; bit 3 = sign (zero is
+ * always code 0). */
+uint8_t kvqo_e2m1_rn(float v)
+{
+    double a = fabs((double)v);
+    int best = 0;
+    double bd = INFINITY;
+    for (int m = 0; m < 8; m++) {
+        double dd = fabs(a - e2m1_mag[m]);
+        if (dd < bd || (dd == bd && !(m & 1))) {
+            bd = dd;
+            best = m;
+        }
+    }
+    if (best == 0) return 0;
+    return (uint8_t)((signbit(v) ? 8 : 0) | best);
+}
+
+static double e2m1_value(uint8_t c) { return ((c & 8) ? -1.0 : 1.0) * e2m1_mag[c & 7]; }
+
+/* Codes of a 16-element block under scale code sc: v = y / scale (fp32),
+ * code = e2m1 of v; all zero when the scale is 0. */
+static void nvfp4_codes(const float *y, uint8_t sc, uint8_t *code)
+{
+    float sf = (float)kvqo_e4m3_value(sc);
+    for (int i = 0; i < 16; i++) code[i] = sf > 0.0f ? kvqo_e2m1_rn(y[i] / sf) : 0;
+}
+
+/* Squared reconstruction error of a block in fp32: per run of four
+ * elements ((e0^2 + e1^2) + e2^2) + e3^2, then (r0 + r1) + (r2 + r3); each
+ * e = y - code value x scale (that product is exact), each operation
+ * rounded. */
+static float nvfp4_sq_error(const float *y, uint8_t sc)
+{
+    uint8_t code[16];
+    nvfp4_codes(y, sc, code);
+    float sf = (float)kvqo_e4m3_value(sc), r[4];
+    for (int q = 0; q < 4; q++) {
+        float acc = 0.0f;
+        for (int i = 0; i < 4; i++) {
+            float e = y[4 * q + i] - (float)e2m1_value(code[4 * q + i]) * sf;
+            float e2 = e * e;
+            acc = i == 0 ? e2 : acc + e2;
+        }
+        r[q] = acc;
+    }
+    return (r[0] + r[1]) + (r[2] + r[3]);
+}
+
+/* One row of d elements: per block of 16, amax = max |y| (fp32), default
+ * scale code = E4M3 RN (saturating) of amax / 6 (fp32 division); with
+ * search ([ScaleSearch] ScaleSearch) the codes b0 + f, f tried as 0, -1, 1,
+ * -2, 2, 3, 4, 5, 6 (positive finite codes only, b0 itself nonzero and
+ * finite), keep the least squared error, a later one only if strictly
+ * smaller. */
+static void nvfp4_quantize_row(const float *y, int d, int search, uint8_t *code, uint8_t *scale)
+{
+    for (int g = 0; g < d / 16; g++) {
+        const float *yg = y + 16 * g;
+        float amax = 0.0f;
+        for (int i = 0; i < 16; i++) amax = fmaxf(amax, fabsf(yg[i]));
+        uint8_t b0 = kvqo_e4m3_rn_sat(amax / 6.0f), best = b0;
+        if (search && b0 != 0 && b0 <= 0x7E) {
+            static const int offs[9] = {0, -1, 1, -2, 2, 3, 4, 5, 6};
+            float be = 0.0f;
+            for (int k = 0; k < 9; k++) {
+                int b = (int)b0 + offs[k];
+                if (b < 1 || b > 0x7E) continue;
+                float e = nvfp4_sq_error(yg, (uint8_t)b);
+                if (k == 0 || e < be) {
+                    be = e;
+                    best = (uint8_t)b;
+                }
+            }
+        }
+        scale[g] = best;
+        nvfp4_codes(yg, best, code + 16 * g);
+    }
+}
+
+/* ------------------------------------------------------------------------- */
 /* Paged pool layout (restated here from the written layout definition)      */
 /* ------------------------------------------------------------------------- */
 /* pool  = [header: 256 B][pages: num_pages x page_bytes][descriptors]
@@ -588,10 +705,18 @@ static void hqmq_dequant_block(uint32_t field, int is_outlier, const uint16_t *o
  * radius code) as one little-endian bit stream; meta = fp16 radius step,
  * 2 zero bytes, the 32-bit outlier mask, KVQO_HQMQ_NO outlier slots of four
  * fp16 values (in block order). */
-static int row_code_bytes(int fmt, int d) { return fmt == KVQO_HQMQ ? d * 5 / 8 : d * fmt_bits(fmt) / 8; }
+/* NVFP4 rows: d/2 code bytes (byte j = code[2j] | code[2j+1] << 4) stored
+ * token-major, meta = d/16 E4M3 scale bytes. */
+static int row_code_bytes(int fmt, int d)
+{
+    if (fmt == KVQO_HQMQ) return d * 5 / 8;
+    if (fmt == KVQO_NVFP4) return d / 2;
+    return d * fmt_bits(fmt) / 8;
+}
 static int row_meta_bytes(int fmt, int d, int group)
 {
     if (fmt == KVQO_HQMQ) return 8 + 8 * KVQO_HQMQ_NO;
+    if (fmt == KVQO_NVFP4) return d / 16;
     return fmt == KVQO_INT8_SYM ? 2 : 4 * (d / group);
 }
 static size_t region_code_bytes(int fmt, int d) { return (size_t)KVQO_PAGE_TOKENS * row_code_bytes(fmt, d); }
@@ -719,6 +844,31 @@ void kvqo_hqmq_read_row(const kvqo_config *c, const uint8_t *pool, int slot, int
     memcpy(outl, meta + 8, 8 * KVQO_HQMQ_NO);
 }
 
+static void nvfp4_pack_row(const kvqo_config *c, uint8_t *pool, int page, int tok, int kvh, int tensor,
+                           const uint8_t *code, const uint8_t *scale)
+{
+    int d = c->head_dim;
+    uint8_t *row = pool + region_base(c, page, kvh, tensor, 0) + (size_t)tok * row_code_bytes(KVQO_NVFP4, d);
+    for (int j = 0; j < d / 2; j++) row[j] = (uint8_t)(code[2 * j] | (code[2 * j + 1] << 4));
+    memcpy(pool + region_base(c, page, kvh, tensor, 1) + (size_t)tok * row_meta_bytes(KVQO_NVFP4, d, 16), scale,
+           (size_t)(d / 16));
+}
+
+/* Read an NVFP4 row back: codes (one per element) and scale bytes. */
+void kvqo_nvfp4_read_row(const kvqo_config *c, const uint8_t *pool, int slot, int kvh, int tensor, uint8_t *code,
+                         uint8_t *scale)
+{
+    int d = c->head_dim;
+    int page = slot / KVQO_PAGE_TOKENS, tok = slot % KVQO_PAGE_TOKENS;
+    const uint8_t *row = pool + region_base(c, page, kvh, tensor, 0) + (size_t)tok * row_code_bytes(KVQO_NVFP4, d);
+    for (int j = 0; j < d / 2; j++) {
+        code[2 * j] = row[j] & 15;
+        code[2 * j + 1] = row[j] >> 4;
+    }
+    memcpy(scale, pool + region_base(c, page, kvh, tensor, 1) + (size_t)tok * row_meta_bytes(KVQO_NVFP4, d, 16),
+           (size_t)(d / 16));
+}
+
 /* Read back the codes, scales and zeros of one stored row (inverse of
  * pack_row). */
 void kvqo_read_row(const kvqo_config *c, const uint8_t *pool, int slot, int kvh, int tensor, int16_t *code,
@@ -771,6 +921,12 @@ void kvqo_dequant_row(const kvqo_config *c, const uint8_t *pool, int slot, int k
         }
         return;
     }
+    if (fmt == KVQO_NVFP4) {  /* e2m1 value x E4M3 scale */
+        uint8_t nc[KVQO_MAXD], ns[KVQO_MAXD / 16];
+        kvqo_nvfp4_read_row(c, pool, slot, kvh, tensor, nc, ns);
+        for (int i = 0; i < d; i++) out[i] = e2m1_value(nc[i]) * kvqo_e4m3_value(ns[i / 16]);
+        return;
+    }
     int16_t code[KVQO_MAXD];
     uint16_t sh[KVQO_MAXD], zh[KVQO_MAXD];
     kvqo_read_row(c, pool, slot, kvh, tensor, code, sh, zh);
@@ -792,6 +948,7 @@ static int fmt_ok(int fmt, int group, int d)
 {
     if (fmt == KVQO_INT8_SYM) return 1;
     if (fmt == KVQO_HQMQ) return group == 4 && d == 128;
+    if (fmt == KVQO_NVFP4) return group == 16 && d == 128;
     if (fmt != KVQO_INT4_ASYM && fmt != KVQO_INT2_ASYM) return 0;
     if (group <= 0 || d % group) return 0;
     return 1;
@@ -809,6 +966,8 @@ int kvqo_config_ok(const kvqo_config *c)
     if (c->scale_search != 0 && c->scale_search != 1) return 0;
     if ((c->k_fmt == KVQO_HQMQ) != (c->v_fmt == KVQO_HQMQ)) return 0;  /* both or neither */
     if (c->k_fmt == KVQO_HQMQ && (c->bound_block_tokens != 0 || c->scale_search)) return 0;
+    if ((c->k_fmt == KVQO_NVFP4) != (c->v_fmt == KVQO_NVFP4)) return 0;
+    if (c->k_fmt == KVQO_NVFP4 && c->bound_block_tokens != 0) return 0;
     return 1;
 }
 
@@ -849,6 +1008,12 @@ int kvqo_append(const kvqo_config *c, uint8_t *pool, const uint16_t *k, const ui
                     uint16_t step, outl[KVQO_HQMQ_NO][4];
                     hqmq_quantize_row(y, d, hqmq_table(c, pool, kvh, tensor), field, &step, &mask, outl);
                     hqmq_pack_row(c, pool, page, tok, kvh, tensor, field, step, mask, outl);
+                    continue;
+                }
+                if (fmt == KVQO_NVFP4) {
+                    uint8_t nc[KVQO_MAXD], ns[KVQO_MAXD / 16];
+                    nvfp4_quantize_row(y, d, c->scale_search, nc, ns);
+                    nvfp4_pack_row(c, pool, page, tok, kvh, tensor, nc, ns);
                     continue;
                 }
                 int16_t code[KVQO_MAXD];
@@ -1671,6 +1836,21 @@ void kvqo_hqmq_quantize_rows(const float *y, int n, int d, const float *S, uint3
     for (int r = 0; r < n; r++)
         hqmq_quantize_row(y + (size_t)r * d, d, S, field + (size_t)r * (d / 4), step + r, mask + r,
                           (uint16_t(*)[4])(outl + (size_t)r * KVQO_HQMQ_NO * 4));
+}
+
+void kvqo_nvfp4_quantize_rows(const float *y, int n, int d, int search, uint8_t *code, uint8_t *scale)
+{
+    for (int r = 0; r < n; r++) nvfp4_quantize_row(y + (size_t)r * d, d, search, code + (size_t)r * d, scale + (size_t)r * (d / 16));
+}
+
+void kvqo_e2m1_rn_n(const float *v, uint8_t *c, size_t n)
+{
+    for (size_t i = 0; i < n; i++) c[i] = kvqo_e2m1_rn(v[i]);
+}
+
+void kvqo_e4m3_rn_sat_n(const float *x, uint8_t *b, size_t n)
+{
+    for (size_t i = 0; i < n; i++) b[i] = kvqo_e4m3_rn_sat(x[i]);
 }
 
 void kvqo_hqmq_encode_dirs(const float *u, int n, const float *S, int32_t *idx)
