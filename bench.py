@@ -76,7 +76,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-steps", type=int, default=4, help="oracle steps in the CPU baseline sample")
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, append and CPU legs")
-    ap.add_argument("--leg", choices=["certified", "ladder", "windows", "hqmq"],
+    ap.add_argument("--leg", choices=["certified", "ladder", "windows", "hqmq", "nvfp4"],
                     help="run only this leg (one GPU, --steps calls) and print its JSON")
     ap.add_argument("--ctx", type=int, default=0, help="context length of --leg (default: its workload's)")
     return ap.parse_args()
@@ -397,6 +397,7 @@ def run_ours(args, dist: Dist):
         result["ladder"] = ladder_leg(min(K, 100))
         result["windows"] = windows_leg(min(K, 200))
         result["hqmq"] = hqmq_leg(min(K, 200))
+        result["nvfp4"] = nvfp4_leg(min(K, 200))
     if dist.rank == 0:
         if not args.no_extras:
             result["cpu_baseline"] = cpu_leg(wk, args.cpu_steps)
@@ -671,6 +672,85 @@ def windows_leg(steps: int, T: int = 0, sink: int = 128, recent: int = 1024):
             "cache_bytes": kv_bytes, "window_bytes": win_bytes, "steps": steps}
 
 
+def nvfp4_leg(steps: int, T: int = 0):
+    """The NVFP4 codec at Llama-3-8B layer shape (batch 1, 32/8 heads,
+    d=128, context 32768, rotated, ScaleSearch on the E4M3 scales): the bulk
+    append of the whole context and a one-token append timed with events;
+    the decode replayed in a CUDA graph over four cache copies (151 MB, above
+    L2), beside the same decode of a cache without ScaleSearch."""
+    import torch
+
+    import quantized_kv_cache_16_b200 as K
+    import workloads as W
+    wl = W.nvfp4(T) if T else W.nvfp4()
+    T, copies = wl.ctx[0], 4
+    dev = torch.device("cuda", torch.cuda.current_device())
+    tabs = W.page_table(wl, copies=copies, extra_tokens=8)
+    rt = Cudart()
+    stream = torch.cuda.Stream()
+    e0, e1 = rt.event(), rt.event()
+    kd, vd = W.prefix_kv_device(wl, 0, dev)
+    res = {}
+    for search in (1, 0):
+        cfg = K.make_config(wl.Hq, wl.Hkv, wl.d, wl.k_fmt, wl.v_fmt, wl.k_group, wl.v_group, wl.clip,
+                            wl.rotation_seed, rotate=wl.rotate, num_pages=tabs[0].num_pages, scale_search=search)
+        cache = K.Cache(cfg)
+        bulk_ms = []
+        for c in range(copies):
+            sl = torch.from_numpy(tabs[c].slots(0, 0, T)).to(dev)
+            rt.record(e0, stream.cuda_stream)
+            with torch.cuda.stream(stream):
+                cache.append(kd, vd, sl, stream=stream)
+            rt.record(e1, stream.cuda_stream)
+            torch.cuda.synchronize()
+            bulk_ms.append(rt.elapsed_ms(e0, e1))
+        kn, vn = (torch.from_numpy(x).to(dev) for x in W.step_kv(wl, 0))
+        tok_slots = [torch.from_numpy(tabs[0].slots(0, T + i, T + i + 1)).to(dev) for i in range(8)]
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                cache.append(kn, vn, tok_slots[i], stream=stream)
+        torch.cuda.synchronize()
+        rt.record(e0, stream.cuda_stream)
+        with torch.cuda.stream(stream):
+            for i in range(50):
+                cache.append(kn, vn, tok_slots[i % 8], stream=stream)
+        rt.record(e1, stream.cuda_stream)
+        torch.cuda.synchronize()
+        tok_us = rt.elapsed_ms(e0, e1) * 1e3 / 50
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(wl.seed)
+        nq = 8
+        qs = torch.randn((nq, wl.B, wl.Hq, wl.d), generator=gen, device=dev).half()
+        bts = [torch.from_numpy(t.block_table).to(dev) for t in tabs]
+        max_pages = bts[0].shape[1]
+        ctx = torch.tensor(wl.ctx, dtype=torch.int32, device=dev)
+        ws = cache.workspace_for(wl.B, max_pages)
+        out = torch.empty((wl.B, wl.Hq, wl.d), dtype=torch.float32, device=dev)
+
+        def dec(s):
+            K.kvq_decode_attn(cache.handle, qs[s % nq], bts[s % copies], max_pages, ctx, wl.B, 0.0, None, ws,
+                              ws.numel(), out, None, stream)
+
+        d_us = _graph_time(dec, steps, stream)
+        assert cache.sync_status() == 0
+        res[search] = (min(bulk_ms), tok_us, d_us)
+        del cache
+    del kd, vd
+    row_bytes = wl.d // 2 + wl.d // 16  # e2m1 codes + E4M3 scales
+    kv_bytes = T * wl.Hkv * 2 * row_bytes
+    rows = 2 * T * wl.Hkv
+    peak, kind = measured_peaks()
+    bulk, tok_us, d_us = res[1]
+    return {"workload": f"NVFP4 K/V, B=1, 32/8 heads, d=128, context {T}, rotated, ScaleSearch on",
+            "decode_us": round(d_us, 2), "decode_gbs": round(kv_bytes / d_us / 1e3, 1),
+            "decode_pct_hbm_peak": kv_bytes / d_us / 1e3 / peak, "peak_kind": kind, "cache_bytes": kv_bytes,
+            "bits_per_element": row_bytes * 8 / wl.d, "bulk_append_ms": round(bulk, 3),
+            "bulk_append_rows_per_s": round(rows / bulk * 1e3, 1), "token_append_us": round(tok_us, 2),
+            "no_search": {"bulk_append_ms": round(res[0][0], 3), "token_append_us": round(res[0][1], 2),
+                          "decode_us": round(res[0][2], 2)},
+            "steps": steps}
+
+
 def hqmq_leg(steps: int, T: int = 0):
     """The HQMQ codec at Llama-3-8B layer shape (batch 1, 32/8 heads, d=128,
     context 32768, K and V coded from the raw rows): the bulk append of the
@@ -909,7 +989,8 @@ def main():
     if args.leg:
         import torch
         torch.cuda.set_device(0)
-        leg = {"certified": certified_leg, "ladder": ladder_leg, "windows": windows_leg, "hqmq": hqmq_leg}[args.leg]
+        leg = {"certified": certified_leg, "ladder": ladder_leg, "windows": windows_leg, "hqmq": hqmq_leg,
+               "nvfp4": nvfp4_leg}[args.leg]
         print(json.dumps(leg(args.steps, args.ctx)), flush=True)
         return
     if args.impl == "reference":

@@ -62,9 +62,28 @@ typedef enum {
     KVQ_INT4_ASYM = 0, /* 4-bit codes, group 32, fp16 scale + fp16 zero         */
     KVQ_INT8_SYM = 1,  /* 8-bit signed codes, one fp16 scale per token-head     */
     KVQ_INT2_ASYM = 2, /* 2-bit codes, group = head_dim, fp16 scale + fp16 zero */
-    KVQ_HQMQ = 3       /* Hurwitz-quaternion codes of 4-element blocks (group 4,
+    KVQ_HQMQ = 3,      /* Hurwitz-quaternion codes of 4-element blocks (group 4,
+                          head_dim 128, keys and values both), see below       */
+    KVQ_NVFP4 = 4      /* e2m1 codes, one E4M3 scale per 16 elements (group 16,
                           head_dim 128, keys and values both), see below       */
 } kvq_fmt;
+
+/* NVFP4 ["Search Your Block Floating Point Scales!", NVFP4 and ScaleSearch].
+ * Per block of 16 rotated elements: scale byte = E4M3 (OCP E4M3FN) of
+ * max|x| / 6 (fp32 division; nearest, ties to the even code, above 448 to
+ * 448); code of x = e2m1 of x / scale (fp32 division): the nearest of
+ * +-{0, 0.5, 1, 1.5, 2, 3, 4, 6}, ties to the even magnitude index, beyond
+ * 6 to 6, zero (and NaN) code 0, bit 3 the sign; all codes 0 when the scale
+ * is 0.  With scale_search = 1 the scale bytes b0 + f, f tried as 0, -1, 1,
+ * -2, 2, 3, 4, 5, 6 (positive finite codes only; b0 nonzero and finite),
+ * each quantise the block and the least squared error wins, a later one only
+ * if strictly smaller; the error is fp32, per run of four elements ((e0^2 +
+ * e1^2) + e2^2) + e3^2 with e = x - value, then (r0 + r1) + (r2 + r3).
+ * Storage (token-major rows): 64 code bytes (byte j = code[2j] |
+ * code[2j+1] << 4), then per region 16 meta rows of the 8 scale bytes.  A
+ * value decodes to e2m1 x scale, exact in fp16.  kvq_append, kvq_decode_attn
+ * (without tier 2) and kvq_decode_attn_static serve NVFP4 caches; the other
+ * decode calls return KVQ_ERR_UNSUPPORTED. */
 
 /* HQMQ ["Hurwitz Quaternion Multiplicative Quantization for KV Cache
  * Compression", 1-3].  A rotated row is cut into d/4 blocks x (a quaternion);
@@ -100,17 +119,17 @@ typedef enum {
  *     fp16 values in block order (unused slots zero).  The codebooks sit in
  *     the pool after the pages (and descriptors): [Hkv][2][1024] x 4 fp32.
  * A block decodes to (radius code x step) x q_p q_s, an outlier to its fp16
- * values.  HQMQ caches have no descriptors and no scale search; kvq_append
- * and kvq_decode_attn (without tier 2) serve them, the other decode calls
- * return KVQ_ERR_UNSUPPORTED. */
+ * values.  HQMQ caches have no descriptors and no scale search; kvq_append,
+ * kvq_decode_attn (without tier 2) and kvq_decode_attn_static serve them,
+ * the other decode calls return KVQ_ERR_UNSUPPORTED. */
 
 typedef struct {
     int32_t num_q_heads;        /* Hq; Hq / Hkv (the GQA group) must be 1..8          */
     int32_t num_kv_heads;       /* Hkv                                                */
     int32_t head_dim;           /* d: 64 or 128                                       */
     int32_t k_fmt, v_fmt;       /* kvq_fmt of keys / values (values: int4, int2, or
-                                   HQMQ with HQMQ keys)                              */
-    int32_t k_group, v_group;   /* int4: 32; int2: head_dim; int8: head_dim; HQMQ: 4  */
+                                   HQMQ / NVFP4 with keys of the same format)        */
+    int32_t k_group, v_group;   /* int4: 32; int2, int8: head_dim; HQMQ: 4; NVFP4: 16 */
     float clip_ratio;           /* (0, 1]; scales both ends of int2/int4 groups       */
     uint64_t rotation_seed;     /* SplitMix64 state that draws the sign vector        */
     int32_t rotate;             /* 1 = sign + Hadamard rotation, 0 = identity         */

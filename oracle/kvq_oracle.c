@@ -605,11 +605,12 @@ uint8_t kvqo_e4m3_rn_sat(float x)
 static const double e2m1_mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
 
 /* v to a 4-bit e2m1 code: the nearest of +-{0, 0.5, 1, 1.5, 2, 3, 4, 6},
- * ties to the even magnitude index, beyond 6 to 6; bit 3 = sign (zero is
- * always code 0). */
+ * ties to the even magnitude index, beyond 6 (infinity included) to 6; bit
+ * 3 = sign (zero is always code 0; NaN is code 0). */
 uint8_t kvqo_e2m1_rn(float v)
 {
     double a = fabs((double)v);
+    if (isinf(a)) return (uint8_t)((signbit(v) ? 8 : 0) | 7);
     int best = 0;
     double bd = INFINITY;
     for (int m = 0; m < 8; m++) {

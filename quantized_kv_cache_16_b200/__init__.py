@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(HERE, "libkvq.so")
 
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY = 0, 1, 2, 3
 KVQ_ERR_OUT_OF_RANGE, KVQ_ERR_CUDA, KVQ_ERR_TIMEOUT = 4, 5, 6
-KVQ_INT4_ASYM, KVQ_INT8_SYM, KVQ_INT2_ASYM, KVQ_HQMQ = 0, 1, 2, 3
+KVQ_INT4_ASYM, KVQ_INT8_SYM, KVQ_INT2_ASYM, KVQ_HQMQ, KVQ_NVFP4 = 0, 1, 2, 3, 4
 PAGE_TOKENS = 16
 
 # Every symbol include/kvq.h declares (checked by the ABI test).

@@ -77,12 +77,18 @@ kvq_status check_config(const kvq_config *c)
         case KVQ_HQMQ:
             if (groups[t] != 4 || c->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
             break;
+        case KVQ_NVFP4:
+            if (groups[t] != 16 || c->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+            break;
         default: return KVQ_ERR_INVALID_ARG;
         }
     }
     const bool hq = c->k_fmt == KVQ_HQMQ;
     if (hq != (c->v_fmt == KVQ_HQMQ)) return KVQ_ERR_UNSUPPORTED;  // HQMQ keys and values, or neither
     if (hq && (c->bound_block_tokens != 0 || c->scale_search != 0)) return KVQ_ERR_UNSUPPORTED;
+    const bool nv = c->k_fmt == KVQ_NVFP4;
+    if (nv != (c->v_fmt == KVQ_NVFP4)) return KVQ_ERR_UNSUPPORTED;  // NVFP4 keys and values, or neither
+    if (nv && c->bound_block_tokens != 0) return KVQ_ERR_UNSUPPORTED;
     if (!(c->clip_ratio > 0.0f && c->clip_ratio <= 1.0f)) return KVQ_ERR_INVALID_ARG;
     if (c->bound_block_tokens < 0 || c->bound_block_tokens % kPageTokens) return KVQ_ERR_INVALID_ARG;
     if (c->rotate != 0 && c->rotate != 1) return KVQ_ERR_INVALID_ARG;
@@ -354,6 +360,8 @@ kvq_status kvq_append(kvq_cache *c, const void *k, const void *v, const int32_t 
     memcpy(p.sign_xor, c->sign_xor, sizeof(p.sign_xor));
     c->last_stream = stream;
     if (c->L.hq_tab) return cuda_status(launch_hqmq_append(p, c->num_sms, static_cast<cudaStream_t>(stream)));
+    if (c->L.k_fmt == KVQ_NVFP4)
+        return cuda_status(launch_nvfp4_append(p, c->num_sms, static_cast<cudaStream_t>(stream)));
     return cuda_status(launch_append(p, c->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
@@ -472,7 +480,7 @@ kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const
     if (!q || !block_table || !ctx_lens || !out || !workspace) return KVQ_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
     if (k_new && (!v_new || !slot_mapping || !aligned(k_new, 16) || !aligned(v_new, 16))) return KVQ_ERR_INVALID_ARG;
-    if (c->L.hq_tab) {  // HQMQ: its own decode kernel, no fused append, no tier 2
+    if (c->L.hq_tab || c->L.k_fmt == KVQ_NVFP4) {  // HQMQ, NVFP4: own decode kernels, no fused append, no tier 2
         if (k_new || tier2) return KVQ_ERR_UNSUPPORTED;
         if (ws_bytes < kvq_decode_workspace_bytes(c, batch, max_pages_per_seq)) return KVQ_ERR_CAPACITY;
         const SplitPlan s = plan_splits(c, batch, max_pages_per_seq);
@@ -480,8 +488,9 @@ kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const
         const DecodeParams p =
             decode_params(c, s, q, block_table, max_pages_per_seq, ctx_lens, batch, scale, workspace, out);
         c->last_stream = stream;
-        return cuda_status(
-            launch_hqmq_decode(p, dim3(s.n_splits, c->L.hkv, batch), static_cast<cudaStream_t>(stream)));
+        const dim3 grid(s.n_splits, c->L.hkv, batch);
+        return cuda_status(c->L.hq_tab ? launch_hqmq_decode(p, grid, static_cast<cudaStream_t>(stream))
+                                       : launch_nvfp4_decode(p, grid, static_cast<cudaStream_t>(stream)));
     }
     if (!decode_supported(c->L)) return KVQ_ERR_UNSUPPORTED;
     // certified mode: checks and the tier-2 device view
@@ -701,7 +710,7 @@ kvq_status kvq_dequant_debug(kvq_cache *c, const int32_t *slots, int32_t n, floa
                              uint8_t *codes_out, uint16_t *meta_out, void *stream)
 {
     if (!c || n < 0) return KVQ_ERR_INVALID_ARG;
-    if (c->L.hq_tab) return KVQ_ERR_UNSUPPORTED;  // integer formats only
+    if (c->L.hq_tab || c->L.k_fmt == KVQ_NVFP4) return KVQ_ERR_UNSUPPORTED;  // integer formats only
     if (n == 0) return KVQ_OK;
     if (!slots) return KVQ_ERR_INVALID_ARG;
     DequantParams p{};

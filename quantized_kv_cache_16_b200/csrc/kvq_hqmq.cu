@@ -108,18 +108,8 @@ struct HqRow {
 
 __device__ __forceinline__ void hq_prepare(const AppendParams &p, const __half *src, int lane, HqRow &R)
 {
-    uint2 raw = *reinterpret_cast<const uint2 *>(src + 4 * lane);
-    if (p.rotate) {
-        raw.x ^= p.sign_xor[2 * lane];
-        raw.y ^= p.sign_xor[2 * lane + 1];
-    }
-    const float2 a = __half22float2(bits_h2(raw.x)), b = __half22float2(bits_h2(raw.y));
-    float x[4] = {a.x, a.y, b.x, b.y};
-    if (p.rotate) {
-        fwht_warp<kHqD>(x, lane);  // butterfly stages h = 1, 2, ..., 64, each add rounded
-#pragma unroll
-        for (int e = 0; e < 4; e++) x[e] = __fmul_rn(x[e], p.rot_scale);
-    }
+    float x[4];
+    rotated_row_lane4(p, src, lane, x);  // butterfly stages h = 1, 2, ..., 64, each add rounded
 #pragma unroll
     for (int e = 0; e < 4; e++) R.x[e] = x[e];
     const float r = __fsqrt_rn(__fadd_rn(__fadd_rn(__fadd_rn(__fmul_rn(x[0], x[0]), __fmul_rn(x[1], x[1])),

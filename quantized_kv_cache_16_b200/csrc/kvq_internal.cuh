@@ -30,7 +30,7 @@ constexpr int kHqmqRowMeta = 8 + 8 * kHqmqOut;
 
 inline __host__ __device__ int fmt_bits(int fmt)
 {
-    return fmt == KVQ_INT4_ASYM ? 4 : fmt == KVQ_INT8_SYM ? 8 : fmt == KVQ_HQMQ ? 5 : 2;
+    return fmt == KVQ_INT4_ASYM || fmt == KVQ_NVFP4 ? 4 : fmt == KVQ_INT8_SYM ? 8 : fmt == KVQ_HQMQ ? 5 : 2;
 }
 
 // Byte layout of the pool (see kvq_pool_bytes in kvq.h).
@@ -59,8 +59,14 @@ inline __host__ Layout make_layout(const kvq_config &c)
     L.v_fmt = c.v_fmt;
     L.k_row_code = L.d * fmt_bits(c.k_fmt) / 8;
     L.v_row_code = L.d * fmt_bits(c.v_fmt) / 8;
-    L.k_row_meta = c.k_fmt == KVQ_HQMQ ? kHqmqRowMeta : c.k_fmt == KVQ_INT8_SYM ? 2 : 4 * (L.d / c.k_group);
-    L.v_row_meta = c.v_fmt == KVQ_HQMQ ? kHqmqRowMeta : c.v_fmt == KVQ_INT8_SYM ? 2 : 4 * (L.d / c.v_group);
+    L.k_row_meta = c.k_fmt == KVQ_HQMQ    ? kHqmqRowMeta
+                   : c.k_fmt == KVQ_NVFP4 ? L.d / 16
+                   : c.k_fmt == KVQ_INT8_SYM ? 2
+                                              : 4 * (L.d / c.k_group);
+    L.v_row_meta = c.v_fmt == KVQ_HQMQ    ? kHqmqRowMeta
+                   : c.v_fmt == KVQ_NVFP4 ? L.d / 16
+                   : c.v_fmt == KVQ_INT8_SYM ? 2
+                                              : 4 * (L.d / c.v_group);
     L.k_codes = 0;
     L.k_meta = kPageTokens * L.k_row_code;
     L.v_codes = L.k_meta + kPageTokens * L.k_row_meta;
@@ -239,6 +245,8 @@ cudaError_t launch_ladder_finish(const CertParams &p, int batch, cudaStream_t s)
 cudaError_t launch_windows(const CertParams &p, int batch, cudaStream_t s);
 cudaError_t launch_hqmq_append(const AppendParams &p, int num_sms, cudaStream_t s);
 cudaError_t launch_hqmq_decode(const DecodeParams &p, dim3 grid, cudaStream_t s);
+cudaError_t launch_nvfp4_append(const AppendParams &p, int num_sms, cudaStream_t s);
+cudaError_t launch_nvfp4_decode(const DecodeParams &p, dim3 grid, cudaStream_t s);
 bool decode_supported(const Layout &L);
 int decode_max_splits(const Layout &L);
 constexpr int kDecodeWarps = 8;

@@ -67,4 +67,27 @@ __device__ __forceinline__ void fwht_warp2(float (&x)[D / 32], float (&y)[D / 32
         }
 }
 
+// A head_dim-128 fp16 row at `src` as rotated fp32, lane holding elements
+// 4 lane .. 4 lane + 3: signs flipped on the fp16 bits (exact), the
+// butterflies of fwht_warp, then each value times rot_scale (rounded once);
+// the raw values when the cache does not rotate.
+__device__ __forceinline__ void rotated_row_lane4(const AppendParams &p, const __half *src, int lane, float (&x)[4])
+{
+    uint2 raw = *reinterpret_cast<const uint2 *>(src + 4 * lane);
+    if (p.rotate) {
+        raw.x ^= p.sign_xor[2 * lane];
+        raw.y ^= p.sign_xor[2 * lane + 1];
+    }
+    const float2 a = __half22float2(bits_h2(raw.x)), b = __half22float2(bits_h2(raw.y));
+    x[0] = a.x;
+    x[1] = a.y;
+    x[2] = b.x;
+    x[3] = b.y;
+    if (p.rotate) {
+        fwht_warp<128>(x, lane);
+#pragma unroll
+        for (int e = 0; e < 4; e++) x[e] = __fmul_rn(x[e], p.rot_scale);
+    }
+}
+
 }  // namespace kvq

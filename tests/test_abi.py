@@ -37,6 +37,8 @@ CONFIGS = [
     dict(num_q_heads=64, num_kv_heads=8, head_dim=128, num_pages=3),
     dict(num_q_heads=32, num_kv_heads=8, head_dim=128, k_fmt=3, v_fmt=3, k_group=4, v_group=4),
     dict(num_q_heads=8, num_kv_heads=1, head_dim=128, k_fmt=3, v_fmt=3, k_group=4, v_group=4, num_pages=5),
+    dict(num_q_heads=32, num_kv_heads=8, head_dim=128, k_fmt=4, v_fmt=4, k_group=16, v_group=16),
+    dict(num_q_heads=32, num_kv_heads=8, head_dim=128, k_fmt=4, v_fmt=4, k_group=16, v_group=16, scale_search=1),
 ]
 
 
@@ -56,6 +58,10 @@ def test_pool_bytes_matches_oracle_layout(kw):
     dict(k_fmt=3, v_fmt=3, k_group=4, v_group=4, head_dim=64, num_q_heads=8, num_kv_heads=2),
     dict(k_fmt=3, v_fmt=3, k_group=4, v_group=4, bound_block_tokens=64),
     dict(k_fmt=3, v_fmt=3, k_group=4, v_group=4, scale_search=1),
+    # NVFP4: keys and values both, group 16, head_dim 128, no descriptors
+    dict(k_fmt=4, k_group=16), dict(k_fmt=4, v_fmt=4, k_group=16, v_group=32),
+    dict(k_fmt=4, v_fmt=4, k_group=16, v_group=16, head_dim=64, num_q_heads=8, num_kv_heads=2),
+    dict(k_fmt=4, v_fmt=4, k_group=16, v_group=16, bound_block_tokens=64),
 ])
 def test_invalid_configs_have_no_pool(bad):
     kw = dict(num_q_heads=32, num_kv_heads=8, head_dim=128, num_pages=4)

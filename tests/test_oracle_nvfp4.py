@@ -50,6 +50,7 @@ def test_e2m1_grid_ties_and_saturation():
     assert O.e2m1_rn([-0.75, -5.0]).tolist() == [8 | 2, 8 | 6]
     assert O.e2m1_rn([6.5, 1e9, -7.0]).tolist() == [7, 7, 15]  # saturating at 6
     assert O.e2m1_rn([0.0, -0.0, -0.2]).tolist() == [0, 0, 0]  # zero is code 0
+    assert O.e2m1_rn([np.inf, -np.inf, np.nan]).tolist() == [7, 15, 0]
 
 
 def test_e2m1_codes_are_nearest_by_brute_force():

@@ -26,6 +26,8 @@ Recipes (numpy ``default_rng``; every stream is keyed by (seed, stream id)):
               N(0,1) + 14*u of their kv head.
   hqmq        llama's geometry, distributions and context with the HQMQ codec
               for K and V.
+  nvfp4       llama's geometry, distributions and context, rotated, NVFP4 K and
+              V with ScaleSearch on the E4M3 scales.
   int2        prefill of 65536 tokens x 8 kv heads x d=128 per sequence, K and
               V ~ Laplace(0,1) with 1% of elements x30; 2-bit g128, clip 0.9;
               decode B=4, Hq=32, T=65536 (four independent prefills).
@@ -38,7 +40,7 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-INT4_ASYM, INT8_SYM, INT2_ASYM, HQMQ_FMT = 0, 1, 2, 3
+INT4_ASYM, INT8_SYM, INT2_ASYM, HQMQ_FMT, NVFP4_FMT = 0, 1, 2, 3, 4
 PAGE_TOKENS = 16
 
 # stream ids
@@ -118,6 +120,13 @@ def hqmq(T: int = 32768) -> Workload:
                                 "radii, Med3x fp16 outliers)")
 
 
+def nvfp4(T: int = 32768, search: int = 1) -> Workload:
+    return Workload(f"nvfp4-llama3-8b-layer-T{T}", 1, 32, 8, 128, [T], k_fmt=NVFP4_FMT, v_fmt=NVFP4_FMT, k_group=16,
+                    v_group=16, dist="llama", seed=7, steps=1, scale_search=search,
+                    description="batch 1, 32/8 heads, head_dim 128, llama's K/V, rotated, NVFP4 K and V (e2m1 codes, "
+                                "an E4M3 scale per 16 elements, ScaleSearch on the scales)")
+
+
 def int2(B: int = 4, T: int = 65536) -> Workload:
     return Workload(f"int2-g128-clip0.9-B{B}-T{T}", B, 32, 8, 128, [T] * B, k_fmt=INT2_ASYM, v_fmt=INT2_ASYM,
                     k_group=128, v_group=128, clip=0.9, dist="laplace", seed=4, steps=1,
@@ -126,7 +135,7 @@ def int2(B: int = 4, T: int = 65536) -> Workload:
 
 
 ALL = {"tiny": tiny, "llama": llama, "paged": paged, "certified": certified, "ladder": ladder, "int2": int2,
-       "hqmq": hqmq}
+       "hqmq": hqmq, "nvfp4": nvfp4}
 
 
 def scaled(wl: Workload, ctx, steps: int = 1) -> Workload:
