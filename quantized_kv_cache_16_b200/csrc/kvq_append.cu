@@ -478,8 +478,9 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(const __grid_
 template <int D, int KF, int VF, bool SEARCH>
 cudaError_t launch_one_s(const AppendParams &p, long long want, int num_sms, cudaStream_t st)
 {
-    static int resident = 0;
-    if (resident == 0) {
+    static DeviceOnce once;
+    static int resident = 1;
+    if (once.needed()) {
         cudaError_t e = cudaFuncSetAttribute(append_kernel<D, KF, VF, SEARCH>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, AppendSmem<D>::BYTES);
         if (e != cudaSuccess) return e;
@@ -488,6 +489,7 @@ cudaError_t launch_one_s(const AppendParams &p, long long want, int num_sms, cud
                                                           AppendSmem<D>::BYTES);
         if (e != cudaSuccess) return e;
         resident = n < 1 ? 1 : (n > 2 ? 2 : n);
+        once.mark();
     }
     const long long cap = (long long)resident * num_sms;
     const int blocks = (int)(want < cap ? want : cap);

@@ -613,17 +613,17 @@ cudaError_t launch_cert_blocks(const CertParams &p, int batch, cudaStream_t s)
 
 cudaError_t launch_cert_select(const CertParams &p, int batch, cudaStream_t s)
 {
-    static bool configured[2] = {false, false};
+    static DeviceOnce once[2];
     const int di = p.L.d == 64 ? 0 : 1;
     const size_t smem = (size_t)p.sort_cap * sizeof(unsigned long long);
-    if (!configured[di]) {
+    if (once[di].needed()) {
         const cudaError_t e =
             di ? cudaFuncSetAttribute(cert_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       kCertMaxBlocks * (int)sizeof(unsigned long long))
                : cudaFuncSetAttribute(cert_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       kCertMaxBlocks * (int)sizeof(unsigned long long));
         if (e != cudaSuccess) return e;
-        configured[di] = true;
+        once[di].mark();
     }
     const dim3 grid(p.L.hkv, batch);
     return di ? launch_pdl(cert_select_kernel<128>, grid, kSelThreads, smem, s, p)
@@ -633,13 +633,13 @@ cudaError_t launch_cert_select(const CertParams &p, int batch, cudaStream_t s)
 template <int D, int G, bool WIN>
 cudaError_t launch_promote_t(const CertParams &p, int batch, cudaStream_t s)
 {
-    static bool configured = false;
-    if (!configured) {
+    static DeviceOnce once;
+    if (once.needed()) {
         const int cap = kPromWarps * G * 3 * D * (int)sizeof(float);
         const cudaError_t e =
             cudaFuncSetAttribute(cert_promote_kernel<D, G, WIN>, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
         if (e != cudaSuccess) return e;
-        configured = true;
+        once.mark();
     }
     const size_t smem = (size_t)kPromWarps * p.L.g * 3 * D * sizeof(float);
     const dim3 grid(p.n_chunks, p.L.hkv, batch);

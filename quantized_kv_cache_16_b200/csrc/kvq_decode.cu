@@ -1163,12 +1163,12 @@ template <int D, int KF, int VF, bool G8>
 cudaError_t launch_t(const DecodeParams &p, dim3 grid, cudaStream_t s)
 {
     using C = Cfg<KF, VF, D, G8>;
-    static bool configured = false;
-    if (!configured) {
+    static DeviceOnce once;
+    if (once.needed()) {
         cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, KF, VF, G8>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
-        configured = true;
+        once.mark();
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;

@@ -716,12 +716,12 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
 template <int G>
 cudaError_t launch_hq_decode_g(const DecodeParams &p, dim3 grid, cudaStream_t s)
 {
-    static bool configured = false;
-    if (!configured) {
+    static DeviceOnce once;
+    if (once.needed()) {
         const cudaError_t e =
             cudaFuncSetAttribute(hqmq_decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHqSmem);
         if (e != cudaSuccess) return e;
-        configured = true;
+        once.mark();
     }
     if (p.n_splits > kHqMaxSplits || p.L.chunk_bytes != kHqChunk) return cudaErrorInvalidValue;
     hqmq_decode_kernel<G><<<grid, kHqThreads, kHqSmem, s>>>(p);

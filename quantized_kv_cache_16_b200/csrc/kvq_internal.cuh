@@ -259,6 +259,27 @@ inline size_t decode_counter_bytes(int batch, int hkv)
 }
 constexpr int kDecodeThreads = kDecodeWarps * 32;
 
+// One-time setup per device (a kernel's shared-memory attribute is a
+// property of the device it was set on): a bit per device, 64 devices.
+struct DeviceOnce {
+    unsigned long long done = 0;
+    static int device()
+    {
+        int dev = 0;
+        return cudaGetDevice(&dev) == cudaSuccess ? dev : 0;
+    }
+    bool needed() const
+    {
+        const int dev = device();
+        return dev >= 64 || !((done >> dev) & 1ull);
+    }
+    void mark()
+    {
+        const int dev = device();
+        if (dev < 64) done |= 1ull << dev;
+    }
+};
+
 // ------------------------------------------------------------- device util ---
 
 __device__ __forceinline__ void set_status(const unsigned char *pool, unsigned int code)

@@ -541,15 +541,15 @@ __global__ void __launch_bounds__(kPromThreads) ladder_dense_kernel(const __grid
 
 cudaError_t launch_ladder_select(const CertParams &p, int batch, cudaStream_t s)
 {
-    static bool configured[2] = {false, false};
+    static DeviceOnce once[2];
     const int di = p.L.d == 64 ? 0 : 1;
-    if (!configured[di]) {
+    if (once[di].needed()) {
         const int cap = kCertMaxBlocks * (int)(sizeof(unsigned long long) + 1);
         const cudaError_t e =
             di ? cudaFuncSetAttribute(ladder_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, cap)
                : cudaFuncSetAttribute(ladder_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
         if (e != cudaSuccess) return e;
-        configured[di] = true;
+        once[di].mark();
     }
     const size_t smem = (size_t)p.sort_cap * (sizeof(unsigned long long) + 1);
     const dim3 grid(p.L.hkv, batch);
@@ -559,9 +559,9 @@ cudaError_t launch_ladder_select(const CertParams &p, int batch, cudaStream_t s)
 
 cudaError_t launch_ladder_finish(const CertParams &p, int batch, cudaStream_t s)
 {
-    static bool configured[2] = {false, false};
+    static DeviceOnce once[2];
     const int di = p.L.d == 64 ? 0 : 1;
-    if (!configured[di]) {
+    if (once[di].needed()) {
         const int cap = kCertMaxBlocks * (int)sizeof(unsigned long long);
         const int dcap = kPromWarps * kMaxGqa * kMaxD * (int)sizeof(float);
         cudaError_t e =
@@ -571,7 +571,7 @@ cudaError_t launch_ladder_finish(const CertParams &p, int batch, cudaStream_t s)
         e = di ? cudaFuncSetAttribute(ladder_dense_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, dcap)
                : cudaFuncSetAttribute(ladder_dense_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, dcap);
         if (e != cudaSuccess) return e;
-        configured[di] = true;
+        once[di].mark();
     }
     const size_t smem = (size_t)p.sort_cap * sizeof(unsigned long long);
     const dim3 grid(p.L.hkv, batch);

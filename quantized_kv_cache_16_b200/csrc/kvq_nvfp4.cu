@@ -490,12 +490,12 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
 template <int G>
 cudaError_t launch_nv_decode_g(const DecodeParams &p, dim3 grid, cudaStream_t s)
 {
-    static bool configured = false;
-    if (!configured) {
+    static DeviceOnce once;
+    if (once.needed()) {
         const cudaError_t e =
             cudaFuncSetAttribute(nvfp4_decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kNvSmem);
         if (e != cudaSuccess) return e;
-        configured = true;
+        once.mark();
     }
     if (p.n_splits > kNvMaxSplits || p.L.chunk_bytes != kNvChunk) return cudaErrorInvalidValue;
     nvfp4_decode_kernel<G><<<grid, kNvThreads, kNvSmem, s>>>(p);
