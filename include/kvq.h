@@ -360,6 +360,26 @@ kvq_status kvq_decode_step(kvq_cache *cache, const void *k_new, const void *v_ne
                            const int32_t *ctx_lens, int32_t batch, float softmax_scale, void *workspace,
                            size_t ws_bytes, void *out, void *stream);
 
+/* Bytes of the host record of kvq_decode_step_host for `batch` sequences:
+ * q fp16 [batch][Hq][d], then k_new fp16 [batch][Hkv][d], v_new fp16
+ * [batch][Hkv][d], slot_mapping int32 [batch], ctx_lens int32 [batch], each
+ * section starting at a multiple of 16 bytes.  0 for a NULL cache or
+ * batch < 1. */
+size_t kvq_step_record_bytes(const kvq_cache *cache, int32_t batch);
+
+/* One decode step from and to host memory: enqueues on `stream` the copy of
+ * the pinned host record `host_in` (kvq_step_record_bytes long, layout
+ * above) into the device buffer `dev_rec` (as long, 16-byte aligned) and
+ * kvq_decode_step on that record, whose kernel writes the fp32 output
+ * [batch][Hq][d] straight to pinned `host_out` (16-byte aligned) through
+ * its device mapping (no separate copy back).  Synchronise the stream
+ * before reading host_out.  block_table stays in device memory.  Host
+ * buffers that are not page-locked (cudaHostAlloc / cudaHostRegister)
+ * return KVQ_ERR_INVALID_ARG, as do the cases kvq_decode_step rejects. */
+kvq_status kvq_decode_step_host(kvq_cache *cache, const void *host_in, void *dev_rec, const int32_t *block_table,
+                                int32_t max_pages_per_seq, int32_t batch, float softmax_scale, void *workspace,
+                                size_t ws_bytes, void *host_out, void *stream);
+
 /* Decode attention that allocates nothing and takes no workspace, for
  * callers that cannot allocate device memory: an engine that reserves all of
  * the GPU's memory up front for its own pools (so any later cudaMalloc fails

@@ -25,7 +25,7 @@ PAGE_TOKENS = 16
 EXPORTS = (
     "kvq_pool_bytes", "kvq_create_cache", "kvq_destroy_cache", "kvq_append", "kvq_reset_pages",
     "kvq_decode_workspace_bytes", "kvq_decode_attn", "kvq_decode_certified", "kvq_decode_windows",
-    "kvq_decode_windows_workspace_bytes", "kvq_decode_step",
+    "kvq_decode_windows_workspace_bytes", "kvq_decode_step", "kvq_step_record_bytes", "kvq_decode_step_host",
     "kvq_decode_attn_static", "kvq_dequant_debug", "kvq_sync_status",
     "kvq_status_string",
 )
@@ -91,6 +91,8 @@ def lib() -> C.CDLL:
             "kvq_decode_windows": (i32, [P, P, P, i32, P, i32, C.c_float, P, P, i32, i32, P, sz, P, P]),
             "kvq_decode_windows_workspace_bytes": (sz, [P, i32, i32]),
             "kvq_decode_step": (i32, [P, P, P, P, P, P, i32, P, i32, C.c_float, P, sz, P, P]),
+            "kvq_step_record_bytes": (sz, [P, i32]),
+            "kvq_decode_step_host": (i32, [P, P, P, P, i32, i32, C.c_float, P, sz, P, P]),
             "kvq_decode_attn_static": (i32, [P, P, P, i32, P, i32, C.c_float, P, P]),
             "kvq_dequant_debug": (i32, [P, P, i32, P, P, P, P, P]),
             "kvq_sync_status": (i32, [P]),
@@ -201,6 +203,21 @@ def kvq_decode_step(cache, k_new, v_new, slot_mapping, q, block_table, max_pages
            lib().kvq_decode_step(cache, _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(q), _ptr(block_table),
                                  max_pages_per_seq, _ptr(ctx_lens), batch, softmax_scale, _ptr(workspace), ws_bytes,
                                  _ptr(out), _stream(stream)))
+
+
+def kvq_step_record_bytes(cache, batch: int) -> int:
+    return int(lib().kvq_step_record_bytes(cache, batch))
+
+
+def kvq_decode_step_host(cache, host_in, dev_rec, block_table, max_pages_per_seq: int, batch: int,
+                         softmax_scale: float, workspace, ws_bytes: int, host_out, stream=None) -> None:
+    """host_in / host_out: pinned host tensors (or addresses); the record
+    layout is kvq_step_record_bytes' (q, k_new, v_new, slots, ctx_lens);
+    dev_rec: a device buffer of that size."""
+    _check("kvq_decode_step_host",
+           lib().kvq_decode_step_host(cache, _ptr(host_in), _ptr(dev_rec), _ptr(block_table), max_pages_per_seq,
+                                      batch, softmax_scale, _ptr(workspace), ws_bytes, _ptr(host_out),
+                                      _stream(stream)))
 
 
 def kvq_decode_attn_static(cache, q, block_table, max_pages_per_seq: int, ctx_lens, batch: int,

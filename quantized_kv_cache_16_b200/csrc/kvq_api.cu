@@ -706,6 +706,68 @@ kvq_status kvq_decode_step(kvq_cache *c, const void *k_new, const void *v_new, c
                        softmax_scale, nullptr, workspace, ws_bytes, out, nullptr, stream);
 }
 
+}  // extern "C"
+
+namespace {
+
+struct StepRecord {
+    size_t q, k, v, slot, ctx, bytes;
+};
+
+size_t up16(size_t n) { return (n + 15) / 16 * 16; }
+
+StepRecord step_record(const kvq_cache *c, int batch)
+{
+    StepRecord r{};
+    const size_t b = (size_t)batch, d = (size_t)c->L.d;
+    r.q = 0;
+    r.k = up16(b * c->L.hq * d * 2);
+    r.v = r.k + up16(b * c->L.hkv * d * 2);
+    r.slot = r.v + up16(b * c->L.hkv * d * 2);
+    r.ctx = r.slot + up16(b * 4);
+    r.bytes = r.ctx + up16(b * 4);
+    return r;
+}
+
+bool pinned_host(const void *p)
+{
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeHost;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kvq_step_record_bytes(const kvq_cache *c, int32_t batch)
+{
+    if (!c || batch < 1) return 0;
+    return step_record(c, batch).bytes;
+}
+
+kvq_status kvq_decode_step_host(kvq_cache *c, const void *host_in, void *dev_rec, const int32_t *block_table,
+                                int32_t max_pages_per_seq, int32_t batch, float softmax_scale, void *workspace,
+                                size_t ws_bytes, void *host_out, void *stream)
+{
+    if (!c || batch < 1 || !host_in || !dev_rec || !host_out || !aligned(dev_rec, 16)) return KVQ_ERR_INVALID_ARG;
+    if (!pinned_host(host_in) || !pinned_host(host_out)) return KVQ_ERR_INVALID_ARG;
+    void *o = const_cast<void *>(device_view(host_out));
+    if (!o || !aligned(o, 16)) return KVQ_ERR_INVALID_ARG;
+    if (c->cfg.scale_search || c->L.hq_tab || c->L.k_fmt == KVQ_NVFP4) return KVQ_ERR_UNSUPPORTED;
+    const StepRecord r = step_record(c, batch);
+    if (cudaMemcpyAsync(dev_rec, host_in, r.bytes, cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return KVQ_ERR_CUDA;
+    const unsigned char *d = static_cast<const unsigned char *>(dev_rec);
+    return decode_impl(c, d + r.k, d + r.v, reinterpret_cast<const int32_t *>(d + r.slot), d + r.q, block_table,
+                       max_pages_per_seq, reinterpret_cast<const int32_t *>(d + r.ctx), batch, softmax_scale, nullptr,
+                       workspace, ws_bytes, o, nullptr, stream);
+}
+
 kvq_status kvq_dequant_debug(kvq_cache *c, const int32_t *slots, int32_t n, float *k_out, float *v_out,
                              uint8_t *codes_out, uint16_t *meta_out, void *stream)
 {

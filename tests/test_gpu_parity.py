@@ -194,3 +194,56 @@ def test_decode_step_rejects_a_slot_off_the_last_position():
                     torch.from_numpy(W.queries(wl, 0)).cuda(), pair.block_table(), pair.ctx(1))
     assert pair.cache.sync_status() == 4  # KVQ_ERR_OUT_OF_RANGE
     assert np.array_equal(pair.cache.pool.cpu().numpy()[256:], before[256:])
+
+
+def _host_record(cache, wl, step, slots, ctx):
+    """The pinned host record of kvq_decode_step_host (q, k_new, v_new, slots,
+    ctx lengths, sections 16-byte aligned)."""
+    import torch
+    import quantized_kv_cache_16_b200 as K
+    k, v = W.step_kv(wl, step)
+    q = W.queries(wl, step)
+    up = lambda n: (n + 15) // 16 * 16
+    parts = [q.view(np.uint8).ravel(), k.view(np.uint8).ravel(), v.view(np.uint8).ravel(),
+             np.asarray(slots, np.int32).view(np.uint8), np.asarray(ctx, np.int32).view(np.uint8)]
+    rec = np.zeros(K.kvq_step_record_bytes(cache.handle, wl.B), np.uint8)
+    off = 0
+    for a in parts:
+        rec[off:off + a.size] = a
+        off += up(a.size)
+    assert off == rec.size
+    return torch.from_numpy(rec).pin_memory()
+
+
+def test_decode_step_host_equals_the_device_step():
+    """kvq_decode_step_host (the pinned host record copied in, the kernel
+    writing the pinned host output through its device mapping) stores the
+    same bytes and returns the same output as kvq_decode_step on device
+    copies of the same inputs; pageable host memory is refused."""
+    import torch
+    import quantized_kv_cache_16_b200 as K
+    wl = W.scaled(W.llama(), [1000, 31, 16])
+    host = build_pair(wl, extra_tokens=2, oracle=False)
+    devp = build_pair(wl, extra_tokens=2, oracle=False)
+    ws = host.cache.workspace_for(wl.B, host.pages.block_table.shape[1])
+    h_out = torch.empty((wl.B, wl.Hq, wl.d), dtype=torch.float32).pin_memory()
+    d_rec = torch.empty(K.kvq_step_record_bytes(host.cache.handle, wl.B), dtype=torch.uint8, device="cuda")
+    for step in range(2):
+        slots = np.array([host.pages.slot(b, wl.ctx[b] + step) for b in range(wl.B)], np.int32)
+        ctx = [t + step + 1 for t in wl.ctx]
+        h_in = _host_record(host.cache, wl, step, slots, ctx)
+        K.kvq_decode_step_host(host.cache.handle, h_in, d_rec, host.block_table(), host.pages.block_table.shape[1],
+                               wl.B, 0.0, ws, ws.numel(), h_out)
+        torch.cuda.synchronize()
+        k, v = W.step_kv(wl, step)
+        want = devp.cache.step(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(),
+                               torch.from_numpy(slots).cuda(), torch.from_numpy(W.queries(wl, step)).cuda(),
+                               devp.block_table(), devp.ctx(step + 1))
+        assert np.array_equal(h_out.numpy(), want.cpu().numpy())
+        assert np.array_equal(host.cache.pool.cpu().numpy()[256:], devp.cache.pool.cpu().numpy()[256:])
+    assert host.cache.sync_status() == 0
+    pageable = torch.zeros_like(h_out)
+    with pytest.raises(K.KvqError) as e:
+        K.kvq_decode_step_host(host.cache.handle, h_in, d_rec, host.block_table(), host.pages.block_table.shape[1],
+                               wl.B, 0.0, ws, ws.numel(), pageable)
+    assert e.value.status == K.KVQ_ERR_INVALID_ARG
