@@ -15,10 +15,11 @@
 // single fp16 operands straight from the hardware conversions: each lane
 // turns a byte of two codes into an fp16 pair and multiplies it by its
 // block's scale.  The query and the softmax weights are hi + lo fp16 pairs.
-// The layout of the fragments is the HQMQ decode's: scores K Q^T (M = the
-// page's 16 tokens, N = 8 heads), output V^T P^T (M = dims), with the
-// contraction index and the output rows permuted so that a lane reads whole
-// 4-element groups of a row.
+// Fragments as in the HQMQ decode (scores K Q^T with M = the page's 16
+// tokens and N = 8 heads, output V^T P^T with M = dims), but the contraction
+// index and the output rows are permuted so that a lane reads one 16-byte
+// span of each of its two key rows and one 8-byte span of each of its four
+// value rows.
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <math.h>
@@ -265,18 +266,26 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
         for (int e = 0; e < 4; e++) sq[warp * kNvD + lane * 4 + e] = x[e] * p.qscale;
     }
     __syncthreads();
-    // Fragments (r = lane / 4, j = lane % 4): k-slice ks position {2j, 2j+1,
-    // 2j+8, 2j+9} = dims 16 ks + 4j .. + 3 (lane reads 2 code bytes of tokens
-    // r and r + 8); m-tiles 2i, 2i + 1 rows r / r + 8 = dims 0 / 1 and 2 / 3 of
-    // the group 32 i + 4 r .. + 3 (lane reads it for tokens 2j, 2j+1, 2j+8,
-    // 2j+9); the score fragments become P^T by two 8x8 transposes.
+    // Fragments (r = lane / 4, j = lane % 4).  Rows of the score tile and
+    // the contraction index of PV are the page's tokens in the order
+    // tok(m) = m ^ ((m >> 1) & 1), so the four token rows a value load of a
+    // half-warp touches alternate between the two bank halves of a 128-byte
+    // line (64-byte rows).  Scores S^T = K Q^T: k-slice ks position {2j,
+    // 2j+1, 2j+8, 2j+9} = dims 32j + 4ks .. + 3, so a lane's eight slices are
+    // the 16 code bytes [16j, 16j + 16) of tokens tok(r) and tok(r + 8)
+    // (one conflict-free 16-byte load each).  Output O^T = V^T P^T: m-tiles
+    // 2ib, 2ib + 1 rows r / r + 8 = dims 0 / 1 and 2 / 3 of 16r + 4ib, so a
+    // lane's four tile pairs are the 8 code bytes [8r, 8r + 8) of tokens
+    // tok(2j), tok(2j+1), tok(2j+8), tok(2j+9).  The score fragments become
+    // P^T by two 8x8 transposes.
     const int r = lane >> 2, j = lane & 3;
+    auto tok = [](int m) { return m ^ ((m >> 1) & 1); };
     uint32_t qb[8][2], ql[8][2];
 #pragma unroll
     for (int ks = 0; ks < 8; ks++) {
         qb[ks][0] = qb[ks][1] = ql[ks][0] = ql[ks][1] = 0u;
         if (r < g) {
-            const float4 q4 = *reinterpret_cast<const float4 *>(sq + r * kNvD + 16 * ks + 4 * j);
+            const float4 q4 = *reinterpret_cast<const float4 *>(sq + r * kNvD + 32 * j + 4 * ks);
             split_h2(q4.x, q4.y, qb[ks][0], ql[ks][0]);
             split_h2(q4.z, q4.w, qb[ks][1], ql[ks][1]);
         }
@@ -285,6 +294,8 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
     float acc[8][4];
 #pragma unroll
     for (int mt = 0; mt < 8; mt++) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    const int ta = tok(r), tb = tok(r + 8);
+    const int tv[4] = {tok(2 * j), tok(2 * j + 1), tok(2 * j + 8), tok(2 * j + 9)};
 
     for (int i = 0; i < npg; i++) {
         const int st = i % kNvStages;
@@ -299,17 +310,20 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
         const int t_page = (p_begin + i) * kPageTokens;
         const int nvalid = ((vbits >> st) & 1u) ? min(kPageTokens, T - t_page) : 0;
 
-        // ---- scores of tokens r, r + 8 for heads 2j, 2j + 1 ----
+        // ---- scores of tokens tok(r), tok(r + 8) for heads 2j, 2j + 1 ----
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        const bool va = ta < nvalid, vb = tb < nvalid;
         {
-            const bool va = r < nvalid, vb = r + 8 < nvalid;
-            const unsigned char *ra = chunk + L.k_codes + r * kNvRowCode, *rb = ra + 8 * kNvRowCode;
-            const unsigned char *ma = chunk + L.k_meta + r * kNvRowMeta, *mb = ma + 8 * kNvRowMeta;
+            const uint4 ka = *reinterpret_cast<const uint4 *>(chunk + L.k_codes + ta * kNvRowCode + 16 * j);
+            const uint4 kb = *reinterpret_cast<const uint4 *>(chunk + L.k_codes + tb * kNvRowCode + 16 * j);
+            const uint32_t sa2 = *reinterpret_cast<const uint16_t *>(chunk + L.k_meta + ta * kNvRowMeta + 2 * j);
+            const uint32_t sb2 = *reinterpret_cast<const uint16_t *>(chunk + L.k_meta + tb * kNvRowMeta + 2 * j);
+            const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w}, wb[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
             for (int ks = 0; ks < 8; ks++) {
-                const uint32_t ca = *reinterpret_cast<const uint16_t *>(ra + 8 * ks + 2 * j);
-                const uint32_t cb = *reinterpret_cast<const uint16_t *>(rb + 8 * ks + 2 * j);
-                const __half2 sa = scale_h2(ma[ks]), sb = scale_h2(mb[ks]);
+                const __half2 sa = scale_h2((uint8_t)(sa2 >> (ks < 4 ? 0 : 8)));
+                const __half2 sb = scale_h2((uint8_t)(sb2 >> (ks < 4 ? 0 : 8)));
+                const uint32_t ca = wa[ks >> 1] >> (16 * (ks & 1)), cb = wb[ks >> 1] >> (16 * (ks & 1));
                 uint32_t a[4];
                 a[0] = va ? h2_bits(fp4x2_scaled(ca, sa)) : 0u;
                 a[1] = vb ? h2_bits(fp4x2_scaled(cb, sb)) : 0u;
@@ -349,7 +363,7 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
             acc[mt][2] *= al0;
             acc[mt][3] *= al1;
         }
-        uint32_t pb[2][2];  // P^T (hi, lo): tokens 2j, 2j+1 (b0) and 2j+8, 2j+9 (b1) of head r
+        uint32_t pb[2][2];  // P^T (hi, lo): tokens tok(2j), tok(2j+1) (b0) and tok(2j+8), tok(2j+9) (b1) of head r
         {
             uint32_t t[2][2];
             split_h2(p0, p1, t[0][0], t[1][0]);
@@ -360,20 +374,27 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
                 for (int k = 0; k < 2; k++)
                     asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(pb[hl][k]) : "r"(t[hl][k]));
         }
-        // ---- values: dims 32 ib + 4r .. + 3 of tokens 2j, 2j+1, 2j+8, 2j+9 ----
+        // ---- values: dims 16r .. 16r + 15 of the lane's four tokens ----
         {
-            const int tk[4] = {2 * j, 2 * j + 1, 2 * j + 8, 2 * j + 9};
+            uint2 cv[4];
+            __half2 s2[4];
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                cv[u] = *reinterpret_cast<const uint2 *>(chunk + L.v_codes + tv[u] * kNvRowCode + 8 * r);
+                s2[u] = scale_h2(chunk[L.v_meta + tv[u] * kNvRowMeta + r]);
+                if (tv[u] >= nvalid) {  // zero codes and scale (a stale scale byte may be NaN)
+                    cv[u] = make_uint2(0u, 0u);
+                    s2[u] = __float2half2_rn(0.f);
+                }
+            }
 #pragma unroll
             for (int ib = 0; ib < 4; ib++) {
                 __half2 v01[4], v23[4];
 #pragma unroll
                 for (int u = 0; u < 4; u++) {
-                    const unsigned char *row = chunk + L.v_codes + tk[u] * kNvRowCode;
-                    const uint32_t cv = *reinterpret_cast<const uint16_t *>(row + 16 * ib + 2 * r);
-                    const __half2 s2 = scale_h2(chunk[L.v_meta + tk[u] * kNvRowMeta + 2 * ib + (r >> 2)]);
-                    const bool ok_t = tk[u] < nvalid;
-                    v01[u] = ok_t ? fp4x2_scaled(cv, s2) : __float2half2_rn(0.f);
-                    v23[u] = ok_t ? fp4x2_scaled(cv >> 8, s2) : __float2half2_rn(0.f);
+                    const uint32_t w = ((ib < 2 ? cv[u].x : cv[u].y) >> (16 * (ib & 1))) & 0xFFFFu;
+                    v01[u] = fp4x2_scaled(w, s2[u]);
+                    v23[u] = fp4x2_scaled(w >> 8, s2[u]);
                 }
                 uint32_t a[4];
                 a[0] = h2_bits(__lows2half2(v01[0], v01[1]));
@@ -403,7 +424,7 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
         if (h < g) {
 #pragma unroll
             for (int ib = 0; ib < 4; ib++)
-                *reinterpret_cast<float4 *>(wacc + (warp * G + h) * kNvD + 32 * ib + 4 * r) =
+                *reinterpret_cast<float4 *>(wacc + (warp * G + h) * kNvD + 16 * r + 4 * ib) =
                     make_float4(acc[2 * ib][hh], acc[2 * ib][2 + hh], acc[2 * ib + 1][hh], acc[2 * ib + 1][2 + hh]);
             if (r == 0) {
                 wm[warp][h] = hh ? m1 : m0;
