@@ -169,3 +169,23 @@ def test_tie_rules_of_med3x():
     y2[0, 0::4] = 1.0
     y2[0, 4 * 2], y2[0, 4 * 7] = 3.0, 5.0
     assert int(O.hqmq_quantize_rows(y2, S)[2][0]) == 1 << 7
+
+
+def test_covering_rate_of_the_product_codebook():
+    """The page's Proposition 3.1: the product codebook of 24 Hurwitz units
+    and S random unit quaternions covers S^3 at the rate O((24 S)^(-1/3)).
+    With the first S of a generated codebook (S = 32 .. 1024), the mean angle
+    from a random direction to its nearest codeword falls with slope -1/3 in
+    log-log."""
+    rng = np.random.default_rng(0)
+    u = rng.standard_normal((3000, 4))
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    S = O.hqmq_codebook(3, 0, 0).astype(np.float64)
+    xs, ys = [], []
+    for n in (32, 64, 128, 256, 512, 1024):
+        C = hamilton(P[:, None, :], S[None, :n, :]).reshape(-1, 4)
+        theta = np.arccos(np.clip(np.max(u @ C.T, axis=1), -1, 1))
+        xs.append(np.log(24 * n))
+        ys.append(np.log(theta.mean()))
+    slope = np.polyfit(xs, ys, 1)[0]
+    assert -0.38 < slope < -0.29, slope
