@@ -33,7 +33,6 @@
 // dominates: the path is bound by instruction issue, not by HBM.
 #include <math.h>
 
-#include "kvq_cert.cuh"
 #include "kvq_internal.cuh"
 #include "kvq_warp.cuh"
 
@@ -344,12 +343,12 @@ __device__ __forceinline__ uint32_t hq_field(const unsigned char *row, int blk)
     return __funnelshift_r(lo, hi, sh) & kHqFieldMask;
 }
 
-// Block `lane` of a row: (radius code x step) x q_p q_s with q_s from the
+// Block `blk` of a row: (radius code x step) x q_p q_s with q_s from the
 // codebook and q_p from the unit table (both in shared memory), or the fp16
 // outlier values.  meta = the row's meta (shared memory): step | 0, outlier
 // mask, two outlier slots.  The unit table holds 8 copies of the 24 units,
-// copy r of unit p at p * 8 + r: lane reads copy lane % 8, so the eight
-// lanes of each 16-byte load phase hit eight different bank groups.
+// copy r of unit p at p * 8 + r: a lane reads copy `cpy` = lane % 8, so the
+// eight lanes of each 16-byte load phase hit eight different bank groups.
 __device__ __forceinline__ void hq_block(uint32_t f, const unsigned char *meta, const float4 *S, const float4 *units,
                                          int blk, int cpy, float (&c)[4])
 {
