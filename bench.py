@@ -685,7 +685,8 @@ def nvfp4_leg(steps: int, T: int = 0):
     d=128, context 32768, rotated, ScaleSearch on the E4M3 scales): the bulk
     append of the whole context and a one-token append timed with events;
     the decode replayed in a CUDA graph over four cache copies (151 MB, above
-    L2), beside the same decode of a cache without ScaleSearch."""
+    L2), beside the same decode of a cache without ScaleSearch and that
+    cache's fused append + decode step (kvq_decode_step, one launch)."""
     import torch
 
     import quantized_kv_cache_16_b200 as K
@@ -740,22 +741,32 @@ def nvfp4_leg(steps: int, T: int = 0):
                               ws.numel(), out, None, stream)
 
         d_us = _graph_time(dec, steps, stream)
+        step_us = None
+        if not search:  # the fused append + decode step (default scales): the token at position T
+            ctx1 = torch.tensor([T + 1], dtype=torch.int32, device=dev)
+            st_slots = [torch.from_numpy(t.slots(0, T, T + 1)).to(dev) for t in tabs]
+
+            def step(s):
+                K.kvq_decode_step(cache.handle, kn, vn, st_slots[s % copies], qs[s % nq], bts[s % copies], max_pages,
+                                  ctx1, wl.B, 0.0, ws, ws.numel(), out, stream)
+
+            step_us = _graph_time(step, steps, stream)
         assert cache.sync_status() == 0
-        res[search] = (min(bulk_ms), tok_us, d_us)
+        res[search] = (min(bulk_ms), tok_us, d_us, step_us)
         del cache
     del kd, vd
     row_bytes = wl.d // 2 + wl.d // 16  # e2m1 codes + E4M3 scales
     kv_bytes = T * wl.Hkv * 2 * row_bytes
     rows = 2 * T * wl.Hkv
     peak, kind = measured_peaks()
-    bulk, tok_us, d_us = res[1]
+    bulk, tok_us, d_us, _ = res[1]
     return {"workload": f"NVFP4 K/V, B=1, 32/8 heads, d=128, context {T}, rotated, ScaleSearch on",
             "decode_us": round(d_us, 2), "decode_gbs": round(kv_bytes / d_us / 1e3, 1),
             "decode_pct_hbm_peak": kv_bytes / d_us / 1e3 / peak, "peak_kind": kind, "cache_bytes": kv_bytes,
             "bits_per_element": row_bytes * 8 / wl.d, "bulk_append_ms": round(bulk, 3),
             "bulk_append_rows_per_s": round(rows / bulk * 1e3, 1), "token_append_us": round(tok_us, 2),
             "no_search": {"bulk_append_ms": round(res[0][0], 3), "token_append_us": round(res[0][1], 2),
-                          "decode_us": round(res[0][2], 2)},
+                          "decode_us": round(res[0][2], 2), "fused_step_us": round(res[0][3], 2)},
             "steps": steps}
 
 

@@ -82,8 +82,10 @@ typedef enum {
  * Storage (token-major rows): 64 code bytes (byte j = code[2j] |
  * code[2j+1] << 4), then per region 16 meta rows of the 8 scale bytes.  A
  * value decodes to e2m1 x scale, exact in fp16.  kvq_append, kvq_decode_attn
- * (without tier 2) and kvq_decode_attn_static serve NVFP4 caches; the other
- * decode calls return KVQ_ERR_UNSUPPORTED. */
+ * (without tier 2) and kvq_decode_attn_static serve NVFP4 caches, and
+ * kvq_decode_step / kvq_decode_step_host when scale_search is 0 (the fused
+ * append codes the new token with the default scales); the other decode
+ * calls return KVQ_ERR_UNSUPPORTED. */
 
 /* HQMQ ["Hurwitz Quaternion Multiplicative Quantization for KV Cache
  * Compression", 1-3].  A rotated row is cut into d/4 blocks x (a quaternion);

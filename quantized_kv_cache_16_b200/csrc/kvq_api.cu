@@ -480,13 +480,15 @@ kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const
     if (!q || !block_table || !ctx_lens || !out || !workspace) return KVQ_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
     if (k_new && (!v_new || !slot_mapping || !aligned(k_new, 16) || !aligned(v_new, 16))) return KVQ_ERR_INVALID_ARG;
-    if (c->L.hq_tab || c->L.k_fmt == KVQ_NVFP4) {  // HQMQ, NVFP4: own decode kernels, no fused append, no tier 2
-        if (k_new || tier2) return KVQ_ERR_UNSUPPORTED;
+    if (c->L.hq_tab || c->L.k_fmt == KVQ_NVFP4) {  // HQMQ, NVFP4: own decode kernels, no tier 2
+        if (tier2 || (k_new && c->L.hq_tab)) return KVQ_ERR_UNSUPPORTED;  // NVFP4 fuses the step's append
         if (ws_bytes < kvq_decode_workspace_bytes(c, batch, max_pages_per_seq)) return KVQ_ERR_CAPACITY;
         const SplitPlan s = plan_splits(c, batch, max_pages_per_seq);
         const float scale = softmax_scale > 0.0f ? softmax_scale : (float)(1.0 / sqrt((double)c->L.d));
-        const DecodeParams p =
-            decode_params(c, s, q, block_table, max_pages_per_seq, ctx_lens, batch, scale, workspace, out);
+        DecodeParams p = decode_params(c, s, q, block_table, max_pages_per_seq, ctx_lens, batch, scale, workspace, out);
+        p.new_k = static_cast<const __half *>(k_new);
+        p.new_v = static_cast<const __half *>(v_new);
+        p.new_slots = slot_mapping;
         c->last_stream = stream;
         const dim3 grid(s.n_splits, c->L.hkv, batch);
         return cuda_status(c->L.hq_tab ? launch_hqmq_decode(p, grid, static_cast<cudaStream_t>(stream))
@@ -757,7 +759,7 @@ kvq_status kvq_decode_step_host(kvq_cache *c, const void *host_in, void *dev_rec
     if (!pinned_host(host_in) || !pinned_host(host_out)) return KVQ_ERR_INVALID_ARG;
     void *o = const_cast<void *>(device_view(host_out));
     if (!o || !aligned(o, 16)) return KVQ_ERR_INVALID_ARG;
-    if (c->cfg.scale_search || c->L.hq_tab || c->L.k_fmt == KVQ_NVFP4) return KVQ_ERR_UNSUPPORTED;
+    if (c->cfg.scale_search || c->L.hq_tab) return KVQ_ERR_UNSUPPORTED;
     const StepRecord r = step_record(c, batch);
     if (cudaMemcpyAsync(dev_rec, host_in, r.bytes, cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream)) !=
         cudaSuccess)

@@ -88,6 +88,27 @@ __device__ __forceinline__ float block_sq_error(const float (&x)[4], float sf)
     return __fadd_rn(acc, __shfl_xor_sync(kFull, acc, 2));
 }
 
+// The default scale byte of the lane's block: E4M3 (nearest, saturating) of
+// max |x| / 6 over the block's four lanes.
+__device__ __forceinline__ int default_scale(const float (&x)[4])
+{
+    float am = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+    am = fmaxf(am, __shfl_xor_sync(kFull, am, 1));
+    am = fmaxf(am, __shfl_xor_sync(kFull, am, 2));
+    return (int)__nv_cvt_float_to_fp8(__fdiv_rn(am, 6.0f), __NV_SATFINITE, __NV_E4M3);
+}
+
+// Code the lane's four elements under scale byte sc and store them (two
+// code bytes a lane) and the block's scale byte (its first lane).
+__device__ __forceinline__ void store_row(const float (&x)[4], int sc, unsigned char *codes, unsigned char *meta,
+                                          int lane)
+{
+    uint32_t c[4];
+    lane_codes(x, e4m3_f((uint8_t)sc), c);
+    reinterpret_cast<uint16_t *>(codes)[lane] = (uint16_t)(c[0] | (c[1] << 4) | (c[2] << 8) | (c[3] << 12));
+    if ((lane & 3) == 0) meta[lane >> 2] = (unsigned char)sc;
+}
+
 // Grid: persistent CTAs, a warp codes rows r, r + all warps, ... (K rows
 // then V rows, row = token * Hkv + kv head).
 template <bool SEARCH>
@@ -110,11 +131,7 @@ __global__ void __launch_bounds__(kNvThreads) nvfp4_append_kernel(const __grid_c
         }
         float x[4];
         rotated_row_lane4(p, (tensor ? p.v : p.k) + rr * kNvD, lane, x);
-        // the block's max |x| (lanes 4k .. 4k + 3), the default scale
-        float am = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
-        am = fmaxf(am, __shfl_xor_sync(kFull, am, 1));
-        am = fmaxf(am, __shfl_xor_sync(kFull, am, 2));
-        const int b0 = (int)__nv_cvt_float_to_fp8(__fdiv_rn(am, 6.0f), __NV_SATFINITE, __NV_E4M3);
+        const int b0 = default_scale(x);  // the block's (lanes 4k .. 4k + 3)
         int best = b0;
         if constexpr (SEARCH) {
             // candidates b0 + f, f = 0, -1, 1, -2, 2, 3, 4, 5, 6: positive finite
@@ -133,14 +150,10 @@ __global__ void __launch_bounds__(kNvThreads) nvfp4_append_kernel(const __grid_c
                 }
             }
         }
-        uint32_t c[4];
-        lane_codes(x, e4m3_f((uint8_t)best), c);
         const int page = slot / kPageTokens, tok = slot % kPageTokens;
         unsigned char *chunk = p.pool + kHeaderBytes + (long long)page * L.page_bytes + (long long)kvh * L.chunk_bytes;
-        unsigned char *codes = chunk + (tensor ? L.v_codes : L.k_codes) + tok * kNvRowCode;
-        unsigned char *meta = chunk + (tensor ? L.v_meta : L.k_meta) + tok * kNvRowMeta;
-        reinterpret_cast<uint16_t *>(codes)[lane] = (uint16_t)(c[0] | (c[1] << 4) | (c[2] << 8) | (c[3] << 12));
-        if ((lane & 3) == 0) meta[lane >> 2] = (unsigned char)best;
+        store_row(x, best, chunk + (tensor ? L.v_codes : L.k_codes) + tok * kNvRowCode,
+                  chunk + (tensor ? L.v_meta : L.k_meta) + tok * kNvRowMeta, lane);
     }
 }
 
@@ -248,6 +261,38 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
         pg = __shfl_sync(kFull, pg, 0);
         vbits = (vbits & ~(1u << st)) | ((pg >= 0 ? 1u : 0u) << st);
     };
+    // fused append (decode step): the warp that owns the page of position
+    // T - 1 codes the new token's K and V rows into it (default scales)
+    // before any copy of that page
+    if (p.new_k != nullptr && T > 0 && n_pages - 1 >= p_begin && n_pages - 1 < p_begin + npg) {
+        const int pg = bt[n_pages - 1];
+        const int slot = p.new_slots[b];
+        const int tok = (T - 1) % kPageTokens;
+        if (pg < 0 || pg >= L.num_pages || slot != pg * kPageTokens + tok) {
+            if (lane == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
+        } else {
+            unsigned char *chunk = const_cast<unsigned char *>(kv_base) + (long long)pg * L.page_bytes;
+#pragma unroll 1
+            for (int tensor = 0; tensor < 2; tensor++) {
+                const __half *src = (tensor ? p.new_v : p.new_k) + ((long long)b * L.hkv + kvh) * kNvD + 4 * lane;
+                const uint2 raw = *reinterpret_cast<const uint2 *>(src);
+                const float2 a = __half22float2(bits_h2(raw.x)), c = __half22float2(bits_h2(raw.y));
+                float x[4] = {a.x, a.y, c.x, c.y};
+                if (p.rotate) {  // the append's rotation: exact sign flips, butterflies, one rounded scale
+#pragma unroll
+                    for (int e = 0; e < 4; e++) x[e] = __fmul_rn(x[e], p.signs[4 * lane + e]);
+                    fwht_warp<kNvD>(x, lane);
+#pragma unroll
+                    for (int e = 0; e < 4; e++) x[e] = __fmul_rn(x[e], p.rot_scale);
+                }
+                store_row(x, default_scale(x), chunk + (tensor ? L.v_codes : L.k_codes) + tok * kNvRowCode,
+                          chunk + (tensor ? L.v_meta : L.k_meta) + tok * kNvRowMeta, lane);
+            }
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+    }
     for (int i = 0; i < kNvStages && i < npg; i++) issue(i);
 
     if (warp < g) {  // the rotated query in log2 units

@@ -110,6 +110,8 @@ def test_bad_and_skipped_slots():
 
 
 def test_calls_nvfp4_does_not_serve():
+    """With ScaleSearch the fused step refuses the cache (its append codes
+    with the default scales); the integer read-back refuses NVFP4."""
     import torch
     import quantized_kv_cache_16_b200 as K
     wl = dataclasses.replace(W.scaled(NV, [32]), Hq=8, Hkv=2)
@@ -139,3 +141,30 @@ def test_full_size_bit_exact_and_decode():
     max_abs, rel = attn_errors(got, want)
     assert max_abs <= TOL_MAX_ABS and rel <= TOL_REL_L2, f"max_abs={max_abs:.3e} rel={rel:.3e}"
     assert pair.cache.sync_status() == 0
+
+
+@pytest.mark.parametrize("rotate", [1, 0])
+def test_decode_step_fuses_append_and_decode(rotate):
+    """Without ScaleSearch, kvq_decode_step on an NVFP4 cache stores exactly
+    the bytes kvq_append (and the oracle) stores and returns exactly what
+    kvq_append followed by kvq_decode_attn returns."""
+    import torch
+    wl = dataclasses.replace(W.scaled(NV, [300, 31, 16]), scale_search=0, rotate=rotate)
+    fused = build_pair(wl, extra_tokens=2)
+    split = build_pair(wl, extra_tokens=2, oracle=False)
+    for step in range(2):
+        k, v = W.step_kv(wl, step)
+        slots = np.array([fused.pages.slot(b, wl.ctx[b] + step) for b in range(wl.B)], np.int32)
+        q = torch.from_numpy(W.queries(wl, step)).cuda()
+        kd, vd, sd = torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(), torch.from_numpy(slots).cuda()
+        out_f = fused.cache.step(kd, vd, sd, q, fused.block_table(), fused.ctx(step + 1))
+        split.cache.append(kd, vd, sd)
+        out_s = split.cache.decode(q, split.block_table(), split.ctx(step + 1))
+        assert O.append(fused.ocfg, fused.opool, k, v, slots) == 0
+        assert fused.cache.sync_status() == 0
+        _bytes_equal(fused)
+        assert np.array_equal(out_f.cpu().numpy(), out_s.cpu().numpy())
+        want = O.decode(fused.ocfg, fused.opool, W.queries(wl, step), fused.pages.block_table,
+                        [t + step + 1 for t in wl.ctx])
+        max_abs, rel = attn_errors(out_f.cpu().numpy(), want)
+        assert max_abs <= TOL_MAX_ABS and rel <= TOL_REL_L2, f"max_abs={max_abs:.3e} rel={rel:.3e}"
