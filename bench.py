@@ -410,7 +410,8 @@ def e2e_leg(wk: Workload, K: int, stream, dist: Dist):
     """The same steps through the public C ABI with host buffers: one
     kvq_decode_step_host call a step enqueues the copy of that step's pinned
     host record (q, the new token's k and v, its slot and the context length)
-    to the device and the fused append + decode, whose kernel writes the
+    to the device (on the library's copy stream, overlapping the previous
+    step's kernel) and the fused append + decode, whose kernel writes the
     output to pinned host memory through its device mapping.  The call's
     arguments are marshalled once, before the timed region."""
     import ctypes as C
@@ -437,7 +438,7 @@ def e2e_leg(wk: Workload, K: int, stream, dist: Dist):
             h_in[c, u, off_c:off_c + 4] = np.array([wk.h_ctx[u]], np.int32).view(np.uint8)
     h_in = torch.from_numpy(h_in).pin_memory()
     h_out = torch.empty((wk.window,) + tuple(wk.out.shape), dtype=torch.float32).pin_memory()
-    d_rec = torch.empty(rec, dtype=torch.uint8, device=dev)
+    d_rec = torch.empty(2 * rec, dtype=torch.uint8, device=dev)  # two records, used alternately
     fn = Kb.lib().kvq_decode_step_host
     st = C.c_void_p(stream.cuda_stream)
     args = {}
@@ -469,8 +470,9 @@ def e2e_leg(wk: Workload, K: int, stream, dist: Dist):
     return {"value": round(bytes_rank * dist.world / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
             "us_per_step": 1e3 * ms / K, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "how": "one kvq_decode_step_host call per step: the step's pinned host record (q, k, v, slot, ctx) "
-                   "copied to the device, the fused append + decode, whose kernel writes the output to pinned host "
-                   "memory through its device mapping, inside the event-timed region"}
+                   "copied to the device on the library's copy stream (overlapping the previous step's kernel), "
+                   "the fused append + decode, whose kernel writes the output to pinned host memory through its "
+                   "device mapping, inside the event-timed region"}
 
 
 def append_leg():

@@ -369,15 +369,20 @@ kvq_status kvq_decode_step(kvq_cache *cache, const void *k_new, const void *v_ne
  * batch < 1. */
 size_t kvq_step_record_bytes(const kvq_cache *cache, int32_t batch);
 
-/* One decode step from and to host memory: enqueues on `stream` the copy of
+/* One decode step from and to host memory: kvq_decode_step on a copy of
  * the pinned host record `host_in` (kvq_step_record_bytes long, layout
- * above) into the device buffer `dev_rec` (as long, 16-byte aligned) and
- * kvq_decode_step on that record, whose kernel writes the fp32 output
- * [batch][Hq][d] straight to pinned `host_out` (16-byte aligned) through
- * its device mapping (no separate copy back).  Synchronise the stream
- * before reading host_out.  block_table stays in device memory.  Host
- * buffers that are not page-locked (cudaHostAlloc / cudaHostRegister)
- * return KVQ_ERR_INVALID_ARG, as do the cases kvq_decode_step rejects. */
+ * above), whose kernel writes the fp32 output [batch][Hq][d] straight to
+ * pinned `host_out` (16-byte aligned) through its device mapping (no copy
+ * back).  `dev_rec` is device memory for two records (2 x
+ * kvq_step_record_bytes, 16-byte aligned), used alternately: the record is
+ * copied on a stream of the library's own, waiting only for the step that
+ * last used the same half, so the copy overlaps the previous step's kernel;
+ * the kernel, on `stream`, waits for its copy.  Synchronise `stream` before
+ * reading host_out; host_in too must stay unchanged until then (its copy
+ * runs asynchronously).  One thread at a time per cache.  block_table stays
+ * in device memory.  Host buffers
+ * that are not page-locked (cudaHostAlloc / cudaHostRegister) return
+ * KVQ_ERR_INVALID_ARG, as do the cases kvq_decode_step rejects. */
 kvq_status kvq_decode_step_host(kvq_cache *cache, const void *host_in, void *dev_rec, const int32_t *block_table,
                                 int32_t max_pages_per_seq, int32_t batch, float softmax_scale, void *workspace,
                                 size_t ws_bytes, void *host_out, void *stream);

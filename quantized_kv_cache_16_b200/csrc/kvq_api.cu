@@ -335,6 +335,14 @@ kvq_status kvq_create_cache(const kvq_config *cfg, void *pool_dev, size_t pool_b
 kvq_status kvq_destroy_cache(kvq_cache *cache)
 {
     if (!cache) return KVQ_ERR_INVALID_ARG;
+    if (cache->copy_stream) {
+        cudaStreamSynchronize(cache->copy_stream);
+        cudaStreamDestroy(cache->copy_stream);
+    }
+    for (int b = 0; b < 2; b++) {
+        if (cache->ev_copied[b]) cudaEventDestroy(cache->ev_copied[b]);
+        if (cache->ev_consumed[b]) cudaEventDestroy(cache->ev_consumed[b]);
+    }
     delete cache;
     return KVQ_OK;
 }
@@ -760,14 +768,31 @@ kvq_status kvq_decode_step_host(kvq_cache *c, const void *host_in, void *dev_rec
     void *o = const_cast<void *>(device_view(host_out));
     if (!o || !aligned(o, 16)) return KVQ_ERR_INVALID_ARG;
     if (c->cfg.scale_search || c->L.hq_tab) return KVQ_ERR_UNSUPPORTED;
+    if (!c->copy_stream) {
+        if (cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking) != cudaSuccess) return KVQ_ERR_CUDA;
+        for (int b = 0; b < 2; b++)
+            if (cudaEventCreateWithFlags(&c->ev_copied[b], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&c->ev_consumed[b], cudaEventDisableTiming) != cudaSuccess)
+                return KVQ_ERR_CUDA;
+    }
     const StepRecord r = step_record(c, batch);
-    if (cudaMemcpyAsync(dev_rec, host_in, r.bytes, cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream)) !=
-        cudaSuccess)
+    const int b = c->io_next;
+    unsigned char *d = static_cast<unsigned char *>(dev_rec) + (size_t)b * r.bytes;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the copy of this step's record overlaps the previous step's kernel: it
+    // waits only for the kernel that last read the same buffer
+    if (cudaStreamWaitEvent(c->copy_stream, c->ev_consumed[b], 0) != cudaSuccess ||
+        cudaMemcpyAsync(d, host_in, r.bytes, cudaMemcpyHostToDevice, c->copy_stream) != cudaSuccess ||
+        cudaEventRecord(c->ev_copied[b], c->copy_stream) != cudaSuccess ||
+        cudaStreamWaitEvent(st, c->ev_copied[b], 0) != cudaSuccess)
         return KVQ_ERR_CUDA;
-    const unsigned char *d = static_cast<const unsigned char *>(dev_rec);
-    return decode_impl(c, d + r.k, d + r.v, reinterpret_cast<const int32_t *>(d + r.slot), d + r.q, block_table,
-                       max_pages_per_seq, reinterpret_cast<const int32_t *>(d + r.ctx), batch, softmax_scale, nullptr,
-                       workspace, ws_bytes, o, nullptr, stream);
+    const kvq_status rc = decode_impl(c, d + r.k, d + r.v, reinterpret_cast<const int32_t *>(d + r.slot), d + r.q,
+                                      block_table, max_pages_per_seq, reinterpret_cast<const int32_t *>(d + r.ctx),
+                                      batch, softmax_scale, nullptr, workspace, ws_bytes, o, nullptr, stream);
+    if (rc != KVQ_OK) return rc;
+    if (cudaEventRecord(c->ev_consumed[b], st) != cudaSuccess) return KVQ_ERR_CUDA;
+    c->io_next = b ^ 1;
+    return KVQ_OK;
 }
 
 kvq_status kvq_dequant_debug(kvq_cache *c, const int32_t *slots, int32_t n, float *k_out, float *v_out,

@@ -96,6 +96,12 @@ struct kvq_cache {
     uint32_t sign_xor[kvq::kMaxD / 2];  // per half2 word: 0x8000 / 0x80000000 where the sign is -1
     float rot_scale;               // fp32(1/sqrt(d))
     void *last_stream;
+    // kvq_decode_step_host: record copies on their own stream, two record
+    // buffers used alternately (created on first use)
+    cudaStream_t copy_stream = nullptr;
+    cudaEvent_t ev_copied[2] = {nullptr, nullptr};   // record b is on the device
+    cudaEvent_t ev_consumed[2] = {nullptr, nullptr}; // the kernel that read record b is done
+    int io_next = 0;
 };
 
 namespace kvq {

@@ -216,19 +216,21 @@ def _host_record(cache, wl, step, slots, ctx):
 
 
 def test_decode_step_host_equals_the_device_step():
-    """kvq_decode_step_host (the pinned host record copied in, the kernel
-    writing the pinned host output through its device mapping) stores the
-    same bytes and returns the same output as kvq_decode_step on device
-    copies of the same inputs; pageable host memory is refused."""
+    """kvq_decode_step_host (the pinned host record copied in on the
+    library's copy stream into alternating buffers, the kernel writing the
+    pinned host output through its device mapping) stores the same bytes and
+    returns the same output as kvq_decode_step on device copies of the same
+    inputs, over steps that use both buffers; pageable host memory is
+    refused."""
     import torch
     import quantized_kv_cache_16_b200 as K
     wl = W.scaled(W.llama(), [1000, 31, 16])
-    host = build_pair(wl, extra_tokens=2, oracle=False)
-    devp = build_pair(wl, extra_tokens=2, oracle=False)
+    host = build_pair(wl, extra_tokens=3, oracle=False)
+    devp = build_pair(wl, extra_tokens=3, oracle=False)
     ws = host.cache.workspace_for(wl.B, host.pages.block_table.shape[1])
     h_out = torch.empty((wl.B, wl.Hq, wl.d), dtype=torch.float32).pin_memory()
-    d_rec = torch.empty(K.kvq_step_record_bytes(host.cache.handle, wl.B), dtype=torch.uint8, device="cuda")
-    for step in range(2):
+    d_rec = torch.empty(2 * K.kvq_step_record_bytes(host.cache.handle, wl.B), dtype=torch.uint8, device="cuda")
+    for step in range(3):
         slots = np.array([host.pages.slot(b, wl.ctx[b] + step) for b in range(wl.B)], np.int32)
         ctx = [t + step + 1 for t in wl.ctx]
         h_in = _host_record(host.cache, wl, step, slots, ctx)
