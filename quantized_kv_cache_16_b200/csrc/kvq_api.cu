@@ -776,6 +776,12 @@ kvq_status kvq_decode_step_host(kvq_cache *c, const void *host_in, void *dev_rec
                 return KVQ_ERR_CUDA;
     }
     const StepRecord r = step_record(c, batch);
+    if (r.bytes != c->io_bytes || dev_rec != c->io_buf) {  // another layout: no half may still be in use
+        if (cudaStreamWaitEvent(c->copy_stream, c->ev_consumed[c->io_next ^ 1], 0) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        c->io_bytes = r.bytes;
+        c->io_buf = dev_rec;
+    }
     const int b = c->io_next;
     unsigned char *d = static_cast<unsigned char *>(dev_rec) + (size_t)b * r.bytes;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -102,6 +102,8 @@ struct kvq_cache {
     cudaEvent_t ev_copied[2] = {nullptr, nullptr};   // record b is on the device
     cudaEvent_t ev_consumed[2] = {nullptr, nullptr}; // the kernel that read record b is done
     int io_next = 0;
+    size_t io_bytes = 0;        // record size and buffer of the last call:
+    const void *io_buf = nullptr;  // when either changes, the copy waits for both halves
 };
 
 namespace kvq {
