@@ -35,10 +35,11 @@ METRIC = "int4-KV decode attn: KV-bytes GB/s as % of HBM peak; µs/step; append 
 NOMINAL_HBM_GBS = 8000.0
 
 
-# DRAM bytes (read + write) per launch of the dominant kernel from the ncu
-# capture summarised under profiles/ (decode_kernel_llama3-8b-layer-T32768.md).
-# Reported as roofline.traffic only while the decode kernel's sources hash to
-# the digest they had when the counters were taken; null otherwise.
+# DRAM bytes (read + write) per launch of the dominant kernel, as an ncu
+# capture of the decode kernel at this workload counted them
+# (dram__bytes_read.sum + dram__bytes_write.sum).  Reported as
+# roofline.traffic only while the decode kernel's sources hash to the digest
+# they had when the counters were taken; null otherwise.
 PROFILED_DECODE = {"sources_sha256": "4f2686c25844259234cdd81d4fac3484f962ce661750f6a10d1b6afab05f5edb",
                    "dram_bytes_per_launch": 42147456}
 DECODE_SOURCES = ("kvq_decode.cu", "kvq_internal.cuh", "kvq_warp.cuh")
@@ -76,7 +77,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-steps", type=int, default=4, help="oracle steps in the CPU baseline sample")
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, append and CPU legs")
-    ap.add_argument("--leg", choices=["certified", "ladder", "windows", "hqmq", "nvfp4"],
+    ap.add_argument("--leg", choices=["paged", "certified", "ladder", "windows", "hqmq", "nvfp4"],
                     help="run only this leg (one GPU, --steps calls) and print its JSON")
     ap.add_argument("--ctx", type=int, default=0, help="context length of --leg (default: its workload's)")
     return ap.parse_args()
@@ -227,6 +228,11 @@ class ClockSampler(threading.Thread):
 
 # ----------------------------------------------------------- the workload ---
 
+def workload_name(T: int, window: int) -> str:
+    return (f"llama3-8b layer decode step: B=1, Hq=32, Hkv=8, d=128, int4 g32 K/V, sign+Hadamard rotation, "
+            f"16-token shuffled pages, context {T + 1}..{T + window} (append 1 token + decode per step)")
+
+
 def kv_bytes_per_token(d: int, hkv: int) -> int:
     # int4 g32: d/2 code bytes + (d/32) x (scale, zero) fp16, for K and for V
     return hkv * 2 * (d // 2 + (d // 32) * 4)
@@ -374,9 +380,7 @@ def run_ours(args, dist: Dist):
         "warmup": max(args.warmup, 3), "ms_per_step": elapsed_ms / K, "us_per_step": 1e3 * elapsed_ms / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int4 codes; f16 mma with f32 accumulate", "data": "synthetic",
-        "config": {"workload": f"llama3-8b layer decode step: B=1, Hq=32, Hkv=8, d=128, int4 g32 K/V, "
-                               f"sign+Hadamard rotation, 16-token shuffled pages, context {wk.T + 1}.."
-                               f"{wk.T + wk.window} (append 1 token + decode per step)",
+        "config": {"workload": workload_name(wk.T, wk.window),
                    "global_batch": dist.world, "seq_len": wk.T, "parallelism": f"replicas x{dist.world}",
                    "l2_policy": f"{wk.copies} rotating cache copies ({wk.copies * (wk.T + wk.window) * kv_bytes_per_token(128, 8) / 1e6:.0f} MB) > 3x L2 ({wk.l2 / 1e6:.0f} MB)",
                    "cuda_graph": True},
@@ -393,6 +397,7 @@ def run_ours(args, dist: Dist):
     if not args.no_extras:
         result["e2e"] = e2e_leg(wk, K, stream, dist)
         result["append"] = append_leg()
+        result["paged"] = paged_leg(min(K, 200))
         result["certified"] = certified_leg(min(K, 200))
         result["ladder"] = ladder_leg(min(K, 100))
         result["windows"] = windows_leg(min(K, 200))
@@ -621,6 +626,68 @@ def certified_leg(steps: int, T: int = 0):
             "quantised_only_GB/s": round(hbm / (res["quantised_only"] * 1e-6) / 1e9, 1),
             "quantised_only_pct_hbm_peak": hbm / (res["quantised_only"] * 1e-6) / 1e9 / peak, "peak_kind": kind,
             "l2_policy": "2 cache copies (440 MB) alternate", "steps": steps}
+
+
+def paged_leg(steps: int, T: int = 0):
+    """Batched paged decode: batch 16, 32/8 heads, d=128, int4 g32 rotated,
+    context lengths uniform in [1024, 8192] from the seed, 16-token pages
+    shuffled in the block table.  Each step appends one token per sequence
+    and attends (kvq_decode_step, one launch); steps replayed in a CUDA graph
+    that rotates over enough cache copies to exceed 3x L2."""
+    import torch
+
+    import quantized_kv_cache_16_b200 as K
+    import workloads as W
+    wl = W.paged()
+    window = 16
+    dev = torch.device("cuda", torch.cuda.current_device())
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20))
+    per_copy = sum(wl.ctx) * kv_bytes_per_token(wl.d, wl.Hkv)
+    copies = max(2, math.ceil(3 * l2 / per_copy))
+    tabs = W.page_table(wl, extra_tokens=window, copies=copies)
+    cfg = K.make_config(wl.Hq, wl.Hkv, wl.d, wl.k_fmt, wl.v_fmt, wl.k_group, wl.v_group, wl.clip, wl.rotation_seed,
+                        num_pages=tabs[0].num_pages)
+    cache = K.Cache(cfg)
+    for b in range(wl.B):
+        kd, vd = W.prefix_kv_device(wl, b, dev)
+        for c in range(copies):
+            cache.append(kd, vd, torch.from_numpy(tabs[c].slots(b, 0, wl.ctx[b])).to(dev))
+        del kd, vd
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed)
+    newk = torch.randn((window, wl.B, wl.Hkv, wl.d), generator=gen, device=dev).half()
+    newv = (0.5 * torch.randn((window, wl.B, wl.Hkv, wl.d), generator=gen, device=dev)).half()
+    qs = torch.randn((window, wl.B, wl.Hq, wl.d), generator=gen, device=dev).half()
+    slots = torch.tensor([[[tabs[c].slot(b, wl.ctx[b] + u) for b in range(wl.B)] for u in range(window)]
+                          for c in range(copies)], dtype=torch.int32, device=dev)  # [C, window, B]
+    ctxs = torch.tensor([[t + u + 1 for t in wl.ctx] for u in range(window)], dtype=torch.int32, device=dev)
+    bts = [torch.from_numpy(t.block_table).to(dev) for t in tabs]
+    max_pages = bts[0].shape[1]
+    ws = cache.workspace_for(wl.B, max_pages)
+    out = torch.empty((wl.B, wl.Hq, wl.d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream()
+    n = (steps // (copies * window) + 1) * copies * window  # whole passes over (copy, step)
+
+    def step(s):
+        c, u = s % copies, (s // copies) % window
+        K.kvq_decode_step(cache.handle, newk[u], newv[u], slots[c, u], qs[u], bts[c], max_pages, ctxs[u], wl.B, 0.0,
+                          ws, ws.numel(), out, stream)
+
+    us = _graph_time(step, n, stream)
+    assert cache.sync_status() == 0
+    mean_ctx = sum(wl.ctx) + wl.B * (window + 1) / 2
+    kv = mean_ctx * kv_bytes_per_token(wl.d, wl.Hkv)
+    alg = kv + wl.B * wl.Hq * wl.d * (2 + 4) + 4 * sum((t + window + 15) // 16 for t in wl.ctx) + \
+        wl.B * wl.Hkv * wl.d * 2 * 2
+    peak, kind = measured_peaks()
+    gbs = alg / (us * 1e-6) / 1e9
+    return {"workload": f"batched paged decode step: B={wl.B}, 32/8 heads, d=128, int4 g32 rotated, context "
+                        f"lengths U[1024, 8192] (sum {sum(wl.ctx)}), shuffled 16-token pages, append 1 token per "
+                        f"sequence + decode (one launch)",
+            "us_per_step": round(us, 2), "kv_bytes_per_step": int(kv), "algorithmic_bytes_per_step": int(alg),
+            "gbs": round(gbs, 1), "pct_hbm_peak": gbs / peak, "peak_kind": kind,
+            "pct_hbm_nominal_8tbs": gbs / NOMINAL_HBM_GBS, "steps": n,
+            "l2_policy": f"{copies} rotating cache copies ({copies * per_copy / 1e6:.0f} MB) > 3x L2"}
 
 
 def windows_leg(steps: int, T: int = 0, sink: int = 128, recent: int = 1024):
@@ -936,28 +1003,53 @@ def ladder_leg(steps: int, T: int = 0):
             "steps": steps, "queries": nq}
 
 
-def cpu_leg(wk: Workload, n_steps: int):
-    """The CPU oracle on a bounded sample of the same steps (single thread)."""
-    import numpy as np
+def host_cpu():
+    """The host's logical CPU count and model name (from /proc/cpuinfo)."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count() or 1, model
 
+
+def cpu_leg(wk: Workload, n_steps: int):
+    """The CPU oracle on a bounded sample of the same steps: one thread, then
+    its (sequence, kv head) loop on all cores (OpenMP)."""
     import oracle as O
     wl = wk.wl
     ocfg = O.make_config(**wk.cfg_kw)
     pool = O.new_pool(ocfg)
     k, v = wk.W.prefix_kv(wl, 0)
     O.append(ocfg, pool, k, v, wk.tabs[0].slots(0, 0, wk.T))
-    times, nbytes = [], 0
-    for u in range(n_steps):
-        t = time.perf_counter()
-        O.append(ocfg, pool, wk.h_newk[u], wk.h_newv[u], wk.h_slots[0, u:u + 1])
-        O.decode(ocfg, pool, wk.h_q[u], wk.tabs[0].block_table, [int(wk.h_ctx[u])])
-        times.append(time.perf_counter() - t)
-        nbytes += int(wk.h_ctx[u]) * kv_bytes_per_token(wl.d, wl.Hkv)
-    sec = sum(times)
-    return {"value": round(nbytes / sec / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "us_per_step": 1e6 * sec / n_steps,
+    nproc, model = host_cpu()
+
+    def timed(threads, steps, first):
+        used = O.set_threads(threads)
+        times, nbytes = [], 0
+        for u in range(first, first + steps):
+            t = time.perf_counter()
+            O.append(ocfg, pool, wk.h_newk[u], wk.h_newv[u], wk.h_slots[0, u:u + 1])
+            O.decode(ocfg, pool, wk.h_q[u], wk.tabs[0].block_table, [int(wk.h_ctx[u])])
+            times.append(time.perf_counter() - t)
+            nbytes += int(wk.h_ctx[u]) * kv_bytes_per_token(wl.d, wl.Hkv)
+        return nbytes, sum(times), min(used, wl.B * wl.Hkv)
+
+    nb1, sec1, _ = timed(1, n_steps, 0)
+    nbn, secn, used = timed(nproc, 2 * n_steps, n_steps)
+    O.set_threads(1)
+    return {"value": round(nb1 / sec1 / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "us_per_step": 1e6 * sec1 / n_steps, "host": {"nproc": nproc, "cpu_model": model},
             "sample": f"{n_steps} of the window's steps (append 1 token + fp64 decode over the full context), "
-                      f"C oracle -O2 single thread, {sec:.1f} s"}
+                      f"C oracle -O2 single thread, {sec1:.1f} s",
+            "all_cores": {"value": round(nbn / secn / 1e9, 4), "unit": "GB/s", "cores": used,
+                          "us_per_step": 1e6 * secn / (2 * n_steps),
+                          "sample": f"the next {2 * n_steps} steps, OpenMP over the (sequence, kv head) pairs: "
+                                    f"{used} threads busy of {nproc} ({wl.B * wl.Hkv} pairs), {secn:.1f} s"}}
 
 
 def run_reference(args, dist: Dist):
@@ -984,22 +1076,27 @@ def run_reference(args, dist: Dist):
         O.decode(ocfg, pool, W.queries(wl, u), tab.block_table, [T + u + 1])
         return (T + u + 1) * per_tok
 
-    # the oracle takes seconds per step: a bounded sample of the K steps
+    # the oracle takes seconds per step: a bounded sample of the K steps, its
+    # (sequence, kv head) loop spread over the host's cores
+    nproc, model = host_cpu()
+    used = min(O.set_threads(nproc), wl.B * wl.Hkv)
     n_w = min(args.warmup, 1)
-    n_t = max(1, min(args.steps, 4))
+    n_t = max(1, min(args.steps, 8))
     for u in range(n_w):
         step(u)
     t = time.perf_counter()
     nbytes = sum(step(u % wl.steps) for u in range(n_t))
     sec = time.perf_counter() - t
     val = nbytes / sec / 1e9
+    sample = (f"{n_t} steps of the 100-step window (append 1 token + fp64 decode), C oracle -O2, OpenMP over "
+              f"the {wl.B * wl.Hkv} (sequence, kv head) pairs on {used} of {nproc} threads ({model}), {sec:.1f} s")
     line = {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": dist.world,
             "steps": n_t, "warmup": n_w, "ms_per_step": 1e3 * sec / n_t, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32 codec / f64 attention", "data": "synthetic",
-            "config": {"workload": "llama3-8b layer decode step (CPU oracle)", "global_batch": 1, "seq_len": T,
-                       "parallelism": "host, single thread"},
-            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{n_t} steps of the 100-step window"},
+            "config": {"workload": workload_name(T, wl.steps), "global_batch": dist.world, "seq_len": T,
+                       "parallelism": f"host CPU oracle, {used} threads"},
+            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": used, "kind": "oracle",
+                             "sample": sample, "host": {"nproc": nproc, "cpu_model": model}},
             "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -1010,7 +1107,7 @@ def main():
     if args.leg:
         import torch
         torch.cuda.set_device(0)
-        leg = {"certified": certified_leg, "ladder": ladder_leg, "windows": windows_leg, "hqmq": hqmq_leg,
+        leg = {"paged": paged_leg, "certified": certified_leg, "ladder": ladder_leg, "windows": windows_leg, "hqmq": hqmq_leg,
                "nvfp4": nvfp4_leg}[args.leg]
         print(json.dumps(leg(args.steps, args.ctx)), flush=True)
         return

@@ -31,7 +31,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.run(
-            ["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+            ["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
              "-Wall", "-o", tmp, _SRC, "-lm"],
             check=True,
         )
@@ -139,13 +139,21 @@ def lib():
             "kvqo_decode_windows": (i32, [cfgp, P, P, P, i32, i32, P, P, i32, P, i32, f64, P]),
             "kvqo_decode_ladder": (i32, [cfgp, P, P, P, P, P, i32, P, i32, f64, C.POINTER(Ladder), P, P,
                                          C.POINTER(LadderOut)]),
+            "kvqo_set_threads": (i32, [i32]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
+        L.kvqo_set_threads(1)  # one thread unless a caller asks for more
         _lib = L
     return _lib
+
+
+def set_threads(n: int) -> int:
+    """Threads of the decode's (sequence, kv head) loop (timing only: the
+    results do not depend on it); returns the count in effect."""
+    return int(lib().kvqo_set_threads(int(n)))
 
 
 def _p(a):

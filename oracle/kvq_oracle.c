@@ -38,6 +38,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define KVQO_INT4_ASYM 0
 #define KVQO_INT8_SYM 1
@@ -1120,6 +1123,20 @@ static int decode_args_ok(const kvqo_config *c, const int32_t *block_table, int 
     return 1;
 }
 
+/* Threads of the decode's (sequence, kv head) loop; returns the count in
+ * effect (1 when the oracle is built without OpenMP).  Timing only: the
+ * results do not depend on it. */
+int kvqo_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
 /* Decode attention over the quantised cache ([OSCAR] 2.2b fused kernel:
  * unpack, dequantise, attention, inverse rotation; the split/LSE merge is the
  * flash-decoding form the hot path uses).  Per sequence b and query head h:
@@ -1139,9 +1156,14 @@ int kvqo_decode(const kvqo_config *c, const uint8_t *pool, const uint16_t *q, co
     if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
     float s[KVQO_MAXD];
     kvqo_signs(c->rotation_seed, d, s);
+    /* (sequence, kv head) pairs are independent; with OpenMP they run on the
+     * threads kvqo_set_threads chose, each pair's arithmetic unchanged */
+#ifdef _OPENMP
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+#endif
     for (int b = 0; b < B; b++) {
-        int T = ctx_lens[b];
         for (int kvh = 0; kvh < hkv; kvh++) {
+            int T = ctx_lens[b];
             if (sel && !sel[b * hkv + kvh]) continue;
             double *K = (double *)malloc(sizeof(double) * ((size_t)T * d + 1));
             double *V = (double *)malloc(sizeof(double) * ((size_t)T * d + 1));
@@ -1604,8 +1626,10 @@ int kvqo_decode_ladder(const kvqo_config *c, const uint8_t *pool, const uint16_t
             }
             int k_cov = 0;
             if (pol->tau_cov > 0.0) {
+                /* tau_cov >= 1 is all of the mass: every block (a rounded
+                 * running sum can reach 1 before the last block joins) */
                 k_cov = nb;
-                for (int K = 0; K <= nb; K++)
+                for (int K = 0; K <= nb && pol->tau_cov < 1.0; K++)
                     if (cov[K] >= pol->tau_cov) {
                         k_cov = K;
                         break;

@@ -26,7 +26,7 @@ EXPORTS = (
     "kvq_pool_bytes", "kvq_create_cache", "kvq_destroy_cache", "kvq_append", "kvq_reset_pages",
     "kvq_decode_workspace_bytes", "kvq_decode_attn", "kvq_decode_certified", "kvq_decode_windows",
     "kvq_decode_windows_workspace_bytes", "kvq_decode_step", "kvq_step_record_bytes", "kvq_decode_step_host",
-    "kvq_decode_attn_static", "kvq_dequant_debug", "kvq_sync_status",
+    "kvq_decode_attn_static", "kvq_dequant_debug", "kvq_debug_expire_first_wait", "kvq_sync_status",
     "kvq_status_string",
 )
 
@@ -95,6 +95,7 @@ def lib() -> C.CDLL:
             "kvq_decode_step_host": (i32, [P, P, P, P, i32, i32, C.c_float, P, sz, P, P]),
             "kvq_decode_attn_static": (i32, [P, P, P, i32, P, i32, C.c_float, P, P]),
             "kvq_dequant_debug": (i32, [P, P, i32, P, P, P, P, P]),
+            "kvq_debug_expire_first_wait": (i32, [P, i32]),
             "kvq_sync_status": (i32, [P]),
             "kvq_status_string": (C.c_char_p, [i32]),
         }
@@ -232,6 +233,10 @@ def kvq_dequant_debug(cache, slots, n: int | None = None, k_out=None, v_out=None
     n = slots.shape[0] if n is None else n
     _check("kvq_dequant_debug", lib().kvq_dequant_debug(cache, _ptr(slots), n, _ptr(k_out), _ptr(v_out),
                                                         _ptr(codes_out), _ptr(meta_out), _stream(stream)))
+
+
+def kvq_debug_expire_first_wait(cache, on: int) -> None:
+    _check("kvq_debug_expire_first_wait", lib().kvq_debug_expire_first_wait(cache, int(on)))
 
 
 def kvq_sync_status(cache) -> int:

@@ -425,6 +425,7 @@ DecodeParams decode_params(kvq_cache *c, const SplitPlan &s, const void *q, cons
     p.part = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + counters_bytes(batch, c->L.hkv));
     p.out = static_cast<float *>(out);
     p.clip = c->cfg.clip_ratio;
+    p.expire_first_wait = c->expire_first_wait;
     return p;
 }
 
@@ -759,6 +760,13 @@ size_t kvq_step_record_bytes(const kvq_cache *c, int32_t batch)
     return step_record(c, batch).bytes;
 }
 
+kvq_status kvq_debug_expire_first_wait(kvq_cache *c, int32_t on)
+{
+    if (!c || (on != 0 && on != 1)) return KVQ_ERR_INVALID_ARG;
+    c->expire_first_wait = on;
+    return KVQ_OK;
+}
+
 kvq_status kvq_decode_step_host(kvq_cache *c, const void *host_in, void *dev_rec, const int32_t *block_table,
                                 int32_t max_pages_per_seq, int32_t batch, float softmax_scale, void *workspace,
                                 size_t ws_bytes, void *host_out, void *stream)
@@ -769,11 +777,24 @@ kvq_status kvq_decode_step_host(kvq_cache *c, const void *host_in, void *dev_rec
     if (!o || !aligned(o, 16)) return KVQ_ERR_INVALID_ARG;
     if (c->cfg.scale_search || c->L.hq_tab) return KVQ_ERR_UNSUPPORTED;
     if (!c->copy_stream) {
-        if (cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking) != cudaSuccess) return KVQ_ERR_CUDA;
-        for (int b = 0; b < 2; b++)
-            if (cudaEventCreateWithFlags(&c->ev_copied[b], cudaEventDisableTiming) != cudaSuccess ||
-                cudaEventCreateWithFlags(&c->ev_consumed[b], cudaEventDisableTiming) != cudaSuccess)
-                return KVQ_ERR_CUDA;
+        // the stream and its four events are created into locals and kept
+        // only if all five exist, so a failure here leaves the handle as it
+        // was and the next call tries again
+        cudaStream_t cs = nullptr;
+        cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+        bool ok = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) == cudaSuccess;
+        for (int i = 0; ok && i < 4; i++) ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) {
+            for (int i = 0; i < 4; i++)
+                if (ev[i]) cudaEventDestroy(ev[i]);
+            if (cs) cudaStreamDestroy(cs);
+            return KVQ_ERR_CUDA;
+        }
+        c->ev_copied[0] = ev[0];
+        c->ev_copied[1] = ev[1];
+        c->ev_consumed[0] = ev[2];
+        c->ev_consumed[1] = ev[3];
+        c->copy_stream = cs;
     }
     const StepRecord r = step_record(c, batch);
     if (r.bytes != c->io_bytes || dev_rec != c->io_buf) {  // another layout: no half may still be in use

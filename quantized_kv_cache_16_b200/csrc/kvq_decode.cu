@@ -39,7 +39,6 @@ namespace kvq {
 namespace {
 
 constexpr int kCombineSplits = 40;  // most splits per (sequence, kv head)
-constexpr int kMergeBatch = 10;     // split records a merging warp loads at once
 
 // fp16x2 constants (bit patterns)
 constexpr uint32_t kH1024 = 0x64006400u;  // (1024, 1024)
@@ -84,11 +83,9 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) { return h2_bits
 // values at once (one packed conversion each way): rx for x, ry for y
 __device__ __forceinline__ void hilo_pair(float x, float y, uint32_t &rx, uint32_t &ry)
 {
-    const __half2 h = __floats2half2_rn(x, y);
-    const float2 hf = __half22float2(h);
-    const uint32_t hb = h2_bits(h), lb = h2_bits(__floats2half2_rn(x - hf.x, y - hf.y));
-    rx = __byte_perm(hb, lb, 0x5410);
-    ry = __byte_perm(hb, lb, 0x7632);
+    const float2 hf = __half22float2(__floats2half2_rn(x, y));
+    rx = pack_h2(hf.x, x - hf.x);  // hf.x is an fp16 value: packing it is exact
+    ry = pack_h2(hf.y, y - hf.y);
 }
 
 // NG fp16 values stored consecutively (4-byte aligned for NG >= 2) as fp32
@@ -126,6 +123,25 @@ __device__ __forceinline__ void imma16832(int *d, const uint32_t (&a)[4], uint32
         "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D(16x8 s32) = A(16x32 s8, row) * B(32x8 s8, col), no accumulator input
+__device__ __forceinline__ void imma16832_z(int *d, const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
+}
+
+// D(16x8 f32) = A(16x16 f16, row) * B(16x8 f16, col), no accumulator input
+__device__ __forceinline__ void mma16816_z(float *d, const uint32_t *a, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
 
@@ -426,14 +442,25 @@ template <int KF, int VF, int D, bool G8> struct Cfg {
     static constexpr int OFF_QEXP = OFF_QSUM + kMaxGqa * 4 * 4;      // i32 [8]
     static constexpr int OFF_BAR = OFF_QEXP + kMaxGqa * 4;
     static constexpr int END = OFF_BAR + kDecodeWarps * NST * 8;
-    static constexpr int OFF_FLAG = (END + 7) / 8 * 8;
-    static constexpr int SMEM = OFF_FLAG + 16;  // the last-CTA flag (int)
-    // merge scratch (aliases the ring after the page loop)
-    static constexpr int MERGE_ACC = 0;                                         // [W][8][D]
-    static constexpr int MERGE_Z = MERGE_ACC + kDecodeWarps * kMaxGqa * D * 4;    // [W][4][8]
-    static constexpr int MERGE_M = MERGE_Z + kDecodeWarps * 4 * kMaxGqa * 4;      // [W][8]
-    static constexpr int MERGE_L = MERGE_M + kDecodeWarps * kMaxGqa * 4;          // [W][8]
-    static_assert(MERGE_L + kDecodeWarps * kMaxGqa * 4 <= RING, "merge scratch must fit in the ring");
+    static constexpr int OFF_FLAG = (END + 7) / 8 * 8;                   // the last-CTA flag (int)
+    static constexpr int OFF_RBAR = OFF_FLAG + 8;                         // mbarrier of the record copy
+    // final merge: split weights [kCombineSplits][8], per-head rescale,
+    // max and sum [8] each, the normalised rows [8][D]
+    static constexpr int OFF_FW = OFF_RBAR + 8;
+    static constexpr int OFF_FC = OFF_FW + kCombineSplits * kMaxGqa * 4;
+    static constexpr int OFF_FM = OFF_FC + kMaxGqa * 4;
+    static constexpr int OFF_FL = OFF_FM + kMaxGqa * 4;
+    static constexpr int OFF_FROW = (OFF_FL + kMaxGqa * 4 + 15) / 16 * 16;
+    static constexpr int SMEM = OFF_FROW + kMaxGqa * D * 4;
+    // split records staged per piece of the final merge (in the ring)
+    static constexpr int REC = D + 4;
+    // merge scratch (aliases the ring after the page loop): per warp and
+    // head a row of D sums at a padded stride (the four heads a warp stores
+    // at once then fall on different banks), and the (max, sum) pairs
+    static constexpr int MS = D + 8;
+    static constexpr int MERGE_ACC = 0;                                       // [W][8][MS] f32
+    static constexpr int MERGE_ML = MERGE_ACC + kDecodeWarps * kMaxGqa * MS * 4;  // [W][8] float2
+    static_assert(MERGE_ML + kDecodeWarps * kMaxGqa * 8 <= RING, "merge scratch must fit in the ring");
     static_assert(OFF_BAR % 8 == 0, "mbarriers need 8-byte alignment");
 };
 
@@ -524,18 +551,43 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     constexpr int NH = C::NH;
     constexpr int NT = C::NT;
 
-    // Launched as a programmatic dependent of the stream's previous kernel:
-    // wait for that grid to complete (its writes visible) before touching
-    // memory, then let the next dependent grid be set up early.  No work of
-    // this grid overlaps the previous one; only the launch latency is hidden.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
     const Layout &L = p.L;
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r = lane >> 2, j = lane & 3;
     const int g = L.g;
+
+    // Launched as a programmatic dependent of the stream's previous kernel,
+    // this CTA may start while that grid is still finishing.  Until
+    // griddepcontrol.wait returns, nothing read can be trusted (the previous
+    // kernel may be writing the context lengths, the block table, the query
+    // or the pages), so this phase only warms L2: the context length and this
+    // warp's block-table entries are read as hints (L2 only, never kept in
+    // L1), clamped into the pool, and the pages they name are prefetched
+    // into L2.  A stale hint costs a wasted prefetch, never a wrong result:
+    // every value used below is read again after the wait.
+    {
+        int Th = __ldcg(p.ctx_lens + b);
+        Th = min(max(Th, 0), p.max_pages * kPageTokens);
+        const int pg0 = split * p.pages_per_split + warp * p.pages_per_warp;
+        const int npg_h = min(pg0 + p.pages_per_warp, (Th + kPageTokens - 1) / kPageTokens) - pg0;
+        if (lane < npg_h) {
+            const int pg = __ldcg(p.block_table + (long long)b * p.max_pages + pg0 + lane);
+            if (pg >= 0 && pg < L.num_pages)
+                bulk_prefetch_l2(p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes + (long long)pg * L.page_bytes,
+                                 L.chunk_bytes);
+        }
+        // the group's query rows (contiguous) and the rows the step appends
+        if (warp == 0 && lane == 31) bulk_prefetch_l2(p.q + ((long long)b * L.hq + kvh * g) * D, g * D * 2);
+        if (warp == 1 && lane == 31 && p.new_k != nullptr) {
+            bulk_prefetch_l2(p.new_k + ((long long)b * L.hkv + kvh) * D, D * 2);
+            bulk_prefetch_l2(p.new_v + ((long long)b * L.hkv + kvh) * D, D * 2);
+        }
+    }
+    // wait for the previous grid to complete (its writes visible), then let
+    // the next dependent grid be set up early
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // independent loads first: the context length, this warp's first 32
     // block-table entries (speculative) and the query row all go out together
@@ -599,23 +651,25 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         }
     }
     uint32_t vbits = 0;      // bit s: stage s holds a valid page
-    auto issue = [&](int i) {  // every lane calls this
+    auto issue = [&](int i) {  // every lane calls this; lane 0 alone copies (predicated, no branch)
         const int pg = __shfl_sync(kFull, ids, i & 31);
         const int st = i % NST;
         vbits = (vbits & ~(1u << st)) | ((pg >= 0 ? 1u : 0u) << st);
         // (a stage was last read by this warp's ldmatrix loads, complete before
         // the __syncwarp that precedes every refill; no generic-proxy write to
         // the ring precedes the copy, so no proxy fence)
-        if (lane == 0) {
-            if (pg >= 0)
-                bulk_load(stage0 + st * C::STAGE, kv_base + (long long)pg * L.page_bytes, C::CHUNK, bar0 + 8 * st);
-            else
-                asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar0 + 8 * st) : "memory");
-        }
+        bulk_load_or_arrive(lane == 0 && pg >= 0, lane == 0 && pg < 0, stage0 + st * C::STAGE,
+                            kv_base + (long long)max(pg, 0) * L.page_bytes, C::CHUNK, bar0 + 8 * st);
     };
     // fused append: the warp that owns the page of position T-1 quantises
-    // the new token's K and V rows into it before any copy of that page
-    if (p.new_k != nullptr && T > 0 && n_pages - 1 >= p_begin && n_pages - 1 < p_end) {
+    // the new token's K and V rows into it before any copy of that page.
+    // That page is the warp's last; the copies of the pages before it go out
+    // first, so the append's latency overlaps them.
+    const bool appends = p.new_k != nullptr && T > 0 && n_pages - 1 >= p_begin && n_pages - 1 < p_end;
+    const int n_first = min(NST, npg);
+    const int n_pre = (appends && n_first == npg) ? npg - 1 : n_first;
+    for (int i = 0; i < n_pre; i++) issue(i);
+    if (appends) {
         const int pg = bt[n_pages - 1];
         const int slot = p.new_slots[b];
         const int tok = (T - 1) % kPageTokens;
@@ -636,7 +690,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             if (lane == 0) asm volatile("fence.proxy.async.global;" ::: "memory");
         }
     }
-    for (int i = 0; i < NST && i < npg; i++) issue(i);
+    for (int i = n_pre; i < n_first; i++) issue(i);
 
     // ---- query (warp h): rotate, pre-scale, group sums, and the three signed
     //      7-bit digits of q * 2^E written straight into the B layout ----
@@ -760,25 +814,49 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         l_part[t] = 0.f;
     }
 
-    for (int i = 0; i < npg; i++) {
-        const int st = i % NST;
-        const bool ok = mbar_wait_bounded(bar0 + 8 * st, (i / NST) & 1, kWaitLimitNs);
-        if (!__all_sync(kFull, ok)) {
-            // give up on this warp's run: record it, then wait (bounded) for
-            // the copies still in flight so none lands after the ring is reused
-            if (lane == 0) set_status(p.pool, KVQ_ERR_TIMEOUT);
-            for (int k = i; k < npg && k < i + NST; k++)
-                (void)mbar_wait_bounded(bar0 + 8 * (k % NST), (k / NST) & 1, kWaitLimitNs);
-            break;
+    // Pages whose 16 tokens are all attended here and whose copy exists take
+    // the plain path; the first/last pages of the context or of a window
+    // boundary, and pages the block table got wrong, mask their tokens.
+    // Iterations [i_full0, i_full1) are the warp's pages inside [q_lo, q_hi).
+    const int i_full0 = (q_lo + kPageTokens - 1) / kPageTokens - p_begin;
+    const int i_full1 = q_hi / kPageTokens - p_begin;
+    int st = 0;
+    uint32_t ph = 0;  // the ring stage and its barrier phase of page i
+    int n_loop = npg;
+    if (p.expire_first_wait && npg > 0) {
+        // test hook: the first wait counts as expired.  The timeout path
+        // runs as it would: record the status, then wait (bounded, the
+        // normal limit) for the copies in flight; no page is attended.
+        if (lane == 0) set_status(p.pool, KVQ_ERR_TIMEOUT);
+        for (int k = 0; k < npg && k < NST; k++)
+            (void)mbar_wait_bounded(bar0 + 8 * (k % NST), (k / NST) & 1, kWaitLimitNs);
+        n_loop = 0;
+    }
+    for (int i = 0; i < n_loop; i++) {
+        const uint32_t bar = bar0 + 8 * st;
+        if (!__all_sync(kFull, mbar_try_wait(bar, ph))) {
+            // slow path: the page is not in yet; wait, but not forever
+            if (!__all_sync(kFull, mbar_wait_bounded(bar, ph, kWaitLimitNs))) {
+                // give up on this warp's run: record it, then wait (bounded) for
+                // the copies still in flight so none lands after the ring is reused
+                if (lane == 0) set_status(p.pool, KVQ_ERR_TIMEOUT);
+                for (int k = i; k < npg && k < i + NST; k++)
+                    (void)mbar_wait_bounded(bar0 + 8 * (k % NST), (k / NST) & 1, kWaitLimitNs);
+                break;
+            }
         }
-        const int t0 = (p_begin + i) * kPageTokens;
-        // valid tokens of the page: [vlo, vhi) (the tail, and windows attended elsewhere)
-        const int vlo = min(max(q_lo - t0, 0), kPageTokens);
-        const int vhi = min(max(q_hi - t0, 0), kPageTokens);
         const uint32_t sb = stage0 + st * C::STAGE;
         const unsigned char *sp = stage0_ptr + st * C::STAGE;
         const bool page_ok = (vbits >> st) & 1u;
-        const bool ragged = vlo > 0 || vhi < kPageTokens || !page_ok;
+        const bool ragged = i < i_full0 || i >= i_full1 || !page_ok;  // warp-uniform
+        // valid tokens of a ragged page: r in [vlo, vhi) (the tail, windows attended elsewhere)
+        int vlo = 0, vhi = kPageTokens;
+        if (ragged) {
+            const int t0 = (p_begin + i) * kPageTokens;
+            vlo = page_ok ? min(max(q_lo - t0, 0), kPageTokens) : kPageTokens;
+            vhi = page_ok ? min(max(q_hi - t0, 0), kPageTokens) : 0;
+        }
+        const bool tv_r = r >= vlo && r < vhi, tv_r8 = r + 8 >= vlo && r + 8 < vhi;
 
         // ---------------- QK: scores of tokens r, r+8 for the lane's heads ----
         float s_r[NH], s_r8[NH];
@@ -791,44 +869,49 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
 #pragma unroll
             for (int t = 0; t < NH; t++) zr[t] = zr8[t] = 0.f;
             if constexpr (KC::ZERO) {
+                // zeros of groups (2j, 2j+1) of tokens r and r+8 as the A
+                // fragment; lanes j with no such group read an in-row word
+                // and drop it (their B rows are zero as well)
                 uint32_t a[4] = {0u, 0u, 0u, 0u};
                 if constexpr (KC::NG >= 2) {
-                    if (2 * j < KC::NG) {
-                        a[0] = *reinterpret_cast<const uint32_t *>(meta_r + 2 * KC::NG + 4 * j);
-                        a[1] = *reinterpret_cast<const uint32_t *>(meta_r8 + 2 * KC::NG + 4 * j);
-                    }
+                    const int jj = (2 * j < KC::NG) ? j : 0;
+                    const uint32_t z0 = *reinterpret_cast<const uint32_t *>(meta_r + 2 * KC::NG + 4 * jj);
+                    const uint32_t z1 = *reinterpret_cast<const uint32_t *>(meta_r8 + 2 * KC::NG + 4 * jj);
+                    a[0] = (2 * j < KC::NG) ? z0 : 0u;
+                    a[1] = (2 * j < KC::NG) ? z1 : 0u;
                 } else {
-                    if (j == 0) {
-                        a[0] = *reinterpret_cast<const uint16_t *>(meta_r + 2);
-                        a[1] = *reinterpret_cast<const uint16_t *>(meta_r8 + 2);
-                    }
+                    const uint32_t z0 = *reinterpret_cast<const uint16_t *>(meta_r + 2);
+                    const uint32_t z1 = *reinterpret_cast<const uint16_t *>(meta_r8 + 2);
+                    a[0] = j == 0 ? z0 : 0u;
+                    a[1] = j == 0 ? z1 : 0u;
                 }
 #pragma unroll
                 for (int t = 0; t < NH; t++) {
-                    float dz[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma16816(dz, a, zb[t], 0u);
+                    float dz[4];
+                    mma16816_z(dz, a, zb[t], 0u);
                     zr[t] = dz[0] + dz[1];
                     zr8[t] = dz[2] + dz[3];
                 }
             }
             float acc_r[NH], acc_r8[NH];
-#pragma unroll
-            for (int t = 0; t < NH; t++) acc_r[t] = acc_r8[t] = 0.f;
             float skr[KC::NG], skr8[KC::NG];  // the rows' group scales
             load_h<KC::NG>(meta_r, skr);
             load_h<KC::NG>(meta_r8, skr8);
 #pragma unroll
             for (int gi = 0; gi < KC::NG; gi++) {
                 int d[NT][4];
-#pragma unroll
-                for (int nt = 0; nt < NT; nt++) d[nt][0] = d[nt][1] = d[nt][2] = d[nt][3] = 0;
+                bool first = true;
 #pragma unroll
                 for (int kq = 0; kq < KC::KQ; kq++) {
                     if (KC::group_of_kq(kq) != gi) continue;
                     uint32_t a[4];
                     KC::afrag(kw, kw8, kq, a);
 #pragma unroll
-                    for (int nt = 0; nt < NT; nt++) imma16832(d[nt], a, qb[nt][kq][0], qb[nt][kq][1]);
+                    for (int nt = 0; nt < NT; nt++) {
+                        if (first) imma16832_z(d[nt], a, qb[nt][kq][0], qb[nt][kq][1]);
+                        else imma16832(d[nt], a, qb[nt][kq][0], qb[nt][kq][1]);
+                    }
+                    first = false;
                 }
                 const float sk_r = skr[gi], sk_r8 = skr8[gi];
 #pragma unroll
@@ -845,18 +928,19 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
                         v_r = __int2float_rn(d[n12][0] * 16384 + d[n12][1] * 128 + d[n3][c3]);
                         v_r8 = __int2float_rn(d[n12][2] * 16384 + d[n12][3] * 128 + d[n3][2 + c3]);
                     }
-                    acc_r[t] = fmaf(sk_r, v_r, acc_r[t]);
-                    acc_r8[t] = fmaf(sk_r8, v_r8, acc_r8[t]);
+                    if (gi == 0) {
+                        acc_r[t] = sk_r * v_r;
+                        acc_r8[t] = sk_r8 * v_r8;
+                    } else {
+                        acc_r[t] = fmaf(sk_r, v_r, acc_r[t]);
+                        acc_r8[t] = fmaf(sk_r8, v_r8, acc_r8[t]);
+                    }
                 }
             }
 #pragma unroll
             for (int t = 0; t < NH; t++) {
-                s_r[t] = fmaf(acc_r[t], qinv[t], zr[t]);
-                s_r8[t] = fmaf(acc_r8[t], qinv[t], zr8[t]);
-                if (ragged) {
-                    if (r < vlo || r >= vhi || !page_ok) s_r[t] = -INFINITY;
-                    if (r + 8 < vlo || r + 8 >= vhi || !page_ok) s_r8[t] = -INFINITY;
-                }
+                s_r[t] = tv_r ? fmaf(acc_r[t], qinv[t], zr[t]) : -INFINITY;
+                s_r8[t] = tv_r8 ? fmaf(acc_r8[t], qinv[t], zr8[t]) : -INFINITY;
             }
         }
 
@@ -896,9 +980,11 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             }
 #pragma unroll
             for (int t = 0; t < NH; t++) {
-                const bool live = m_run[t] != -INFINITY;
-                p_r[t] = live ? ex2(s_r[t] - m_run[t]) : 0.f;
-                p_r8[t] = live ? ex2(s_r8[t] - m_run[t]) : 0.f;
+                // m_run is finite once any token was seen; before that every
+                // score is -inf and ex2(-inf - (-inf)) would be NaN
+                const float mr = m_run[t] == -INFINITY ? 0.f : m_run[t];
+                p_r[t] = ex2(s_r[t] - mr);
+                p_r8[t] = ex2(s_r8[t] - mr);
                 l_part[t] += p_r[t] + p_r8[t];
             }
             if (p.page_stats != nullptr) {  // certified mode: this page's (m, l) per head
@@ -921,30 +1007,31 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             float sv_r[VC::NG], sv_r8[VC::NG];
             load_h<VC::NG>(vmeta_r, sv_r);
             load_h<VC::NG>(vmeta_r8, sv_r8);
-            if (ragged) {
-                const bool v_r = page_ok && r >= vlo && r < vhi, v_r8 = page_ok && r + 8 >= vlo && r + 8 < vhi;
-#pragma unroll
-                for (int gi = 0; gi < VC::NG; gi++) {
-                    sv_r[gi] = v_r ? sv_r[gi] : 0.f;
-                    sv_r8[gi] = v_r8 ? sv_r8[gi] : 0.f;
-                }
-            }
-            // zero term: A = zeros^T (group r, tokens 2j, 2j+1 | 2j+8, 2j+9)
+            // zero term: A = zeros^T (group r, tokens 2j, 2j+1 | 2j+8, 2j+9);
+            // rows r >= NG read group r % NG and drop it
             uint32_t az[4] = {0u, 0u, 0u, 0u};
-            if (r < VC::NG) {
-                const unsigned char *zrow = sp + C::V_META + 2 * VC::NG + 2 * r;
+            {
+                const unsigned char *zrow = sp + C::V_META + 2 * VC::NG + 2 * (r % VC::NG);
                 uint32_t z0 = *reinterpret_cast<const uint16_t *>(zrow + (2 * j) * VC::ROW_META);
                 uint32_t z1 = *reinterpret_cast<const uint16_t *>(zrow + (2 * j + 1) * VC::ROW_META);
                 uint32_t z2 = *reinterpret_cast<const uint16_t *>(zrow + (2 * j + 8) * VC::ROW_META);
                 uint32_t z3 = *reinterpret_cast<const uint16_t *>(zrow + (2 * j + 9) * VC::ROW_META);
                 if (ragged) {
-                    if (!page_ok || 2 * j < vlo || 2 * j >= vhi) z0 = 0;
-                    if (!page_ok || 2 * j + 1 < vlo || 2 * j + 1 >= vhi) z1 = 0;
-                    if (!page_ok || 2 * j + 8 < vlo || 2 * j + 8 >= vhi) z2 = 0;
-                    if (!page_ok || 2 * j + 9 < vlo || 2 * j + 9 >= vhi) z3 = 0;
+                    // masked tokens: weight and zero both 0 (their stage bytes may be stale)
+#pragma unroll
+                    for (int gi = 0; gi < VC::NG; gi++) {
+                        sv_r[gi] = tv_r ? sv_r[gi] : 0.f;
+                        sv_r8[gi] = tv_r8 ? sv_r8[gi] : 0.f;
+                    }
+                    if (2 * j < vlo || 2 * j >= vhi) z0 = 0;
+                    if (2 * j + 1 < vlo || 2 * j + 1 >= vhi) z1 = 0;
+                    if (2 * j + 8 < vlo || 2 * j + 8 >= vhi) z2 = 0;
+                    if (2 * j + 9 < vlo || 2 * j + 9 >= vhi) z3 = 0;
                 }
-                az[0] = z0 | (z1 << 16);
-                az[2] = z2 | (z3 << 16);
+                if (r < VC::NG) {
+                    az[0] = z0 | (z1 << 16);
+                    az[2] = z2 | (z3 << 16);
+                }
             }
             uint32_t vA[VC::NCH], vB[VC::NCH];
             ld_vrows_t<VC::NCH>(sb + C::V_CODES, lane, vA, vB);
@@ -982,61 +1069,76 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             if ((nxt & 31) == 0) ids = fetch_ids(nxt);
             issue(nxt);
         }
+        if (++st == NST) {
+            st = 0;
+            ph ^= 1u;
+        }
     }
 
     // ---- warp state -> shared memory, CTA merge ----
+    // The zero term of group gi for head j sits in lane (gi, j): add it to
+    // the accumulator rows of that group, and the row pair (c, c + 1) a lane
+    // holds becomes two finished sums.
 #pragma unroll
     for (int t = 0; t < NH; t++) {
         l_part[t] += __shfl_xor_sync(kFull, l_part[t], 4);
         l_part[t] += __shfl_xor_sync(kFull, l_part[t], 8);
         l_part[t] += __shfl_xor_sync(kFull, l_part[t], 16);
+        const float zs = oz[t][0] + oz[t][1];
+        float zg[VC::NG];
+#pragma unroll
+        for (int gi = 0; gi < VC::NG; gi++) zg[gi] = __shfl_sync(kFull, zs, gi * 4 + j);
+#pragma unroll
+        for (int mt = 0; mt < C::MT; mt++) {
+            const float z = zg[VC::group_of_mt(mt)];
+            oacc[t][mt][0] = oacc[t][mt][0] + oacc[t][mt][1] + z;
+            oacc[t][mt][2] = oacc[t][mt][2] + oacc[t][mt][3] + z;
+        }
     }
     __syncthreads();  // every warp is done with the stage ring
-    float *macc = reinterpret_cast<float *>(smem + C::MERGE_ACC);
-    float *mz = reinterpret_cast<float *>(smem + C::MERGE_Z);
-    float *mm = reinterpret_cast<float *>(smem + C::MERGE_M);
-    float *ml = reinterpret_cast<float *>(smem + C::MERGE_L);
+    float *macc = reinterpret_cast<float *>(smem + C::MERGE_ACC);  // [warp][head][MS]
+    float2 *mml = reinterpret_cast<float2 *>(smem + C::MERGE_ML);  // [warp][head] (max, sum)
 #pragma unroll
     for (int t = 0; t < NH; t++) {
         const int head = j + 4 * t;
         if (head < g) {
+            float *row = macc + (warp * kMaxGqa + head) * C::MS;
 #pragma unroll
-            for (int mt = 0; mt < C::MT; mt++) {
-                macc[(warp * kMaxGqa + head) * D + VC::chan(mt, r)] = oacc[t][mt][0] + oacc[t][mt][1];
-                macc[(warp * kMaxGqa + head) * D + VC::chan(mt, r + 8)] = oacc[t][mt][2] + oacc[t][mt][3];
-            }
-            if (r < VC::NG) mz[(warp * 4 + r) * kMaxGqa + head] = oz[t][0] + oz[t][1];
-            if (r == 0) {
-                mm[warp * kMaxGqa + head] = m_run[t];
-                ml[warp * kMaxGqa + head] = l_part[t];
-            }
+            for (int mt = 0; mt < C::MT; mt++)
+                *reinterpret_cast<float2 *>(row + VC::chan(mt, r)) = make_float2(oacc[t][mt][0], oacc[t][mt][2]);
+            if (r == 0) mml[warp * kMaxGqa + head] = make_float2(m_run[t], l_part[t]);
         }
     }
     __syncthreads();
 
+    // thread: head h, channels (ch, ch + 1); the 8 warps' (max, sum) of the
+    // head are broadcast reads, their weights 2^(m_w - M) computed here
     const int n_splits = p.n_splits;
     float *part_base = p.part + (((long long)b * L.hkv + kvh) * n_splits) * g * (D + 4);
-    for (int idx = tid; idx < g * D; idx += kDecodeThreads) {
-        const int h = idx / D, ch = idx % D;
+    for (int idx = tid; idx < g * (D / 2); idx += kDecodeThreads) {
+        const int h = idx / (D / 2), ch = 2 * (idx % (D / 2));
+        float2 mlw[kDecodeWarps];
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kDecodeWarps; w++) M = fmaxf(M, mm[w * kMaxGqa + h]);
-        float acc = 0.f, Lsum = 0.f;
+        for (int w = 0; w < kDecodeWarps; w++) {
+            mlw[w] = mml[w * kMaxGqa + h];
+            M = fmaxf(M, mlw[w].x);
+        }
+        float2 acc = make_float2(0.f, 0.f);
+        float Lsum = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
             for (int w = 0; w < kDecodeWarps; w++) {
-                const float mw = mm[w * kMaxGqa + h];
-                const float f = (mw == -INFINITY) ? 0.f : ex2(mw - M);
-                acc += f * (macc[(w * kMaxGqa + h) * D + ch] + mz[(w * 4 + VC::group_of_chan(ch)) * kMaxGqa + h]);
-                Lsum += f * ml[w * kMaxGqa + h];
+                const float f = (mlw[w].x == -INFINITY) ? 0.f : ex2(mlw[w].x - M);
+                const float2 a = *reinterpret_cast<const float2 *>(macc + (w * kMaxGqa + h) * C::MS + ch);
+                acc.x = fmaf(f, a.x, acc.x);
+                acc.y = fmaf(f, a.y, acc.y);
+                Lsum = fmaf(f, mlw[w].y, Lsum);
             }
         }
         float *dst = part_base + ((long long)split * g + h) * (D + 4);
-        dst[ch] = acc;
-        if (ch == 0) {
-            dst[D] = M;
-            dst[D + 1] = Lsum;
-        }
+        *reinterpret_cast<float2 *>(dst + ch) = acc;
+        if (ch == 0) *reinterpret_cast<float2 *>(dst + D) = make_float2(M, Lsum);
     }
 
     // ---- last CTA of this (sequence, kv head) merges the splits ----
@@ -1053,108 +1155,134 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     }
     __syncthreads();
     if (!*sflag) return;
-    if (tid == 0) p.counters[b * L.hkv + kvh] = 0u;
 
-    // merge the splits' records straight from L2.  kDecodeWarps / g warps per
-    // head split the records between them; a warp first issues the loads of
-    // all its accumulator rows (lane l: channels l*E .. l*E+E-1), its lanes
-    // load the records' (max, sum) pairs in parallel, then the weighted sum
-    // runs from registers.  The parts meet in shared memory; warp h
-    // normalises head h, applies the inverse rotation and stores.
-    constexpr int REC = D + 4;
-    constexpr int MB = kMergeBatch;
-    const int parts = kDecodeWarps / g;  // >= 1
-    float *wacc = reinterpret_cast<float *>(smem);            // [warp][D]
-    float *wml = wacc + kDecodeWarps * D;                      // [warp][2]
-    if (warp < parts * g) {
-        const int h = warp % g, part = warp / g;
-        const int nmine = (n_active - part + parts - 1) / parts;  // records part, part + parts, ...
-        const float *rec0 = part_base + (long long)h * REC;
-        const long long rstride = (long long)parts * g * REC;     // between this warp's records
-        float M = -INFINITY, Ls = 0.f, o[E];
+    // The splits' records (contiguous, [split][head][D + 4]) come into the
+    // free ring with one bulk copy per piece; warp h turns the piece's
+    // (max, sum) pairs of head h into weights 2^(m_s - M) and the running
+    // (M, L); every thread then accumulates its (head, channel pair) over
+    // the piece from shared memory.
+    float *fw = reinterpret_cast<float *>(smem + C::OFF_FW);  // [split in piece][8]
+    float *fc = reinterpret_cast<float *>(smem + C::OFF_FC);  // [8] rescale of what came before
+    float *fM = reinterpret_cast<float *>(smem + C::OFF_FM);
+    float *fL = reinterpret_cast<float *>(smem + C::OFF_FL);
+    float *frow = reinterpret_cast<float *>(smem + C::OFF_FROW);  // [8][D]
+    const float *recs = reinterpret_cast<const float *>(smem);
+    const uint32_t rbar = smem_u32(smem + C::OFF_RBAR);
+    constexpr int REC = C::REC;
+    const int split_bytes = g * REC * 4;
+    const int per_piece = min(n_active, C::RING / split_bytes);
+    constexpr int OPT = (kMaxGqa * (D / 2) + kDecodeThreads - 1) / kDecodeThreads;  // pairs a thread owns
+    float2 o[OPT];
 #pragma unroll
-        for (int e = 0; e < E; e++) o[e] = 0.f;
-        for (int i0 = 0; i0 < nmine; i0 += MB) {
-            const float *rb = rec0 + (part + (long long)i0 * parts) * g * REC;
-            float a[MB][E];
-#pragma unroll
-            for (int i = 0; i < MB; i++) {  // every load of the batch goes out first
-                if (i0 + i < nmine) {
-                    if constexpr (E == 4) {
-                        const float4 v = __ldcg(reinterpret_cast<const float4 *>(rb + i * rstride + lane * E));
-                        a[i][0] = v.x;
-                        a[i][1] = v.y;
-                        a[i][2] = v.z;
-                        a[i][3] = v.w;
-                    } else {
-                        const float2 v = __ldcg(reinterpret_cast<const float2 *>(rb + i * rstride + lane * E));
-                        a[i][0] = v.x;
-                        a[i][1] = v.y;
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < E; e++) a[i][e] = 0.f;
-                }
+    for (int k = 0; k < OPT; k++) o[k] = make_float2(0.f, 0.f);
+    if (tid < kMaxGqa) {
+        fM[tid] = -INFINITY;
+        fL[tid] = 0.f;
+    }
+    if (tid == 0) {
+        p.counters[b * L.hkv + kvh] = 0u;  // self-resetting for the next call
+        mbar_init(rbar, 1);
+        fence_mbar_init();
+        // the records were written by other CTAs through the generic proxy
+        // and are read here by the bulk-copy (async) proxy
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
+    __syncthreads();
+    bool rec_ok = true;
+    uint32_t rph = 0;
+    for (int s0 = 0; s0 < n_active; s0 += per_piece) {
+        const int ns = min(per_piece, n_active - s0);
+        if (tid == 0)
+            bulk_load(smem_u32(smem), part_base + (long long)s0 * g * REC, (uint32_t)(ns * split_bytes), rbar);
+        rec_ok = __syncthreads_and(mbar_wait_bounded(rbar, rph, kWaitLimitNs));
+        if (!rec_ok) {
+            // record it; wait (bounded) once more so the copy is not left
+            // landing in the shared memory of an exited CTA; no output
+            if (tid == 0) {
+                set_status(p.pool, KVQ_ERR_TIMEOUT);
+                (void)mbar_wait_bounded(rbar, rph, kWaitLimitNs);
             }
-            // lane i: (max, sum) of record i0 + i; the running max moves to
-            // the batch's, rescaling what came before (online merge)
-            float2 ml = make_float2(-INFINITY, 0.f);
-            if (lane < MB && i0 + lane < nmine) ml = __ldcg(reinterpret_cast<const float2 *>(rb + lane * rstride + D));
-            float Mb = ml.x;
+            return;
+        }
+        rph ^= 1u;
+        if (warp < g) {
+            const int h = warp;
+            const float Mold = fM[h];
+            float mloc = -INFINITY, lloc = 0.f, mloc2 = -INFINITY, lloc2 = 0.f;
+            if (lane < ns) {
+                const float2 ml = *reinterpret_cast<const float2 *>(recs + (lane * g + h) * REC + D);
+                mloc = ml.x;
+                lloc = ml.y;
+            }
+            if (lane + 32 < ns) {
+                const float2 ml = *reinterpret_cast<const float2 *>(recs + ((lane + 32) * g + h) * REC + D);
+                mloc2 = ml.x;
+                lloc2 = ml.y;
+            }
+            float Mp = fmaxf(mloc, mloc2);
 #pragma unroll
-            for (int m = 16; m >= 1; m >>= 1) Mb = fmaxf(Mb, __shfl_xor_sync(kFull, Mb, m));
-            const float Mn = fmaxf(M, Mb);
-            const float sc = (M == -INFINITY) ? 0.f : ex2(M - Mn);
-            M = Mn;
-            Ls *= sc;
+            for (int m = 16; m >= 1; m >>= 1) Mp = fmaxf(Mp, __shfl_xor_sync(kFull, Mp, m));
+            const float Mn = fmaxf(Mold, Mp);
+            const float f1 = mloc == -INFINITY ? 0.f : ex2(mloc - Mn);
+            const float f2 = mloc2 == -INFINITY ? 0.f : ex2(mloc2 - Mn);
+            if (lane < ns) fw[lane * kMaxGqa + h] = f1;
+            if (lane + 32 < ns) fw[(lane + 32) * kMaxGqa + h] = f2;
+            float Lp = f1 * lloc + f2 * lloc2;
 #pragma unroll
-            for (int e = 0; e < E; e++) o[e] *= sc;
-            const float f = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M);
-            Ls = fmaf(f, ml.y, Ls);
-#pragma unroll
-            for (int i = 0; i < MB; i++) {
-                const float fi = __shfl_sync(kFull, f, i);
-#pragma unroll
-                for (int e = 0; e < E; e++) o[e] = fmaf(fi, a[i][e], o[e]);
+            for (int m = 16; m >= 1; m >>= 1) Lp += __shfl_xor_sync(kFull, Lp, m);
+            if (lane == 0) {
+                const float c = Mold == -INFINITY ? 0.f : ex2(Mold - Mn);
+                fc[h] = c;
+                fM[h] = Mn;
+                fL[h] = fL[h] * c + Lp;
             }
         }
+        __syncthreads();
 #pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) Ls += __shfl_xor_sync(kFull, Ls, m);
+        for (int k = 0; k < OPT; k++) {
+            const int idx = tid + k * kDecodeThreads;
+            if (idx < g * (D / 2)) {
+                const int h = idx / (D / 2), ch = 2 * (idx % (D / 2));
+                const float c = fc[h];
+                float2 a = make_float2(o[k].x * c, o[k].y * c);
+                for (int sp = 0; sp < ns; sp++) {
+                    const float f = fw[sp * kMaxGqa + h];
+                    const float2 v = *reinterpret_cast<const float2 *>(recs + (sp * g + h) * REC + ch);
+                    a.x = fmaf(f, v.x, a.x);
+                    a.y = fmaf(f, v.y, a.y);
+                }
+                o[k] = a;
+            }
+        }
+        __syncthreads();  // the next piece overwrites the staged records
+    }
 #pragma unroll
-        for (int e = 0; e < E; e++) wacc[warp * D + lane * E + e] = o[e];
-        if (lane == 0) {
-            wml[2 * warp] = M;
-            wml[2 * warp + 1] = Ls;
+    for (int k = 0; k < OPT; k++) {
+        const int idx = tid + k * kDecodeThreads;
+        if (idx < g * (D / 2)) {
+            const int h = idx / (D / 2), ch = 2 * (idx % (D / 2));
+            const float Ls = fL[h];
+            const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+            *reinterpret_cast<float2 *>(frow + h * D + ch) = make_float2(o[k].x * inv, o[k].y * inv);
         }
     }
     __syncthreads();
+    // warp h: inverse rotation of head h's normalised row, then the output
     for (int h = warp; h < g; h += kDecodeWarps) {
-        float M = -INFINITY;
-        for (int pt = 0; pt < parts; pt++) M = fmaxf(M, wml[2 * (pt * g + h)]);
-        float Ls = 0.f, o[E];
+        float v[E];
 #pragma unroll
-        for (int e = 0; e < E; e++) o[e] = 0.f;
-        for (int pt = 0; pt < parts; pt++) {
-            const int w = pt * g + h;
-            const float f = (wml[2 * w] == -INFINITY) ? 0.f : ex2(wml[2 * w] - M);
-            Ls = fmaf(f, wml[2 * w + 1], Ls);
-#pragma unroll
-            for (int e = 0; e < E; e++) o[e] = fmaf(f, wacc[w * D + lane * E + e], o[e]);
-        }
-        if (lane == 0 && p.head_ml) p.head_ml[((long long)b * L.hkv + kvh) * g + h] = make_float2(M, Ls);
-        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-#pragma unroll
-        for (int e = 0; e < E; e++) o[e] *= inv;
+        for (int e = 0; e < E; e++) v[e] = frow[h * D + lane * E + e];
+        if (lane == 0 && p.head_ml) p.head_ml[((long long)b * L.hkv + kvh) * g + h] = make_float2(fM[h], fL[h]);
         if (p.rotate) {
-            fwht_warp<D>(o, lane);
+            fwht_warp<D>(v, lane);
 #pragma unroll
-            for (int e = 0; e < E; e++) o[e] *= p.rot_scale * p.signs[lane * E + e];
+            for (int e = 0; e < E; e++) v[e] *= p.rot_scale * p.signs[lane * E + e];
         }
         float *dst = p.out + ((long long)b * L.hq + kvh * g + h) * D + lane * E;
         if constexpr (E == 4) {
-            *reinterpret_cast<float4 *>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
         } else {
-            *reinterpret_cast<float2 *>(dst) = make_float2(o[0], o[1]);
+            *reinterpret_cast<float2 *>(dst) = make_float2(v[0], v[1]);
         }
     }
 }

@@ -104,6 +104,7 @@ struct kvq_cache {
     int io_next = 0;
     size_t io_bytes = 0;        // record size and buffer of the last call:
     const void *io_buf = nullptr;  // when either changes, the copy waits for both halves
+    int expire_first_wait = 0;  // test hook (kvq_debug_expire_first_wait)
 };
 
 namespace kvq {
@@ -154,6 +155,7 @@ struct DecodeParams {
     // [min(sink, T), max(that, T - recent)) are attended here
     int win_sink, win_recent;
     float2 *head_ml;          // [B][Hkv][g]: totals (M, L) of the softmax, certified mode only
+    int expire_first_wait;    // test hook: each warp's first page wait counts as expired
 };
 
 struct DequantParams {
@@ -330,6 +332,33 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
+}
+
+// The warp-uniform form of a ring refill: every lane executes it, only the
+// lane whose `copy` is set arms the barrier and starts the bulk copy, and only
+// the lane whose `skip` is set arrives on the barrier without a copy (a slot
+// with nothing to load).  Predicated instructions, no branch.
+__device__ __forceinline__ void bulk_load_or_arrive(bool copy, bool skip, uint32_t dst, const void *src,
+                                                    uint32_t bytes, uint32_t bar)
+{
+    asm volatile(
+        "{\n"
+        " .reg .pred pc, ps;\n"
+        " setp.ne.u32 pc, %4, 0;\n"
+        " setp.ne.u32 ps, %5, 0;\n"
+        " @pc mbarrier.arrive.expect_tx.relaxed.cta.shared::cta.b64 _, [%3], %2;\n"
+        " @pc cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+        " @ps mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%3];\n"
+        "}\n" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "r"((uint32_t)copy), "r"((uint32_t)skip)
+        : "memory");
+}
+
+// Hint: bring `bytes` at src into L2 (no data returned, no completion to
+// wait for).  src 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase)

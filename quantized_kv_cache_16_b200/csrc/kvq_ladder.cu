@@ -155,7 +155,9 @@ __global__ void __launch_bounds__(kSelThreads) ladder_select_kernel(const __grid
     for (int bb = tid; bb < nb; bb += kSelThreads) fl[bb] = 0;
     __syncthreads();
 
-    const int k_cov = p.tau_cov > 0.f ? (kcov_s == kNoK ? nb : kcov_s) : 0;
+    // tau_cov >= 1 asks for all of the mass: every block, whatever the
+    // rounded running sum of the estimated masses reaches first
+    const int k_cov = p.tau_cov >= 1.f ? nb : p.tau_cov > 0.f ? (kcov_s == kNoK ? nb : kcov_s) : 0;
     const int k_key = kkey_s == kNoK ? nb : kkey_s;
     int k_cap = 0;
     if (p.frac > 0.f && nb > 0) {

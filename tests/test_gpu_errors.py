@@ -83,3 +83,37 @@ def test_decode_checks_arguments_and_indices():
     K.kvq_decode_attn(c.handle, q, bt, bt.shape[1], ctx, 1, 0.0, None, ws, ws_need, out)
     assert c.sync_status() == K.KVQ_OK
     assert torch.isfinite(out).all()
+
+
+def test_timeout_path_reports_and_recovers():
+    """The bounded-wait path, driven by the library's test hook (no copy is
+    made to stall): every warp's first page wait counts as expired, the warp
+    waits out the copies it started and attends nothing, and the call leaves
+    KVQ_ERR_TIMEOUT for kvq_sync_status.  With the hook off, the next call on
+    the same cache is the oracle's attention again."""
+    torch = _torch()
+    from _cases import TOL_MAX_ABS, TOL_REL_L2, attn_errors
+    import oracle as O
+    wl = W.scaled(W.llama(), [1000])
+    pair = build_pair(wl)
+    c = pair.cache
+    qn = W.queries(wl, 0)
+    q = torch.from_numpy(qn).cuda()
+    bt = pair.block_table()
+    ctx = pair.ctx()
+    ws_need = K.kvq_decode_workspace_bytes(c.handle, 1, bt.shape[1])
+    ws = torch.zeros(ws_need, dtype=torch.uint8, device="cuda")
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    with pytest.raises(K.KvqError):
+        K.kvq_debug_expire_first_wait(c.handle, 2)
+    K.kvq_debug_expire_first_wait(c.handle, 1)
+    try:
+        K.kvq_decode_attn(c.handle, q, bt, bt.shape[1], ctx, 1, 0.0, None, ws, ws_need, out)
+        assert c.sync_status() == K.KVQ_ERR_TIMEOUT
+    finally:
+        K.kvq_debug_expire_first_wait(c.handle, 0)
+    K.kvq_decode_attn(c.handle, q, bt, bt.shape[1], ctx, 1, 0.0, None, ws, ws_need, out)
+    assert c.sync_status() == K.KVQ_OK
+    want = O.decode(pair.ocfg, pair.opool, qn, pair.pages.block_table, wl.ctx)
+    max_abs, rel = attn_errors(out.cpu().numpy(), want)
+    assert max_abs <= TOL_MAX_ABS and rel <= TOL_REL_L2, (max_abs, rel)

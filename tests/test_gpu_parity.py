@@ -215,6 +215,69 @@ def _host_record(cache, wl, step, slots, ctx):
     return torch.from_numpy(rec).pin_memory()
 
 
+def _record_of(cache, q, k, v, slots, ctx):
+    """kvq_decode_step_host's pinned record of explicit arrays (sections
+    16-byte aligned: q, k_new, v_new, slots, ctx lengths)."""
+    import torch
+    import quantized_kv_cache_16_b200 as K
+    up = lambda n: (n + 15) // 16 * 16
+    parts = [q.view(np.uint8).ravel(), k.view(np.uint8).ravel(), v.view(np.uint8).ravel(),
+             np.asarray(slots, np.int32).view(np.uint8), np.asarray(ctx, np.int32).view(np.uint8)]
+    rec = np.zeros(K.kvq_step_record_bytes(cache.handle, q.shape[0]), np.uint8)
+    off = 0
+    for a in parts:
+        rec[off:off + a.size] = a
+        off += up(a.size)
+    assert off == rec.size
+    return torch.from_numpy(rec).pin_memory()
+
+
+def test_decode_step_host_back_to_back():
+    """Six kvq_decode_step_host calls issued with no synchronisation between
+    them, each with its own pinned record and output: the record copy of a
+    step runs on the library's copy stream while the previous step's kernel
+    may still read the other buffer half.  In mid-run the device record
+    buffer changes (step 2) and so does the batch, hence the record size
+    (step 4): both must wait for the two halves still in use.  After one
+    synchronisation every step's output and the final pool bytes equal those
+    of kvq_decode_step run one step at a time on device copies."""
+    import torch
+    import quantized_kv_cache_16_b200 as K
+    wl = W.scaled(W.llama(), [700, 45, 16])
+    host = build_pair(wl, extra_tokens=8, oracle=False)
+    devp = build_pair(wl, extra_tokens=8, oracle=False)
+    P = host.pages.block_table.shape[1]
+    ws = host.cache.workspace_for(wl.B, P)
+    d_recs = [torch.empty(2 * K.kvq_step_record_bytes(host.cache.handle, wl.B), dtype=torch.uint8, device="cuda")
+              for _ in range(2)]
+    plan = [(0, 3), (0, 3), (1, 3), (1, 3), (1, 2), (1, 2)]  # (device record buffer, batch) of each step
+    pos = list(wl.ctx)
+    rng = np.random.default_rng(11)
+    bt_h = host.block_table()
+    steps = []
+    for step, (buf, B) in enumerate(plan):
+        q = rng.standard_normal((B, wl.Hq, wl.d)).astype(np.float16)
+        k = rng.standard_normal((B, wl.Hkv, wl.d)).astype(np.float16)
+        v = (0.5 * rng.standard_normal((B, wl.Hkv, wl.d))).astype(np.float16)
+        slots = np.array([host.pages.slot(b, pos[b]) for b in range(B)], np.int32)
+        ctx = np.array([pos[b] + 1 for b in range(B)], np.int32)
+        for b in range(B):
+            pos[b] += 1
+        h_in = _record_of(host.cache, q, k, v, slots, ctx)
+        h_out = torch.full((B, wl.Hq, wl.d), float("nan"), dtype=torch.float32).pin_memory()
+        K.kvq_decode_step_host(host.cache.handle, h_in, d_recs[buf], bt_h[:B], P, B, 0.0, ws, ws.numel(), h_out)
+        steps.append((q, k, v, slots, ctx, B, h_in, h_out))
+    torch.cuda.synchronize()
+    bt_d = devp.block_table()
+    for step, (q, k, v, slots, ctx, B, _, h_out) in enumerate(steps):
+        want = devp.cache.step(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(), torch.from_numpy(slots).cuda(),
+                               torch.from_numpy(q).cuda(), bt_d[:B], torch.from_numpy(ctx).cuda())
+        torch.cuda.synchronize()
+        assert np.array_equal(h_out.numpy(), want.cpu().numpy()), f"step {step}"
+    assert np.array_equal(host.cache.pool.cpu().numpy()[256:], devp.cache.pool.cpu().numpy()[256:])
+    assert host.cache.sync_status() == 0 and devp.cache.sync_status() == 0
+
+
 def test_decode_step_host_equals_the_device_step():
     """kvq_decode_step_host (the pinned host record copied in on the
     library's copy stream into alternating buffers, the kernel writing the
