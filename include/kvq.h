@@ -420,15 +420,20 @@ kvq_status kvq_decode_attn_static(kvq_cache *cache, const void *q, const int32_t
 kvq_status kvq_dequant_debug(kvq_cache *cache, const int32_t *slots, int32_t n, float *k_out, float *v_out,
                              uint8_t *codes_out, uint16_t *meta_out, void *stream);
 
-/* Test hook for the bounded waits (the pages have no counterpart of it).
- * With on = 1, the decode kernels that kvq_decode_attn and kvq_decode_step
- * launch treat each warp's first page wait as expired: the warp records
- * KVQ_ERR_TIMEOUT in the status word, waits (bounded, the normal one-second
- * limit) for the page copies it has already started, and attends no page,
- * so the output of such a call is not the attention.  on = 0 restores the
- * normal waits.  It lets a test drive the timeout path, which otherwise
- * needs a copy that never completes, without hanging or faulting the GPU.
- * Returns KVQ_ERR_INVALID_ARG for a null cache or on outside {0, 1}. */
+/* Test hooks of the decode kernels that kvq_decode_attn and kvq_decode_step
+ * launch (the pages have no counterpart of them).  They let a test drive
+ * paths that otherwise need a copy that never completes or a block table
+ * changed by the previous kernel, without hanging or faulting the GPU.
+ *   on = 1: each warp's first page wait counts as expired: the warp records
+ *           KVQ_ERR_TIMEOUT in the status word, waits (bounded, the normal
+ *           one-second limit) for the page copies it has already started,
+ *           and attends no page, so the output is not the attention;
+ *   on = 2: the page copies a warp starts from the block-table entries it
+ *           read before the previous kernel finished count as wrong guesses:
+ *           it waits them out and copies those pages again (the output is
+ *           the attention);
+ *   on = 0: normal operation.
+ * Returns KVQ_ERR_INVALID_ARG for a null cache or on outside {0, 1, 2}. */
 kvq_status kvq_debug_expire_first_wait(kvq_cache *cache, int32_t on);
 
 /* Synchronise the cache's last stream use and return (then clear) the device

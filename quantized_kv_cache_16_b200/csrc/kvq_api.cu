@@ -418,6 +418,8 @@ DecodeParams decode_params(kvq_cache *c, const SplitPlan &s, const void *q, cons
     p.rot_scale = c->rot_scale;
     p.rotate = c->cfg.rotate;
     memcpy(p.signs, c->signs, sizeof(p.signs));
+    for (int i = 0; i < kMaxD; i++)
+        if (c->signs[i] < 0.0f) p.sign_bits[i / 32] |= 1u << (i % 32);
     p.pages_per_split = s.pages_per_split;
     p.pages_per_warp = s.pages_per_warp;
     p.n_splits = s.n_splits;
@@ -762,7 +764,7 @@ size_t kvq_step_record_bytes(const kvq_cache *c, int32_t batch)
 
 kvq_status kvq_debug_expire_first_wait(kvq_cache *c, int32_t on)
 {
-    if (!c || (on != 0 && on != 1)) return KVQ_ERR_INVALID_ARG;
+    if (!c || on < 0 || on > 2) return KVQ_ERR_INVALID_ARG;
     c->expire_first_wait = on;
     return KVQ_OK;
 }

@@ -66,6 +66,29 @@ __device__ __forceinline__ void quant_pair(float2 y, float2 z2, float2 inv2, flo
     c1 = __float_as_uint(t.y);
 }
 
+// The same codes for rows whose largest element already codes at most the
+// top code: every step (subtract, multiply by inv > 0 or 0, add the rounding
+// magic) is monotone in y, so no element needs the upper clamp.  The lower
+// clamp stays: it also keeps the multiply and the add apart (fused into one
+// multiply-add they would round once where the codec rounds twice, and a
+// product just below a half-way point that rounds up onto it would then
+// code differently).
+__device__ __forceinline__ void quant_pair_lo(float2 y, float2 z2, float2 inv2, float lo, uint32_t &c0, uint32_t &c1)
+{
+    float2 t = __fmul2_rn(sub2(y, z2), inv2);
+    t.x = fmaxf(t.x, lo);
+    t.y = fmaxf(t.y, lo);
+    t = __fadd2_rn(t, make_float2(kRoundMagic, kRoundMagic));
+    c0 = __float_as_uint(t.x);
+    c1 = __float_as_uint(t.y);
+}
+
+// The unclamped integer code of one value, by the same operations.
+__device__ __forceinline__ int code_of(float y, float z, float inv)
+{
+    return (int)(__float_as_uint(__fadd_rn(__fmul_rn(__fsub_rn(y, z), inv), kRoundMagic)) - 0x4B400000u);
+}
+
 // min / max over the row's lanes (lane and lane ^ 16 for d = 128)
 template <int LANES> __device__ __forceinline__ float row_min(float v)
 {
@@ -239,11 +262,14 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
     if (FMT == KVQ_INT4_ASYM) {
         // two groups of 32 per lane (16 pairs each), one 16-byte chunk each
         uint32_t sz[2][2];  // [scale|zero][group] fp16 bits
+        float zfs[2], infs[2], sfs[2];
+        bool fits = true;  // both groups' largest elements code at most 15
 #pragma unroll
         for (int gq = 0; gq < 2; gq++) {
             const float2 *yg = y + 16 * gq;
             float lo, hi;
             pair_minmax<16>(yg, lo, hi);
+            const float hi_y = hi;
             if (p.clip < 1.0f) {
                 lo = __fmul_rn(lo, p.clip);
                 hi = __fmul_rn(hi, p.clip);
@@ -251,25 +277,47 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
             __half shh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
             const __half zhh = __float2half_rn(lo);
             if constexpr (SEARCH) shh = search_scale<16, 1>(yg, shh, __half2float(zhh), 0.0f, 15.0f);
-            const float sf = __half2float(shh), zf = __half2float(zhh);
-            const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
-            const float2 z2 = make_float2(zf, zf), inv2 = make_float2(inv, inv), s2 = make_float2(sf, sf);
-            uint32_t w[4];
-#pragma unroll
-            for (int m = 0; m < 4; m++) {
-                uint32_t bb[4];
-#pragma unroll
-                for (int k = 0; k < 4; k++) {
-                    uint32_t c0, c1;
-                    quant_pair(yg[4 * m + k], z2, inv2, 0.0f, 15.0f, c0, c1);
-                    if (want_desc) pair_err(yg[4 * m + k], c0, c1, s2, z2, emax, amax);
-                    bb[k] = c0 + (c1 << 4);
-                }
-                w[m] = pack4bytes(bb[0], bb[1], bb[2], bb[3]);
-            }
-            if (active) *reinterpret_cast<uint4 *>(codes + ((2 * s + gq) * 16 + tok) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+            sfs[gq] = __half2float(shh);
+            zfs[gq] = __half2float(zhh);
+            infs[gq] = (sfs[gq] == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sfs[gq]);
+            fits = fits && code_of(hi_y, zfs[gq], infs[gq]) <= 15;
             sz[0][gq] = __half_as_ushort(shh);
             sz[1][gq] = __half_as_ushort(zhh);
+        }
+        fits = __all_sync(kFull, fits || !active);
+#pragma unroll
+        for (int gq = 0; gq < 2; gq++) {
+            const float2 *yg = y + 16 * gq;
+            const float2 z2 = make_float2(zfs[gq], zfs[gq]), inv2 = make_float2(infs[gq], infs[gq]);
+            const float2 s2 = make_float2(sfs[gq], sfs[gq]);
+            uint32_t w[4];
+            if (fits && !want_desc) {
+#pragma unroll
+                for (int m = 0; m < 4; m++) {
+                    uint32_t bb[4];
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        uint32_t c0, c1;
+                        quant_pair_lo(yg[4 * m + k], z2, inv2, 0.0f, c0, c1);
+                        bb[k] = c0 + (c1 << 4);
+                    }
+                    w[m] = pack4bytes(bb[0], bb[1], bb[2], bb[3]);
+                }
+            } else {
+#pragma unroll
+                for (int m = 0; m < 4; m++) {
+                    uint32_t bb[4];
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        uint32_t c0, c1;
+                        quant_pair(yg[4 * m + k], z2, inv2, 0.0f, 15.0f, c0, c1);
+                        if (want_desc) pair_err(yg[4 * m + k], c0, c1, s2, z2, emax, amax);
+                        bb[k] = c0 + (c1 << 4);
+                    }
+                    w[m] = pack4bytes(bb[0], bb[1], bb[2], bb[3]);
+                }
+            }
+            if (active) *reinterpret_cast<uint4 *>(codes + ((2 * s + gq) * 16 + tok) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         if (active) {
             constexpr int NG = D / 32;
@@ -282,6 +330,7 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
         pair_minmax<32>(y, lo, hi);
         lo = row_min<LANES>(lo);
         hi = row_max<LANES>(hi);
+        const float hi_y = hi;
         if (p.clip < 1.0f) {
             lo = __fmul_rn(lo, p.clip);
             hi = __fmul_rn(hi, p.clip);
@@ -292,22 +341,40 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
         const float sf = __half2float(shh), zf = __half2float(zhh);
         const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
         const float2 z2 = make_float2(zf, zf), inv2 = make_float2(inv, inv), s2 = make_float2(sf, sf);
+        // the row's largest element codes at most 3 (clipping leaves it there
+        // for rows around zero): then no element needs the upper clamp
+        const bool fits = __all_sync(kFull, code_of(hi_y, zf, inv) <= 3 || !active);
         uint32_t w[4];
+        if (fits && !want_desc) {
 #pragma unroll
-        for (int m = 0; m < 4; m++) {
-            uint32_t bb[4];
+            for (int m = 0; m < 4; m++) {
+                uint32_t bb[4];
 #pragma unroll
-            for (int k = 0; k < 4; k++) {
-                uint32_t c[4];
-                quant_pair(y[8 * m + 2 * k], z2, inv2, 0.0f, 3.0f, c[0], c[1]);
-                quant_pair(y[8 * m + 2 * k + 1], z2, inv2, 0.0f, 3.0f, c[2], c[3]);
-                if (want_desc) {
-                    pair_err(y[8 * m + 2 * k], c[0], c[1], s2, z2, emax, amax);
-                    pair_err(y[8 * m + 2 * k + 1], c[2], c[3], s2, z2, emax, amax);
+                for (int k = 0; k < 4; k++) {
+                    uint32_t c[4];
+                    quant_pair_lo(y[8 * m + 2 * k], z2, inv2, 0.0f, c[0], c[1]);
+                    quant_pair_lo(y[8 * m + 2 * k + 1], z2, inv2, 0.0f, c[2], c[3]);
+                    bb[k] = c[0] + (c[1] << 2) + (c[2] << 4) + (c[3] << 6);
                 }
-                bb[k] = c[0] + (c[1] << 2) + (c[2] << 4) + (c[3] << 6);
+                w[m] = pack4bytes(bb[0], bb[1], bb[2], bb[3]);
             }
-            w[m] = pack4bytes(bb[0], bb[1], bb[2], bb[3]);
+        } else {
+#pragma unroll
+            for (int m = 0; m < 4; m++) {
+                uint32_t bb[4];
+#pragma unroll
+                for (int k = 0; k < 4; k++) {
+                    uint32_t c[4];
+                    quant_pair(y[8 * m + 2 * k], z2, inv2, 0.0f, 3.0f, c[0], c[1]);
+                    quant_pair(y[8 * m + 2 * k + 1], z2, inv2, 0.0f, 3.0f, c[2], c[3]);
+                    if (want_desc) {
+                        pair_err(y[8 * m + 2 * k], c[0], c[1], s2, z2, emax, amax);
+                        pair_err(y[8 * m + 2 * k + 1], c[2], c[3], s2, z2, emax, amax);
+                    }
+                    bb[k] = c[0] + (c[1] << 2) + (c[2] << 4) + (c[3] << 6);
+                }
+                w[m] = pack4bytes(bb[0], bb[1], bb[2], bb[3]);
+            }
         }
         if (active) {
             *reinterpret_cast<uint4 *>(codes + (s * 16 + tok) * 16) = make_uint4(w[0], w[1], w[2], w[3]);

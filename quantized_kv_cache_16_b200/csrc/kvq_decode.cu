@@ -53,13 +53,36 @@ __device__ __forceinline__ uint32_t hfma2u(uint32_t a, uint32_t b, uint32_t c)
     return h2_bits(__hfma2(bits_h2(a), bits_h2(b), bits_h2(c)));
 }
 
+// (a & m) | c in one three-input logic instruction.  The masks come in as
+// registers (see nib_masks): with both as immediates the compiler splits the
+// operation in two.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t m, uint32_t c)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(m), "r"(c));
+    return d;
+}
+
+// The three constants of nib, held in registers for the whole loop.
+struct NibMasks {
+    uint32_t lo, hi, h1024;
+};
+__device__ __forceinline__ NibMasks nib_masks()
+{
+    NibMasks m;
+    asm volatile("mov.b32 %0, 0x000F000F;" : "=r"(m.lo));
+    asm volatile("mov.b32 %0, 0x00F000F0;" : "=r"(m.hi));
+    asm volatile("mov.b32 %0, 0x64006400;" : "=r"(m.h1024));
+    return m;
+}
+
 // Nibble n (0..3) of each 16-bit half of w as exact fp16 integers:
 // (w & mask) | 0x6400 is 1024 + c * 16^(n&1); subtract / rescale exactly.
-__device__ __forceinline__ uint32_t nib(uint32_t w, int n)
+__device__ __forceinline__ uint32_t nib(uint32_t w, int n, const NibMasks &k)
 {
     const uint32_t x = (n & 2) ? (w >> 8) : w;
-    if (n & 1) return hfma2u((x & 0x00F000F0u) | kH1024, 0x2C002C00u /*1/16*/, 0xD400D400u /*-64*/);
-    return hsub2u((x & 0x000F000Fu) | kH1024, kH1024);
+    if (n & 1) return hfma2u(and_or(x, k.hi, k.h1024), 0x2C002C00u /*1/16*/, 0xD400D400u /*-64*/);
+    return hsub2u(and_or(x, k.lo, k.h1024), kH1024);
 }
 
 // 2-bit field f (0..7) of each 16-bit half as exact fp16 integers.
@@ -145,6 +168,22 @@ __device__ __forceinline__ void mma16816_z(float *d, const uint32_t *a, uint32_t
 }
 
 
+// The signs of a lane's E consecutive elements (lane*E .. lane*E+E-1) as
+// bits (1 = negative), from the per-call bit words: a per-lane index into
+// the parameter space touches at most four words, not one address per lane.
+template <int E>
+__device__ __forceinline__ uint32_t lane_sign_bits(const uint32_t (&bits)[kMaxD / 32], int lane)
+{
+    return (bits[(lane * E) >> 5] >> ((lane * E) & 31)) & ((1u << E) - 1u);
+}
+
+// x with its sign flipped where bit e of sg is set (multiplication by +-1,
+// exactly)
+__device__ __forceinline__ float flip_sign(float x, uint32_t sg, int e)
+{
+    return __uint_as_float(__float_as_uint(x) ^ (((sg >> e) & 1u) << 31));
+}
+
 // ------------------------------------------------------------ fused append ---
 // Quantise-on-append of one K or V row by a whole warp: lane l holds elements
 // [l*E, l*E+E).  Same fp32 operations in the same order as the append kernel
@@ -177,7 +216,7 @@ template <int LANES> __device__ __forceinline__ float group_max(float v)
 }
 
 template <int D, int FMT>
-__device__ __forceinline__ void warp_append_row(const __half *src, const float *signs, int rotate, float rot_scale,
+__device__ __forceinline__ void warp_append_row(const __half *src, uint32_t sg, int rotate, float rot_scale,
                                                 float clip, unsigned char *codes, unsigned char *meta_row, int tok,
                                                 unsigned int *desc, int tensor, int lane)
 {
@@ -197,7 +236,7 @@ __device__ __forceinline__ void warp_append_row(const __half *src, const float *
     }
     if (rotate) {
 #pragma unroll
-        for (int e = 0; e < E; e++) x[e] = __fmul_rn(x[e], signs[lane * E + e]);
+        for (int e = 0; e < E; e++) x[e] = flip_sign(x[e], sg, e);
 #pragma unroll
         for (int h = 1; h < E; h <<= 1)
 #pragma unroll
@@ -395,12 +434,12 @@ template <int D> struct VCodec<KVQ_INT4_ASYM, D> {
     __device__ static int chan(int mt, int row) { return 32 * (mt >> 1) + 4 * (row & 7) + 2 * (mt & 1) + (row >> 3); }
     __device__ static int group_of_mt(int mt) { return mt >> 1; }
     __device__ static int group_of_chan(int ch) { return ch / 32; }
-    __device__ static void afrag(uint32_t wA, uint32_t wB, int u, uint32_t (&a)[4])
+    __device__ static void afrag(uint32_t wA, uint32_t wB, int u, uint32_t (&a)[4], const NibMasks &k)
     {
-        a[0] = nib(wA, 2 * u);
-        a[1] = nib(wA, 2 * u + 1);
-        a[2] = nib(wB, 2 * u);
-        a[3] = nib(wB, 2 * u + 1);
+        a[0] = nib(wA, 2 * u, k);
+        a[1] = nib(wA, 2 * u + 1, k);
+        a[2] = nib(wB, 2 * u, k);
+        a[3] = nib(wB, 2 * u + 1, k);
     }
 };
 
@@ -412,7 +451,7 @@ template <int D> struct VCodec<KVQ_INT2_ASYM, D> {
     __device__ static int chan(int mt, int row) { return 64 * (mt >> 2) + 8 * (row & 7) + 2 * (mt & 3) + (row >> 3); }
     __device__ static int group_of_mt(int) { return 0; }
     __device__ static int group_of_chan(int) { return 0; }
-    __device__ static void afrag(uint32_t wA, uint32_t wB, int u, uint32_t (&a)[4])
+    __device__ static void afrag(uint32_t wA, uint32_t wB, int u, uint32_t (&a)[4], const NibMasks &)
     {
         a[0] = fld2(wA, 2 * u);
         a[1] = fld2(wA, 2 * u + 1);
@@ -561,21 +600,25 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     // this CTA may start while that grid is still finishing.  Until
     // griddepcontrol.wait returns, nothing read can be trusted (the previous
     // kernel may be writing the context lengths, the block table, the query
-    // or the pages), so this phase only warms L2: the context length and this
-    // warp's block-table entries are read as hints (L2 only, never kept in
-    // L1), clamped into the pool, and the pages they name are prefetched
-    // into L2.  A stale hint costs a wasted prefetch, never a wrong result:
-    // every value used below is read again after the wait.
+    // or the pages), so this phase only reads hints and warms L2: the context
+    // length and this warp's block-table entries are read (L2 only, never
+    // kept in L1), clamped into the pool, and the pages they name, the
+    // query rows and the appended rows are prefetched into L2.
+    extern __shared__ __align__(128) unsigned char smem[];
+    const uint32_t bar0 = smem_u32(smem + C::OFF_BAR) + warp * NST * 8;
+    const int p_begin = split * p.pages_per_split + warp * p.pages_per_warp;
+    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
+    int Th, id_h = -1;  // hints: the context length, page p_begin + lane
     {
-        int Th = __ldcg(p.ctx_lens + b);
-        Th = min(max(Th, 0), p.max_pages * kPageTokens);
-        const int pg0 = split * p.pages_per_split + warp * p.pages_per_warp;
-        const int npg_h = min(pg0 + p.pages_per_warp, (Th + kPageTokens - 1) / kPageTokens) - pg0;
-        if (lane < npg_h) {
-            const int pg = __ldcg(p.block_table + (long long)b * p.max_pages + pg0 + lane);
-            if (pg >= 0 && pg < L.num_pages)
+        Th = min(max(__ldcg(p.ctx_lens + b), 0), p.max_pages * kPageTokens);
+        const int npg_h = min(p_begin + p.pages_per_warp, (Th + kPageTokens - 1) / kPageTokens) - p_begin;
+        if (lane < npg_h && lane < 32) {
+            const int pg = __ldcg(bt + p_begin + lane);
+            if (pg >= 0 && pg < L.num_pages) {
+                id_h = pg;
                 bulk_prefetch_l2(p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes + (long long)pg * L.page_bytes,
                                  L.chunk_bytes);
+            }
         }
         // the group's query rows (contiguous) and the rows the step appends
         if (warp == 0 && lane == 31) bulk_prefetch_l2(p.q + ((long long)b * L.hq + kvh * g) * D, g * D * 2);
@@ -583,17 +626,19 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             bulk_prefetch_l2(p.new_k + ((long long)b * L.hkv + kvh) * D, D * 2);
             bulk_prefetch_l2(p.new_v + ((long long)b * L.hkv + kvh) * D, D * 2);
         }
+        if (lane == 0) {  // the ring's barriers (this CTA's own shared memory)
+            for (int s = 0; s < NST; s++) mbar_init(bar0 + 8 * s, 1);
+            fence_mbar_init();
+        }
     }
     // wait for the previous grid to complete (its writes visible), then let
     // the next dependent grid be set up early
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    // independent loads first: the context length, this warp's first 32
-    // block-table entries (speculative) and the query row all go out together
+    // the true values: the context length, this warp's first 32 block-table
+    // entries and the query row all go out together, ahead of any copy
     int T = p.ctx_lens[b];
-    const int p_begin = split * p.pages_per_split + warp * p.pages_per_warp;
-    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
     const int id_raw = (lane < p.pages_per_warp && p_begin + lane < p.max_pages) ? bt[p_begin + lane] : -1;
     uint2 q_raw = make_uint2(0u, 0u);
     if (warp < g) {
@@ -601,34 +646,42 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         if constexpr (E == 4) q_raw = *reinterpret_cast<const uint2 *>(qh);
         else q_raw.x = *reinterpret_cast<const uint32_t *>(qh);
     }
-    extern __shared__ __align__(128) unsigned char smem[];
-    const uint32_t bar0 = smem_u32(smem + C::OFF_BAR) + warp * NST * 8;
-    if (lane == 0) {  // the ring's barriers, while the loads above are in flight
-        for (int s = 0; s < NST; s++) mbar_init(bar0 + 8 * s, 1);
-        fence_mbar_init();
+
+    // The contents of every page are final now; only the page ids of the
+    // hints are guesses.  The first copies go out at once from them, while
+    // the loads above are in flight.  A guess that turns out wrong is waited
+    // out and its copy made again.
+    const uint32_t stage0 = smem_u32(smem) + warp * NST * C::STAGE;
+    const unsigned char *stage0_ptr = smem + warp * NST * C::STAGE;
+    const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
+    int n_spec = 0;
+    {
+        const unsigned lead = __ballot_sync(kFull, id_h >= 0);
+        n_spec = min(NST, __ffs(~lead) - 1 < 0 ? 32 : __ffs(~lead) - 1);
+        for (int i = 0; i < n_spec; i++) {
+            const int pg = __shfl_sync(kFull, id_h, i);
+            bulk_load_or_arrive(lane == 0, false, stage0 + i * C::STAGE, kv_base + (long long)pg * L.page_bytes,
+                                C::CHUNK, bar0 + 8 * i);
+        }
     }
+
     if (T < 0 || T > p.max_pages * kPageTokens) {
         if (split == 0 && tid == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
         T = T < 0 ? 0 : p.max_pages * kPageTokens;
     }
     const int n_pages = (T + kPageTokens - 1) / kPageTokens;
     const int n_active = max(1, (n_pages + p.pages_per_split - 1) / p.pages_per_split);
-    if (split >= n_active) return;
     const int q_lo = min(p.win_sink, T), q_hi = max(q_lo, T - p.win_recent);  // tokens attended here
 
     int8_t *qv = reinterpret_cast<int8_t *>(smem + C::OFF_QV);
     float *qsum = reinterpret_cast<float *>(smem + C::OFF_QSUM);
     int *qexp = reinterpret_cast<int *>(smem + C::OFF_QEXP);
     int *sflag = reinterpret_cast<int *>(smem + C::OFF_FLAG);
-    const uint32_t stage0 = smem_u32(smem) + warp * NST * C::STAGE;
-    const unsigned char *stage0_ptr = smem + warp * NST * C::STAGE;
 
-    // ---- this warp's pages: barriers and the first copies go out before
-    //      any query work, so the page data is in flight during it ----
+    // ---- this warp's pages: the first copies go out before any query work,
+    //      so the page data is in flight during it ----
     const int p_end = min(p_begin + p.pages_per_warp, n_pages);
-    const int npg = max(0, p_end - p_begin);
-    const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
-    __syncwarp();
+    const int npg = split >= n_active ? 0 : max(0, p_end - p_begin);
 
     auto fetch_ids = [&](int i0) -> int {
         const int i = i0 + lane;
@@ -650,7 +703,23 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             ids = -1;
         }
     }
-    uint32_t vbits = 0;      // bit s: stage s holds a valid page
+    const bool appends = p.new_k != nullptr && T > 0 && npg > 0 && n_pages - 1 >= p_begin && n_pages - 1 < p_end;
+    // the guesses hold if page i < n_spec is the true page i (the test
+    // hook's mode 2 discards them all)
+    const bool spec_ok = __all_sync(kFull, lane >= n_spec || (lane < npg && ids == id_h)) && p.expire_first_wait != 2;
+    uint32_t phm = 0;  // bit s: the parity stage s's next page completes
+    int n_done = n_spec;
+    if (!spec_ok && n_spec > 0) {
+        // wait (bounded) for the guessed copies, so none lands on a stage that
+        // is refilled or of a CTA that has left; their stages move on a phase
+        bool landed = true;
+        for (int i = 0; i < n_spec; i++) landed &= mbar_wait_bounded(bar0 + 8 * i, 0, kWaitLimitNs);
+        if (!__all_sync(kFull, landed) && lane == 0) set_status(p.pool, KVQ_ERR_TIMEOUT);
+        phm = (1u << n_spec) - 1u;
+        n_done = 0;
+    }
+    if (split >= n_active) return;
+    uint32_t vbits = (1u << n_done) - 1u;  // bit s: stage s holds a valid page
     auto issue = [&](int i) {  // every lane calls this; lane 0 alone copies (predicated, no branch)
         const int pg = __shfl_sync(kFull, ids, i & 31);
         const int st = i % NST;
@@ -661,36 +730,34 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         bulk_load_or_arrive(lane == 0 && pg >= 0, lane == 0 && pg < 0, stage0 + st * C::STAGE,
                             kv_base + (long long)max(pg, 0) * L.page_bytes, C::CHUNK, bar0 + 8 * st);
     };
-    // fused append: the warp that owns the page of position T-1 quantises
-    // the new token's K and V rows into it before any copy of that page.
-    // That page is the warp's last; the copies of the pages before it go out
-    // first, so the append's latency overlaps them.
-    const bool appends = p.new_k != nullptr && T > 0 && n_pages - 1 >= p_begin && n_pages - 1 < p_end;
     const int n_first = min(NST, npg);
-    const int n_pre = (appends && n_first == npg) ? npg - 1 : n_first;
-    for (int i = 0; i < n_pre; i++) issue(i);
+    for (int i = n_done; i < n_first; i++) issue(i);
+    // Fused append: the warp that owns the page of position T-1 quantises
+    // the new token's K and V rows into the pool.  Its copy of that page (its
+    // last) may or may not see those stores, so when the page arrives the
+    // warp writes the same row into the staged copy too (see the page loop);
+    // nothing orders the stores before the copy, and no other warp waits.
+    const int app_tok = (T - 1) % kPageTokens;
+    bool app_ok = false;
+    const long long app_row = ((long long)b * L.hkv + kvh) * D;
+    const uint32_t app_sg = lane_sign_bits<E>(p.sign_bits, lane);
     if (appends) {
         const int pg = bt[n_pages - 1];
         const int slot = p.new_slots[b];
-        const int tok = (T - 1) % kPageTokens;
-        if (pg < 0 || pg >= L.num_pages || slot != pg * kPageTokens + tok) {
+        if (pg < 0 || pg >= L.num_pages || slot != pg * kPageTokens + app_tok) {
             if (lane == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
         } else {
+            app_ok = true;
             unsigned char *chunk = const_cast<unsigned char *>(kv_base) + (long long)pg * L.page_bytes;
             unsigned int *desc = L.desc_off ? reinterpret_cast<unsigned int *>(const_cast<unsigned char *>(p.pool) +
                                                                                 L.desc_off + ((long long)pg * L.hkv + kvh) * 16)
                                             : nullptr;
-            const long long row = ((long long)b * L.hkv + kvh) * D;
-            warp_append_row<D, KF>(p.new_k + row, p.signs, p.rotate, p.rot_scale, p.clip, chunk + L.k_codes,
-                                   chunk + L.k_meta + tok * L.k_row_meta, tok, desc, 0, lane);
-            warp_append_row<D, VF>(p.new_v + row, p.signs, p.rotate, p.rot_scale, p.clip, chunk + L.v_codes,
-                                   chunk + L.v_meta + tok * L.v_row_meta, tok, desc, 1, lane);
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) asm volatile("fence.proxy.async.global;" ::: "memory");
+            warp_append_row<D, KF>(p.new_k + app_row, app_sg, p.rotate, p.rot_scale, p.clip, chunk + L.k_codes,
+                                   chunk + L.k_meta + app_tok * L.k_row_meta, app_tok, desc, 0, lane);
+            warp_append_row<D, VF>(p.new_v + app_row, app_sg, p.rotate, p.rot_scale, p.clip, chunk + L.v_codes,
+                                   chunk + L.v_meta + app_tok * L.v_row_meta, app_tok, desc, 1, lane);
         }
     }
-    for (int i = n_pre; i < n_first; i++) issue(i);
 
     // ---- query (warp h): rotate, pre-scale, group sums, and the three signed
     //      7-bit digits of q * 2^E written straight into the B layout ----
@@ -712,7 +779,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         float sc = p.qscale;
         if (p.rotate) {
 #pragma unroll
-            for (int e = 0; e < E; e++) x[e] *= p.signs[lane * E + e];
+            for (int e = 0; e < E; e++) x[e] = flip_sign(x[e], lane_sign_bits<E>(p.sign_bits, lane), e);
             fwht_warp<D>(x, lane);
             sc *= p.rot_scale;
         }
@@ -804,9 +871,12 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
 
     float oacc[NH][C::MT][4];
     float oz[NH][4];
-    float m_run[NH], l_part[NH];
+    // m_ref: the exponentials' reference, m_run while it is finite; before
+    // any token every score is -inf and ex2(-inf - (-inf)) would be NaN
+    float m_run[NH], l_part[NH], m_ref[NH];
 #pragma unroll
     for (int t = 0; t < NH; t++) {
+        m_ref[t] = 0.f;
 #pragma unroll
         for (int mt = 0; mt < C::MT; mt++) oacc[t][mt][0] = oacc[t][mt][1] = oacc[t][mt][2] = oacc[t][mt][3] = 0.f;
         oz[t][0] = oz[t][1] = oz[t][2] = oz[t][3] = 0.f;
@@ -820,20 +890,19 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     // Iterations [i_full0, i_full1) are the warp's pages inside [q_lo, q_hi).
     const int i_full0 = (q_lo + kPageTokens - 1) / kPageTokens - p_begin;
     const int i_full1 = q_hi / kPageTokens - p_begin;
-    int st = 0;
-    uint32_t ph = 0;  // the ring stage and its barrier phase of page i
+    const NibMasks nmask = nib_masks();
+    int st = 0;  // the ring stage of page i
     int n_loop = npg;
-    if (p.expire_first_wait && npg > 0) {
+    if (p.expire_first_wait == 1 && npg > 0) {
         // test hook: the first wait counts as expired.  The timeout path
         // runs as it would: record the status, then wait (bounded, the
         // normal limit) for the copies in flight; no page is attended.
         if (lane == 0) set_status(p.pool, KVQ_ERR_TIMEOUT);
-        for (int k = 0; k < npg && k < NST; k++)
-            (void)mbar_wait_bounded(bar0 + 8 * (k % NST), (k / NST) & 1, kWaitLimitNs);
+        for (int k = 0; k < npg && k < NST; k++) (void)mbar_wait_bounded(bar0 + 8 * k, (phm >> k) & 1u, kWaitLimitNs);
         n_loop = 0;
     }
     for (int i = 0; i < n_loop; i++) {
-        const uint32_t bar = bar0 + 8 * st;
+        const uint32_t bar = bar0 + 8 * st, ph = (phm >> st) & 1u;
         if (!__all_sync(kFull, mbar_try_wait(bar, ph))) {
             // slow path: the page is not in yet; wait, but not forever
             if (!__all_sync(kFull, mbar_wait_bounded(bar, ph, kWaitLimitNs))) {
@@ -841,12 +910,22 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
                 // the copies still in flight so none lands after the ring is reused
                 if (lane == 0) set_status(p.pool, KVQ_ERR_TIMEOUT);
                 for (int k = i; k < npg && k < i + NST; k++)
-                    (void)mbar_wait_bounded(bar0 + 8 * (k % NST), (k / NST) & 1, kWaitLimitNs);
+                    (void)mbar_wait_bounded(bar0 + 8 * (k % NST), (phm >> (k % NST)) & 1u, kWaitLimitNs);
                 break;
             }
         }
         const uint32_t sb = stage0 + st * C::STAGE;
         const unsigned char *sp = stage0_ptr + st * C::STAGE;
+        if (app_ok && i == npg - 1) {
+            // the appended row, into the staged copy of its page (the same
+            // bytes the append stored; the copy may have missed them)
+            unsigned char *sw = const_cast<unsigned char *>(sp);
+            warp_append_row<D, KF>(p.new_k + app_row, app_sg, p.rotate, p.rot_scale, p.clip, sw + C::K_CODES,
+                                   sw + C::K_META + app_tok * KC::ROW_META, app_tok, nullptr, 0, lane);
+            warp_append_row<D, VF>(p.new_v + app_row, app_sg, p.rotate, p.rot_scale, p.clip, sw + C::V_CODES,
+                                   sw + C::V_META + app_tok * VC::ROW_META, app_tok, nullptr, 1, lane);
+            __syncwarp();
+        }
         const bool page_ok = (vbits >> st) & 1u;
         const bool ragged = i < i_full0 || i >= i_full1 || !page_ok;  // warp-uniform
         // valid tokens of a ragged page: r in [vlo, vhi) (the tail, windows attended elsewhere)
@@ -939,8 +1018,15 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             }
 #pragma unroll
             for (int t = 0; t < NH; t++) {
-                s_r[t] = tv_r ? fmaf(acc_r[t], qinv[t], zr[t]) : -INFINITY;
-                s_r8[t] = tv_r8 ? fmaf(acc_r8[t], qinv[t], zr8[t]) : -INFINITY;
+                s_r[t] = fmaf(acc_r[t], qinv[t], zr[t]);
+                s_r8[t] = fmaf(acc_r8[t], qinv[t], zr8[t]);
+            }
+            if (ragged) {
+#pragma unroll
+                for (int t = 0; t < NH; t++) {
+                    s_r[t] = tv_r ? s_r[t] : -INFINITY;
+                    s_r8[t] = tv_r8 ? s_r8[t] : -INFINITY;
+                }
             }
         }
 
@@ -964,6 +1050,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
                     const float m_new = mx[t] > m_run[t] + 8.0f ? mx[t] : m_run[t];
                     const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_run[t] - m_new);
                     m_run[t] = m_new;
+                    m_ref[t] = m_new == -INFINITY ? 0.f : m_new;
                     l_part[t] *= alpha;
 #pragma unroll
                     for (int mt = 0; mt < C::MT; mt++) {
@@ -980,11 +1067,8 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             }
 #pragma unroll
             for (int t = 0; t < NH; t++) {
-                // m_run is finite once any token was seen; before that every
-                // score is -inf and ex2(-inf - (-inf)) would be NaN
-                const float mr = m_run[t] == -INFINITY ? 0.f : m_run[t];
-                p_r[t] = ex2(s_r[t] - mr);
-                p_r8[t] = ex2(s_r8[t] - mr);
+                p_r[t] = ex2(s_r[t] - m_ref[t]);
+                p_r8[t] = ex2(s_r8[t] - m_ref[t]);
                 l_part[t] += p_r[t] + p_r8[t];
             }
             if (p.page_stats != nullptr) {  // certified mode: this page's (m, l) per head
@@ -1054,7 +1138,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
                     for (int u = 0; u < VC::MT_PER_CHUNK; u++) {
                         const int mt = c * VC::MT_PER_CHUNK + u;
                         uint32_t a[4];
-                        VC::afrag(vA[c], vB[c], u, a);
+                        VC::afrag(vA[c], vB[c], u, a, nmask);
                         const int gi = VC::group_of_mt(mt);
                         mma16816(oacc[t][mt], a, wb[gi][0], wb[gi][1]);
                     }
@@ -1069,10 +1153,8 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             if ((nxt & 31) == 0) ids = fetch_ids(nxt);
             issue(nxt);
         }
-        if (++st == NST) {
-            st = 0;
-            ph ^= 1u;
-        }
+        phm ^= 1u << st;
+        if (++st == NST) st = 0;
     }
 
     // ---- warp state -> shared memory, CTA merge ----
@@ -1275,8 +1357,9 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         if (lane == 0 && p.head_ml) p.head_ml[((long long)b * L.hkv + kvh) * g + h] = make_float2(fM[h], fL[h]);
         if (p.rotate) {
             fwht_warp<D>(v, lane);
+            const uint32_t sg = lane_sign_bits<E>(p.sign_bits, lane);
 #pragma unroll
-            for (int e = 0; e < E; e++) v[e] *= p.rot_scale * p.signs[lane * E + e];
+            for (int e = 0; e < E; e++) v[e] = flip_sign(v[e] * p.rot_scale, sg, e);
         }
         float *dst = p.out + ((long long)b * L.hq + kvh * g + h) * D + lane * E;
         if constexpr (E == 4) {

@@ -137,6 +137,7 @@ struct DecodeParams {
     float rot_scale;
     int rotate;
     float signs[kMaxD];
+    uint32_t sign_bits[kMaxD / 32];  // bit i % 32 of word i / 32: sign i is -1
     int pages_per_split;
     int pages_per_warp;
     int n_splits;

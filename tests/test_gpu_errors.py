@@ -105,7 +105,7 @@ def test_timeout_path_reports_and_recovers():
     ws = torch.zeros(ws_need, dtype=torch.uint8, device="cuda")
     out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
     with pytest.raises(K.KvqError):
-        K.kvq_debug_expire_first_wait(c.handle, 2)
+        K.kvq_debug_expire_first_wait(c.handle, 3)
     K.kvq_debug_expire_first_wait(c.handle, 1)
     try:
         K.kvq_decode_attn(c.handle, q, bt, bt.shape[1], ctx, 1, 0.0, None, ws, ws_need, out)
@@ -117,3 +117,30 @@ def test_timeout_path_reports_and_recovers():
     want = O.decode(pair.ocfg, pair.opool, qn, pair.pages.block_table, wl.ctx)
     max_abs, rel = attn_errors(out.cpu().numpy(), want)
     assert max_abs <= TOL_MAX_ABS and rel <= TOL_REL_L2, (max_abs, rel)
+
+
+def test_wrong_block_table_guesses_are_redone():
+    """A decode CTA may start while the previous kernel is still running and
+    reads the block table early to start its first page copies; with the
+    test hook's mode 2 every such guess counts as wrong, so each warp waits
+    its early copies out and copies the pages again.  The result is still
+    the oracle's attention, for a single sequence and a ragged batch."""
+    torch = _torch()
+    from _cases import TOL_MAX_ABS, TOL_REL_L2, attn_errors
+    import oracle as O
+    for ctx in ([1000], [700, 31, 16]):
+        wl = W.scaled(W.llama(), ctx)
+        pair = build_pair(wl)
+        c = pair.cache
+        qn = W.queries(wl, 0)
+        q = torch.from_numpy(qn).cuda()
+        bt = pair.block_table()
+        K.kvq_debug_expire_first_wait(c.handle, 2)
+        try:
+            out = c.decode(q, bt, pair.ctx())
+            assert c.sync_status() == K.KVQ_OK
+        finally:
+            K.kvq_debug_expire_first_wait(c.handle, 0)
+        want = O.decode(pair.ocfg, pair.opool, qn, pair.pages.block_table, wl.ctx)
+        max_abs, rel = attn_errors(out.cpu().numpy(), want)
+        assert max_abs <= TOL_MAX_ABS and rel <= TOL_REL_L2, (ctx, max_abs, rel)
