@@ -100,24 +100,25 @@ struct SplitPlan {
     int pages_per_warp, pages_per_split, n_splits;
 };
 
-// Split the context so that the largest sequence fills about two CTAs per SM
-// when every sequence is as long as the block table allows.
+// Split the context so that the grid of (split, kv head, sequence) CTAs
+// fills the two CTA slots of every SM in one wave when every sequence is as
+// long as the block table allows: as many splits as the slots allow per
+// (sequence, kv head) pair (at most the final merge's limit), pages spread
+// evenly over them in whole pages per warp.  More pairs than slots take one
+// split each.
 SplitPlan plan_splits(const kvq_cache *c, int batch, int max_pages)
 {
     SplitPlan s{};
-    const long long work = (long long)batch * c->L.hkv * max_pages;
-    const long long target = 2LL * c->num_sms;
-    long long per_cta = (work + target - 1) / target;
-    if (per_cta < 1) per_cta = 1;
-    s.pages_per_warp = (int)((per_cta + kDecodeWarps - 1) / kDecodeWarps);
+    const long long pairs = (long long)batch * c->L.hkv;
+    const long long slots = 2LL * c->num_sms;
+    long long want = pairs > 0 ? slots / pairs : 1;
+    if (want < 1) want = 1;
+    if (want > decode_max_splits(c->L)) want = decode_max_splits(c->L);
+    const long long per_split = (max_pages + want - 1) / want;
+    s.pages_per_warp = (int)((per_split + kDecodeWarps - 1) / kDecodeWarps);
+    if (s.pages_per_warp < 1) s.pages_per_warp = 1;
     s.pages_per_split = s.pages_per_warp * kDecodeWarps;
     s.n_splits = (max_pages + s.pages_per_split - 1) / s.pages_per_split;
-    // the final merge holds every split's weight in shared memory
-    while (s.n_splits > decode_max_splits(c->L)) {
-        s.pages_per_warp *= 2;
-        s.pages_per_split = s.pages_per_warp * kDecodeWarps;
-        s.n_splits = (max_pages + s.pages_per_split - 1) / s.pages_per_split;
-    }
     if (s.n_splits < 1) s.n_splits = 1;
     return s;
 }

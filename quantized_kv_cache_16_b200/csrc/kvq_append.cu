@@ -49,19 +49,39 @@ __device__ __forceinline__ float max3(float a, float b, float c)
     return r;
 }
 
+// A constant pair held in a register pair: the packed instructions take
+// their operands from registers, and a pair the compiler may re-materialise
+// costs a move at every use.
+__device__ __forceinline__ float2 reg_pair(float x, float y)
+{
+    float2 r;
+    asm volatile("mov.b32 %0, %2;\n\tmov.b32 %1, %3;" : "=f"(r.x), "=f"(r.y) : "f"(x), "f"(y));
+    return r;
+}
+
+// The constant pairs of the packed arithmetic: (-1, -1) and the rounding
+// magic, set up once per row.
+struct PackC {
+    float2 m1, magic;
+};
+__device__ __forceinline__ PackC pack_consts()
+{
+    return PackC{reg_pair(-1.0f, -1.0f), reg_pair(kRoundMagic, kRoundMagic)};
+}
+
 // a - b, rounded once: fma(b, -1, a)
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b, const PackC &k) { return __ffma2_rn(b, k.m1, a); }
 
 // codes of a pair: clamp(rint((y - z) * inv), lo, hi) as the low bits of
 // (value + magic); the clamp comes before the rounding, which gives the same
 // integer
 __device__ __forceinline__ void quant_pair(float2 y, float2 z2, float2 inv2, float lo, float hi, uint32_t &c0,
-                                           uint32_t &c1)
+                                           uint32_t &c1, const PackC &k)
 {
-    float2 t = __fmul2_rn(sub2(y, z2), inv2);
+    float2 t = __fmul2_rn(sub2(y, z2, k), inv2);
     t.x = fminf(fmaxf(t.x, lo), hi);
     t.y = fminf(fmaxf(t.y, lo), hi);
-    t = __fadd2_rn(t, make_float2(kRoundMagic, kRoundMagic));
+    t = __fadd2_rn(t, k.magic);
     c0 = __float_as_uint(t.x);
     c1 = __float_as_uint(t.y);
 }
@@ -73,12 +93,13 @@ __device__ __forceinline__ void quant_pair(float2 y, float2 z2, float2 inv2, flo
 // multiply-add they would round once where the codec rounds twice, and a
 // product just below a half-way point that rounds up onto it would then
 // code differently).
-__device__ __forceinline__ void quant_pair_lo(float2 y, float2 z2, float2 inv2, float lo, uint32_t &c0, uint32_t &c1)
+__device__ __forceinline__ void quant_pair_lo(float2 y, float2 z2, float2 inv2, float lo, uint32_t &c0, uint32_t &c1,
+                                              const PackC &k)
 {
-    float2 t = __fmul2_rn(sub2(y, z2), inv2);
+    float2 t = __fmul2_rn(sub2(y, z2, k), inv2);
     t.x = fmaxf(t.x, lo);
     t.y = fmaxf(t.y, lo);
-    t = __fadd2_rn(t, make_float2(kRoundMagic, kRoundMagic));
+    t = __fadd2_rn(t, k.magic);
     c0 = __float_as_uint(t.x);
     c1 = __float_as_uint(t.y);
 }
@@ -87,6 +108,14 @@ __device__ __forceinline__ void quant_pair_lo(float2 y, float2 z2, float2 inv2, 
 __device__ __forceinline__ int code_of(float y, float z, float inv)
 {
     return (int)(__float_as_uint(__fadd_rn(__fmul_rn(__fsub_rn(y, z), inv), kRoundMagic)) - 0x4B400000u);
+}
+
+// The value of lane ^ 16, every operand an immediate.
+__device__ __forceinline__ float shfl_xor16(float v)
+{
+    float r;
+    asm volatile("shfl.sync.bfly.b32 %0, %1, 16, 0x1f, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
 }
 
 // min / max over the row's lanes (lane and lane ^ 16 for d = 128)
@@ -127,11 +156,11 @@ __device__ __forceinline__ void pair_minmax(const float2 *y, float &lo, float &h
 // Dequantisation error and magnitude of a pair (descriptors): the stored
 // value is code * scale + zero, each step rounded.
 __device__ __forceinline__ void pair_err(float2 y, uint32_t c0, uint32_t c1, float2 s2, float2 z2, float &emax,
-                                         float &amax)
+                                         float &amax, const PackC &k)
 {
     float2 yh = make_float2(code_value(c0), code_value(c1));
     yh = __fadd2_rn(__fmul2_rn(yh, s2), z2);
-    const float2 e = sub2(y, yh);
+    const float2 e = sub2(y, yh, k);
     emax = max3(emax, fabsf(e.x), fabsf(e.y));
     amax = max3(amax, fabsf(y.x), fabsf(y.y));
 }
@@ -143,7 +172,7 @@ __device__ __forceinline__ void pair_err(float2 y, uint32_t c0, uint32_t c1, flo
 // fused square-and-add rounds once instead of twice and was seen to move a
 // near-tie decision).
 template <int NP>
-__device__ __forceinline__ float run_sq_error(const float2 *y, float2 z2, float sf, float lo, float hi)
+__device__ __forceinline__ float run_sq_error(const float2 *y, float2 z2, float sf, float lo, float hi, const PackC &k)
 {
     const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
     const float2 inv2 = make_float2(inv, inv);
@@ -151,7 +180,7 @@ __device__ __forceinline__ float run_sq_error(const float2 *y, float2 z2, float 
 #pragma unroll
     for (int i = 0; i < NP; i++) {
         uint32_t c0, c1;
-        quant_pair(y[i], z2, inv2, lo, hi, c0, c1);
+        quant_pair(y[i], z2, inv2, lo, hi, c0, c1, k);
         const float h0 = __fadd_rn(__fmul_rn(code_value(c0), sf), z2.x);
         const float h1 = __fadd_rn(__fmul_rn(code_value(c1), sf), z2.x);
         const float e0 = __fsub_rn(y[i].x, h0), e1 = __fsub_rn(y[i].y, h1);
@@ -169,7 +198,7 @@ __device__ __forceinline__ float run_sq_error(const float2 *y, float2 z2, float 
 // holds a run of 64 consecutive elements).  Every lane of the warp runs every
 // candidate, so the shuffle never diverges.
 template <int NP, int LANES>
-__device__ __forceinline__ __half search_scale(const float2 *y, __half sh0, float zf, float lo, float hi)
+__device__ __forceinline__ __half search_scale(const float2 *y, __half sh0, float zf, float lo, float hi, const PackC &kc)
 {
     const int b0 = __half_as_ushort(sh0);
     const bool searchable = b0 != 0 && b0 < 0x7C00;
@@ -182,7 +211,7 @@ __device__ __forceinline__ __half search_scale(const float2 *y, __half sh0, floa
         const int bits = b0 + f;
         const bool valid = searchable && bits > 0 && bits < 0x7C00;
         const float sf = valid ? __half2float(__ushort_as_half((unsigned short)bits)) : 0.0f;
-        float err = run_sq_error<NP>(y, z2, sf, lo, hi);
+        float err = run_sq_error<NP>(y, z2, sf, lo, hi, kc);
         if constexpr (LANES == 2) err = __fadd_rn(err, __shfl_xor_sync(kFull, err, 16));
         if (valid && (k == 0 || err < best_err)) {
             best = bits;
@@ -200,6 +229,7 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
     constexpr int LANES = D / 64;
     constexpr unsigned PARTNER = 16;  // the row's other lane (d = 128)
     const Layout &L = p.L;
+    const PackC kc = pack_consts();
     // ---- 64 fp16 from the staged row (shared memory), flip signs (exact), widen to 32 pairs ----
     float2 y[32];
     {
@@ -236,7 +266,7 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
                 if (!(i & hh)) {
                     const float2 a = y[i], b = y[i + hh];
                     y[i] = __fadd2_rn(a, b);
-                    y[i + hh] = sub2(a, b);
+                    y[i + hh] = sub2(a, b, kc);
                 }
         if constexpr (LANES == 2) {
             // lower lane: a + b; upper lane: a - b with a = the lower lane's value
@@ -244,12 +274,11 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
             const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
             for (int i = 0; i < 32; i++) {
-                const float2 o = make_float2(__shfl_xor_sync(kFull, y[i].x, PARTNER),
-                                             __shfl_xor_sync(kFull, y[i].y, PARTNER));
+                const float2 o = make_float2(shfl_xor16(y[i].x), shfl_xor16(y[i].y));
                 y[i] = __ffma2_rn(sg2, y[i], o);
             }
         }
-        const float2 c2 = make_float2(p.rot_scale, p.rot_scale);
+        const float2 c2 = reg_pair(p.rot_scale, p.rot_scale);
 #pragma unroll
         for (int i = 0; i < 32; i++) y[i] = __fmul2_rn(y[i], c2);
     }
@@ -276,7 +305,7 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
             }
             __half shh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
             const __half zhh = __float2half_rn(lo);
-            if constexpr (SEARCH) shh = search_scale<16, 1>(yg, shh, __half2float(zhh), 0.0f, 15.0f);
+            if constexpr (SEARCH) shh = search_scale<16, 1>(yg, shh, __half2float(zhh), 0.0f, 15.0f, kc);
             sfs[gq] = __half2float(shh);
             zfs[gq] = __half2float(zhh);
             infs[gq] = (sfs[gq] == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sfs[gq]);
@@ -298,7 +327,7 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
 #pragma unroll
                     for (int k = 0; k < 4; k++) {
                         uint32_t c0, c1;
-                        quant_pair_lo(yg[4 * m + k], z2, inv2, 0.0f, c0, c1);
+                        quant_pair_lo(yg[4 * m + k], z2, inv2, 0.0f, c0, c1, kc);
                         bb[k] = c0 + (c1 << 4);
                     }
                     w[m] = pack4bytes(bb[0], bb[1], bb[2], bb[3]);
@@ -310,8 +339,8 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
 #pragma unroll
                     for (int k = 0; k < 4; k++) {
                         uint32_t c0, c1;
-                        quant_pair(yg[4 * m + k], z2, inv2, 0.0f, 15.0f, c0, c1);
-                        if (want_desc) pair_err(yg[4 * m + k], c0, c1, s2, z2, emax, amax);
+                        quant_pair(yg[4 * m + k], z2, inv2, 0.0f, 15.0f, c0, c1, kc);
+                        if (want_desc) pair_err(yg[4 * m + k], c0, c1, s2, z2, emax, amax, kc);
                         bb[k] = c0 + (c1 << 4);
                     }
                     w[m] = pack4bytes(bb[0], bb[1], bb[2], bb[3]);
@@ -337,7 +366,7 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
         }
         __half shh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 3.0f));
         const __half zhh = __float2half_rn(lo);
-        if constexpr (SEARCH) shh = search_scale<32, LANES>(y, shh, __half2float(zhh), 0.0f, 3.0f);
+        if constexpr (SEARCH) shh = search_scale<32, LANES>(y, shh, __half2float(zhh), 0.0f, 3.0f, kc);
         const float sf = __half2float(shh), zf = __half2float(zhh);
         const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
         const float2 z2 = make_float2(zf, zf), inv2 = make_float2(inv, inv), s2 = make_float2(sf, sf);
@@ -352,8 +381,8 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
 #pragma unroll
                 for (int k = 0; k < 4; k++) {
                     uint32_t c[4];
-                    quant_pair_lo(y[8 * m + 2 * k], z2, inv2, 0.0f, c[0], c[1]);
-                    quant_pair_lo(y[8 * m + 2 * k + 1], z2, inv2, 0.0f, c[2], c[3]);
+                    quant_pair_lo(y[8 * m + 2 * k], z2, inv2, 0.0f, c[0], c[1], kc);
+                    quant_pair_lo(y[8 * m + 2 * k + 1], z2, inv2, 0.0f, c[2], c[3], kc);
                     bb[k] = c[0] + (c[1] << 2) + (c[2] << 4) + (c[3] << 6);
                 }
                 w[m] = pack4bytes(bb[0], bb[1], bb[2], bb[3]);
@@ -365,11 +394,11 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
 #pragma unroll
                 for (int k = 0; k < 4; k++) {
                     uint32_t c[4];
-                    quant_pair(y[8 * m + 2 * k], z2, inv2, 0.0f, 3.0f, c[0], c[1]);
-                    quant_pair(y[8 * m + 2 * k + 1], z2, inv2, 0.0f, 3.0f, c[2], c[3]);
+                    quant_pair(y[8 * m + 2 * k], z2, inv2, 0.0f, 3.0f, c[0], c[1], kc);
+                    quant_pair(y[8 * m + 2 * k + 1], z2, inv2, 0.0f, 3.0f, c[2], c[3], kc);
                     if (want_desc) {
-                        pair_err(y[8 * m + 2 * k], c[0], c[1], s2, z2, emax, amax);
-                        pair_err(y[8 * m + 2 * k + 1], c[2], c[3], s2, z2, emax, amax);
+                        pair_err(y[8 * m + 2 * k], c[0], c[1], s2, z2, emax, amax, kc);
+                        pair_err(y[8 * m + 2 * k + 1], c[2], c[3], s2, z2, emax, amax, kc);
                     }
                     bb[k] = c[0] + (c[1] << 2) + (c[2] << 4) + (c[3] << 6);
                 }
@@ -393,7 +422,7 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
         float a = fmaxf(max3(am[0], am[1], am[2]), am[3]);
         a = row_max<LANES>(a);
         __half shh = __float2half_ru(__fdiv_rn(a, 127.0f));
-        if constexpr (SEARCH) shh = search_scale<32, LANES>(y, shh, 0.0f, -127.0f, 127.0f);
+        if constexpr (SEARCH) shh = search_scale<32, LANES>(y, shh, 0.0f, -127.0f, 127.0f, kc);
         const float sf = __half2float(shh);
         const float inv = (sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sf);
         if (want_desc) amax = a;
@@ -404,12 +433,12 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
 #pragma unroll
             for (int m = 0; m < 4; m++) {
                 uint32_t cw[4];
-                quant_pair(y[8 * c + 2 * m], z2, inv2, -127.0f, 127.0f, cw[0], cw[1]);
-                quant_pair(y[8 * c + 2 * m + 1], z2, inv2, -127.0f, 127.0f, cw[2], cw[3]);
+                quant_pair(y[8 * c + 2 * m], z2, inv2, -127.0f, 127.0f, cw[0], cw[1], kc);
+                quant_pair(y[8 * c + 2 * m + 1], z2, inv2, -127.0f, 127.0f, cw[2], cw[3], kc);
                 if (want_desc) {
                     float unused = 0.0f;
-                    pair_err(y[8 * c + 2 * m], cw[0], cw[1], s2, z2, emax, unused);
-                    pair_err(y[8 * c + 2 * m + 1], cw[2], cw[3], s2, z2, emax, unused);
+                    pair_err(y[8 * c + 2 * m], cw[0], cw[1], s2, z2, emax, unused, kc);
+                    pair_err(y[8 * c + 2 * m + 1], cw[2], cw[3], s2, z2, emax, unused, kc);
                 }
                 w[m] = pack4bytes(cw[0], cw[1], cw[2], cw[3]);
             }
@@ -493,14 +522,14 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(const __grid_
                          "r"((uint32_t)(nrows * S::ROW_BYTES))
                          : "memory");
         __syncwarp();
-        if (lane < nrows) {
-            const __half *src = (tensor ? p.v : p.k) + (long long)(row0 + lane) * D;
-            asm volatile(
-                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                    smem_u32(buf0 + bsel * S::BUF + lane * S::STRIDE)),
-                "l"(src), "r"((uint32_t)S::ROW_BYTES), "r"(bar)
-                : "memory");
-        }
+        // lanes 0 .. nrows-1 copy one row each (predicated, no branch)
+        const __half *src = (tensor ? p.v : p.k) + (long long)(row0 + min(lane, nrows - 1)) * D;
+        asm volatile(
+            "{\n .reg .pred pc;\n setp.ne.u32 pc, %4, 0;\n"
+            " @pc cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}" ::"r"(
+                smem_u32(buf0 + bsel * S::BUF + lane * S::STRIDE)),
+            "l"(src), "r"((uint32_t)S::ROW_BYTES), "r"(bar), "r"((uint32_t)(lane < nrows))
+            : "memory");
     };
 
     if (g0 < n_groups) issue(g0, 0);

@@ -602,7 +602,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     // kernel may be writing the context lengths, the block table, the query
     // or the pages), so this phase only reads hints and warms L2: the context
     // length and this warp's block-table entries are read (L2 only, never
-    // kept in L1), clamped into the pool, and the pages they name, the
+    // kept in L1), clamped into the pool, and the first pages they name, the
     // query rows and the appended rows are prefetched into L2.
     extern __shared__ __align__(128) unsigned char smem[];
     const uint32_t bar0 = smem_u32(smem + C::OFF_BAR) + warp * NST * 8;
@@ -616,7 +616,9 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             const int pg = __ldcg(bt + p_begin + lane);
             if (pg >= 0 && pg < L.num_pages) {
                 id_h = pg;
-                bulk_prefetch_l2(p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes + (long long)pg * L.page_bytes,
+                // only the ring's first fill: prefetching the whole run at once
+                // queued the first pages behind the rest (measured slower)
+                if (lane < NST) bulk_prefetch_l2(p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes + (long long)pg * L.page_bytes,
                                  L.chunk_bytes);
             }
         }
@@ -1276,28 +1278,21 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         const int ns = min(per_piece, n_active - s0);
         if (tid == 0)
             bulk_load(smem_u32(smem), part_base + (long long)s0 * g * REC, (uint32_t)(ns * split_bytes), rbar);
-        rec_ok = __syncthreads_and(mbar_wait_bounded(rbar, rph, kWaitLimitNs));
-        if (!rec_ok) {
-            // record it; wait (bounded) once more so the copy is not left
-            // landing in the shared memory of an exited CTA; no output
-            if (tid == 0) {
-                set_status(p.pool, KVQ_ERR_TIMEOUT);
-                (void)mbar_wait_bounded(rbar, rph, kWaitLimitNs);
-            }
-            return;
-        }
-        rph ^= 1u;
+        // while the accumulators stream in: warp h reads the piece's (max,
+        // sum) pairs of head h straight from the records and turns them into
+        // weights 2^(m_s - M) and the running (M, L)
         if (warp < g) {
             const int h = warp;
             const float Mold = fM[h];
             float mloc = -INFINITY, lloc = 0.f, mloc2 = -INFINITY, lloc2 = 0.f;
             if (lane < ns) {
-                const float2 ml = *reinterpret_cast<const float2 *>(recs + (lane * g + h) * REC + D);
+                const float2 ml = __ldcg(reinterpret_cast<const float2 *>(part_base + ((long long)(s0 + lane) * g + h) * REC + D));
                 mloc = ml.x;
                 lloc = ml.y;
             }
             if (lane + 32 < ns) {
-                const float2 ml = *reinterpret_cast<const float2 *>(recs + ((lane + 32) * g + h) * REC + D);
+                const float2 ml =
+                    __ldcg(reinterpret_cast<const float2 *>(part_base + ((long long)(s0 + lane + 32) * g + h) * REC + D));
                 mloc2 = ml.x;
                 lloc2 = ml.y;
             }
@@ -1319,21 +1314,42 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
                 fL[h] = fL[h] * c + Lp;
             }
         }
-        __syncthreads();
+        rec_ok = __syncthreads_and(mbar_wait_bounded(rbar, rph, kWaitLimitNs));
+        if (!rec_ok) {
+            // record it; wait (bounded) once more so the copy is not left
+            // landing in the shared memory of an exited CTA; no output
+            if (tid == 0) {
+                set_status(p.pool, KVQ_ERR_TIMEOUT);
+                (void)mbar_wait_bounded(rbar, rph, kWaitLimitNs);
+            }
+            return;
+        }
+        rph ^= 1u;
 #pragma unroll
         for (int k = 0; k < OPT; k++) {
             const int idx = tid + k * kDecodeThreads;
             if (idx < g * (D / 2)) {
                 const int h = idx / (D / 2), ch = 2 * (idx % (D / 2));
                 const float c = fc[h];
-                float2 a = make_float2(o[k].x * c, o[k].y * c);
-                for (int sp = 0; sp < ns; sp++) {
+                // two independent chains (even and odd records)
+                float2 a = make_float2(o[k].x * c, o[k].y * c), a2 = make_float2(0.f, 0.f);
+                int sp = 0;
+                for (; sp + 1 < ns; sp += 2) {
+                    const float f = fw[sp * kMaxGqa + h], f2 = fw[(sp + 1) * kMaxGqa + h];
+                    const float2 v = *reinterpret_cast<const float2 *>(recs + (sp * g + h) * REC + ch);
+                    const float2 v2 = *reinterpret_cast<const float2 *>(recs + ((sp + 1) * g + h) * REC + ch);
+                    a.x = fmaf(f, v.x, a.x);
+                    a.y = fmaf(f, v.y, a.y);
+                    a2.x = fmaf(f2, v2.x, a2.x);
+                    a2.y = fmaf(f2, v2.y, a2.y);
+                }
+                if (sp < ns) {
                     const float f = fw[sp * kMaxGqa + h];
                     const float2 v = *reinterpret_cast<const float2 *>(recs + (sp * g + h) * REC + ch);
                     a.x = fmaf(f, v.x, a.x);
                     a.y = fmaf(f, v.y, a.y);
                 }
-                o[k] = a;
+                o[k] = make_float2(a.x + a2.x, a.y + a2.y);
             }
         }
         __syncthreads();  // the next piece overwrites the staged records
