@@ -177,7 +177,7 @@ cudaError_t launch_nv_append(const AppendParams &p, int num_sms, cudaStream_t st
 // ------------------------------------------------------------------ decode --
 
 constexpr int kNvChunk = 2 * kPageTokens * (kNvRowCode + kNvRowMeta);  // 2304 bytes
-constexpr int kNvStages = 2;
+constexpr int kNvStages = 4;
 constexpr int kNvOffBar = kNvWarps * kNvStages * kNvChunk;
 constexpr int kNvSmem = kNvOffBar + kNvWarps * kNvStages * 8;
 constexpr int kNvMaxSplits = 64;
@@ -222,7 +222,44 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
     __shared__ float wm[kNvWarps][G], wl[kNvWarps][G];
     __shared__ int sflag;
 
+    const int p_begin = split * p.pages_per_split + warp * p.pages_per_warp;
+    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
+    const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
+    const uint32_t stage0 = smem_u32(smem) + warp * kNvStages * kNvChunk;
+    const unsigned char *stage0_ptr = smem + warp * kNvStages * kNvChunk;
+    const uint32_t bar0 = smem_u32(smem + kNvOffBar) + warp * kNvStages * 8;
+
+    // Launched as a programmatic dependent of the stream's previous kernel:
+    // until griddepcontrol.wait returns nothing read is trusted, so this
+    // phase reads the context length and this warp's block-table entries as
+    // hints only (L2, never L1) and prefetches the pages of the ring's first
+    // fill, the query rows and the appended rows into L2.
+    {
+        const int Th = min(max(__ldcg(p.ctx_lens + b), 0), p.max_pages * kPageTokens);
+        const int npg_h = min(p_begin + p.pages_per_warp, (Th + kPageTokens - 1) / kPageTokens) - p_begin;
+        if (lane < npg_h && lane < kNvStages) {
+            const int pg = __ldcg(bt + p_begin + lane);
+            if (pg >= 0 && pg < L.num_pages) bulk_prefetch_l2(kv_base + (long long)pg * L.page_bytes, kNvChunk);
+        }
+        if (warp == 0 && lane == 31) bulk_prefetch_l2(p.q + ((long long)b * L.hq + kvh * g) * kNvD, g * kNvD * 2);
+        if (warp == 1 && lane == 31 && p.new_k != nullptr) {
+            bulk_prefetch_l2(p.new_k + ((long long)b * L.hkv + kvh) * kNvD, kNvD * 2);
+            bulk_prefetch_l2(p.new_v + ((long long)b * L.hkv + kvh) * kNvD, kNvD * 2);
+        }
+        if (lane == 0) {
+            for (int st = 0; st < kNvStages; st++) mbar_init(bar0 + 8 * st, 1);
+            fence_mbar_init();
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // the true context length, this warp's first 32 block-table entries and
+    // the query row go out together
     int T = p.ctx_lens[b];
+    const int id_raw = (lane < p.pages_per_warp && p_begin + lane < p.max_pages) ? bt[p_begin + lane] : -1;
+    uint2 q_raw = make_uint2(0u, 0u);
+    if (warp < g) q_raw = *reinterpret_cast<const uint2 *>(p.q + ((long long)b * L.hq + kvh * g + warp) * kNvD + lane * 4);
     if (T < 0 || T > p.max_pages * kPageTokens) {
         if (split == 0 && tid == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
         T = T < 0 ? 0 : p.max_pages * kPageTokens;
@@ -230,79 +267,78 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
     const int n_pages = (T + kPageTokens - 1) / kPageTokens;
     const int n_act = max(1, (n_pages + p.pages_per_split - 1) / p.pages_per_split);
     if (split >= n_act) return;
-
-    const int p_begin = split * p.pages_per_split + warp * p.pages_per_warp;
     const int npg = max(0, min(p_begin + p.pages_per_warp, n_pages) - p_begin);
-    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
-    const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
-    const uint32_t stage0 = smem_u32(smem) + warp * kNvStages * kNvChunk;
-    const unsigned char *stage0_ptr = smem + warp * kNvStages * kNvChunk;
-    const uint32_t bar0 = smem_u32(smem + kNvOffBar) + warp * kNvStages * 8;
-    if (lane == 0) {
-        for (int st = 0; st < kNvStages; st++) mbar_init(bar0 + 8 * st, 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
-    uint32_t vbits = 0;  // bit st: stage st holds a valid page
-    auto issue = [&](int i) {  // every lane calls this
-        const int st = i % kNvStages;
-        int pg = 0;
-        if (lane == 0) {
+    auto fetch_ids = [&](int i0) -> int {
+        const int i = i0 + lane;
+        int pg = -1;
+        if (i < npg) {
             pg = bt[p_begin + i];
             if (pg < 0 || pg >= L.num_pages) {
                 set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
                 pg = -1;
             }
-            if (pg >= 0)
-                bulk_load(stage0 + st * kNvChunk, kv_base + (long long)pg * L.page_bytes, kNvChunk, bar0 + 8 * st);
-            else
-                asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar0 + 8 * st) : "memory");
         }
-        pg = __shfl_sync(kFull, pg, 0);
-        vbits = (vbits & ~(1u << st)) | ((pg >= 0 ? 1u : 0u) << st);
+        return pg;
     };
+    int ids = -1;  // page ids of the issue window [32k, 32k + 32)
+    if (lane < npg) {
+        ids = id_raw;
+        if (ids < 0 || ids >= L.num_pages) {
+            set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
+            ids = -1;
+        }
+    }
+    uint32_t vbits = 0;  // bit st: stage st holds a valid page
+    auto issue = [&](int i) {  // every lane calls this; lane 0 alone copies (predicated)
+        const int pg = __shfl_sync(kFull, ids, i & 31);
+        const int st = i % kNvStages;
+        vbits = (vbits & ~(1u << st)) | ((pg >= 0 ? 1u : 0u) << st);
+        bulk_load_or_arrive(lane == 0 && pg >= 0, lane == 0 && pg < 0, stage0 + st * kNvChunk,
+                            kv_base + (long long)max(pg, 0) * L.page_bytes, kNvChunk, bar0 + 8 * st);
+    };
+    for (int i = 0; i < kNvStages && i < npg; i++) issue(i);
     // fused append (decode step): the warp that owns the page of position
-    // T - 1 codes the new token's K and V rows into it (default scales)
-    // before any copy of that page
+    // T - 1 codes the new token's K and V rows into the pool (default
+    // scales).  Its ring copy of that page may miss those stores, so the
+    // warp writes the same row into the staged copy when the page arrives.
+    const uint32_t sgb = (p.sign_bits[lane >> 3] >> ((lane & 7) * 4)) & 0xFu;  // signs of elements 4 lane .. + 3
+    const int app_tok = (T - 1) % kPageTokens;
+    bool app_ok = false;
+    auto append_rows = [&](unsigned char *chunk) {
+#pragma unroll 1
+        for (int tensor = 0; tensor < 2; tensor++) {
+            const __half *src = (tensor ? p.new_v : p.new_k) + ((long long)b * L.hkv + kvh) * kNvD + 4 * lane;
+            const uint2 raw = *reinterpret_cast<const uint2 *>(src);
+            const float2 a = __half22float2(bits_h2(raw.x)), c = __half22float2(bits_h2(raw.y));
+            float x[4] = {a.x, a.y, c.x, c.y};
+            if (p.rotate) {  // the append's rotation: exact sign flips, butterflies, one rounded scale
+#pragma unroll
+                for (int e = 0; e < 4; e++) x[e] = __uint_as_float(__float_as_uint(x[e]) ^ (((sgb >> e) & 1u) << 31));
+                fwht_warp<kNvD>(x, lane);
+#pragma unroll
+                for (int e = 0; e < 4; e++) x[e] = __fmul_rn(x[e], p.rot_scale);
+            }
+            store_row(x, default_scale(x), chunk + (tensor ? L.v_codes : L.k_codes) + app_tok * kNvRowCode,
+                      chunk + (tensor ? L.v_meta : L.k_meta) + app_tok * kNvRowMeta, lane);
+        }
+    };
     if (p.new_k != nullptr && T > 0 && n_pages - 1 >= p_begin && n_pages - 1 < p_begin + npg) {
         const int pg = bt[n_pages - 1];
         const int slot = p.new_slots[b];
-        const int tok = (T - 1) % kPageTokens;
-        if (pg < 0 || pg >= L.num_pages || slot != pg * kPageTokens + tok) {
+        if (pg < 0 || pg >= L.num_pages || slot != pg * kPageTokens + app_tok) {
             if (lane == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
         } else {
-            unsigned char *chunk = const_cast<unsigned char *>(kv_base) + (long long)pg * L.page_bytes;
-#pragma unroll 1
-            for (int tensor = 0; tensor < 2; tensor++) {
-                const __half *src = (tensor ? p.new_v : p.new_k) + ((long long)b * L.hkv + kvh) * kNvD + 4 * lane;
-                const uint2 raw = *reinterpret_cast<const uint2 *>(src);
-                const float2 a = __half22float2(bits_h2(raw.x)), c = __half22float2(bits_h2(raw.y));
-                float x[4] = {a.x, a.y, c.x, c.y};
-                if (p.rotate) {  // the append's rotation: exact sign flips, butterflies, one rounded scale
-#pragma unroll
-                    for (int e = 0; e < 4; e++) x[e] = __fmul_rn(x[e], p.signs[4 * lane + e]);
-                    fwht_warp<kNvD>(x, lane);
-#pragma unroll
-                    for (int e = 0; e < 4; e++) x[e] = __fmul_rn(x[e], p.rot_scale);
-                }
-                store_row(x, default_scale(x), chunk + (tensor ? L.v_codes : L.k_codes) + tok * kNvRowCode,
-                          chunk + (tensor ? L.v_meta : L.k_meta) + tok * kNvRowMeta, lane);
-            }
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) asm volatile("fence.proxy.async.global;" ::: "memory");
+            app_ok = true;
+            append_rows(const_cast<unsigned char *>(kv_base) + (long long)pg * L.page_bytes);
         }
     }
-    for (int i = 0; i < kNvStages && i < npg; i++) issue(i);
 
     if (warp < g) {  // the rotated query in log2 units
-        const __half *qh = p.q + ((long long)b * L.hq + kvh * g + warp) * kNvD + lane * 4;
-        const uint2 raw = *reinterpret_cast<const uint2 *>(qh);
-        const float2 a = __half22float2(bits_h2(raw.x)), c = __half22float2(bits_h2(raw.y));
+        const float2 a = __half22float2(bits_h2(q_raw.x)), c = __half22float2(bits_h2(q_raw.y));
         float x[4] = {a.x, a.y, c.x, c.y};
         if (p.rotate) {
 #pragma unroll
-            for (int e = 0; e < 4; e++) x[e] *= p.signs[lane * 4 + e];
+            for (int e = 0; e < 4; e++) x[e] = __uint_as_float(__float_as_uint(x[e]) ^ (((sgb >> e) & 1u) << 31));
             fwht_warp<kNvD>(x, lane);
 #pragma unroll
             for (int e = 0; e < 4; e++) x[e] *= p.rot_scale;
@@ -352,6 +388,10 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
             break;
         }
         const unsigned char *chunk = stage0_ptr + st * kNvChunk;
+        if (app_ok && i == npg - 1) {  // the appended row, into the staged copy of its page
+            append_rows(const_cast<unsigned char *>(chunk));
+            __syncwarp();
+        }
         const int t_page = (p_begin + i) * kPageTokens;
         const int nvalid = ((vbits >> st) & 1u) ? min(kPageTokens, T - t_page) : 0;
 
@@ -457,7 +497,11 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
             }
         }
         __syncwarp();
-        if (i + kNvStages < npg) issue(i + kNvStages);
+        const int nxt = i + kNvStages;
+        if (nxt < npg) {
+            if ((nxt & 31) == 0) ids = fetch_ids(nxt);
+            issue(nxt);
+        }
     }
 
     // warps -> one partial per head (the ring holds the warps' sums now)
@@ -545,7 +589,7 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
         if (p.rotate) {  // back to the original domain: diag(s) H c
             fwht_warp<kNvD>(o4, lane);
 #pragma unroll
-            for (int e = 0; e < 4; e++) o4[e] *= p.rot_scale * p.signs[lane * 4 + e];
+            for (int e = 0; e < 4; e++) o4[e] = __uint_as_float(__float_as_uint(o4[e] * p.rot_scale) ^ (((sgb >> e) & 1u) << 31));
         }
         float *out = p.out + ((long long)b * L.hq + kvh * g + h) * kNvD + lane * 4;
         *reinterpret_cast<float4 *>(out) = Ls > 0.f ? make_float4(o4[0] / Ls, o4[1] / Ls, o4[2] / Ls, o4[3] / Ls)
@@ -564,8 +608,17 @@ cudaError_t launch_nv_decode_g(const DecodeParams &p, dim3 grid, cudaStream_t s)
         once.mark();
     }
     if (p.n_splits > kNvMaxSplits || p.L.chunk_bytes != kNvChunk) return cudaErrorInvalidValue;
-    nvfp4_decode_kernel<G><<<grid, kNvThreads, kNvSmem, s>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kNvThreads);
+    cfg.dynamicSmemBytes = kNvSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, nvfp4_decode_kernel<G>, p);
 }
 
 }  // namespace
