@@ -77,7 +77,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-steps", type=int, default=4, help="oracle steps in the CPU baseline sample")
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, append and CPU legs")
-    ap.add_argument("--leg", choices=["paged", "certified", "ladder", "windows", "hqmq", "nvfp4"],
+    ap.add_argument("--leg", choices=["paged", "certified", "ladder", "windows", "hqmq", "nvfp4", "contexts"],
                     help="run only this leg (one GPU, --steps calls) and print its JSON")
     ap.add_argument("--ctx", type=int, default=0, help="context length of --leg (default: its workload's)")
     return ap.parse_args()
@@ -241,7 +241,7 @@ def kv_bytes_per_token(d: int, hkv: int) -> int:
 class Workload:
     """Llama-3-8B layer decode steps over C rotating cache copies."""
 
-    def __init__(self, dist: Dist):
+    def __init__(self, dist: Dist, T: int = 0, window: int = 100):
         import numpy as np
         import torch
 
@@ -249,7 +249,7 @@ class Workload:
         import workloads as W
 
         self.K, self.W = K, W
-        self.wl = wl = W.llama()
+        self.wl = wl = W.llama() if not T else W.llama(T=T, steps=window)
         self.T, self.window = wl.ctx[0], wl.steps
         dev = torch.device("cuda", torch.cuda.current_device())
         props = torch.cuda.get_device_properties(dev)
@@ -264,8 +264,11 @@ class Workload:
                   num_pages=tabs[0].num_pages)
         self.cfg_kw = kw
         self.cache = K.Cache(K.make_config(**kw))
-        k, v = W.prefix_kv(wl, 0)
-        kd, vd = torch.from_numpy(k).to(dev), torch.from_numpy(v).to(dev)
+        if T:  # other contexts (timing only): the prefix is drawn on the device
+            kd, vd = W.prefix_kv_device(wl, 0, dev)
+        else:
+            k, v = W.prefix_kv(wl, 0)
+            kd, vd = torch.from_numpy(k).to(dev), torch.from_numpy(v).to(dev)
         for c in range(self.copies):  # same prefix values, distinct memory per copy
             self.cache.append(kd, vd, torch.from_numpy(tabs[c].slots(0, 0, self.T)).to(dev))
         del kd, vd
@@ -403,6 +406,7 @@ def run_ours(args, dist: Dist):
         result["windows"] = windows_leg(min(K, 200))
         result["hqmq"] = hqmq_leg(min(K, 200))
         result["nvfp4"] = nvfp4_leg(min(K, 200))
+        result["contexts"] = contexts_leg(min(K, 200))
     if dist.rank == 0:
         if not args.no_extras:
             result["cpu_baseline"] = cpu_leg(wk, args.cpu_steps)
@@ -747,6 +751,42 @@ def windows_leg(steps: int, T: int = 0, sink: int = 128, recent: int = 1024):
                         f"recent {recent} tokens per sequence from a device store",
             "us": round(w_us, 2), "quantised_only_us": round(q_us, 2), "overhead_x": round(w_us / q_us, 3),
             "cache_bytes": kv_bytes, "window_bytes": win_bytes, "steps": steps}
+
+
+CONTEXTS = (4096, 8192, 16384, 32768, 65536, 131072, 262144)
+
+
+def contexts_leg(steps: int, T: int = 0):
+    """The headline decode step (batch 1, int4 g32, append + decode, rotating
+    cache copies > 3x L2) at contexts from 4K to 256K tokens, and a least
+    squares fit of step time = fixed + bytes / stream bandwidth over them: the
+    fixed part is what a step costs whatever the context (launch, prologue,
+    the two merges), the bandwidth is the page stream's."""
+    import numpy as np
+    import torch
+    stream = torch.cuda.Stream()
+    peak, peak_kind = measured_peaks()
+    rows = []
+    for ctx in ((T,) if T else CONTEXTS):
+        wk = Workload(Dist(), T=ctx, window=16)
+        us = _graph_time(lambda s: wk.launch_step(s, stream), steps, stream)
+        assert wk.cache.sync_status() == 0
+        alg = statistics.mean(wk.decode_algorithmic_bytes(s) for s in range(steps))
+        rows.append({"context": ctx + 1, "us": round(us, 2), "bytes": int(alg), "gbs": round(alg / us / 1e3, 1),
+                     "frac": round(alg / us / 1e3 / peak, 4), "copies": wk.copies})
+        del wk
+        torch.cuda.empty_cache()
+    out = {"workload": "llama3-8b layer decode step (B=1, 32/8 heads, d=128, int4 g32, append 1 token + decode) "
+                       "at each context; cache copies rotate over > 3x L2",
+           "peak_gbs": peak, "peak_kind": peak_kind, "points": rows, "steps": steps}
+    if len(rows) >= 3:
+        x = np.array([r["bytes"] for r in rows], float)
+        y = np.array([r["us"] for r in rows], float)
+        slope, fixed = np.polyfit(x, y, 1)
+        out["fit"] = {"fixed_us": round(float(fixed), 2), "stream_gbs": round(1e-3 / float(slope), 1),
+                      "stream_frac": round(1e-3 / float(slope) / peak, 4),
+                      "model": "us = fixed_us + bytes / stream_gbs"}
+    return out
 
 
 def nvfp4_leg(steps: int, T: int = 0):
@@ -1108,7 +1148,7 @@ def main():
         import torch
         torch.cuda.set_device(0)
         leg = {"paged": paged_leg, "certified": certified_leg, "ladder": ladder_leg, "windows": windows_leg, "hqmq": hqmq_leg,
-               "nvfp4": nvfp4_leg}[args.leg]
+               "nvfp4": nvfp4_leg, "contexts": contexts_leg}[args.leg]
         print(json.dumps(leg(args.steps, args.ctx)), flush=True)
         return
     if args.impl == "reference":

@@ -215,22 +215,35 @@ template <int LANES> __device__ __forceinline__ float group_max(float v)
     return v;
 }
 
+// A store of the appended row's bytes to the pool's page and, when stage is
+// not null, to the same offset of the page's staged copy.
+template <typename T>
+__device__ __forceinline__ void put2(unsigned char *pool, unsigned char *stage, int off, T v)
+{
+    *reinterpret_cast<T *>(pool + off) = v;
+    if (stage) *reinterpret_cast<T *>(stage + off) = v;
+}
+
+// The new token's row (raw: this lane's E fp16 values, already loaded) coded
+// into the pool's page (codes[], scale and zero at meta_row[]) and, when
+// codes_s and meta_s are not null, into the page's staged copy at the same
+// offsets.
 template <int D, int FMT>
-__device__ __forceinline__ void warp_append_row(const __half *src, uint32_t sg, int rotate, float rot_scale,
-                                                float clip, unsigned char *codes, unsigned char *meta_row, int tok,
-                                                unsigned int *desc, int tensor, int lane)
+__device__ __forceinline__ void warp_append_row(uint2 raw, uint32_t sg, int rotate, float rot_scale, float clip,
+                                                unsigned char *codes, unsigned char *meta_row, unsigned char *codes_s,
+                                                unsigned char *meta_s, int tok, unsigned int *desc, int tensor,
+                                                int lane)
 {
     constexpr int E = D / 32;
     float x[E];
     if constexpr (E == 4) {
-        const uint2 u = *reinterpret_cast<const uint2 *>(src + lane * E);
-        const float2 f0 = __half22float2(bits_h2(u.x)), f1 = __half22float2(bits_h2(u.y));
+        const float2 f0 = __half22float2(bits_h2(raw.x)), f1 = __half22float2(bits_h2(raw.y));
         x[0] = f0.x;
         x[1] = f0.y;
         x[2] = f1.x;
         x[3] = f1.y;
     } else {
-        const float2 f0 = __half22float2(bits_h2(*reinterpret_cast<const uint32_t *>(src + lane * E)));
+        const float2 f0 = __half22float2(bits_h2(raw.x));
         x[0] = f0.x;
         x[1] = f0.y;
     }
@@ -274,10 +287,10 @@ __device__ __forceinline__ void warp_append_row(const __half *src, uint32_t sg, 
             emax = fmaxf(emax, fabsf(__fsub_rn(x[e], __fmul_rn(code_value(c, true), sf))));
         }
         const int byte0 = lane * E;  // stream byte
-        unsigned char *dst = codes + ((byte0 / 16) * 16 + tok) * 16 + byte0 % 16;
-        if constexpr (E == 4) *reinterpret_cast<uint32_t *>(dst) = packed;
-        else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)packed;
-        if (lane == 0) *reinterpret_cast<uint16_t *>(meta_row) = __half_as_ushort(shh);
+        const int off = ((byte0 / 16) * 16 + tok) * 16 + byte0 % 16;
+        if constexpr (E == 4) put2<uint32_t>(codes, codes_s, off, packed);
+        else put2<uint16_t>(codes, codes_s, off, (uint16_t)packed);
+        if (lane == 0) put2<uint16_t>(meta_row, meta_s, 0, __half_as_ushort(shh));
     } else {
         constexpr bool I4 = FMT == KVQ_INT4_ASYM;
         constexpr int GL = I4 ? 32 / E : 32;  // lanes per group
@@ -309,18 +322,18 @@ __device__ __forceinline__ void warp_append_row(const __half *src, uint32_t sg, 
         }
         if constexpr (I4) {
             const int gi = lane / GL, q = lane % GL;  // q-th run of E codes in group gi
-            unsigned char *dst = codes + (gi * 16 + tok) * 16 + (q * E) / 2;
-            if constexpr (E == 4) *reinterpret_cast<uint16_t *>(dst) = (uint16_t)packed;
-            else *dst = (unsigned char)packed;
+            const int off = (gi * 16 + tok) * 16 + (q * E) / 2;
+            if constexpr (E == 4) put2<uint16_t>(codes, codes_s, off, (uint16_t)packed);
+            else put2<uint8_t>(codes, codes_s, off, (uint8_t)packed);
             if (q == 0) {
-                reinterpret_cast<uint16_t *>(meta_row)[gi] = __half_as_ushort(shh);
-                reinterpret_cast<uint16_t *>(meta_row)[NG + gi] = __half_as_ushort(zhh);
+                put2<uint16_t>(meta_row, meta_s, 2 * gi, __half_as_ushort(shh));
+                put2<uint16_t>(meta_row, meta_s, 2 * (NG + gi), __half_as_ushort(zhh));
             }
         } else {
             static_assert(I4 || E == 4, "2-bit fused append needs head_dim 128");
-            codes[((lane / 16) * 16 + tok) * 16 + lane % 16] = (unsigned char)packed;  // stream byte = lane
+            put2<uint8_t>(codes, codes_s, ((lane / 16) * 16 + tok) * 16 + lane % 16, (uint8_t)packed);  // stream byte = lane
             if (lane == 0)
-                *reinterpret_cast<uint32_t *>(meta_row) = __half_as_ushort(shh) | (uint32_t(__half_as_ushort(zhh)) << 16);
+                put2<uint32_t>(meta_row, meta_s, 0, __half_as_ushort(shh) | (uint32_t(__half_as_ushort(zhh)) << 16));
         }
     }
     if (want_desc) {
@@ -734,32 +747,59 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     };
     const int n_first = min(NST, npg);
     for (int i = n_done; i < n_first; i++) issue(i);
-    // Fused append: the warp that owns the page of position T-1 quantises
-    // the new token's K and V rows into the pool.  Its copy of that page (its
-    // last) may or may not see those stores, so when the page arrives the
-    // warp writes the same row into the staged copy too (see the page loop);
-    // nothing orders the stores before the copy, and no other warp waits.
+    // Fused append: the warp that owns the page of position T-1 (its last
+    // page) codes the new token's K and V rows into it once that page's copy
+    // has landed, storing the bytes both to the pool and to the staged copy
+    // (see the page loop); no other warp waits for it.  The rows and the
+    // slot are copied now (cp.async) into the final merge's row buffer,
+    // unused until every warp has left its page loop, so their latency
+    // hides behind the query work and the first pages.
     const int app_tok = (T - 1) % kPageTokens;
-    bool app_ok = false;
-    const long long app_row = ((long long)b * L.hkv + kvh) * D;
-    const uint32_t app_sg = lane_sign_bits<E>(p.sign_bits, lane);
+    bool app_pending = appends;  // the rows are yet to be stored
+    unsigned char *app_buf = smem + C::OFF_FROW;  // K row, V row, slot
     if (appends) {
-        const int pg = bt[n_pages - 1];
-        const int slot = p.new_slots[b];
-        if (pg < 0 || pg >= L.num_pages || slot != pg * kPageTokens + app_tok) {
-            if (lane == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
-        } else {
-            app_ok = true;
-            unsigned char *chunk = const_cast<unsigned char *>(kv_base) + (long long)pg * L.page_bytes;
-            unsigned int *desc = L.desc_off ? reinterpret_cast<unsigned int *>(const_cast<unsigned char *>(p.pool) +
-                                                                                L.desc_off + ((long long)pg * L.hkv + kvh) * 16)
-                                            : nullptr;
-            warp_append_row<D, KF>(p.new_k + app_row, app_sg, p.rotate, p.rot_scale, p.clip, chunk + L.k_codes,
-                                   chunk + L.k_meta + app_tok * L.k_row_meta, app_tok, desc, 0, lane);
-            warp_append_row<D, VF>(p.new_v + app_row, app_sg, p.rotate, p.rot_scale, p.clip, chunk + L.v_codes,
-                                   chunk + L.v_meta + app_tok * L.v_row_meta, app_tok, desc, 1, lane);
-        }
+        const long long app_row = ((long long)b * L.hkv + kvh) * D + lane * E;
+        const uint32_t dst = smem_u32(app_buf) + lane * E * 2;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(dst), "l"(p.new_k + app_row), "n"(E * 2) : "memory");
+        asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(dst + D * 2), "l"(p.new_v + app_row), "n"(E * 2)
+                     : "memory");
+        if (lane == 0)
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(app_buf) + D * 4), "l"(p.new_slots + b)
+                         : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
     }
+    // codes the rows into the pool's page app_pg and, if stage is not null,
+    // into its staged copy
+    auto append_rows = [&](int app_pg, unsigned char *stage) {
+        app_pending = false;
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncwarp();
+        const int app_slot = *reinterpret_cast<const int *>(app_buf + D * 4);
+        if (app_pg < 0 || app_pg >= L.num_pages || app_slot != app_pg * kPageTokens + app_tok) {
+            if (lane == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
+            return false;
+        }
+        uint2 app_k = make_uint2(0u, 0u), app_v = make_uint2(0u, 0u);
+        if constexpr (E == 4) {
+            app_k = *reinterpret_cast<const uint2 *>(app_buf + lane * 8);
+            app_v = *reinterpret_cast<const uint2 *>(app_buf + D * 2 + lane * 8);
+        } else {
+            app_k.x = *reinterpret_cast<const uint32_t *>(app_buf + lane * 4);
+            app_v.x = *reinterpret_cast<const uint32_t *>(app_buf + D * 2 + lane * 4);
+        }
+        unsigned char *chunk = const_cast<unsigned char *>(kv_base) + (long long)app_pg * L.page_bytes;
+        unsigned int *desc = L.desc_off ? reinterpret_cast<unsigned int *>(const_cast<unsigned char *>(p.pool) +
+                                                                            L.desc_off + ((long long)app_pg * L.hkv + kvh) * 16)
+                                        : nullptr;
+        const uint32_t sg = lane_sign_bits<E>(p.sign_bits, lane);
+        warp_append_row<D, KF>(app_k, sg, p.rotate, p.rot_scale, p.clip, chunk + L.k_codes,
+                               chunk + L.k_meta + app_tok * L.k_row_meta, stage ? stage + C::K_CODES : nullptr,
+                               stage ? stage + C::K_META + app_tok * KC::ROW_META : nullptr, app_tok, desc, 0, lane);
+        warp_append_row<D, VF>(app_v, sg, p.rotate, p.rot_scale, p.clip, chunk + L.v_codes,
+                               chunk + L.v_meta + app_tok * L.v_row_meta, stage ? stage + C::V_CODES : nullptr,
+                               stage ? stage + C::V_META + app_tok * VC::ROW_META : nullptr, app_tok, desc, 1, lane);
+        return true;
+    };
 
     // ---- query (warp h): rotate, pre-scale, group sums, and the three signed
     //      7-bit digits of q * 2^E written straight into the B layout ----
@@ -918,15 +958,10 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         }
         const uint32_t sb = stage0 + st * C::STAGE;
         const unsigned char *sp = stage0_ptr + st * C::STAGE;
-        if (app_ok && i == npg - 1) {
-            // the appended row, into the staged copy of its page (the same
-            // bytes the append stored; the copy may have missed them)
-            unsigned char *sw = const_cast<unsigned char *>(sp);
-            warp_append_row<D, KF>(p.new_k + app_row, app_sg, p.rotate, p.rot_scale, p.clip, sw + C::K_CODES,
-                                   sw + C::K_META + app_tok * KC::ROW_META, app_tok, nullptr, 0, lane);
-            warp_append_row<D, VF>(p.new_v + app_row, app_sg, p.rotate, p.rot_scale, p.clip, sw + C::V_CODES,
-                                   sw + C::V_META + app_tok * VC::ROW_META, app_tok, nullptr, 1, lane);
-            __syncwarp();
+        if (app_pending && i == npg - 1) {
+            // the appended row: into the pool and into the staged copy of its
+            // page, which was copied before the row existed
+            if (append_rows(__shfl_sync(kFull, ids, i & 31), const_cast<unsigned char *>(sp))) __syncwarp();
         }
         const bool page_ok = (vbits >> st) & 1u;
         const bool ragged = i < i_full0 || i >= i_full1 || !page_ok;  // warp-uniform
@@ -1158,6 +1193,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         phm ^= 1u << st;
         if (++st == NST) st = 0;
     }
+    if (app_pending) (void)append_rows(bt[n_pages - 1], nullptr);  // the run ended early: the pool still gets the rows
 
     // ---- warp state -> shared memory, CTA merge ----
     // The zero term of group gi for head j sits in lane (gi, j): add it to

@@ -100,13 +100,19 @@ __device__ __forceinline__ int default_scale(const float (&x)[4])
 
 // Code the lane's four elements under scale byte sc and store them (two
 // code bytes a lane) and the block's scale byte (its first lane).
+// (and, when codes_s / meta_s are not null, the same bytes there too)
 __device__ __forceinline__ void store_row(const float (&x)[4], int sc, unsigned char *codes, unsigned char *meta,
-                                          int lane)
+                                          int lane, unsigned char *codes_s = nullptr, unsigned char *meta_s = nullptr)
 {
     uint32_t c[4];
     lane_codes(x, e4m3_f((uint8_t)sc), c);
-    reinterpret_cast<uint16_t *>(codes)[lane] = (uint16_t)(c[0] | (c[1] << 4) | (c[2] << 8) | (c[3] << 12));
-    if ((lane & 3) == 0) meta[lane >> 2] = (unsigned char)sc;
+    const uint16_t w = (uint16_t)(c[0] | (c[1] << 4) | (c[2] << 8) | (c[3] << 12));
+    reinterpret_cast<uint16_t *>(codes)[lane] = w;
+    if (codes_s) reinterpret_cast<uint16_t *>(codes_s)[lane] = w;
+    if ((lane & 3) == 0) {
+        meta[lane >> 2] = (unsigned char)sc;
+        if (meta_s) meta_s[lane >> 2] = (unsigned char)sc;
+    }
 }
 
 // Grid: persistent CTAs, a warp codes rows r, r + all warps, ... (K rows
@@ -298,17 +304,39 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
     };
     for (int i = 0; i < kNvStages && i < npg; i++) issue(i);
     // fused append (decode step): the warp that owns the page of position
-    // T - 1 codes the new token's K and V rows into the pool (default
-    // scales).  Its ring copy of that page may miss those stores, so the
-    // warp writes the same row into the staged copy when the page arrives.
+    // T - 1 (its last page) codes the new token's K and V rows (default
+    // scales) once that page's copy has landed, storing the bytes both to
+    // the pool and to the staged copy; no other warp waits for it.  The rows
+    // and the slot are copied now (cp.async) into app_buf, so their latency
+    // hides behind the query work and the first pages.
     const uint32_t sgb = (p.sign_bits[lane >> 3] >> ((lane & 7) * 4)) & 0xFu;  // signs of elements 4 lane .. + 3
     const int app_tok = (T - 1) % kPageTokens;
-    bool app_ok = false;
-    auto append_rows = [&](unsigned char *chunk) {
+    __shared__ __align__(16) unsigned char app_buf[2 * kNvD * 2 + 16];  // K row, V row, slot
+    bool app_pending = p.new_k != nullptr && T > 0 && n_pages - 1 >= p_begin && n_pages - 1 < p_begin + npg;
+    if (app_pending) {
+        const long long row = ((long long)b * L.hkv + kvh) * kNvD + 4 * lane;
+        const uint32_t dst = smem_u32(app_buf) + lane * 8;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(p.new_k + row) : "memory");
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst + kNvD * 2), "l"(p.new_v + row) : "memory");
+        if (lane == 0)
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(app_buf) + kNvD * 4), "l"(p.new_slots + b)
+                         : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    // codes the rows into the pool's page pg and, if stage is not null, into its staged copy
+    auto append_rows = [&](int pg, unsigned char *stage) -> bool {
+        app_pending = false;
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncwarp();
+        const int slot = *reinterpret_cast<const int *>(app_buf + kNvD * 4);
+        if (pg < 0 || pg >= L.num_pages || slot != pg * kPageTokens + app_tok) {
+            if (lane == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
+            return false;
+        }
+        unsigned char *chunk = const_cast<unsigned char *>(kv_base) + (long long)pg * L.page_bytes;
 #pragma unroll 1
         for (int tensor = 0; tensor < 2; tensor++) {
-            const __half *src = (tensor ? p.new_v : p.new_k) + ((long long)b * L.hkv + kvh) * kNvD + 4 * lane;
-            const uint2 raw = *reinterpret_cast<const uint2 *>(src);
+            const uint2 raw = *reinterpret_cast<const uint2 *>(app_buf + tensor * kNvD * 2 + lane * 8);
             const float2 a = __half22float2(bits_h2(raw.x)), c = __half22float2(bits_h2(raw.y));
             float x[4] = {a.x, a.y, c.x, c.y};
             if (p.rotate) {  // the append's rotation: exact sign flips, butterflies, one rounded scale
@@ -318,20 +346,13 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
 #pragma unroll
                 for (int e = 0; e < 4; e++) x[e] = __fmul_rn(x[e], p.rot_scale);
             }
-            store_row(x, default_scale(x), chunk + (tensor ? L.v_codes : L.k_codes) + app_tok * kNvRowCode,
-                      chunk + (tensor ? L.v_meta : L.k_meta) + app_tok * kNvRowMeta, lane);
+            const int co = (tensor ? L.v_codes : L.k_codes) + app_tok * kNvRowCode;
+            const int mo = (tensor ? L.v_meta : L.k_meta) + app_tok * kNvRowMeta;
+            store_row(x, default_scale(x), chunk + co, chunk + mo, lane, stage ? stage + co : nullptr,
+                      stage ? stage + mo : nullptr);
         }
+        return true;
     };
-    if (p.new_k != nullptr && T > 0 && n_pages - 1 >= p_begin && n_pages - 1 < p_begin + npg) {
-        const int pg = bt[n_pages - 1];
-        const int slot = p.new_slots[b];
-        if (pg < 0 || pg >= L.num_pages || slot != pg * kPageTokens + app_tok) {
-            if (lane == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
-        } else {
-            app_ok = true;
-            append_rows(const_cast<unsigned char *>(kv_base) + (long long)pg * L.page_bytes);
-        }
-    }
 
     if (warp < g) {  // the rotated query in log2 units
         const float2 a = __half22float2(bits_h2(q_raw.x)), c = __half22float2(bits_h2(q_raw.y));
@@ -388,9 +409,8 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
             break;
         }
         const unsigned char *chunk = stage0_ptr + st * kNvChunk;
-        if (app_ok && i == npg - 1) {  // the appended row, into the staged copy of its page
-            append_rows(const_cast<unsigned char *>(chunk));
-            __syncwarp();
+        if (app_pending && i == npg - 1) {  // the appended row: into the pool and the staged copy of its page
+            if (append_rows(__shfl_sync(kFull, ids, i & 31), const_cast<unsigned char *>(chunk))) __syncwarp();
         }
         const int t_page = (p_begin + i) * kPageTokens;
         const int nvalid = ((vbits >> st) & 1u) ? min(kPageTokens, T - t_page) : 0;
@@ -503,6 +523,7 @@ __global__ void __launch_bounds__(kNvThreads, 2) nvfp4_decode_kernel(const __gri
             issue(nxt);
         }
     }
+    if (app_pending) (void)append_rows(bt[n_pages - 1], nullptr);  // the run ended early: the pool still gets the rows
 
     // warps -> one partial per head (the ring holds the warps' sums now)
     __syncthreads();
