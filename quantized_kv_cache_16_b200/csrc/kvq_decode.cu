@@ -63,34 +63,43 @@ __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t m, uint32_t c)
     return d;
 }
 
-// The three constants of nib, held in registers for the whole loop.
-struct NibMasks {
-    uint32_t lo, hi, h1024;
+// The constants of nib (4-bit values: two masks) and fld2 (2-bit values:
+// four masks), held in registers for the whole loop.
+template <int VF> struct NibMasks {
+    uint32_t m[VF == KVQ_INT2_ASYM ? 4 : 2];
+    uint32_t h1024;
 };
-__device__ __forceinline__ NibMasks nib_masks()
+template <int VF> __device__ __forceinline__ NibMasks<VF> nib_masks()
 {
-    NibMasks m;
-    asm volatile("mov.b32 %0, 0x000F000F;" : "=r"(m.lo));
-    asm volatile("mov.b32 %0, 0x00F000F0;" : "=r"(m.hi));
-    asm volatile("mov.b32 %0, 0x64006400;" : "=r"(m.h1024));
-    return m;
+    NibMasks<VF> k;
+    if constexpr (VF == KVQ_INT2_ASYM) {
+        asm volatile("mov.b32 %0, 0x00030003;" : "=r"(k.m[0]));
+        asm volatile("mov.b32 %0, 0x000C000C;" : "=r"(k.m[1]));
+        asm volatile("mov.b32 %0, 0x00300030;" : "=r"(k.m[2]));
+        asm volatile("mov.b32 %0, 0x00C000C0;" : "=r"(k.m[3]));
+    } else {
+        asm volatile("mov.b32 %0, 0x000F000F;" : "=r"(k.m[0]));
+        asm volatile("mov.b32 %0, 0x00F000F0;" : "=r"(k.m[1]));
+    }
+    asm volatile("mov.b32 %0, 0x64006400;" : "=r"(k.h1024));
+    return k;
 }
 
 // Nibble n (0..3) of each 16-bit half of w as exact fp16 integers:
 // (w & mask) | 0x6400 is 1024 + c * 16^(n&1); subtract / rescale exactly.
-__device__ __forceinline__ uint32_t nib(uint32_t w, int n, const NibMasks &k)
+template <int VF> __device__ __forceinline__ uint32_t nib(uint32_t w, int n, const NibMasks<VF> &k)
 {
     const uint32_t x = (n & 2) ? (w >> 8) : w;
-    if (n & 1) return hfma2u(and_or(x, k.hi, k.h1024), 0x2C002C00u /*1/16*/, 0xD400D400u /*-64*/);
-    return hsub2u(and_or(x, k.lo, k.h1024), kH1024);
+    if (n & 1) return hfma2u(and_or(x, k.m[1], k.h1024), 0x2C002C00u /*1/16*/, 0xD400D400u /*-64*/);
+    return hsub2u(and_or(x, k.m[0], k.h1024), kH1024);
 }
 
 // 2-bit field f (0..7) of each 16-bit half as exact fp16 integers.
-__device__ __forceinline__ uint32_t fld2(uint32_t w, int f)
+template <int VF> __device__ __forceinline__ uint32_t fld2(uint32_t w, int f, const NibMasks<VF> &k)
 {
     const uint32_t x = (f >= 4) ? (w >> 8) : w;
     const int q = f & 3;
-    const uint32_t v = (x & (0x00030003u << (2 * q))) | kH1024;  // 1024 + c * 4^q
+    const uint32_t v = and_or(x, k.m[q], k.h1024);  // 1024 + c * 4^q
     switch (q) {
     case 0: return hsub2u(v, kH1024);
     case 1: return hfma2u(v, 0x34003400u /*1/4*/, 0xDC00DC00u /*-256*/);
@@ -447,7 +456,7 @@ template <int D> struct VCodec<KVQ_INT4_ASYM, D> {
     __device__ static int chan(int mt, int row) { return 32 * (mt >> 1) + 4 * (row & 7) + 2 * (mt & 1) + (row >> 3); }
     __device__ static int group_of_mt(int mt) { return mt >> 1; }
     __device__ static int group_of_chan(int ch) { return ch / 32; }
-    __device__ static void afrag(uint32_t wA, uint32_t wB, int u, uint32_t (&a)[4], const NibMasks &k)
+    __device__ static void afrag(uint32_t wA, uint32_t wB, int u, uint32_t (&a)[4], const NibMasks<KVQ_INT4_ASYM> &k)
     {
         a[0] = nib(wA, 2 * u, k);
         a[1] = nib(wA, 2 * u + 1, k);
@@ -464,12 +473,12 @@ template <int D> struct VCodec<KVQ_INT2_ASYM, D> {
     __device__ static int chan(int mt, int row) { return 64 * (mt >> 2) + 8 * (row & 7) + 2 * (mt & 3) + (row >> 3); }
     __device__ static int group_of_mt(int) { return 0; }
     __device__ static int group_of_chan(int) { return 0; }
-    __device__ static void afrag(uint32_t wA, uint32_t wB, int u, uint32_t (&a)[4], const NibMasks &)
+    __device__ static void afrag(uint32_t wA, uint32_t wB, int u, uint32_t (&a)[4], const NibMasks<KVQ_INT2_ASYM> &k)
     {
-        a[0] = fld2(wA, 2 * u);
-        a[1] = fld2(wA, 2 * u + 1);
-        a[2] = fld2(wB, 2 * u);
-        a[3] = fld2(wB, 2 * u + 1);
+        a[0] = fld2(wA, 2 * u, k);
+        a[1] = fld2(wA, 2 * u + 1, k);
+        a[2] = fld2(wB, 2 * u, k);
+        a[3] = fld2(wB, 2 * u + 1, k);
     }
 };
 
@@ -932,7 +941,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     // Iterations [i_full0, i_full1) are the warp's pages inside [q_lo, q_hi).
     const int i_full0 = (q_lo + kPageTokens - 1) / kPageTokens - p_begin;
     const int i_full1 = q_hi / kPageTokens - p_begin;
-    const NibMasks nmask = nib_masks();
+    const NibMasks<VF> nmask = nib_masks<VF>();
     int st = 0;  // the ring stage of page i
     int n_loop = npg;
     if (p.expire_first_wait == 1 && npg > 0) {
