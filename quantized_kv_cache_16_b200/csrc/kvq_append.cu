@@ -221,44 +221,68 @@ __device__ __forceinline__ __half search_scale(const float2 *y, __half sh0, floa
     return __ushort_as_half((unsigned short)best);
 }
 
+// (a + b, a - b) of the fp16 halves (a low, b high) of w: the exact fp16
+// values added and subtracted in fp32 with one rounding each (b widened,
+// then two mixed-precision operations)
+__device__ __forceinline__ float2 h1_butterfly(uint32_t w)
+{
+    float s, d, b;
+    asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %3;\n cvt.f32.f16 %2, hi;\n"
+        " add.rn.f32.f16 %0, lo, %2;\n sub.rn.f32.f16 %1, lo, %2;\n}"
+        : "=f"(s), "=f"(d), "=f"(b)
+        : "r"(w));
+    return make_float2(s, d);
+}
+
 template <int D, int FMT, bool SEARCH>
 __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *sign_xor, const unsigned char *src,
                                          unsigned char *chunk, int tok, int tensor, int s, bool active,
-                                         unsigned int *desc)
+                                         unsigned int *desc, int x, const float (&csc)[8])
 {
     constexpr int LANES = D / 64;
     constexpr unsigned PARTNER = 16;  // the row's other lane (d = 128)
     const Layout &L = p.L;
     const PackC kc = pack_consts();
     // ---- 64 fp16 from the staged row (shared memory), flip signs (exact), widen to 32 pairs ----
+    // Slot i takes the row's 16-byte chunk i ^ x (x = this lane's row mod 8
+    // when rotating, else 0), so that the lanes of a row group read distinct
+    // banks of the densely staged rows.  The butterflies undo the
+    // permutation: a Sylvester Hadamard transform of a vector whose index is
+    // XORed with x is the transform of the vector with entry k negated when
+    // popcount(k & x) is odd.  Each butterfly then forms the same sum (its
+    // operands swapped) or the negated difference of the unpermuted order,
+    // so every value is exactly plus or minus the unpermuted one, and the
+    // final scale by +-c_d (csc, per chunk) restores the signs exactly.
     float2 y[32];
     {
         const uint4 *s4 = reinterpret_cast<const uint4 *>(src + 128 * s);
         uint4 w[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) w[i] = s4[i];
+        for (int i = 0; i < 8; i++) w[i] = s4[i ^ x];
         const uint4 *sx4 = reinterpret_cast<const uint4 *>(sign_xor + 32 * s);
 #pragma unroll
         for (int i = 0; i < 8; i++) {
             uint32_t ww[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
             if (p.rotate) {
-                const uint4 m = sx4[i];
+                const uint4 m = sx4[i ^ x];
                 ww[0] ^= m.x;
                 ww[1] ^= m.y;
                 ww[2] ^= m.z;
                 ww[3] ^= m.w;
             }
+            if (p.rotate) {
+                // butterfly h = 1 straight from the fp16 pair: (a + b, a - b),
+                // each rounded once in fp32 from the exact fp16 values
 #pragma unroll
-            for (int e = 0; e < 4; e++) y[4 * i + e] = __half22float2(bits_h2(ww[e]));
+                for (int e = 0; e < 4; e++) y[4 * i + e] = h1_butterfly(ww[e]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; e++) y[4 * i + e] = __half22float2(bits_h2(ww[e]));
+            }
         }
     }
-    // ---- butterflies: h = 1 inside a pair, h = 2..32 across pairs, h = 64 across lanes ----
+    // ---- butterflies: h = 2..32 across pairs, h = 64 across lanes ----
     if (p.rotate) {
-#pragma unroll
-        for (int i = 0; i < 32; i++) {
-            const float a = y[i].x, b = y[i].y;
-            y[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
-        }
 #pragma unroll
         for (int hh = 1; hh < 32; hh <<= 1)
 #pragma unroll
@@ -278,9 +302,8 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
                 y[i] = __ffma2_rn(sg2, y[i], o);
             }
         }
-        const float2 c2 = reg_pair(p.rot_scale, p.rot_scale);
 #pragma unroll
-        for (int i = 0; i < 32; i++) y[i] = __fmul2_rn(y[i], c2);
+        for (int i = 0; i < 32; i++) y[i] = __fmul2_rn(y[i], reg_pair(csc[i >> 2], csc[i >> 2]));
     }
 
     unsigned char *codes = chunk + (tensor ? L.v_codes : L.k_codes);
@@ -462,25 +485,26 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
 }
 
 // Rows are processed in groups of 32/LANES consecutive rows of one tensor per
-// warp (16 rows for d = 128).  Each group is staged in shared memory by one
-// bulk copy per row (whole 256-byte rows: full DRAM sectors), double-buffered
-// so the next group streams in while this one is computed; rows sit at a
-// stride of 2d+16 bytes and lane (row = lane & 15, half = lane >> 4) reads its
-// half-row with conflict-free 16-byte loads.  Persistent grid: each warp
-// takes groups g, g + all warps, ...
+// warp (16 rows for d = 128).  Each group (contiguous in the input) is staged
+// in shared memory by one bulk copy, double-buffered so the next group
+// streams in while this one is computed; lane (row = lane & 15, half =
+// lane >> 4) reads its half-row with 16-byte loads in the chunk order
+// i ^ (row & 7), which keeps the eight rows of a load phase on distinct banks
+// (see half_row).  Persistent grid: each warp takes groups g, g + all
+// warps, ...
 constexpr int kAppendWarps = 8;
 
 template <int D> struct AppendSmem {
     static constexpr int LANES = D / 64;
     static constexpr int ROWS = 32 / LANES;       // rows per group
     static constexpr int ROW_BYTES = 2 * D;
-    static constexpr int STRIDE = ROW_BYTES + 16;
+    static constexpr int STRIDE = ROW_BYTES;
     static constexpr int BUF = ROWS * STRIDE;
     static constexpr int BYTES = kAppendWarps * 2 * BUF + kAppendWarps * 2 * 8;  // buffers + mbarriers
 };
 
 template <int D, int KF, int VF, bool SEARCH>
-__global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(const __grid_constant__ AppendParams p)
+__global__ void __launch_bounds__(kAppendWarps * 32, SEARCH ? 1 : 2) append_kernel(const __grid_constant__ AppendParams p)
 {
     using S = AppendSmem<D>;
     constexpr int LANES = S::LANES, ROWS = S::ROWS;
@@ -506,30 +530,23 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(const __grid_
     const bool hkv_pow2 = (p.L.hkv & (p.L.hkv - 1)) == 0;
     const int hkv_shift = __ffs(p.L.hkv) - 1;
     const int g0 = blockIdx.x * kAppendWarps + warp;
+    // this lane's chunk order and the signed output scales it implies (half_row)
+    const int xr = p.rotate ? (r & 7) : 0;
+    float csc[8];
+#pragma unroll
+    for (int c = 0; c < 8; c++) csc[c] = (__popc(c & xr) & 1) ? -p.rot_scale : p.rot_scale;
 
-    // start the copies of group gi into buffer bsel (lanes 0..ROWS-1 one row each)
+    // start the copy of group gi (its nrows rows, contiguous) into buffer bsel
     auto issue = [&](int gi, int bsel) {
         const int tensor = gi >= groups_per_tensor;
         const int row0 = (gi - tensor * groups_per_tensor) * ROWS;
         const int nrows = min(ROWS, rows_per_tensor - row0);
-        const uint32_t bar = bar0 + 8 * bsel;
         // relaxed arm, no proxy fence: the buffer was last read (generic
         // loads, complete before the __syncwarp ending its group) and the
-        // copy's completion is what publishes the data; a release arrive
-        // would wait for this lane's code stores of the previous group
+        // copy's completion is what publishes the data
         if (lane == 0)
-            asm volatile("mbarrier.arrive.expect_tx.relaxed.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
-                         "r"((uint32_t)(nrows * S::ROW_BYTES))
-                         : "memory");
-        __syncwarp();
-        // lanes 0 .. nrows-1 copy one row each (predicated, no branch)
-        const __half *src = (tensor ? p.v : p.k) + (long long)(row0 + min(lane, nrows - 1)) * D;
-        asm volatile(
-            "{\n .reg .pred pc;\n setp.ne.u32 pc, %4, 0;\n"
-            " @pc cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}" ::"r"(
-                smem_u32(buf0 + bsel * S::BUF + lane * S::STRIDE)),
-            "l"(src), "r"((uint32_t)S::ROW_BYTES), "r"(bar), "r"((uint32_t)(lane < nrows))
-            : "memory");
+            bulk_load(smem_u32(buf0 + bsel * S::BUF), (tensor ? p.v : p.k) + (long long)row0 * D,
+                      (uint32_t)(nrows * S::ROW_BYTES), bar0 + 8 * bsel);
     };
 
     if (g0 < n_groups) issue(g0, 0);
@@ -562,8 +579,8 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(const __grid_
             break;
         }
         const unsigned char *src = buf0 + bsel * S::BUF + r * S::STRIDE;
-        if (tensor == 0) half_row<D, KF, SEARCH>(p, sign_xor, src, chunk, tok, 0, s, active, desc);
-        else half_row<D, VF, SEARCH>(p, sign_xor, src, chunk, tok, 1, s, active, desc);
+        if (tensor == 0) half_row<D, KF, SEARCH>(p, sign_xor, src, chunk, tok, 0, s, active, desc, xr, csc);
+        else half_row<D, VF, SEARCH>(p, sign_xor, src, chunk, tok, 1, s, active, desc, xr, csc);
         __syncwarp();  // every lane is done with this buffer before it is refilled
     }
     (void)LANES;
