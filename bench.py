@@ -40,8 +40,8 @@ NOMINAL_HBM_GBS = 8000.0
 # (dram__bytes_read.sum + dram__bytes_write.sum).  Reported as
 # roofline.traffic only while the decode kernel's sources hash to the digest
 # they had when the counters were taken; null otherwise.
-PROFILED_DECODE = {"sources_sha256": "4f2686c25844259234cdd81d4fac3484f962ce661750f6a10d1b6afab05f5edb",
-                   "dram_bytes_per_launch": 42147456}
+PROFILED_DECODE = {"sources_sha256": "08ee6edcd41e16f3d8ff189c5fa8abe6197003818227c472005f5fe3182e8492",
+                   "dram_bytes_per_launch": 42157568}
 DECODE_SOURCES = ("kvq_decode.cu", "kvq_internal.cuh", "kvq_warp.cuh")
 
 
