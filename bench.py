@@ -77,7 +77,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-steps", type=int, default=4, help="oracle steps in the CPU baseline sample")
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, append and CPU legs")
-    ap.add_argument("--leg", choices=["paged", "certified", "ladder", "windows", "hqmq", "nvfp4", "contexts", "append"],
+    ap.add_argument("--leg", choices=["paged", "certified", "ladder", "windows", "hqmq", "nvfp4", "contexts", "append",
+                                      "e2e"],
                     help="run only this leg (one GPU, --steps calls) and print its JSON")
     ap.add_argument("--ctx", type=int, default=0, help="context length of --leg (default: its workload's)")
     return ap.parse_args()
@@ -477,8 +478,10 @@ def e2e_leg(wk: Workload, K: int, stream, dist: Dist):
     dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    t0 = time.perf_counter()
     for s in range(K):
         step(s)
+    t_host = time.perf_counter() - t0
     e1.record(stream)
     torch.cuda.synchronize()
     ms = dist.max(e0.elapsed_time(e1))
@@ -487,6 +490,7 @@ def e2e_leg(wk: Workload, K: int, stream, dist: Dist):
     bytes_rank = sum(wk.kv_bytes(s) for s in range(K))
     return {"value": round(bytes_rank * dist.world / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
             "us_per_step": 1e3 * ms / K, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "host_us_per_step": round(1e6 * t_host / K, 2),
             "how": "one kvq_decode_step_host call per step: the step's pinned host record (q, k, v, slot, ctx) "
                    "copied to the device on the library's copy stream (overlapping the previous step's kernel), "
                    "the fused append + decode, whose kernel writes the output to pinned host memory through its "
@@ -1157,7 +1161,8 @@ def main():
         import torch
         torch.cuda.set_device(0)
         leg = {"paged": paged_leg, "certified": certified_leg, "ladder": ladder_leg, "windows": windows_leg, "hqmq": hqmq_leg,
-               "nvfp4": nvfp4_leg, "contexts": contexts_leg, "append": lambda steps, ctx: append_leg()}[args.leg]
+               "nvfp4": nvfp4_leg, "contexts": contexts_leg, "append": lambda steps, ctx: append_leg(),
+               "e2e": lambda steps, ctx: e2e_leg(Workload(dist), steps, torch.cuda.Stream(), dist)}[args.leg]
         print(json.dumps(leg(args.steps, args.ctx)), flush=True)
         return
     if args.impl == "reference":

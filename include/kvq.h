@@ -377,10 +377,16 @@ size_t kvq_step_record_bytes(const kvq_cache *cache, int32_t batch);
  * kvq_step_record_bytes, 16-byte aligned), used alternately: the record is
  * copied on a stream of the library's own, waiting only for the step that
  * last used the same half, so the copy overlaps the previous step's kernel;
- * the kernel, on `stream`, waits for its copy.  Synchronise `stream` before
- * reading host_out; host_in too must stay unchanged until then (its copy
- * runs asynchronously).  One thread at a time per cache.  block_table stays
- * in device memory.  Host buffers
+ * the kernel, on `stream`, waits for its copy.  For the integer formats the
+ * two sides meet through 32-bit flags in device memory (stream memory
+ * operations on the copy stream; the kernel waits for its record's flag,
+ * bounded, else KVQ_ERR_TIMEOUT, and marks the previous record consumed), so
+ * that `stream` holds nothing between the steps' kernels and they overlap
+ * through the dependent launch; NVFP4 caches use events.  All steps of a
+ * cache go on the same `stream`.  Synchronise `stream` before reading
+ * host_out; host_in too must stay unchanged until then (its copy runs
+ * asynchronously).  One thread at a time per cache.  block_table stays in
+ * device memory.  Host buffers
  * that are not page-locked (cudaHostAlloc / cudaHostRegister) return
  * KVQ_ERR_INVALID_ARG, as do the cases kvq_decode_step rejects. */
 kvq_status kvq_decode_step_host(kvq_cache *cache, const void *host_in, void *dev_rec, const int32_t *block_table,

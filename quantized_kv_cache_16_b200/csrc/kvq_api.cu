@@ -6,6 +6,8 @@
 
 #include <new>
 
+#include <cuda.h>
+
 #include "kvq_internal.cuh"
 
 using namespace kvq;
@@ -337,9 +339,17 @@ kvq_status kvq_destroy_cache(kvq_cache *cache)
 {
     if (!cache) return KVQ_ERR_INVALID_ARG;
     if (cache->copy_stream) {
+        // a copy may wait for a step's mark that no later kernel will set:
+        // raise both marks to the last step first
+        if (cache->io_marks) {
+            volatile unsigned int *m = cache->io_marks;
+            m[0] = m[1] = cache->io_seq;
+        }
         cudaStreamSynchronize(cache->copy_stream);
         cudaStreamDestroy(cache->copy_stream);
     }
+    if (cache->io_flags) cudaFree(cache->io_flags);
+    if (cache->io_marks) cudaFreeHost(cache->io_marks);
     for (int b = 0; b < 2; b++) {
         if (cache->ev_copied[b]) cudaEventDestroy(cache->ev_copied[b]);
         if (cache->ev_consumed[b]) cudaEventDestroy(cache->ev_consumed[b]);
@@ -482,10 +492,39 @@ kvq_status cert_shape_ok(const kvq_cache *c, int max_pages)
     return KVQ_OK;
 }
 
+// Stream memory operations (driver entry points, resolved once): the host
+// step's copy stream waits for, and announces with, 32-bit flags in device
+// memory.  ok is false where they cannot be had (the host step then takes
+// events).
+typedef CUresult (*StreamValueFn)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+struct StreamMemOps {
+    StreamValueFn wait = nullptr, write = nullptr;
+    bool ok = false;
+};
+const StreamMemOps &stream_mem_ops()
+{
+    static const StreamMemOps ops = [] {
+        StreamMemOps o;
+        void *w = nullptr, *x = nullptr;
+        cudaDriverEntryPointQueryResult q1 = cudaDriverEntryPointSymbolNotFound, q2 = q1;
+        if (cudaGetDriverEntryPointByVersion("cuStreamWaitValue32", &w, 12000, cudaEnableDefault, &q1) == cudaSuccess &&
+            cudaGetDriverEntryPointByVersion("cuStreamWriteValue32", &x, 12000, cudaEnableDefault, &q2) == cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess && q2 == cudaDriverEntryPointSuccess && w && x) {
+            o.wait = reinterpret_cast<StreamValueFn>(w);
+            o.write = reinterpret_cast<StreamValueFn>(x);
+            o.ok = true;
+        }
+        cudaGetLastError();
+        return o;
+    }();
+    return ops;
+}
+
 kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const int32_t *slot_mapping,
                        const void *q, const int32_t *block_table, int32_t max_pages_per_seq, const int32_t *ctx_lens,
                        int32_t batch, float softmax_scale, const kvq_tier2 *tier2, void *workspace, size_t ws_bytes,
-                       void *out, int32_t *promoted_out, void *stream)
+                       void *out, int32_t *promoted_out, void *stream, const unsigned int *rec_ready = nullptr,
+                       unsigned int *rec_consumed = nullptr, unsigned int rec_seq = 0)
 {
     if (!c || batch < 0 || max_pages_per_seq < 1) return KVQ_ERR_INVALID_ARG;
     if (batch == 0) return KVQ_OK;
@@ -529,6 +568,9 @@ kvq_status decode_impl(kvq_cache *c, const void *k_new, const void *v_new, const
     p.new_k = static_cast<const __half *>(k_new);
     p.new_v = static_cast<const __half *>(v_new);
     p.new_slots = slot_mapping;
+    p.rec_ready = rec_ready;
+    p.rec_consumed = rec_consumed;
+    p.rec_seq = rec_seq;
     c->last_stream = stream;
     const dim3 grid(s.n_splits, c->L.hkv, batch);
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -753,6 +795,17 @@ bool pinned_host(const void *p)
     return a.type == cudaMemoryTypeHost;
 }
 
+// The device view of page-locked host memory; null for anything else.
+void *pinned_device_view(const void *p)
+{
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
 }  // namespace
 
 extern "C" {
@@ -775,8 +828,8 @@ kvq_status kvq_decode_step_host(kvq_cache *c, const void *host_in, void *dev_rec
                                 size_t ws_bytes, void *host_out, void *stream)
 {
     if (!c || batch < 1 || !host_in || !dev_rec || !host_out || !aligned(dev_rec, 16)) return KVQ_ERR_INVALID_ARG;
-    if (!pinned_host(host_in) || !pinned_host(host_out)) return KVQ_ERR_INVALID_ARG;
-    void *o = const_cast<void *>(device_view(host_out));
+    if (!pinned_host(host_in)) return KVQ_ERR_INVALID_ARG;
+    void *o = pinned_device_view(host_out);
     if (!o || !aligned(o, 16)) return KVQ_ERR_INVALID_ARG;
     if (c->cfg.scale_search || c->L.hq_tab) return KVQ_ERR_UNSUPPORTED;
     if (!c->copy_stream) {
@@ -799,16 +852,73 @@ kvq_status kvq_decode_step_host(kvq_cache *c, const void *host_in, void *dev_rec
         c->ev_consumed[1] = ev[3];
         c->copy_stream = cs;
     }
+    // The integer decode takes the flag handshake: nothing but the steps'
+    // kernels on `stream`, so consecutive steps overlap through the dependent
+    // launch.  NVFP4 (its own decode kernel) takes events between the steps.
+    const StreamMemOps &ops = stream_mem_ops();
+    const bool flags = ops.ok && c->L.k_fmt != KVQ_NVFP4;
+    if (flags && !c->io_flags) {
+        // ready flags in device memory; consumed marks in mapped page-locked
+        // host memory, which the host reads to skip the copy's wait when the
+        // mark is already there
+        unsigned int *f = nullptr, *m = nullptr, *md = nullptr;
+        bool ok = cudaMalloc(&f, 2 * sizeof(unsigned int)) == cudaSuccess &&
+                  cudaMemset(f, 0, 2 * sizeof(unsigned int)) == cudaSuccess &&
+                  cudaHostAlloc(&m, 2 * sizeof(unsigned int), cudaHostAllocMapped) == cudaSuccess &&
+                  cudaHostGetDevicePointer(&md, m, 0) == cudaSuccess;
+        if (!ok) {
+            if (f) cudaFree(f);
+            if (m) cudaFreeHost(m);
+            return KVQ_ERR_CUDA;
+        }
+        m[0] = m[1] = 0u;
+        c->io_flags = f;
+        c->io_marks = m;
+        c->io_marks_dev = md;
+        c->io_seq = 0;
+    }
     const StepRecord r = step_record(c, batch);
-    if (r.bytes != c->io_bytes || dev_rec != c->io_buf) {  // another layout: no half may still be in use
-        if (cudaStreamWaitEvent(c->copy_stream, c->ev_consumed[c->io_next ^ 1], 0) != cudaSuccess)
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool relayout = r.bytes != c->io_bytes || dev_rec != c->io_buf;
+    if (relayout) {
+        // another layout: no half may still be in use, so the copy waits for
+        // every kernel enqueued on `stream` so far
+        if (cudaEventRecord(c->ev_consumed[0], st) != cudaSuccess ||
+            cudaStreamWaitEvent(c->copy_stream, c->ev_consumed[0], 0) != cudaSuccess)
             return KVQ_ERR_CUDA;
         c->io_bytes = r.bytes;
         c->io_buf = dev_rec;
     }
     const int b = c->io_next;
     unsigned char *d = static_cast<unsigned char *>(dev_rec) + (size_t)b * r.bytes;
-    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int32_t *ctx = reinterpret_cast<const int32_t *>(d + r.ctx);
+    const int32_t *slots = reinterpret_cast<const int32_t *>(d + r.slot);
+    if (flags) {
+        // Step n copies into half n & 1 once the kernel of step n - 1 has
+        // started, which it does only after the kernel of step n - 2 (the
+        // half's last reader) is complete: that kernel marks consumed[half]
+        // = n - 2.  The copy then raises ready[half] to n, which the
+        // kernel of step n waits for.  Both compare in modular order.
+        unsigned int *ready = c->io_flags, *consumed = c->io_marks_dev;
+        const unsigned int n = ++c->io_seq;
+        const volatile unsigned int *seen = c->io_marks;
+        if (!relayout && n >= 3 && (int)(seen[b] - (n - 2u)) < 0 &&
+            ops.wait(c->copy_stream, (CUdeviceptr)(consumed + b), n - 2u, CU_STREAM_WAIT_VALUE_GEQ) != CUDA_SUCCESS)
+            return KVQ_ERR_CUDA;
+        if (cudaMemcpyAsync(d, host_in, r.bytes, cudaMemcpyHostToDevice, c->copy_stream) != cudaSuccess ||
+            ops.write(c->copy_stream, (CUdeviceptr)(ready + b), n, CU_STREAM_WRITE_VALUE_DEFAULT) != CUDA_SUCCESS)
+            return KVQ_ERR_CUDA;
+        c->io_next = b ^ 1;
+        unsigned int *mark = n >= 2 ? consumed + (b ^ 1) : nullptr;
+        const kvq_status rc = decode_impl(c, d + r.k, d + r.v, slots, d + r.q, block_table, max_pages_per_seq, ctx,
+                                          batch, softmax_scale, nullptr, workspace, ws_bytes, o, nullptr, stream,
+                                          ready + b, mark, n);
+        // a step whose kernel did not launch still marks the previous half
+        // consumed (after the kernels before it), or the next copy would wait
+        // for a mark that never comes
+        if (rc != KVQ_OK && mark) ops.write(st, (CUdeviceptr)mark, n - 1u, CU_STREAM_WRITE_VALUE_DEFAULT);
+        return rc;
+    }
     // the copy of this step's record overlaps the previous step's kernel: it
     // waits only for the kernel that last read the same buffer
     if (cudaStreamWaitEvent(c->copy_stream, c->ev_consumed[b], 0) != cudaSuccess ||
@@ -816,9 +926,8 @@ kvq_status kvq_decode_step_host(kvq_cache *c, const void *host_in, void *dev_rec
         cudaEventRecord(c->ev_copied[b], c->copy_stream) != cudaSuccess ||
         cudaStreamWaitEvent(st, c->ev_copied[b], 0) != cudaSuccess)
         return KVQ_ERR_CUDA;
-    const kvq_status rc = decode_impl(c, d + r.k, d + r.v, reinterpret_cast<const int32_t *>(d + r.slot), d + r.q,
-                                      block_table, max_pages_per_seq, reinterpret_cast<const int32_t *>(d + r.ctx),
-                                      batch, softmax_scale, nullptr, workspace, ws_bytes, o, nullptr, stream);
+    const kvq_status rc = decode_impl(c, d + r.k, d + r.v, slots, d + r.q, block_table, max_pages_per_seq, ctx, batch,
+                                      softmax_scale, nullptr, workspace, ws_bytes, o, nullptr, stream);
     if (rc != KVQ_OK) return rc;
     if (cudaEventRecord(c->ev_consumed[b], st) != cudaSuccess) return KVQ_ERR_CUDA;
     c->io_next = b ^ 1;

@@ -660,6 +660,20 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
+    if (p.rec_ready != nullptr) {
+        // a step from host buffers: the previous step's record is consumed
+        // (its grid is complete); this step's record comes on the library's
+        // copy stream, announced by its flag.  The mark is a plain store:
+        // nothing written before it needs ordering (the previous grid only
+        // read the record, and its completion is what the mark says)
+        if (p.rec_consumed != nullptr && split == 0 && kvh == 0 && b == 0 && tid == 0)
+            asm volatile("st.relaxed.sys.global.u32 [%0], %1;" ::"l"(p.rec_consumed), "r"(p.rec_seq - 1u) : "memory");
+        bool ok = true;
+        if (lane == 0) ok = flag_wait_bounded(p.rec_ready, p.rec_seq, kWaitLimitNs);
+        __syncwarp();  // the other lanes' record loads come after lane 0's acquire
+        if (!__shfl_sync(kFull, ok, 0) && lane == 0) set_status(p.pool, KVQ_ERR_TIMEOUT);
+    }
+
     // the true values: the context length, this warp's first 32 block-table
     // entries and the query row all go out together, ahead of any copy
     int T = p.ctx_lens[b];

@@ -104,6 +104,14 @@ struct kvq_cache {
     int io_next = 0;
     size_t io_bytes = 0;        // record size and buffer of the last call:
     const void *io_buf = nullptr;  // when either changes, the copy waits for both halves
+    // the integer decode's record handshake (no event between the steps'
+    // kernels, so they overlap through the dependent launch): ready[2] in
+    // device memory, consumed[2] in mapped page-locked host memory (and its
+    // device view), the step number of the last call
+    unsigned int *io_flags = nullptr;
+    unsigned int *io_marks = nullptr;
+    unsigned int *io_marks_dev = nullptr;
+    unsigned int io_seq = 0;
     int expire_first_wait = 0;  // test hook (kvq_debug_expire_first_wait)
 };
 
@@ -157,6 +165,14 @@ struct DecodeParams {
     int win_sink, win_recent;
     float2 *head_ml;          // [B][Hkv][g]: totals (M, L) of the softmax, certified mode only
     int expire_first_wait;    // test hook: each warp's first page wait counts as expired
+    // kvq_decode_step_host: the step's record (context lengths, query, new
+    // rows) is on the device once *rec_ready reaches rec_seq (written after
+    // its copy on the library's copy stream); CTA (0, 0, 0) marks the previous
+    // step's record consumed (*rec_consumed = rec_seq - 1) once the previous
+    // grid is complete.  Null otherwise.
+    const unsigned int *rec_ready;
+    unsigned int *rec_consumed;
+    unsigned int rec_seq;
 };
 
 struct DequantParams {
@@ -387,6 +403,24 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t phase, 
     unsigned long long t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait(bar, phase)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+// Wait until the 32-bit flag *f (written by a stream memory operation, i.e.
+// from outside the SMs) reaches v in modular order, giving up after
+// ~limit_ns.  Acquire at system scope: what was written before the flag is
+// visible after it.
+__device__ __forceinline__ bool flag_wait_bounded(const unsigned int *f, unsigned int v, unsigned long long limit_ns)
+{
+    unsigned int x;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(x) : "l"(f) : "memory");
+    if ((int)(x - v) >= 0) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(32);
+        asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(x) : "l"(f) : "memory");
+        if ((int)(x - v) >= 0) return true;
         if (globaltimer_ns() - t0 > limit_ns) return false;
     }
 }
