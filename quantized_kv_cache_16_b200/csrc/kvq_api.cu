@@ -343,7 +343,7 @@ kvq_status kvq_destroy_cache(kvq_cache *cache)
         // raise both marks to the last step first
         if (cache->io_marks) {
             volatile unsigned int *m = cache->io_marks;
-            m[0] = m[1] = cache->io_seq;
+            m[0] = m[1] = (unsigned int)cache->io_seq;
         }
         cudaStreamSynchronize(cache->copy_stream);
         cudaStreamDestroy(cache->copy_stream);
@@ -899,24 +899,27 @@ kvq_status kvq_decode_step_host(kvq_cache *c, const void *host_in, void *dev_rec
         // half's last reader) is complete: that kernel marks consumed[half]
         // = n - 2.  The copy then raises ready[half] to n, which the
         // kernel of step n waits for.  Both compare in modular order.
+        // (the step count is 64-bit; the flags hold its low 32 bits)
         unsigned int *ready = c->io_flags, *consumed = c->io_marks_dev;
-        const unsigned int n = ++c->io_seq;
+        const unsigned long long n64 = ++c->io_seq;
+        const unsigned int n = (unsigned int)n64;
         const volatile unsigned int *seen = c->io_marks;
-        if (!relayout && n >= 3 && (int)(seen[b] - (n - 2u)) < 0 &&
-            ops.wait(c->copy_stream, (CUdeviceptr)(consumed + b), n - 2u, CU_STREAM_WAIT_VALUE_GEQ) != CUDA_SUCCESS)
+        // any failure from here on makes the next call start afresh (as after
+        // a layout change: its copy waits for every kernel enqueued before it)
+        bool fail = !relayout && n64 >= 3 && (int)(seen[b] - (n - 2u)) < 0 &&
+                    ops.wait(c->copy_stream, (CUdeviceptr)(consumed + b), n - 2u, CU_STREAM_WAIT_VALUE_GEQ) != CUDA_SUCCESS;
+        fail = fail || cudaMemcpyAsync(d, host_in, r.bytes, cudaMemcpyHostToDevice, c->copy_stream) != cudaSuccess ||
+               ops.write(c->copy_stream, (CUdeviceptr)(ready + b), n, CU_STREAM_WRITE_VALUE_DEFAULT) != CUDA_SUCCESS;
+        if (fail) {
+            c->io_bytes = 0;
             return KVQ_ERR_CUDA;
-        if (cudaMemcpyAsync(d, host_in, r.bytes, cudaMemcpyHostToDevice, c->copy_stream) != cudaSuccess ||
-            ops.write(c->copy_stream, (CUdeviceptr)(ready + b), n, CU_STREAM_WRITE_VALUE_DEFAULT) != CUDA_SUCCESS)
-            return KVQ_ERR_CUDA;
+        }
         c->io_next = b ^ 1;
-        unsigned int *mark = n >= 2 ? consumed + (b ^ 1) : nullptr;
+        unsigned int *mark = n64 >= 2 ? consumed + (b ^ 1) : nullptr;
         const kvq_status rc = decode_impl(c, d + r.k, d + r.v, slots, d + r.q, block_table, max_pages_per_seq, ctx,
                                           batch, softmax_scale, nullptr, workspace, ws_bytes, o, nullptr, stream,
                                           ready + b, mark, n);
-        // a step whose kernel did not launch still marks the previous half
-        // consumed (after the kernels before it), or the next copy would wait
-        // for a mark that never comes
-        if (rc != KVQ_OK && mark) ops.write(st, (CUdeviceptr)mark, n - 1u, CU_STREAM_WRITE_VALUE_DEFAULT);
+        if (rc != KVQ_OK) c->io_bytes = 0;
         return rc;
     }
     // the copy of this step's record overlaps the previous step's kernel: it

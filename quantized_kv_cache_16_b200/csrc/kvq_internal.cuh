@@ -111,7 +111,7 @@ struct kvq_cache {
     unsigned int *io_flags = nullptr;
     unsigned int *io_marks = nullptr;
     unsigned int *io_marks_dev = nullptr;
-    unsigned int io_seq = 0;
+    unsigned long long io_seq = 0;
     int expire_first_wait = 0;  // test hook (kvq_debug_expire_first_wait)
 };
 
