@@ -40,8 +40,8 @@ NOMINAL_HBM_GBS = 8000.0
 # (dram__bytes_read.sum + dram__bytes_write.sum).  Reported as
 # roofline.traffic only while the decode kernel's sources hash to the digest
 # they had when the counters were taken; null otherwise.
-PROFILED_DECODE = {"sources_sha256": "86b66c39f33e9b490ea6f69cdbeb1d0e39875f8641574b4f47057eddae55fc7c",
-                   "dram_bytes_per_launch": 42155392}
+PROFILED_DECODE = {"sources_sha256": "06a6c67390f8ad439fa7fb5e40db4464bd2d94c0456c6c0ca69e99b5226958c8",
+                   "dram_bytes_per_launch": 42154880}
 DECODE_SOURCES = ("kvq_decode.cu", "kvq_internal.cuh", "kvq_warp.cuh")
 
 
