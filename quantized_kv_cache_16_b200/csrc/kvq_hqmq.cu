@@ -403,6 +403,46 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
     __shared__ float wm[kHqWarps][G], wl[kHqWarps][G];
     __shared__ int sflag;
 
+    const int p_begin = split * p.pages_per_split + warp * p.pages_per_warp;
+    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
+    const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
+    const uint32_t stage0 = smem_u32(smem + kHqOffStage) + warp * kHqStages * kHqChunk;
+    const unsigned char *stage0_ptr = smem + kHqOffStage + warp * kHqStages * kHqChunk;
+    const uint32_t bar0 = smem_u32(smem + kHqOffBar) + warp * kHqStages * 8;
+
+    // Launched as a programmatic dependent of the stream's previous kernel:
+    // until griddepcontrol.wait returns, only what no kernel writes is read
+    // for use (the codebooks, fixed when the cache was created, and the unit
+    // table); the context length and block-table entries are read as hints
+    // (L2 only) to prefetch the ring's first pages and the query rows.
+    {
+        const float4 *S = reinterpret_cast<const float4 *>(p.pool + L.hq_tab) + (long long)kvh * 2 * kHqmqNS;
+        for (int i = tid; i < 2 * kHqmqNS; i += kHqThreads) tab[i] = __ldg(S + i);
+        // the 24 unit Hurwitz quaternions: p < 8 are +-1, +-i, +-j, +-k; p >= 8
+        // are (+-1 +-i +-j +-k)/2 with component c negative iff bit c of p - 8
+        if (tid < 24 * 8) {
+            const int pu = tid >> 3;
+            float u4[4];
+#pragma unroll
+            for (int c = 0; c < 4; c++)
+                u4[c] = pu < 8 ? (pu / 2 == c ? ((pu & 1) ? -1.f : 1.f) : 0.f) : ((((pu - 8) >> c) & 1) ? -0.5f : 0.5f);
+            units[tid] = make_float4(u4[0], u4[1], u4[2], u4[3]);
+        }
+        const int Th = min(max(__ldcg(p.ctx_lens + b), 0), p.max_pages * kPageTokens);
+        const int npg_h = min(p_begin + p.pages_per_warp, (Th + kPageTokens - 1) / kPageTokens) - p_begin;
+        if (lane < npg_h && lane < kHqStages) {
+            const int pg = __ldcg(bt + p_begin + lane);
+            if (pg >= 0 && pg < L.num_pages) bulk_prefetch_l2(kv_base + (long long)pg * L.page_bytes, kHqChunk);
+        }
+        if (warp == 0 && lane == 31) bulk_prefetch_l2(p.q + ((long long)b * L.hq + kvh * g) * kHqD, g * kHqD * 2);
+        if (lane == 0) {
+            for (int st = 0; st < kHqStages; st++) mbar_init(bar0 + 8 * st, 1);
+            fence_mbar_init();
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
     int T = p.ctx_lens[b];
     if (T < 0 || T > p.max_pages * kPageTokens) {
         if (split == 0 && tid == 0) set_status(p.pool, KVQ_ERR_OUT_OF_RANGE);
@@ -413,17 +453,7 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
     if (split >= n_act) return;
 
     // this warp's pages and its ring; the first copies go out first
-    const int p_begin = split * p.pages_per_split + warp * p.pages_per_warp;
     const int npg = max(0, min(p_begin + p.pages_per_warp, n_pages) - p_begin);
-    const int32_t *bt = p.block_table + (long long)b * p.max_pages;
-    const unsigned char *kv_base = p.pool + kHeaderBytes + (long long)kvh * L.chunk_bytes;
-    const uint32_t stage0 = smem_u32(smem + kHqOffStage) + warp * kHqStages * kHqChunk;
-    const unsigned char *stage0_ptr = smem + kHqOffStage + warp * kHqStages * kHqChunk;
-    const uint32_t bar0 = smem_u32(smem + kHqOffBar) + warp * kHqStages * 8;
-    if (lane == 0) {
-        for (int st = 0; st < kHqStages; st++) mbar_init(bar0 + 8 * st, 1);
-        fence_mbar_init();
-    }
     __syncwarp();
     uint32_t vbits = 0;  // bit st: stage st holds a valid page
     auto issue = [&](int i) {  // every lane calls this
@@ -445,20 +475,6 @@ __global__ void __launch_bounds__(kHqThreads, 2) hqmq_decode_kernel(const __grid
     };
     for (int i = 0; i < kHqStages && i < npg; i++) issue(i);
 
-    {
-        const float4 *S = reinterpret_cast<const float4 *>(p.pool + L.hq_tab) + (long long)kvh * 2 * kHqmqNS;
-        for (int i = tid; i < 2 * kHqmqNS; i += kHqThreads) tab[i] = __ldg(S + i);
-        // the 24 unit Hurwitz quaternions: p < 8 are +-1, +-i, +-j, +-k; p >= 8
-        // are (+-1 +-i +-j +-k)/2 with component c negative iff bit c of p - 8
-        if (tid < 24 * 8) {
-            const int pu = tid >> 3;
-            float u4[4];
-#pragma unroll
-            for (int c = 0; c < 4; c++)
-                u4[c] = pu < 8 ? (pu / 2 == c ? ((pu & 1) ? -1.f : 1.f) : 0.f) : ((((pu - 8) >> c) & 1) ? -0.5f : 0.5f);
-            units[tid] = make_float4(u4[0], u4[1], u4[2], u4[3]);
-        }
-    }
     if (warp < g) {  // the rotated query in log2 units
         const __half *qh = p.q + ((long long)b * L.hq + kvh * g + warp) * kHqD + lane * 4;
         const uint2 raw = *reinterpret_cast<const uint2 *>(qh);
@@ -723,8 +739,17 @@ cudaError_t launch_hq_decode_g(const DecodeParams &p, dim3 grid, cudaStream_t s)
         once.mark();
     }
     if (p.n_splits > kHqMaxSplits || p.L.chunk_bytes != kHqChunk) return cudaErrorInvalidValue;
-    hqmq_decode_kernel<G><<<grid, kHqThreads, kHqSmem, s>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kHqThreads);
+    cfg.dynamicSmemBytes = kHqSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, hqmq_decode_kernel<G>, p);
 }
 
 // CTAs per (kv head, tensor) column: what stays resident in one wave (the
