@@ -278,6 +278,50 @@ def test_decode_step_host_back_to_back():
     assert host.cache.sync_status() == 0 and devp.cache.sync_status() == 0
 
 
+def test_decode_step_host_many_steps_unsynchronised():
+    """Forty kvq_decode_step_host calls in one layout with no
+    synchronisation between them: the record copies and the kernels meet
+    only through the library's ready and consumed flags, so the copy of step
+    n must wait for the kernel of step n - 1 to start (its half's last reader
+    done) whether or not the host already sees the mark.  Every step's output
+    and the final pool bytes equal those of kvq_decode_step run one step at
+    a time on device copies."""
+    import torch
+    import quantized_kv_cache_16_b200 as K
+    n_steps = 40
+    wl = W.scaled(W.llama(), [900, 60, 17])
+    host = build_pair(wl, extra_tokens=n_steps, oracle=False)
+    devp = build_pair(wl, extra_tokens=n_steps, oracle=False)
+    P = host.pages.block_table.shape[1]
+    ws = host.cache.workspace_for(wl.B, P)
+    d_rec = torch.empty(2 * K.kvq_step_record_bytes(host.cache.handle, wl.B), dtype=torch.uint8, device="cuda")
+    pos = list(wl.ctx)
+    rng = np.random.default_rng(12)
+    bt_h = host.block_table()
+    steps = []
+    for step in range(n_steps):
+        q = rng.standard_normal((wl.B, wl.Hq, wl.d)).astype(np.float16)
+        k = rng.standard_normal((wl.B, wl.Hkv, wl.d)).astype(np.float16)
+        v = (0.5 * rng.standard_normal((wl.B, wl.Hkv, wl.d))).astype(np.float16)
+        slots = np.array([host.pages.slot(b, pos[b]) for b in range(wl.B)], np.int32)
+        ctx = np.array([pos[b] + 1 for b in range(wl.B)], np.int32)
+        for b in range(wl.B):
+            pos[b] += 1
+        h_in = _record_of(host.cache, q, k, v, slots, ctx)
+        h_out = torch.full((wl.B, wl.Hq, wl.d), float("nan"), dtype=torch.float32).pin_memory()
+        K.kvq_decode_step_host(host.cache.handle, h_in, d_rec, bt_h, P, wl.B, 0.0, ws, ws.numel(), h_out)
+        steps.append((q, k, v, slots, ctx, h_in, h_out))
+    torch.cuda.synchronize()
+    bt_d = devp.block_table()
+    for step, (q, k, v, slots, ctx, _, h_out) in enumerate(steps):
+        want = devp.cache.step(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(), torch.from_numpy(slots).cuda(),
+                               torch.from_numpy(q).cuda(), bt_d, torch.from_numpy(ctx).cuda())
+        torch.cuda.synchronize()
+        assert np.array_equal(h_out.numpy(), want.cpu().numpy()), f"step {step}"
+    assert np.array_equal(host.cache.pool.cpu().numpy()[256:], devp.cache.pool.cpu().numpy()[256:])
+    assert host.cache.sync_status() == 0 and devp.cache.sync_status() == 0
+
+
 def test_decode_step_host_equals_the_device_step():
     """kvq_decode_step_host (the pinned host record copied in on the
     library's copy stream into alternating buffers, the kernel writing the
