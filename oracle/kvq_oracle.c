@@ -184,6 +184,45 @@ void kvqo_signs(uint64_t seed, int d, float *s)
 /* c_d = 1/sqrt(d) rounded to fp32. */
 float kvqo_rot_scale_f32(int d) { return (float)(1.0 / sqrt((double)d)); }
 
+/* [OSCAR] 2.2(a): P_br, the bit-reversal permutation of the channel index.
+ * With rotate = 2 the rotation is R = H_Had P_br in the page's row-vector
+ * form x R (U, the data-derived eigenbasis, left out): the Hadamard output t
+ * is permuted after the scale, y_j = t_{br(j)}, br(j) = j with its log2(d)
+ * bits in reverse order.  br is its own inverse. */
+int kvqo_bitrev(int j, int d)
+{
+    int r = 0;
+    for (int b = 1; b < d; b <<= 1) {
+        r = (r << 1) | (j & 1);
+        j >>= 1;
+    }
+    return r;
+}
+
+static void bitrev_f32(float *y, int d)
+{
+    for (int j = 0; j < d; j++) {
+        const int k = kvqo_bitrev(j, d);
+        if (k > j) {
+            const float t = y[j];
+            y[j] = y[k];
+            y[k] = t;
+        }
+    }
+}
+
+static void bitrev_f64(double *y, int d)
+{
+    for (int j = 0; j < d; j++) {
+        const int k = kvqo_bitrev(j, d);
+        if (k > j) {
+            const double t = y[j];
+            y[j] = y[k];
+            y[k] = t;
+        }
+    }
+}
+
 /* [SRFT] Methodology 1-2 with the Hadamard choice (SRHT), [OSCAR] 2.2
  * (H_Had factor): y = c_d * H_d * diag(s) * x in fp32.  H_d is the Sylvester
  * (natural-order) Hadamard matrix applied as log2(d) butterfly stages with
@@ -206,6 +245,7 @@ void kvqo_rotate_f32(const float *x, const float *s, int d, int rotate, float *y
             }
     float c = kvqo_rot_scale_f32(d);
     for (int i = 0; i < d; i++) y[i] = y[i] * c;
+    if (rotate == 2) bitrev_f32(y, d);
 }
 
 static void fwht_f64(double *y, int d)
@@ -230,10 +270,12 @@ void kvqo_rotate_f64(const double *x, const float *s, int d, int rotate, double 
     fwht_f64(y, d);
     double c = 1.0 / sqrt((double)d);
     for (int i = 0; i < d; i++) y[i] *= c;
+    if (rotate == 2) bitrev_f64(y, d);
 }
 
 /* fp64 inverse rotation R^T x = diag(s) * H_d * c_d * x ([OSCAR] 2.2b: the
- * fused kernel applies the inverse rotation to the attention output). */
+ * fused kernel applies the inverse rotation to the attention output); with
+ * rotate = 2 the bit reversal is undone first. */
 void kvqo_inv_rotate_f64(const double *x, const float *s, int d, int rotate, double *y)
 {
     if (!rotate) {
@@ -241,6 +283,7 @@ void kvqo_inv_rotate_f64(const double *x, const float *s, int d, int rotate, dou
         return;
     }
     for (int i = 0; i < d; i++) y[i] = x[i];
+    if (rotate == 2) bitrev_f64(y, d);
     fwht_f64(y, d);
     double c = 1.0 / sqrt((double)d);
     for (int i = 0; i < d; i++) y[i] = y[i] * c * (double)s[i];
