@@ -78,7 +78,7 @@ def parse():
     ap.add_argument("--cpu-steps", type=int, default=4, help="oracle steps in the CPU baseline sample")
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, append and CPU legs")
     ap.add_argument("--leg", choices=["paged", "certified", "ladder", "windows", "hqmq", "nvfp4", "contexts", "append",
-                                      "e2e"],
+                                      "e2e", "bitrev"],
                     help="run only this leg (one GPU, --steps calls) and print its JSON")
     ap.add_argument("--ctx", type=int, default=0, help="context length of --leg (default: its workload's)")
     return ap.parse_args()
@@ -248,7 +248,7 @@ def kv_bytes_per_token(d: int, hkv: int) -> int:
 class Workload:
     """Llama-3-8B layer decode steps over C rotating cache copies."""
 
-    def __init__(self, dist: Dist, T: int = 0, window: int = 100):
+    def __init__(self, dist: Dist, T: int = 0, window: int = 100, rotate: int = 1):
         import numpy as np
         import torch
 
@@ -268,7 +268,7 @@ class Workload:
         self.tabs = tabs
         kw = dict(num_q_heads=wl.Hq, num_kv_heads=wl.Hkv, head_dim=wl.d, k_fmt=wl.k_fmt, v_fmt=wl.v_fmt,
                   k_group=wl.k_group, v_group=wl.v_group, clip_ratio=wl.clip, rotation_seed=wl.rotation_seed,
-                  num_pages=tabs[0].num_pages)
+                  rotate=rotate, num_pages=tabs[0].num_pages)
         self.cfg_kw = kw
         self.cache = K.Cache(K.make_config(**kw))
         if T:  # other contexts (timing only): the prefix is drawn on the device
@@ -802,6 +802,29 @@ def contexts_leg(steps: int, T: int = 0):
     return out
 
 
+def bitrev_leg(steps: int, T: int = 0):
+    """The headline decode step with the sign + Hadamard rotation (rotate 1)
+    and with OSCAR's bit-reversal permutation after it (rotate 2), on the
+    same rows and the same rotating cache copies: what the permutation costs
+    the append and the decode."""
+    import torch
+    stream = torch.cuda.Stream()
+    peak, peak_kind = measured_peaks()
+    rows = []
+    for rot in (1, 2):
+        wk = Workload(Dist(), T=T, window=100, rotate=rot)
+        us = _graph_time(lambda s: wk.launch_step(s, stream), steps, stream)
+        assert wk.cache.sync_status() == 0
+        alg = statistics.mean(wk.decode_algorithmic_bytes(s) for s in range(steps))
+        rows.append({"rotate": rot, "context": wk.T + 1, "us": round(us, 2), "gbs": round(alg / us / 1e3, 1),
+                     "frac": round(alg / us / 1e3 / peak, 4)})
+        del wk
+        torch.cuda.empty_cache()
+    return {"workload": "llama3-8b layer decode step (B=1, 32/8 heads, d=128, int4 g32, append 1 token + decode), "
+                        "rotate 1 (signs + Hadamard) vs rotate 2 (then bit reversal); cache copies rotate over > 3x L2",
+            "peak_gbs": peak, "peak_kind": peak_kind, "points": rows, "steps": steps}
+
+
 def nvfp4_leg(steps: int, T: int = 0):
     """The NVFP4 codec at Llama-3-8B layer shape (batch 1, 32/8 heads,
     d=128, context 32768, rotated, ScaleSearch on the E4M3 scales): the bulk
@@ -1161,7 +1184,7 @@ def main():
         import torch
         torch.cuda.set_device(0)
         leg = {"paged": paged_leg, "certified": certified_leg, "ladder": ladder_leg, "windows": windows_leg, "hqmq": hqmq_leg,
-               "nvfp4": nvfp4_leg, "contexts": contexts_leg, "append": lambda steps, ctx: append_leg(),
+               "nvfp4": nvfp4_leg, "contexts": contexts_leg, "bitrev": bitrev_leg, "append": lambda steps, ctx: append_leg(),
                "e2e": lambda steps, ctx: e2e_leg(Workload(dist), steps, torch.cuda.Stream(), dist)}[args.leg]
         print(json.dumps(leg(args.steps, args.ctx)), flush=True)
         return

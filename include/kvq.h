@@ -134,7 +134,13 @@ typedef struct {
     int32_t k_group, v_group;   /* int4: 32; int2, int8: head_dim; HQMQ: 4; NVFP4: 16 */
     float clip_ratio;           /* (0, 1]; scales both ends of int2/int4 groups       */
     uint64_t rotation_seed;     /* SplitMix64 state that draws the sign vector        */
-    int32_t rotate;             /* 1 = sign + Hadamard rotation, 0 = identity         */
+    int32_t rotate;             /* 1 = sign + Hadamard rotation, 0 = identity,
+                                   2 = sign + Hadamard + bit-reversal permutation of
+                                   the channels ["OSCAR", 2.2(a): R = H_Had P_br,
+                                   without the data-derived U; the channel j of
+                                   the rotated row is channel br(j) of H's output,
+                                   br reversing the log2(head_dim) index bits;
+                                   integer formats only]                            */
     int32_t page_tokens;        /* tokens per page; must be 16                        */
     int32_t num_pages;          /* pages in the pool                                  */
     int32_t bound_block_tokens; /* 0 = no error descriptors; else a multiple of 16    */

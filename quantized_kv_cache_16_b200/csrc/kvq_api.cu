@@ -93,7 +93,8 @@ kvq_status check_config(const kvq_config *c)
     if (nv && c->bound_block_tokens != 0) return KVQ_ERR_UNSUPPORTED;
     if (!(c->clip_ratio > 0.0f && c->clip_ratio <= 1.0f)) return KVQ_ERR_INVALID_ARG;
     if (c->bound_block_tokens < 0 || c->bound_block_tokens % kPageTokens) return KVQ_ERR_INVALID_ARG;
-    if (c->rotate != 0 && c->rotate != 1) return KVQ_ERR_INVALID_ARG;
+    if (c->rotate < 0 || c->rotate > 2) return KVQ_ERR_INVALID_ARG;
+    if (c->rotate == 2 && (hq || nv)) return KVQ_ERR_UNSUPPORTED;  // the bit reversal: integer formats
     if (c->scale_search != 0 && c->scale_search != 1) return KVQ_ERR_INVALID_ARG;
     return KVQ_OK;
 }

@@ -234,6 +234,38 @@ __device__ __forceinline__ float2 h1_butterfly(uint32_t w)
     return make_float2(s, d);
 }
 
+// v with its low n bits in reverse order
+__host__ __device__ constexpr int rev_bits(int v, int n) { return n == 0 ? 0 : ((v & 1) << (n - 1)) | rev_bits(v >> 1, n - 1); }
+
+// OSCAR's bit-reversal permutation P_br of a rotated row, after H and c_d
+// ("OSCAR", 2.2(a)): element i moves to position br(i), br reversing the
+// log2(d) index bits.  d = 128, two lanes a row: half s holds elements
+// 64 s + k as pairs y[t] = (k = 2t, 2t + 1); element (s, t, c) lands in half
+// c at pair br5(t), component s.  So lane s keeps component s of each pair,
+// trades the other with its partner (one shuffle a pair) and the pairs move
+// to slot br5(t).  d = 64, one lane a row: a fixed reordering of the lane's
+// registers.  A permutation: every value is moved, none is changed.
+template <int LANES>
+__device__ __forceinline__ void bitrev_row(float2 (&y)[32], int s)
+{
+    float2 z[32];
+    if constexpr (LANES == 2) {
+#pragma unroll
+        for (int t = 0; t < 32; t++) {
+            const float recv = shfl_xor16(s ? y[t].x : y[t].y);
+            z[rev_bits(t, 5)] = s ? make_float2(recv, y[t].y) : make_float2(y[t].x, recv);
+        }
+    } else {
+#pragma unroll
+        for (int u = 0; u < 32; u++) {
+            const int k0 = rev_bits(2 * u, 6), k1 = rev_bits(2 * u + 1, 6);
+            z[u] = make_float2((k0 & 1) ? y[k0 >> 1].y : y[k0 >> 1].x, (k1 & 1) ? y[k1 >> 1].y : y[k1 >> 1].x);
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < 32; t++) y[t] = z[t];
+}
+
 template <int D, int FMT, bool SEARCH>
 __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *sign_xor, const unsigned char *src,
                                          unsigned char *chunk, int tok, int tensor, int s, bool active,
@@ -304,6 +336,7 @@ __device__ __forceinline__ void half_row(const AppendParams &p, const uint32_t *
         }
 #pragma unroll
         for (int i = 0; i < 32; i++) y[i] = __fmul2_rn(y[i], reg_pair(csc[i >> 2], csc[i >> 2]));
+        if (p.rotate == 2) bitrev_row<LANES>(y, s);
     }
 
     unsigned char *codes = chunk + (tensor ? L.v_codes : L.k_codes);

@@ -63,6 +63,7 @@ __device__ __forceinline__ void rotated_query(const CertParams &p, int b, int he
         fwht_warp<D>(x, lane);
 #pragma unroll
         for (int e = 0; e < E; e++) x[e] *= p.rot_scale;
+        if (p.rotate == 2) warp_bitrev<D>(x, lane);  // ["OSCAR", 2.2(a)] P_br after H
     }
 }
 

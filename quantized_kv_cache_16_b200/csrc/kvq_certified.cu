@@ -592,6 +592,7 @@ __global__ void __launch_bounds__(kPromThreads, WIN ? 2 : 1) cert_promote_kernel
 #pragma unroll
         for (int e = 0; e < E; e++) dlt[e] = a[1][e] * fe - a[2][e] * fq;
         if (p.rotate) {
+            if (p.rotate == 2) warp_bitrev<D>(dlt, lane);  // undo P_br first
             fwht_warp<D>(dlt, lane);
 #pragma unroll
             for (int e = 0; e < E; e++) dlt[e] *= p.rot_scale * p.signs[lane * E + e];

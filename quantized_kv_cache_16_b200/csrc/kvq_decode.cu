@@ -236,12 +236,12 @@ __device__ __forceinline__ void put2(unsigned char *pool, unsigned char *stage, 
 // The new token's row (raw: this lane's E fp16 values, already loaded) coded
 // into the pool's page (codes[], scale and zero at meta_row[]) and, when
 // codes_s and meta_s are not null, into the page's staged copy at the same
-// offsets.
+// offsets.  perm: D floats of shared memory for the bit reversal (rotate 2).
 template <int D, int FMT>
 __device__ __forceinline__ void warp_append_row(uint2 raw, uint32_t sg, int rotate, float rot_scale, float clip,
                                                 unsigned char *codes, unsigned char *meta_row, unsigned char *codes_s,
                                                 unsigned char *meta_s, int tok, unsigned int *desc, int tensor,
-                                                int lane)
+                                                int lane, float *perm)
 {
     constexpr int E = D / 32;
     float x[E];
@@ -276,6 +276,15 @@ __device__ __forceinline__ void warp_append_row(uint2 raw, uint32_t sg, int rota
         }
 #pragma unroll
         for (int e = 0; e < E; e++) x[e] = __fmul_rn(x[e], rot_scale);
+        if (rotate == 2) {  // ["OSCAR", 2.2(a)] P_br after H: a permutation (exact), through shared memory
+            __syncwarp();
+#pragma unroll
+            for (int e = 0; e < E; e++) perm[lane * E + e] = x[e];
+            __syncwarp();
+#pragma unroll
+            for (int e = 0; e < E; e++) x[e] = perm[bitrev_index<D>(lane * E + e)];
+            __syncwarp();
+        }
     }
     const bool want_desc = desc != nullptr;
     float emax = 0.f, amax = 0.f;
@@ -779,7 +788,8 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     // hides behind the query work and the first pages.
     const int app_tok = (T - 1) % kPageTokens;
     bool app_pending = appends;  // the rows are yet to be stored
-    unsigned char *app_buf = smem + C::OFF_FROW;  // K row, V row, slot
+    unsigned char *app_buf = smem + C::OFF_FROW;  // K row, V row, slot; at +1024 the bit-reversal scratch
+    static_assert(kMaxGqa * D * 4 >= 1024 + D * 4, "the append's scratch fits in the row buffer");
     if (appends) {
         const long long app_row = ((long long)b * L.hkv + kvh) * D + lane * E;
         const uint32_t dst = smem_u32(app_buf) + lane * E * 2;
@@ -815,12 +825,15 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
                                                                             L.desc_off + ((long long)app_pg * L.hkv + kvh) * 16)
                                         : nullptr;
         const uint32_t sg = lane_sign_bits<E>(p.sign_bits, lane);
+        float *perm = reinterpret_cast<float *>(app_buf + 1024);  // past the rows and the slot
         warp_append_row<D, KF>(app_k, sg, p.rotate, p.rot_scale, p.clip, chunk + L.k_codes,
                                chunk + L.k_meta + app_tok * L.k_row_meta, stage ? stage + C::K_CODES : nullptr,
-                               stage ? stage + C::K_META + app_tok * KC::ROW_META : nullptr, app_tok, desc, 0, lane);
+                               stage ? stage + C::K_META + app_tok * KC::ROW_META : nullptr, app_tok, desc, 0, lane,
+                               perm);
         warp_append_row<D, VF>(app_v, sg, p.rotate, p.rot_scale, p.clip, chunk + L.v_codes,
                                chunk + L.v_meta + app_tok * L.v_row_meta, stage ? stage + C::V_CODES : nullptr,
-                               stage ? stage + C::V_META + app_tok * VC::ROW_META : nullptr, app_tok, desc, 1, lane);
+                               stage ? stage + C::V_META + app_tok * VC::ROW_META : nullptr, app_tok, desc, 1, lane,
+                               perm);
         return true;
     };
 
@@ -864,7 +877,8 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         const float pw2 = __int_as_float((127 + Eh) << 23);
 #pragma unroll
         for (int e = 0; e < E; e++) {
-            const int ch = lane * E + e;
+            // ["OSCAR", 2.2(a)] P_br after H (rotate 2): element i is channel br(i)
+            const int ch = p.rotate == 2 ? bitrev_index<D>(lane * E + e) : lane * E + e;
             const int Q = __float2int_rn(x[e] * pw2);
             const int d3 = ((Q + 64) & 127) - 64;
             const int R = (Q - d3) >> 7;
@@ -881,13 +895,25 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             }
         }
         if constexpr (KC::ZERO) {
-            float sm = 0.f;
+            if (KF == KVQ_INT4_ASYM && p.rotate == 2) {
+                // with P_br a lane's element e falls in group br(e) / 32 of
+                // every lane's, whatever the lane: one warp sum per element
 #pragma unroll
-            for (int e = 0; e < E; e++) sm += x[e];
-            constexpr int LANES = (KF == KVQ_INT4_ASYM) ? 32 / E : 32;
+                for (int e = 0; e < E; e++) {
+                    float sm = x[e];
 #pragma unroll
-            for (int m = 1; m < LANES; m <<= 1) sm += __shfl_xor_sync(kFull, sm, m);
-            if ((lane % LANES) == 0) qsum[h * 4 + (lane * E) / (KF == KVQ_INT4_ASYM ? 32 : D)] = sm;
+                    for (int m = 1; m < 32; m <<= 1) sm += __shfl_xor_sync(kFull, sm, m);
+                    if (lane == 0) qsum[h * 4 + bitrev_index<D>(e) / 32] = sm;
+                }
+            } else {
+                float sm = 0.f;
+#pragma unroll
+                for (int e = 0; e < E; e++) sm += x[e];
+                constexpr int LANES = (KF == KVQ_INT4_ASYM) ? 32 / E : 32;
+#pragma unroll
+                for (int m = 1; m < LANES; m <<= 1) sm += __shfl_xor_sync(kFull, sm, m);
+                if ((lane % LANES) == 0) qsum[h * 4 + (lane * E) / (KF == KVQ_INT4_ASYM ? 32 : D)] = sm;
+            }
         }
     }
     // warps without a head clear the digit columns no head writes
@@ -1427,8 +1453,10 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     // warp h: inverse rotation of head h's normalised row, then the output
     for (int h = warp; h < g; h += kDecodeWarps) {
         float v[E];
+        // (with P_br the row is in the reversed channel order: gather it back)
 #pragma unroll
-        for (int e = 0; e < E; e++) v[e] = frow[h * D + lane * E + e];
+        for (int e = 0; e < E; e++)
+            v[e] = frow[h * D + (p.rotate == 2 ? bitrev_index<D>(lane * E + e) : lane * E + e)];
         if (lane == 0 && p.head_ml) p.head_ml[((long long)b * L.hkv + kvh) * g + h] = make_float2(fM[h], fL[h]);
         if (p.rotate) {
             fwht_warp<D>(v, lane);

@@ -1,6 +1,7 @@
 // kvq_warp.cuh -- warp-level helpers shared by the decode kernels: the full
-// lane mask, the bounded-wait limit, a base-2 exponential and the fp32
-// Walsh-Hadamard transform of a head_dim vector spread over a warp.
+// lane mask, the bounded-wait limit, a base-2 exponential, the fp32
+// Walsh-Hadamard transform of a head_dim vector spread over a warp and the
+// bit-reversal permutation of such a vector.
 #pragma once
 
 #include "kvq_internal.cuh"
@@ -39,6 +40,39 @@ __device__ __forceinline__ void fwht_warp(float (&x)[D / 32], int lane)
             const float o = __shfl_xor_sync(kFull, x[e], m);
             x[e] = (lane & m) ? (o - x[e]) : (x[e] + o);
         }
+}
+
+// OSCAR's bit-reversal permutation P_br of a warp-wide vector (element
+// lane*E + e): element j becomes element br(j) of the input, br reversing the
+// log2(D) bits of the index.  br is its own inverse, so the same call undoes
+// it.  A lane gathers its E elements with E shuffles each (one per possible
+// source register) and keeps the right one.
+template <int D> __device__ __forceinline__ int bitrev_index(int j)
+{
+    constexpr int BITS = D == 128 ? 7 : D == 64 ? 6 : D == 32 ? 5 : 0;
+    static_assert(BITS > 0, "head_dim 32, 64 or 128");
+    return (int)(__brev((unsigned)j) >> (32 - BITS));
+}
+
+template <int D>
+__device__ __forceinline__ void warp_bitrev(float (&x)[D / 32], int lane)
+{
+    constexpr int E = D / 32;
+    float y[E];
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        const int i = bitrev_index<D>(lane * E + e);  // the source element
+        const int src = i / E, se = i % E;
+        float v = 0.f;
+#pragma unroll
+        for (int r = 0; r < E; r++) {
+            const float t = __shfl_sync(kFull, x[r], src);
+            v = r == se ? t : v;
+        }
+        y[e] = v;
+    }
+#pragma unroll
+    for (int e = 0; e < E; e++) x[e] = y[e];
 }
 
 // Two vectors transformed together (independent shuffle chains interleave).

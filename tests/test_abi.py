@@ -52,16 +52,18 @@ def test_pool_bytes_matches_oracle_layout(kw):
 @pytest.mark.parametrize("bad", [
     dict(head_dim=96), dict(num_q_heads=12, num_kv_heads=8), dict(num_q_heads=72, num_kv_heads=8),
     dict(num_pages=0), dict(k_group=64), dict(v_fmt=1, v_group=128), dict(clip_ratio=0.0),
-    dict(clip_ratio=1.5), dict(bound_block_tokens=100), dict(k_fmt=7), dict(rotate=2),
+    dict(clip_ratio=1.5), dict(bound_block_tokens=100), dict(k_fmt=7), dict(rotate=3), dict(rotate=-1),
     # HQMQ: keys and values both, group 4, head_dim 128, no descriptors or scale search
     dict(k_fmt=3, k_group=4), dict(v_fmt=3, v_group=4), dict(k_fmt=3, v_fmt=3, k_group=4, v_group=32),
     dict(k_fmt=3, v_fmt=3, k_group=4, v_group=4, head_dim=64, num_q_heads=8, num_kv_heads=2),
     dict(k_fmt=3, v_fmt=3, k_group=4, v_group=4, bound_block_tokens=64),
     dict(k_fmt=3, v_fmt=3, k_group=4, v_group=4, scale_search=1),
+    dict(k_fmt=3, v_fmt=3, k_group=4, v_group=4, rotate=2),
     # NVFP4: keys and values both, group 16, head_dim 128, no descriptors
     dict(k_fmt=4, k_group=16), dict(k_fmt=4, v_fmt=4, k_group=16, v_group=32),
     dict(k_fmt=4, v_fmt=4, k_group=16, v_group=16, head_dim=64, num_q_heads=8, num_kv_heads=2),
     dict(k_fmt=4, v_fmt=4, k_group=16, v_group=16, bound_block_tokens=64),
+    dict(k_fmt=4, v_fmt=4, k_group=16, v_group=16, rotate=2),
 ])
 def test_invalid_configs_have_no_pool(bad):
     kw = dict(num_q_heads=32, num_kv_heads=8, head_dim=128, num_pages=4)
