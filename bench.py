@@ -40,8 +40,8 @@ NOMINAL_HBM_GBS = 8000.0
 # (dram__bytes_read.sum + dram__bytes_write.sum).  Reported as
 # roofline.traffic only while the decode kernel's sources hash to the digest
 # they had when the counters were taken; null otherwise.
-PROFILED_DECODE = {"sources_sha256": "06a6c67390f8ad439fa7fb5e40db4464bd2d94c0456c6c0ca69e99b5226958c8",
-                   "dram_bytes_per_launch": 42154880}
+PROFILED_DECODE = {"sources_sha256": "68a5966ba0077c3d81b76da4febfd0eb4c02930aa13b99ee59dc681e7cad4261",
+                   "dram_bytes_per_launch": 42157056}
 DECODE_SOURCES = ("kvq_decode.cu", "kvq_internal.cuh", "kvq_warp.cuh")
 
 

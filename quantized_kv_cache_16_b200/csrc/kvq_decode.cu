@@ -867,6 +867,9 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             x[e] *= sc;
             amax = fmaxf(amax, fabsf(x[e]));
         }
+        // ["OSCAR", 2.2(a)] P_br after H (rotate 2): the query in the stored
+        // channel order, so the digits and group sums below are the plain ones
+        if (p.rotate == 2) warp_bitrev<D>(x, lane);
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, m));
         // amax < 2^ex with ex = biased exponent - 126; E = 20 - ex keeps
@@ -877,8 +880,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         const float pw2 = __int_as_float((127 + Eh) << 23);
 #pragma unroll
         for (int e = 0; e < E; e++) {
-            // ["OSCAR", 2.2(a)] P_br after H (rotate 2): element i is channel br(i)
-            const int ch = p.rotate == 2 ? bitrev_index<D>(lane * E + e) : lane * E + e;
+            const int ch = lane * E + e;
             const int Q = __float2int_rn(x[e] * pw2);
             const int d3 = ((Q + 64) & 127) - 64;
             const int R = (Q - d3) >> 7;
@@ -895,25 +897,13 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
             }
         }
         if constexpr (KC::ZERO) {
-            if (KF == KVQ_INT4_ASYM && p.rotate == 2) {
-                // with P_br a lane's element e falls in group br(e) / 32 of
-                // every lane's, whatever the lane: one warp sum per element
+            float sm = 0.f;
 #pragma unroll
-                for (int e = 0; e < E; e++) {
-                    float sm = x[e];
+            for (int e = 0; e < E; e++) sm += x[e];
+            constexpr int LANES = (KF == KVQ_INT4_ASYM) ? 32 / E : 32;
 #pragma unroll
-                    for (int m = 1; m < 32; m <<= 1) sm += __shfl_xor_sync(kFull, sm, m);
-                    if (lane == 0) qsum[h * 4 + bitrev_index<D>(e) / 32] = sm;
-                }
-            } else {
-                float sm = 0.f;
-#pragma unroll
-                for (int e = 0; e < E; e++) sm += x[e];
-                constexpr int LANES = (KF == KVQ_INT4_ASYM) ? 32 / E : 32;
-#pragma unroll
-                for (int m = 1; m < LANES; m <<= 1) sm += __shfl_xor_sync(kFull, sm, m);
-                if ((lane % LANES) == 0) qsum[h * 4 + (lane * E) / (KF == KVQ_INT4_ASYM ? 32 : D)] = sm;
-            }
+            for (int m = 1; m < LANES; m <<= 1) sm += __shfl_xor_sync(kFull, sm, m);
+            if ((lane % LANES) == 0) qsum[h * 4 + (lane * E) / (KF == KVQ_INT4_ASYM ? 32 : D)] = sm;
         }
     }
     // warps without a head clear the digit columns no head writes
@@ -1453,10 +1443,13 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     // warp h: inverse rotation of head h's normalised row, then the output
     for (int h = warp; h < g; h += kDecodeWarps) {
         float v[E];
-        // (with P_br the row is in the reversed channel order: gather it back)
+        if (p.rotate == 2) {  // the row is in the stored (bit-reversed) channel order: gather it back
 #pragma unroll
-        for (int e = 0; e < E; e++)
-            v[e] = frow[h * D + (p.rotate == 2 ? bitrev_index<D>(lane * E + e) : lane * E + e)];
+            for (int e = 0; e < E; e++) v[e] = frow[h * D + bitrev_index<D>(lane * E + e)];
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; e++) v[e] = frow[h * D + lane * E + e];
+        }
         if (lane == 0 && p.head_ml) p.head_ml[((long long)b * L.hkv + kvh) * g + h] = make_float2(fM[h], fL[h]);
         if (p.rotate) {
             fwht_warp<D>(v, lane);
