@@ -40,8 +40,8 @@ NOMINAL_HBM_GBS = 8000.0
 # (dram__bytes_read.sum + dram__bytes_write.sum).  Reported as
 # roofline.traffic only while the decode kernel's sources hash to the digest
 # they had when the counters were taken; null otherwise.
-PROFILED_DECODE = {"sources_sha256": "68a5966ba0077c3d81b76da4febfd0eb4c02930aa13b99ee59dc681e7cad4261",
-                   "dram_bytes_per_launch": 42157056}
+PROFILED_DECODE = {"sources_sha256": "626c094f50917150a990ae7d752084cea4bba58f6ee155bac8bdcc98e96b37b0",
+                   "dram_bytes_per_launch": 42160768}
 DECODE_SOURCES = ("kvq_decode.cu", "kvq_internal.cuh", "kvq_warp.cuh")
 
 

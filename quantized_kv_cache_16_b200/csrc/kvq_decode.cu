@@ -236,8 +236,9 @@ __device__ __forceinline__ void put2(unsigned char *pool, unsigned char *stage, 
 // The new token's row (raw: this lane's E fp16 values, already loaded) coded
 // into the pool's page (codes[], scale and zero at meta_row[]) and, when
 // codes_s and meta_s are not null, into the page's staged copy at the same
-// offsets.  perm: D floats of shared memory for the bit reversal (rotate 2).
-template <int D, int FMT>
+// offsets.  BR: OSCAR's bit reversal after H (rotate 2), through perm, D
+// floats of shared memory.
+template <int D, int FMT, bool BR>
 __device__ __forceinline__ void warp_append_row(uint2 raw, uint32_t sg, int rotate, float rot_scale, float clip,
                                                 unsigned char *codes, unsigned char *meta_row, unsigned char *codes_s,
                                                 unsigned char *meta_s, int tok, unsigned int *desc, int tensor,
@@ -276,7 +277,7 @@ __device__ __forceinline__ void warp_append_row(uint2 raw, uint32_t sg, int rota
         }
 #pragma unroll
         for (int e = 0; e < E; e++) x[e] = __fmul_rn(x[e], rot_scale);
-        if (rotate == 2) {  // ["OSCAR", 2.2(a)] P_br after H: a permutation (exact), through shared memory
+        if constexpr (BR) {  // ["OSCAR", 2.2(a)] P_br after H: a permutation (exact), through shared memory
             __syncwarp();
 #pragma unroll
             for (int e = 0; e < E; e++) perm[lane * E + e] = x[e];
@@ -610,7 +611,9 @@ __device__ __forceinline__ void digit_col(int h, int dg, int &nt, int &col)
     }
 }
 
-template <int D, int KF, int VF, bool G8>
+// BR: the cache stores the rotated channels in bit-reversed order (rotate 2);
+// a template parameter so that the rotate 0/1 kernels carry none of it.
+template <int D, int KF, int VF, bool G8, bool BR>
 __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(const __grid_constant__ DecodeParams p)
 {
     using C = Cfg<KF, VF, D, G8>;
@@ -826,11 +829,11 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
                                         : nullptr;
         const uint32_t sg = lane_sign_bits<E>(p.sign_bits, lane);
         float *perm = reinterpret_cast<float *>(app_buf + 1024);  // past the rows and the slot
-        warp_append_row<D, KF>(app_k, sg, p.rotate, p.rot_scale, p.clip, chunk + L.k_codes,
+        warp_append_row<D, KF, BR>(app_k, sg, p.rotate, p.rot_scale, p.clip, chunk + L.k_codes,
                                chunk + L.k_meta + app_tok * L.k_row_meta, stage ? stage + C::K_CODES : nullptr,
                                stage ? stage + C::K_META + app_tok * KC::ROW_META : nullptr, app_tok, desc, 0, lane,
                                perm);
-        warp_append_row<D, VF>(app_v, sg, p.rotate, p.rot_scale, p.clip, chunk + L.v_codes,
+        warp_append_row<D, VF, BR>(app_v, sg, p.rotate, p.rot_scale, p.clip, chunk + L.v_codes,
                                chunk + L.v_meta + app_tok * L.v_row_meta, stage ? stage + C::V_CODES : nullptr,
                                stage ? stage + C::V_META + app_tok * VC::ROW_META : nullptr, app_tok, desc, 1, lane,
                                perm);
@@ -869,7 +872,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
         }
         // ["OSCAR", 2.2(a)] P_br after H (rotate 2): the query in the stored
         // channel order, so the digits and group sums below are the plain ones
-        if (p.rotate == 2) warp_bitrev<D>(x, lane);
+        if constexpr (BR) warp_bitrev<D>(x, lane);
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, m));
         // amax < 2^ex with ex = biased exponent - 126; E = 20 - ex keeps
@@ -1443,7 +1446,7 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     // warp h: inverse rotation of head h's normalised row, then the output
     for (int h = warp; h < g; h += kDecodeWarps) {
         float v[E];
-        if (p.rotate == 2) {  // the row is in the stored (bit-reversed) channel order: gather it back
+        if constexpr (BR) {  // the row is in the stored (bit-reversed) channel order: gather it back
 #pragma unroll
             for (int e = 0; e < E; e++) v[e] = frow[h * D + bitrev_index<D>(lane * E + e)];
         } else {
@@ -1466,13 +1469,13 @@ __global__ void __launch_bounds__(kDecodeThreads, G8 ? 1 : 2) decode_kernel(cons
     }
 }
 
-template <int D, int KF, int VF, bool G8>
+template <int D, int KF, int VF, bool G8, bool BR>
 cudaError_t launch_t(const DecodeParams &p, dim3 grid, cudaStream_t s)
 {
     using C = Cfg<KF, VF, D, G8>;
     static DeviceOnce once;
     if (once.needed()) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, KF, VF, G8>,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, KF, VF, G8, BR>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         once.mark();
@@ -1487,13 +1490,15 @@ cudaError_t launch_t(const DecodeParams &p, dim3 grid, cudaStream_t s)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<D, KF, VF, G8>, p);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<D, KF, VF, G8, BR>, p);
 }
 
 template <int D, int KF, int VF>
 cudaError_t launch_g(const DecodeParams &p, dim3 grid, cudaStream_t s)
 {
-    return p.L.g > 4 ? launch_t<D, KF, VF, true>(p, grid, s) : launch_t<D, KF, VF, false>(p, grid, s);
+    if (p.rotate == 2)
+        return p.L.g > 4 ? launch_t<D, KF, VF, true, true>(p, grid, s) : launch_t<D, KF, VF, false, true>(p, grid, s);
+    return p.L.g > 4 ? launch_t<D, KF, VF, true, false>(p, grid, s) : launch_t<D, KF, VF, false, false>(p, grid, s);
 }
 
 }  // namespace
