@@ -32,6 +32,8 @@ def test_library_exports_every_declared_symbol():
 CONFIGS = [
     dict(num_q_heads=8, num_kv_heads=2, head_dim=64),
     dict(num_q_heads=32, num_kv_heads=8, head_dim=128),
+    dict(num_q_heads=8, num_kv_heads=2, head_dim=64, rotate=2),
+    dict(num_q_heads=32, num_kv_heads=8, head_dim=128, k_fmt=2, v_fmt=2, k_group=128, v_group=128, rotate=2),
     dict(num_q_heads=32, num_kv_heads=8, head_dim=128, k_fmt=1, k_group=128, bound_block_tokens=128),
     dict(num_q_heads=32, num_kv_heads=8, head_dim=128, k_fmt=2, v_fmt=2, k_group=128, v_group=128, clip_ratio=0.9),
     dict(num_q_heads=64, num_kv_heads=8, head_dim=128, num_pages=3),
