@@ -68,6 +68,23 @@ def test_rotate2_is_the_dense_hadamard_then_bit_reversal(d):
     assert abs(got[0] @ got[1] - q @ k) <= 1e-12 * (abs(q @ k) + 1)
 
 
+@pytest.mark.parametrize("d", [8, 64, 128])
+def test_bit_reversal_commutes_with_the_sylvester_hadamard(d):
+    """H[i][j] = (-1)^popcount(i & j) and br permutes the bits of i and j
+    alike, so H[br(i)][br(j)] = H[i][j]: P_br H = H P_br.  Which side of H
+    the permutation stands on changes no value, only the fp32 rounding
+    order; the rotate = 2 output is also H applied to the bit-reversed
+    signed input."""
+    br = _bitrev(d)
+    H = scipy.linalg.hadamard(d)
+    assert np.array_equal(H[np.ix_(br, br)], H)
+    seed = 0x51
+    s = O.signs(seed, d).astype(np.float64)
+    X = np.random.default_rng(6).standard_normal((5, d))
+    want = ((X * s)[:, br] @ H.T.astype(np.float64)) / math.sqrt(d)
+    assert np.allclose(O.rotate_f64(X, seed, rotate=2), want, rtol=0, atol=1e-12)
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_rotate2_f32_is_the_f32_rotation_reordered_bit_for_bit(d):
     x = np.random.default_rng(5).standard_normal((40, d)).astype(np.float16).astype(np.float32)
