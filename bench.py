@@ -417,6 +417,7 @@ def run_ours(args, dist: Dist):
         result["hqmq"] = hqmq_leg(min(K, 200))
         result["nvfp4"] = nvfp4_leg(min(K, 200))
         result["contexts"] = contexts_leg(min(K, 200))
+        result["bitrev"] = bitrev_leg(min(K, 200))
     if dist.rank == 0:
         if not args.no_extras:
             result["cpu_baseline"] = cpu_leg(wk, args.cpu_steps)
